@@ -1,0 +1,204 @@
+"""fp64 CPU oracle of the tensor-parallel (Megatron) Transformer sublayer.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
+reference arm may call it.  It shares no code with the CUDA path.
+
+It computes the plain, unsharded definition of what the tensor-parallel split
+computes exactly (up to rounding order).  Every input is the exact value the
+GPU receives (bf16 or f32), widened to float64; every intermediate stays in
+float64.  A matmul is done by numpy (a library primitive); nothing is blocked,
+fused or reordered beyond the definition.  Where memory demands it, a product
+is produced a block of *output columns* at a time, which leaves every output
+element's own dot product unchanged.
+
+Pages cited (by title and section):
+  [TYPC]  "张量并行：千亿大模型突破单卡显存限制的底层技术" (typc.net)
+  [0539]  "1. 张量并行：Tensor Parallelism" (0539edu.com news 288531)
+  [PWWT]  "TP到底在切什么——从一次矩阵乘法说起" (pwwt.cn news 5934571)
+
+Readings where the pages are silent or garbled (each is listed in the design doc):
+  * A is split by columns and B by rows ([TYPC] §3 MLP bullet; [0539] §1.2.1);
+    the [PWWT] §2.3 labels are swapped and are not followed.
+  * Post-LN: Y = LN(X + sum_i Act(X A_i) B_i); no LayerNorm on the input.
+  * LayerNorm: biased variance (divide by H), eps inside the square root,
+    Y = (Z - mean) / sqrt(var + eps) * gamma + beta.
+  * GeLU: the tanh form 0.5 u (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3)))
+    (Hendrycks & Gimpel 2016); the erf form 0.5 u (1 + erf(u / sqrt 2)) and
+    ReLU are the other activations ([0539] §1.2.1 names "ReLU or GeLU").
+  * Attention: per head, softmax(Q K^T / sqrt(d)) V, non-causal, no mask,
+    max-subtracted softmax; heads concatenated in head order, then O W_O.
+  * No biases, no dropout.
+
+Parity status: every function below is pinned by tests/test_oracle_pins.py
+(brute force on exact small inputs, closed forms, invariants, library
+special cases); none is "parity unpinned".
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+from scipy.special import erf as _erf
+
+__all__ = [
+    "gelu_tanh", "gelu_erf", "relu", "activation",
+    "layernorm", "mlp_block", "mlp_block_sharded",
+    "linear_column", "linear_row",
+    "attention_heads", "attention_sublayer",
+]
+
+_COL_BLOCK = 2048  # output-column block for products whose fp64 weight copy is large
+
+
+def _f64(a) -> np.ndarray:
+    """Exact widening of the GPU's input values (torch or numpy, bf16/f32) to fp64."""
+    try:
+        import torch
+        if isinstance(a, torch.Tensor):
+            return a.detach().to("cpu").to(torch.float64).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(a, dtype=np.float64)
+
+
+# ---------------------------------------------------------------- activations
+# [0539] §1.2.1: Act is applied elementwise ("ReLU 或 GeLU"), so it can be
+# applied to each column shard on its own.
+
+def gelu_tanh(u: np.ndarray) -> np.ndarray:
+    """tanh-approximated GeLU (Hendrycks & Gimpel 2016)."""
+    c = math.sqrt(2.0 / math.pi)
+    return 0.5 * u * (1.0 + np.tanh(c * (u + 0.044715 * u * u * u)))
+
+
+def gelu_erf(u: np.ndarray) -> np.ndarray:
+    """Exact GeLU, u * Phi(u) written through erf."""
+    return 0.5 * u * (1.0 + _erf(u / math.sqrt(2.0)))
+
+
+def relu(u: np.ndarray) -> np.ndarray:
+    return np.maximum(u, 0.0)
+
+
+_ACTS = {"none": lambda u: u, "gelu_tanh": gelu_tanh, "gelu_erf": gelu_erf, "relu": relu}
+
+
+def activation(u: np.ndarray, act: str) -> np.ndarray:
+    return _ACTS[act](u)
+
+
+# ------------------------------------------------------------------ LayerNorm
+# [PWWT] §2.3 and §5.3: the shard reduction is followed by the residual add and
+# the next LayerNorm, whose row statistics are taken over the full hidden row.
+
+def layernorm(Z: np.ndarray, gamma=None, beta=None, eps: float = 1e-5) -> np.ndarray:
+    Z = np.asarray(Z, dtype=np.float64)
+    H = Z.shape[-1]
+    mean = Z.sum(axis=-1, keepdims=True) / H
+    D = Z - mean
+    var = (D * D).sum(axis=-1, keepdims=True) / H
+    Y = D / np.sqrt(var + eps)
+    if gamma is not None:
+        Y = Y * _f64(gamma)
+    if beta is not None:
+        Y = Y + _f64(beta)
+    return Y
+
+
+# ------------------------------------------------------------------- products
+
+def _matmul_cols(Xr: np.ndarray, W, act: str = "none") -> np.ndarray:
+    """act(Xr @ W) with W widened to fp64 one block of output columns at a time."""
+    n = W.shape[1]
+    out = np.empty((Xr.shape[0], n), dtype=np.float64)
+    for c0 in range(0, n, _COL_BLOCK):
+        c1 = min(n, c0 + _COL_BLOCK)
+        out[:, c0:c1] = activation(Xr @ _f64(W[:, c0:c1]), act)
+    return out
+
+
+def _rows(X, rows):
+    X64 = _f64(X)
+    return X64 if rows is None else X64[np.asarray(rows, dtype=np.int64)]
+
+
+# ---------------------------------------------------------------------- MLP
+# [0539] §1.2.1, eqs (1.2)-(1.5): Y_mlp = Act(X A) B.  Column-splitting A gives
+# Act(X A) = [Act(X A_1) ... Act(X A_t)] ([TYPC] §2.1; [0539] §1.1 列切分), and
+# row-splitting B gives [G_1 ... G_t] B = sum_i G_i B_i ([TYPC] §2.2; [0539]
+# §1.1, eq (1.1) 外积和切分).  The oracle computes the unsplit left-hand sides.
+
+def mlp_block(X, A, B, gamma=None, beta=None, eps: float = 1e-5,
+              act: str = "gelu_tanh", rows=None) -> np.ndarray:
+    """Y = LN(X + Act(X A) B) for the requested rows (all rows if None).
+
+    Each output row depends only on the same row of X, so a row sample is
+    exactly the corresponding rows of the full result."""
+    Xr = _rows(X, rows)
+    G = _matmul_cols(Xr, A, act)          # step 1-2: U = X A, G = Act(U)
+    V = _matmul_cols(G, B)                # step 3:   V = G B
+    Z = Xr + V                            # step 4:   residual
+    return layernorm(Z, gamma, beta, eps)  # step 5:  LayerNorm
+
+
+def mlp_block_sharded(X, A_shards, B_shards, gamma=None, beta=None, eps: float = 1e-5,
+                      act: str = "gelu_tanh", rows=None) -> np.ndarray:
+    """The split form sum_i Act(X A_i) B_i, shard by shard (self-tests only:
+    it checks the block identities the method relies on)."""
+    Xr = _rows(X, rows)
+    acc = np.zeros((Xr.shape[0], _f64(B_shards[0]).shape[1]))
+    for Ai, Bi in zip(A_shards, B_shards):
+        acc += _f64(activation(Xr @ _f64(Ai), act)) @ _f64(Bi)
+    return layernorm(Xr + acc, gamma, beta, eps)
+
+
+# ------------------------------------------------------------ single linears
+# [TYPC] §2.1 / [PWWT] §1.1 figure 1: the column-split linear concatenates
+# X W_i, which equals X W.  [TYPC] §2.2 / [PWWT] §1.2 figure 2: the row-split
+# linear sums X_i W_i (X split by columns, W by rows), which equals X W.
+
+def linear_column(X, W, act: str = "none", rows=None) -> np.ndarray:
+    return _matmul_cols(_rows(X, rows), W, act)
+
+
+def linear_row(X, W, rows=None) -> np.ndarray:
+    return _matmul_cols(_rows(X, rows), W)
+
+
+# ---------------------------------------------------------------- attention
+# [0539] §1.2.2 (eqs (1.6)-(1.13), formulas lost in extraction) and [PWWT]
+# §2.2 figure 4: every head computes softmax(Q_h K_h^T / sqrt(d)) V_h on its own;
+# the heads' outputs are concatenated and multiplied by W_O, which is why W_O
+# is row-split by head ([0539] §1.2.2; [PWWT] §2.1 O 投影).
+
+def attention_heads(Q: np.ndarray, K: np.ndarray, V: np.ndarray, nh: int, d: int) -> np.ndarray:
+    """O = concat_h softmax(Q_h K_h^T / sqrt d) V_h; Q [r, nh*d], K, V [S, nh*d]."""
+    O = np.empty((Q.shape[0], nh * d), dtype=np.float64)
+    scale = 1.0 / math.sqrt(d)
+    for h in range(nh):
+        c = slice(h * d, (h + 1) * d)
+        s = (Q[:, c] @ K[:, c].T) * scale
+        s = s - s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        p = p / p.sum(axis=1, keepdims=True)
+        O[:, c] = p @ V[:, c]
+    return O
+
+
+def attention_sublayer(X, Wqkv, Wo, nh: int, d: int, gamma=None, beta=None,
+                       eps: float = 1e-5, rows=None) -> np.ndarray:
+    """Y = LN(X + concat_h(attn_h) W_O) for the requested query rows.
+
+    Wqkv is [H, 3H] = [W_Q | W_K | W_V]; head h owns columns h*d..(h+1)*d-1 of
+    each block.  K and V are needed for every row; Q only for the sampled rows."""
+    X64 = _f64(X)
+    H = X64.shape[1]
+    assert nh * d == H
+    Xr = X64 if rows is None else X64[np.asarray(rows, dtype=np.int64)]
+    Q = _matmul_cols(Xr, Wqkv[:, 0:H])
+    K = _matmul_cols(X64, Wqkv[:, H:2 * H])
+    V = _matmul_cols(X64, Wqkv[:, 2 * H:3 * H])
+    O = attention_heads(Q, K, V, nh, d)
+    Z = Xr + _matmul_cols(O, Wo)
+    return layernorm(Z, gamma, beta, eps)

@@ -1,0 +1,166 @@
+/*
+ * tpblock — the Megatron tensor-parallel Transformer sublayer on one B200.
+ *
+ *   MLP sublayer:        Y = LN( X + sum_i Act(X A_i) B_i )
+ *   attention sublayer:  Y = LN( X + sum_s O_s Wo_s ),
+ *                        O_s = concat_{h in shard s} softmax(Q_h K_h^T / sqrt d) V_h
+ *
+ * The t tensor-parallel shards are logical partitions held in one GPU's HBM:
+ * the column split's concatenation is a memory layout and the row split's
+ * reduction happens in the tensor-core accumulator or in the fused
+ * reduce + residual + LayerNorm kernel.  No second device, no collective.
+ *
+ * Pages that define the operations (cited by title and section):
+ *   [TYPC] "张量并行：千亿大模型突破单卡显存限制的底层技术" (typc.net)
+ *   [0539] "1. 张量并行：Tensor Parallelism" (0539edu.com news 288531)
+ *   [PWWT] "TP到底在切什么——从一次矩阵乘法说起" (pwwt.cn news 5934571)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  Layout     Row-major everywhere.  Weights use the pages' [in, out] layout
+ *             (Y = X W with X [seq, H], W [H, N]; [PWWT] §1.1).
+ *  Shards     Each shard is its own contiguous device buffer, as the pages'
+ *             weight chunking makes one ([PWWT] §3.1).  `*_shards` arguments
+ *             are HOST arrays of t DEVICE pointers.  1 <= t <= TP_MAX_SHARDS.
+ *  Ownership  Every pointer is owned by the caller.  The library allocates
+ *             no device memory: scratch comes from the caller's `workspace`,
+ *             sized by the matching *_workspace_bytes() query.
+ *  Alignment  Every device pointer must be 16-byte aligned.
+ *  Ordering   Work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ *             default stream).  No call synchronises; results are valid once
+ *             the caller has synchronised the stream.
+ *  Errors     Arguments are checked before anything is launched; a failed
+ *             check returns its status and enqueues nothing.  A CUDA launch
+ *             error returns TP_ERR_CUDA.  Every device-side wait is bounded:
+ *             if one gives up, the kernel returns early and tp_device_error()
+ *             reports TP_ERR_TIMEOUT after the stream is synchronised.  No C++
+ *             exception crosses this interface.
+ *  Types      dtype TP_DTYPE_BF16: bf16 storage, f32 accumulation on the
+ *             tensor cores (tcgen05).  dtype TP_DTYPE_F32: f32 storage and
+ *             f32 CUDA-core arithmetic.  gamma/beta are always f32 (NULL means
+ *             gamma = 1, beta = 0).
+ */
+#ifndef TPBLOCK_H_
+#define TPBLOCK_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TP_MAX_SHARDS 8
+#define TP_API_VERSION 1
+
+typedef enum {
+  TP_OK = 0,
+  TP_ERR_INVALID_ARG = 1,        /* null pointer, t out of range, bad enum, misaligned pointer */
+  TP_ERR_UNSUPPORTED_SHAPE = 2,  /* shape outside the supported set (see each entry point) */
+  TP_ERR_WORKSPACE_TOO_SMALL = 3,
+  TP_ERR_CUDA = 4,               /* a CUDA runtime/driver call failed */
+  TP_ERR_TIMEOUT = 5,            /* a bounded device-side wait gave up (tp_device_error) */
+  TP_ERR_NO_DEVICE = 6           /* no sm_100 device current */
+} tp_status;
+
+typedef enum { TP_DTYPE_F32 = 0, TP_DTYPE_BF16 = 1 } tp_dtype;
+
+/* Elementwise activation between the two MLP products ([0539] §1.2.1: "ReLU 或
+ * GeLU").  GELU_TANH: 0.5 u (1 + tanh(sqrt(2/pi) (u + 0.044715 u^3)));
+ * GELU_ERF: 0.5 u (1 + erf(u / sqrt 2)); RELU: max(u, 0). */
+typedef enum { TP_ACT_NONE = 0, TP_ACT_GELU_TANH = 1, TP_ACT_GELU_ERF = 2, TP_ACT_RELU = 3 } tp_act;
+
+/* Library version (TP_API_VERSION) and a static string for a status code. */
+int tp_version(void);
+const char* tp_status_string(int status);
+
+/* Reads and clears the device-side error word of the current device (0 when no
+ * bounded wait gave up).  Call after synchronising the streams that ran the
+ * library's kernels.  Returns TP_OK or TP_ERR_TIMEOUT (or TP_ERR_CUDA). */
+int tp_device_error(void);
+
+/* ------------------------------------------------------------------ MLP ----
+ * Y = LN(X + sum_i Act(X A_i) B_i), post-LN, no biases, no dropout.
+ * [0539] §1.2.1 eqs (1.2)-(1.5) (Act(X A) B with A column-split and B
+ * row-split, one reduction); [TYPC] §3 (MLP: column split then row split);
+ * [PWWT] §2.3 (the reduction fused with the residual add and the next
+ * LayerNorm's statistics).
+ *
+ *   S, H, F   sequence rows, hidden size, FFN size; F % t == 0.
+ *   X         [S, H] dtype.
+ *   A_shards  t pointers, A_i = columns [i F/t, (i+1) F/t) of A [H, F]: [H, F/t].
+ *   B_shards  t pointers, B_i = rows    [i F/t, (i+1) F/t) of B [F, H]: [F/t, H].
+ *   gamma, beta  [H] f32 or NULL.  eps > 0.
+ *   Y         [S, H] out_dtype (bf16 or f32 for dtype bf16; f32 for dtype f32).
+ *   workspace caller-owned device scratch of >= tp_mlp_workspace_bytes().
+ * Supported: S >= 1; H % 8 == 0 and 8 <= H <= 16384; (F/t) % 8 == 0.
+ * Kernels (bf16): column-split GEMM with the activation in its epilogue
+ * (writes Act(X A_i) into its column slice of a [S, F] bf16 buffer), row-split
+ * GEMM summing every shard in the TMEM accumulator ([S, H] f32), then the
+ * reduce + residual + LayerNorm kernel. */
+size_t tp_mlp_workspace_bytes(int S, int H, int F, int t, int dtype);
+int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype,
+                   const void* X, const void* const* A_shards, const void* const* B_shards,
+                   const float* gamma, const float* beta, float eps, int act,
+                   void* Y, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------------ attention ----
+ * Y = LN(X + concat_h(softmax(Q_h K_h^T / sqrt d) V_h) Wo), non-causal, no
+ * mask, heads split over t shards of nh/t heads.  [0539] §1.2.2 (every head
+ * is independent; W_O row-split by head; one reduction); [TYPC] §3 (64 heads
+ * on 4 shards, 16 per shard); [PWWT] §2.1-§2.2 (QKV column-split, O row-split).
+ *
+ *   Full weights: Wqkv = [W_Q | W_K | W_V], [H, 3H], head j in columns
+ *   j d .. j d + d - 1 of each block; Wo [H, H], rows in the same head order.
+ *   Wqkv_shards[s]: [H, 3 (nh/t) d] = [Q cols of shard s's heads | K cols | V cols].
+ *   Wo_shards[s]:   [(nh/t) d, H] = rows s (nh/t) d .. of Wo.
+ *   X [S, H] bf16; Y [S, H] out_dtype; gamma, beta [H] f32 or NULL.
+ * Supported: dtype bf16; d == 128; H == nh * d; nh % t == 0; S % 128 == 0;
+ * H <= 16384. */
+size_t tp_attn_workspace_bytes(int S, int H, int nh, int d, int t, int dtype);
+int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int out_dtype,
+                              const void* X, const void* const* Wqkv_shards, const void* const* Wo_shards,
+                              const float* gamma, const float* beta, float eps,
+                              void* Y, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------------------------ single linears ----
+ * Column-split linear ([TYPC] §2.1; [PWWT] §1.1 figure 1; [0539] §1.1 列切分):
+ *   Y[:, i N/t : (i+1) N/t] = Act(X W_i),  X [M, K], W_i [K, N/t]  (concat in place).
+ * Row-split linear ([TYPC] §2.2; [PWWT] §1.2 figure 2; [0539] eq. (1.1)):
+ *   Y = sum_i X[:, i K/t : (i+1) K/t] W_i,  X [M, K] (full), W_i [K/t, N].
+ * Y is [M, N] out_dtype (bf16 or f32; f32 only for dtype f32).
+ * Supported: M >= 1; K % 8 == 0, N % 8 == 0, (N/t) % 8 (column) or (K/t) % 8
+ * (row) == 0.  The row-split linear accumulates every shard in the tensor-core
+ * accumulator and needs no workspace (workspace may be NULL). */
+int tp_linear_column_forward(int M, int K, int N, int t, int dtype, int out_dtype,
+                             const void* X, const void* const* W_shards, int act,
+                             void* Y, void* stream);
+int tp_linear_row_forward(int M, int K, int N, int t, int dtype, int out_dtype,
+                          const void* X, const void* const* W_shards,
+                          void* Y, void* workspace, size_t workspace_bytes, void* stream);
+
+/* ------------------------------------- reduce + residual + LayerNorm ----
+ * Y = LN(X + sum_{p < nparts} P_p) per row over H ([PWWT] §2.3, §5.3): mean,
+ * then the biased variance (divide by H), eps inside the square root.
+ *   parts  nparts f32 buffers [S, H] laid out back to back (may be NULL if
+ *          nparts == 0).  X [S, H] x_dtype; Y [S, H] out_dtype.
+ * Supported: H % 8 == 0, 8 <= H <= 16384. */
+int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts,
+                                 const void* X, int x_dtype, const float* gamma, const float* beta,
+                                 float eps, void* Y, int out_dtype, void* stream);
+
+/* ----------------------------------------------------- kernel timing ----
+ * When enabled, every kernel the library launches is bracketed by CUDA events
+ * recorded on its stream (at most 4096 launches between two collects).
+ * tp_profile_collect synchronises those events, writes per kernel kind the
+ * launch count and summed device milliseconds (kinds: 0 tensor-core GEMM,
+ * 1 reduce+residual+LayerNorm, 2 f32 CUDA-core GEMM, 3 attention), and
+ * clears the record.  Returns the number of kinds written (<= max_kinds). */
+int tp_profile_enable(int on);
+int tp_profile_collect(int* launches, double* ms, int max_kinds);
+const char* tp_kernel_kind_name(int kind);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TPBLOCK_H_ */

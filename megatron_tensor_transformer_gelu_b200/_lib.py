@@ -1,0 +1,169 @@
+"""ctypes binding of libtpblock.so (argument marshalling only).
+
+Every step of the sublayer runs in the library's CUDA kernels; this module
+only turns torch tensors into pointers and sizes and maps status codes to
+exceptions.  If the library is missing it raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtpblock.so")
+
+TP_OK = 0
+STATUS = {
+    0: "TP_OK", 1: "TP_ERR_INVALID_ARG", 2: "TP_ERR_UNSUPPORTED_SHAPE",
+    3: "TP_ERR_WORKSPACE_TOO_SMALL", 4: "TP_ERR_CUDA", 5: "TP_ERR_TIMEOUT", 6: "TP_ERR_NO_DEVICE",
+}
+DTYPE = {torch.float32: 0, torch.bfloat16: 1}
+ACT = {"none": 0, "gelu_tanh": 1, "gelu_erf": 2, "relu": 3}
+MAX_SHARDS = 8
+
+# name -> (restype, argtypes)
+_c_int, _c_size, _c_float, _vp = ctypes.c_int, ctypes.c_size_t, ctypes.c_float, ctypes.c_void_p
+_vpp = ctypes.POINTER(ctypes.c_void_p)
+SIGNATURES = {
+    "tp_version": (_c_int, []),
+    "tp_status_string": (ctypes.c_char_p, [_c_int]),
+    "tp_device_error": (_c_int, []),
+    "tp_mlp_workspace_bytes": (_c_size, [_c_int] * 5),
+    "tp_mlp_forward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vpp, _vp, _vp, _c_float, _c_int, _vp, _vp, _c_size, _vp]),
+    "tp_attn_workspace_bytes": (_c_size, [_c_int] * 6),
+    "tp_qkv_attn_oproj_forward": (_c_int, [_c_int] * 7 + [_vp, _vpp, _vpp, _vp, _vp, _c_float, _vp, _vp, _c_size, _vp]),
+    "tp_linear_column_forward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _c_int, _vp, _vp]),
+    "tp_linear_row_forward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vp, _vp, _c_size, _vp]),
+    "tp_reduce_residual_layernorm": (_c_int, [_c_int] * 3 + [_vp, _vp, _c_int, _vp, _vp, _c_float, _vp, _c_int, _vp]),
+    "tp_profile_enable": (_c_int, [_c_int]),
+    "tp_profile_collect": (_c_int, [ctypes.POINTER(_c_int), ctypes.POINTER(ctypes.c_double), _c_int]),
+    "tp_kernel_kind_name": (ctypes.c_char_p, [_c_int]),
+}
+
+_lib = None
+
+
+class TPError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load libtpblock.so (built by ``build()``); raise if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is not built: run megatron_tensor_transformer_gelu_b200.build")
+        l = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(l, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = l
+    return _lib
+
+
+def _check(code: int, where: str):
+    if code != TP_OK:
+        raise TPError(code, where)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _ptrs(ts):
+    arr = (ctypes.c_void_p * len(ts))(*[t.data_ptr() for t in ts])
+    return ctypes.cast(arr, _vpp), arr
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def mlp_workspace_bytes(S, H, F, t, dtype) -> int:
+    return lib().tp_mlp_workspace_bytes(S, H, F, t, DTYPE[dtype])
+
+
+def attn_workspace_bytes(S, H, nh, d, t, dtype=torch.bfloat16) -> int:
+    return lib().tp_attn_workspace_bytes(S, H, nh, d, t, DTYPE[dtype])
+
+
+def mlp_forward(X, A_shards, B_shards, Y, workspace, gamma=None, beta=None, eps=1e-5,
+                act="gelu_tanh", stream=None):
+    S, H = X.shape
+    t = len(A_shards)
+    F = sum(a.shape[1] for a in A_shards)
+    pa, ka = _ptrs(A_shards)
+    pb, kb = _ptrs(B_shards)
+    code = lib().tp_mlp_forward(S, H, F, t, DTYPE[X.dtype], DTYPE[Y.dtype], _ptr(X), pa, pb,
+                                _ptr(gamma), _ptr(beta), float(eps), ACT[act], _ptr(Y),
+                                _ptr(workspace), workspace.numel() * workspace.element_size()
+                                if workspace is not None else 0, _stream(stream))
+    _check(code, "tp_mlp_forward")
+
+
+def attn_forward(X, Wqkv_shards, Wo_shards, nh, d, Y, workspace, gamma=None, beta=None, eps=1e-5,
+                 stream=None):
+    S, H = X.shape
+    t = len(Wqkv_shards)
+    pq, kq = _ptrs(Wqkv_shards)
+    po, ko = _ptrs(Wo_shards)
+    code = lib().tp_qkv_attn_oproj_forward(S, H, nh, d, t, DTYPE[X.dtype], DTYPE[Y.dtype], _ptr(X), pq, po,
+                                           _ptr(gamma), _ptr(beta), float(eps), _ptr(Y), _ptr(workspace),
+                                           workspace.numel() * workspace.element_size()
+                                           if workspace is not None else 0, _stream(stream))
+    _check(code, "tp_qkv_attn_oproj_forward")
+
+
+def linear_column_forward(X, W_shards, Y, act="none", stream=None):
+    M, K = X.shape
+    t = len(W_shards)
+    N = sum(w.shape[1] for w in W_shards)
+    pw, kw = _ptrs(W_shards)
+    code = lib().tp_linear_column_forward(M, K, N, t, DTYPE[X.dtype], DTYPE[Y.dtype], _ptr(X), pw, ACT[act],
+                                          _ptr(Y), _stream(stream))
+    _check(code, "tp_linear_column_forward")
+
+
+def linear_row_forward(X, W_shards, Y, stream=None):
+    M, K = X.shape
+    t = len(W_shards)
+    N = W_shards[0].shape[1]
+    pw, kw = _ptrs(W_shards)
+    code = lib().tp_linear_row_forward(M, K, N, t, DTYPE[X.dtype], DTYPE[Y.dtype], _ptr(X), pw, _ptr(Y),
+                                       None, 0, _stream(stream))
+    _check(code, "tp_linear_row_forward")
+
+
+def reduce_residual_layernorm(parts, X, Y, gamma=None, beta=None, eps=1e-5, stream=None):
+    """parts: None or an f32 tensor [nparts, S, H] (contiguous)."""
+    S, H = X.shape
+    nparts = 0 if parts is None else parts.shape[0]
+    code = lib().tp_reduce_residual_layernorm(S, H, nparts, _ptr(parts), _ptr(X), DTYPE[X.dtype], _ptr(gamma),
+                                              _ptr(beta), float(eps), _ptr(Y), DTYPE[Y.dtype], _stream(stream))
+    _check(code, "tp_reduce_residual_layernorm")
+
+
+def device_error() -> int:
+    return lib().tp_device_error()
+
+
+def profile_enable(on: bool):
+    _check(lib().tp_profile_enable(1 if on else 0), "tp_profile_enable")
+
+
+def profile_collect(nkinds: int = 4):
+    launches = (ctypes.c_int * nkinds)()
+    ms = (ctypes.c_double * nkinds)()
+    n = lib().tp_profile_collect(launches, ms, nkinds)
+    if n < 0:
+        raise TPError(-n, "tp_profile_collect")
+    return {lib().tp_kernel_kind_name(k).decode(): (launches[k], ms[k]) for k in range(n)}

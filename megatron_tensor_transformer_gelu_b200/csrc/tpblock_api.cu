@@ -1,0 +1,469 @@
+// C ABI of the tensor-parallel sublayer library (declared in include/tpblock.h).
+//
+// Host side only: argument checks, workspace carving, TMA tensor-map encoding,
+// launch sequencing on the caller's stream, optional per-kernel event timing.
+// Every step of the computation runs in this library's kernels.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/tpblock.h"
+#include "attention.cuh"
+#include "gemm_tcgen05.cuh"
+#include "reduce_ln.cuh"
+#include "simt_f32.cuh"
+
+namespace {
+
+using tp::MAX_SHARDS;
+static_assert(MAX_SHARDS == TP_MAX_SHARDS, "shard limit mismatch");
+
+constexpr int MAX_DEVICES = 64;
+
+struct DeviceInfo {
+  bool ready = false;
+  bool ok = false;
+  int sm_count = 0;
+};
+
+std::mutex g_mu;
+DeviceInfo g_dev[MAX_DEVICES];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+// ------------------------------------------------------------ event timing
+constexpr int PROF_CAP = 4096;
+constexpr int PROF_KINDS = 4;
+bool g_prof_on = false;
+bool g_prof_events_made = false;
+cudaEvent_t g_ev_start[PROF_CAP];
+cudaEvent_t g_ev_stop[PROF_CAP];
+int g_prof_kind[PROF_CAP];
+int g_prof_n = 0;
+
+enum Kind { K_GEMM_TC = 0, K_REDUCE_LN = 1, K_GEMM_SIMT = 2, K_ATTN = 3 };
+
+struct ProfScope {
+  int slot = -1;
+  cudaStream_t st;
+  ProfScope(int kind, cudaStream_t s) : st(s) {
+    if (!g_prof_on || g_prof_n >= PROF_CAP) return;
+    slot = g_prof_n++;
+    g_prof_kind[slot] = kind;
+    cudaEventRecord(g_ev_start[slot], st);
+  }
+  ~ProfScope() {
+    if (slot >= 0) cudaEventRecord(g_ev_stop[slot], st);
+  }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+// Resolve the current device's properties and the tensor-map encoder once.
+int device_ready(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return TP_ERR_NO_DEVICE;
+  if (dev < 0 || dev >= MAX_DEVICES) return TP_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    d.ready = true;
+    int major = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      d.ok = false;
+    } else {
+      d.ok = (major == 10);
+      d.sm_count = sms;
+    }
+    if (d.ok) {
+      if (cudaFuncSetAttribute(tp::gemm_tcgen05_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tp::gemm::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(tp::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tp::attn::SMEM_BYTES) != cudaSuccess)
+        d.ok = false;
+    }
+    if (d.ok && !g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        d.ok = false;
+      else
+        g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  if (!d.ok) return TP_ERR_NO_DEVICE;
+  *out = &d;
+  return TP_OK;
+}
+
+// 2-D bf16 tensor map over a row-major matrix [rows, cols] with a row stride of
+// `ld` elements; box {box_cols, box_rows}; 128-byte swizzle; OOB reads give 0.
+bool tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long cols, long long ld, int box_cols,
+               int box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(ld) * 2u};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_cols), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA; }
+
+// Tensor-core GEMM.  Column mode: B shard s is [K, shard_n], output columns
+// [s*shard_n, (s+1)*shard_n).  Row mode: B shard s is [shard_k, shard_n] and
+// multiplies A's columns [s*shard_k, (s+1)*shard_k); all shards are summed.
+int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, const void* const* B, int t,
+                int row_mode, int shard_k, int shard_n, void* C, long long ldc, int out_f32, int act,
+                cudaStream_t st) {
+  using namespace tp::gemm;
+  if (M == 0) return TP_OK;
+  tp::GemmArgs p;
+  std::memset(&p, 0, sizeof(p));
+  const long long K_total = row_mode ? static_cast<long long>(shard_k) * t : shard_k;
+  if (!tmap_bf16(&p.tmA, A, M, K_total, lda, BK, BM)) return TP_ERR_CUDA;
+  for (int s = 0; s < t; ++s)
+    if (!tmap_bf16(&p.tmB[s], B[s], shard_k, shard_n, shard_n, B_BOX_N, BK)) return TP_ERR_CUDA;
+  p.C = C;
+  p.ldc = ldc;
+  p.M = M;
+  p.t = t;
+  p.row_mode = row_mode;
+  p.shard_n = shard_n;
+  p.shard_k = shard_k;
+  p.m_blocks = ceil_div(M, BM);
+  if (row_mode) {
+    p.N = shard_n;
+    p.n_blocks = ceil_div(shard_n, BN);
+    p.n_blocks_per_shard = p.n_blocks;
+    p.k_blocks_per_shard = ceil_div(shard_k, BK);
+    p.k_blocks = p.k_blocks_per_shard * t;
+  } else {
+    p.N = shard_n * t;
+    p.n_blocks_per_shard = ceil_div(shard_n, BN);
+    p.n_blocks = p.n_blocks_per_shard * t;
+    p.k_blocks_per_shard = ceil_div(shard_k, BK);
+    p.k_blocks = p.k_blocks_per_shard;
+  }
+  p.act = act;
+  p.out_f32 = out_f32;
+  const long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks;
+  const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
+  ProfScope ps(K_GEMM_TC, st);
+  tp::gemm_tcgen05_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
+  return launch_status();
+}
+
+int run_gemm_simt(const float* A, long long lda, int M, const void* const* B, int t, int row_mode, int shard_k,
+                  int shard_n, float* C, long long ldc, int act, cudaStream_t st) {
+  if (M == 0) return TP_OK;
+  tp::SimtArgs p;
+  std::memset(&p, 0, sizeof(p));
+  p.A = A;
+  p.lda = lda;
+  for (int s = 0; s < t; ++s) p.B[s] = static_cast<const float*>(B[s]);
+  p.C = C;
+  p.ldc = ldc;
+  p.M = M;
+  p.row_mode = row_mode;
+  p.shard_n = shard_n;
+  p.shard_k = shard_k;
+  p.N = row_mode ? shard_n : shard_n * t;
+  p.K = row_mode ? shard_k * t : shard_k;
+  p.act = act;
+  dim3 grid(ceil_div(p.N, tp::simt::TN), ceil_div(M, tp::simt::TM));
+  ProfScope ps(K_GEMM_SIMT, st);
+  tp::simt_gemm_f32_kernel<<<grid, tp::simt::THREADS, 0, st>>>(p);
+  return launch_status();
+}
+
+int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, int x_bf16, const float* gamma,
+                  const float* beta, float eps, void* Y, int y_bf16, cudaStream_t st) {
+  if (S == 0) return TP_OK;
+  tp::ReduceLnArgs p;
+  p.S = S;
+  p.H = H;
+  p.nparts = nparts;
+  p.parts = parts;
+  p.part_stride = static_cast<long long>(S) * H;
+  p.X = X;
+  p.x_bf16 = x_bf16;
+  p.gamma = gamma;
+  p.beta = beta;
+  p.eps = eps;
+  p.Y = Y;
+  p.y_bf16 = y_bf16;
+  const int chunks = ceil_div(H, 8 * tp::rln::THREADS);
+  ProfScope ps(K_REDUCE_LN, st);
+  if (chunks <= 1) tp::reduce_residual_ln_kernel<1><<<S, tp::rln::THREADS, 0, st>>>(p);
+  else if (chunks <= 2) tp::reduce_residual_ln_kernel<2><<<S, tp::rln::THREADS, 0, st>>>(p);
+  else if (chunks <= 4) tp::reduce_residual_ln_kernel<4><<<S, tp::rln::THREADS, 0, st>>>(p);
+  else tp::reduce_residual_ln_kernel<8><<<S, tp::rln::THREADS, 0, st>>>(p);
+  return launch_status();
+}
+
+bool valid_dtype(int d) { return d == TP_DTYPE_F32 || d == TP_DTYPE_BF16; }
+bool valid_act(int a) { return a >= TP_ACT_NONE && a <= TP_ACT_RELU; }
+bool valid_out(int dtype, int out) {
+  if (!valid_dtype(dtype) || !valid_dtype(out)) return false;
+  return dtype == TP_DTYPE_BF16 || out == TP_DTYPE_F32;
+}
+bool shards_ok(const void* const* s, int t) {
+  if (!s) return false;
+  for (int i = 0; i < t; ++i)
+    if (!s[i] || !aligned16(s[i])) return false;
+  return true;
+}
+bool ptr_ok(const void* p) { return p && aligned16(p); }
+bool opt_ptr_ok(const void* p) { return !p || aligned16(p); }
+bool hidden_ok(int H) { return H >= 8 && H % 8 == 0 && H <= 8 * tp::rln::THREADS * tp::rln::MAX_CHUNKS; }
+
+}  // namespace
+
+extern "C" {
+
+int tp_version(void) { return TP_API_VERSION; }
+
+const char* tp_status_string(int s) {
+  switch (s) {
+    case TP_OK: return "ok";
+    case TP_ERR_INVALID_ARG: return "invalid argument";
+    case TP_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case TP_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case TP_ERR_CUDA: return "CUDA error";
+    case TP_ERR_TIMEOUT: return "device-side wait timed out";
+    case TP_ERR_NO_DEVICE: return "no sm_100 device";
+    default: return "unknown status";
+  }
+}
+
+int tp_device_error(void) {
+  DeviceInfo* dev = nullptr;
+  int st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, tp::g_tp_device_error, sizeof(int)) != cudaSuccess) return TP_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(tp::g_tp_device_error, &zero, sizeof(int)) != cudaSuccess) return TP_ERR_CUDA;
+  return v == 0 ? TP_OK : TP_ERR_TIMEOUT;
+}
+
+// ------------------------------------------------------------------- MLP
+size_t tp_mlp_workspace_bytes(int S, int H, int F, int t, int dtype) {
+  if (S < 0 || H <= 0 || F <= 0 || t < 1 || !valid_dtype(dtype)) return 0;
+  (void)t;
+  const size_t eh = dtype == TP_DTYPE_BF16 ? 2 : 4;
+  return align256(static_cast<size_t>(S) * F * eh) + static_cast<size_t>(S) * H * 4;
+}
+
+int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype, const void* X,
+                   const void* const* A_shards, const void* const* B_shards, const float* gamma,
+                   const float* beta, float eps, int act, void* Y, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  if (t < 1 || t > TP_MAX_SHARDS || S < 0 || H <= 0 || F <= 0) return TP_ERR_INVALID_ARG;
+  if (!valid_out(dtype, out_dtype) || !valid_act(act) || !(eps > 0.0f) || !std::isfinite(eps))
+    return TP_ERR_INVALID_ARG;
+  if (!ptr_ok(X) || !ptr_ok(Y) || !shards_ok(A_shards, t) || !shards_ok(B_shards, t) || !opt_ptr_ok(gamma) ||
+      !opt_ptr_ok(beta) || !opt_ptr_ok(workspace))
+    return TP_ERR_INVALID_ARG;
+  if (F % t != 0 || (F / t) % 8 != 0 || !hidden_ok(H)) return TP_ERR_UNSUPPORTED_SHAPE;
+  const size_t need = tp_mlp_workspace_bytes(S, H, F, t, dtype);
+  if (workspace_bytes < need || (need > 0 && !workspace)) return TP_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  int st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  if (S == 0) return TP_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int Fs = F / t;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t eh = dtype == TP_DTYPE_BF16 ? 2 : 4;
+  void* Hbuf = ws;
+  float* Zsum = reinterpret_cast<float*>(ws + align256(static_cast<size_t>(S) * F * eh));
+  if (dtype == TP_DTYPE_BF16) {
+    // H_i = Act(X A_i) into columns [i Fs, (i+1) Fs) of Hbuf [S, F] (bf16).
+    st = run_gemm_tc(*dev, X, H, S, A_shards, t, /*row_mode=*/0, /*shard_k=*/H, /*shard_n=*/Fs, Hbuf, F,
+                     /*out_f32=*/0, act, s);
+    if (st != TP_OK) return st;
+    // Zsum = sum_i H_i B_i, accumulated in TMEM across the shards (f32).
+    st = run_gemm_tc(*dev, Hbuf, F, S, B_shards, t, /*row_mode=*/1, /*shard_k=*/Fs, /*shard_n=*/H, Zsum, H,
+                     /*out_f32=*/1, TP_ACT_NONE, s);
+    if (st != TP_OK) return st;
+  } else {
+    st = run_gemm_simt(static_cast<const float*>(X), H, S, A_shards, t, 0, H, Fs, static_cast<float*>(Hbuf), F,
+                       act, s);
+    if (st != TP_OK) return st;
+    st = run_gemm_simt(static_cast<const float*>(Hbuf), F, S, B_shards, t, 1, Fs, H, Zsum, H, TP_ACT_NONE, s);
+    if (st != TP_OK) return st;
+  }
+  return run_reduce_ln(S, H, 1, Zsum, X, dtype == TP_DTYPE_BF16, gamma, beta, eps, Y,
+                       out_dtype == TP_DTYPE_BF16, s);
+}
+
+// -------------------------------------------------------------- attention
+size_t tp_attn_workspace_bytes(int S, int H, int nh, int d, int t, int dtype) {
+  if (S < 0 || H <= 0 || nh <= 0 || d <= 0 || t < 1 || dtype != TP_DTYPE_BF16) return 0;
+  const size_t s = static_cast<size_t>(S), h = static_cast<size_t>(H);
+  return align256(s * 3 * h * 2) + align256(s * h * 2) + s * h * 4;
+}
+
+int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int out_dtype, const void* X,
+                              const void* const* Wqkv_shards, const void* const* Wo_shards, const float* gamma,
+                              const float* beta, float eps, void* Y, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  if (t < 1 || t > TP_MAX_SHARDS || S < 0 || H <= 0 || nh <= 0 || d <= 0) return TP_ERR_INVALID_ARG;
+  if (dtype != TP_DTYPE_BF16 || !valid_out(dtype, out_dtype) || !(eps > 0.0f) || !std::isfinite(eps))
+    return TP_ERR_INVALID_ARG;
+  if (!ptr_ok(X) || !ptr_ok(Y) || !shards_ok(Wqkv_shards, t) || !shards_ok(Wo_shards, t) || !opt_ptr_ok(gamma) ||
+      !opt_ptr_ok(beta) || !opt_ptr_ok(workspace))
+    return TP_ERR_INVALID_ARG;
+  if (d != tp::attn::D || static_cast<long long>(nh) * d != H || nh % t != 0 || S % tp::attn::BQ != 0 ||
+      !hidden_ok(H))
+    return TP_ERR_UNSUPPORTED_SHAPE;
+  const size_t need = tp_attn_workspace_bytes(S, H, nh, d, t, dtype);
+  if (workspace_bytes < need || (need > 0 && !workspace)) return TP_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  int st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  if (S == 0) return TP_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int Hs = H / t;  // columns of one shard's heads
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* QKV = ws;                                                            // [S, 3H] bf16
+  void* Obuf = ws + align256(static_cast<size_t>(S) * 3 * H * 2);            // [S, H]  bf16
+  float* Zsum = reinterpret_cast<float*>(static_cast<uint8_t*>(Obuf) + align256(static_cast<size_t>(S) * H * 2));
+  // [Q_s | K_s | V_s] = X Wqkv_s into columns [3 s Hs, 3 (s+1) Hs) of QKV.
+  st = run_gemm_tc(*dev, X, H, S, Wqkv_shards, t, 0, H, 3 * Hs, QKV, 3LL * H, 0, TP_ACT_NONE, s);
+  if (st != TP_OK) return st;
+  // O_h = softmax(Q_h K_h^T / sqrt d) V_h, written to columns [h d, (h+1) d) of O.
+  {
+    tp::AttnArgs a;
+    std::memset(&a, 0, sizeof(a));
+    const int nhs = nh / t;
+    // Q/K/V boxes: 64 columns (128 B) x BQ or BKV rows of the [S, 3H] buffer.
+    if (!tmap_bf16(&a.tmQKV, QKV, S, 3LL * H, 3LL * H, 64, tp::attn::BQ)) return TP_ERR_CUDA;
+    a.O = Obuf;
+    a.S = S;
+    a.H = H;
+    a.nh = nh;
+    a.heads_per_shard = nhs;
+    a.shard_cols = 3 * Hs;
+    a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+    dim3 grid(S / tp::attn::BQ, nh);
+    ProfScope ps(K_ATTN, s);
+    tp::attn_fwd_kernel<<<grid, tp::attn::NUM_THREADS, tp::attn::SMEM_BYTES, s>>>(a);
+    st = launch_status();
+    if (st != TP_OK) return st;
+  }
+  // sum_s O_s Wo_s, the O projection row-split by head, summed in TMEM.
+  st = run_gemm_tc(*dev, Obuf, H, S, Wo_shards, t, 1, Hs, H, Zsum, H, 1, TP_ACT_NONE, s);
+  if (st != TP_OK) return st;
+  return run_reduce_ln(S, H, 1, Zsum, X, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s);
+}
+
+// ---------------------------------------------------------------- linears
+int tp_linear_column_forward(int M, int K, int N, int t, int dtype, int out_dtype, const void* X,
+                             const void* const* W_shards, int act, void* Y, void* stream) {
+  if (t < 1 || t > TP_MAX_SHARDS || M < 0 || K <= 0 || N <= 0) return TP_ERR_INVALID_ARG;
+  if (!valid_out(dtype, out_dtype) || !valid_act(act)) return TP_ERR_INVALID_ARG;
+  if (!ptr_ok(X) || !ptr_ok(Y) || !shards_ok(W_shards, t)) return TP_ERR_INVALID_ARG;
+  if (K % 8 != 0 || N % t != 0 || (N / t) % 8 != 0) return TP_ERR_UNSUPPORTED_SHAPE;
+  DeviceInfo* dev = nullptr;
+  int st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == TP_DTYPE_BF16)
+    return run_gemm_tc(*dev, X, K, M, W_shards, t, 0, K, N / t, Y, N, out_dtype == TP_DTYPE_F32, act, s);
+  return run_gemm_simt(static_cast<const float*>(X), K, M, W_shards, t, 0, K, N / t, static_cast<float*>(Y), N,
+                       act, s);
+}
+
+int tp_linear_row_forward(int M, int K, int N, int t, int dtype, int out_dtype, const void* X,
+                          const void* const* W_shards, void* Y, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (t < 1 || t > TP_MAX_SHARDS || M < 0 || K <= 0 || N <= 0) return TP_ERR_INVALID_ARG;
+  if (!valid_out(dtype, out_dtype)) return TP_ERR_INVALID_ARG;
+  if (!ptr_ok(X) || !ptr_ok(Y) || !shards_ok(W_shards, t)) return TP_ERR_INVALID_ARG;
+  if (K % t != 0 || (K / t) % 8 != 0 || N % 8 != 0) return TP_ERR_UNSUPPORTED_SHAPE;
+  DeviceInfo* dev = nullptr;
+  int st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == TP_DTYPE_BF16)
+    return run_gemm_tc(*dev, X, K, M, W_shards, t, 1, K / t, N, Y, N, out_dtype == TP_DTYPE_F32, TP_ACT_NONE, s);
+  return run_gemm_simt(static_cast<const float*>(X), K, M, W_shards, t, 1, K / t, N, static_cast<float*>(Y), N,
+                       TP_ACT_NONE, s);
+}
+
+// -------------------------------------------- reduce + residual + LayerNorm
+int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts, const void* X, int x_dtype,
+                                 const float* gamma, const float* beta, float eps, void* Y, int out_dtype,
+                                 void* stream) {
+  if (S < 0 || nparts < 0 || !valid_dtype(x_dtype) || !valid_dtype(out_dtype) || !(eps > 0.0f) ||
+      !std::isfinite(eps))
+    return TP_ERR_INVALID_ARG;
+  if (!ptr_ok(X) || !ptr_ok(Y) || (nparts > 0 && !ptr_ok(parts)) || !opt_ptr_ok(gamma) || !opt_ptr_ok(beta))
+    return TP_ERR_INVALID_ARG;
+  if (!hidden_ok(H)) return TP_ERR_UNSUPPORTED_SHAPE;
+  DeviceInfo* dev = nullptr;
+  int st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  return run_reduce_ln(S, H, nparts, parts, X, x_dtype == TP_DTYPE_BF16, gamma, beta, eps, Y,
+                       out_dtype == TP_DTYPE_BF16, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------- profiling
+int tp_profile_enable(int on) {
+  if (on && !g_prof_events_made) {
+    for (int i = 0; i < PROF_CAP; ++i) {
+      if (cudaEventCreate(&g_ev_start[i]) != cudaSuccess || cudaEventCreate(&g_ev_stop[i]) != cudaSuccess)
+        return TP_ERR_CUDA;
+    }
+    g_prof_events_made = true;
+  }
+  g_prof_on = on != 0;
+  g_prof_n = 0;
+  return TP_OK;
+}
+
+int tp_profile_collect(int* launches, double* ms, int max_kinds) {
+  const int nk = max_kinds < PROF_KINDS ? max_kinds : PROF_KINDS;
+  for (int k = 0; k < nk; ++k) {
+    if (launches) launches[k] = 0;
+    if (ms) ms[k] = 0.0;
+  }
+  for (int i = 0; i < g_prof_n; ++i) {
+    const int k = g_prof_kind[i];
+    if (k >= nk) continue;
+    float t = 0.0f;
+    if (cudaEventSynchronize(g_ev_stop[i]) != cudaSuccess ||
+        cudaEventElapsedTime(&t, g_ev_start[i], g_ev_stop[i]) != cudaSuccess)
+      return -TP_ERR_CUDA;
+    if (launches) launches[k] += 1;
+    if (ms) ms[k] += t;
+  }
+  g_prof_n = 0;
+  return nk;
+}
+
+const char* tp_kernel_kind_name(int kind) {
+  switch (kind) {
+    case K_GEMM_TC: return "gemm_tcgen05";
+    case K_REDUCE_LN: return "reduce_residual_layernorm";
+    case K_GEMM_SIMT: return "gemm_simt_f32";
+    case K_ATTN: return "attention_fwd";
+    default: return "unknown";
+  }
+}
+
+}  // extern "C"

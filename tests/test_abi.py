@@ -1,0 +1,151 @@
+"""Host-only checks of the C ABI: the library loads, exports every function the
+header declares, and rejects bad arguments before anything is launched.
+
+No compute call is made here.  Argument checks run before any CUDA call, so
+fake (aligned, never dereferenced) pointers are safe; the single case with
+valid arguments is only run when no CUDA device is present, where it must
+return TP_ERR_NO_DEVICE instead of launching.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from megatron_tensor_transformer_gelu_b200 import _lib as L
+from megatron_tensor_transformer_gelu_b200 import build as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tpblock.h")
+
+OK, INVALID, UNSUPPORTED, WS_SMALL, NO_DEVICE = 0, 1, 2, 3, 6
+FAKE = 0x10000  # aligned, never dereferenced
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tp_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("tp_mlp_forward", "tp_qkv_attn_oproj_forward", "tp_linear_column_forward",
+              "tp_linear_row_forward", "tp_reduce_residual_layernorm", "tp_mlp_workspace_bytes",
+              "tp_attn_workspace_bytes", "tp_status_string", "tp_device_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+        assert n in L.SIGNATURES, f"binding lacks {n}"
+
+
+def test_exports_only_c_symbols():
+    out = os.popen(f"nm -D --defined-only {L.LIB_PATH}").read()
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    tp_syms = {s for s in exported if s.startswith("tp_")}
+    assert tp_syms == set(declared_functions())
+
+
+def test_version_and_status_strings(lib):
+    assert lib.tp_version() == 1
+    assert lib.tp_status_string(0) == b"ok"
+    assert lib.tp_status_string(3) == b"workspace too small"
+    assert lib.tp_status_string(99) == b"unknown status"
+
+
+def test_workspace_sizes(lib):
+    S, H, F = 2048, 4096, 16384
+    assert lib.tp_mlp_workspace_bytes(S, H, F, 4, 1) == S * F * 2 + S * H * 4
+    assert lib.tp_mlp_workspace_bytes(S, H, F, 4, 0) == S * F * 4 + S * H * 4
+    assert lib.tp_mlp_workspace_bytes(-1, H, F, 4, 1) == 0
+    assert lib.tp_attn_workspace_bytes(2048, 8192, 64, 128, 4, 1) == 2048 * 8192 * (6 + 2 + 4)
+    assert lib.tp_attn_workspace_bytes(2048, 8192, 64, 128, 4, 0) == 0
+
+
+def _ptrs(n, base=FAKE):
+    arr = (ctypes.c_void_p * n)(*[base + 256 * i for i in range(n)])
+    return ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p)), arr
+
+
+def _mlp(lib, S=128, H=256, F=1024, t=2, dtype=1, out=1, X=FAKE, A=None, Bp=None, eps=1e-5, act=1,
+         Y=FAKE, ws=FAKE, ws_bytes=1 << 30):
+    pa, ka = A if A is not None else _ptrs(t)
+    pb, kb = Bp if Bp is not None else _ptrs(t)
+    return lib.tp_mlp_forward(S, H, F, t, dtype, out, ctypes.c_void_p(X), pa, pb, None, None, eps, act,
+                              ctypes.c_void_p(Y), ctypes.c_void_p(ws), ws_bytes, None)
+
+
+def test_mlp_argument_checks(lib):
+    assert _mlp(lib, t=0) == INVALID
+    assert _mlp(lib, t=9) == INVALID
+    assert _mlp(lib, X=0) == INVALID
+    assert _mlp(lib, X=FAKE + 4) == INVALID            # misaligned
+    assert _mlp(lib, Y=FAKE + 8) == INVALID
+    assert _mlp(lib, eps=0.0) == INVALID
+    assert _mlp(lib, eps=float("nan")) == INVALID
+    assert _mlp(lib, act=7) == INVALID
+    assert _mlp(lib, dtype=0, out=1) == INVALID        # f32 storage cannot write bf16
+    assert _mlp(lib, dtype=5) == INVALID
+    assert _mlp(lib, F=1000, t=3) == UNSUPPORTED      # F % t
+    assert _mlp(lib, F=1020, t=2) == UNSUPPORTED      # shard width % 8
+    assert _mlp(lib, H=260) == UNSUPPORTED            # H % 8
+    assert _mlp(lib, H=16392) == UNSUPPORTED          # above the LayerNorm row limit
+    assert _mlp(lib, ws_bytes=100) == WS_SMALL
+    pa, ka = _ptrs(2)
+    ka[1] = None
+    assert _mlp(lib, A=(pa, ka)) == INVALID            # null shard
+
+
+def test_attention_argument_checks(lib):
+    pq, kq = _ptrs(4)
+    po, ko = _ptrs(4)
+
+    def call(S=2048, H=8192, nh=64, d=128, t=4, dtype=1, ws_bytes=1 << 34):
+        return lib.tp_qkv_attn_oproj_forward(S, H, nh, d, t, dtype, 1, ctypes.c_void_p(FAKE), pq, po, None, None,
+                                             1e-5, ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE), ws_bytes, None)
+    assert call(dtype=0) == INVALID
+    assert call(d=64, H=4096) == UNSUPPORTED
+    assert call(nh=63, H=63 * 128) == UNSUPPORTED      # nh % t
+    assert call(H=8000) == UNSUPPORTED                 # H != nh * d
+    assert call(S=2000) == UNSUPPORTED                 # S % 128
+    assert call(ws_bytes=10) == WS_SMALL
+
+
+def test_linear_and_layernorm_argument_checks(lib):
+    pw, kw = _ptrs(2)
+    assert lib.tp_linear_column_forward(64, 100, 256, 2, 1, 0, ctypes.c_void_p(FAKE), pw, 0,
+                                        ctypes.c_void_p(FAKE), None) == UNSUPPORTED
+    assert lib.tp_linear_column_forward(64, 128, 250, 2, 1, 0, ctypes.c_void_p(FAKE), pw, 0,
+                                        ctypes.c_void_p(FAKE), None) == UNSUPPORTED
+    assert lib.tp_linear_row_forward(64, 100, 256, 2, 1, 0, ctypes.c_void_p(FAKE), pw, ctypes.c_void_p(FAKE),
+                                     None, 0, None) == UNSUPPORTED
+    assert lib.tp_linear_row_forward(64, 128, 256, 0, 1, 0, ctypes.c_void_p(FAKE), pw, ctypes.c_void_p(FAKE),
+                                     None, 0, None) == INVALID
+    assert lib.tp_reduce_residual_layernorm(8, 12, 0, None, ctypes.c_void_p(FAKE), 1, None, None, 1e-5,
+                                            ctypes.c_void_p(FAKE), 1, None) == UNSUPPORTED
+    assert lib.tp_reduce_residual_layernorm(8, 16, 1, None, ctypes.c_void_p(FAKE), 1, None, None, 1e-5,
+                                            ctypes.c_void_p(FAKE), 1, None) == INVALID
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a CUDA device")
+def test_valid_call_without_device_reports_no_device(lib):
+    assert _mlp(lib) == NO_DEVICE
+
+
+def test_binding_raises_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(L, "_lib", None)
+    monkeypatch.setattr(L, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="not built"):
+        L.lib()

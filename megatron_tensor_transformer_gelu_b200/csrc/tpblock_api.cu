@@ -272,8 +272,9 @@ int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype, const v
   if (t < 1 || t > TP_MAX_SHARDS || S < 0 || H <= 0 || F <= 0) return TP_ERR_INVALID_ARG;
   if (!valid_out(dtype, out_dtype) || !valid_act(act) || !(eps > 0.0f) || !std::isfinite(eps))
     return TP_ERR_INVALID_ARG;
-  if (!ptr_ok(X) || !ptr_ok(Y) || !shards_ok(A_shards, t) || !shards_ok(B_shards, t) || !opt_ptr_ok(gamma) ||
-      !opt_ptr_ok(beta) || !opt_ptr_ok(workspace))
+  // With S == 0 nothing is read or written, so X, Y and workspace may be null.
+  if ((S > 0 && (!ptr_ok(X) || !ptr_ok(Y))) || !opt_ptr_ok(X) || !opt_ptr_ok(Y) || !shards_ok(A_shards, t) ||
+      !shards_ok(B_shards, t) || !opt_ptr_ok(gamma) || !opt_ptr_ok(beta) || !opt_ptr_ok(workspace))
     return TP_ERR_INVALID_ARG;
   if (F % t != 0 || (F / t) % 8 != 0 || !hidden_ok(H)) return TP_ERR_UNSUPPORTED_SHAPE;
   const size_t need = tp_mlp_workspace_bytes(S, H, F, t, dtype);
@@ -322,8 +323,8 @@ int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int
   if (t < 1 || t > TP_MAX_SHARDS || S < 0 || H <= 0 || nh <= 0 || d <= 0) return TP_ERR_INVALID_ARG;
   if (dtype != TP_DTYPE_BF16 || !valid_out(dtype, out_dtype) || !(eps > 0.0f) || !std::isfinite(eps))
     return TP_ERR_INVALID_ARG;
-  if (!ptr_ok(X) || !ptr_ok(Y) || !shards_ok(Wqkv_shards, t) || !shards_ok(Wo_shards, t) || !opt_ptr_ok(gamma) ||
-      !opt_ptr_ok(beta) || !opt_ptr_ok(workspace))
+  if ((S > 0 && (!ptr_ok(X) || !ptr_ok(Y))) || !opt_ptr_ok(X) || !opt_ptr_ok(Y) || !shards_ok(Wqkv_shards, t) ||
+      !shards_ok(Wo_shards, t) || !opt_ptr_ok(gamma) || !opt_ptr_ok(beta) || !opt_ptr_ok(workspace))
     return TP_ERR_INVALID_ARG;
   if (d != tp::attn::D || static_cast<long long>(nh) * d != H || nh % t != 0 || S % tp::attn::BQ != 0 ||
       !hidden_ok(H))
@@ -374,7 +375,8 @@ int tp_linear_column_forward(int M, int K, int N, int t, int dtype, int out_dtyp
                              const void* const* W_shards, int act, void* Y, void* stream) {
   if (t < 1 || t > TP_MAX_SHARDS || M < 0 || K <= 0 || N <= 0) return TP_ERR_INVALID_ARG;
   if (!valid_out(dtype, out_dtype) || !valid_act(act)) return TP_ERR_INVALID_ARG;
-  if (!ptr_ok(X) || !ptr_ok(Y) || !shards_ok(W_shards, t)) return TP_ERR_INVALID_ARG;
+  if ((M > 0 && (!ptr_ok(X) || !ptr_ok(Y))) || !opt_ptr_ok(X) || !opt_ptr_ok(Y) || !shards_ok(W_shards, t))
+    return TP_ERR_INVALID_ARG;
   if (K % 8 != 0 || N % t != 0 || (N / t) % 8 != 0) return TP_ERR_UNSUPPORTED_SHAPE;
   DeviceInfo* dev = nullptr;
   int st = device_ready(&dev);
@@ -393,7 +395,8 @@ int tp_linear_row_forward(int M, int K, int N, int t, int dtype, int out_dtype, 
   (void)workspace_bytes;
   if (t < 1 || t > TP_MAX_SHARDS || M < 0 || K <= 0 || N <= 0) return TP_ERR_INVALID_ARG;
   if (!valid_out(dtype, out_dtype)) return TP_ERR_INVALID_ARG;
-  if (!ptr_ok(X) || !ptr_ok(Y) || !shards_ok(W_shards, t)) return TP_ERR_INVALID_ARG;
+  if ((M > 0 && (!ptr_ok(X) || !ptr_ok(Y))) || !opt_ptr_ok(X) || !opt_ptr_ok(Y) || !shards_ok(W_shards, t))
+    return TP_ERR_INVALID_ARG;
   if (K % t != 0 || (K / t) % 8 != 0 || N % 8 != 0) return TP_ERR_UNSUPPORTED_SHAPE;
   DeviceInfo* dev = nullptr;
   int st = device_ready(&dev);
@@ -412,7 +415,8 @@ int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts, c
   if (S < 0 || nparts < 0 || !valid_dtype(x_dtype) || !valid_dtype(out_dtype) || !(eps > 0.0f) ||
       !std::isfinite(eps))
     return TP_ERR_INVALID_ARG;
-  if (!ptr_ok(X) || !ptr_ok(Y) || (nparts > 0 && !ptr_ok(parts)) || !opt_ptr_ok(gamma) || !opt_ptr_ok(beta))
+  if ((S > 0 && (!ptr_ok(X) || !ptr_ok(Y) || (nparts > 0 && !ptr_ok(parts)))) || !opt_ptr_ok(X) ||
+      !opt_ptr_ok(Y) || !opt_ptr_ok(parts) || !opt_ptr_ok(gamma) || !opt_ptr_ok(beta))
     return TP_ERR_INVALID_ARG;
   if (!hidden_ok(H)) return TP_ERR_UNSUPPORTED_SHAPE;
   DeviceInfo* dev = nullptr;

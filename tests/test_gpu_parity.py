@@ -122,6 +122,9 @@ def test_mlp_empty_rows(cuda_device):
     Y = torch.empty(0, 64, dtype=torch.bfloat16, device="cuda")
     ws = torch.empty(16, dtype=torch.uint8, device="cuda")
     L.mlp_forward(X, _dev(synth.split_columns(inp.A, 2)), _dev(synth.split_rows(inp.B, 2)), Y, ws)
+    Xl = torch.empty(0, 64, dtype=torch.bfloat16, device="cuda")
+    Yl = torch.empty(0, 128, dtype=torch.float32, device="cuda")
+    L.linear_column_forward(Xl, _dev(synth.split_columns(inp.A, 2)), Yl)
     torch.cuda.synchronize()
 
 
@@ -219,14 +222,19 @@ def test_attention_small_full(cuda_device, S, nh, t):
     assert rel_err(Y, O.attention_sublayer(inp.X, inp.Wqkv, inp.Wo, nh, d)) <= TOL_BF16
 
 
-def test_attention_peaked_scores_rescale(cuda_device):
-    """Large-magnitude inputs make the running max jump by more than the lazy
-    rescale threshold, exercising the O rescale in TMEM."""
+def test_attention_late_large_keys_rescale(cuda_device):
+    """Keys of the last 128-key block are 4x larger, so for the unscaled query
+    rows 0..383 that block's row max exceeds the running max by more than the
+    lazy-rescale threshold (2^8): the O accumulator is rescaled in TMEM."""
     d, nh, S = 128, 2, 512
     inp = synth.gen_attn(S, nh * d, seed=21)
-    inp.X = (inp.X.float() * 4.0).to(torch.bfloat16)
+    X = inp.X.float()
+    X[384:] *= 4.0
+    inp.X = X.to(torch.bfloat16)
     Y = run_attn(inp, nh, d, 2)
-    assert rel_err(Y, O.attention_sublayer(inp.X, inp.Wqkv, inp.Wo, nh, d)) <= TOL_BF16
+    rows = list(range(384))
+    ref = O.attention_sublayer(inp.X, inp.Wqkv, inp.Wo, nh, d, rows=rows)
+    assert rel_err(Y[:384], ref) <= TOL_BF16
 
 
 # ------------------------------------------------------ full-size workloads

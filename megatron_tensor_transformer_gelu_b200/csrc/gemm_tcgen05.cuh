@@ -13,14 +13,22 @@
 //    accumulator, so the sum (the AllReduce of the multi-GPU form) costs no
 //    extra memory traffic.
 //
-// Design (sm_100a): one CTA per SM, 6 warps.
-//   warp 0      TMA producer: A box 128x64 (K-major, 128B swizzle), B as four
-//               64(k) x 64(n) boxes (N-major, 128B swizzle), 4-stage ring.
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
-//               (M=128, N=256, K=16 per instruction, f32 accumulate in TMEM).
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator, activation, store.
+// Design (sm_100a), one CTA per SM, 6 warps, CG = 1 (one CTA per tile) or
+// CG = 2 (a cluster of two CTAs on two SMs shares one tile through
+// tcgen05.mma.cta_group::2):
+//   warp 0      TMA producer.  Per stage each CTA loads its 128 rows of A
+//               (box 128 x 64, K-major, 128-byte swizzle) and its BN/CG
+//               columns of B (64 x 64 boxes, N-major, 128-byte swizzle).  In a
+//               pair both CTAs' copies complete on the leader's barrier.
+//   warp 1      TMEM allocator; lane 0 of the leader issues tcgen05.mma
+//               (M = 128*CG, N = 256, K = 16 per instruction) into an f32
+//               accumulator in TMEM and commits stage/accumulator releases
+//               to both CTAs.
+//   warps 2..5  epilogue: tcgen05.ld of this CTA's 128 accumulator rows,
+//               activation, 16-byte stores.
 // The accumulator is double-buffered in TMEM (2 x 256 of the 512 columns), so
-// the epilogue of tile i overlaps the main loop of tile i+1.
+// the epilogue of tile i overlaps the main loop of tile i+1.  No load uses
+// cluster multicast: every CTA fetches its own operand boxes.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -33,21 +41,24 @@ constexpr int MAX_SHARDS = 8;
 
 enum : int { ACT_NONE = 0, ACT_GELU_TANH = 1, ACT_GELU_ERF = 2, ACT_RELU = 3 };
 
-namespace gemm {
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int BK = 64;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;          // 16 KiB
-constexpr int B_BOX_N = 64;                   // 64 bf16 = one 128-byte swizzle row
-constexpr int B_BOX_BYTES = BK * B_BOX_N * 2; // 8 KiB
-constexpr int B_BOXES = BN / B_BOX_N;         // 4
-constexpr int B_BYTES = BK * BN * 2;          // 32 KiB
-constexpr int NUM_THREADS = 192;
-constexpr int TMEM_COLS = 512;
-constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*barriers*/;
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*a_mn=*/false, /*b_mn=*/true);
-}  // namespace gemm
+template <int CG>
+struct GemmCfg {
+  static constexpr int BM = 128;                    // accumulator rows per CTA
+  static constexpr int TILE_M = BM * CG;            // rows per (cluster) tile
+  static constexpr int BN = 256;                    // columns per tile
+  static constexpr int BK = 64;
+  static constexpr int STAGES = CG == 2 ? 6 : 4;
+  static constexpr int A_BYTES = BM * BK * 2;       // 16 KiB
+  static constexpr int B_BOX_N = 64;                // 64 bf16 = one 128-byte swizzle row
+  static constexpr int B_BOX_BYTES = BK * B_BOX_N * 2;  // 8 KiB
+  static constexpr int B_COLS_CTA = BN / CG;        // B columns each CTA loads
+  static constexpr int B_BOXES = B_COLS_CTA / B_BOX_N;
+  static constexpr int B_BYTES = BK * B_COLS_CTA * 2;
+  static constexpr int NUM_THREADS = 192;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN, /*a_mn=*/false, /*b_mn=*/true);
+};
 
 struct GemmArgs {
   CUtensorMap tmA;               // A [M, K] bf16 row-major, box {64, 128}
@@ -62,7 +73,7 @@ struct GemmArgs {
   int shard_k;                   // rows of each B shard
   int n_blocks_per_shard;        // column mode
   int k_blocks_per_shard;        // row mode (column mode: k blocks of K)
-  int m_blocks, n_blocks, k_blocks;
+  int m_blocks, n_blocks, k_blocks;  // m_blocks counts TILE_M-row tiles
   int act;
   int out_f32;
 };
@@ -86,39 +97,51 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 // Tile coordinates shared by the three roles.
 struct TileCoord {
-  int m0;        // first row
+  int m0;        // first row of the (cluster) tile
   int shard;     // column mode: shard owning the tile's columns
   int n_in;      // first column inside the B operand (shard-local in column mode)
   int out_col0;  // first column of C
   int n_valid;   // valid columns in this tile (<= BN)
 };
 
+template <int CG>
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& p, int tile) {
+  using C = GemmCfg<CG>;
   TileCoord c;
   const int mb = tile % p.m_blocks;
   const int nb = tile / p.m_blocks;
-  c.m0 = mb * gemm::BM;
+  c.m0 = mb * C::TILE_M;
   if (!p.row_mode) {
     c.shard = nb / p.n_blocks_per_shard;
-    c.n_in = (nb % p.n_blocks_per_shard) * gemm::BN;
+    c.n_in = (nb % p.n_blocks_per_shard) * C::BN;
     c.out_col0 = c.shard * p.shard_n + c.n_in;
-    c.n_valid = min(gemm::BN, p.shard_n - c.n_in);
   } else {
     c.shard = 0;
-    c.n_in = nb * gemm::BN;
+    c.n_in = nb * C::BN;
     c.out_col0 = c.n_in;
-    c.n_valid = min(gemm::BN, p.shard_n - c.n_in);
   }
+  c.n_valid = min(C::BN, p.shard_n - c.n_in);
   return c;
 }
 
-__global__ void __launch_bounds__(gemm::NUM_THREADS, 1) gemm_tcgen05_kernel(const __grid_constant__ GemmArgs p) {
-  using namespace gemm;
+// Number of 64-column B boxes CTA `rank` of the pair loads for a tile.
+template <int CG>
+__device__ __forceinline__ int b_boxes_for(int n_valid, int rank) {
+  using C = GemmCfg<CG>;
+  const int cols = n_valid - rank * C::B_COLS_CTA;
+  if (cols <= 0) return 0;
+  return min(C::B_BOXES, (cols + C::B_BOX_N - 1) / C::B_BOX_N);
+}
+
+template <int CG>
+__global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kernel(const __grid_constant__ GemmArgs p) {
+  using C = GemmCfg<CG>;
+  constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
-  uint8_t* sB = smem + STAGES * A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint8_t* sB = smem + STAGES * C::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -127,6 +150,8 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1) gemm_tcgen05_kernel(cons
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = CG == 2 ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -135,7 +160,7 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1) gemm_tcgen05_kernel(cons
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 128);
+      mbar_init(&tempty[a], CG == 2 ? 4 * CG : 128);
     }
     mbar_init(drain, 1);
     mbar_fence_init();
@@ -145,15 +170,18 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1) gemm_tcgen05_kernel(cons
     for (int s = 0; s < p.t; ++s) tma_prefetch_desc(&p.tmB[s]);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc<CG>(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish<CG>();
   }
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) cluster_sync();
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
   const int num_tiles = p.m_blocks * p.n_blocks;
+  const int cluster_id = blockIdx.x / CG;
+  const int num_clusters = gridDim.x / CG;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -161,36 +189,53 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1) gemm_tcgen05_kernel(cons
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int armed[STAGES];  // parity of the last phase this thread armed per stage
+      int armed[STAGES];  // parity of the last phase this thread armed per stage (leader)
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) armed[s] = -1;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const TileCoord tc = tile_coord(p, tile);
-        const int nboxes = min(B_BOXES, (tc.n_valid + B_BOX_N - 1) / B_BOX_N);
-        const uint32_t bytes = A_BYTES + nboxes * B_BOX_BYTES;
+      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+        const TileCoord tc = tile_coord<CG>(p, tile);
+        const int my_row0 = tc.m0 + static_cast<int>(rank) * C::BM;
+        const bool my_a = my_row0 < p.M;
+        const int my_boxes = b_boxes_for<CG>(tc.n_valid, rank);
+        uint32_t bytes = 0;  // leader: bytes the whole tile stage brings in
+        for (int r = 0; r < CG; ++r)
+          bytes += (tc.m0 + r * C::BM < p.M ? C::A_BYTES : 0) + b_boxes_for<CG>(tc.n_valid, r) * C::B_BOX_BYTES;
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           int shard, a_x, b_y;
           if (p.row_mode) {
             shard = kb / p.k_blocks_per_shard;
-            b_y = (kb % p.k_blocks_per_shard) * BK;
+            b_y = (kb % p.k_blocks_per_shard) * C::BK;
             a_x = shard * p.shard_k + b_y;
           } else {
             shard = tc.shard;
-            b_y = kb * BK;
+            b_y = kb * C::BK;
             a_x = b_y;
           }
-          mbar_arrive_expect_tx(&full[stage], bytes);
-          armed[stage] = static_cast<int>(phase);
-          tma_load_2d(sA + stage * A_BYTES, &p.tmA, a_x, tc.m0, &full[stage]);
-          for (int j = 0; j < nboxes; ++j)
-            tma_load_2d(sB + stage * B_BYTES + j * B_BOX_BYTES, &p.tmB[shard], tc.n_in + j * B_BOX_N, b_y,
-                        &full[stage]);
+          uint8_t* dA = sA + stage * C::A_BYTES;
+          uint8_t* dB = sB + stage * C::B_BYTES;
+          const int b_x0 = tc.n_in + static_cast<int>(rank) * C::B_COLS_CTA;
+          if constexpr (CG == 1) {
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            armed[stage] = static_cast<int>(phase);
+            tma_load_2d(dA, &p.tmA, a_x, my_row0, &full[stage]);
+            for (int j = 0; j < my_boxes; ++j)
+              tma_load_2d(dB + j * C::B_BOX_BYTES, &p.tmB[shard], b_x0 + j * C::B_BOX_N, b_y, &full[stage]);
+          } else {
+            const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
+            if (leader) {
+              mbar_arrive_expect_tx(&full[stage], bytes);
+              armed[stage] = static_cast<int>(phase);
+            }
+            if (my_a) tma_load_2d_pair(dA, &p.tmA, a_x, my_row0, bar);
+            for (int j = 0; j < my_boxes; ++j)
+              tma_load_2d_pair(dB + j * C::B_BOX_BYTES, &p.tmB[shard], b_x0 + j * C::B_BOX_N, b_y, bar);
+          }
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
       }
       if (!ok) {
-        // Let every copy already issued land before the CTA can exit.
+        // Let every copy this CTA's barriers still expect land before exit.
         for (int s = 0; s < STAGES; ++s) {
           if (armed[s] < 0) continue;
           const uint32_t a = smem_u32(&full[s]);
@@ -201,40 +246,44 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1) gemm_tcgen05_kernel(cons
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
         for (int kb = 0; kb < p.k_blocks; ++kb) {
           if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a0 = smem_u32(sA + stage * A_BYTES);
-          const uint32_t b0 = smem_u32(sB + stage * B_BYTES);
+          const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
+          const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
+          for (int kk = 0; kk < C::BK / 16; ++kk) {
             // A: K-major, 16 k-elements = 32 bytes further along the swizzled row.
             const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
             // B: N-major, 16 k-rows = 2 x (8 rows x 128 B) further; 64-column
             // chunks are B_BOX_BYTES apart (leading offset), 8-row groups 1 KiB.
-            const uint64_t bd = sdesc_sw128(b0 + kk * 2048, B_BOX_BYTES, 1024);
-            umma_bf16(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            const uint64_t bd = sdesc_sw128(b0 + kk * 2048, C::B_BOX_BYTES, 1024);
+            if constexpr (CG == 1) umma_bf16(d_tmem, ad, bd, C::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            else umma_bf16_pair(d_tmem, ad, bd, C::IDESC, (kb | kk) != 0 ? 1u : 0u);
           }
-          umma_commit(&empty[stage]);
+          if constexpr (CG == 1) umma_commit(&empty[stage]);
+          else umma_commit_pair_mc(&empty[stage], 0x3);
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
         if (!ok) break;
-        umma_commit(&tfull[acc]);
+        if constexpr (CG == 1) umma_commit(&tfull[acc]);
+        else umma_commit_pair_mc(&tfull[acc], 0x3);
         if (++acc == 2) { acc = 0; acc_phase ^= 1; }
       }
       if (!ok) {
         // Wait (bounded) for every MMA already issued before TMEM is freed.
-        umma_commit(drain);
+        if constexpr (CG == 1) umma_commit(drain);
+        else umma_commit_pair_mc(drain, 0x1);
         const uint32_t a = smem_u32(drain);
         const long long t0 = clock64();
         while (!mbar_try_wait(a, 0) && clock64() - t0 < WAIT_LIMIT_CYCLES) {}
@@ -246,13 +295,14 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1) gemm_tcgen05_kernel(cons
     const int row_local = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const TileCoord tc = tile_coord(p, tile);
+    const uint32_t tempty_leader0 = CG == 2 ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
+    for (int tile = cluster_id; tile < num_tiles; tile += num_clusters) {
+      const TileCoord tc = tile_coord<CG>(p, tile);
       if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase))) break;
       tc_fence_after();
-      const int grow = tc.m0 + row_local;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      for (int c = 0; c < BN / 32; ++c) {
+      const int grow = tc.m0 + static_cast<int>(rank) * C::BM + row_local;
+      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
+      for (int c = 0; c < C::BN / 32; ++c) {
         if (c * 32 >= tc.n_valid) break;  // uniform across the CTA
         uint32_t r[32];
         tmem_ld_32x32b_x32(t_row + c * 32, r);
@@ -283,16 +333,22 @@ __global__ void __launch_bounds__(gemm::NUM_THREADS, 1) gemm_tcgen05_kernel(cons
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      if constexpr (CG == 1) {
+        mbar_arrive(&tempty[acc]);
+      } else {
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(tempty_leader0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+      }
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
   }
 
   tc_fence_before();
-  __syncthreads();
+  if constexpr (CG == 2) cluster_sync();
+  else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    tmem_dealloc<CG>(tmem_base, C::TMEM_COLS);
   }
 }
 

@@ -29,7 +29,14 @@ struct DeviceInfo {
   bool ready = false;
   bool ok = false;
   int sm_count = 0;
+  int max_pairs = 0;  // co-resident CTA pairs of the cta_group::2 GEMM
 };
+
+// GEMM flavour: CTA pairs (cta_group::2, 256-row tiles) unless the problem has
+// at most 128 rows, where a pair would leave half of every tile empty.
+#ifndef TP_GEMM_PAIR_MIN_ROWS
+#define TP_GEMM_PAIR_MIN_ROWS 129
+#endif
 
 std::mutex g_mu;
 DeviceInfo g_dev[MAX_DEVICES];
@@ -83,11 +90,30 @@ int device_ready(DeviceInfo** out) {
       d.sm_count = sms;
     }
     if (d.ok) {
-      if (cudaFuncSetAttribute(tp::gemm_tcgen05_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               tp::gemm::SMEM_BYTES) != cudaSuccess ||
+      if (cudaFuncSetAttribute(tp::gemm_tcgen05_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tp::GemmCfg<1>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(tp::gemm_tcgen05_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tp::GemmCfg<2>::SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(tp::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                tp::attn::SMEM_BYTES) != cudaSuccess)
         d.ok = false;
+    }
+    if (d.ok) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 2;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(2 * (sms / 2), 1, 1);
+      cfg.blockDim = dim3(tp::GemmCfg<2>::NUM_THREADS, 1, 1);
+      cfg.dynamicSmemBytes = tp::GemmCfg<2>::SMEM_BYTES;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int pairs = 0;
+      if (cudaOccupancyMaxActiveClusters(&pairs, tp::gemm_tcgen05_kernel<2>, &cfg) != cudaSuccess || pairs < 1)
+        d.ok = false;
+      d.max_pairs = pairs;
     }
     if (d.ok && !g_encode) {
       void* fn = nullptr;
@@ -123,17 +149,51 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_
 // Tensor-core GEMM.  Column mode: B shard s is [K, shard_n], output columns
 // [s*shard_n, (s+1)*shard_n).  Row mode: B shard s is [shard_k, shard_n] and
 // multiplies A's columns [s*shard_k, (s+1)*shard_k); all shards are summed.
+template <int CG>
+int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, cudaStream_t st) {
+  using C = tp::GemmCfg<CG>;
+  p.m_blocks = ceil_div(p.M, C::TILE_M);
+  if (p.row_mode) {
+    p.n_blocks = ceil_div(p.shard_n, C::BN);
+    p.n_blocks_per_shard = p.n_blocks;
+  } else {
+    p.n_blocks_per_shard = ceil_div(p.shard_n, C::BN);
+    p.n_blocks = p.n_blocks_per_shard * p.t;
+  }
+  const long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks;
+  const int slots = CG == 2 ? dev.max_pairs : dev.sm_count;
+  const int clusters = static_cast<int>(tiles < slots ? tiles : slots);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = CG;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(clusters * CG, 1, 1);
+  cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = CG == 2 ? 1 : 0;
+  ProfScope ps(K_GEMM_TC, st);
+  if (cudaLaunchKernelEx(&cfg, tp::gemm_tcgen05_kernel<CG>, p) != cudaSuccess) return TP_ERR_CUDA;
+  return launch_status();
+}
+
+// Tensor-core GEMM.  Column mode: B shard s is [K, shard_n], output columns
+// [s*shard_n, (s+1)*shard_n).  Row mode: B shard s is [shard_k, shard_n] and
+// multiplies A's columns [s*shard_k, (s+1)*shard_k); all shards are summed.
 int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, const void* const* B, int t,
                 int row_mode, int shard_k, int shard_n, void* C, long long ldc, int out_f32, int act,
                 cudaStream_t st) {
-  using namespace tp::gemm;
+  using G = tp::GemmCfg<1>;
   if (M == 0) return TP_OK;
   tp::GemmArgs p;
   std::memset(&p, 0, sizeof(p));
   const long long K_total = row_mode ? static_cast<long long>(shard_k) * t : shard_k;
-  if (!tmap_bf16(&p.tmA, A, M, K_total, lda, BK, BM)) return TP_ERR_CUDA;
+  if (!tmap_bf16(&p.tmA, A, M, K_total, lda, G::BK, G::BM)) return TP_ERR_CUDA;
   for (int s = 0; s < t; ++s)
-    if (!tmap_bf16(&p.tmB[s], B[s], shard_k, shard_n, shard_n, B_BOX_N, BK)) return TP_ERR_CUDA;
+    if (!tmap_bf16(&p.tmB[s], B[s], shard_k, shard_n, shard_n, G::B_BOX_N, G::BK)) return TP_ERR_CUDA;
   p.C = C;
   p.ldc = ldc;
   p.M = M;
@@ -141,27 +201,13 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
   p.row_mode = row_mode;
   p.shard_n = shard_n;
   p.shard_k = shard_k;
-  p.m_blocks = ceil_div(M, BM);
-  if (row_mode) {
-    p.N = shard_n;
-    p.n_blocks = ceil_div(shard_n, BN);
-    p.n_blocks_per_shard = p.n_blocks;
-    p.k_blocks_per_shard = ceil_div(shard_k, BK);
-    p.k_blocks = p.k_blocks_per_shard * t;
-  } else {
-    p.N = shard_n * t;
-    p.n_blocks_per_shard = ceil_div(shard_n, BN);
-    p.n_blocks = p.n_blocks_per_shard * t;
-    p.k_blocks_per_shard = ceil_div(shard_k, BK);
-    p.k_blocks = p.k_blocks_per_shard;
-  }
+  p.N = row_mode ? shard_n : shard_n * t;
+  p.k_blocks_per_shard = ceil_div(shard_k, G::BK);
+  p.k_blocks = row_mode ? p.k_blocks_per_shard * t : p.k_blocks_per_shard;
   p.act = act;
   p.out_f32 = out_f32;
-  const long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks;
-  const int grid = static_cast<int>(tiles < dev.sm_count ? tiles : dev.sm_count);
-  ProfScope ps(K_GEMM_TC, st);
-  tp::gemm_tcgen05_kernel<<<grid, NUM_THREADS, SMEM_BYTES, st>>>(p);
-  return launch_status();
+  if (M >= TP_GEMM_PAIR_MIN_ROWS) return launch_gemm_tc<2>(dev, p, st);
+  return launch_gemm_tc<1>(dev, p, st);
 }
 
 int run_gemm_simt(const float* A, long long lda, int M, const void* const* B, int t, int row_mode, int shard_k,

@@ -266,8 +266,8 @@ def run_ours(args, rank, world, local):
         ms_step = ms_total / args.steps
         value = whole_job_tflops(w.flops, args.steps, world, ms_total)
         e2e_value = whole_job_tflops(w.flops, e2e_steps, world, e2e_ms)
-        g_launch, g_ms = prof.get("gemm_tcgen05", (0, 0.0))
-        ln_launch, ln_ms = prof.get("reduce_residual_layernorm", (0, 0.0))
+        _, g_launch, g_ms = prof.get("gemm_tcgen05", (0, 0, 0.0))
+        _, ln_launch, ln_ms = prof.get("reduce_residual_layernorm", (0, 0, 0.0))
         launches = sum(v[0] for v in prof.values())
         gemm_flops_per_launch = w.flops / 2  # both GEMMs are 2*S*H*F
         achieved = gemm_flops_per_launch / (g_ms / g_launch * 1e-3) / 1e12 if g_launch else None

@@ -91,12 +91,16 @@ int tp_device_error(void);
  *   B_shards  t pointers, B_i = rows    [i F/t, (i+1) F/t) of B [F, H]: [F/t, H].
  *   gamma, beta  [H] f32 or NULL.  eps > 0.
  *   Y         [S, H] out_dtype (bf16 or f32 for dtype bf16; f32 for dtype f32).
- *   workspace caller-owned device scratch of >= tp_mlp_workspace_bytes().
+ *   workspace caller-owned device scratch of >= tp_mlp_workspace_bytes():
+ *             the [S, F] activation buffer plus (bf16) up to 4 f32 [S, H]
+ *             partial-sum slots; its contents on return are unspecified.
  * Supported: S >= 1; H % 8 == 0 and 8 <= H <= 16384; (F/t) % 8 == 0.
  * Kernels (bf16): column-split GEMM with the activation in its epilogue
  * (writes Act(X A_i) into its column slice of a [S, F] bf16 buffer), row-split
- * GEMM summing every shard in the TMEM accumulator ([S, H] f32), then the
- * reduce + residual + LayerNorm kernel. */
+ * GEMM summing every shard in the TMEM accumulator ([S, H] f32; its K loop
+ * is cut into up to 4 ranges with one f32 partial slot each when that fills
+ * the GPU's last wave better), then the reduce + residual + LayerNorm kernel
+ * that adds the slots. */
 size_t tp_mlp_workspace_bytes(int S, int H, int F, int t, int dtype);
 int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype,
                    const void* X, const void* const* A_shards, const void* const* B_shards,
@@ -149,14 +153,17 @@ int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts,
                                  float eps, void* Y, int out_dtype, void* stream);
 
 /* ----------------------------------------------------- kernel timing ----
- * When enabled, every kernel the library launches is bracketed by CUDA events
- * recorded on its stream (at most 4096 launches between two collects).
- * tp_profile_collect synchronises those events, writes per kernel kind the
- * launch count and summed device milliseconds (kinds: 0 tensor-core GEMM,
- * 1 reduce+residual+LayerNorm, 2 f32 CUDA-core GEMM, 3 attention), and
- * clears the record.  Returns the number of kinds written (<= max_kinds). */
+ * When enabled, every kernel the library launches is counted, and the first
+ * 16384 launches between two collects are bracketed by CUDA events recorded on
+ * the launch's stream.  tp_profile_collect synchronises those events and
+ * writes per kernel kind (0 tensor-core GEMM, 1 reduce+residual+LayerNorm,
+ * 2 f32 CUDA-core GEMM, 3 attention): `launches` = all launches, `timed` = the
+ * launches with events, `ms` = their summed device milliseconds; then it
+ * clears the record.  Any output array may be NULL.  Returns the number of
+ * kinds written (<= max_kinds), or -TP_ERR_CUDA.  Not thread-safe: enable,
+ * launch and collect from one host thread. */
 int tp_profile_enable(int on);
-int tp_profile_collect(int* launches, double* ms, int max_kinds);
+int tp_profile_collect(int* launches, int* timed, double* ms, int max_kinds);
 const char* tp_kernel_kind_name(int kind);
 
 #ifdef __cplusplus

@@ -38,7 +38,8 @@ SIGNATURES = {
     "tp_linear_row_forward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vp, _vp, _c_size, _vp]),
     "tp_reduce_residual_layernorm": (_c_int, [_c_int] * 3 + [_vp, _vp, _c_int, _vp, _vp, _c_float, _vp, _c_int, _vp]),
     "tp_profile_enable": (_c_int, [_c_int]),
-    "tp_profile_collect": (_c_int, [ctypes.POINTER(_c_int), ctypes.POINTER(ctypes.c_double), _c_int]),
+    "tp_profile_collect": (_c_int, [ctypes.POINTER(_c_int), ctypes.POINTER(_c_int), ctypes.POINTER(ctypes.c_double),
+                                    _c_int]),
     "tp_kernel_kind_name": (ctypes.c_char_p, [_c_int]),
 }
 
@@ -161,9 +162,11 @@ def profile_enable(on: bool):
 
 
 def profile_collect(nkinds: int = 4):
+    """{kernel kind: (launches, timed launches, summed ms of the timed ones)}"""
     launches = (ctypes.c_int * nkinds)()
+    timed = (ctypes.c_int * nkinds)()
     ms = (ctypes.c_double * nkinds)()
-    n = lib().tp_profile_collect(launches, ms, nkinds)
+    n = lib().tp_profile_collect(launches, timed, ms, nkinds)
     if n < 0:
         raise TPError(-n, "tp_profile_collect")
-    return {lib().tp_kernel_kind_name(k).decode(): (launches[k], ms[k]) for k in range(n)}
+    return {lib().tp_kernel_kind_name(k).decode(): (launches[k], timed[k], ms[k]) for k in range(n)}

@@ -47,7 +47,14 @@ struct GemmCfg {
   static constexpr int TILE_M = BM * CG;            // rows per (cluster) tile
   static constexpr int BN = 256;                    // columns per tile
   static constexpr int BK = 64;
-  static constexpr int STAGES = CG == 2 ? 6 : 4;
+#ifndef TP_GEMM_PAIR_STAGES
+#define TP_GEMM_PAIR_STAGES 6
+#endif
+#ifndef TP_GEMM_L2_PREFETCH
+#define TP_GEMM_L2_PREFETCH 0
+#endif
+  static constexpr int STAGES = CG == 2 ? TP_GEMM_PAIR_STAGES : 4;
+  static constexpr int PREFETCH = TP_GEMM_L2_PREFETCH;  // k-blocks ahead (0 = off)
   static constexpr int A_BYTES = BM * BK * 2;       // 16 KiB
   static constexpr int B_BOX_N = 64;                // 64 bf16 = one 128-byte swizzle row
   static constexpr int B_BOX_BYTES = BK * B_BOX_N * 2;  // 8 KiB
@@ -56,13 +63,20 @@ struct GemmCfg {
   static constexpr int B_BYTES = BK * B_COLS_CTA * 2;
   static constexpr int NUM_THREADS = 192;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES) + 1024 /*align*/ + 256 /*barriers*/;
+  // Epilogue staging: two buffers of 128 rows x 128 bytes (32 f32 or 64 bf16
+  // columns), 128-byte swizzled, drained by TMA stores.
+  static constexpr int EPI_BUF_BYTES = BM * 128;
+  static constexpr int SMEM_BYTES =
+      STAGES * (A_BYTES + B_BYTES) + 2 * EPI_BUF_BYTES + 1024 /*align*/ + 256 /*barriers*/;
   static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN, /*a_mn=*/false, /*b_mn=*/true);
 };
 
 struct GemmArgs {
   CUtensorMap tmA;               // A [M, K] bf16 row-major, box {64, 128}
   CUtensorMap tmB[MAX_SHARDS];   // B shard s, bf16 row-major [rows, cols], box {64, 64}
+  // Output maps, 3-D {cols, M, splits}, box {128 B of columns, 128, 1}, 128-byte
+  // swizzle: column mode one per shard (its column slice of C), row mode one.
+  CUtensorMap tmC[MAX_SHARDS];
   void* C;                       // output, row-major, ldc elements per row
   long long ldc;
   int M;
@@ -76,7 +90,17 @@ struct GemmArgs {
   int m_blocks, n_blocks, k_blocks;  // m_blocks counts TILE_M-row tiles
   int act;
   int out_f32;
+  // Split of the K loop into `splits` contiguous k-block ranges.  Work unit u
+  // is (split u / tiles, tile u % tiles); split j writes its partial sum to
+  // C + j * slot_stride (f32 only), and a later kernel adds the slots.
+  int splits;
+  long long slot_stride;
 };
+
+__device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& kb0, int& kb1) {
+  kb0 = static_cast<int>(static_cast<long long>(split) * p.k_blocks / p.splits);
+  kb1 = static_cast<int>(static_cast<long long>(split + 1) * p.k_blocks / p.splits);
+}
 
 __device__ __forceinline__ float apply_act(float u, int act) {
   if (act == ACT_GELU_TANH) {
@@ -124,6 +148,21 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& p, int tile) {
   return c;
 }
 
+// Shard, A column and B row of k-block kb.
+__device__ __forceinline__ void kblock_coords(const GemmArgs& p, const TileCoord& tc, int kb, int& shard, int& a_x,
+                                              int& b_y) {
+  constexpr int BK = 64;
+  if (p.row_mode) {
+    shard = kb / p.k_blocks_per_shard;
+    b_y = (kb % p.k_blocks_per_shard) * BK;
+    a_x = shard * p.shard_k + b_y;
+  } else {
+    shard = tc.shard;
+    b_y = kb * BK;
+    a_x = b_y;
+  }
+}
+
 // Number of 64-column B boxes CTA `rank` of the pair loads for a tile.
 template <int CG>
 __device__ __forceinline__ int b_boxes_for(int n_valid, int rank) {
@@ -141,7 +180,8 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * C::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_BYTES);
+  uint8_t* sEpi = sB + STAGES * C::B_BYTES;  // 2 x EPI_BUF_BYTES
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + 2 * C::EPI_BUF_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -169,6 +209,9 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
     tma_prefetch_desc(&p.tmA);
     for (int s = 0; s < p.t; ++s) tma_prefetch_desc(&p.tmB[s]);
   }
+  if (warp == 2 && lane == 0) {
+    for (int s = 0; s < (p.row_mode ? 1 : p.t); ++s) tma_prefetch_desc(&p.tmC[s]);
+  }
   if (warp == 1) {
     tmem_alloc<CG>(tmem_holder, C::TMEM_COLS);
     tmem_relinquish<CG>();
@@ -180,6 +223,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
   const uint32_t tmem_base = *tmem_holder;
 
   const int num_tiles = p.m_blocks * p.n_blocks;
+  const int num_units = num_tiles * p.splits;
   const int cluster_id = blockIdx.x / CG;
   const int num_clusters = gridDim.x / CG;
 
@@ -192,7 +236,10 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       int armed[STAGES];  // parity of the last phase this thread armed per stage (leader)
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) armed[s] = -1;
-      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+      for (int unit = cluster_id; unit < num_units && ok; unit += num_clusters) {
+        const int tile = unit % num_tiles;
+        int kb_begin, kb_end;
+        split_range(p, unit / num_tiles, kb_begin, kb_end);
         const TileCoord tc = tile_coord<CG>(p, tile);
         const int my_row0 = tc.m0 + static_cast<int>(rank) * C::BM;
         const bool my_a = my_row0 < p.M;
@@ -200,21 +247,22 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         uint32_t bytes = 0;  // leader: bytes the whole tile stage brings in
         for (int r = 0; r < CG; ++r)
           bytes += (tc.m0 + r * C::BM < p.M ? C::A_BYTES : 0) + b_boxes_for<CG>(tc.n_valid, r) * C::B_BOX_BYTES;
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        const int b_x0 = tc.n_in + static_cast<int>(rank) * C::B_COLS_CTA;
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
+          if constexpr (C::PREFETCH > 0) {
+            const int kp = kb + C::PREFETCH;
+            if (kp < kb_end) {
+              int ps, pa, pb;
+              kblock_coords(p, tc, kp, ps, pa, pb);
+              if (my_a) tma_prefetch_l2_2d(&p.tmA, pa, my_row0);
+              for (int j = 0; j < my_boxes; ++j) tma_prefetch_l2_2d(&p.tmB[ps], b_x0 + j * C::B_BOX_N, pb);
+            }
+          }
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           int shard, a_x, b_y;
-          if (p.row_mode) {
-            shard = kb / p.k_blocks_per_shard;
-            b_y = (kb % p.k_blocks_per_shard) * C::BK;
-            a_x = shard * p.shard_k + b_y;
-          } else {
-            shard = tc.shard;
-            b_y = kb * C::BK;
-            a_x = b_y;
-          }
+          kblock_coords(p, tc, kb, shard, a_x, b_y);
           uint8_t* dA = sA + stage * C::A_BYTES;
           uint8_t* dB = sB + stage * C::B_BYTES;
-          const int b_x0 = tc.n_in + static_cast<int>(rank) * C::B_COLS_CTA;
           if constexpr (CG == 1) {
             mbar_arrive_expect_tx(&full[stage], bytes);
             armed[stage] = static_cast<int>(phase);
@@ -252,11 +300,13 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = cluster_id; tile < num_tiles && ok; tile += num_clusters) {
+      for (int unit = cluster_id; unit < num_units && ok; unit += num_clusters) {
+        int kb_begin, kb_end;
+        split_range(p, unit / num_tiles, kb_begin, kb_end);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
-        for (int kb = 0; kb < p.k_blocks; ++kb) {
+        for (int kb = kb_begin; kb < kb_end; ++kb) {
           if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
@@ -268,8 +318,9 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
             // B: N-major, 16 k-rows = 2 x (8 rows x 128 B) further; 64-column
             // chunks are B_BOX_BYTES apart (leading offset), 8-row groups 1 KiB.
             const uint64_t bd = sdesc_sw128(b0 + kk * 2048, C::B_BOX_BYTES, 1024);
-            if constexpr (CG == 1) umma_bf16(d_tmem, ad, bd, C::IDESC, (kb | kk) != 0 ? 1u : 0u);
-            else umma_bf16_pair(d_tmem, ad, bd, C::IDESC, (kb | kk) != 0 ? 1u : 0u);
+            const uint32_t accum = (kb != kb_begin || kk != 0) ? 1u : 0u;
+            if constexpr (CG == 1) umma_bf16(d_tmem, ad, bd, C::IDESC, accum);
+            else umma_bf16_pair(d_tmem, ad, bd, C::IDESC, accum);
           }
           if constexpr (CG == 1) umma_commit(&empty[stage]);
           else umma_commit_pair_mc(&empty[stage], 0x3);
@@ -291,56 +342,90 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Per 128-byte column chunk: tcgen05.ld of this thread's accumulator row,
+    // activation, conversion, a swizzled row write into a staging buffer, then
+    // one TMA store of the 128 x chunk box (double-buffered).  TMA clips rows
+    // beyond M and columns beyond the shard / output width.
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     const int row_local = q * 32 + lane;
+    const bool elected = threadIdx.x == 64;
+    const int cw = p.out_f32 ? 32 : 64;  // columns per 128-byte chunk
     int acc = 0;
     uint32_t acc_phase = 0;
+    int buf = 0;
     const uint32_t tempty_leader0 = CG == 2 ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
-    for (int tile = cluster_id; tile < num_tiles; tile += num_clusters) {
-      const TileCoord tc = tile_coord<CG>(p, tile);
-      if (!__all_sync(0xffffffffu, mbar_wait(&tfull[acc], acc_phase))) break;
+    for (int unit = cluster_id; unit < num_units; unit += num_clusters) {
+      const TileCoord tc = tile_coord<CG>(p, unit % num_tiles);
+      const int split = unit / num_tiles;
+      const CUtensorMap* tmC = &p.tmC[p.row_mode ? 0 : tc.shard];
+      const int y0 = tc.m0 + static_cast<int>(rank) * C::BM;
+      // All 128 epilogue threads take the same decision (they meet at named
+      // barriers below).
+      if (!named_barrier_and(1, 128, mbar_wait(&tfull[acc], acc_phase))) break;
       tc_fence_after();
-      const int grow = tc.m0 + static_cast<int>(rank) * C::BM + row_local;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
-      for (int c = 0; c < C::BN / 32; ++c) {
-        if (c * 32 >= tc.n_valid) break;  // uniform across the CTA
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_row + c * 32, r);
-        tmem_wait_ld();
-        if (grow < p.M) {
+      const int nchunks = (tc.n_valid + cw - 1) / cw;
+      for (int c = 0; c < nchunks; ++c) {
+        // The TMA store that last read this staging buffer must be done with it.
+        if (elected) bulk_wait_group_read<1>();
+        named_barrier_sync(1, 128);
+        uint8_t* stage_row = sEpi + buf * C::EPI_BUF_BYTES + row_local * 128;
+        if (p.out_f32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + c * 32, r);
+          tmem_wait_ld();
 #pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const int col = c * 32 + g * 8;
-            if (col < tc.n_valid) {
-              float v[8];
+          for (int j = 0; j < 8; ++j) {  // 16-byte chunk j = 4 f32
+            uint4 w;
+            w.x = __float_as_uint(apply_act(__uint_as_float(r[4 * j + 0]), p.act));
+            w.y = __float_as_uint(apply_act(__uint_as_float(r[4 * j + 1]), p.act));
+            w.z = __float_as_uint(apply_act(__uint_as_float(r[4 * j + 2]), p.act));
+            w.w = __float_as_uint(apply_act(__uint_as_float(r[4 * j + 3]), p.act));
+            *reinterpret_cast<uint4*>(stage_row + ((j ^ (row_local & 7)) << 4)) = w;
+          }
+        } else {
 #pragma unroll
-              for (int e = 0; e < 8; ++e) v[e] = apply_act(__uint_as_float(r[g * 8 + e]), p.act);
-              const long long off = static_cast<long long>(grow) * p.ldc + tc.out_col0 + col;
-              if (p.out_f32) {
-                float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.C) + off);
-                dst[0] = make_float4(v[0], v[1], v[2], v[3]);
-                dst[1] = make_float4(v[4], v[5], v[6], v[7]);
-              } else {
-                uint4 w;
-                w.x = pack_bf16x2(v[0], v[1]);
-                w.y = pack_bf16x2(v[2], v[3]);
-                w.z = pack_bf16x2(v[4], v[5]);
-                w.w = pack_bf16x2(v[6], v[7]);
-                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + off) = w;
-              }
+          for (int h = 0; h < 2; ++h) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_row + c * 64 + h * 32, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {  // 16-byte chunk 4h+j = 8 bf16
+              uint4 w;
+              w.x = pack_bf16x2(apply_act(__uint_as_float(r[8 * j + 0]), p.act),
+                                apply_act(__uint_as_float(r[8 * j + 1]), p.act));
+              w.y = pack_bf16x2(apply_act(__uint_as_float(r[8 * j + 2]), p.act),
+                                apply_act(__uint_as_float(r[8 * j + 3]), p.act));
+              w.z = pack_bf16x2(apply_act(__uint_as_float(r[8 * j + 4]), p.act),
+                                apply_act(__uint_as_float(r[8 * j + 5]), p.act));
+              w.w = pack_bf16x2(apply_act(__uint_as_float(r[8 * j + 6]), p.act),
+                                apply_act(__uint_as_float(r[8 * j + 7]), p.act));
+              *reinterpret_cast<uint4*>(stage_row + (((4 * h + j) ^ (row_local & 7)) << 4)) = w;
             }
           }
         }
-      }
-      tc_fence_before();
-      if constexpr (CG == 1) {
-        mbar_arrive(&tempty[acc]);
-      } else {
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(tempty_leader0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+        if (c == nchunks - 1) {
+          // Every accumulator column of this tile has been read: hand the
+          // TMEM buffer back to the MMA issuer before the last store.
+          tc_fence_before();
+          if constexpr (CG == 1) {
+            mbar_arrive(&tempty[acc]);
+          } else {
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(tempty_leader0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+          }
+        }
+        fence_proxy_async_smem();
+        named_barrier_sync(1, 128);
+        if (elected && y0 < p.M) {
+          tma_store_3d(tmC, sEpi + buf * C::EPI_BUF_BYTES, tc.n_in + c * cw, y0, split);
+          bulk_commit_group();
+        }
+        buf ^= 1;
       }
       if (++acc == 2) { acc = 0; acc_phase ^= 1; }
     }
+    if (elected) bulk_wait_group_all();
   }
 
   tc_fence_before();

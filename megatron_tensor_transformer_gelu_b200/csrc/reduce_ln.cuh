@@ -1,4 +1,4 @@
-// Shard reduce + residual + LayerNorm, one CTA per row:
+// Shard reduce + residual + LayerNorm, 1 to 8 rows per CTA:
 //
 //   Z = X + sum_p P_p ;   Y = (Z - mean(Z)) / sqrt(var(Z) + eps) * gamma + beta
 //
@@ -8,10 +8,11 @@
 // row in a fixed order (two passes over registers: mean, then the biased
 // variance of the centred values), so a run is bitwise repeatable.
 //
-// Memory access: every thread moves 8 consecutive elements per step with
+// Memory access: every lane moves 8 consecutive elements per chunk with
 // 128-bit loads/stores (2 x float4 of each f32 partial, one uint4 of bf16 X or
-// Y), consecutive threads take consecutive 8-element chunks, so each warp
-// touches 1 KiB (f32) / 512 B (bf16) contiguous per step.
+// Y); consecutive lanes take consecutive chunks, so each warp touches 1 KiB
+// (f32) / 512 B (bf16) contiguous per step.  The f32 partials are read once,
+// with the streaming (evict-first) cache hint.
 #pragma once
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -19,8 +20,10 @@
 namespace tp {
 
 namespace rln {
-constexpr int THREADS = 256;
-constexpr int MAX_CHUNKS = 8;  // 8-element chunks per thread: H <= 8 * 8 * 256 = 16384
+constexpr int THREADS = 256;       // 8 warps per CTA
+constexpr int CH = 8;              // 8-element chunks per lane (64 values in registers)
+constexpr int MAX_WPR = 8;         // warps per row: H <= MAX_WPR * 32 * CH * 8 = 16384
+constexpr int MAX_H = MAX_WPR * 32 * CH * 8;
 }
 
 struct ReduceLnArgs {
@@ -37,19 +40,6 @@ struct ReduceLnArgs {
   int y_bf16;
 };
 
-__device__ __forceinline__ float block_sum_256(float v, float* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-  __syncthreads();  // `red` may still be read from a previous call
-  if (l == 0) red[w] = v;
-  __syncthreads();
-  float t = 0.0f;
-#pragma unroll
-  for (int i = 0; i < rln::THREADS / 32; ++i) t += red[i];  // same order in every thread
-  return t;
-}
-
 __device__ __forceinline__ void load8_bf16(const __nv_bfloat16* src, float* v) {
   const uint4 u = *reinterpret_cast<const uint4*>(src);
   const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
@@ -61,42 +51,82 @@ __device__ __forceinline__ void load8_bf16(const __nv_bfloat16* src, float* v) {
   }
 }
 
+// Streaming load (read once: evict first).
 __device__ __forceinline__ void load8_f32(const float* src, float* v) {
+  const float4 a = __ldcs(reinterpret_cast<const float4*>(src));
+  const float4 b = __ldcs(reinterpret_cast<const float4*>(src) + 1);
+  v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+  v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// Cached load (gamma/beta are read by every row).
+__device__ __forceinline__ void load8_f32_keep(const float* src, float* v) {
   const float4 a = reinterpret_cast<const float4*>(src)[0];
   const float4 b = reinterpret_cast<const float4*>(src)[1];
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-template <int CHUNKS>
+// One row is handled by WPR consecutive warps; a CTA holds 8 / WPR rows.  Lane
+// l of warp w (of the row) owns chunks c = 0..CH-1 at column
+// ((c * WPR + w) * 32 + l) * 8, so each warp reads 32 consecutive 8-element
+// chunks per step.  Every load of a lane is issued before the first reduction.
+template <int WPR>
 __global__ void __launch_bounds__(rln::THREADS) reduce_residual_ln_kernel(const ReduceLnArgs p) {
-  __shared__ float red[rln::THREADS / 32];
-  const long long row = blockIdx.x;
+  constexpr int RPC = rln::THREADS / 32 / WPR;  // rows per CTA
+  constexpr int CH = rln::CH;
+  __shared__ float red[2][RPC][WPR];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rloc = warp / WPR, wr = warp % WPR;
+  const long long row = static_cast<long long>(blockIdx.x) * RPC + rloc;
+  const bool live = row < p.S && rloc < RPC;
   const long long base = row * p.H;
-  float v[CHUNKS][8];
+  float v[CH][8];
   float s = 0.0f;
 #pragma unroll
-  for (int c = 0; c < CHUNKS; ++c) {
-    const int col = (c * rln::THREADS + threadIdx.x) * 8;
-    if (col < p.H) {
+  for (int c = 0; c < CH; ++c) {
+    const int col = ((c * WPR + wr) * 32 + lane) * 8;
+    if (live && col < p.H) {
       if (p.x_bf16) load8_bf16(static_cast<const __nv_bfloat16*>(p.X) + base + col, v[c]);
       else load8_f32(static_cast<const float*>(p.X) + base + col, v[c]);
-      for (int q = 0; q < p.nparts; ++q) {
+    }
+  }
+  for (int q = 0; q < p.nparts; ++q) {
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = ((c * WPR + wr) * 32 + lane) * 8;
+      if (live && col < p.H) {
         float w[8];
         load8_f32(p.parts + q * p.part_stride + base + col, w);
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[c][e] += w[e];
       }
+    }
+  }
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    const int col = ((c * WPR + wr) * 32 + lane) * 8;
+    if (live && col < p.H) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) s += v[c][e];
     }
   }
-  const float mean = block_sum_256(s, red) / static_cast<float>(p.H);
+  // mean over the row: warp shuffle, then the row's WPR warps in fixed order
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  if (lane == 0 && rloc < RPC) red[0][rloc][wr] = s;
+  __syncthreads();
+  float tot = 0.0f;
+  if (rloc < RPC) {
+#pragma unroll
+    for (int i = 0; i < WPR; ++i) tot += red[0][rloc][i];
+  }
+  const float mean = tot / static_cast<float>(p.H);
   float s2 = 0.0f;
 #pragma unroll
-  for (int c = 0; c < CHUNKS; ++c) {
-    const int col = (c * rln::THREADS + threadIdx.x) * 8;
-    if (col < p.H) {
+  for (int c = 0; c < CH; ++c) {
+    const int col = ((c * WPR + wr) * 32 + lane) * 8;
+    if (live && col < p.H) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const float d = v[c][e] - mean;
@@ -104,19 +134,35 @@ __global__ void __launch_bounds__(rln::THREADS) reduce_residual_ln_kernel(const 
       }
     }
   }
-  const float var = block_sum_256(s2, red) / static_cast<float>(p.H);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+  if (lane == 0 && rloc < RPC) red[1][rloc][wr] = s2;
+  __syncthreads();
+  float tot2 = 0.0f;
+  if (rloc < RPC) {
+#pragma unroll
+    for (int i = 0; i < WPR; ++i) tot2 += red[1][rloc][i];
+  }
+  const float var = tot2 / static_cast<float>(p.H);
   const float rstd = 1.0f / sqrtf(var + p.eps);
 #pragma unroll
-  for (int c = 0; c < CHUNKS; ++c) {
-    const int col = (c * rln::THREADS + threadIdx.x) * 8;
-    if (col < p.H) {
+  for (int c = 0; c < CH; ++c) {
+    const int col = ((c * WPR + wr) * 32 + lane) * 8;
+    if (live && col < p.H) {
+      float g[8], b[8];
+      if (p.gamma) load8_f32_keep(p.gamma + col, g);
+      else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) g[e] = 1.0f;
+      }
+      if (p.beta) load8_f32_keep(p.beta + col, b);
+      else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) b[e] = 0.0f;
+      }
       float y[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float g = p.gamma ? p.gamma[col + e] : 1.0f;
-        const float b = p.beta ? p.beta[col + e] : 0.0f;
-        y[e] = fmaf((v[c][e] - mean) * rstd, g, b);
-      }
+      for (int e = 0; e < 8; ++e) y[e] = fmaf((v[c][e] - mean) * rstd, g[e], b[e]);
       if (p.y_bf16) {
         uint4 u;
         __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]);

@@ -32,6 +32,9 @@ struct DeviceInfo {
   int max_pairs = 0;  // co-resident CTA pairs of the cta_group::2 GEMM
 };
 
+// Most K-split partial-sum slots a row-split GEMM feeding the LayerNorm may use.
+#define TP_MAX_K_SPLITS 4
+
 // GEMM flavour: CTA pairs (cta_group::2, 256-row tiles) unless the problem has
 // at most 128 rows, where a pair would leave half of every tile empty.
 #ifndef TP_GEMM_PAIR_MIN_ROWS
@@ -43,7 +46,7 @@ DeviceInfo g_dev[MAX_DEVICES];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 // ------------------------------------------------------------ event timing
-constexpr int PROF_CAP = 4096;
+constexpr int PROF_CAP = 16384;  // launches timed between two collects
 constexpr int PROF_KINDS = 4;
 bool g_prof_on = false;
 bool g_prof_events_made = false;
@@ -51,6 +54,7 @@ cudaEvent_t g_ev_start[PROF_CAP];
 cudaEvent_t g_ev_stop[PROF_CAP];
 int g_prof_kind[PROF_CAP];
 int g_prof_n = 0;
+long long g_prof_launches[PROF_KINDS];  // every launch while enabled, timed or not
 
 enum Kind { K_GEMM_TC = 0, K_REDUCE_LN = 1, K_GEMM_SIMT = 2, K_ATTN = 3 };
 
@@ -58,7 +62,9 @@ struct ProfScope {
   int slot = -1;
   cudaStream_t st;
   ProfScope(int kind, cudaStream_t s) : st(s) {
-    if (!g_prof_on || g_prof_n >= PROF_CAP) return;
+    if (!g_prof_on) return;
+    ++g_prof_launches[kind];
+    if (g_prof_n >= PROF_CAP) return;
     slot = g_prof_n++;
     g_prof_kind[slot] = kind;
     cudaEventRecord(g_ev_start[slot], st);
@@ -144,13 +150,54 @@ bool tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long cols,
   return r == CUDA_SUCCESS;
 }
 
+// 3-D output map {cols, rows, slots} over row-major [slots][rows][ld] (f32 or
+// bf16); box {128 bytes of columns, 128 rows, 1 slot}; 128-byte swizzle.  TMA
+// stores through it write nothing outside [cols] x [rows] x [slots].
+bool tmap_out(CUtensorMap* m, void* base, int f32, long long cols, long long rows, long long slots, long long ld,
+              long long slot_stride) {
+  const cuuint64_t es = f32 ? 4u : 2u;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(slots)};
+  const long long ss = slot_stride > 0 ? slot_stride : rows * ld;
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * es, static_cast<cuuint64_t>(ss) * es};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), 128u, 1u};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 int launch_status() { return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA; }
 
 // Tensor-core GEMM.  Column mode: B shard s is [K, shard_n], output columns
 // [s*shard_n, (s+1)*shard_n).  Row mode: B shard s is [shard_k, shard_n] and
 // multiplies A's columns [s*shard_k, (s+1)*shard_k); all shards are summed.
+// Number of K splits for `tiles` output tiles on `slots` persistent clusters,
+// from a small cost model: the main loop costs (waves x k-blocks per unit) k-
+// block times (about 0.5 us each for a 256 x 256 x 64 pair step), and every
+// extra f32 partial slot costs one write and one read of M x N x 4 bytes at
+// HBM speed (the reduce + LayerNorm kernel adds the slots).
+int choose_splits(long long tiles, int slots, int k_blocks, int max_splits, long long out_elems) {
+  const double t_kb = 0.48e-6;
+  const double slot_cost = static_cast<double>(out_elems) * 8.0 / 6.0e12;
+  int best = 1;
+  double best_t = 1e30;
+  for (int s = 1; s <= max_splits && s <= k_blocks; ++s) {
+    const long long units = tiles * s;
+    const long long waves = (units + slots - 1) / slots;
+    const long long kb = (k_blocks + s - 1) / s;
+    const double t = static_cast<double>(waves * kb) * t_kb + (s - 1) * slot_cost;
+    if (t < best_t * 0.98) {  // a split must buy at least 2%
+      best_t = t;
+      best = s;
+    }
+  }
+  return best;
+}
+
 template <int CG>
-int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, cudaStream_t st) {
+int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, int max_splits, cudaStream_t st) {
   using C = tp::GemmCfg<CG>;
   p.m_blocks = ceil_div(p.M, C::TILE_M);
   if (p.row_mode) {
@@ -162,7 +209,20 @@ int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, cudaStream_t st) {
   }
   const long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks;
   const int slots = CG == 2 ? dev.max_pairs : dev.sm_count;
-  const int clusters = static_cast<int>(tiles < slots ? tiles : slots);
+  p.splits = max_splits > 1
+                 ? choose_splits(tiles, slots, p.k_blocks, max_splits, static_cast<long long>(p.M) * p.shard_n)
+                 : 1;
+  const long long es = p.out_f32 ? 4 : 2;
+  if (p.row_mode) {
+    if (!tmap_out(&p.tmC[0], p.C, p.out_f32, p.shard_n, p.M, p.splits, p.ldc, p.slot_stride)) return TP_ERR_CUDA;
+  } else {
+    for (int s = 0; s < p.t; ++s) {
+      void* base = static_cast<uint8_t*>(p.C) + static_cast<long long>(s) * p.shard_n * es;
+      if (!tmap_out(&p.tmC[s], base, p.out_f32, p.shard_n, p.M, 1, p.ldc, 0)) return TP_ERR_CUDA;
+    }
+  }
+  const long long units = tiles * p.splits;
+  const int clusters = static_cast<int>(units < slots ? units : slots);
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeClusterDimension;
@@ -183,9 +243,13 @@ int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, cudaStream_t st) {
 // Tensor-core GEMM.  Column mode: B shard s is [K, shard_n], output columns
 // [s*shard_n, (s+1)*shard_n).  Row mode: B shard s is [shard_k, shard_n] and
 // multiplies A's columns [s*shard_k, (s+1)*shard_k); all shards are summed.
+// With max_splits > 1 (f32 output only) the K loop may be cut into up to
+// max_splits ranges whose partial sums land in slots `slot_stride` elements
+// apart; *splits_out tells the caller how many slots to add.
 int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, const void* const* B, int t,
                 int row_mode, int shard_k, int shard_n, void* C, long long ldc, int out_f32, int act,
-                cudaStream_t st) {
+                cudaStream_t st, int max_splits = 1, long long slot_stride = 0, int* splits_out = nullptr) {
+  if (splits_out) *splits_out = 1;
   using G = tp::GemmCfg<1>;
   if (M == 0) return TP_OK;
   tp::GemmArgs p;
@@ -206,8 +270,13 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
   p.k_blocks = row_mode ? p.k_blocks_per_shard * t : p.k_blocks_per_shard;
   p.act = act;
   p.out_f32 = out_f32;
-  if (M >= TP_GEMM_PAIR_MIN_ROWS) return launch_gemm_tc<2>(dev, p, st);
-  return launch_gemm_tc<1>(dev, p, st);
+  p.splits = 1;
+  p.slot_stride = slot_stride;
+  if (!out_f32) max_splits = 1;
+  const int r = M >= TP_GEMM_PAIR_MIN_ROWS ? launch_gemm_tc<2>(dev, p, max_splits, st)
+                                           : launch_gemm_tc<1>(dev, p, max_splits, st);
+  if (splits_out) *splits_out = p.splits;
+  return r;
 }
 
 int run_gemm_simt(const float* A, long long lda, int M, const void* const* B, int t, int row_mode, int shard_k,
@@ -249,11 +318,12 @@ int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, i
   p.eps = eps;
   p.Y = Y;
   p.y_bf16 = y_bf16;
-  const int chunks = ceil_div(H, 8 * tp::rln::THREADS);
+  // warps per row: each lane holds CH chunks of 8 values
+  const int wpr_needed = ceil_div(H, 32 * tp::rln::CH * 8);
   ProfScope ps(K_REDUCE_LN, st);
-  if (chunks <= 1) tp::reduce_residual_ln_kernel<1><<<S, tp::rln::THREADS, 0, st>>>(p);
-  else if (chunks <= 2) tp::reduce_residual_ln_kernel<2><<<S, tp::rln::THREADS, 0, st>>>(p);
-  else if (chunks <= 4) tp::reduce_residual_ln_kernel<4><<<S, tp::rln::THREADS, 0, st>>>(p);
+  if (wpr_needed <= 1) tp::reduce_residual_ln_kernel<1><<<ceil_div(S, 8), tp::rln::THREADS, 0, st>>>(p);
+  else if (wpr_needed <= 2) tp::reduce_residual_ln_kernel<2><<<ceil_div(S, 4), tp::rln::THREADS, 0, st>>>(p);
+  else if (wpr_needed <= 4) tp::reduce_residual_ln_kernel<4><<<ceil_div(S, 2), tp::rln::THREADS, 0, st>>>(p);
   else tp::reduce_residual_ln_kernel<8><<<S, tp::rln::THREADS, 0, st>>>(p);
   return launch_status();
 }
@@ -272,7 +342,7 @@ bool shards_ok(const void* const* s, int t) {
 }
 bool ptr_ok(const void* p) { return p && aligned16(p); }
 bool opt_ptr_ok(const void* p) { return !p || aligned16(p); }
-bool hidden_ok(int H) { return H >= 8 && H % 8 == 0 && H <= 8 * tp::rln::THREADS * tp::rln::MAX_CHUNKS; }
+bool hidden_ok(int H) { return H >= 8 && H % 8 == 0 && H <= tp::rln::MAX_H; }
 
 }  // namespace
 
@@ -308,7 +378,8 @@ size_t tp_mlp_workspace_bytes(int S, int H, int F, int t, int dtype) {
   if (S < 0 || H <= 0 || F <= 0 || t < 1 || !valid_dtype(dtype)) return 0;
   (void)t;
   const size_t eh = dtype == TP_DTYPE_BF16 ? 2 : 4;
-  return align256(static_cast<size_t>(S) * F * eh) + static_cast<size_t>(S) * H * 4;
+  const size_t slots = dtype == TP_DTYPE_BF16 ? TP_MAX_K_SPLITS : 1;
+  return align256(static_cast<size_t>(S) * F * eh) + slots * static_cast<size_t>(S) * H * 4;
 }
 
 int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype, const void* X,
@@ -331,6 +402,7 @@ int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype, const v
   if (S == 0) return TP_OK;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int Fs = F / t;
+  int nparts = 1;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t eh = dtype == TP_DTYPE_BF16 ? 2 : 4;
   void* Hbuf = ws;
@@ -340,9 +412,10 @@ int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype, const v
     st = run_gemm_tc(*dev, X, H, S, A_shards, t, /*row_mode=*/0, /*shard_k=*/H, /*shard_n=*/Fs, Hbuf, F,
                      /*out_f32=*/0, act, s);
     if (st != TP_OK) return st;
-    // Zsum = sum_i H_i B_i, accumulated in TMEM across the shards (f32).
+    // Zsum = sum_i H_i B_i, accumulated in TMEM across the shards (f32); the K
+    // loop may be cut into `nparts` ranges (partial-sum slots) to fill the GPU.
     st = run_gemm_tc(*dev, Hbuf, F, S, B_shards, t, /*row_mode=*/1, /*shard_k=*/Fs, /*shard_n=*/H, Zsum, H,
-                     /*out_f32=*/1, TP_ACT_NONE, s);
+                     /*out_f32=*/1, TP_ACT_NONE, s, TP_MAX_K_SPLITS, static_cast<long long>(S) * H, &nparts);
     if (st != TP_OK) return st;
   } else {
     st = run_gemm_simt(static_cast<const float*>(X), H, S, A_shards, t, 0, H, Fs, static_cast<float*>(Hbuf), F,
@@ -351,7 +424,7 @@ int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype, const v
     st = run_gemm_simt(static_cast<const float*>(Hbuf), F, S, B_shards, t, 1, Fs, H, Zsum, H, TP_ACT_NONE, s);
     if (st != TP_OK) return st;
   }
-  return run_reduce_ln(S, H, 1, Zsum, X, dtype == TP_DTYPE_BF16, gamma, beta, eps, Y,
+  return run_reduce_ln(S, H, nparts, Zsum, X, dtype == TP_DTYPE_BF16, gamma, beta, eps, Y,
                        out_dtype == TP_DTYPE_BF16, s);
 }
 
@@ -359,7 +432,7 @@ int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype, const v
 size_t tp_attn_workspace_bytes(int S, int H, int nh, int d, int t, int dtype) {
   if (S < 0 || H <= 0 || nh <= 0 || d <= 0 || t < 1 || dtype != TP_DTYPE_BF16) return 0;
   const size_t s = static_cast<size_t>(S), h = static_cast<size_t>(H);
-  return align256(s * 3 * h * 2) + align256(s * h * 2) + s * h * 4;
+  return align256(s * 3 * h * 2) + align256(s * h * 2) + TP_MAX_K_SPLITS * s * h * 4;
 }
 
 int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int out_dtype, const void* X,
@@ -411,9 +484,11 @@ int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int
     if (st != TP_OK) return st;
   }
   // sum_s O_s Wo_s, the O projection row-split by head, summed in TMEM.
-  st = run_gemm_tc(*dev, Obuf, H, S, Wo_shards, t, 1, Hs, H, Zsum, H, 1, TP_ACT_NONE, s);
+  int nparts = 1;
+  st = run_gemm_tc(*dev, Obuf, H, S, Wo_shards, t, 1, Hs, H, Zsum, H, 1, TP_ACT_NONE, s, TP_MAX_K_SPLITS,
+                   static_cast<long long>(S) * H, &nparts);
   if (st != TP_OK) return st;
-  return run_reduce_ln(S, H, 1, Zsum, X, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s);
+  return run_reduce_ln(S, H, nparts, Zsum, X, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s);
 }
 
 // ---------------------------------------------------------------- linears
@@ -483,13 +558,15 @@ int tp_profile_enable(int on) {
   }
   g_prof_on = on != 0;
   g_prof_n = 0;
+  for (int k = 0; k < PROF_KINDS; ++k) g_prof_launches[k] = 0;
   return TP_OK;
 }
 
-int tp_profile_collect(int* launches, double* ms, int max_kinds) {
+int tp_profile_collect(int* launches, int* timed, double* ms, int max_kinds) {
   const int nk = max_kinds < PROF_KINDS ? max_kinds : PROF_KINDS;
   for (int k = 0; k < nk; ++k) {
-    if (launches) launches[k] = 0;
+    if (launches) launches[k] = static_cast<int>(g_prof_launches[k]);
+    if (timed) timed[k] = 0;
     if (ms) ms[k] = 0.0;
   }
   for (int i = 0; i < g_prof_n; ++i) {
@@ -499,10 +576,11 @@ int tp_profile_collect(int* launches, double* ms, int max_kinds) {
     if (cudaEventSynchronize(g_ev_stop[i]) != cudaSuccess ||
         cudaEventElapsedTime(&t, g_ev_start[i], g_ev_stop[i]) != cudaSuccess)
       return -TP_ERR_CUDA;
-    if (launches) launches[k] += 1;
+    if (timed) timed[k] += 1;
     if (ms) ms[k] += t;
   }
   g_prof_n = 0;
+  for (int k = 0; k < PROF_KINDS; ++k) g_prof_launches[k] = 0;
   return nk;
 }
 

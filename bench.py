@@ -301,6 +301,8 @@ def run_ours(args, rank, world, local):
                 "peak_source": peaks["source"] + " bf16 burst (MEASURED_PEAKS.json bf16_tflops)",
                 "unit": "TFLOP/s",
                 "frac": round(achieved / peaks["bf16_tflops"], 4) if achieved else None,
+                "frac_of_sustained": (round(achieved / peaks["bf16_tflops_sustained"], 4)
+                                      if achieved and peaks.get("bf16_tflops_sustained") else None),
                 "traffic": traffic,
                 "flops_per_launch": gemm_flops_per_launch,
                 "avg_launch_ms": round(g_ms / g_launch, 5) if g_launch else None,

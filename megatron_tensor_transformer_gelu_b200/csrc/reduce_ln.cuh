@@ -21,9 +21,9 @@ namespace tp {
 
 namespace rln {
 constexpr int THREADS = 256;       // 8 warps per CTA
-constexpr int CH = 8;              // 8-element chunks per lane (64 values in registers)
-constexpr int MAX_WPR = 8;         // warps per row: H <= MAX_WPR * 32 * CH * 8 = 16384
-constexpr int MAX_H = MAX_WPR * 32 * CH * 8;
+constexpr int MAX_WPR = 8;         // warps per row
+constexpr int MAX_CH = 8;          // 8-element chunks per lane
+constexpr int MAX_H = MAX_WPR * 32 * MAX_CH * 8;  // 16384
 }
 
 struct ReduceLnArgs {
@@ -70,11 +70,11 @@ __device__ __forceinline__ void load8_f32_keep(const float* src, float* v) {
 // One row is handled by WPR consecutive warps; a CTA holds 8 / WPR rows.  Lane
 // l of warp w (of the row) owns chunks c = 0..CH-1 at column
 // ((c * WPR + w) * 32 + l) * 8, so each warp reads 32 consecutive 8-element
-// chunks per step.  Every load of a lane is issued before the first reduction.
-template <int WPR>
+// chunks per step.  CH = 4 (32 values per lane, ~60 registers, 4 CTAs per SM)
+// up to H = 8192; CH = 8 beyond.
+template <int WPR, int CH>
 __global__ void __launch_bounds__(rln::THREADS) reduce_residual_ln_kernel(const ReduceLnArgs p) {
   constexpr int RPC = rln::THREADS / 32 / WPR;  // rows per CTA
-  constexpr int CH = rln::CH;
   __shared__ float red[2][RPC][WPR];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rloc = warp / WPR, wr = warp % WPR;

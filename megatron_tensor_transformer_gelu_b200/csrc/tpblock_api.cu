@@ -318,13 +318,14 @@ int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, i
   p.eps = eps;
   p.Y = Y;
   p.y_bf16 = y_bf16;
-  // warps per row: each lane holds CH chunks of 8 values
-  const int wpr_needed = ceil_div(H, 32 * tp::rln::CH * 8);
+  // warps per row (each lane holds CH chunks of 8 values); 8 / WPR rows per CTA
   ProfScope ps(K_REDUCE_LN, st);
-  if (wpr_needed <= 1) tp::reduce_residual_ln_kernel<1><<<ceil_div(S, 8), tp::rln::THREADS, 0, st>>>(p);
-  else if (wpr_needed <= 2) tp::reduce_residual_ln_kernel<2><<<ceil_div(S, 4), tp::rln::THREADS, 0, st>>>(p);
-  else if (wpr_needed <= 4) tp::reduce_residual_ln_kernel<4><<<ceil_div(S, 2), tp::rln::THREADS, 0, st>>>(p);
-  else tp::reduce_residual_ln_kernel<8><<<S, tp::rln::THREADS, 0, st>>>(p);
+  const int T = tp::rln::THREADS;
+  if (H <= 1024) tp::reduce_residual_ln_kernel<1, 4><<<ceil_div(S, 8), T, 0, st>>>(p);
+  else if (H <= 2048) tp::reduce_residual_ln_kernel<2, 4><<<ceil_div(S, 4), T, 0, st>>>(p);
+  else if (H <= 4096) tp::reduce_residual_ln_kernel<4, 4><<<ceil_div(S, 2), T, 0, st>>>(p);
+  else if (H <= 8192) tp::reduce_residual_ln_kernel<8, 4><<<S, T, 0, st>>>(p);
+  else tp::reduce_residual_ln_kernel<8, 8><<<S, T, 0, st>>>(p);
   return launch_status();
 }
 

@@ -107,6 +107,29 @@ int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype,
                    const float* gamma, const float* beta, float eps, int act,
                    void* Y, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------- MLP without allocation ----
+ * The pages have no counterpart to this entry point: it exists for callers
+ * that cannot allocate device memory (plugin hosts that forbid allocation in
+ * their execute hook, latency-critical loops that cannot afford cudaMalloc's
+ * implicit synchronisation, programs whose own allocator holds the device
+ * memory).  Same arguments and result as tp_mlp_forward, minus the workspace:
+ * the scratch is a fixed device array inside the library, of
+ * tp_noalloc_scratch_bytes() bytes (32 MiB), held on every GPU that loads the
+ * library until the process exits.
+ *  - Sizes whose tp_mlp_workspace_bytes() exceeds that maximum are rejected
+ *    with TP_ERR_WORKSPACE_TOO_SMALL before anything is launched.
+ *  - The call allocates nothing.  Its first call on a device looks up the
+ *    array's device address (with that device current); make that first call
+ *    before any stream capture.
+ *  - Every call on a device shares the array: calls whose kernels may overlap
+ *    on the GPU race on it; order them on one stream.  Nothing in it needs to
+ *    start at zero. */
+size_t tp_noalloc_scratch_bytes(void);
+int tp_mlp_forward_noalloc(int S, int H, int F, int t, int dtype, int out_dtype,
+                           const void* X, const void* const* A_shards, const void* const* B_shards,
+                           const float* gamma, const float* beta, float eps, int act,
+                           void* Y, void* stream);
+
 /* ------------------------------------------------------------ attention ----
  * Y = LN(X + concat_h(softmax(Q_h K_h^T / sqrt d) V_h) Wo), non-causal, no
  * mask, heads split over t shards of nh/t heads.  [0539] §1.2.2 (every head

@@ -32,6 +32,8 @@ SIGNATURES = {
     "tp_device_error": (_c_int, []),
     "tp_mlp_workspace_bytes": (_c_size, [_c_int] * 5),
     "tp_mlp_forward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vpp, _vp, _vp, _c_float, _c_int, _vp, _vp, _c_size, _vp]),
+    "tp_noalloc_scratch_bytes": (_c_size, []),
+    "tp_mlp_forward_noalloc": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vpp, _vp, _vp, _c_float, _c_int, _vp, _vp]),
     "tp_attn_workspace_bytes": (_c_size, [_c_int] * 6),
     "tp_qkv_attn_oproj_forward": (_c_int, [_c_int] * 7 + [_vp, _vpp, _vpp, _vp, _vp, _c_float, _vp, _vp, _c_size, _vp]),
     "tp_linear_column_forward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _c_int, _vp, _vp]),
@@ -109,6 +111,19 @@ def mlp_forward(X, A_shards, B_shards, Y, workspace, gamma=None, beta=None, eps=
                                 _ptr(workspace), workspace.numel() * workspace.element_size()
                                 if workspace is not None else 0, _stream(stream))
     _check(code, "tp_mlp_forward")
+
+
+def mlp_forward_noalloc(X, A_shards, B_shards, Y, gamma=None, beta=None, eps=1e-5, act="gelu_tanh",
+                       stream=None):
+    """tp_mlp_forward with the library's fixed scratch array instead of a workspace."""
+    S, H = X.shape
+    t = len(A_shards)
+    F = sum(a.shape[1] for a in A_shards)
+    pa, ka = _ptrs(A_shards)
+    pb, kb = _ptrs(B_shards)
+    code = lib().tp_mlp_forward_noalloc(S, H, F, t, DTYPE[X.dtype], DTYPE[Y.dtype], _ptr(X), pa, pb,
+                                        _ptr(gamma), _ptr(beta), float(eps), ACT[act], _ptr(Y), _stream(stream))
+    _check(code, "tp_mlp_forward_noalloc")
 
 
 def attn_forward(X, Wqkv_shards, Wo_shards, nh, d, Y, workspace, gamma=None, beta=None, eps=1e-5,

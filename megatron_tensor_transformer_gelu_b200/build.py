@@ -13,7 +13,7 @@ import sys
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-SRC = os.path.join(HERE, "csrc", "tpblock_api.cu")
+SRCS = [os.path.join(HERE, "csrc", "tpblock_api.cu"), os.path.join(HERE, "csrc", "tp_noalloc.cu")]
 OUT = os.path.join(HERE, "libtpblock.so")
 
 NVCC_FLAGS = [
@@ -47,7 +47,7 @@ def up_to_date() -> bool:
 def build(force: bool = False, verbose: bool = False, extra: list[str] | None = None) -> str:
     if not force and up_to_date():
         return OUT
-    cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), SRC, "-o", OUT + ".tmp"]
+    cmd = [nvcc(), *NVCC_FLAGS, *(extra or []), *SRCS, "-o", OUT + ".tmp"]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)

@@ -169,6 +169,58 @@ def whole_job_tflops(flops_per_step: int, steps: int, world: int, ms_max: float)
 
 # ----------------------------------------------------------------- our arm
 
+class Problem:
+    """Device inputs and the step of one workload, plus the algorithmic work of
+    each kernel kind per step (FLOPs for tensor-core kinds, bytes for the
+    LayerNorm kind)."""
+
+    def __init__(self, w, dev, rank, L, synth, torch):
+        self.w = w
+        t = w.t
+        bf = torch.bfloat16
+        if w.kind == "mlp":
+            S, H, F = w.S, w.H, w.F
+            inp = synth.gen_mlp(S, H, F, seed=w.seed + rank)
+            self.X = inp.X.to(dev)
+            self.W1 = [a.to(dev) for a in synth.split_columns(inp.A, t)]
+            self.W2 = [b.to(dev) for b in synth.split_rows(inp.B, t)]
+            self.Y = torch.empty(S, H, dtype=bf, device=dev)
+            self.ws = torch.empty(L.mlp_workspace_bytes(S, H, F, t, bf), dtype=torch.uint8, device=dev)
+            self.work = {"gemm_tcgen05": 2 * 2 * S * H * F,
+                         "reduce_residual_layernorm": S * H * 4 + S * H * 2 * 2 + H * 8}
+            self.Xh_src = inp.X
+            self.run = lambda X, Y, st: L.mlp_forward(X, self.W1, self.W2, Y, self.ws, stream=st)
+        elif w.kind == "attn":
+            S, H = w.S, w.H
+            inp = synth.gen_attn(S, H, seed=w.seed + rank)
+            self.X = inp.X.to(dev)
+            self.W1 = [q.to(dev) for q in synth.split_qkv_by_head(inp.Wqkv, w.nh, w.d, t)]
+            self.W2 = [o.to(dev) for o in synth.split_rows_by_head(inp.Wo, w.nh, w.d, t)]
+            self.Y = torch.empty(S, H, dtype=bf, device=dev)
+            self.ws = torch.empty(L.attn_workspace_bytes(S, H, w.nh, w.d, t), dtype=torch.uint8, device=dev)
+            self.work = {"gemm_tcgen05": 2 * S * H * 3 * H + 2 * S * H * H,
+                         "attention_fwd": 4 * S * S * w.d * w.nh,
+                         "reduce_residual_layernorm": S * H * 4 + S * H * 2 * 2 + H * 8}
+            self.Xh_src = inp.X
+            self.run = lambda X, Y, st: L.attn_forward(X, self.W1, self.W2, w.nh, w.d, Y, self.ws, stream=st)
+        else:
+            M, K, N = w.M, w.K, w.N
+            inp = synth.gen_linear(M, K, N, seed=w.seed + rank)
+            self.X = inp.X.to(dev)
+            split = synth.split_columns if w.kind == "linear_col" else synth.split_rows
+            self.W1 = [s_.to(dev) for s_ in split(inp.W, t)]
+            self.W2 = []
+            self.Y = torch.empty(M, N, dtype=torch.float32, device=dev)
+            self.ws = None
+            self.work = {"gemm_tcgen05": 2 * M * K * N}
+            self.Xh_src = inp.X
+            if w.kind == "linear_col":
+                self.run = lambda X, Y, st: L.linear_column_forward(X, self.W1, Y, stream=st)
+            else:
+                self.run = lambda X, Y, st: L.linear_row_forward(X, self.W1, Y, stream=st)
+        self.input_bytes = sum(x.numel() * x.element_size() for x in [self.X, *self.W1, *self.W2])
+
+
 def run_ours(args, rank, world, local):
     import torch
     import torch.distributed as dist
@@ -178,7 +230,7 @@ def run_ours(args, rank, world, local):
     from megatron_tensor_transformer_gelu_b200.workloads import HEADLINE, WORKLOADS
 
     w = WORKLOADS[args.workload or HEADLINE]
-    assert w.kind == "mlp" and w.dtype == "bf16"
+    assert w.dtype == "bf16", "the benchmark times the bf16 tensor-core path"
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
@@ -191,18 +243,12 @@ def run_ours(args, rank, world, local):
     if world > 1:
         dist.barrier()
     L.lib()  # load the CUDA library (raises if it is not built)
-    S, H, F, t = w.S, w.H, w.F, w.t
-    inp = synth.gen_mlp(S, H, F, seed=w.seed + rank)
-    X = inp.X.to(dev)
-    As = [a.to(dev) for a in synth.split_columns(inp.A, t)]
-    Bs = [b.to(dev) for b in synth.split_rows(inp.B, t)]
-    Y = torch.empty(S, H, dtype=torch.bfloat16, device=dev)
-    ws = torch.empty(L.mlp_workspace_bytes(S, H, F, t, torch.bfloat16), dtype=torch.uint8, device=dev)
+    P = Problem(w, dev, rank, L, synth, torch)
+    X, Y = P.X, P.Y
     stream = torch.cuda.Stream(device=dev)
-    input_bytes = (X.numel() + sum(a.numel() for a in As) + sum(b.numel() for b in Bs)) * 2
 
     def step():
-        L.mlp_forward(X, As, Bs, Y, ws, stream=stream)
+        P.run(X, Y, stream)
 
     def barrier():
         torch.cuda.synchronize()
@@ -212,9 +258,8 @@ def run_ours(args, rank, world, local):
 
     sampler = ClockSampler(local)
     time.sleep(0.3)
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            step()
+    for _ in range(args.warmup):
+        step()
     barrier()
     # ---- timed region: K steps, device time on the launching stream
     L.profile_enable(True)
@@ -232,28 +277,53 @@ def run_ours(args, rank, world, local):
     L.profile_enable(False)
     assert L.device_error() == 0, "a device-side wait timed out"
 
-    # ---- end to end through the public call with host buffers
-    Xh = inp.X.pin_memory()
-    Yh = torch.empty(S, H, dtype=torch.bfloat16).pin_memory()
-    Xd = torch.empty_like(X)
+    # ---- end to end through the public call with host buffers.  Step i copies
+    # its X from pinned host memory (copy stream h2d), runs the sublayer (compute
+    # stream) and copies its Y back to pinned host memory (copy stream d2h);
+    # device buffers are double-buffered so step i+1's upload and step i-1's
+    # download overlap step i's compute.  The timed region spans the first
+    # upload to the last download.
+    nbuf = 2
+    Xh = [P.Xh_src.pin_memory() for _ in range(nbuf)]
+    Yh = [torch.empty(Y.shape, dtype=Y.dtype).pin_memory() for _ in range(nbuf)]
+    Xd = [torch.empty_like(X) for _ in range(nbuf)]
+    Yd = [torch.empty_like(Y) for _ in range(nbuf)]
+    h2d = torch.cuda.Stream(device=dev)
+    d2h = torch.cuda.Stream(device=dev)
+    ev_up = [torch.cuda.Event() for _ in range(nbuf)]      # X[b] uploaded
+    ev_done = [torch.cuda.Event() for _ in range(nbuf)]    # sublayer on buffer b finished
+    ev_down = [torch.cuda.Event() for _ in range(nbuf)]    # Y[b] downloaded
 
-    def e2e_step():
-        Xd.copy_(Xh, non_blocking=True)
-        L.mlp_forward(Xd, As, Bs, Y, ws, stream=stream)
-        Yh.copy_(Y, non_blocking=True)
+    def e2e_run(n, first=None, last=None):
+        if first is not None:
+            first.record(h2d)
+        for i in range(n):
+            b = i % nbuf
+            if i >= nbuf:
+                h2d.wait_event(ev_done[b])      # X[b] free again
+            with torch.cuda.stream(h2d):
+                Xd[b].copy_(Xh[b], non_blocking=True)
+            ev_up[b].record(h2d)
+            stream.wait_event(ev_up[b])
+            if i >= nbuf:
+                stream.wait_event(ev_down[b])   # Y[b] free again
+            P.run(Xd[b], Yd[b], stream)
+            ev_done[b].record(stream)
+            d2h.wait_event(ev_done[b])
+            with torch.cuda.stream(d2h):
+                Yh[b].copy_(Yd[b], non_blocking=True)
+            ev_down[b].record(d2h)
+        if last is not None:
+            for b in range(nbuf):
+                h2d.wait_event(ev_down[b])
+            last.record(h2d)
 
-    e2e_steps = max(1, min(args.steps, 200))
-    with torch.cuda.stream(stream):
-        for _ in range(max(1, min(args.warmup, 5))):
-            e2e_step()
+    e2e_steps = max(nbuf, min(args.steps, 200))
+    e2e_run(max(nbuf, min(args.warmup, 5)))
     barrier()
-    with torch.cuda.stream(stream):
-        f0 = torch.cuda.Event(enable_timing=True)
-        f1 = torch.cuda.Event(enable_timing=True)
-        f0.record(stream)
-        for _ in range(e2e_steps):
-            e2e_step()
-        f1.record(stream)
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    e2e_run(e2e_steps, f0, f1)
     barrier()
     e2e_ms = f0.elapsed_time(f1)
     sampler.stop()
@@ -266,14 +336,46 @@ def run_ours(args, rank, world, local):
         ms_step = ms_total / args.steps
         value = whole_job_tflops(w.flops, args.steps, world, ms_total)
         e2e_value = whole_job_tflops(w.flops, e2e_steps, world, e2e_ms)
-        _, g_launch, g_ms = prof.get("gemm_tcgen05", (0, 0, 0.0))
-        _, ln_launch, ln_ms = prof.get("reduce_residual_layernorm", (0, 0, 0.0))
         launches = sum(v[0] for v in prof.values())
-        gemm_flops_per_launch = w.flops / 2  # both GEMMs are 2*S*H*F
-        achieved = gemm_flops_per_launch / (g_ms / g_launch * 1e-3) / 1e12 if g_launch else None
-        traffic = stored_traffic("gemm_tcgen05", w.name)
+        kinds = {}
+        for kind, work in P.work.items():
+            n_all, n_timed, ms_k = prof.get(kind, (0, 0, 0.0))
+            if not n_timed:
+                continue
+            per_launch_ms = ms_k / n_timed
+            launches_per_step = n_all / args.steps
+            tensor = kind != "reduce_residual_layernorm"
+            work_per_launch = work / launches_per_step
+            rate = work_per_launch / (per_launch_ms * 1e-3)
+            if tensor:
+                ach, pk, unit = rate / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+            else:
+                ach, pk, unit = rate / 1e9, peaks["hbm_gbs"], "GB/s"
+            kinds[kind] = {"bound": "tensor" if tensor else "hbm", "achieved": round(ach, 2), "peak": pk,
+                           "unit": unit, "frac": round(ach / pk, 4), "launches": n_all,
+                           "avg_launch_ms": round(per_launch_ms, 5),
+                           ("flops_per_launch" if tensor else "bytes_per_launch"): int(work_per_launch),
+                           "device_ms": ms_k}
+        total_k_ms = sum(k["device_ms"] for k in kinds.values())
+        for k in kinds.values():
+            k["share_of_step"] = round(k.pop("device_ms") / total_k_ms, 4)
+        dom = max(kinds, key=lambda k: kinds[k]["share_of_step"])
+        roof = dict(kinds.pop(dom))
+        roof = {"kernel": dom, **roof}
+        roof["peak_source"] = (peaks["source"] + (" bf16 burst (MEASURED_PEAKS.json bf16_tflops)"
+                                                  if roof["bound"] == "tensor" else " copy (MEASURED_PEAKS.json hbm_gbs)"))
+        if roof["bound"] == "tensor" and peaks.get("bf16_tflops_sustained"):
+            roof["frac_of_sustained"] = round(roof["achieved"] / peaks["bf16_tflops_sustained"], 4)
+        roof["traffic"] = stored_traffic(dom, w.name) if dom == "gemm_tcgen05" else None
         clocks = sampler.summary(t_wall0, t_wall1)
-        ln_bytes = S * H * 4 + S * H * 2 * 2 + H * 8  # Zsum f32 read, X read, Y written, gamma/beta
+        cfg = {"workload": w.name, "t": w.t, "flops_per_step": w.flops,
+               "parallelism": f"{w.t} logical TP shards per GPU; {world} independent replica(s)",
+               "l2": f"inputs larger than L2 ({P.input_bytes / 2**20:.0f} MiB resident vs {L2_BYTES // 2**20} MiB L2)"}
+        for key in ("S", "H", "F", "nh", "d", "M", "K", "N"):
+            if getattr(w, key):
+                cfg[key] = getattr(w, key)
+        if w.kind == "mlp":
+            cfg["act"] = "gelu_tanh"
         result = {
             "metric": METRIC,
             "value": round(value, 2),
@@ -287,40 +389,18 @@ def run_ours(args, rank, world, local):
             "vs_baseline": None,
             "dtype": "bf16",
             "data": "synthetic (seeded torch.randn; X~N(0,1), weights~N(0,1/fan_in))",
-            "config": {
-                "workload": w.name, "S": S, "H": H, "F": F, "t": t, "act": "gelu_tanh",
-                "flops_per_step": w.flops, "parallelism": f"{t} logical TP shards per GPU; {world} independent replicas",
-                "l2": f"inputs larger than L2 ({input_bytes / 2**20:.0f} MiB resident vs {L2_BYTES // 2**20} MiB L2)",
-            },
+            "config": cfg,
             "pct_of_peak": round(100 * value / world / peaks["bf16_tflops"], 2),
-            "roofline": {
-                "kernel": "gemm_tcgen05",
-                "bound": "tensor",
-                "achieved": round(achieved, 2) if achieved else None,
-                "peak": peaks["bf16_tflops"],
-                "peak_source": peaks["source"] + " bf16 burst (MEASURED_PEAKS.json bf16_tflops)",
-                "unit": "TFLOP/s",
-                "frac": round(achieved / peaks["bf16_tflops"], 4) if achieved else None,
-                "frac_of_sustained": (round(achieved / peaks["bf16_tflops_sustained"], 4)
-                                      if achieved and peaks.get("bf16_tflops_sustained") else None),
-                "traffic": traffic,
-                "flops_per_launch": gemm_flops_per_launch,
-                "avg_launch_ms": round(g_ms / g_launch, 5) if g_launch else None,
-                "launches": g_launch,
-                "share_of_step": round(g_ms / (g_ms + ln_ms), 4) if g_launch else None,
-            },
-            "other_kernels": {
-                "reduce_residual_layernorm": {
-                    "launches": ln_launch, "avg_launch_ms": round(ln_ms / max(ln_launch, 1), 5),
-                    "bound": "hbm", "bytes_per_launch": ln_bytes,
-                    "achieved_gbs": round(ln_bytes / (ln_ms / max(ln_launch, 1) * 1e-3) / 1e9, 1) if ln_launch else None,
-                    "peak_gbs": peaks["hbm_gbs"],
-                },
-            },
+            "roofline": roof,
+            "other_kernels": kinds,
             "e2e": {"value": round(e2e_value, 2), "unit": UNIT,
-                    "h2d_bytes_per_step": X.numel() * 2, "d2h_bytes_per_step": Y.numel() * 2,
+                    "h2d_bytes_per_step": X.numel() * X.element_size(),
+                    "d2h_bytes_per_step": Y.numel() * Y.element_size(),
                     "steps": e2e_steps,
-                    "note": "pinned host X -> device, tp_mlp_forward, device Y -> pinned host, one stream"},
+                    "note": ("per step: pinned host X -> device (copy stream), the C-ABI sublayer call (compute "
+                             "stream), device Y -> pinned host (copy stream); double-buffered so the copies of "
+                             "neighbouring steps overlap the compute; timed from the first upload to the last "
+                             "download")},
             "gpu_launches": launches,
             "clocks": clocks,
         }
@@ -333,30 +413,43 @@ def run_ours(args, rank, world, local):
 # -------------------------------------------------- oracle on host cores
 
 def cpu_oracle_timing(w, rows_per_step: int, steps: int, warmup: int):
-    """Time the fp64 oracle (as it stands) on a row sample of the workload."""
-    import numpy as np
-    import torch
+    """Time the fp64 oracle (as it stands) on a row sample of the workload.
 
+    `value` is workload-equivalent throughput: the workload's FLOPs times the
+    fraction of output rows produced, per second (for the attention sublayer
+    the oracle also recomputes every K and V row on each call)."""
     from megatron_tensor_transformer_gelu_b200 import synth
     from oracle import tp_oracle as O
 
-    inp = synth.gen_mlp(w.S, w.H, w.F, seed=w.seed)
-    rows = list(range(min(rows_per_step, w.S)))
+    if w.kind == "mlp":
+        inp = synth.gen_mlp(w.S, w.H, w.F, seed=w.seed)
+        nrows = w.S
+        call = lambda rows: O.mlp_block(inp.X, inp.A, inp.B, rows=rows)
+    elif w.kind == "attn":
+        inp = synth.gen_attn(w.S, w.H, seed=w.seed)
+        nrows = w.S
+        call = lambda rows: O.attention_sublayer(inp.X, inp.Wqkv, inp.Wo, w.nh, w.d, rows=rows)
+    else:
+        inp = synth.gen_linear(w.M, w.K, w.N, seed=w.seed)
+        nrows = w.M
+        call = lambda rows: O.linear_column(inp.X, inp.W, rows=rows)
+    rows = list(range(min(rows_per_step, nrows)))
     try:
         from threadpoolctl import threadpool_info
         cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=os.cpu_count())
     except Exception:  # pragma: no cover
         cores = os.cpu_count()
     for _ in range(warmup):
-        O.mlp_block(inp.X, inp.A, inp.B, rows=rows)
+        call(rows)
     t0 = time.perf_counter()
     for _ in range(steps):
-        O.mlp_block(inp.X, inp.A, inp.B, rows=rows)
+        call(rows)
     dt = time.perf_counter() - t0
-    flops = 4 * w.H * w.F * len(rows) * steps
-    del np, torch
+    flops = w.flops * len(rows) / nrows * steps
     return {"value": round(flops / dt / 1e12, 5), "unit": UNIT, "cores": int(cores), "kind": "oracle",
-            "sample": f"{len(rows)} of {w.S} rows of {w.name} per step, {steps} step(s), fp64 numpy/OpenBLAS",
+            "sample": (f"{len(rows)} of {nrows} output rows of {w.name} per step, {steps} step(s), "
+                       "fp64 numpy/OpenBLAS" + ("; every call also computes all K and V rows"
+                                                if w.kind == "attn" else "")),
             "seconds": round(dt, 3)}
 
 
@@ -382,8 +475,7 @@ def run_reference(args, rank, world):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded torch.randn)",
-        "config": {"workload": w.name, "S": w.S, "H": w.H, "F": w.F, "t": w.t,
-                   "sample_rows_per_step": rows},
+        "config": {"workload": w.name, "t": w.t, "flops_per_step": w.flops, "sample_rows_per_step": rows},
         "cpu_baseline": {k: cb[k] for k in ("value", "unit", "cores", "kind", "sample")},
         "e2e": {"value": cb["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -402,7 +494,8 @@ def main():
         from megatron_tensor_transformer_gelu_b200.workloads import HEADLINE, WORKLOADS
         if not args.no_cpu_baseline:
             w = WORKLOADS[args.workload or HEADLINE]
-            res["cpu_baseline"] = cpu_oracle_timing(w, args.cpu_sample_rows, 1, 0)
+            rows = args.cpu_sample_rows if w.kind == "mlp" else min(args.cpu_sample_rows, 64)
+            res["cpu_baseline"] = cpu_oracle_timing(w, rows, 1, 0)
         print(json.dumps(res), flush=True)
 
 

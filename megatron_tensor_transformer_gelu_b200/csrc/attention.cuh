@@ -6,20 +6,25 @@
 // head across tensor-parallel shards with no exchange until the O projection
 // ("1. 张量并行：Tensor Parallelism" §1.2.2; "TP到底在切什么" §2.2 figure 4).
 //
-// One CTA per (head, 128 query rows), 6 warps:
-//   warp 0      TMA: the Q tile once, then K_j and V_j tiles (128 keys each)
-//               into a 2-stage ring.
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer.
-//               S_j = Q K_j^T into one of two TMEM score buffers, then
-//               O += P_{j-1} V_{j-1}, so the scores of block j are computed
-//               while the softmax warps still work on block j-1.
-//   warps 2..5  one query row per thread: row max, exp2, row sum (online
-//               softmax), P_j as bf16 into shared memory in the 128-byte
-//               swizzled K-major layout the MMA reads, rescaling of the O
-//               accumulator in TMEM, final O / l to global memory.
+// One CTA per (head, 256 query rows) = two 128-row query tiles that share
+// every K and V tile, 11 warps:
+//   warp 0      TMA: Q0, Q1 once, then K_j (128 keys) into a 2-stage ring.
+//   warp 10     TMA: V_j into a 2-stage ring.
+//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer, in the
+//               order P0_j V_j, S0_{j+1}, P1_j V_j, S1_{j+1} (S_t = Q_t K^T).
+//   warps 2..5  softmax of tile 0, one query row per thread;
+//   warps 6..9  softmax of tile 1.  While one group runs its exponentials
+//               (bound by the MUFU units), the other loads scores, reduces,
+//               or waits for its MMAs, so the two tiles ping-pong.
+// TMEM: S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512) f32 columns.
+// P_t (bf16 pairs) is written over the first 64 columns of S_t once S_t has
+// been read and P_t(j-1) V has been consumed, and is fed to the P V product
+// straight from TMEM (no shared-memory round trip); S_t(j+1) is issued after
+// P_t(j) V_j by the same thread.
 // The running max is only raised when a block's max exceeds it by more than
-// 2^8 (log2 domain), so O is rescaled rarely; P then stays below 2^8, which
-// bf16 and the f32 accumulator carry without loss of relative precision.
+// 2^8 (log2 domain), so O is rescaled in TMEM rarely; P then stays below
+// 2^8, which bf16 and the f32 accumulator carry without loss of relative
+// precision.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -31,15 +36,18 @@ namespace tp {
 
 namespace attn {
 constexpr int D = 128;            // head dimension
-constexpr int BQ = 128;           // query rows per CTA
+constexpr int BQ = 128;           // query rows per tile
+constexpr int TILES = 2;          // query tiles per CTA
 constexpr int BKV = 128;          // keys per block
-constexpr int NUM_THREADS = 192;
-constexpr int HALF_BYTES = BQ * 64 * 2;   // one 64-column (128 B) box of 128 rows: 16 KiB
+constexpr int NUM_THREADS = 352;  // 11 warps
+constexpr int K_STAGES = 2;
+constexpr int V_STAGES = 2;
+constexpr int HALF_BYTES = BQ * 64 * 2;     // one 64-column (128 B) box of 128 rows: 16 KiB
 constexpr int TILE_BYTES = 2 * HALF_BYTES;  // 128 rows x 128 bf16: 32 KiB
-constexpr int SMEM_BYTES = TILE_BYTES * (1 + 2 + 2 + 1) + 1024 + 256;
+constexpr int SMEM_BYTES = TILE_BYTES * (TILES + K_STAGES + V_STAGES) + 1024 + 256;
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(BQ, BKV, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(BQ, D, false, true);
-constexpr uint32_t TMEM_COLS = 512;       // S0 [0,128), S1 [128,256), O [256,384)
+constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;
 }  // namespace attn
 
@@ -56,25 +64,24 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
   using namespace attn;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + TILE_BYTES;        // 2 stages
-  uint8_t* sV = sK + 2 * TILE_BYTES;    // 2 stages
-  uint8_t* sP = sV + 2 * TILE_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + TILE_BYTES);
+  uint8_t* sQ = smem;                            // TILES tiles
+  uint8_t* sK = sQ + TILES * TILE_BYTES;         // K_STAGES stages
+  uint8_t* sV = sK + K_STAGES * TILE_BYTES;      // V_STAGES stages
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + V_STAGES * TILE_BYTES);
   uint64_t* q_full = bars + 0;
-  uint64_t* k_full = bars + 1;    // [2]
-  uint64_t* v_full = bars + 3;    // [2]
-  uint64_t* kv_empty = bars + 5;  // [2]
-  uint64_t* s_full = bars + 7;    // [2]
-  uint64_t* s_free = bars + 9;    // [2]
-  uint64_t* p_full = bars + 11;
-  uint64_t* pv_done = bars + 12;
-  uint64_t* drain = bars + 13;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 14);
+  uint64_t* k_full = bars + 1;                   // [K_STAGES]
+  uint64_t* k_empty = k_full + K_STAGES;         // [K_STAGES]
+  uint64_t* v_full = k_empty + K_STAGES;         // [V_STAGES]
+  uint64_t* v_empty = v_full + V_STAGES;         // [V_STAGES]
+  uint64_t* s_full = v_empty + V_STAGES;         // [TILES]
+  uint64_t* p_full = s_full + TILES;             // [TILES]
+  uint64_t* pv_done = p_full + TILES;            // [TILES]
+  uint64_t* drain = pv_done + TILES;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * BQ;
+  const int q0 = blockIdx.x * (TILES * BQ);
   const int h = blockIdx.y;
   const int shard = h / a.heads_per_shard;
   const int hj = h % a.heads_per_shard;
@@ -86,15 +93,19 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < K_STAGES; ++i) {
       mbar_init(&k_full[i], 1);
-      mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&s_free[i], 128);
+      mbar_init(&k_empty[i], 1);
     }
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
+    for (int i = 0; i < V_STAGES; ++i) {
+      mbar_init(&v_full[i], 1);
+      mbar_init(&v_empty[i], 1);
+    }
+    for (int t = 0; t < TILES; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&pv_done[t], 1);
+    }
     mbar_init(drain, 1);
     mbar_fence_init();
   }
@@ -107,77 +118,93 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const uint32_t tS0 = tmem_base;
-  const uint32_t tO = tmem_base + 256;
 
-  if (warp == 0) {
+  if (warp == 0 || warp == 10) {
+    // ---------------------------------------------- producers (Q + K, V)
     if (lane == 0) {
-      int armed[5] = {-1, -1, -1, -1, -1};  // q, k0, k1, v0, v1
+      const bool is_k = warp == 0;
+      const int nst = is_k ? K_STAGES : V_STAGES;
+      uint64_t* fullb = is_k ? k_full : v_full;
+      uint64_t* emptyb = is_k ? k_empty : v_empty;
+      uint8_t* base = is_k ? sK : sV;
+      const int col = is_k ? kcol : vcol;
+      int armed[K_STAGES + 1];
+#pragma unroll
+      for (int i = 0; i <= K_STAGES; ++i) armed[i] = -1;
       bool ok = true;
-      mbar_arrive_expect_tx(q_full, TILE_BYTES);
-      armed[0] = 0;
-      tma_load_2d(sQ, &a.tmQKV, qcol, q0, q_full);
-      tma_load_2d(sQ + HALF_BYTES, &a.tmQKV, qcol + 64, q0, q_full);
+      if (is_k) {
+        // Tiles past S (an odd tile count) are zero-filled by the TMA.
+        mbar_arrive_expect_tx(q_full, TILES * TILE_BYTES);
+        armed[K_STAGES] = 0;
+        for (int t = 0; t < TILES; ++t) {
+          tma_load_2d(sQ + t * TILE_BYTES, &a.tmQKV, qcol, q0 + t * BQ, q_full);
+          tma_load_2d(sQ + t * TILE_BYTES + HALF_BYTES, &a.tmQKV, qcol + 64, q0 + t * BQ, q_full);
+        }
+      }
       for (int j = 0; j < nkv; ++j) {
-        const int st = j & 1;
-        const uint32_t ph = (j >> 1) & 1;
-        if (!mbar_wait(&kv_empty[st], ph ^ 1)) { ok = false; break; }
-        uint8_t* dk = sK + st * TILE_BYTES;
-        uint8_t* dv = sV + st * TILE_BYTES;
-        mbar_arrive_expect_tx(&k_full[st], TILE_BYTES);
-        armed[1 + st] = static_cast<int>(ph);
-        tma_load_2d(dk, &a.tmQKV, kcol, j * BKV, &k_full[st]);
-        tma_load_2d(dk + HALF_BYTES, &a.tmQKV, kcol + 64, j * BKV, &k_full[st]);
-        mbar_arrive_expect_tx(&v_full[st], TILE_BYTES);
-        armed[3 + st] = static_cast<int>(ph);
-        tma_load_2d(dv, &a.tmQKV, vcol, j * BKV, &v_full[st]);
-        tma_load_2d(dv + HALF_BYTES, &a.tmQKV, vcol + 64, j * BKV, &v_full[st]);
+        const int st = j % nst;
+        const uint32_t ph = (j / nst) & 1;
+        if (!mbar_wait(&emptyb[st], ph ^ 1)) { ok = false; break; }
+        uint8_t* d = base + st * TILE_BYTES;
+        mbar_arrive_expect_tx(&fullb[st], TILE_BYTES);
+        armed[st] = static_cast<int>(ph);
+        tma_load_2d(d, &a.tmQKV, col, j * BKV, &fullb[st]);
+        tma_load_2d(d + HALF_BYTES, &a.tmQKV, col + 64, j * BKV, &fullb[st]);
       }
       if (!ok) {
-        uint64_t* bl[5] = {q_full, &k_full[0], &k_full[1], &v_full[0], &v_full[1]};
-        for (int i = 0; i < 5; ++i) {
-          if (armed[i] < 0) continue;
-          const uint32_t ad = smem_u32(bl[i]);
+        for (int i = 0; i <= K_STAGES; ++i) {
+          if (armed[i] < 0 || (i < K_STAGES && i >= nst)) continue;
+          const uint32_t ad = smem_u32(i == K_STAGES ? q_full : &fullb[i]);
           const long long t0 = clock64();
           while (!mbar_try_wait(ad, static_cast<uint32_t>(armed[i])) && clock64() - t0 < WAIT_LIMIT_CYCLES) {}
         }
       }
     }
   } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
     if (lane == 0) {
       bool ok = mbar_wait(q_full, 0);
       const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t p_addr = smem_u32(sP);
-      for (int j = 0; j <= nkv && ok; ++j) {
-        if (j < nkv) {
-          const int b = j & 1;
-          const uint32_t ph = (j >> 1) & 1;
-          if (!mbar_wait(&k_full[b], ph) || !mbar_wait(&s_free[b], ph ^ 1)) { ok = false; break; }
+      // S_t(j) = Q_t K_j^T into columns [t*128, t*128+128).  Tile 0 waits for
+      // K_j; tile 1 releases its stage.
+      auto issue_s = [&](int j, int t) -> bool {
+        const int ks = j % K_STAGES;
+        if (t == 0) {
+          if (!mbar_wait(&k_full[ks], (j / K_STAGES) & 1)) return false;
           tc_fence_after();
-          const uint32_t k_addr = smem_u32(sK + b * TILE_BYTES);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            umma_bf16(tS0 + b * 128, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
-                      IDESC_QK, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&s_full[b]);
         }
-        if (j >= 1) {
-          const int i = j - 1;
-          const int st = i & 1;
-          const uint32_t ph = (i >> 1) & 1;
-          if (!mbar_wait(&v_full[st], ph) || !mbar_wait(p_full, i & 1)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(sV + st * TILE_BYTES);
+        const uint32_t k_addr = smem_u32(sK + ks * TILE_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < BKV / 16; ++kk) {
-            const uint32_t poff = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-            umma_bf16(tO, sdesc_sw128(p_addr + poff, 16, 1024), sdesc_sw128(v_addr + kk * 2048, HALF_BYTES, 1024),
-                      IDESC_PV, (i > 0 || kk > 0) ? 1u : 0u);
-          }
-          umma_commit(pv_done);
-          umma_commit(&kv_empty[st]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
+          umma_bf16(tmem_base + t * 128, sdesc_sw128(q_addr + t * TILE_BYTES + off, 16, 1024),
+                    sdesc_sw128(k_addr + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[t]);
+        if (t == TILES - 1) umma_commit(&k_empty[ks]);
+        return true;
+      };
+      for (int t = 0; t < TILES && ok && nkv > 0; ++t) ok = issue_s(0, t);
+      // Per block: P0 V, S0(j+1), P1 V, S1(j+1).  Tile 0's next scores are
+      // ready while tile 1 is still in its exponentials, and the reverse.
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int vs = j % V_STAGES;
+        if (!mbar_wait(&v_full[vs], (j / V_STAGES) & 1)) { ok = false; break; }
+        const uint32_t v_addr = smem_u32(sV + vs * TILE_BYTES);
+        for (int t = 0; t < TILES && ok; ++t) {
+          // P_t(j) sits in the first 64 columns of S_t once the softmax arrived.
+          if (!mbar_wait(&p_full[t], j & 1)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t tP = tmem_base + t * 128;
+          const uint32_t tO = tmem_base + 256 + t * 128;
+#pragma unroll
+          for (int kk = 0; kk < BKV / 16; ++kk)
+            umma_bf16_tmem_a(tO, tP + kk * 8, sdesc_sw128(v_addr + kk * 2048, HALF_BYTES, 1024), IDESC_PV,
+                             (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(&pv_done[t]);
+          if (t == TILES - 1) umma_commit(&v_empty[vs]);
+          // S_t(j+1) overwrites P_t(j): issued after P_t(j) V_j above.
+          if (j + 1 < nkv && !issue_s(j + 1, t)) { ok = false; break; }
         }
       }
       if (!ok) {
@@ -189,34 +216,44 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
     }
   } else {
     // --------------------------------------------------- softmax / epilogue
-    const int q = warp & 3;
-    const int r = q * 32 + lane;  // query row inside the tile == TMEM lane
+    const int tile = warp < 6 ? 0 : 1;                 // warps 2..5 -> tile 0, 6..9 -> tile 1
+    const int q = warp & 3;                            // TMEM lane quarter
+    const int r = q * 32 + lane;                       // query row inside the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t tS = tmem_base + tile * 128 + lane_off;
+    const uint32_t tO = tmem_base + 256 + tile * 128 + lane_off;
     float m_run = -INFINITY;
     float l_run = 0.0f;
     bool ok = true;
-    uint8_t* prow0 = sP + r * 128;               // keys 0..63 of this row
-    uint8_t* prow1 = sP + HALF_BYTES + r * 128;  // keys 64..127
     for (int j = 0; j < nkv; ++j) {
-      const int b = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (j >> 1) & 1))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[tile], j & 1))) { ok = false; break; }
       tc_fence_after();
       float s[BKV];
       {
-        uint32_t u[32];
+        uint32_t u0[32], u1[32], u2[32], u3[32];
+        tmem_ld_32x32b_x32(tS + 0, u0);
+        tmem_ld_32x32b_x32(tS + 32, u1);
+        tmem_ld_32x32b_x32(tS + 64, u2);
+        tmem_ld_32x32b_x32(tS + 96, u3);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < BKV / 32; ++c) {
-          tmem_ld_32x32b_x32(tS0 + b * 128 + lane_off + c * 32, u);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(u[e]);
+        for (int e = 0; e < 32; ++e) {
+          s[e] = __uint_as_float(u0[e]);
+          s[32 + e] = __uint_as_float(u1[e]);
+          s[64 + e] = __uint_as_float(u2[e]);
+          s[96 + e] = __uint_as_float(u3[e]);
         }
       }
-      tc_fence_before();
-      mbar_arrive(&s_free[b]);
-      float mx = s[0];
+      // Row max with 8 independent chains, then a tree.
+      float m8[8];
 #pragma unroll
-      for (int e = 1; e < BKV; ++e) mx = fmaxf(mx, s[e]);
+      for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#pragma unroll
+      for (int e = 8; e < BKV; e += 8)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[e + i]);
+      const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                             fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
       const float m_blk = mx * a.scale_log2;
       const bool resc = m_blk > m_run + RESCALE_THRESHOLD;
       float alpha = 1.0f;
@@ -224,57 +261,54 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
         alpha = exp2_fast(m_run - m_blk);  // 0 on the first block
         m_run = m_blk;
       }
-      float sum = 0.0f;
-      uint32_t pk[BKV / 2];
+      // p = 2^(s * scale_log2 - m) in f32, kept as bf16 pairs for the P V
+      // product; the row sum adds the f32 values in 8 independent chains.
+      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      uint32_t pk0[32], pk1[32];
 #pragma unroll
       for (int e = 0; e < BKV; e += 2) {
         const float p0 = exp2_fast(fmaf(s[e], a.scale_log2, -m_run));
         const float p1 = exp2_fast(fmaf(s[e + 1], a.scale_log2, -m_run));
-        __nv_bfloat162 hp = __floats2bfloat162_rn(p0, p1);
-        const float2 back = __bfloat1622float2(hp);
-        sum += back.x + back.y;
-        pk[e / 2] = *reinterpret_cast<uint32_t*>(&hp);
+        sum8[(e / 2) & 7] += p0 + p1;
+        if (e < 64) pk0[e / 2] = pack_bf16x2(p0, p1);
+        else pk1[(e - 64) / 2] = pack_bf16x2(p0, p1);
       }
+      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l_run = l_run * alpha + sum;
       if (j > 0) {
-        // P_{j-1} V_{j-1} must be done before sP is overwritten and O rescaled.
-        if (!__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1))) { ok = false; break; }
+        // P_t(j-1) V_{j-1} must be done before P_t(j) replaces it and O_t is
+        // rescaled.
+        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[tile], (j - 1) & 1))) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t u[32];
-            tmem_ld_32x32b_x32(tO + lane_off + c * 32, u);
+            tmem_ld_32x32b_x32(tO + c * 32, u);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-            tmem_st_32x32b_x32(tO + lane_off + c * 32, u);
+            tmem_st_32x32b_x32(tO + c * 32, u);
           }
-          tmem_wait_st();
         }
       }
-      // P row -> shared memory, 128-byte swizzle: 16-byte chunk c of row r is
-      // stored at chunk (c ^ (r & 7)).
-#pragma unroll
-      for (int c = 0; c < 16; ++c) {
-        uint8_t* rowp = c < 8 ? prow0 : prow1;
-        const int cc = c & 7;
-        uint4 w = make_uint4(pk[c * 4 + 0], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
-        *reinterpret_cast<uint4*>(rowp + ((cc ^ (r & 7)) << 4)) = w;
-      }
-      fence_proxy_async_smem();
+      // P_t(j): 128 keys of row r as 64 columns of bf16 pairs over S_t.
+      tmem_st_32x32b_x32(tS + 0, pk0);
+      tmem_st_32x32b_x32(tS + 32, pk1);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[tile]);
     }
-    if (ok && __all_sync(0xffffffffu, mbar_wait(pv_done, (nkv - 1) & 1))) {
+    const bool tile_valid = q0 + tile * BQ < a.S;  // the second tile of an odd tile count is not stored
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&pv_done[tile], (nkv - 1) & 1)) && tile_valid) {
       tc_fence_after();
       const float inv = 1.0f / l_run;
-      const int grow = q0 + r;
+      const int grow = q0 + tile * BQ + r;
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.O) + static_cast<long long>(grow) * a.H + h * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t u[32];
-        tmem_ld_32x32b_x32(tO + lane_off + c * 32, u);
+        tmem_ld_32x32b_x32(tO + c * 32, u);
         tmem_wait_ld();
 #pragma unroll
         for (int g = 0; g < 4; ++g) {

@@ -478,7 +478,7 @@ int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int
     a.heads_per_shard = nhs;
     a.shard_cols = 3 * Hs;
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
-    dim3 grid(S / tp::attn::BQ, nh);
+    dim3 grid((S + tp::attn::TILES * tp::attn::BQ - 1) / (tp::attn::TILES * tp::attn::BQ), nh);
     ProfScope ps(K_ATTN, s);
     tp::attn_fwd_kernel<<<grid, tp::attn::NUM_THREADS, tp::attn::SMEM_BYTES, s>>>(a);
     st = launch_status();

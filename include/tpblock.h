@@ -75,7 +75,10 @@ const char* tp_status_string(int status);
 
 /* Reads and clears the device-side error word of the current device (0 when no
  * bounded wait gave up).  Call after synchronising the streams that ran the
- * library's kernels.  Returns TP_OK or TP_ERR_TIMEOUT (or TP_ERR_CUDA). */
+ * library's kernels.  Returns TP_OK or TP_ERR_TIMEOUT (or TP_ERR_CUDA).  While
+ * the word is set, the library's kernels give up any wait that does not
+ * complete at once (their outputs are then unspecified), so a failure is not
+ * silently followed by more work: read the word to re-arm the library. */
 int tp_device_error(void);
 
 /* ------------------------------------------------------------------ MLP ----
@@ -174,6 +177,15 @@ int tp_linear_row_forward(int M, int K, int N, int t, int dtype, int out_dtype,
 int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts,
                                  const void* X, int x_dtype, const float* gamma, const float* beta,
                                  float eps, void* Y, int out_dtype, void* stream);
+
+/* ------------------------------------------------------------ self-test ----
+ * Diagnostic for the bounded-wait path every kernel here takes when one of its
+ * device-side waits gives up: launches one CTA whose mbarrier wait nothing can
+ * complete, so the wait ends after `limit_cycles` SM cycles (> 0), raises the
+ * device error word and returns.  After the caller synchronises `stream`,
+ * tp_device_error() returns TP_ERR_TIMEOUT (and clears the word); the context
+ * stays usable.  Returns TP_ERR_INVALID_ARG for limit_cycles < 1. */
+int tp_selftest_wait_timeout(long long limit_cycles, void* stream);
 
 /* ----------------------------------------------------- kernel timing ----
  * When enabled, every kernel the library launches is counted, and the first

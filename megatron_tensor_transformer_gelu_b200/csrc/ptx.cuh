@@ -61,9 +61,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 }
 
 // Wait until the phase with the given parity has completed.  Returns false
-// (and raises the device error word) if it did not within WAIT_LIMIT_CYCLES,
+// (and raises the device error word) if it did not within `limit` SM cycles,
 // or if another role already raised it.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long limit = WAIT_LIMIT_CYCLES) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const long long t0 = clock64();
@@ -72,11 +72,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     if (mbar_try_wait(a, parity)) return true;
     if ((++n & 255u) == 0u) {
       if (error_raised()) return false;
-      if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+      if (clock64() - t0 > limit) {
         flag_error(DEV_ERR_TIMEOUT);
         return false;
       }
     }
+  }
+}
+
+// Diagnostic: one thread waits on an mbarrier that nothing completes, so the
+// bounded wait above gives up after `limit` cycles and raises the error word.
+__global__ void selftest_wait_timeout_kernel(long long limit) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    mbar_fence_init();
+    (void)mbar_wait(&bar, 0, limit);
   }
 }
 

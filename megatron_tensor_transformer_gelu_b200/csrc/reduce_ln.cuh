@@ -20,10 +20,12 @@
 namespace tp {
 
 namespace rln {
-constexpr int THREADS = 256;       // 8 warps per CTA
-constexpr int MAX_WPR = 8;         // warps per row
-constexpr int MAX_CH = 8;          // 8-element chunks per lane
+constexpr int THREADS = 256;       // 8 warps per CTA (up to 8 warps per row)
+constexpr int MAX_WPR = 16;        // warps per row (CTAs grow to 16 warps)
+constexpr int MAX_CH = 4;          // 8-element chunks per lane
 constexpr int MAX_H = MAX_WPR * 32 * MAX_CH * 8;  // 16384
+// CTA size for WPR warps per row: 8 warps, or one row of WPR warps.
+__host__ __device__ constexpr int cta_threads(int wpr) { return wpr > 8 ? wpr * 32 : THREADS; }
 }
 
 struct ReduceLnArgs {
@@ -67,119 +69,144 @@ __device__ __forceinline__ void load8_f32_keep(const float* src, float* v) {
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// One row is handled by WPR consecutive warps; a CTA holds 8 / WPR rows.  Lane
-// l of warp w (of the row) owns chunks c = 0..CH-1 at column
-// ((c * WPR + w) * 32 + l) * 8, so each warp reads 32 consecutive 8-element
-// chunks per step.  CH = 4 (32 values per lane, ~60 registers, 4 CTAs per SM)
-// up to H = 8192; CH = 8 beyond.
-template <int WPR, int CH>
-__global__ void __launch_bounds__(rln::THREADS) reduce_residual_ln_kernel(const ReduceLnArgs p) {
-  constexpr int RPC = rln::THREADS / 32 / WPR;  // rows per CTA
+// One row is handled by WPR consecutive warps; a CTA holds max(1, 8 / WPR)
+// rows at a time and walks row groups blockIdx.x, blockIdx.x + gridDim.x, ...
+// (the grid is sized to the number of CTAs resident at once, so there is no
+// partial last wave).  Lane l of warp w (of the row) owns chunks c = 0..CH-1
+// at column ((c * WPR + w) * 32 + l) * 8, so each warp reads 32 consecutive
+// 8-element chunks per step.  Few values per lane (CH = 2 up to H = 4096, 4
+// beyond) keep registers low and occupancy high; larger H uses more warps per
+// row.  NP1 specialises the common single partial so that every load of a row
+// is issued before its first add.
+template <int WPR, int CH, bool NP1>
+__global__ void __launch_bounds__(rln::cta_threads(WPR)) reduce_residual_ln_kernel(const ReduceLnArgs p) {
+  constexpr int RPC = WPR > 8 ? 1 : rln::THREADS / 32 / WPR;  // rows per CTA
   __shared__ float red[2][RPC][WPR];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rloc = warp / WPR, wr = warp % WPR;
-  const long long row = static_cast<long long>(blockIdx.x) * RPC + rloc;
-  const bool live = row < p.S && rloc < RPC;
-  const long long base = row * p.H;
-  float v[CH][8];
-  float s = 0.0f;
+  const int groups = (p.S + RPC - 1) / RPC;
+  for (int g = blockIdx.x; g < groups; g += gridDim.x) {
+    const long long row = static_cast<long long>(g) * RPC + rloc;
+    const bool live = row < p.S && rloc < RPC;
+    const long long base = row * p.H;
+    float v[CH][8];
+    if (NP1) {
+      float w[CH][8];
 #pragma unroll
-  for (int c = 0; c < CH; ++c) {
-    const int col = ((c * WPR + wr) * 32 + lane) * 8;
-    if (live && col < p.H) {
-      if (p.x_bf16) load8_bf16(static_cast<const __nv_bfloat16*>(p.X) + base + col, v[c]);
-      else load8_f32(static_cast<const float*>(p.X) + base + col, v[c]);
+      for (int c = 0; c < CH; ++c) {
+        const int col = ((c * WPR + wr) * 32 + lane) * 8;
+        if (live && col < p.H) {
+          if (p.x_bf16) load8_bf16(static_cast<const __nv_bfloat16*>(p.X) + base + col, v[c]);
+          else load8_f32(static_cast<const float*>(p.X) + base + col, v[c]);
+          load8_f32(p.parts + base + col, w[c]);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < CH; ++c)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[c][e] += w[c][e];
+    } else {
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int col = ((c * WPR + wr) * 32 + lane) * 8;
+        if (live && col < p.H) {
+          if (p.x_bf16) load8_bf16(static_cast<const __nv_bfloat16*>(p.X) + base + col, v[c]);
+          else load8_f32(static_cast<const float*>(p.X) + base + col, v[c]);
+        }
+      }
+      for (int q = 0; q < p.nparts; ++q) {
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+          const int col = ((c * WPR + wr) * 32 + lane) * 8;
+          if (live && col < p.H) {
+            float w[8];
+            load8_f32(p.parts + q * p.part_stride + base + col, w);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[c][e] += w[e];
+          }
+        }
+      }
     }
-  }
-  for (int q = 0; q < p.nparts; ++q) {
+    float s = 0.0f;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int col = ((c * WPR + wr) * 32 + lane) * 8;
       if (live && col < p.H) {
-        float w[8];
-        load8_f32(p.parts + q * p.part_stride + base + col, w);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[c][e] += w[e];
+        for (int e = 0; e < 8; ++e) s += v[c][e];
       }
     }
-  }
+    // mean over the row: warp shuffle, then the row's WPR warps in fixed order
 #pragma unroll
-  for (int c = 0; c < CH; ++c) {
-    const int col = ((c * WPR + wr) * 32 + lane) * 8;
-    if (live && col < p.H) {
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0 && rloc < RPC) red[0][rloc][wr] = s;
+    __syncthreads();
+    float tot = 0.0f;
+    if (rloc < RPC) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) s += v[c][e];
+      for (int i = 0; i < WPR; ++i) tot += red[0][rloc][i];
     }
-  }
-  // mean over the row: warp shuffle, then the row's WPR warps in fixed order
+    const float mean = tot / static_cast<float>(p.H);
+    float s2 = 0.0f;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-  if (lane == 0 && rloc < RPC) red[0][rloc][wr] = s;
-  __syncthreads();
-  float tot = 0.0f;
-  if (rloc < RPC) {
+    for (int c = 0; c < CH; ++c) {
+      const int col = ((c * WPR + wr) * 32 + lane) * 8;
+      if (live && col < p.H) {
 #pragma unroll
-    for (int i = 0; i < WPR; ++i) tot += red[0][rloc][i];
-  }
-  const float mean = tot / static_cast<float>(p.H);
-  float s2 = 0.0f;
-#pragma unroll
-  for (int c = 0; c < CH; ++c) {
-    const int col = ((c * WPR + wr) * 32 + lane) * 8;
-    if (live && col < p.H) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float d = v[c][e] - mean;
-        s2 = fmaf(d, d, s2);
+        for (int e = 0; e < 8; ++e) {
+          const float d = v[c][e] - mean;
+          s2 = fmaf(d, d, s2);
+        }
       }
     }
-  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
-  if (lane == 0 && rloc < RPC) red[1][rloc][wr] = s2;
-  __syncthreads();
-  float tot2 = 0.0f;
-  if (rloc < RPC) {
+    for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    if (lane == 0 && rloc < RPC) red[1][rloc][wr] = s2;
+    __syncthreads();
+    float tot2 = 0.0f;
+    if (rloc < RPC) {
 #pragma unroll
-    for (int i = 0; i < WPR; ++i) tot2 += red[1][rloc][i];
-  }
-  const float var = tot2 / static_cast<float>(p.H);
-  const float rstd = 1.0f / sqrtf(var + p.eps);
+      for (int i = 0; i < WPR; ++i) tot2 += red[1][rloc][i];
+    }
+    const float var = tot2 / static_cast<float>(p.H);
+    const float rstd = 1.0f / sqrtf(var + p.eps);
 #pragma unroll
-  for (int c = 0; c < CH; ++c) {
-    const int col = ((c * WPR + wr) * 32 + lane) * 8;
-    if (live && col < p.H) {
-      float g[8], b[8];
-      if (p.gamma) load8_f32_keep(p.gamma + col, g);
-      else {
+    for (int c = 0; c < CH; ++c) {
+      const int col = ((c * WPR + wr) * 32 + lane) * 8;
+      if (live && col < p.H) {
+        float gm[8], bt[8];
+        if (p.gamma) load8_f32_keep(p.gamma + col, gm);
+        else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) g[e] = 1.0f;
-      }
-      if (p.beta) load8_f32_keep(p.beta + col, b);
-      else {
+          for (int e = 0; e < 8; ++e) gm[e] = 1.0f;
+        }
+        if (p.beta) load8_f32_keep(p.beta + col, bt);
+        else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) b[e] = 0.0f;
-      }
-      float y[8];
+          for (int e = 0; e < 8; ++e) bt[e] = 0.0f;
+        }
+        float y[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) y[e] = fmaf((v[c][e] - mean) * rstd, g[e], b[e]);
-      if (p.y_bf16) {
-        uint4 u;
-        __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]);
-        __nv_bfloat162 h1 = __floats2bfloat162_rn(y[2], y[3]);
-        __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]);
-        __nv_bfloat162 h3 = __floats2bfloat162_rn(y[6], y[7]);
-        u.x = *reinterpret_cast<uint32_t*>(&h0);
-        u.y = *reinterpret_cast<uint32_t*>(&h1);
-        u.z = *reinterpret_cast<uint32_t*>(&h2);
-        u.w = *reinterpret_cast<uint32_t*>(&h3);
-        *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + base + col) = u;
-      } else {
-        float4* d = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + base + col);
-        d[0] = make_float4(y[0], y[1], y[2], y[3]);
-        d[1] = make_float4(y[4], y[5], y[6], y[7]);
+        for (int e = 0; e < 8; ++e) y[e] = fmaf((v[c][e] - mean) * rstd, gm[e], bt[e]);
+        if (p.y_bf16) {
+          uint4 u;
+          __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]);
+          __nv_bfloat162 h1 = __floats2bfloat162_rn(y[2], y[3]);
+          __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]);
+          __nv_bfloat162 h3 = __floats2bfloat162_rn(y[6], y[7]);
+          u.x = *reinterpret_cast<uint32_t*>(&h0);
+          u.y = *reinterpret_cast<uint32_t*>(&h1);
+          u.z = *reinterpret_cast<uint32_t*>(&h2);
+          u.w = *reinterpret_cast<uint32_t*>(&h3);
+          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + base + col) = u;
+        } else {
+          float4* d = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + base + col);
+          d[0] = make_float4(y[0], y[1], y[2], y[3]);
+          d[1] = make_float4(y[4], y[5], y[6], y[7]);
+        }
       }
     }
+    __syncthreads();  // `red` is reused by the next row group
   }
 }
 

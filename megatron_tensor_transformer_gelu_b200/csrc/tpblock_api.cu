@@ -303,7 +303,7 @@ int run_gemm_simt(const float* A, long long lda, int M, const void* const* B, in
 }
 
 int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, int x_bf16, const float* gamma,
-                  const float* beta, float eps, void* Y, int y_bf16, cudaStream_t st) {
+                  const float* beta, float eps, void* Y, int y_bf16, cudaStream_t st, int dev_sms) {
   if (S == 0) return TP_OK;
   tp::ReduceLnArgs p;
   p.S = S;
@@ -318,14 +318,28 @@ int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, i
   p.eps = eps;
   p.Y = Y;
   p.y_bf16 = y_bf16;
-  // warps per row (each lane holds CH chunks of 8 values); 8 / WPR rows per CTA
+  // WPR warps per row (each lane holds CH chunks of 8 values); max(1, 8 / WPR)
+  // rows per CTA; a grid of the resident CTA count walks the row groups.
   ProfScope ps(K_REDUCE_LN, st);
-  const int T = tp::rln::THREADS;
-  if (H <= 1024) tp::reduce_residual_ln_kernel<1, 4><<<ceil_div(S, 8), T, 0, st>>>(p);
-  else if (H <= 2048) tp::reduce_residual_ln_kernel<2, 4><<<ceil_div(S, 4), T, 0, st>>>(p);
-  else if (H <= 4096) tp::reduce_residual_ln_kernel<4, 4><<<ceil_div(S, 2), T, 0, st>>>(p);
-  else if (H <= 8192) tp::reduce_residual_ln_kernel<8, 4><<<S, T, 0, st>>>(p);
-  else tp::reduce_residual_ln_kernel<8, 8><<<S, T, 0, st>>>(p);
+  const bool np1 = nparts == 1;
+  auto go = [&](auto kern, int wpr, int rows_per_cta) {
+    const int threads = tp::rln::cta_threads(wpr);
+    const int groups = ceil_div(S, rows_per_cta);
+    int per_sm = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0) != cudaSuccess || per_sm < 1)
+      per_sm = 1;
+    const int grid = groups < per_sm * dev_sms ? groups : per_sm * dev_sms;
+    kern<<<grid, threads, 0, st>>>(p);
+  };
+  using namespace tp;
+  if (H <= 512) np1 ? go(reduce_residual_ln_kernel<1, 2, true>, 1, 8) : go(reduce_residual_ln_kernel<1, 2, false>, 1, 8);
+  else if (H <= 1024) np1 ? go(reduce_residual_ln_kernel<2, 2, true>, 2, 4) : go(reduce_residual_ln_kernel<2, 2, false>, 2, 4);
+  else if (H <= 2048) np1 ? go(reduce_residual_ln_kernel<4, 2, true>, 4, 2) : go(reduce_residual_ln_kernel<4, 2, false>, 4, 2);
+  else if (H <= 4096) np1 ? go(reduce_residual_ln_kernel<8, 2, true>, 8, 1) : go(reduce_residual_ln_kernel<8, 2, false>, 8, 1);
+  else if (H <= 8192) np1 ? go(reduce_residual_ln_kernel<8, 4, true>, 8, 1) : go(reduce_residual_ln_kernel<8, 4, false>, 8, 1);
+  // (one-row CTAs of 12 or 16 warps keep the generic loop: fewer registers, two CTAs per SM)
+  else if (H <= 12288) go(reduce_residual_ln_kernel<12, 4, false>, 12, 1);
+  else go(reduce_residual_ln_kernel<16, 4, false>, 16, 1);
   return launch_status();
 }
 
@@ -426,7 +440,7 @@ int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype, const v
     if (st != TP_OK) return st;
   }
   return run_reduce_ln(S, H, nparts, Zsum, X, dtype == TP_DTYPE_BF16, gamma, beta, eps, Y,
-                       out_dtype == TP_DTYPE_BF16, s);
+                       out_dtype == TP_DTYPE_BF16, s, dev->sm_count);
 }
 
 // -------------------------------------------------------------- attention
@@ -489,7 +503,7 @@ int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int
   st = run_gemm_tc(*dev, Obuf, H, S, Wo_shards, t, 1, Hs, H, Zsum, H, 1, TP_ACT_NONE, s, TP_MAX_K_SPLITS,
                    static_cast<long long>(S) * H, &nparts);
   if (st != TP_OK) return st;
-  return run_reduce_ln(S, H, nparts, Zsum, X, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s);
+  return run_reduce_ln(S, H, nparts, Zsum, X, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s, dev->sm_count);
 }
 
 // ---------------------------------------------------------------- linears
@@ -545,7 +559,17 @@ int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts, c
   int st = device_ready(&dev);
   if (st != TP_OK) return st;
   return run_reduce_ln(S, H, nparts, parts, X, x_dtype == TP_DTYPE_BF16, gamma, beta, eps, Y,
-                       out_dtype == TP_DTYPE_BF16, static_cast<cudaStream_t>(stream));
+                       out_dtype == TP_DTYPE_BF16, static_cast<cudaStream_t>(stream), dev->sm_count);
+}
+
+// ------------------------------------------------------------- self-test
+int tp_selftest_wait_timeout(long long limit_cycles, void* stream) {
+  if (limit_cycles < 1) return TP_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  int st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  tp::selftest_wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles);
+  return launch_status();
 }
 
 // ------------------------------------------------------------- profiling

@@ -152,6 +152,27 @@ int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int
                               const float* gamma, const float* beta, float eps,
                               void* Y, void* workspace, size_t workspace_bytes, void* stream);
 
+/* ---------------------------------------------------- Transformer block ----
+ * The attention sublayer followed by the MLP sublayer, the two TP pairs of one
+ * Transformer block ([PWWT] §2.1 figure 3: QKV/O one pair, the two MLP
+ * layers the other, two reductions per block).
+ *   pre_ln = 0 (post-LN):  Y1 = LN1(X + Attn(X));  Y = LN2(Y1 + MLP(Y1))
+ *   pre_ln = 1 (pre-LN, the order [PWWT] §2.1 lists):
+ *                          Z1 = X + Attn(LN1(X)); Y = Z1 + MLP(LN2(Z1))
+ * Attn and MLP are the sublayers above without their residual and LayerNorm;
+ * the intermediate Y1 / Z1 / LN outputs are bf16.  Weights as in
+ * tp_qkv_attn_oproj_forward and tp_mlp_forward; ln*_gamma/beta [H] f32 or
+ * NULL.  dtype bf16; out_dtype bf16 or f32.  Shapes: the union of both
+ * sublayers' limits (d == 128, H == nh d, nh % t == 0, S % 128 == 0,
+ * (F/t) % 8 == 0, H <= 16384).  workspace >= tp_block_workspace_bytes(). */
+size_t tp_block_workspace_bytes(int S, int H, int F, int nh, int d, int t, int dtype);
+int tp_transformer_block_forward(int S, int H, int F, int nh, int d, int t, int dtype, int out_dtype, int pre_ln,
+                                 const void* X, const void* const* Wqkv_shards, const void* const* Wo_shards,
+                                 const void* const* A_shards, const void* const* B_shards,
+                                 const float* ln1_gamma, const float* ln1_beta,
+                                 const float* ln2_gamma, const float* ln2_beta, float eps, int act,
+                                 void* Y, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------------ single linears ----
  * Column-split linear ([TYPC] §2.1; [PWWT] §1.1 figure 1; [0539] §1.1 列切分):
  *   Y[:, i N/t : (i+1) N/t] = Act(X W_i),  X [M, K], W_i [K, N/t]  (concat in place).

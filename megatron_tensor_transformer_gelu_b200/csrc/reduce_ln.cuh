@@ -40,6 +40,7 @@ struct ReduceLnArgs {
   float eps;
   void* Y;                    // [S, H], bf16 or f32
   int y_bf16;
+  int apply_ln;               // 0: Y = X + sum_p P_p only (pre-LN residual stream)
 };
 
 __device__ __forceinline__ void load8_bf16(const __nv_bfloat16* src, float* v) {
@@ -67,6 +68,26 @@ __device__ __forceinline__ void load8_f32_keep(const float* src, float* v) {
   const float4 b = reinterpret_cast<const float4*>(src)[1];
   v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
+// 8 consecutive output values, bf16 (one 16-byte store) or f32 (two).
+__device__ __forceinline__ void store8(const ReduceLnArgs& p, long long off, const float* y) {
+  if (p.y_bf16) {
+    uint4 u;
+    __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]);
+    __nv_bfloat162 h1 = __floats2bfloat162_rn(y[2], y[3]);
+    __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]);
+    __nv_bfloat162 h3 = __floats2bfloat162_rn(y[6], y[7]);
+    u.x = *reinterpret_cast<uint32_t*>(&h0);
+    u.y = *reinterpret_cast<uint32_t*>(&h1);
+    u.z = *reinterpret_cast<uint32_t*>(&h2);
+    u.w = *reinterpret_cast<uint32_t*>(&h3);
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + off) = u;
+  } else {
+    float4* d = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + off);
+    d[0] = make_float4(y[0], y[1], y[2], y[3]);
+    d[1] = make_float4(y[4], y[5], y[6], y[7]);
+  }
 }
 
 // One row is handled by WPR consecutive warps; a CTA holds max(1, 8 / WPR)
@@ -126,6 +147,15 @@ __global__ void __launch_bounds__(rln::cta_threads(WPR)) reduce_residual_ln_kern
           }
         }
       }
+    }
+    if (!p.apply_ln) {
+      // residual add only: Y = X + sum of the partials
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int col = ((c * WPR + wr) * 32 + lane) * 8;
+        if (live && col < p.H) store8(p, base + col, v[c]);
+      }
+      continue;  // no shared memory touched: no barrier needed
     }
     float s = 0.0f;
 #pragma unroll
@@ -188,22 +218,7 @@ __global__ void __launch_bounds__(rln::cta_threads(WPR)) reduce_residual_ln_kern
         float y[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) y[e] = fmaf((v[c][e] - mean) * rstd, gm[e], bt[e]);
-        if (p.y_bf16) {
-          uint4 u;
-          __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]);
-          __nv_bfloat162 h1 = __floats2bfloat162_rn(y[2], y[3]);
-          __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]);
-          __nv_bfloat162 h3 = __floats2bfloat162_rn(y[6], y[7]);
-          u.x = *reinterpret_cast<uint32_t*>(&h0);
-          u.y = *reinterpret_cast<uint32_t*>(&h1);
-          u.z = *reinterpret_cast<uint32_t*>(&h2);
-          u.w = *reinterpret_cast<uint32_t*>(&h3);
-          *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + base + col) = u;
-        } else {
-          float4* d = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + base + col);
-          d[0] = make_float4(y[0], y[1], y[2], y[3]);
-          d[1] = make_float4(y[4], y[5], y[6], y[7]);
-        }
+        store8(p, base + col, y);
       }
     }
     __syncthreads();  // `red` is reused by the next row group

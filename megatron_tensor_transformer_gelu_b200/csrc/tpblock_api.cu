@@ -303,9 +303,11 @@ int run_gemm_simt(const float* A, long long lda, int M, const void* const* B, in
 }
 
 int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, int x_bf16, const float* gamma,
-                  const float* beta, float eps, void* Y, int y_bf16, cudaStream_t st, int dev_sms) {
+                  const float* beta, float eps, void* Y, int y_bf16, cudaStream_t st, int dev_sms,
+                  int apply_ln = 1) {
   if (S == 0) return TP_OK;
   tp::ReduceLnArgs p;
+  p.apply_ln = apply_ln;
   p.S = S;
   p.H = H;
   p.nparts = nparts;
@@ -397,93 +399,65 @@ size_t tp_mlp_workspace_bytes(int S, int H, int F, int t, int dtype) {
   return align256(static_cast<size_t>(S) * F * eh) + slots * static_cast<size_t>(S) * H * 4;
 }
 
-int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype, const void* X,
-                   const void* const* A_shards, const void* const* B_shards, const float* gamma,
-                   const float* beta, float eps, int act, void* Y, void* workspace, size_t workspace_bytes,
-                   void* stream) {
-  if (t < 1 || t > TP_MAX_SHARDS || S < 0 || H <= 0 || F <= 0) return TP_ERR_INVALID_ARG;
-  if (!valid_out(dtype, out_dtype) || !valid_act(act) || !(eps > 0.0f) || !std::isfinite(eps))
-    return TP_ERR_INVALID_ARG;
-  // With S == 0 nothing is read or written, so X, Y and workspace may be null.
-  if ((S > 0 && (!ptr_ok(X) || !ptr_ok(Y))) || !opt_ptr_ok(X) || !opt_ptr_ok(Y) || !shards_ok(A_shards, t) ||
-      !shards_ok(B_shards, t) || !opt_ptr_ok(gamma) || !opt_ptr_ok(beta) || !opt_ptr_ok(workspace))
-    return TP_ERR_INVALID_ARG;
-  if (F % t != 0 || (F / t) % 8 != 0 || !hidden_ok(H)) return TP_ERR_UNSUPPORTED_SHAPE;
-  const size_t need = tp_mlp_workspace_bytes(S, H, F, t, dtype);
-  if (workspace_bytes < need || (need > 0 && !workspace)) return TP_ERR_WORKSPACE_TOO_SMALL;
-  DeviceInfo* dev = nullptr;
-  int st = device_ready(&dev);
-  if (st != TP_OK) return st;
+}  // extern "C"
+
+namespace {
+
+// MLP sublayer on `in` with residual `res`: Y = LN(res + sum_i Act(in A_i) B_i),
+// or Y = res + sum_i Act(in A_i) B_i without the LayerNorm (apply_ln = 0).
+// Arguments are already checked.
+int mlp_core(const DeviceInfo& dev, int S, int H, int F, int t, int dtype, int out_dtype, const void* in,
+             const void* res, const void* const* A_shards, const void* const* B_shards, const float* gamma,
+             const float* beta, float eps, int act, int apply_ln, void* Y, void* workspace, cudaStream_t s) {
   if (S == 0) return TP_OK;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int Fs = F / t;
   int nparts = 1;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t eh = dtype == TP_DTYPE_BF16 ? 2 : 4;
   void* Hbuf = ws;
   float* Zsum = reinterpret_cast<float*>(ws + align256(static_cast<size_t>(S) * F * eh));
+  int st;
   if (dtype == TP_DTYPE_BF16) {
-    // H_i = Act(X A_i) into columns [i Fs, (i+1) Fs) of Hbuf [S, F] (bf16).
-    st = run_gemm_tc(*dev, X, H, S, A_shards, t, /*row_mode=*/0, /*shard_k=*/H, /*shard_n=*/Fs, Hbuf, F,
+    // H_i = Act(in A_i) into columns [i Fs, (i+1) Fs) of Hbuf [S, F] (bf16).
+    st = run_gemm_tc(dev, in, H, S, A_shards, t, /*row_mode=*/0, /*shard_k=*/H, /*shard_n=*/Fs, Hbuf, F,
                      /*out_f32=*/0, act, s);
     if (st != TP_OK) return st;
     // Zsum = sum_i H_i B_i, accumulated in TMEM across the shards (f32); the K
     // loop may be cut into `nparts` ranges (partial-sum slots) to fill the GPU.
-    st = run_gemm_tc(*dev, Hbuf, F, S, B_shards, t, /*row_mode=*/1, /*shard_k=*/Fs, /*shard_n=*/H, Zsum, H,
+    st = run_gemm_tc(dev, Hbuf, F, S, B_shards, t, /*row_mode=*/1, /*shard_k=*/Fs, /*shard_n=*/H, Zsum, H,
                      /*out_f32=*/1, TP_ACT_NONE, s, TP_MAX_K_SPLITS, static_cast<long long>(S) * H, &nparts);
     if (st != TP_OK) return st;
   } else {
-    st = run_gemm_simt(static_cast<const float*>(X), H, S, A_shards, t, 0, H, Fs, static_cast<float*>(Hbuf), F,
+    st = run_gemm_simt(static_cast<const float*>(in), H, S, A_shards, t, 0, H, Fs, static_cast<float*>(Hbuf), F,
                        act, s);
     if (st != TP_OK) return st;
     st = run_gemm_simt(static_cast<const float*>(Hbuf), F, S, B_shards, t, 1, Fs, H, Zsum, H, TP_ACT_NONE, s);
     if (st != TP_OK) return st;
   }
-  return run_reduce_ln(S, H, nparts, Zsum, X, dtype == TP_DTYPE_BF16, gamma, beta, eps, Y,
-                       out_dtype == TP_DTYPE_BF16, s, dev->sm_count);
+  return run_reduce_ln(S, H, nparts, Zsum, res, dtype == TP_DTYPE_BF16, gamma, beta, eps, Y,
+                       out_dtype == TP_DTYPE_BF16, s, dev.sm_count, apply_ln);
 }
 
-// -------------------------------------------------------------- attention
-size_t tp_attn_workspace_bytes(int S, int H, int nh, int d, int t, int dtype) {
-  if (S < 0 || H <= 0 || nh <= 0 || d <= 0 || t < 1 || dtype != TP_DTYPE_BF16) return 0;
-  const size_t s = static_cast<size_t>(S), h = static_cast<size_t>(H);
-  return align256(s * 3 * h * 2) + align256(s * h * 2) + TP_MAX_K_SPLITS * s * h * 4;
-}
-
-int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int out_dtype, const void* X,
-                              const void* const* Wqkv_shards, const void* const* Wo_shards, const float* gamma,
-                              const float* beta, float eps, void* Y, void* workspace, size_t workspace_bytes,
-                              void* stream) {
-  if (t < 1 || t > TP_MAX_SHARDS || S < 0 || H <= 0 || nh <= 0 || d <= 0) return TP_ERR_INVALID_ARG;
-  if (dtype != TP_DTYPE_BF16 || !valid_out(dtype, out_dtype) || !(eps > 0.0f) || !std::isfinite(eps))
-    return TP_ERR_INVALID_ARG;
-  if ((S > 0 && (!ptr_ok(X) || !ptr_ok(Y))) || !opt_ptr_ok(X) || !opt_ptr_ok(Y) || !shards_ok(Wqkv_shards, t) ||
-      !shards_ok(Wo_shards, t) || !opt_ptr_ok(gamma) || !opt_ptr_ok(beta) || !opt_ptr_ok(workspace))
-    return TP_ERR_INVALID_ARG;
-  if (d != tp::attn::D || static_cast<long long>(nh) * d != H || nh % t != 0 || S % tp::attn::BQ != 0 ||
-      !hidden_ok(H))
-    return TP_ERR_UNSUPPORTED_SHAPE;
-  const size_t need = tp_attn_workspace_bytes(S, H, nh, d, t, dtype);
-  if (workspace_bytes < need || (need > 0 && !workspace)) return TP_ERR_WORKSPACE_TOO_SMALL;
-  DeviceInfo* dev = nullptr;
-  int st = device_ready(&dev);
-  if (st != TP_OK) return st;
+// Attention sublayer on `in` with residual `res` (bf16): Y = LN(res + O Wo)
+// or Y = res + O Wo (apply_ln = 0).  Arguments are already checked.
+int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out_dtype, const void* in,
+              const void* res, const void* const* Wqkv_shards, const void* const* Wo_shards, const float* gamma,
+              const float* beta, float eps, int apply_ln, void* Y, void* workspace, cudaStream_t s) {
   if (S == 0) return TP_OK;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int Hs = H / t;  // columns of one shard's heads
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* QKV = ws;                                                            // [S, 3H] bf16
   void* Obuf = ws + align256(static_cast<size_t>(S) * 3 * H * 2);            // [S, H]  bf16
   float* Zsum = reinterpret_cast<float*>(static_cast<uint8_t*>(Obuf) + align256(static_cast<size_t>(S) * H * 2));
-  // [Q_s | K_s | V_s] = X Wqkv_s into columns [3 s Hs, 3 (s+1) Hs) of QKV.
-  st = run_gemm_tc(*dev, X, H, S, Wqkv_shards, t, 0, H, 3 * Hs, QKV, 3LL * H, 0, TP_ACT_NONE, s);
+  // [Q_s | K_s | V_s] = in Wqkv_s into columns [3 s Hs, 3 (s+1) Hs) of QKV.
+  int st = run_gemm_tc(dev, in, H, S, Wqkv_shards, t, 0, H, 3 * Hs, QKV, 3LL * H, 0, TP_ACT_NONE, s);
   if (st != TP_OK) return st;
   // O_h = softmax(Q_h K_h^T / sqrt d) V_h, written to columns [h d, (h+1) d) of O.
   {
     tp::AttnArgs a;
     std::memset(&a, 0, sizeof(a));
     const int nhs = nh / t;
-    // Q/K/V boxes: 64 columns (128 B) x BQ or BKV rows of the [S, 3H] buffer.
+    // Q/K/V boxes: 64 columns (128 B) x 128 rows of the [S, 3H] buffer.
     if (!tmap_bf16(&a.tmQKV, QKV, S, 3LL * H, 3LL * H, 64, tp::attn::BQ)) return TP_ERR_CUDA;
     a.O = Obuf;
     a.S = S;
@@ -500,10 +474,137 @@ int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int
   }
   // sum_s O_s Wo_s, the O projection row-split by head, summed in TMEM.
   int nparts = 1;
-  st = run_gemm_tc(*dev, Obuf, H, S, Wo_shards, t, 1, Hs, H, Zsum, H, 1, TP_ACT_NONE, s, TP_MAX_K_SPLITS,
+  st = run_gemm_tc(dev, Obuf, H, S, Wo_shards, t, 1, Hs, H, Zsum, H, 1, TP_ACT_NONE, s, TP_MAX_K_SPLITS,
                    static_cast<long long>(S) * H, &nparts);
   if (st != TP_OK) return st;
-  return run_reduce_ln(S, H, nparts, Zsum, X, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s, dev->sm_count);
+  return run_reduce_ln(S, H, nparts, Zsum, res, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s, dev.sm_count,
+                       apply_ln);
+}
+
+int check_mlp_args(int S, int H, int F, int t, int dtype, int out_dtype, const void* X, const void* const* A_shards,
+                   const void* const* B_shards, const float* gamma, const float* beta, float eps, int act,
+                   const void* Y) {
+  if (t < 1 || t > TP_MAX_SHARDS || S < 0 || H <= 0 || F <= 0) return TP_ERR_INVALID_ARG;
+  if (!valid_out(dtype, out_dtype) || !valid_act(act) || !(eps > 0.0f) || !std::isfinite(eps))
+    return TP_ERR_INVALID_ARG;
+  // With S == 0 nothing is read or written, so X and Y may be null.
+  if ((S > 0 && (!ptr_ok(X) || !ptr_ok(Y))) || !opt_ptr_ok(X) || !opt_ptr_ok(Y) || !shards_ok(A_shards, t) ||
+      !shards_ok(B_shards, t) || !opt_ptr_ok(gamma) || !opt_ptr_ok(beta))
+    return TP_ERR_INVALID_ARG;
+  if (F % t != 0 || (F / t) % 8 != 0 || !hidden_ok(H)) return TP_ERR_UNSUPPORTED_SHAPE;
+  return TP_OK;
+}
+
+int check_attn_args(int S, int H, int nh, int d, int t, int dtype, int out_dtype, const void* X,
+                    const void* const* Wqkv_shards, const void* const* Wo_shards, const float* gamma,
+                    const float* beta, float eps, const void* Y) {
+  if (t < 1 || t > TP_MAX_SHARDS || S < 0 || H <= 0 || nh <= 0 || d <= 0) return TP_ERR_INVALID_ARG;
+  if (dtype != TP_DTYPE_BF16 || !valid_out(dtype, out_dtype) || !(eps > 0.0f) || !std::isfinite(eps))
+    return TP_ERR_INVALID_ARG;
+  if ((S > 0 && (!ptr_ok(X) || !ptr_ok(Y))) || !opt_ptr_ok(X) || !opt_ptr_ok(Y) || !shards_ok(Wqkv_shards, t) ||
+      !shards_ok(Wo_shards, t) || !opt_ptr_ok(gamma) || !opt_ptr_ok(beta))
+    return TP_ERR_INVALID_ARG;
+  if (d != tp::attn::D || static_cast<long long>(nh) * d != H || nh % t != 0 || S % tp::attn::BQ != 0 ||
+      !hidden_ok(H))
+    return TP_ERR_UNSUPPORTED_SHAPE;
+  return TP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype, const void* X,
+                   const void* const* A_shards, const void* const* B_shards, const float* gamma,
+                   const float* beta, float eps, int act, void* Y, void* workspace, size_t workspace_bytes,
+                   void* stream) {
+  int st = check_mlp_args(S, H, F, t, dtype, out_dtype, X, A_shards, B_shards, gamma, beta, eps, act, Y);
+  if (st != TP_OK) return st;
+  if (!opt_ptr_ok(workspace)) return TP_ERR_INVALID_ARG;
+  const size_t need = tp_mlp_workspace_bytes(S, H, F, t, dtype);
+  if (workspace_bytes < need || (need > 0 && !workspace)) return TP_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  return mlp_core(*dev, S, H, F, t, dtype, out_dtype, X, X, A_shards, B_shards, gamma, beta, eps, act, 1, Y,
+                  workspace, static_cast<cudaStream_t>(stream));
+}
+
+// -------------------------------------------------------------- attention
+size_t tp_attn_workspace_bytes(int S, int H, int nh, int d, int t, int dtype) {
+  if (S < 0 || H <= 0 || nh <= 0 || d <= 0 || t < 1 || dtype != TP_DTYPE_BF16) return 0;
+  const size_t s = static_cast<size_t>(S), h = static_cast<size_t>(H);
+  return align256(s * 3 * h * 2) + align256(s * h * 2) + TP_MAX_K_SPLITS * s * h * 4;
+}
+
+int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int out_dtype, const void* X,
+                              const void* const* Wqkv_shards, const void* const* Wo_shards, const float* gamma,
+                              const float* beta, float eps, void* Y, void* workspace, size_t workspace_bytes,
+                              void* stream) {
+  int st = check_attn_args(S, H, nh, d, t, dtype, out_dtype, X, Wqkv_shards, Wo_shards, gamma, beta, eps, Y);
+  if (st != TP_OK) return st;
+  if (!opt_ptr_ok(workspace)) return TP_ERR_INVALID_ARG;
+  const size_t need = tp_attn_workspace_bytes(S, H, nh, d, t, dtype);
+  if (workspace_bytes < need || (need > 0 && !workspace)) return TP_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  return attn_core(*dev, S, H, nh, d, t, out_dtype, X, X, Wqkv_shards, Wo_shards, gamma, beta, eps, 1, Y, workspace,
+                   static_cast<cudaStream_t>(stream));
+}
+
+// ---------------------------------------------------------- Transformer block
+size_t tp_block_workspace_bytes(int S, int H, int F, int nh, int d, int t, int dtype) {
+  if (S < 0 || H <= 0 || F <= 0 || nh <= 0 || d <= 0 || t < 1 || dtype != TP_DTYPE_BF16) return 0;
+  const size_t a = tp_attn_workspace_bytes(S, H, nh, d, t, dtype);
+  const size_t m = tp_mlp_workspace_bytes(S, H, F, t, dtype);
+  const size_t core = align256(a > m ? a : m);
+  const size_t act = align256(static_cast<size_t>(S) * H * 2);
+  return core + 2 * act;
+}
+
+int tp_transformer_block_forward(int S, int H, int F, int nh, int d, int t, int dtype, int out_dtype, int pre_ln,
+                                 const void* X, const void* const* Wqkv_shards, const void* const* Wo_shards,
+                                 const void* const* A_shards, const void* const* B_shards, const float* ln1_gamma,
+                                 const float* ln1_beta, const float* ln2_gamma, const float* ln2_beta, float eps,
+                                 int act, void* Y, void* workspace, size_t workspace_bytes, void* stream) {
+  if (pre_ln != 0 && pre_ln != 1) return TP_ERR_INVALID_ARG;
+  int st = check_attn_args(S, H, nh, d, t, dtype, TP_DTYPE_BF16, X, Wqkv_shards, Wo_shards, ln1_gamma, ln1_beta,
+                           eps, Y);
+  if (st != TP_OK) return st;
+  st = check_mlp_args(S, H, F, t, dtype, out_dtype, X, A_shards, B_shards, ln2_gamma, ln2_beta, eps, act, Y);
+  if (st != TP_OK) return st;
+  if (!opt_ptr_ok(workspace)) return TP_ERR_INVALID_ARG;
+  const size_t need = tp_block_workspace_bytes(S, H, F, nh, d, t, dtype);
+  if (workspace_bytes < need || (need > 0 && !workspace)) return TP_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  if (S == 0) return TP_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t a = tp_attn_workspace_bytes(S, H, nh, d, t, dtype);
+  const size_t m = tp_mlp_workspace_bytes(S, H, F, t, dtype);
+  uint8_t* core = static_cast<uint8_t*>(workspace);
+  uint8_t* buf1 = core + align256(a > m ? a : m);                    // [S, H] bf16
+  uint8_t* buf2 = buf1 + align256(static_cast<size_t>(S) * H * 2);   // [S, H] bf16
+  if (!pre_ln) {
+    // Y1 = LN1(X + Attn(X));  Y = LN2(Y1 + MLP(Y1))
+    st = attn_core(*dev, S, H, nh, d, t, TP_DTYPE_BF16, X, X, Wqkv_shards, Wo_shards, ln1_gamma, ln1_beta, eps, 1,
+                   buf1, core, s);
+    if (st != TP_OK) return st;
+    return mlp_core(*dev, S, H, F, t, dtype, out_dtype, buf1, buf1, A_shards, B_shards, ln2_gamma, ln2_beta, eps,
+                    act, 1, Y, core, s);
+  }
+  // h1 = LN1(X);  Z1 = X + Attn(h1);  h2 = LN2(Z1);  Y = Z1 + MLP(h2)
+  st = run_reduce_ln(S, H, 0, nullptr, X, 1, ln1_gamma, ln1_beta, eps, buf1, 1, s, dev->sm_count, 1);
+  if (st != TP_OK) return st;
+  st = attn_core(*dev, S, H, nh, d, t, TP_DTYPE_BF16, buf1, X, Wqkv_shards, Wo_shards, nullptr, nullptr, eps, 0,
+                 buf2, core, s);
+  if (st != TP_OK) return st;
+  st = run_reduce_ln(S, H, 0, nullptr, buf2, 1, ln2_gamma, ln2_beta, eps, buf1, 1, s, dev->sm_count, 1);
+  if (st != TP_OK) return st;
+  return mlp_core(*dev, S, H, F, t, dtype, out_dtype, buf1, buf2, A_shards, B_shards, nullptr, nullptr, eps, act, 0,
+                  Y, core, s);
 }
 
 // ---------------------------------------------------------------- linears

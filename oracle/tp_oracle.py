@@ -45,7 +45,7 @@ __all__ = [
     "gelu_tanh", "gelu_erf", "relu", "activation",
     "layernorm", "mlp_block", "mlp_block_sharded",
     "linear_column", "linear_row",
-    "attention_heads", "attention_sublayer",
+    "attention_heads", "attention_sublayer", "attention_out", "mlp_out", "transformer_block",
 ]
 
 _COL_BLOCK = 2048  # output-column block for products whose fp64 weight copy is large
@@ -184,6 +184,41 @@ def attention_heads(Q: np.ndarray, K: np.ndarray, V: np.ndarray, nh: int, d: int
         p = p / p.sum(axis=1, keepdims=True)
         O[:, c] = p @ V[:, c]
     return O
+
+
+def attention_out(Xin, Wqkv, Wo, nh: int, d: int, rows=None) -> np.ndarray:
+    """concat_h(softmax(Q_h K_h^T / sqrt d) V_h) W_O for the requested query
+    rows of the input Xin (no residual, no LayerNorm)."""
+    X64 = _f64(Xin)
+    H = X64.shape[1]
+    assert nh * d == H
+    Xr = X64 if rows is None else X64[np.asarray(rows, dtype=np.int64)]
+    Q = _matmul_cols(Xr, Wqkv[:, 0:H])
+    K = _matmul_cols(X64, Wqkv[:, H:2 * H])
+    V = _matmul_cols(X64, Wqkv[:, 2 * H:3 * H])
+    return _matmul_cols(attention_heads(Q, K, V, nh, d), Wo)
+
+
+def mlp_out(Xin_rows, A, B, act: str = "gelu_tanh") -> np.ndarray:
+    """Act(Xin A) B for the given input rows (no residual, no LayerNorm)."""
+    return _matmul_cols(_matmul_cols(_f64(Xin_rows), A, act), B)
+
+
+def transformer_block(X, Wqkv, Wo, A, B, nh: int, d: int, ln1=(None, None), ln2=(None, None),
+                      eps: float = 1e-5, act: str = "gelu_tanh", pre_ln: bool = False, rows=None) -> np.ndarray:
+    """One Transformer block: the attention sublayer then the MLP sublayer
+    ("TP到底在切什么" §2.1 figure 3).  post-LN: Y1 = LN1(X + Attn(X)),
+    Y = LN2(Y1 + MLP(Y1)).  pre-LN: Z1 = X + Attn(LN1(X)), Y = Z1 + MLP(LN2(Z1)).
+    Every output row depends on all rows of X only through the attention's K
+    and V, so a row sample is exact."""
+    X64 = _f64(X)
+    Xr = X64 if rows is None else X64[np.asarray(rows, dtype=np.int64)]
+    if not pre_ln:
+        Y1 = layernorm(Xr + attention_out(X64, Wqkv, Wo, nh, d, rows=rows), ln1[0], ln1[1], eps)
+        return layernorm(Y1 + mlp_out(Y1, A, B, act), ln2[0], ln2[1], eps)
+    h1 = layernorm(X64, ln1[0], ln1[1], eps)
+    Z1 = Xr + attention_out(h1, Wqkv, Wo, nh, d, rows=rows)
+    return Z1 + mlp_out(layernorm(Z1, ln2[0], ln2[1], eps), A, B, act)
 
 
 def attention_sublayer(X, Wqkv, Wo, nh: int, d: int, gamma=None, beta=None,

@@ -276,3 +276,27 @@ def _cached_mlp(w):
     if w.name not in _CACHE:
         _CACHE[w.name] = synth.gen_mlp(w.S, w.H, w.F, seed=w.seed)
     return _CACHE[w.name]
+
+
+# --------------------------------------------------------- Transformer block
+
+@pytest.mark.parametrize("pre_ln", [False, True])
+@pytest.mark.parametrize("S,nh,F,t", [(256, 2, 1024, 2), (384, 4, 2048, 4)])
+def test_transformer_block(cuda_device, pre_ln, S, nh, F, t):
+    d = 128
+    H = nh * d
+    a = synth.gen_attn(S, H, seed=S + 1)
+    m = synth.gen_mlp(S, H, F, seed=S + 2)
+    g = torch.Generator().manual_seed(3)
+    ln1 = (torch.randn(H, generator=g) * 0.2 + 1.0, torch.randn(H, generator=g) * 0.1)
+    ln2 = (torch.randn(H, generator=g) * 0.2 + 1.0, torch.randn(H, generator=g) * 0.1)
+    X = a.X.cuda()
+    Y = torch.empty(S, H, dtype=torch.float32, device="cuda")
+    ws = torch.empty(L.block_workspace_bytes(S, H, F, nh, d, t), dtype=torch.uint8, device="cuda")
+    L.block_forward(X, _dev(synth.split_qkv_by_head(a.Wqkv, nh, d, t)), _dev(synth.split_rows_by_head(a.Wo, nh, d, t)),
+                    _dev(synth.split_columns(m.A, t)), _dev(synth.split_rows(m.B, t)), nh, d, Y, ws, pre_ln=pre_ln,
+                    ln1=(ln1[0].cuda(), ln1[1].cuda()), ln2=(ln2[0].cuda(), ln2[1].cuda()))
+    torch.cuda.synchronize()
+    assert L.device_error() == 0
+    ref = O.transformer_block(a.X, a.Wqkv, a.Wo, m.A, m.B, nh, d, ln1=ln1, ln2=ln2, pre_ln=pre_ln)
+    assert rel_err(Y, ref) <= TOL_BF16

@@ -229,11 +229,42 @@ def check_attention_row_equivariance():
     np.testing.assert_allclose(O.attention_sublayer(inp.X[p], inp.Wqkv, inp.Wo, nh, d), Y[p], atol=1e-12)
 
 
+def check_block_composition():
+    S, nh, d, F = 16, 2, 8, 48
+    H = nh * d
+    a = synth.gen_attn(S, H, seed=12, dtype=torch.float32)
+    m = synth.gen_mlp(S, H, F, seed=13, dtype=torch.float32)
+    # post-LN block = the two pinned sublayers applied in turn
+    Y1 = O.attention_sublayer(a.X, a.Wqkv, a.Wo, nh, d)
+    ref = O.mlp_block(Y1, m.A, m.B)
+    np.testing.assert_allclose(O.transformer_block(a.X, a.Wqkv, a.Wo, m.A, m.B, nh, d), ref, atol=1e-11)
+    # zero output projections make the pre-LN block the identity on X ...
+    Z = np.zeros_like(a.Wo.numpy())
+    Zb = np.zeros_like(m.B.numpy())
+    np.testing.assert_allclose(O.transformer_block(a.X, a.Wqkv, Z, m.A, Zb, nh, d, pre_ln=True),
+                               a.X.double().numpy(), atol=0)
+    # ... and the post-LN block LN(LN(X))
+    np.testing.assert_allclose(O.transformer_block(a.X, a.Wqkv, Z, m.A, Zb, nh, d),
+                               O.layernorm(O.layernorm(a.X.double().numpy())), atol=1e-12)
+    # pre-LN: the MLP sees LN2 of the attention residual stream, the residual is unnormalised
+    h1 = O.layernorm(a.X.double().numpy())
+    Zr = a.X.double().numpy() + O.attention_out(h1, a.Wqkv, a.Wo, nh, d)
+    pre = O.transformer_block(a.X, a.Wqkv, a.Wo, m.A, m.B, nh, d, pre_ln=True)
+    np.testing.assert_allclose(pre, Zr + O.mlp_out(O.layernorm(Zr), m.A, m.B), atol=1e-11)
+    # attention_out + residual + LN is the pinned attention sublayer
+    np.testing.assert_allclose(O.layernorm(a.X.double().numpy() + O.attention_out(a.X, a.Wqkv, a.Wo, nh, d)), Y1,
+                               atol=1e-12)
+    rows = [1, 9, 15]
+    np.testing.assert_allclose(O.transformer_block(a.X, a.Wqkv, a.Wo, m.A, m.B, nh, d, pre_ln=True, rows=rows),
+                               pre[rows], atol=1e-12)
+
+
 ALL_CHECKS = [
     check_gelu_library, check_gelu_identities, check_layernorm_hand, check_layernorm_invariants,
     check_mlp_exact_bruteforce, check_mlp_closed_forms, check_mlp_block_identities,
     check_mlp_symmetries, check_linears_exact, check_attention_hand,
     check_attention_uniform_keys, check_attention_library, check_attention_row_equivariance,
+    check_block_composition,
 ]
 
 

@@ -69,6 +69,13 @@ typedef enum { TP_DTYPE_F32 = 0, TP_DTYPE_BF16 = 1 } tp_dtype;
  * GELU_ERF: 0.5 u (1 + erf(u / sqrt 2)); RELU: max(u, 0). */
 typedef enum { TP_ACT_NONE = 0, TP_ACT_GELU_TANH = 1, TP_ACT_GELU_ERF = 2, TP_ACT_RELU = 3 } tp_act;
 
+/* Weight layouts.  TP_W_IN_OUT: the pages' [in, out] (Y = X W, [PWWT] §1.1),
+ * the layout every entry point without `_ex` takes.  TP_W_OUT_IN: nn.Linear's
+ * [out, in] (`x @ W.T`, [PWWT] §3.2-§3.3): each shard is the transpose of the
+ * [in, out] shard, read K-major by the tensor cores (no transpose pass). */
+#define TP_W_IN_OUT 0
+#define TP_W_OUT_IN 1
+
 /* Library version (TP_API_VERSION) and a static string for a status code. */
 int tp_version(void);
 const char* tp_status_string(int status);
@@ -109,6 +116,14 @@ int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype,
                    const void* X, const void* const* A_shards, const void* const* B_shards,
                    const float* gamma, const float* beta, float eps, int act,
                    void* Y, void* workspace, size_t workspace_bytes, void* stream);
+
+/* tp_mlp_forward with a weight layout: for TP_W_OUT_IN, A_shards[i] is
+ * [F/t, H] (rows i F/t .. of the [F, H] expansion weight) and B_shards[i] is
+ * [H, F/t] (columns i F/t .. of the [H, F] compression weight). */
+int tp_mlp_forward_ex(int S, int H, int F, int t, int dtype, int out_dtype, int w_layout,
+                      const void* X, const void* const* A_shards, const void* const* B_shards,
+                      const float* gamma, const float* beta, float eps, int act,
+                      void* Y, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------- MLP without allocation ----
  * The pages have no counterpart to this entry point: it exists for callers
@@ -152,6 +167,13 @@ int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int
                               const float* gamma, const float* beta, float eps,
                               void* Y, void* workspace, size_t workspace_bytes, void* stream);
 
+/* tp_qkv_attn_oproj_forward with a weight layout: for TP_W_OUT_IN,
+ * Wqkv_shards[s] is [3 (nh/t) d, H] and Wo_shards[s] is [H, (nh/t) d]. */
+int tp_qkv_attn_oproj_forward_ex(int S, int H, int nh, int d, int t, int dtype, int out_dtype, int w_layout,
+                                 const void* X, const void* const* Wqkv_shards, const void* const* Wo_shards,
+                                 const float* gamma, const float* beta, float eps,
+                                 void* Y, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------- Transformer block ----
  * The attention sublayer followed by the MLP sublayer, the two TP pairs of one
  * Transformer block ([PWWT] §2.1 figure 3: QKV/O one pair, the two MLP
@@ -188,6 +210,13 @@ int tp_linear_column_forward(int M, int K, int N, int t, int dtype, int out_dtyp
 int tp_linear_row_forward(int M, int K, int N, int t, int dtype, int out_dtype,
                           const void* X, const void* const* W_shards,
                           void* Y, void* workspace, size_t workspace_bytes, void* stream);
+/* The same with a weight layout: for TP_W_OUT_IN the column-split shard i is
+ * [N/t, K] and the row-split shard i is [N, K/t]. */
+int tp_linear_column_forward_ex(int M, int K, int N, int t, int dtype, int out_dtype, int w_layout,
+                                const void* X, const void* const* W_shards, int act, void* Y, void* stream);
+int tp_linear_row_forward_ex(int M, int K, int N, int t, int dtype, int out_dtype, int w_layout,
+                             const void* X, const void* const* W_shards,
+                             void* Y, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------- reduce + residual + LayerNorm ----
  * Y = LN(X + sum_{p < nparts} P_p) per row over H ([PWWT] §2.3, §5.3): mean,

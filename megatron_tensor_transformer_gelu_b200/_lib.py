@@ -40,6 +40,12 @@ SIGNATURES = {
     "tp_transformer_block_forward": (_c_int, [_c_int] * 9 + [_vp, _vpp, _vpp, _vpp, _vpp, _vp, _vp, _vp, _vp, _c_float,
                                                               _c_int, _vp, _vp, _c_size, _vp]),
     "tp_linear_column_forward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _c_int, _vp, _vp]),
+    "tp_linear_column_forward_ex": (_c_int, [_c_int] * 7 + [_vp, _vpp, _c_int, _vp, _vp]),
+    "tp_linear_row_forward_ex": (_c_int, [_c_int] * 7 + [_vp, _vpp, _vp, _vp, _c_size, _vp]),
+    "tp_mlp_forward_ex": (_c_int, [_c_int] * 7 + [_vp, _vpp, _vpp, _vp, _vp, _c_float, _c_int, _vp, _vp, _c_size,
+                                                   _vp]),
+    "tp_qkv_attn_oproj_forward_ex": (_c_int, [_c_int] * 8 + [_vp, _vpp, _vpp, _vp, _vp, _c_float, _vp, _vp, _c_size,
+                                                              _vp]),
     "tp_linear_row_forward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vp, _vp, _c_size, _vp]),
     "tp_reduce_residual_layernorm": (_c_int, [_c_int] * 3 + [_vp, _vp, _c_int, _vp, _vp, _c_float, _vp, _c_int, _vp]),
     "tp_selftest_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
@@ -103,17 +109,26 @@ def attn_workspace_bytes(S, H, nh, d, t, dtype=torch.bfloat16) -> int:
     return lib().tp_attn_workspace_bytes(S, H, nh, d, t, DTYPE[dtype])
 
 
+LAYOUT = {"in_out": 0, "out_in": 1}
+
+
 def mlp_forward(X, A_shards, B_shards, Y, workspace, gamma=None, beta=None, eps=1e-5,
-                act="gelu_tanh", stream=None):
+                act="gelu_tanh", stream=None, layout="in_out"):
+    """layout "in_out": A_i [H, F/t], B_i [F/t, H]; "out_in" (nn.Linear): A_i [F/t, H], B_i [H, F/t]."""
     S, H = X.shape
     t = len(A_shards)
-    F = sum(a.shape[1] for a in A_shards)
+    F = sum(a.shape[1 if layout == "in_out" else 0] for a in A_shards)
     pa, ka = _ptrs(A_shards)
     pb, kb = _ptrs(B_shards)
-    code = lib().tp_mlp_forward(S, H, F, t, DTYPE[X.dtype], DTYPE[Y.dtype], _ptr(X), pa, pb,
-                                _ptr(gamma), _ptr(beta), float(eps), ACT[act], _ptr(Y),
-                                _ptr(workspace), workspace.numel() * workspace.element_size()
-                                if workspace is not None else 0, _stream(stream))
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    if layout == "in_out":
+        code = lib().tp_mlp_forward(S, H, F, t, DTYPE[X.dtype], DTYPE[Y.dtype], _ptr(X), pa, pb,
+                                    _ptr(gamma), _ptr(beta), float(eps), ACT[act], _ptr(Y),
+                                    _ptr(workspace), ws_bytes, _stream(stream))
+    else:
+        code = lib().tp_mlp_forward_ex(S, H, F, t, DTYPE[X.dtype], DTYPE[Y.dtype], LAYOUT[layout], _ptr(X), pa, pb,
+                                       _ptr(gamma), _ptr(beta), float(eps), ACT[act], _ptr(Y),
+                                       _ptr(workspace), ws_bytes, _stream(stream))
     _check(code, "tp_mlp_forward")
 
 
@@ -131,15 +146,15 @@ def mlp_forward_noalloc(X, A_shards, B_shards, Y, gamma=None, beta=None, eps=1e-
 
 
 def attn_forward(X, Wqkv_shards, Wo_shards, nh, d, Y, workspace, gamma=None, beta=None, eps=1e-5,
-                 stream=None):
+                 stream=None, layout="in_out"):
     S, H = X.shape
     t = len(Wqkv_shards)
     pq, kq = _ptrs(Wqkv_shards)
     po, ko = _ptrs(Wo_shards)
-    code = lib().tp_qkv_attn_oproj_forward(S, H, nh, d, t, DTYPE[X.dtype], DTYPE[Y.dtype], _ptr(X), pq, po,
-                                           _ptr(gamma), _ptr(beta), float(eps), _ptr(Y), _ptr(workspace),
-                                           workspace.numel() * workspace.element_size()
-                                           if workspace is not None else 0, _stream(stream))
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    code = lib().tp_qkv_attn_oproj_forward_ex(S, H, nh, d, t, DTYPE[X.dtype], DTYPE[Y.dtype], LAYOUT[layout],
+                                              _ptr(X), pq, po, _ptr(gamma), _ptr(beta), float(eps), _ptr(Y),
+                                              _ptr(workspace), ws_bytes, _stream(stream))
     _check(code, "tp_qkv_attn_oproj_forward")
 
 
@@ -164,23 +179,23 @@ def block_forward(X, Wqkv_shards, Wo_shards, A_shards, B_shards, nh, d, Y, works
     _check(code, "tp_transformer_block_forward")
 
 
-def linear_column_forward(X, W_shards, Y, act="none", stream=None):
+def linear_column_forward(X, W_shards, Y, act="none", stream=None, layout="in_out"):
     M, K = X.shape
     t = len(W_shards)
-    N = sum(w.shape[1] for w in W_shards)
+    N = sum(w.shape[1 if layout == "in_out" else 0] for w in W_shards)
     pw, kw = _ptrs(W_shards)
-    code = lib().tp_linear_column_forward(M, K, N, t, DTYPE[X.dtype], DTYPE[Y.dtype], _ptr(X), pw, ACT[act],
-                                          _ptr(Y), _stream(stream))
+    code = lib().tp_linear_column_forward_ex(M, K, N, t, DTYPE[X.dtype], DTYPE[Y.dtype], LAYOUT[layout], _ptr(X), pw,
+                                             ACT[act], _ptr(Y), _stream(stream))
     _check(code, "tp_linear_column_forward")
 
 
-def linear_row_forward(X, W_shards, Y, stream=None):
+def linear_row_forward(X, W_shards, Y, stream=None, layout="in_out"):
     M, K = X.shape
     t = len(W_shards)
-    N = W_shards[0].shape[1]
+    N = W_shards[0].shape[1 if layout == "in_out" else 0]
     pw, kw = _ptrs(W_shards)
-    code = lib().tp_linear_row_forward(M, K, N, t, DTYPE[X.dtype], DTYPE[Y.dtype], _ptr(X), pw, _ptr(Y),
-                                       None, 0, _stream(stream))
+    code = lib().tp_linear_row_forward_ex(M, K, N, t, DTYPE[X.dtype], DTYPE[Y.dtype], LAYOUT[layout], _ptr(X), pw,
+                                          _ptr(Y), None, 0, _stream(stream))
     _check(code, "tp_linear_row_forward")
 
 

@@ -69,11 +69,13 @@ struct GemmCfg {
   static constexpr int SMEM_BYTES =
       STAGES * (A_BYTES + B_BYTES) + 2 * EPI_BUF_BYTES + 1024 /*align*/ + 256 /*barriers*/;
   static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN, /*a_mn=*/false, /*b_mn=*/true);
+  // B given K-major ([out, in] weights): one box of B_COLS_CTA rows x 64 k.
+  static constexpr uint32_t IDESC_BK = idesc_bf16_f32(TILE_M, BN, /*a_mn=*/false, /*b_mn=*/false);
 };
 
 struct GemmArgs {
   CUtensorMap tmA;               // A [M, K] bf16 row-major, box {64, 128}
-  CUtensorMap tmB[MAX_SHARDS];   // B shard s, bf16 row-major [rows, cols], box {64, 64}
+  CUtensorMap tmB[MAX_SHARDS];   // B shard s: [k rows, n cols] box {64, 64}, or K-major [n rows, k cols] box {64, BN/CG}
   // Output maps, 3-D {cols, M, splits}, box {128 B of columns, 128, 1}, 128-byte
   // swizzle: column mode one per shard (its column slice of C), row mode one.
   CUtensorMap tmC[MAX_SHARDS];
@@ -95,6 +97,7 @@ struct GemmArgs {
   // C + j * slot_stride (f32 only), and a later kernel adds the slots.
   int splits;
   long long slot_stride;
+  int b_kmajor;                  // B shards stored [n, k] (nn.Linear [out, in] weights)
 };
 
 __device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& kb0, int& kb1) {
@@ -163,12 +166,14 @@ __device__ __forceinline__ void kblock_coords(const GemmArgs& p, const TileCoord
   }
 }
 
-// Number of 64-column B boxes CTA `rank` of the pair loads for a tile.
+// Number of 64-column B boxes CTA `rank` of the pair loads for a tile (N-major
+// B); a K-major B is one box of B_COLS_CTA rows, counted here as B_BOXES.
 template <int CG>
-__device__ __forceinline__ int b_boxes_for(int n_valid, int rank) {
+__device__ __forceinline__ int b_boxes_for(int n_valid, int rank, int b_kmajor) {
   using C = GemmCfg<CG>;
   const int cols = n_valid - rank * C::B_COLS_CTA;
   if (cols <= 0) return 0;
+  if (b_kmajor) return C::B_BOXES;
   return min(C::B_BOXES, (cols + C::B_BOX_N - 1) / C::B_BOX_N);
 }
 
@@ -243,10 +248,11 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         const TileCoord tc = tile_coord<CG>(p, tile);
         const int my_row0 = tc.m0 + static_cast<int>(rank) * C::BM;
         const bool my_a = my_row0 < p.M;
-        const int my_boxes = b_boxes_for<CG>(tc.n_valid, rank);
+        const int my_boxes = b_boxes_for<CG>(tc.n_valid, rank, p.b_kmajor);
         uint32_t bytes = 0;  // leader: bytes the whole tile stage brings in
         for (int r = 0; r < CG; ++r)
-          bytes += (tc.m0 + r * C::BM < p.M ? C::A_BYTES : 0) + b_boxes_for<CG>(tc.n_valid, r) * C::B_BOX_BYTES;
+          bytes += (tc.m0 + r * C::BM < p.M ? C::A_BYTES : 0) +
+                   b_boxes_for<CG>(tc.n_valid, r, p.b_kmajor) * C::B_BOX_BYTES;
         const int b_x0 = tc.n_in + static_cast<int>(rank) * C::B_COLS_CTA;
         for (int kb = kb_begin; kb < kb_end; ++kb) {
           if constexpr (C::PREFETCH > 0) {
@@ -267,8 +273,12 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
             mbar_arrive_expect_tx(&full[stage], bytes);
             armed[stage] = static_cast<int>(phase);
             tma_load_2d(dA, &p.tmA, a_x, my_row0, &full[stage]);
-            for (int j = 0; j < my_boxes; ++j)
-              tma_load_2d(dB + j * C::B_BOX_BYTES, &p.tmB[shard], b_x0 + j * C::B_BOX_N, b_y, &full[stage]);
+            if (p.b_kmajor) {
+              if (my_boxes) tma_load_2d(dB, &p.tmB[shard], b_y, b_x0, &full[stage]);
+            } else {
+              for (int j = 0; j < my_boxes; ++j)
+                tma_load_2d(dB + j * C::B_BOX_BYTES, &p.tmB[shard], b_x0 + j * C::B_BOX_N, b_y, &full[stage]);
+            }
           } else {
             const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
             if (leader) {
@@ -276,8 +286,12 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
               armed[stage] = static_cast<int>(phase);
             }
             if (my_a) tma_load_2d_pair(dA, &p.tmA, a_x, my_row0, bar);
-            for (int j = 0; j < my_boxes; ++j)
-              tma_load_2d_pair(dB + j * C::B_BOX_BYTES, &p.tmB[shard], b_x0 + j * C::B_BOX_N, b_y, bar);
+            if (p.b_kmajor) {
+              if (my_boxes) tma_load_2d_pair(dB, &p.tmB[shard], b_y, b_x0, bar);
+            } else {
+              for (int j = 0; j < my_boxes; ++j)
+                tma_load_2d_pair(dB + j * C::B_BOX_BYTES, &p.tmB[shard], b_x0 + j * C::B_BOX_N, b_y, bar);
+            }
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -311,16 +325,19 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
+          const uint32_t idesc = p.b_kmajor ? C::IDESC_BK : C::IDESC;
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk) {
             // A: K-major, 16 k-elements = 32 bytes further along the swizzled row.
             const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
-            // B: N-major, 16 k-rows = 2 x (8 rows x 128 B) further; 64-column
+            // B N-major: 16 k-rows = 2 x (8 rows x 128 B) further; 64-column
             // chunks are B_BOX_BYTES apart (leading offset), 8-row groups 1 KiB.
-            const uint64_t bd = sdesc_sw128(b0 + kk * 2048, C::B_BOX_BYTES, 1024);
+            // B K-major: like A.
+            const uint64_t bd = p.b_kmajor ? sdesc_sw128(b0 + kk * 32, 16, 1024)
+                                           : sdesc_sw128(b0 + kk * 2048, C::B_BOX_BYTES, 1024);
             const uint32_t accum = (kb != kb_begin || kk != 0) ? 1u : 0u;
-            if constexpr (CG == 1) umma_bf16(d_tmem, ad, bd, C::IDESC, accum);
-            else umma_bf16_pair(d_tmem, ad, bd, C::IDESC, accum);
+            if constexpr (CG == 1) umma_bf16(d_tmem, ad, bd, idesc, accum);
+            else umma_bf16_pair(d_tmem, ad, bd, idesc, accum);
           }
           if constexpr (CG == 1) umma_commit(&empty[stage]);
           else umma_commit_pair_mc(&empty[stage], 0x3);

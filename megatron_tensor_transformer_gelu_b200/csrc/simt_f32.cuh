@@ -22,6 +22,7 @@ struct SimtArgs {
   int row_mode;
   int shard_n, shard_k;
   int act;
+  int b_kmajor;                   // shards stored [shard_n, shard_k] (nn.Linear [out, in])
 };
 
 namespace simt {
@@ -41,12 +42,18 @@ __device__ __forceinline__ float apply_act_precise(float u, int act) {
 }
 
 __device__ __forceinline__ float simt_b(const SimtArgs& p, int k, int n) {
+  int s, kk, nn;
   if (p.row_mode) {
-    const int s = k / p.shard_k;
-    return p.B[s][static_cast<long long>(k - s * p.shard_k) * p.shard_n + n];
+    s = k / p.shard_k;
+    kk = k - s * p.shard_k;
+    nn = n;
+  } else {
+    s = n / p.shard_n;
+    kk = k;
+    nn = n - s * p.shard_n;
   }
-  const int s = n / p.shard_n;
-  return p.B[s][static_cast<long long>(k) * p.shard_n + (n - s * p.shard_n)];
+  return p.b_kmajor ? p.B[s][static_cast<long long>(nn) * p.shard_k + kk]
+                    : p.B[s][static_cast<long long>(kk) * p.shard_n + nn];
 }
 
 // 64x64 output tile per block, 4x4 per thread, K in steps of 16 through smem.

@@ -170,9 +170,6 @@ bool tmap_out(CUtensorMap* m, void* base, int f32, long long cols, long long row
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA; }
 
-// Tensor-core GEMM.  Column mode: B shard s is [K, shard_n], output columns
-// [s*shard_n, (s+1)*shard_n).  Row mode: B shard s is [shard_k, shard_n] and
-// multiplies A's columns [s*shard_k, (s+1)*shard_k); all shards are summed.
 // Number of K splits for `tiles` output tiles on `slots` persistent clusters,
 // from a small cost model: the main loop costs (waves x k-blocks per unit) k-
 // block times (about 0.5 us each for a 256 x 256 x 64 pair step), and every
@@ -243,21 +240,31 @@ int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, int max_splits, cudaS
 // Tensor-core GEMM.  Column mode: B shard s is [K, shard_n], output columns
 // [s*shard_n, (s+1)*shard_n).  Row mode: B shard s is [shard_k, shard_n] and
 // multiplies A's columns [s*shard_k, (s+1)*shard_k); all shards are summed.
+// With b_kmajor every shard is stored transposed ([shard_n, shard_k], the
+// nn.Linear [out, in] layout) and read K-major.
 // With max_splits > 1 (f32 output only) the K loop may be cut into up to
 // max_splits ranges whose partial sums land in slots `slot_stride` elements
 // apart; *splits_out tells the caller how many slots to add.
 int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, const void* const* B, int t,
                 int row_mode, int shard_k, int shard_n, void* C, long long ldc, int out_f32, int act,
-                cudaStream_t st, int max_splits = 1, long long slot_stride = 0, int* splits_out = nullptr) {
-  if (splits_out) *splits_out = 1;
+                cudaStream_t st, int max_splits = 1, long long slot_stride = 0, int* splits_out = nullptr,
+                int b_kmajor = 0) {
   using G = tp::GemmCfg<1>;
+  if (splits_out) *splits_out = 1;
   if (M == 0) return TP_OK;
+  const bool pair = M >= TP_GEMM_PAIR_MIN_ROWS;
   tp::GemmArgs p;
   std::memset(&p, 0, sizeof(p));
   const long long K_total = row_mode ? static_cast<long long>(shard_k) * t : shard_k;
   if (!tmap_bf16(&p.tmA, A, M, K_total, lda, G::BK, G::BM)) return TP_ERR_CUDA;
-  for (int s = 0; s < t; ++s)
-    if (!tmap_bf16(&p.tmB[s], B[s], shard_k, shard_n, shard_n, G::B_BOX_N, G::BK)) return TP_ERR_CUDA;
+  for (int s = 0; s < t; ++s) {
+    bool ok;
+    if (b_kmajor)  // shard [shard_n rows, shard_k cols]; box 64 k x (BN / CG) rows
+      ok = tmap_bf16(&p.tmB[s], B[s], shard_n, shard_k, shard_k, G::BK, pair ? tp::GemmCfg<2>::B_COLS_CTA : G::BN);
+    else           // shard [shard_k rows, shard_n cols]; box 64 n x 64 k
+      ok = tmap_bf16(&p.tmB[s], B[s], shard_k, shard_n, shard_n, G::B_BOX_N, G::BK);
+    if (!ok) return TP_ERR_CUDA;
+  }
   p.C = C;
   p.ldc = ldc;
   p.M = M;
@@ -272,15 +279,15 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
   p.out_f32 = out_f32;
   p.splits = 1;
   p.slot_stride = slot_stride;
+  p.b_kmajor = b_kmajor;
   if (!out_f32) max_splits = 1;
-  const int r = M >= TP_GEMM_PAIR_MIN_ROWS ? launch_gemm_tc<2>(dev, p, max_splits, st)
-                                           : launch_gemm_tc<1>(dev, p, max_splits, st);
+  const int r = pair ? launch_gemm_tc<2>(dev, p, max_splits, st) : launch_gemm_tc<1>(dev, p, max_splits, st);
   if (splits_out) *splits_out = p.splits;
   return r;
 }
 
 int run_gemm_simt(const float* A, long long lda, int M, const void* const* B, int t, int row_mode, int shard_k,
-                  int shard_n, float* C, long long ldc, int act, cudaStream_t st) {
+                  int shard_n, float* C, long long ldc, int act, cudaStream_t st, int b_kmajor = 0) {
   if (M == 0) return TP_OK;
   tp::SimtArgs p;
   std::memset(&p, 0, sizeof(p));
@@ -296,6 +303,7 @@ int run_gemm_simt(const float* A, long long lda, int M, const void* const* B, in
   p.N = row_mode ? shard_n : shard_n * t;
   p.K = row_mode ? shard_k * t : shard_k;
   p.act = act;
+  p.b_kmajor = b_kmajor;
   dim3 grid(ceil_div(p.N, tp::simt::TN), ceil_div(M, tp::simt::TM));
   ProfScope ps(K_GEMM_SIMT, st);
   tp::simt_gemm_f32_kernel<<<grid, tp::simt::THREADS, 0, st>>>(p);
@@ -408,7 +416,8 @@ namespace {
 // Arguments are already checked.
 int mlp_core(const DeviceInfo& dev, int S, int H, int F, int t, int dtype, int out_dtype, const void* in,
              const void* res, const void* const* A_shards, const void* const* B_shards, const float* gamma,
-             const float* beta, float eps, int act, int apply_ln, void* Y, void* workspace, cudaStream_t s) {
+             const float* beta, float eps, int act, int apply_ln, void* Y, void* workspace, cudaStream_t s,
+             int kmaj = 0) {
   if (S == 0) return TP_OK;
   const int Fs = F / t;
   int nparts = 1;
@@ -420,18 +429,18 @@ int mlp_core(const DeviceInfo& dev, int S, int H, int F, int t, int dtype, int o
   if (dtype == TP_DTYPE_BF16) {
     // H_i = Act(in A_i) into columns [i Fs, (i+1) Fs) of Hbuf [S, F] (bf16).
     st = run_gemm_tc(dev, in, H, S, A_shards, t, /*row_mode=*/0, /*shard_k=*/H, /*shard_n=*/Fs, Hbuf, F,
-                     /*out_f32=*/0, act, s);
+                     /*out_f32=*/0, act, s, 1, 0, nullptr, kmaj);
     if (st != TP_OK) return st;
     // Zsum = sum_i H_i B_i, accumulated in TMEM across the shards (f32); the K
     // loop may be cut into `nparts` ranges (partial-sum slots) to fill the GPU.
     st = run_gemm_tc(dev, Hbuf, F, S, B_shards, t, /*row_mode=*/1, /*shard_k=*/Fs, /*shard_n=*/H, Zsum, H,
-                     /*out_f32=*/1, TP_ACT_NONE, s, TP_MAX_K_SPLITS, static_cast<long long>(S) * H, &nparts);
+                     /*out_f32=*/1, TP_ACT_NONE, s, TP_MAX_K_SPLITS, static_cast<long long>(S) * H, &nparts, kmaj);
     if (st != TP_OK) return st;
   } else {
     st = run_gemm_simt(static_cast<const float*>(in), H, S, A_shards, t, 0, H, Fs, static_cast<float*>(Hbuf), F,
-                       act, s);
+                       act, s, kmaj);
     if (st != TP_OK) return st;
-    st = run_gemm_simt(static_cast<const float*>(Hbuf), F, S, B_shards, t, 1, Fs, H, Zsum, H, TP_ACT_NONE, s);
+    st = run_gemm_simt(static_cast<const float*>(Hbuf), F, S, B_shards, t, 1, Fs, H, Zsum, H, TP_ACT_NONE, s, kmaj);
     if (st != TP_OK) return st;
   }
   return run_reduce_ln(S, H, nparts, Zsum, res, dtype == TP_DTYPE_BF16, gamma, beta, eps, Y,
@@ -442,7 +451,8 @@ int mlp_core(const DeviceInfo& dev, int S, int H, int F, int t, int dtype, int o
 // or Y = res + O Wo (apply_ln = 0).  Arguments are already checked.
 int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out_dtype, const void* in,
               const void* res, const void* const* Wqkv_shards, const void* const* Wo_shards, const float* gamma,
-              const float* beta, float eps, int apply_ln, void* Y, void* workspace, cudaStream_t s) {
+              const float* beta, float eps, int apply_ln, void* Y, void* workspace, cudaStream_t s,
+              int kmaj = 0) {
   if (S == 0) return TP_OK;
   const int Hs = H / t;  // columns of one shard's heads
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -450,7 +460,8 @@ int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out
   void* Obuf = ws + align256(static_cast<size_t>(S) * 3 * H * 2);            // [S, H]  bf16
   float* Zsum = reinterpret_cast<float*>(static_cast<uint8_t*>(Obuf) + align256(static_cast<size_t>(S) * H * 2));
   // [Q_s | K_s | V_s] = in Wqkv_s into columns [3 s Hs, 3 (s+1) Hs) of QKV.
-  int st = run_gemm_tc(dev, in, H, S, Wqkv_shards, t, 0, H, 3 * Hs, QKV, 3LL * H, 0, TP_ACT_NONE, s);
+  int st = run_gemm_tc(dev, in, H, S, Wqkv_shards, t, 0, H, 3 * Hs, QKV, 3LL * H, 0, TP_ACT_NONE, s, 1, 0, nullptr,
+                       kmaj);
   if (st != TP_OK) return st;
   // O_h = softmax(Q_h K_h^T / sqrt d) V_h, written to columns [h d, (h+1) d) of O.
   {
@@ -475,7 +486,7 @@ int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out
   // sum_s O_s Wo_s, the O projection row-split by head, summed in TMEM.
   int nparts = 1;
   st = run_gemm_tc(dev, Obuf, H, S, Wo_shards, t, 1, Hs, H, Zsum, H, 1, TP_ACT_NONE, s, TP_MAX_K_SPLITS,
-                   static_cast<long long>(S) * H, &nparts);
+                   static_cast<long long>(S) * H, &nparts, kmaj);
   if (st != TP_OK) return st;
   return run_reduce_ln(S, H, nparts, Zsum, res, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s, dev.sm_count,
                        apply_ln);
@@ -518,6 +529,15 @@ int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype, const v
                    const void* const* A_shards, const void* const* B_shards, const float* gamma,
                    const float* beta, float eps, int act, void* Y, void* workspace, size_t workspace_bytes,
                    void* stream) {
+  return tp_mlp_forward_ex(S, H, F, t, dtype, out_dtype, TP_W_IN_OUT, X, A_shards, B_shards, gamma, beta, eps, act, Y,
+                           workspace, workspace_bytes, stream);
+}
+
+int tp_mlp_forward_ex(int S, int H, int F, int t, int dtype, int out_dtype, int w_layout, const void* X,
+                      const void* const* A_shards, const void* const* B_shards, const float* gamma,
+                      const float* beta, float eps, int act, void* Y, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+  if (w_layout != TP_W_IN_OUT && w_layout != TP_W_OUT_IN) return TP_ERR_INVALID_ARG;
   int st = check_mlp_args(S, H, F, t, dtype, out_dtype, X, A_shards, B_shards, gamma, beta, eps, act, Y);
   if (st != TP_OK) return st;
   if (!opt_ptr_ok(workspace)) return TP_ERR_INVALID_ARG;
@@ -527,7 +547,7 @@ int tp_mlp_forward(int S, int H, int F, int t, int dtype, int out_dtype, const v
   st = device_ready(&dev);
   if (st != TP_OK) return st;
   return mlp_core(*dev, S, H, F, t, dtype, out_dtype, X, X, A_shards, B_shards, gamma, beta, eps, act, 1, Y,
-                  workspace, static_cast<cudaStream_t>(stream));
+                  workspace, static_cast<cudaStream_t>(stream), w_layout == TP_W_OUT_IN);
 }
 
 // -------------------------------------------------------------- attention
@@ -541,6 +561,15 @@ int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int
                               const void* const* Wqkv_shards, const void* const* Wo_shards, const float* gamma,
                               const float* beta, float eps, void* Y, void* workspace, size_t workspace_bytes,
                               void* stream) {
+  return tp_qkv_attn_oproj_forward_ex(S, H, nh, d, t, dtype, out_dtype, TP_W_IN_OUT, X, Wqkv_shards, Wo_shards, gamma,
+                                      beta, eps, Y, workspace, workspace_bytes, stream);
+}
+
+int tp_qkv_attn_oproj_forward_ex(int S, int H, int nh, int d, int t, int dtype, int out_dtype, int w_layout,
+                                 const void* X, const void* const* Wqkv_shards, const void* const* Wo_shards,
+                                 const float* gamma, const float* beta, float eps, void* Y, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  if (w_layout != TP_W_IN_OUT && w_layout != TP_W_OUT_IN) return TP_ERR_INVALID_ARG;
   int st = check_attn_args(S, H, nh, d, t, dtype, out_dtype, X, Wqkv_shards, Wo_shards, gamma, beta, eps, Y);
   if (st != TP_OK) return st;
   if (!opt_ptr_ok(workspace)) return TP_ERR_INVALID_ARG;
@@ -550,7 +579,7 @@ int tp_qkv_attn_oproj_forward(int S, int H, int nh, int d, int t, int dtype, int
   st = device_ready(&dev);
   if (st != TP_OK) return st;
   return attn_core(*dev, S, H, nh, d, t, out_dtype, X, X, Wqkv_shards, Wo_shards, gamma, beta, eps, 1, Y, workspace,
-                   static_cast<cudaStream_t>(stream));
+                   static_cast<cudaStream_t>(stream), w_layout == TP_W_OUT_IN);
 }
 
 // ---------------------------------------------------------- Transformer block
@@ -610,8 +639,14 @@ int tp_transformer_block_forward(int S, int H, int F, int nh, int d, int t, int 
 // ---------------------------------------------------------------- linears
 int tp_linear_column_forward(int M, int K, int N, int t, int dtype, int out_dtype, const void* X,
                              const void* const* W_shards, int act, void* Y, void* stream) {
+  return tp_linear_column_forward_ex(M, K, N, t, dtype, out_dtype, TP_W_IN_OUT, X, W_shards, act, Y, stream);
+}
+
+int tp_linear_column_forward_ex(int M, int K, int N, int t, int dtype, int out_dtype, int w_layout, const void* X,
+                                const void* const* W_shards, int act, void* Y, void* stream) {
   if (t < 1 || t > TP_MAX_SHARDS || M < 0 || K <= 0 || N <= 0) return TP_ERR_INVALID_ARG;
   if (!valid_out(dtype, out_dtype) || !valid_act(act)) return TP_ERR_INVALID_ARG;
+  if (w_layout != TP_W_IN_OUT && w_layout != TP_W_OUT_IN) return TP_ERR_INVALID_ARG;
   if ((M > 0 && (!ptr_ok(X) || !ptr_ok(Y))) || !opt_ptr_ok(X) || !opt_ptr_ok(Y) || !shards_ok(W_shards, t))
     return TP_ERR_INVALID_ARG;
   if (K % 8 != 0 || N % t != 0 || (N / t) % 8 != 0) return TP_ERR_UNSUPPORTED_SHAPE;
@@ -619,19 +654,29 @@ int tp_linear_column_forward(int M, int K, int N, int t, int dtype, int out_dtyp
   int st = device_ready(&dev);
   if (st != TP_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int kmaj = w_layout == TP_W_OUT_IN;
   if (dtype == TP_DTYPE_BF16)
-    return run_gemm_tc(*dev, X, K, M, W_shards, t, 0, K, N / t, Y, N, out_dtype == TP_DTYPE_F32, act, s);
+    return run_gemm_tc(*dev, X, K, M, W_shards, t, 0, K, N / t, Y, N, out_dtype == TP_DTYPE_F32, act, s, 1, 0, nullptr,
+                       kmaj);
   return run_gemm_simt(static_cast<const float*>(X), K, M, W_shards, t, 0, K, N / t, static_cast<float*>(Y), N,
-                       act, s);
+                       act, s, kmaj);
 }
 
 int tp_linear_row_forward(int M, int K, int N, int t, int dtype, int out_dtype, const void* X,
                           const void* const* W_shards, void* Y, void* workspace, size_t workspace_bytes,
                           void* stream) {
+  return tp_linear_row_forward_ex(M, K, N, t, dtype, out_dtype, TP_W_IN_OUT, X, W_shards, Y, workspace,
+                                  workspace_bytes, stream);
+}
+
+int tp_linear_row_forward_ex(int M, int K, int N, int t, int dtype, int out_dtype, int w_layout, const void* X,
+                             const void* const* W_shards, void* Y, void* workspace, size_t workspace_bytes,
+                             void* stream) {
   (void)workspace;
   (void)workspace_bytes;
   if (t < 1 || t > TP_MAX_SHARDS || M < 0 || K <= 0 || N <= 0) return TP_ERR_INVALID_ARG;
   if (!valid_out(dtype, out_dtype)) return TP_ERR_INVALID_ARG;
+  if (w_layout != TP_W_IN_OUT && w_layout != TP_W_OUT_IN) return TP_ERR_INVALID_ARG;
   if ((M > 0 && (!ptr_ok(X) || !ptr_ok(Y))) || !opt_ptr_ok(X) || !opt_ptr_ok(Y) || !shards_ok(W_shards, t))
     return TP_ERR_INVALID_ARG;
   if (K % t != 0 || (K / t) % 8 != 0 || N % 8 != 0) return TP_ERR_UNSUPPORTED_SHAPE;
@@ -639,10 +684,12 @@ int tp_linear_row_forward(int M, int K, int N, int t, int dtype, int out_dtype, 
   int st = device_ready(&dev);
   if (st != TP_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int kmaj = w_layout == TP_W_OUT_IN;
   if (dtype == TP_DTYPE_BF16)
-    return run_gemm_tc(*dev, X, K, M, W_shards, t, 1, K / t, N, Y, N, out_dtype == TP_DTYPE_F32, TP_ACT_NONE, s);
+    return run_gemm_tc(*dev, X, K, M, W_shards, t, 1, K / t, N, Y, N, out_dtype == TP_DTYPE_F32, TP_ACT_NONE, s, 1,
+                       0, nullptr, kmaj);
   return run_gemm_simt(static_cast<const float*>(X), K, M, W_shards, t, 1, K / t, N, static_cast<float*>(Y), N,
-                       TP_ACT_NONE, s);
+                       TP_ACT_NONE, s, kmaj);
 }
 
 // -------------------------------------------- reduce + residual + LayerNorm

@@ -139,6 +139,18 @@ def test_linear_and_layernorm_argument_checks(lib):
                                             ctypes.c_void_p(FAKE), 1, None) == INVALID
 
 
+def test_weight_layout_argument_checks(lib):
+    pw, kw = _ptrs(2)
+    X, Y = ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE)
+    for layout in (-1, 2):
+        assert lib.tp_linear_column_forward_ex(64, 128, 256, 2, 1, 0, layout, X, pw, 0, Y, None) == INVALID
+        assert lib.tp_linear_row_forward_ex(64, 128, 256, 2, 1, 0, layout, X, pw, Y, None, 0, None) == INVALID
+        assert lib.tp_mlp_forward_ex(64, 128, 256, 2, 1, 1, layout, X, pw, pw, None, None, 1e-5, 1, Y, X,
+                                     1 << 30, None) == INVALID
+        assert lib.tp_qkv_attn_oproj_forward_ex(128, 256, 2, 128, 2, 1, 1, layout, X, pw, pw, None, None, 1e-5,
+                                                Y, X, 1 << 30, None) == INVALID
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a CUDA device")
 def test_valid_call_without_device_reports_no_device(lib):
     assert _mlp(lib) == NO_DEVICE

@@ -228,6 +228,18 @@ int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts,
                                  const void* X, int x_dtype, const float* gamma, const float* beta,
                                  float eps, void* Y, int out_dtype, void* stream);
 
+/* -------------------------------------------------------- GEMM tiling ----
+ * Tuning override for the tensor-core GEMMs (every sublayer and linear here).
+ * tile_n == 0 (the default): a cost model picks, per launch, 256-column tiles
+ * (with an optional K split for f32 partial sums) or wide tiles of up to 512
+ * columns (two MMAs per K step filling TMEM) where they give fuller waves on
+ * the SM pairs.  tile_n in [256, 512], a multiple of 32: every GEMM of at
+ * least 129 rows uses that tile width (rounded up to a multiple of 64 for
+ * bf16 output) and no K split.  Results are the same to rounding either way.
+ * Process-wide, not thread-safe against concurrent launches.  Returns
+ * TP_ERR_INVALID_ARG for other values. */
+int tp_set_gemm_tile_n(int tile_n);
+
 /* ------------------------------------------------------------ self-test ----
  * Diagnostic for the bounded-wait path every kernel here takes when one of its
  * device-side waits gives up: launches one CTA whose mbarrier wait nothing can

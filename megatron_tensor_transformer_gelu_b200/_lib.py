@@ -48,6 +48,7 @@ SIGNATURES = {
                                                               _vp]),
     "tp_linear_row_forward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vp, _vp, _c_size, _vp]),
     "tp_reduce_residual_layernorm": (_c_int, [_c_int] * 3 + [_vp, _vp, _c_int, _vp, _vp, _c_float, _vp, _c_int, _vp]),
+    "tp_set_gemm_tile_n": (_c_int, [_c_int]),
     "tp_selftest_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
     "tp_profile_enable": (_c_int, [_c_int]),
     "tp_profile_collect": (_c_int, [ctypes.POINTER(_c_int), ctypes.POINTER(_c_int), ctypes.POINTER(ctypes.c_double),
@@ -206,6 +207,11 @@ def reduce_residual_layernorm(parts, X, Y, gamma=None, beta=None, eps=1e-5, stre
     code = lib().tp_reduce_residual_layernorm(S, H, nparts, _ptr(parts), _ptr(X), DTYPE[X.dtype], _ptr(gamma),
                                               _ptr(beta), float(eps), _ptr(Y), DTYPE[Y.dtype], _stream(stream))
     _check(code, "tp_reduce_residual_layernorm")
+
+
+def set_gemm_tile_n(tile_n: int) -> None:
+    """0: the library's cost model picks GEMM tiles; 256..512: force that tile width."""
+    _check(lib().tp_set_gemm_tile_n(int(tile_n)), "tp_set_gemm_tile_n")
 
 
 def selftest_wait_timeout(limit_cycles: int, stream=None):

@@ -29,6 +29,12 @@
 // The accumulator is double-buffered in TMEM (2 x 256 of the 512 columns), so
 // the epilogue of tile i overlaps the main loop of tile i+1.  No load uses
 // cluster multicast: every CTA fetches its own operand boxes.
+//
+// Wide tiles (WIDE = true, pairs only): a tile is 256 rows by up to 512
+// columns, computed as two MMAs per K step (N = 256 into TMEM columns
+// [0, 256), N = n2 into [256, 256 + n2)).  The accumulator then fills TMEM and
+// is single-buffered, but every operand byte feeds more MACs and the tile
+// count can be matched to the number of SM pairs (fewer, fuller waves).
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -41,7 +47,7 @@ constexpr int MAX_SHARDS = 8;
 
 enum : int { ACT_NONE = 0, ACT_GELU_TANH = 1, ACT_GELU_ERF = 2, ACT_RELU = 3 };
 
-template <int CG>
+template <int CG, bool WIDE = false>
 struct GemmCfg {
   static constexpr int BM = 128;                    // accumulator rows per CTA
   static constexpr int TILE_M = BM * CG;            // rows per (cluster) tile
@@ -53,14 +59,21 @@ struct GemmCfg {
 #ifndef TP_GEMM_L2_PREFETCH
 #define TP_GEMM_L2_PREFETCH 0
 #endif
-  static constexpr int STAGES = CG == 2 ? TP_GEMM_PAIR_STAGES : 4;
+#ifndef TP_GEMM_WIDE_STAGES
+#define TP_GEMM_WIDE_STAGES 4
+#endif
+  static_assert(!WIDE || CG == 2, "wide tiles need a CTA pair");
+  static constexpr int STAGES = WIDE ? TP_GEMM_WIDE_STAGES : (CG == 2 ? TP_GEMM_PAIR_STAGES : 4);
   static constexpr int PREFETCH = TP_GEMM_L2_PREFETCH;  // k-blocks ahead (0 = off)
   static constexpr int A_BYTES = BM * BK * 2;       // 16 KiB
   static constexpr int B_BOX_N = 64;                // 64 bf16 = one 128-byte swizzle row
   static constexpr int B_BOX_BYTES = BK * B_BOX_N * 2;  // 8 KiB
-  static constexpr int B_COLS_CTA = BN / CG;        // B columns each CTA loads
+  static constexpr int B_COLS_CTA = BN / CG;        // B columns each CTA loads for the first MMA
   static constexpr int B_BOXES = B_COLS_CTA / B_BOX_N;
-  static constexpr int B_BYTES = BK * B_COLS_CTA * 2;
+  static constexpr int B_REGION_BYTES = BK * B_COLS_CTA * 2;
+  // Wide tiles: a second region holds this CTA's half of the second MMA's B.
+  static constexpr int B_BYTES = (WIDE ? 2 : 1) * B_REGION_BYTES;
+  static constexpr int ACC_BUFS = WIDE ? 1 : 2;     // accumulators in TMEM
   static constexpr int NUM_THREADS = 192;
   static constexpr int TMEM_COLS = 512;
   // Epilogue staging: two buffers of 128 rows x 128 bytes (32 f32 or 64 bf16
@@ -98,6 +111,9 @@ struct GemmArgs {
   int splits;
   long long slot_stride;
   int b_kmajor;                  // B shards stored [n, k] (nn.Linear [out, in] weights)
+  int tile_n;                    // columns per tile: BN, or up to 2*BN for wide tiles
+  int n2;                        // wide tiles: N of the second MMA (tile_n - BN), else 0
+  uint32_t idesc2;               // wide tiles: instruction descriptor of the second MMA
 };
 
 __device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& kb0, int& kb1) {
@@ -105,21 +121,69 @@ __device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& k
   kb1 = static_cast<int>(static_cast<long long>(split + 1) * p.k_blocks / p.splits);
 }
 
-__device__ __forceinline__ float apply_act(float u, int act) {
-  if (act == ACT_GELU_TANH) {
-    const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
-    return 0.5f * u * (1.0f + tanh_fast(k0 * fmaf(0.044715f * u, u * u, u)));
-  } else if (act == ACT_GELU_ERF) {
-    return 0.5f * u * (1.0f + erff(u * 0.7071067811865476f));
-  } else if (act == ACT_RELU) {
-    return fmaxf(u, 0.0f);
-  }
-  return u;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Epilogue work on one 128-byte output chunk of this thread's accumulator row:
+// tcgen05.ld, activation, conversion, and a 128-byte-swizzled row write into
+// the staging buffer.  The activation is a template argument so the element
+// loop holds only that activation's instructions (a runtime switch per
+// element gets if-converted into evaluating every activation).
+template <int ACT>
+__device__ __forceinline__ float act_t(float u) {
+  if constexpr (ACT == ACT_GELU_TANH) {
+    const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+    return 0.5f * u * (1.0f + tanh_fast(k0 * fmaf(0.044715f * u, u * u, u)));
+  } else if constexpr (ACT == ACT_GELU_ERF) {
+    return 0.5f * u * (1.0f + erff(u * 0.7071067811865476f));
+  } else if constexpr (ACT == ACT_RELU) {
+    return fmaxf(u, 0.0f);
+  } else {
+    return u;
+  }
+}
+
+template <int ACT>
+__device__ __forceinline__ void epi_chunk_f32(uint32_t taddr, uint8_t* stage_row, int row_local) {
+  uint32_t r[32];
+  tmem_ld_32x32b_x32(taddr, r);
+  tmem_wait_ld();
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {  // 16-byte chunk j = 4 f32
+    uint4 w;
+    w.x = __float_as_uint(act_t<ACT>(__uint_as_float(r[4 * j + 0])));
+    w.y = __float_as_uint(act_t<ACT>(__uint_as_float(r[4 * j + 1])));
+    w.z = __float_as_uint(act_t<ACT>(__uint_as_float(r[4 * j + 2])));
+    w.w = __float_as_uint(act_t<ACT>(__uint_as_float(r[4 * j + 3])));
+    *reinterpret_cast<uint4*>(stage_row + ((j ^ (row_local & 7)) << 4)) = w;
+  }
+}
+
+template <int ACT>
+__device__ __forceinline__ void epi_chunk_bf16(uint32_t taddr, uint8_t* stage_row, int row_local) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(taddr + h * 32, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {  // 16-byte chunk 4h+j = 8 bf16
+      uint4 w;
+      w.x = pack_bf16x2(act_t<ACT>(__uint_as_float(r[8 * j + 0])), act_t<ACT>(__uint_as_float(r[8 * j + 1])));
+      w.y = pack_bf16x2(act_t<ACT>(__uint_as_float(r[8 * j + 2])), act_t<ACT>(__uint_as_float(r[8 * j + 3])));
+      w.z = pack_bf16x2(act_t<ACT>(__uint_as_float(r[8 * j + 4])), act_t<ACT>(__uint_as_float(r[8 * j + 5])));
+      w.w = pack_bf16x2(act_t<ACT>(__uint_as_float(r[8 * j + 6])), act_t<ACT>(__uint_as_float(r[8 * j + 7])));
+      *reinterpret_cast<uint4*>(stage_row + (((4 * h + j) ^ (row_local & 7)) << 4)) = w;
+    }
+  }
+}
+
+template <int ACT>
+__device__ __forceinline__ void epi_chunk(bool out_f32, uint32_t taddr, uint8_t* stage_row, int row_local) {
+  if (out_f32) epi_chunk_f32<ACT>(taddr, stage_row, row_local);
+  else epi_chunk_bf16<ACT>(taddr, stage_row, row_local);
 }
 
 // Tile coordinates shared by the three roles.
@@ -140,14 +204,14 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& p, int tile) {
   c.m0 = mb * C::TILE_M;
   if (!p.row_mode) {
     c.shard = nb / p.n_blocks_per_shard;
-    c.n_in = (nb % p.n_blocks_per_shard) * C::BN;
+    c.n_in = (nb % p.n_blocks_per_shard) * p.tile_n;
     c.out_col0 = c.shard * p.shard_n + c.n_in;
   } else {
     c.shard = 0;
-    c.n_in = nb * C::BN;
+    c.n_in = nb * p.tile_n;
     c.out_col0 = c.n_in;
   }
-  c.n_valid = min(C::BN, p.shard_n - c.n_in);
+  c.n_valid = min(p.tile_n, p.shard_n - c.n_in);
   return c;
 }
 
@@ -171,15 +235,27 @@ __device__ __forceinline__ void kblock_coords(const GemmArgs& p, const TileCoord
 template <int CG>
 __device__ __forceinline__ int b_boxes_for(int n_valid, int rank, int b_kmajor) {
   using C = GemmCfg<CG>;
-  const int cols = n_valid - rank * C::B_COLS_CTA;
+  const int cols = min(n_valid, C::BN) - rank * C::B_COLS_CTA;
   if (cols <= 0) return 0;
   if (b_kmajor) return C::B_BOXES;
   return min(C::B_BOXES, (cols + C::B_BOX_N - 1) / C::B_BOX_N);
 }
 
-template <int CG>
+// Wide tiles: B boxes CTA `rank` loads for the second MMA, whose n2 columns
+// (tile columns [BN, BN + n2)) the pair splits in halves of n2/2.  Counted in
+// B_BOX_BYTES units; a K-major B is one box of up to B_COLS_CTA rows.
+__device__ __forceinline__ int b2_boxes_for(int n_valid, int n2, int rank, int b_kmajor) {
+  using C = GemmCfg<2, true>;
+  const int half = n2 / 2;
+  const int cols = min(n_valid - C::BN - rank * half, half);
+  if (cols <= 0) return 0;
+  if (b_kmajor) return C::B_BOXES;
+  return (cols + C::B_BOX_N - 1) / C::B_BOX_N;
+}
+
+template <int CG, bool WIDE = false>
 __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kernel(const __grid_constant__ GemmArgs p) {
-  using C = GemmCfg<CG>;
+  using C = GemmCfg<CG, WIDE>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -249,11 +325,15 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         const int my_row0 = tc.m0 + static_cast<int>(rank) * C::BM;
         const bool my_a = my_row0 < p.M;
         const int my_boxes = b_boxes_for<CG>(tc.n_valid, rank, p.b_kmajor);
+        const int my_boxes2 = WIDE ? b2_boxes_for(tc.n_valid, p.n2, rank, p.b_kmajor) : 0;
         uint32_t bytes = 0;  // leader: bytes the whole tile stage brings in
-        for (int r = 0; r < CG; ++r)
+        for (int r = 0; r < CG; ++r) {
           bytes += (tc.m0 + r * C::BM < p.M ? C::A_BYTES : 0) +
                    b_boxes_for<CG>(tc.n_valid, r, p.b_kmajor) * C::B_BOX_BYTES;
+          if constexpr (WIDE) bytes += b2_boxes_for(tc.n_valid, p.n2, r, p.b_kmajor) * C::B_BOX_BYTES;
+        }
         const int b_x0 = tc.n_in + static_cast<int>(rank) * C::B_COLS_CTA;
+        const int b_x2 = tc.n_in + C::BN + static_cast<int>(rank) * (p.n2 / 2);  // wide: second region
         for (int kb = kb_begin; kb < kb_end; ++kb) {
           if constexpr (C::PREFETCH > 0) {
             const int kp = kb + C::PREFETCH;
@@ -292,6 +372,15 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
               for (int j = 0; j < my_boxes; ++j)
                 tma_load_2d_pair(dB + j * C::B_BOX_BYTES, &p.tmB[shard], b_x0 + j * C::B_BOX_N, b_y, bar);
             }
+            if constexpr (WIDE) {
+              uint8_t* dB2 = dB + C::B_REGION_BYTES;
+              if (p.b_kmajor) {
+                if (my_boxes2) tma_load_2d_pair(dB2, &p.tmB[shard], b_y, b_x2, bar);
+              } else {
+                for (int j = 0; j < my_boxes2; ++j)
+                  tma_load_2d_pair(dB2 + j * C::B_BOX_BYTES, &p.tmB[shard], b_x2 + j * C::B_BOX_N, b_y, bar);
+              }
+            }
           }
           if (++stage == STAGES) { stage = 0; phase ^= 1; }
         }
@@ -320,6 +409,8 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
+        // Wide tiles: the second MMA only where the tile has columns past BN.
+        const bool two = WIDE && tile_coord<CG>(p, unit % num_tiles).n_valid > C::BN;
         for (int kb = kb_begin; kb < kb_end; ++kb) {
           if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
           tc_fence_after();
@@ -338,6 +429,14 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
             const uint32_t accum = (kb != kb_begin || kk != 0) ? 1u : 0u;
             if constexpr (CG == 1) umma_bf16(d_tmem, ad, bd, idesc, accum);
             else umma_bf16_pair(d_tmem, ad, bd, idesc, accum);
+            if constexpr (WIDE) {
+              if (two) {
+                const uint32_t b2 = b0 + C::B_REGION_BYTES;
+                const uint64_t bd2 = p.b_kmajor ? sdesc_sw128(b2 + kk * 32, 16, 1024)
+                                                : sdesc_sw128(b2 + kk * 2048, C::B_BOX_BYTES, 1024);
+                umma_bf16_pair(d_tmem + C::BN, ad, bd2, p.idesc2, accum);
+              }
+            }
           }
           if constexpr (CG == 1) umma_commit(&empty[stage]);
           else umma_commit_pair_mc(&empty[stage], 0x3);
@@ -346,7 +445,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         if (!ok) break;
         if constexpr (CG == 1) umma_commit(&tfull[acc]);
         else umma_commit_pair_mc(&tfull[acc], 0x3);
-        if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+        if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
       }
       if (!ok) {
         // Wait (bounded) for every MMA already issued before TMEM is freed.
@@ -387,39 +486,12 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         if (elected) bulk_wait_group_read<1>();
         named_barrier_sync(1, 128);
         uint8_t* stage_row = sEpi + buf * C::EPI_BUF_BYTES + row_local * 128;
-        if (p.out_f32) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(t_row + c * 32, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {  // 16-byte chunk j = 4 f32
-            uint4 w;
-            w.x = __float_as_uint(apply_act(__uint_as_float(r[4 * j + 0]), p.act));
-            w.y = __float_as_uint(apply_act(__uint_as_float(r[4 * j + 1]), p.act));
-            w.z = __float_as_uint(apply_act(__uint_as_float(r[4 * j + 2]), p.act));
-            w.w = __float_as_uint(apply_act(__uint_as_float(r[4 * j + 3]), p.act));
-            *reinterpret_cast<uint4*>(stage_row + ((j ^ (row_local & 7)) << 4)) = w;
-          }
-        } else {
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(t_row + c * 64 + h * 32, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {  // 16-byte chunk 4h+j = 8 bf16
-              uint4 w;
-              w.x = pack_bf16x2(apply_act(__uint_as_float(r[8 * j + 0]), p.act),
-                                apply_act(__uint_as_float(r[8 * j + 1]), p.act));
-              w.y = pack_bf16x2(apply_act(__uint_as_float(r[8 * j + 2]), p.act),
-                                apply_act(__uint_as_float(r[8 * j + 3]), p.act));
-              w.z = pack_bf16x2(apply_act(__uint_as_float(r[8 * j + 4]), p.act),
-                                apply_act(__uint_as_float(r[8 * j + 5]), p.act));
-              w.w = pack_bf16x2(apply_act(__uint_as_float(r[8 * j + 6]), p.act),
-                                apply_act(__uint_as_float(r[8 * j + 7]), p.act));
-              *reinterpret_cast<uint4*>(stage_row + (((4 * h + j) ^ (row_local & 7)) << 4)) = w;
-            }
-          }
+        const uint32_t taddr = t_row + c * (p.out_f32 ? 32 : 64);
+        switch (p.act) {  // uniform: one branch per chunk
+          case ACT_GELU_TANH: epi_chunk<ACT_GELU_TANH>(p.out_f32, taddr, stage_row, row_local); break;
+          case ACT_GELU_ERF: epi_chunk<ACT_GELU_ERF>(p.out_f32, taddr, stage_row, row_local); break;
+          case ACT_RELU: epi_chunk<ACT_RELU>(p.out_f32, taddr, stage_row, row_local); break;
+          default: epi_chunk<ACT_NONE>(p.out_f32, taddr, stage_row, row_local); break;
         }
         if (c == nchunks - 1) {
           // Every accumulator column of this tile has been read: hand the
@@ -440,7 +512,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         }
         buf ^= 1;
       }
-      if (++acc == 2) { acc = 0; acc_phase ^= 1; }
+      if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
     }
     if (elected) bulk_wait_group_all();
   }

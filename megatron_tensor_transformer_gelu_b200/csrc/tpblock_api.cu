@@ -43,6 +43,7 @@ struct DeviceInfo {
 
 std::mutex g_mu;
 DeviceInfo g_dev[MAX_DEVICES];
+int g_force_tile_n = 0;  // tp_set_gemm_tile_n: 0 = cost model
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 // ------------------------------------------------------------ event timing
@@ -100,6 +101,8 @@ int device_ready(DeviceInfo** out) {
                                tp::GemmCfg<1>::SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(tp::gemm_tcgen05_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                tp::GemmCfg<2>::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(tp::gemm_tcgen05_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tp::GemmCfg<2, true>::SMEM_BYTES) != cudaSuccess ||
           cudaFuncSetAttribute(tp::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                tp::attn::SMEM_BYTES) != cudaSuccess)
         d.ok = false;
@@ -170,45 +173,96 @@ bool tmap_out(CUtensorMap* m, void* base, int f32, long long cols, long long row
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA; }
 
-// Number of K splits for `tiles` output tiles on `slots` persistent clusters,
-// from a small cost model: the main loop costs (waves x k-blocks per unit) k-
-// block times (about 0.5 us each for a 256 x 256 x 64 pair step), and every
-// extra f32 partial slot costs one write and one read of M x N x 4 bytes at
-// HBM speed (the reduce + LayerNorm kernel adds the slots).
-int choose_splits(long long tiles, int slots, int k_blocks, int max_splits, long long out_elems) {
-  const double t_kb = 0.48e-6;
+// Tile plan of a tensor-core GEMM: tile width (256, or 288..512 for wide
+// tiles) and number of K splits, from a small cost model of a persistent
+// launch on `slots` SM pairs, calibrated by timing these kernels on B200
+// under its power cap:
+//  * Main loop: waves x k-blocks per unit x the time of one k-block, about
+//    0.40 us for a 256 x 256 x 64 pair step.  A w-column tile does w/256 of
+//    that MMA work, at a lower time per MAC because every operand byte feeds
+//    more MACs (the main loop is bound by operand traffic from L2): relative
+//    time per MAC 1.0 at w = 256, 0.95 at 384, 0.88 at 448, 0.82 at 480 and
+//    0.78 at 512 (linear in between).
+//  * Every extra f32 partial slot of a K split costs one write and one read of
+//    M x N x 4 bytes at HBM speed (the reduce + LayerNorm kernel adds slots).
+//  * A wide tile fills TMEM, so its epilogue no longer overlaps the next
+//    tile's main loop: each wave but the last pays it (about 3.5 us per 256
+//    columns).
+struct TilePlan {
+  int tile_n = 256;
+  int splits = 1;
+};
+
+constexpr double T_KB = 0.40e-6;
+constexpr double T_EPI_256 = 3.5e-6;
+
+double per_mac_factor(int w) {
+  static const int xs[] = {256, 384, 448, 480, 512};
+  static const double ys[] = {1.0, 0.95, 0.88, 0.82, 0.78};
+  if (w <= xs[0]) return ys[0];
+  for (int i = 1; i < 5; ++i)
+    if (w <= xs[i]) return ys[i - 1] + (ys[i] - ys[i - 1]) * (w - xs[i - 1]) / double(xs[i] - xs[i - 1]);
+  return ys[4];
+}
+
+double kb_cost(int w) { return (w / 256.0) * per_mac_factor(w); }
+
+long long n_blocks_for(const tp::GemmArgs& p, int w) {
+  const long long per_shard = (p.shard_n + w - 1) / w;
+  return p.row_mode ? per_shard : per_shard * p.t;
+}
+
+TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits) {
+  TilePlan best;
+  const long long m_blocks = (p.M + (pair ? 255 : 127)) / (pair ? 256 : 128);
+  const long long out_elems = static_cast<long long>(p.M) * (p.row_mode ? p.shard_n : p.shard_n * p.t);
   const double slot_cost = static_cast<double>(out_elems) * 8.0 / 6.0e12;
-  int best = 1;
+  const long long tiles = m_blocks * n_blocks_for(p, 256);
   double best_t = 1e30;
-  for (int s = 1; s <= max_splits && s <= k_blocks; ++s) {
-    const long long units = tiles * s;
-    const long long waves = (units + slots - 1) / slots;
-    const long long kb = (k_blocks + s - 1) / s;
-    const double t = static_cast<double>(waves * kb) * t_kb + (s - 1) * slot_cost;
+  for (int s = 1; s <= max_splits && s <= p.k_blocks; ++s) {
+    const long long waves = (tiles * s + slots - 1) / slots;
+    const long long kb = (p.k_blocks + s - 1) / s;
+    const double t = static_cast<double>(waves * kb) * T_KB + (s - 1) * slot_cost;
     if (t < best_t * 0.98) {  // a split must buy at least 2%
       best_t = t;
-      best = s;
+      best.splits = s;
+    }
+  }
+  const int step = p.out_f32 ? 32 : 64;  // a 128-byte output chunk must not cross a tile edge
+  if (g_force_tile_n) {
+    if (!pair) return best;
+    best.splits = 1;
+    best.tile_n = (g_force_tile_n + step - 1) / step * step;
+    if (best.tile_n > 512) best.tile_n = 512;
+    return best;
+  }
+  if (!pair) return best;
+  for (int w = 256 + step; w <= 512; w += step) {
+    const long long wt = m_blocks * n_blocks_for(p, w);
+    const long long waves = (wt + slots - 1) / slots;
+    const double t = static_cast<double>(waves * p.k_blocks) * kb_cost(w) * T_KB +
+                     static_cast<double>(waves - 1) * (w / 256.0) * T_EPI_256;
+    if (t < best_t * 0.97) {  // wide tiles must buy at least 3%
+      best_t = t;
+      best.tile_n = w;
+      best.splits = 1;
     }
   }
   return best;
 }
 
-template <int CG>
-int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, int max_splits, cudaStream_t st) {
-  using C = tp::GemmCfg<CG>;
+template <int CG, bool WIDE>
+int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, const TilePlan& plan, cudaStream_t st) {
+  using C = tp::GemmCfg<CG, WIDE>;
   p.m_blocks = ceil_div(p.M, C::TILE_M);
-  if (p.row_mode) {
-    p.n_blocks = ceil_div(p.shard_n, C::BN);
-    p.n_blocks_per_shard = p.n_blocks;
-  } else {
-    p.n_blocks_per_shard = ceil_div(p.shard_n, C::BN);
-    p.n_blocks = p.n_blocks_per_shard * p.t;
-  }
+  p.tile_n = plan.tile_n;
+  p.n2 = WIDE ? plan.tile_n - C::BN : 0;
+  p.idesc2 = WIDE ? tp::idesc_bf16_f32(C::TILE_M, p.n2, false, !p.b_kmajor) : 0u;
+  p.n_blocks_per_shard = ceil_div(p.shard_n, p.tile_n);
+  p.n_blocks = p.row_mode ? p.n_blocks_per_shard : p.n_blocks_per_shard * p.t;
   const long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks;
   const int slots = CG == 2 ? dev.max_pairs : dev.sm_count;
-  p.splits = max_splits > 1
-                 ? choose_splits(tiles, slots, p.k_blocks, max_splits, static_cast<long long>(p.M) * p.shard_n)
-                 : 1;
+  p.splits = plan.splits;
   const long long es = p.out_f32 ? 4 : 2;
   if (p.row_mode) {
     if (!tmap_out(&p.tmC[0], p.C, p.out_f32, p.shard_n, p.M, p.splits, p.ldc, p.slot_stride)) return TP_ERR_CUDA;
@@ -233,7 +287,7 @@ int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, int max_splits, cudaS
   cfg.attrs = at;
   cfg.numAttrs = CG == 2 ? 1 : 0;
   ProfScope ps(K_GEMM_TC, st);
-  if (cudaLaunchKernelEx(&cfg, tp::gemm_tcgen05_kernel<CG>, p) != cudaSuccess) return TP_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, tp::gemm_tcgen05_kernel<CG, WIDE>, p) != cudaSuccess) return TP_ERR_CUDA;
   return launch_status();
 }
 
@@ -281,7 +335,11 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
   p.slot_stride = slot_stride;
   p.b_kmajor = b_kmajor;
   if (!out_f32) max_splits = 1;
-  const int r = pair ? launch_gemm_tc<2>(dev, p, max_splits, st) : launch_gemm_tc<1>(dev, p, max_splits, st);
+  const TilePlan plan = plan_tiles(p, pair, pair ? dev.max_pairs : dev.sm_count, max_splits);
+  int r;
+  if (!pair) r = launch_gemm_tc<1, false>(dev, p, plan, st);
+  else if (plan.tile_n > tp::GemmCfg<2>::BN) r = launch_gemm_tc<2, true>(dev, p, plan, st);
+  else r = launch_gemm_tc<2, false>(dev, p, plan, st);
   if (splits_out) *splits_out = p.splits;
   return r;
 }
@@ -708,6 +766,14 @@ int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts, c
   if (st != TP_OK) return st;
   return run_reduce_ln(S, H, nparts, parts, X, x_dtype == TP_DTYPE_BF16, gamma, beta, eps, Y,
                        out_dtype == TP_DTYPE_BF16, static_cast<cudaStream_t>(stream), dev->sm_count);
+}
+
+// ------------------------------------------------------------- GEMM tiling
+int tp_set_gemm_tile_n(int tile_n) {
+  if (tile_n != 0 && (tile_n < 256 || tile_n > 512 || tile_n % 32 != 0)) return TP_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_force_tile_n = tile_n;
+  return TP_OK;
 }
 
 // ------------------------------------------------------------- self-test

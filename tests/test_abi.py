@@ -139,6 +139,16 @@ def test_linear_and_layernorm_argument_checks(lib):
                                             ctypes.c_void_p(FAKE), 1, None) == INVALID
 
 
+def test_gemm_tile_override_checks(lib):
+    try:
+        for bad in (-32, 100, 224, 300, 544):
+            assert lib.tp_set_gemm_tile_n(bad) == INVALID
+        for good in (256, 288, 480, 512, 0):
+            assert lib.tp_set_gemm_tile_n(good) == OK
+    finally:
+        lib.tp_set_gemm_tile_n(0)
+
+
 def test_weight_layout_argument_checks(lib):
     pw, kw = _ptrs(2)
     X, Y = ctypes.c_void_p(FAKE), ctypes.c_void_p(FAKE)

@@ -18,7 +18,8 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  Layout     Row-major everywhere.  Weights use the pages' [in, out] layout
- *             (Y = X W with X [seq, H], W [H, N]; [PWWT] §1.1).
+ *             (Y = X W with X [seq, H], W [H, N]; [PWWT] §1.1); the `_ex`
+ *             entry points also take nn.Linear's [out, in] (TP_W_OUT_IN).
  *  Shards     Each shard is its own contiguous device buffer, as the pages'
  *             weight chunking makes one ([PWWT] §3.1).  `*_shards` arguments
  *             are HOST arrays of t DEVICE pointers.  1 <= t <= TP_MAX_SHARDS.

@@ -29,6 +29,12 @@ Readings where the pages are silent or garbled (each is listed in the design doc):
   * Attention: per head, softmax(Q K^T / sqrt(d)) V, non-causal, no mask,
     max-subtracted softmax; heads concatenated in head order, then O W_O.
   * No biases, no dropout.
+  * Backward pass: the pages give no formulas, only that each shard computes
+    the gradient of its own weight block ("TP到底在切什么" §4, weight
+    gradients split like the weights) and that the two split directions
+    differ in backward ("张量并行：千亿大模型突破单卡显存限制的底层技术" §2.2).
+    The oracle is the gradient of the forward definition above by the chain
+    rule, for a given upstream gradient dY (the vector-Jacobian product).
 
 Parity status: every function below is pinned by tests/test_oracle_pins.py
 (brute force on exact small inputs, closed forms, invariants, library
@@ -46,6 +52,7 @@ __all__ = [
     "layernorm", "mlp_block", "mlp_block_sharded",
     "linear_column", "linear_row",
     "attention_heads", "attention_sublayer", "attention_out", "mlp_out", "transformer_block",
+    "activation_grad", "layernorm_backward", "mlp_block_backward",
 ]
 
 _COL_BLOCK = 2048  # output-column block for products whose fp64 weight copy is large
@@ -237,3 +244,71 @@ def attention_sublayer(X, Wqkv, Wo, nh: int, d: int, gamma=None, beta=None,
     O = attention_heads(Q, K, V, nh, d)
     Z = Xr + _matmul_cols(O, Wo)
     return layernorm(Z, gamma, beta, eps)
+
+
+# ------------------------------------------------------------- backward pass
+# The gradient of the post-LN MLP sublayer for an upstream gradient dY, by the
+# chain rule through the forward steps of mlp_block:
+#   U = X A, G = Act(U), V = G B, Z = X + V, Y = LN(Z)
+# Column-splitting A and row-splitting B split the weight gradients the same
+# way ("TP到底在切什么" §4: each shard computes the gradient of its own block of
+# W): dA = X^T dU gives dA_i = X^T dU_i (the columns of shard i), and
+# dB = G^T dZ gives dB_i = G_i^T dZ (the rows of shard i); dX sums the row
+# split's contributions, dX = dZ + sum_i dU_i A_i^T.
+
+def activation_grad(u: np.ndarray, act: str) -> np.ndarray:
+    """d Act(u) / du, elementwise.  ReLU's derivative at 0 is taken as 0."""
+    if act == "gelu_tanh":
+        c = math.sqrt(2.0 / math.pi)
+        t = np.tanh(c * (u + 0.044715 * u * u * u))
+        return 0.5 * (1.0 + t) + 0.5 * u * (1.0 - t * t) * c * (1.0 + 3.0 * 0.044715 * u * u)
+    if act == "gelu_erf":
+        return 0.5 * (1.0 + _erf(u / math.sqrt(2.0))) + u * np.exp(-0.5 * u * u) / math.sqrt(2.0 * math.pi)
+    if act == "relu":
+        return (u > 0.0).astype(np.float64)
+    if act == "none":
+        return np.ones_like(u)
+    raise KeyError(act)
+
+
+def layernorm_backward(Z, dY, gamma=None, eps: float = 1e-5):
+    """(dZ, dgamma, dbeta) of Y = (Z - mean) / sqrt(var + eps) * gamma + beta
+    (biased variance over the last axis).  With xh the normalised row, r the
+    reciprocal standard deviation and g = dY * gamma:
+        dZ = r * (g - mean(g) - xh * mean(g * xh)),
+        dgamma = sum over rows of dY * xh,  dbeta = sum over rows of dY."""
+    Z = np.asarray(Z, dtype=np.float64)
+    dY = _f64(dY)
+    H = Z.shape[-1]
+    mean = Z.sum(axis=-1, keepdims=True) / H
+    D = Z - mean
+    var = (D * D).sum(axis=-1, keepdims=True) / H
+    r = 1.0 / np.sqrt(var + eps)
+    xh = D * r
+    g = dY * _f64(gamma) if gamma is not None else dY
+    dZ = r * (g - g.sum(axis=-1, keepdims=True) / H - xh * ((g * xh).sum(axis=-1, keepdims=True) / H))
+    return dZ, (dY * xh).sum(axis=0), dY.sum(axis=0)
+
+
+def mlp_block_backward(X, A, B, dY, gamma=None, beta=None, eps: float = 1e-5,
+                       act: str = "gelu_tanh") -> dict:
+    """Gradients of mlp_block's output Y with respect to X, A, B, gamma and
+    beta, contracted with dY: {"dX", "dA", "dB", "dgamma", "dbeta"}.  beta
+    does not enter any gradient but its own (dbeta = column sums of dY)."""
+    del beta
+    X64 = _f64(X)
+    A64 = _f64(A)
+    B64 = _f64(B)
+    U = X64 @ A64                          # forward, step 1
+    G = activation(U, act)                 # step 2
+    Z = X64 + G @ B64                      # steps 3-4
+    dZ, dgamma, dbeta = layernorm_backward(Z, dY, gamma, eps)   # through step 5
+    dG = dZ @ B64.T                        # through step 3 (V = G B)
+    dU = dG * activation_grad(U, act)      # through step 2
+    return {
+        "dX": dZ + dU @ A64.T,             # residual path + through step 1
+        "dA": X64.T @ dU,
+        "dB": G.T @ dZ,
+        "dgamma": dgamma,
+        "dbeta": dbeta,
+    }

@@ -259,12 +259,99 @@ def check_block_composition():
                                pre[rows], atol=1e-12)
 
 
+# ------------------------------------------------------------ backward pass
+
+def _backward_case(S, H, F, seed):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((S, H))
+    A = rng.standard_normal((H, F)) / math.sqrt(H)
+    B = rng.standard_normal((F, H)) / math.sqrt(F)
+    g = 1.0 + 0.5 * rng.standard_normal(H)
+    b = 0.3 * rng.standard_normal(H)
+    dY = rng.standard_normal((S, H))
+    return X, A, B, g, b, dY
+
+
+def check_backward_finite_differences():
+    """Brute force: every gradient entry against a central difference of the
+    (separately pinned) forward, L = sum(dY * Y), on a tiny rectangular case."""
+    S, H, F = 3, 5, 7
+    h = 1e-5
+    for act in ("gelu_tanh", "gelu_erf", "relu", "none"):
+        X, A, B, g, b, dY = _backward_case(S, H, F, seed=len(act))
+        assert np.abs(X @ A).min() > 1e-3  # keep ReLU away from its kink
+        grads = O.mlp_block_backward(X, A, B, dY, g, b, act=act)
+        params = {"dX": X, "dA": A, "dB": B, "dgamma": g, "dbeta": b}
+
+        def loss():
+            return float((dY * O.mlp_block(X, A, B, g, b, act=act)).sum())
+
+        for key, P in params.items():
+            assert grads[key].shape == P.shape, key
+            for idx in np.ndindex(*P.shape):
+                old = P[idx]
+                P[idx] = old + h
+                lp = loss()
+                P[idx] = old - h
+                lm = loss()
+                P[idx] = old
+                fd = (lp - lm) / (2 * h)
+                assert abs(fd - grads[key][idx]) <= 1e-7 * max(1.0, abs(fd)), (act, key, idx, fd, grads[key][idx])
+
+
+def check_backward_autograd():
+    """Library route: torch autograd (fp64) through torch's own layer_norm and
+    GeLU/ReLU gives the same gradients."""
+    S, H, F = 6, 8, 12
+    fns = {"gelu_tanh": lambda u: torch.nn.functional.gelu(u, approximate="tanh"),
+           "gelu_erf": lambda u: torch.nn.functional.gelu(u), "relu": torch.relu, "none": lambda u: u}
+    for act, fn in fns.items():
+        X, A, B, g, b, dY = _backward_case(S, H, F, seed=7 + len(act))
+        ts = [torch.tensor(v, dtype=torch.float64, requires_grad=True) for v in (X, A, B, g, b)]
+        Xt, At, Bt, gt, bt = ts
+        Y = torch.nn.functional.layer_norm(Xt + fn(Xt @ At) @ Bt, (H,), gt, bt, eps=1e-5)
+        (Y * torch.tensor(dY)).sum().backward()
+        ref = O.mlp_block_backward(X, A, B, dY, g, b, act=act)
+        for key, t in zip(("dX", "dA", "dB", "dgamma", "dbeta"), ts):
+            np.testing.assert_allclose(ref[key], t.grad.numpy(), rtol=1e-10, atol=1e-12, err_msg=f"{act} {key}")
+
+
+def check_backward_invariants():
+    """LayerNorm's input gradient has zero row sums (shifting a row does not
+    change its normalisation); gamma = 0 blocks every gradient but dbeta's and
+    dgamma's; the shard-by-shard form (weight gradients split like the weights,
+    dX summed over the row split) equals the unsplit one."""
+    X, A, B, g, b, dY = _backward_case(5, 8, 16, seed=3)
+    Z = X + O.gelu_tanh(X @ A) @ B
+    dZ, dg, db = O.layernorm_backward(Z, dY, g)
+    np.testing.assert_allclose(dZ.sum(axis=1), 0.0, atol=1e-12)
+    np.testing.assert_allclose(db, dY.sum(axis=0), atol=1e-12)
+    z = O.mlp_block_backward(X, A, B, dY, np.zeros(8), b)
+    for key in ("dX", "dA", "dB"):
+        assert np.abs(z[key]).max() == 0.0, key
+    full = O.mlp_block_backward(X, A, B, dY, g, b)
+    t = 4
+    dZ, _, _ = O.layernorm_backward(Z, dY, g)
+    dX = dZ.copy()
+    for Ai, Bi in zip(np.split(A, t, axis=1), np.split(B, t, axis=0)):
+        Ui = X @ Ai
+        dUi = (dZ @ Bi.T) * O.activation_grad(Ui, "gelu_tanh")
+        dX += dUi @ Ai.T
+    np.testing.assert_allclose(dX, full["dX"], atol=1e-12)
+    for i, (Ai, Bi) in enumerate(zip(np.split(A, t, axis=1), np.split(B, t, axis=0))):
+        Ui = X @ Ai
+        dUi = (dZ @ Bi.T) * O.activation_grad(Ui, "gelu_tanh")
+        np.testing.assert_allclose(X.T @ dUi, full["dA"][:, i * 4:(i + 1) * 4], atol=1e-12)
+        np.testing.assert_allclose(O.gelu_tanh(Ui).T @ dZ, full["dB"][i * 4:(i + 1) * 4], atol=1e-12)
+
+
 ALL_CHECKS = [
     check_gelu_library, check_gelu_identities, check_layernorm_hand, check_layernorm_invariants,
     check_mlp_exact_bruteforce, check_mlp_closed_forms, check_mlp_block_identities,
     check_mlp_symmetries, check_linears_exact, check_attention_hand,
     check_attention_uniform_keys, check_attention_library, check_attention_row_equivariance,
-    check_block_composition,
+    check_block_composition, check_backward_finite_differences, check_backward_autograd,
+    check_backward_invariants,
 ]
 
 
@@ -354,6 +441,38 @@ def _bad_attention_wrong_head_cols(X, Wqkv, Wo, nh, d, gamma=None, beta=None, ep
     return O.layernorm(Xr + Oo @ O._f64(Wo), gamma, beta, eps)
 
 
+def _bad_layernorm_backward_no_projection(Z, dY, gamma=None, eps=1e-5):
+    Z = np.asarray(Z, dtype=np.float64)
+    dY = O._f64(dY)
+    H = Z.shape[-1]
+    D = Z - Z.mean(axis=-1, keepdims=True)
+    r = 1.0 / np.sqrt((D * D).mean(axis=-1, keepdims=True) + eps)
+    g = dY * O._f64(gamma) if gamma is not None else dY
+    return r * (g - g.sum(axis=-1, keepdims=True) / H), (dY * D * r).sum(axis=0), dY.sum(axis=0)
+
+
+def _bad_activation_grad_is_activation(u, act):
+    return O.activation(u, act)
+
+
+def _bad_backward_no_residual(X, A, B, dY, gamma=None, beta=None, eps=1e-5, act="gelu_tanh"):
+    X64, A64, B64 = O._f64(X), O._f64(A), O._f64(B)
+    U = X64 @ A64
+    G = O.activation(U, act)
+    dZ, dg, db = O.layernorm_backward(X64 + G @ B64, dY, gamma, eps)
+    dU = (dZ @ B64.T) * O.activation_grad(U, act)
+    return {"dX": dU @ A64.T, "dA": X64.T @ dU, "dB": G.T @ dZ, "dgamma": dg, "dbeta": db}
+
+
+def _bad_backward_db_from_u(X, A, B, dY, gamma=None, beta=None, eps=1e-5, act="gelu_tanh"):
+    X64, A64, B64 = O._f64(X), O._f64(A), O._f64(B)
+    U = X64 @ A64
+    G = O.activation(U, act)
+    dZ, dg, db = O.layernorm_backward(X64 + G @ B64, dY, gamma, eps)
+    dU = (dZ @ B64.T) * O.activation_grad(U, act)
+    return {"dX": dZ + dU @ A64.T, "dA": X64.T @ dU, "dB": U.T @ dZ, "dgamma": dg, "dbeta": db}
+
+
 _PLANTED = [
     ("layernorm", _bad_layernorm_unbiased),
     ("layernorm", _bad_layernorm_eps_outside),
@@ -364,6 +483,10 @@ _PLANTED = [
     ("attention_heads", _bad_attention_no_scale),
     ("attention_heads", _bad_attention_softmax_axis),
     ("attention_sublayer", _bad_attention_wrong_head_cols),
+    ("layernorm_backward", _bad_layernorm_backward_no_projection),
+    ("activation_grad", _bad_activation_grad_is_activation),
+    ("mlp_block_backward", _bad_backward_no_residual),
+    ("mlp_block_backward", _bad_backward_db_from_u),
 ]
 
 

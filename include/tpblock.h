@@ -126,6 +126,40 @@ int tp_mlp_forward_ex(int S, int H, int F, int t, int dtype, int out_dtype, int 
                       const float* gamma, const float* beta, float eps, int act,
                       void* Y, void* workspace, size_t workspace_bytes, void* stream);
 
+/* -------------------------------------------------- MLP training step ----
+ * Backward pass of the MLP sublayer (post-LN, [in, out] weights, bf16).  The
+ * pages give no backward formulas, only that each shard computes the gradient
+ * of its own weight block ([PWWT] §4) and that the two split directions differ
+ * in backward ([TYPC] §2.2); what is computed is the chain rule through
+ *   U = X A, G = Act(U), V = G B, Z = X + V, Y = LN(Z):
+ *   dZ = LayerNorm backward of dY;  dU_i = (dZ B_i^T) * Act'(U_i);
+ *   dX = dZ + sum_i dU_i A_i^T;  dA_i = X^T dU_i;  dB_i = G_i^T dZ;
+ *   dgamma = sum_rows dY * (Z - mean) / sqrt(var + eps);  dbeta = sum_rows dY.
+ *
+ * tp_mlp_forward_train: tp_mlp_forward (dtype bf16 only) that also keeps, in
+ * the caller's `state` (>= tp_mlp_train_state_bytes()), what the backward
+ * reads: U [S, F] bf16 (pre-activation), G [S, F] bf16 and V [S, H] f32.
+ * Y is the same as tp_mlp_forward's up to rounding.
+ *
+ * tp_mlp_backward: from the same X, shards, gamma, eps, act and the state of
+ * one tp_mlp_forward_train call, and the upstream gradient dY [S, H] bf16,
+ * writes dX [S, H] bf16, dA_shards[i] [H, F/t] f32 and dB_shards[i] [F/t, H]
+ * f32 (the gradients of shard i's weights, same layout as the weights),
+ * dgamma and dbeta [H] f32 (either may be NULL).  workspace >=
+ * tp_mlp_backward_workspace_bytes().  S == 0 writes nothing.  Shapes as
+ * tp_mlp_forward. */
+size_t tp_mlp_train_state_bytes(int S, int H, int F, int t, int dtype);
+int tp_mlp_forward_train(int S, int H, int F, int t, int dtype, int out_dtype, const void* X,
+                         const void* const* A_shards, const void* const* B_shards,
+                         const float* gamma, const float* beta, float eps, int act,
+                         void* Y, void* state, size_t state_bytes, void* stream);
+size_t tp_mlp_backward_workspace_bytes(int S, int H, int F, int t, int dtype);
+int tp_mlp_backward(int S, int H, int F, int t, int dtype, const void* X,
+                    const void* const* A_shards, const void* const* B_shards,
+                    const float* gamma, float eps, int act, const void* state, size_t state_bytes,
+                    const void* dY, void* dX, void* const* dA_shards, void* const* dB_shards,
+                    float* dgamma, float* dbeta, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ------------------------------------------------- MLP without allocation ----
  * The pages have no counterpart to this entry point: it exists for callers
  * that cannot allocate device memory (plugin hosts that forbid allocation in
@@ -255,7 +289,7 @@ int tp_selftest_wait_timeout(long long limit_cycles, void* stream);
  * 16384 launches between two collects are bracketed by CUDA events recorded on
  * the launch's stream.  tp_profile_collect synchronises those events and
  * writes per kernel kind (0 tensor-core GEMM, 1 reduce+residual+LayerNorm,
- * 2 f32 CUDA-core GEMM, 3 attention): `launches` = all launches, `timed` = the
+ * 2 f32 CUDA-core GEMM, 3 attention, 4 LayerNorm backward): `launches` = all launches, `timed` = the
  * launches with events, `ms` = their summed device milliseconds; then it
  * clears the record.  Any output array may be NULL.  Returns the number of
  * kinds written (<= max_kinds), or -TP_ERR_CUDA.  Not thread-safe: enable,

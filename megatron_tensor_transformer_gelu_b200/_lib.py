@@ -48,6 +48,12 @@ SIGNATURES = {
                                                               _vp]),
     "tp_linear_row_forward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vp, _vp, _c_size, _vp]),
     "tp_reduce_residual_layernorm": (_c_int, [_c_int] * 3 + [_vp, _vp, _c_int, _vp, _vp, _c_float, _vp, _c_int, _vp]),
+    "tp_mlp_train_state_bytes": (_c_size, [_c_int] * 5),
+    "tp_mlp_forward_train": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vpp, _vp, _vp, _c_float, _c_int, _vp, _vp, _c_size,
+                                                      _vp]),
+    "tp_mlp_backward_workspace_bytes": (_c_size, [_c_int] * 5),
+    "tp_mlp_backward": (_c_int, [_c_int] * 5 + [_vp, _vpp, _vpp, _vp, _c_float, _c_int, _vp, _c_size, _vp, _vp, _vpp,
+                                                 _vpp, _vp, _vp, _vp, _c_size, _vp]),
     "tp_set_gemm_tile_n": (_c_int, [_c_int]),
     "tp_selftest_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
     "tp_profile_enable": (_c_int, [_c_int]),
@@ -209,6 +215,43 @@ def reduce_residual_layernorm(parts, X, Y, gamma=None, beta=None, eps=1e-5, stre
     _check(code, "tp_reduce_residual_layernorm")
 
 
+def mlp_train_state_bytes(S, H, F, t, dtype=torch.bfloat16) -> int:
+    return int(lib().tp_mlp_train_state_bytes(S, H, F, t, DTYPE[dtype]))
+
+
+def mlp_backward_workspace_bytes(S, H, F, t, dtype=torch.bfloat16) -> int:
+    return int(lib().tp_mlp_backward_workspace_bytes(S, H, F, t, DTYPE[dtype]))
+
+
+def mlp_forward_train(X, A_shards, B_shards, Y, state, gamma=None, beta=None, eps=1e-5, act="gelu_tanh",
+                      stream=None):
+    S, H = X.shape
+    t = len(A_shards)
+    F = sum(a.shape[1] for a in A_shards)
+    pa, ka = _ptrs(A_shards)
+    pb, kb = _ptrs(B_shards)
+    code = lib().tp_mlp_forward_train(S, H, F, t, DTYPE[X.dtype], DTYPE[Y.dtype], _ptr(X), pa, pb, _ptr(gamma),
+                                      _ptr(beta), float(eps), ACT[act], _ptr(Y), _ptr(state),
+                                      state.numel() * state.element_size(), _stream(stream))
+    _check(code, "tp_mlp_forward_train")
+
+
+def mlp_backward(X, A_shards, B_shards, state, dY, dX, dA_shards, dB_shards, workspace, gamma=None, dgamma=None,
+                 dbeta=None, eps=1e-5, act="gelu_tanh", stream=None):
+    S, H = X.shape
+    t = len(A_shards)
+    F = sum(a.shape[1] for a in A_shards)
+    pa, ka = _ptrs(A_shards)
+    pb, kb = _ptrs(B_shards)
+    pda, kda = _ptrs(dA_shards)
+    pdb, kdb = _ptrs(dB_shards)
+    code = lib().tp_mlp_backward(S, H, F, t, DTYPE[X.dtype], _ptr(X), pa, pb, _ptr(gamma), float(eps), ACT[act],
+                                 _ptr(state), state.numel() * state.element_size(), _ptr(dY), _ptr(dX), pda, pdb,
+                                 _ptr(dgamma), _ptr(dbeta), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(code, "tp_mlp_backward")
+
+
 def set_gemm_tile_n(tile_n: int) -> None:
     """0: the library's cost model picks GEMM tiles; 256..512: force that tile width."""
     _check(lib().tp_set_gemm_tile_n(int(tile_n)), "tp_set_gemm_tile_n")
@@ -226,7 +269,7 @@ def profile_enable(on: bool):
     _check(lib().tp_profile_enable(1 if on else 0), "tp_profile_enable")
 
 
-def profile_collect(nkinds: int = 4):
+def profile_collect(nkinds: int = 5):
     """{kernel kind: (launches, timed launches, summed ms of the timed ones)}"""
     launches = (ctypes.c_int * nkinds)()
     timed = (ctypes.c_int * nkinds)()

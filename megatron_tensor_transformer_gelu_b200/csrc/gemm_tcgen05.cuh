@@ -114,7 +114,20 @@ struct GemmArgs {
   int tile_n;                    // columns per tile: BN, or up to 2*BN for wide tiles
   int n2;                        // wide tiles: N of the second MMA (tile_n - BN), else 0
   uint32_t idesc2;               // wide tiles: instruction descriptor of the second MMA
+  // A given M-major: the stored matrix is [K, M] (A^T of a row-major [M, K]),
+  // loaded as two 64 x 64 boxes per CTA and read through an MN-major descriptor.
+  int a_mnmajor;
+  // Epilogue mode.  EPI_PLAIN: C = Act(acc).  EPI_AUX_PRE: also stores the
+  // pre-activation acc (bf16) through tmAux (same tiling as C).  EPI_GRAD: bf16
+  // C = acc * Act'(U), with U read from `aux` (bf16, row stride ld_aux, same
+  // columns as C) — the backward of the activation fused into the GEMM.
+  int epi_mode;
+  CUtensorMap tmAux[MAX_SHARDS];
+  const void* aux;
+  long long ld_aux;
 };
+
+enum : int { EPI_PLAIN = 0, EPI_AUX_PRE = 1, EPI_GRAD = 2 };
 
 __device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& kb0, int& kb1) {
   kb0 = static_cast<int>(static_cast<long long>(split) * p.k_blocks / p.splits);
@@ -142,6 +155,66 @@ __device__ __forceinline__ float act_t(float u) {
     return fmaxf(u, 0.0f);
   } else {
     return u;
+  }
+}
+
+// d Act(u) / du for the backward epilogue (ReLU's derivative at 0 is 0).
+template <int ACT>
+__device__ __forceinline__ float act_grad_t(float u) {
+  if constexpr (ACT == ACT_GELU_TANH) {
+    const float k0 = 0.7978845608028654f;  // sqrt(2/pi)
+    const float t = tanh_fast(k0 * fmaf(0.044715f * u, u * u, u));
+    return 0.5f * (1.0f + t) + 0.5f * u * (1.0f - t * t) * k0 * fmaf(3.0f * 0.044715f, u * u, 1.0f);
+  } else if constexpr (ACT == ACT_GELU_ERF) {
+    return 0.5f * (1.0f + erff(u * 0.7071067811865476f)) + u * 0.3989422804014327f * __expf(-0.5f * u * u);
+  } else if constexpr (ACT == ACT_RELU) {
+    return u > 0.0f ? 1.0f : 0.0f;
+  } else {
+    return 1.0f;
+  }
+}
+
+// Backward epilogue chunk (bf16 out, 64 columns): acc * Act'(U) with this
+// thread's U values read from global memory, 32 at a time (columns past
+// `nvalid` and rows past M read nothing and use U = 0).
+template <int ACT>
+__device__ __forceinline__ void epi_chunk_grad(uint32_t taddr, uint8_t* stage_row, int row_local,
+                                               const __nv_bfloat16* urow, int nvalid) {
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    float u[32];
+    const int nv = nvalid - 32 * h;
+    if (urow != nullptr && nv >= 32) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(urow + 32 * h) + j);
+        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(hv[e]);
+          u[8 * j + 2 * e] = f.x;
+          u[8 * j + 2 * e + 1] = f.y;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) u[j] = (urow != nullptr && j < nv) ? __bfloat162float(urow[32 * h + j]) : 0.0f;
+    }
+    uint32_t r[32];
+    tmem_ld_32x32b_x32(taddr + h * 32, r);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i0 = 8 * j + 2 * e;
+        w4[e] = pack_bf16x2(__uint_as_float(r[i0]) * act_grad_t<ACT>(u[i0]),
+                            __uint_as_float(r[i0 + 1]) * act_grad_t<ACT>(u[i0 + 1]));
+      }
+      *reinterpret_cast<uint4*>(stage_row + (((4 * h + j) ^ (row_local & 7)) << 4)) =
+          make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
   }
 }
 
@@ -241,6 +314,17 @@ __device__ __forceinline__ int b_boxes_for(int n_valid, int rank, int b_kmajor) 
   return min(C::B_BOXES, (cols + C::B_BOX_N - 1) / C::B_BOX_N);
 }
 
+// A bytes a CTA whose rows start at row0 brings into a stage: one 128 x 64
+// K-major box, or (M-major A) one 64 x 64 box per 64 rows that exist.
+__device__ __forceinline__ int a_mn_boxes(const GemmArgs& p, int row0) {
+  const int rows = p.M - row0;
+  return rows <= 0 ? 0 : (rows >= 128 ? 2 : (rows + 63) / 64);
+}
+__device__ __forceinline__ uint32_t a_bytes_for(const GemmArgs& p, int row0) {
+  if (p.a_mnmajor) return static_cast<uint32_t>(a_mn_boxes(p, row0)) * 8192u;
+  return row0 < p.M ? 16384u : 0u;
+}
+
 // Wide tiles: B boxes CTA `rank` loads for the second MMA, whose n2 columns
 // (tile columns [BN, BN + n2)) the pair splits in halves of n2/2.  Counted in
 // B_BOX_BYTES units; a K-major B is one box of up to B_COLS_CTA rows.
@@ -324,12 +408,12 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         const TileCoord tc = tile_coord<CG>(p, tile);
         const int my_row0 = tc.m0 + static_cast<int>(rank) * C::BM;
         const bool my_a = my_row0 < p.M;
+        const int my_aboxes = a_mn_boxes(p, my_row0);  // M-major A: 64-row boxes this CTA loads
         const int my_boxes = b_boxes_for<CG>(tc.n_valid, rank, p.b_kmajor);
         const int my_boxes2 = WIDE ? b2_boxes_for(tc.n_valid, p.n2, rank, p.b_kmajor) : 0;
         uint32_t bytes = 0;  // leader: bytes the whole tile stage brings in
         for (int r = 0; r < CG; ++r) {
-          bytes += (tc.m0 + r * C::BM < p.M ? C::A_BYTES : 0) +
-                   b_boxes_for<CG>(tc.n_valid, r, p.b_kmajor) * C::B_BOX_BYTES;
+          bytes += a_bytes_for(p, tc.m0 + r * C::BM) + b_boxes_for<CG>(tc.n_valid, r, p.b_kmajor) * C::B_BOX_BYTES;
           if constexpr (WIDE) bytes += b2_boxes_for(tc.n_valid, p.n2, r, p.b_kmajor) * C::B_BOX_BYTES;
         }
         const int b_x0 = tc.n_in + static_cast<int>(rank) * C::B_COLS_CTA;
@@ -337,7 +421,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         for (int kb = kb_begin; kb < kb_end; ++kb) {
           if constexpr (C::PREFETCH > 0) {
             const int kp = kb + C::PREFETCH;
-            if (kp < kb_end) {
+            if (kp < kb_end && !p.a_mnmajor) {
               int ps, pa, pb;
               kblock_coords(p, tc, kp, ps, pa, pb);
               if (my_a) tma_prefetch_l2_2d(&p.tmA, pa, my_row0);
@@ -352,7 +436,12 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
           if constexpr (CG == 1) {
             mbar_arrive_expect_tx(&full[stage], bytes);
             armed[stage] = static_cast<int>(phase);
-            tma_load_2d(dA, &p.tmA, a_x, my_row0, &full[stage]);
+            if (p.a_mnmajor) {
+              for (int j = 0; j < my_aboxes; ++j)
+                tma_load_2d(dA + j * C::B_BOX_BYTES, &p.tmA, my_row0 + j * 64, a_x, &full[stage]);
+            } else {
+              tma_load_2d(dA, &p.tmA, a_x, my_row0, &full[stage]);
+            }
             if (p.b_kmajor) {
               if (my_boxes) tma_load_2d(dB, &p.tmB[shard], b_y, b_x0, &full[stage]);
             } else {
@@ -365,7 +454,12 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
               mbar_arrive_expect_tx(&full[stage], bytes);
               armed[stage] = static_cast<int>(phase);
             }
-            if (my_a) tma_load_2d_pair(dA, &p.tmA, a_x, my_row0, bar);
+            if (p.a_mnmajor) {
+              for (int j = 0; j < my_aboxes; ++j)
+                tma_load_2d_pair(dA + j * C::B_BOX_BYTES, &p.tmA, my_row0 + j * 64, a_x, bar);
+            } else if (my_a) {
+              tma_load_2d_pair(dA, &p.tmA, a_x, my_row0, bar);
+            }
             if (p.b_kmajor) {
               if (my_boxes) tma_load_2d_pair(dB, &p.tmB[shard], b_y, b_x0, bar);
             } else {
@@ -416,11 +510,13 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
-          const uint32_t idesc = p.b_kmajor ? C::IDESC_BK : C::IDESC;
+          const uint32_t idesc = (p.b_kmajor ? C::IDESC_BK : C::IDESC) | (p.a_mnmajor ? (1u << 15) : 0u);
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk) {
-            // A: K-major, 16 k-elements = 32 bytes further along the swizzled row.
-            const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
+            // A K-major: 16 k-elements = 32 bytes further along the swizzled row.
+            // A M-major: like an N-major B (64-row chunks 8 KiB apart).
+            const uint64_t ad = p.a_mnmajor ? sdesc_sw128(a0 + kk * 2048, C::B_BOX_BYTES, 1024)
+                                            : sdesc_sw128(a0 + kk * 32, 16, 1024);
             // B N-major: 16 k-rows = 2 x (8 rows x 128 B) further; 64-column
             // chunks are B_BOX_BYTES apart (leading offset), 8-row groups 1 KiB.
             // B K-major: like A.
@@ -474,6 +570,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       const TileCoord tc = tile_coord<CG>(p, unit % num_tiles);
       const int split = unit / num_tiles;
       const CUtensorMap* tmC = &p.tmC[p.row_mode ? 0 : tc.shard];
+      const CUtensorMap* tmAux = &p.tmAux[p.row_mode ? 0 : tc.shard];
       const int y0 = tc.m0 + static_cast<int>(rank) * C::BM;
       // All 128 epilogue threads take the same decision (they meet at named
       // barriers below).
@@ -481,36 +578,57 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
       const int nchunks = (tc.n_valid + cw - 1) / cw;
+      const int parts = p.epi_mode == EPI_AUX_PRE ? 2 : 1;  // aux (pre-activation) store first
+      const int grow = y0 + row_local;
       for (int c = 0; c < nchunks; ++c) {
-        // The TMA store that last read this staging buffer must be done with it.
-        if (elected) bulk_wait_group_read<1>();
-        named_barrier_sync(1, 128);
-        uint8_t* stage_row = sEpi + buf * C::EPI_BUF_BYTES + row_local * 128;
-        const uint32_t taddr = t_row + c * (p.out_f32 ? 32 : 64);
-        switch (p.act) {  // uniform: one branch per chunk
-          case ACT_GELU_TANH: epi_chunk<ACT_GELU_TANH>(p.out_f32, taddr, stage_row, row_local); break;
-          case ACT_GELU_ERF: epi_chunk<ACT_GELU_ERF>(p.out_f32, taddr, stage_row, row_local); break;
-          case ACT_RELU: epi_chunk<ACT_RELU>(p.out_f32, taddr, stage_row, row_local); break;
-          default: epi_chunk<ACT_NONE>(p.out_f32, taddr, stage_row, row_local); break;
-        }
-        if (c == nchunks - 1) {
-          // Every accumulator column of this tile has been read: hand the
-          // TMEM buffer back to the MMA issuer before the last store.
-          tc_fence_before();
-          if constexpr (CG == 1) {
-            mbar_arrive(&tempty[acc]);
+        for (int part = 0; part < parts; ++part) {
+          // The TMA store that last read this staging buffer must be done with it.
+          if (elected) bulk_wait_group_read<1>();
+          named_barrier_sync(1, 128);
+          uint8_t* stage_row = sEpi + buf * C::EPI_BUF_BYTES + row_local * 128;
+          const uint32_t taddr = t_row + c * (p.out_f32 ? 32 : 64);
+          if (p.epi_mode == EPI_GRAD) {
+            const __nv_bfloat16* urow =
+                grow < p.M ? static_cast<const __nv_bfloat16*>(p.aux) + static_cast<long long>(grow) * p.ld_aux +
+                                 tc.out_col0 + c * 64
+                           : nullptr;
+            const int nvalid = tc.n_valid - c * 64;
+            switch (p.act) {  // uniform: one branch per chunk
+              case ACT_GELU_TANH: epi_chunk_grad<ACT_GELU_TANH>(taddr, stage_row, row_local, urow, nvalid); break;
+              case ACT_GELU_ERF: epi_chunk_grad<ACT_GELU_ERF>(taddr, stage_row, row_local, urow, nvalid); break;
+              case ACT_RELU: epi_chunk_grad<ACT_RELU>(taddr, stage_row, row_local, urow, nvalid); break;
+              default: epi_chunk_grad<ACT_NONE>(taddr, stage_row, row_local, urow, nvalid); break;
+            }
+          } else if (part < parts - 1) {
+            epi_chunk<ACT_NONE>(p.out_f32, taddr, stage_row, row_local);
           } else {
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(tempty_leader0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+            switch (p.act) {  // uniform: one branch per chunk
+              case ACT_GELU_TANH: epi_chunk<ACT_GELU_TANH>(p.out_f32, taddr, stage_row, row_local); break;
+              case ACT_GELU_ERF: epi_chunk<ACT_GELU_ERF>(p.out_f32, taddr, stage_row, row_local); break;
+              case ACT_RELU: epi_chunk<ACT_RELU>(p.out_f32, taddr, stage_row, row_local); break;
+              default: epi_chunk<ACT_NONE>(p.out_f32, taddr, stage_row, row_local); break;
+            }
           }
+          if (c == nchunks - 1 && part == parts - 1) {
+            // Every accumulator column of this tile has been read: hand the
+            // TMEM buffer back to the MMA issuer before the last store.
+            tc_fence_before();
+            if constexpr (CG == 1) {
+              mbar_arrive(&tempty[acc]);
+            } else {
+              __syncwarp();
+              if (lane == 0) mbar_arrive_cluster(tempty_leader0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+            }
+          }
+          fence_proxy_async_smem();
+          named_barrier_sync(1, 128);
+          if (elected && y0 < p.M) {
+            const CUtensorMap* map = part < parts - 1 ? tmAux : tmC;
+            tma_store_3d(map, sEpi + buf * C::EPI_BUF_BYTES, tc.n_in + c * cw, y0, split);
+            bulk_commit_group();
+          }
+          buf ^= 1;
         }
-        fence_proxy_async_smem();
-        named_barrier_sync(1, 128);
-        if (elected && y0 < p.M) {
-          tma_store_3d(tmC, sEpi + buf * C::EPI_BUF_BYTES, tc.n_in + c * cw, y0, split);
-          bulk_commit_group();
-        }
-        buf ^= 1;
       }
       if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
     }

@@ -1,0 +1,208 @@
+// Backward of the fused residual + LayerNorm, one row per CTA at a time:
+//
+//   forward   Z = X + sum_p V_p ;  Y = (Z - mean) * r * gamma + beta,  r = 1/sqrt(var + eps)
+//   backward  xh = (Z - mean) * r ;  g = dY * gamma
+//             dZ = r * (g - mean(g) - xh * mean(g * xh))
+//             dgamma = sum over rows of dY * xh ;  dbeta = sum over rows of dY
+//
+// Z and its statistics are recomputed from the forward's inputs (X and the f32
+// partial sums the row-split GEMM left), so the forward keeps no extra tensor.
+// The gradient of the weights of each shard stays with its shard
+// ("TP到底在切什么" §4); dgamma/dbeta are reduced over rows in a fixed order:
+// every CTA accumulates its rows' contributions per column in registers and
+// writes one partial row, and a second kernel adds the partial rows.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace tp {
+
+namespace lnb {
+constexpr int MAX_WARPS = 16;
+}
+
+struct LnBackArgs {
+  int S, H;
+  int nparts;
+  const float* parts;          // nparts x [S, H] f32, part_stride apart
+  long long part_stride;
+  const __nv_bfloat16* X;      // [S, H]
+  const __nv_bfloat16* dY;     // [S, H]
+  const float* gamma;          // [H] or null (= 1)
+  float eps;
+  __nv_bfloat16* dZ;           // [S, H]
+  float* partial;              // [gridDim.x][2][H]: per-CTA (dgamma, dbeta) sums
+};
+
+// Sum of v over the CTA (all threads get it), fixed order: warp shuffles, then
+// the warps' sums in warp order.
+__device__ __forceinline__ float lnb_block_sum(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  __syncthreads();  // red may still be read from the previous reduction
+  if ((threadIdx.x & 31) == 0) red[warp] = v;
+  __syncthreads();
+  float t = 0.0f;
+  for (int w = 0; w < nw; ++w) t += red[w];
+  return t;
+}
+
+__device__ __forceinline__ void lnb_block_sum2(float& a, float& b, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+  }
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) {
+    red[warp] = a;
+    red[lnb::MAX_WARPS + warp] = b;
+  }
+  __syncthreads();
+  float ta = 0.0f, tb = 0.0f;
+  for (int w = 0; w < nw; ++w) {
+    ta += red[w];
+    tb += red[lnb::MAX_WARPS + w];
+  }
+  a = ta;
+  b = tb;
+}
+
+// CH chunks of 8 consecutive elements per thread (CH = 1..4, up to 512
+// threads, so H <= 16384); chunk c of thread i covers elements
+// (c * blockDim.x + i) * 8 ...; chunks past H are masked.  dY is read twice
+// (the second time from cache) to keep registers for Z and the running
+// dgamma/dbeta column sums.
+__device__ __forceinline__ void lnb_load8_bf16(const __nv_bfloat16* src, float (&v)[8]) {
+  const uint4 w = *reinterpret_cast<const uint4*>(src);
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = __bfloat1622float2(h[e]);
+    v[2 * e] = f.x;
+    v[2 * e + 1] = f.y;
+  }
+}
+
+template <int CH>
+__global__ void __launch_bounds__(512) ln_backward_kernel(const LnBackArgs p) {
+  __shared__ float red[2 * lnb::MAX_WARPS];
+  const int nthr = blockDim.x;
+  float z[CH][8], dg[CH][8], db[CH][8];
+#pragma unroll
+  for (int c = 0; c < CH; ++c)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dg[c][e] = db[c][e] = 0.0f;
+  const float inv_h = 1.0f / static_cast<float>(p.H);
+
+  for (int row = blockIdx.x; row < p.S; row += gridDim.x) {
+    const long long base = static_cast<long long>(row) * p.H;
+    float s = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = (c * nthr + threadIdx.x) * 8;
+      if (col < p.H) {
+        lnb_load8_bf16(p.X + base + col, z[c]);
+        for (int q = 0; q < p.nparts; ++q) {
+          const float4* pp = reinterpret_cast<const float4*>(p.parts + q * p.part_stride + base + col);
+          const float4 a = __ldcs(pp), b = __ldcs(pp + 1);
+          z[c][0] += a.x; z[c][1] += a.y; z[c][2] += a.z; z[c][3] += a.w;
+          z[c][4] += b.x; z[c][5] += b.y; z[c][6] += b.z; z[c][7] += b.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s += z[c][e];
+      }
+    }
+    const float mean = lnb_block_sum(s, red) * inv_h;
+    float v = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = (c * nthr + threadIdx.x) * 8;
+      if (col < p.H) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float d = z[c][e] - mean;
+          v = fmaf(d, d, v);
+        }
+      }
+    }
+    const float var = lnb_block_sum(v, red) * inv_h;
+    const float r = rsqrtf(var + p.eps);
+    float sg = 0.0f, sgx = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = (c * nthr + threadIdx.x) * 8;
+      if (col < p.H) {
+        float dy[8];
+        lnb_load8_bf16(p.dY + base + col, dy);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float xh = (z[c][e] - mean) * r;
+          const float g = p.gamma ? dy[e] * __ldg(p.gamma + col + e) : dy[e];
+          z[c][e] = xh;  // z now holds the normalised row
+          sg += g;
+          sgx = fmaf(g, xh, sgx);
+          dg[c][e] = fmaf(dy[e], xh, dg[c][e]);
+          db[c][e] += dy[e];
+        }
+      }
+    }
+    lnb_block_sum2(sg, sgx, red);
+    const float mg = sg * inv_h, mgx = sgx * inv_h;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = (c * nthr + threadIdx.x) * 8;
+      if (col < p.H) {
+        float dy[8];
+        lnb_load8_bf16(p.dY + base + col, dy);
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float o[2];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const int i = 2 * e + k;
+            const float g = p.gamma ? dy[i] * __ldg(p.gamma + col + i) : dy[i];
+            o[k] = r * (g - mg - z[c][i] * mgx);
+          }
+          __nv_bfloat162 h = __floats2bfloat162_rn(o[0], o[1]);
+          w[e] = *reinterpret_cast<uint32_t*>(&h);
+        }
+        *reinterpret_cast<uint4*>(p.dZ + base + col) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+  }
+  // This CTA's per-column partial sums (zero where it had no rows).
+  float* out = p.partial + static_cast<long long>(blockIdx.x) * 2 * p.H;
+#pragma unroll
+  for (int c = 0; c < CH; ++c) {
+    const int col = (c * nthr + threadIdx.x) * 8;
+    if (col < p.H) {
+      float4* og = reinterpret_cast<float4*>(out + col);
+      float4* ob = reinterpret_cast<float4*>(out + p.H + col);
+      og[0] = make_float4(dg[c][0], dg[c][1], dg[c][2], dg[c][3]);
+      og[1] = make_float4(dg[c][4], dg[c][5], dg[c][6], dg[c][7]);
+      ob[0] = make_float4(db[c][0], db[c][1], db[c][2], db[c][3]);
+      ob[1] = make_float4(db[c][4], db[c][5], db[c][6], db[c][7]);
+    }
+  }
+}
+
+// dgamma[j] = sum_b partial[b][0][j], dbeta[j] = sum_b partial[b][1][j], in
+// CTA order (deterministic).  One thread per column; consecutive threads read
+// consecutive columns.
+__global__ void ln_grad_params_kernel(const float* partial, int nblk, int H, float* dgamma, float* dbeta) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j >= H) return;
+  float a = 0.0f, b = 0.0f;
+  for (int k = 0; k < nblk; ++k) {
+    a += partial[static_cast<long long>(k) * 2 * H + j];
+    b += partial[static_cast<long long>(k) * 2 * H + H + j];
+  }
+  if (dgamma) dgamma[j] = a;
+  if (dbeta) dbeta[j] = b;
+}
+
+}  // namespace tp

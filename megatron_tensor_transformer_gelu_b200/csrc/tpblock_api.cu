@@ -15,6 +15,7 @@
 #include "../../include/tpblock.h"
 #include "attention.cuh"
 #include "gemm_tcgen05.cuh"
+#include "ln_backward.cuh"
 #include "reduce_ln.cuh"
 #include "simt_f32.cuh"
 
@@ -48,7 +49,7 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 // ------------------------------------------------------------ event timing
 constexpr int PROF_CAP = 16384;  // launches timed between two collects
-constexpr int PROF_KINDS = 4;
+constexpr int PROF_KINDS = 5;
 bool g_prof_on = false;
 bool g_prof_events_made = false;
 cudaEvent_t g_ev_start[PROF_CAP];
@@ -57,7 +58,7 @@ int g_prof_kind[PROF_CAP];
 int g_prof_n = 0;
 long long g_prof_launches[PROF_KINDS];  // every launch while enabled, timed or not
 
-enum Kind { K_GEMM_TC = 0, K_REDUCE_LN = 1, K_GEMM_SIMT = 2, K_ATTN = 3 };
+enum Kind { K_GEMM_TC = 0, K_REDUCE_LN = 1, K_GEMM_SIMT = 2, K_ATTN = 3, K_LN_BACK = 4 };
 
 struct ProfScope {
   int slot = -1;
@@ -251,13 +252,27 @@ TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits)
   return best;
 }
 
+// Options of a tensor-core GEMM beyond the forward sublayers' needs (the
+// backward pass): M-major A, strided B shards, per-shard output buffers, and
+// the epilogue modes of tp::GemmArgs.
+struct GemmExtra {
+  int a_mnmajor = 0;                 // A stored [K, M] (row stride lda)
+  long long ldb = 0;                 // row stride of every B shard (0: contiguous)
+  void* const* C_shards = nullptr;   // column mode: shard s writes C_shards[s] (row stride ldc_shard)
+  long long ldc_shard = 0;
+  int epi_mode = tp::EPI_PLAIN;
+  const void* aux = nullptr;         // EPI_AUX_PRE: bf16 output laid out like C; EPI_GRAD: bf16 U
+  long long ld_aux = 0;
+};
+
 template <int CG, bool WIDE>
-int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, const TilePlan& plan, cudaStream_t st) {
+int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, const TilePlan& plan, const GemmExtra& ex,
+                   cudaStream_t st) {
   using C = tp::GemmCfg<CG, WIDE>;
   p.m_blocks = ceil_div(p.M, C::TILE_M);
   p.tile_n = plan.tile_n;
   p.n2 = WIDE ? plan.tile_n - C::BN : 0;
-  p.idesc2 = WIDE ? tp::idesc_bf16_f32(C::TILE_M, p.n2, false, !p.b_kmajor) : 0u;
+  p.idesc2 = WIDE ? tp::idesc_bf16_f32(C::TILE_M, p.n2, p.a_mnmajor != 0, !p.b_kmajor) : 0u;
   p.n_blocks_per_shard = ceil_div(p.shard_n, p.tile_n);
   p.n_blocks = p.row_mode ? p.n_blocks_per_shard : p.n_blocks_per_shard * p.t;
   const long long tiles = static_cast<long long>(p.m_blocks) * p.n_blocks;
@@ -268,8 +283,13 @@ int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, const TilePlan& plan,
     if (!tmap_out(&p.tmC[0], p.C, p.out_f32, p.shard_n, p.M, p.splits, p.ldc, p.slot_stride)) return TP_ERR_CUDA;
   } else {
     for (int s = 0; s < p.t; ++s) {
-      void* base = static_cast<uint8_t*>(p.C) + static_cast<long long>(s) * p.shard_n * es;
-      if (!tmap_out(&p.tmC[s], base, p.out_f32, p.shard_n, p.M, 1, p.ldc, 0)) return TP_ERR_CUDA;
+      void* base = ex.C_shards ? ex.C_shards[s] : static_cast<uint8_t*>(p.C) + static_cast<long long>(s) * p.shard_n * es;
+      const long long ld = ex.C_shards ? ex.ldc_shard : p.ldc;
+      if (!tmap_out(&p.tmC[s], base, p.out_f32, p.shard_n, p.M, 1, ld, 0)) return TP_ERR_CUDA;
+      if (ex.epi_mode == tp::EPI_AUX_PRE) {
+        void* abase = static_cast<uint8_t*>(const_cast<void*>(ex.aux)) + static_cast<long long>(s) * p.shard_n * 2;
+        if (!tmap_out(&p.tmAux[s], abase, 0, p.shard_n, p.M, 1, ex.ld_aux, 0)) return TP_ERR_CUDA;
+      }
     }
   }
   const long long units = tiles * p.splits;
@@ -302,7 +322,9 @@ int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, const TilePlan& plan,
 int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, const void* const* B, int t,
                 int row_mode, int shard_k, int shard_n, void* C, long long ldc, int out_f32, int act,
                 cudaStream_t st, int max_splits = 1, long long slot_stride = 0, int* splits_out = nullptr,
-                int b_kmajor = 0) {
+                int b_kmajor = 0, const GemmExtra* extra = nullptr) {
+  const GemmExtra none;
+  const GemmExtra& ex = extra ? *extra : none;
   using G = tp::GemmCfg<1>;
   if (splits_out) *splits_out = 1;
   if (M == 0) return TP_OK;
@@ -310,15 +332,24 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
   tp::GemmArgs p;
   std::memset(&p, 0, sizeof(p));
   const long long K_total = row_mode ? static_cast<long long>(shard_k) * t : shard_k;
-  if (!tmap_bf16(&p.tmA, A, M, K_total, lda, G::BK, G::BM)) return TP_ERR_CUDA;
+  if (ex.a_mnmajor) {  // stored [K, M]; box 64 m x 64 k
+    if (!tmap_bf16(&p.tmA, A, K_total, M, lda, 64, G::BK)) return TP_ERR_CUDA;
+  } else if (!tmap_bf16(&p.tmA, A, M, K_total, lda, G::BK, G::BM)) {
+    return TP_ERR_CUDA;
+  }
   for (int s = 0; s < t; ++s) {
     bool ok;
     if (b_kmajor)  // shard [shard_n rows, shard_k cols]; box 64 k x (BN / CG) rows
-      ok = tmap_bf16(&p.tmB[s], B[s], shard_n, shard_k, shard_k, G::BK, pair ? tp::GemmCfg<2>::B_COLS_CTA : G::BN);
+      ok = tmap_bf16(&p.tmB[s], B[s], shard_n, shard_k, ex.ldb ? ex.ldb : shard_k, G::BK,
+                     pair ? tp::GemmCfg<2>::B_COLS_CTA : G::BN);
     else           // shard [shard_k rows, shard_n cols]; box 64 n x 64 k
-      ok = tmap_bf16(&p.tmB[s], B[s], shard_k, shard_n, shard_n, G::B_BOX_N, G::BK);
+      ok = tmap_bf16(&p.tmB[s], B[s], shard_k, shard_n, ex.ldb ? ex.ldb : shard_n, G::B_BOX_N, G::BK);
     if (!ok) return TP_ERR_CUDA;
   }
+  p.a_mnmajor = ex.a_mnmajor;
+  p.epi_mode = ex.epi_mode;
+  p.aux = ex.aux;
+  p.ld_aux = ex.ld_aux;
   p.C = C;
   p.ldc = ldc;
   p.M = M;
@@ -337,9 +368,9 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
   if (!out_f32) max_splits = 1;
   const TilePlan plan = plan_tiles(p, pair, pair ? dev.max_pairs : dev.sm_count, max_splits);
   int r;
-  if (!pair) r = launch_gemm_tc<1, false>(dev, p, plan, st);
-  else if (plan.tile_n > tp::GemmCfg<2>::BN) r = launch_gemm_tc<2, true>(dev, p, plan, st);
-  else r = launch_gemm_tc<2, false>(dev, p, plan, st);
+  if (!pair) r = launch_gemm_tc<1, false>(dev, p, plan, ex, st);
+  else if (plan.tile_n > tp::GemmCfg<2>::BN) r = launch_gemm_tc<2, true>(dev, p, plan, ex, st);
+  else r = launch_gemm_tc<2, false>(dev, p, plan, ex, st);
   if (splits_out) *splits_out = p.splits;
   return r;
 }
@@ -426,6 +457,84 @@ bool shards_ok(const void* const* s, int t) {
 bool ptr_ok(const void* p) { return p && aligned16(p); }
 bool opt_ptr_ok(const void* p) { return !p || aligned16(p); }
 bool hidden_ok(int H) { return H >= 8 && H % 8 == 0 && H <= tp::rln::MAX_H; }
+
+// ------------------------------------------------------------ training state
+// Saved by tp_mlp_forward_train for tp_mlp_backward: U = X A (pre-activation,
+// bf16 [S, F]), G = Act(U) (bf16 [S, F], the row-split GEMM's input) and
+// V = G B (f32 [S, H], the row-split GEMM's output before the residual).
+struct TrainState {
+  size_t off_u, off_g, off_v, bytes;
+};
+TrainState train_state_layout(int S, int H, int F) {
+  TrainState t;
+  const size_t sf = static_cast<size_t>(S) * F, sh = static_cast<size_t>(S) * H;
+  t.off_u = 0;
+  t.off_g = align256(sf * 2);
+  t.off_v = t.off_g + align256(sf * 2);
+  t.bytes = t.off_v + align256(sh * 4);
+  return t;
+}
+
+// Backward workspace: dZ (bf16 [S, H]), dU (bf16 [S, F]), the f32 row-split
+// partial of dX ([S, H]) and the LayerNorm-backward CTAs' dgamma/dbeta partial
+// rows (at most LNB_MAX_CTAS x 2 x H f32).
+constexpr int LNB_MAX_CTAS = 320;
+struct BackWs {
+  size_t off_dz, off_du, off_dxp, off_part, bytes;
+};
+BackWs back_ws_layout(int S, int H, int F) {
+  BackWs w;
+  const size_t sf = static_cast<size_t>(S) * F, sh = static_cast<size_t>(S) * H;
+  w.off_dz = 0;
+  w.off_du = align256(sh * 2);
+  w.off_dxp = w.off_du + align256(sf * 2);
+  w.off_part = w.off_dxp + align256(sh * 4);
+  w.bytes = w.off_part + align256(static_cast<size_t>(LNB_MAX_CTAS) * 2 * H * 4);
+  return w;
+}
+
+// LayerNorm backward + the dgamma/dbeta reduction.  Chunks of 8 per thread:
+// CH = ceil(H / 8 / 512) (1..4), threads = the chunks per CH rounded up to a
+// warp; CTAs = as many as fit two per SM's worth of threads (at most
+// LNB_MAX_CTAS, at most S).
+int run_ln_backward(int S, int H, const float* V, const void* X, const void* dY, const float* gamma, float eps,
+                    void* dZ, float* partial, float* dgamma, float* dbeta, cudaStream_t st, int dev_sms) {
+  tp::LnBackArgs p;
+  p.S = S;
+  p.H = H;
+  p.nparts = 1;
+  p.parts = V;
+  p.part_stride = static_cast<long long>(S) * H;
+  p.X = static_cast<const __nv_bfloat16*>(X);
+  p.dY = static_cast<const __nv_bfloat16*>(dY);
+  p.gamma = gamma;
+  p.eps = eps;
+  p.dZ = static_cast<__nv_bfloat16*>(dZ);
+  p.partial = partial;
+  const int chunks = H / 8;
+  const int ch = ceil_div(chunks, 512);
+  const int threads = ceil_div(ceil_div(chunks, ch), 32) * 32;
+  int grid = (2048 / threads) * dev_sms / 2;
+  if (grid > LNB_MAX_CTAS) grid = LNB_MAX_CTAS;
+  if (grid > S) grid = S;
+  if (grid < 1) grid = 1;
+  {
+    ProfScope ps(K_LN_BACK, st);
+    switch (ch) {
+      case 1: tp::ln_backward_kernel<1><<<grid, threads, 0, st>>>(p); break;
+      case 2: tp::ln_backward_kernel<2><<<grid, threads, 0, st>>>(p); break;
+      case 3: tp::ln_backward_kernel<3><<<grid, threads, 0, st>>>(p); break;
+      default: tp::ln_backward_kernel<4><<<grid, threads, 0, st>>>(p); break;
+    }
+    if (launch_status() != TP_OK) return TP_ERR_CUDA;
+  }
+  if (dgamma || dbeta) {
+    ProfScope ps(K_LN_BACK, st);
+    tp::ln_grad_params_kernel<<<ceil_div(H, 256), 256, 0, st>>>(partial, grid, H, dgamma, dbeta);
+    return launch_status();
+  }
+  return TP_OK;
+}
 
 }  // namespace
 
@@ -606,6 +715,125 @@ int tp_mlp_forward_ex(int S, int H, int F, int t, int dtype, int out_dtype, int 
   if (st != TP_OK) return st;
   return mlp_core(*dev, S, H, F, t, dtype, out_dtype, X, X, A_shards, B_shards, gamma, beta, eps, act, 1, Y,
                   workspace, static_cast<cudaStream_t>(stream), w_layout == TP_W_OUT_IN);
+}
+
+// ------------------------------------------------------- MLP training step
+size_t tp_mlp_train_state_bytes(int S, int H, int F, int t, int dtype) {
+  if (S < 0 || H <= 0 || F <= 0 || t < 1 || dtype != TP_DTYPE_BF16) return 0;
+  return train_state_layout(S, H, F).bytes;
+}
+
+int tp_mlp_forward_train(int S, int H, int F, int t, int dtype, int out_dtype, const void* X,
+                         const void* const* A_shards, const void* const* B_shards, const float* gamma,
+                         const float* beta, float eps, int act, void* Y, void* state, size_t state_bytes,
+                         void* stream) {
+  if (dtype != TP_DTYPE_BF16) return TP_ERR_UNSUPPORTED_SHAPE;
+  int st = check_mlp_args(S, H, F, t, dtype, out_dtype, X, A_shards, B_shards, gamma, beta, eps, act, Y);
+  if (st != TP_OK) return st;
+  if (!opt_ptr_ok(state)) return TP_ERR_INVALID_ARG;
+  if (S == 0) return TP_OK;
+  const TrainState L = train_state_layout(S, H, F);
+  if (!state || state_bytes < L.bytes) return TP_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(state);
+  void* U = base + L.off_u;
+  void* G = base + L.off_g;
+  float* V = reinterpret_cast<float*>(base + L.off_v);
+  const int Fs = F / t;
+  // G_i = Act(X A_i) into columns [i Fs, (i+1) Fs) of G, and U_i = X A_i (the
+  // pre-activation, from the same accumulator) into the same columns of U.
+  GemmExtra ex;
+  ex.epi_mode = tp::EPI_AUX_PRE;
+  ex.aux = U;
+  ex.ld_aux = F;
+  st = run_gemm_tc(*dev, X, H, S, A_shards, t, 0, H, Fs, G, F, 0, act, s, 1, 0, nullptr, 0, &ex);
+  if (st != TP_OK) return st;
+  // V = sum_i G_i B_i in one f32 slot (no K split: the backward reads one).
+  st = run_gemm_tc(*dev, G, F, S, B_shards, t, 1, Fs, H, V, H, 1, TP_ACT_NONE, s, 1, 0, nullptr, 0);
+  if (st != TP_OK) return st;
+  return run_reduce_ln(S, H, 1, V, X, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s, dev->sm_count);
+}
+
+size_t tp_mlp_backward_workspace_bytes(int S, int H, int F, int t, int dtype) {
+  if (S < 0 || H <= 0 || F <= 0 || t < 1 || dtype != TP_DTYPE_BF16) return 0;
+  return back_ws_layout(S, H, F).bytes;
+}
+
+int tp_mlp_backward(int S, int H, int F, int t, int dtype, const void* X, const void* const* A_shards,
+                    const void* const* B_shards, const float* gamma, float eps, int act, const void* state,
+                    size_t state_bytes, const void* dY, void* dX, void* const* dA_shards, void* const* dB_shards,
+                    float* dgamma, float* dbeta, void* workspace, size_t workspace_bytes, void* stream) {
+  if (dtype != TP_DTYPE_BF16) return TP_ERR_UNSUPPORTED_SHAPE;
+  int st = check_mlp_args(S, H, F, t, dtype, TP_DTYPE_BF16, X, A_shards, B_shards, gamma, nullptr, eps, act, dX);
+  if (st != TP_OK) return st;
+  if ((S > 0 && (!ptr_ok(dY) || !ptr_ok(state))) || !opt_ptr_ok(dY) || !opt_ptr_ok(state) ||
+      !shards_ok(dA_shards, t) || !shards_ok(dB_shards, t) || !opt_ptr_ok(dgamma) || !opt_ptr_ok(dbeta) ||
+      !opt_ptr_ok(workspace))
+    return TP_ERR_INVALID_ARG;
+  if (S == 0) return TP_OK;  // weight gradients of an empty batch: the caller's buffers are left as they are
+  if (state_bytes < train_state_layout(S, H, F).bytes) return TP_ERR_WORKSPACE_TOO_SMALL;
+  const BackWs W = back_ws_layout(S, H, F);
+  if (!workspace || workspace_bytes < W.bytes) return TP_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const TrainState L = train_state_layout(S, H, F);
+  const uint8_t* sb = static_cast<const uint8_t*>(state);
+  const void* U = sb + L.off_u;
+  const uint8_t* G = sb + L.off_g;
+  const float* V = reinterpret_cast<const float*>(sb + L.off_v);
+  uint8_t* wb = static_cast<uint8_t*>(workspace);
+  void* dZ = wb + W.off_dz;
+  uint8_t* dU = wb + W.off_du;
+  float* dXp = reinterpret_cast<float*>(wb + W.off_dxp);
+  float* part = reinterpret_cast<float*>(wb + W.off_part);
+  const int Fs = F / t;
+  // 1. Through the LayerNorm: dZ, dgamma, dbeta.
+  st = run_ln_backward(S, H, V, X, dY, gamma, eps, dZ, part, dgamma, dbeta, s, dev->sm_count);
+  if (st != TP_OK) return st;
+  // 2. Through V = G B and G = Act(U): dU_i = (dZ B_i^T) * Act'(U_i) into the
+  //    columns of shard i (B_i [Fs, H] is read K-major as B_i^T).
+  {
+    GemmExtra ex;
+    ex.epi_mode = tp::EPI_GRAD;
+    ex.aux = U;
+    ex.ld_aux = F;
+    st = run_gemm_tc(*dev, dZ, H, S, B_shards, t, 0, H, Fs, dU, F, 0, act, s, 1, 0, nullptr, 1, &ex);
+    if (st != TP_OK) return st;
+  }
+  // 3. Through U = X A and the residual: dX = dZ + sum_i dU_i A_i^T (row split
+  //    over the shards, A_i [H, Fs] read K-major), then the residual add.
+  st = run_gemm_tc(*dev, dU, F, S, A_shards, t, 1, Fs, H, dXp, H, 1, TP_ACT_NONE, s, 1, 0, nullptr, 1);
+  if (st != TP_OK) return st;
+  st = run_reduce_ln(S, H, 1, dXp, dZ, 1, nullptr, nullptr, 1.0f, dX, 1, s, dev->sm_count, /*apply_ln=*/0);
+  if (st != TP_OK) return st;
+  // 4. Weight gradients, each with its own shard.  dA_i = X^T dU_i: A operand
+  //    X read M-major, B operand the column slice i of dU (row stride F).
+  {
+    const void* dU_sh[TP_MAX_SHARDS];
+    for (int i = 0; i < t; ++i) dU_sh[i] = dU + static_cast<size_t>(i) * Fs * 2;
+    GemmExtra ex;
+    ex.a_mnmajor = 1;
+    ex.ldb = F;
+    ex.C_shards = dA_shards;
+    ex.ldc_shard = Fs;
+    st = run_gemm_tc(*dev, X, H, H, dU_sh, t, 0, S, Fs, nullptr, Fs, 1, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
+    if (st != TP_OK) return st;
+  }
+  //    dB_i = G_i^T dZ: A operand the column slice i of G read M-major.
+  for (int i = 0; i < t; ++i) {
+    const void* dz1[1] = {dZ};
+    GemmExtra ex;
+    ex.a_mnmajor = 1;
+    st = run_gemm_tc(*dev, G + static_cast<size_t>(i) * Fs * 2, F, Fs, dz1, 1, 0, S, H, dB_shards[i], H, 1,
+                     TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
+    if (st != TP_OK) return st;
+  }
+  return TP_OK;
 }
 
 // -------------------------------------------------------------- attention
@@ -829,6 +1057,7 @@ const char* tp_kernel_kind_name(int kind) {
     case K_REDUCE_LN: return "reduce_residual_layernorm";
     case K_GEMM_SIMT: return "gemm_simt_f32";
     case K_ATTN: return "attention_fwd";
+    case K_LN_BACK: return "layernorm_backward";
     default: return "unknown";
   }
 }

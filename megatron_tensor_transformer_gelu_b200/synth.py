@@ -92,6 +92,17 @@ def gen_linear(M: int, K: int, N: int, seed: int = 0, dtype=torch.bfloat16) -> L
     return LinearInputs(X, W)
 
 
+def gen_upstream(S: int, H: int, seed: int = 0, dtype=torch.bfloat16):
+    """Upstream gradient dY ~ N(0, 1) [S, H] and a LayerNorm scale gamma ~
+    1 + N(0, 1)/4, beta ~ N(0, 1)/4 (f32 [H]) for backward tests: the same
+    recipe as the forward inputs, from its own seeded generator."""
+    g = _gen(seed)
+    dY = torch.randn(S, H, generator=g).to(dtype)
+    gamma = 1.0 + 0.25 * torch.randn(H, generator=g)
+    beta = 0.25 * torch.randn(H, generator=g)
+    return dY, gamma, beta
+
+
 def split_columns(W: torch.Tensor, t: int) -> list[torch.Tensor]:
     """t contiguous column shards of a [in, out] matrix."""
     n = W.shape[1]

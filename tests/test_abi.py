@@ -139,6 +139,38 @@ def test_linear_and_layernorm_argument_checks(lib):
                                             ctypes.c_void_p(FAKE), 1, None) == INVALID
 
 
+def test_training_argument_checks(lib):
+    S, H, F, t = 128, 256, 1024, 2
+    pa, ka = _ptrs(t)
+    pb, kb = _ptrs(t)
+    pda, kda = _ptrs(t)
+    pdb, kdb = _ptrs(t)
+    st_bytes = lib.tp_mlp_train_state_bytes(S, H, F, t, 1)
+    assert st_bytes == 2 * S * F * 2 + S * H * 4
+    assert lib.tp_mlp_train_state_bytes(S, H, F, t, 0) == 0      # f32 storage has no training path
+    ws_bytes = lib.tp_mlp_backward_workspace_bytes(S, H, F, t, 1)
+    assert ws_bytes >= S * H * 2 + S * F * 2 + S * H * 4
+    P = ctypes.c_void_p(FAKE)
+
+    def fwd(dtype=1, state_bytes=st_bytes, act=1):
+        return lib.tp_mlp_forward_train(S, H, F, t, dtype, 1, P, pa, pb, None, None, 1e-5, act, P, P, state_bytes,
+                                        None)
+
+    def bwd(dtype=1, dY=P, state_bytes=st_bytes, ws=ws_bytes, dA=pda):
+        return lib.tp_mlp_backward(S, H, F, t, dtype, P, pa, pb, None, 1e-5, 1, P, state_bytes, dY, P, dA, pdb,
+                                   None, None, P, ws, None)
+
+    assert fwd(dtype=0) == UNSUPPORTED
+    assert fwd(act=9) == INVALID
+    assert fwd(state_bytes=st_bytes - 1) == WS_SMALL
+    assert bwd(dtype=0) == UNSUPPORTED
+    assert bwd(dY=None) == INVALID
+    assert bwd(dY=ctypes.c_void_p(FAKE + 8)) == INVALID             # misaligned
+    assert bwd(dA=None) == INVALID
+    assert bwd(state_bytes=1) == WS_SMALL
+    assert bwd(ws=ws_bytes - 1) == WS_SMALL
+
+
 def test_gemm_tile_override_checks(lib):
     try:
         for bad in (-32, 100, 224, 300, 544):

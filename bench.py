@@ -32,6 +32,11 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "TP MLP block fwd TFLOP/s (bf16, 1 B200) and % of dense bf16 tensor peak"
+METRIC_TRAIN = "TP MLP block training step (fwd + bwd) TFLOP/s (bf16, 1 B200) and % of dense bf16 tensor peak"
+
+
+def metric_for(w) -> str:
+    return METRIC_TRAIN if w.kind == "mlp_train" else METRIC
 UNIT = "TFLOP/s"
 L2_BYTES = 126 * 2**20
 
@@ -190,6 +195,36 @@ class Problem:
                          "reduce_residual_layernorm": S * H * 4 + S * H * 2 * 2 + H * 8}
             self.Xh_src = inp.X
             self.run = lambda X, Y, st: L.mlp_forward(X, self.W1, self.W2, Y, self.ws, stream=st)
+        elif w.kind == "mlp_train":
+            S, H, F = w.S, w.H, w.F
+            inp = synth.gen_mlp(S, H, F, seed=w.seed + rank)
+            dY, gamma, _ = synth.gen_upstream(S, H, seed=w.seed + rank + 2)
+            self.X = inp.X.to(dev)
+            self.W1 = [a.to(dev) for a in synth.split_columns(inp.A, t)]
+            self.W2 = [b.to(dev) for b in synth.split_rows(inp.B, t)]
+            self.dY = dY.to(dev)
+            self.gamma = gamma.to(dev)
+            self.Yf = torch.empty(S, H, dtype=bf, device=dev)           # forward output
+            self.Y = torch.empty(S, H, dtype=bf, device=dev)            # the step's result: dX
+            self.state = torch.empty(L.mlp_train_state_bytes(S, H, F, t), dtype=torch.uint8, device=dev)
+            self.ws = torch.empty(L.mlp_backward_workspace_bytes(S, H, F, t), dtype=torch.uint8, device=dev)
+            self.dA = [torch.empty(H, F // t, dtype=torch.float32, device=dev) for _ in range(t)]
+            self.dB = [torch.empty(F // t, H, dtype=torch.float32, device=dev) for _ in range(t)]
+            self.dg = torch.empty(H, dtype=torch.float32, device=dev)
+            self.db = torch.empty(H, dtype=torch.float32, device=dev)
+            # LayerNorm backward reads V (f32), X, dY (twice, the second time from
+            # cache) and writes dZ; the forward LayerNorm and the dX residual
+            # add each move 8 bytes per element.
+            self.work = {"gemm_tcgen05": w.flops,
+                         "reduce_residual_layernorm": 2 * (S * H * 8 + H * 8),
+                         "layernorm_backward": S * H * (4 + 2 + 2 + 2)}
+            self.Xh_src = inp.X
+
+            def train_step(X, Y, st):
+                L.mlp_forward_train(X, self.W1, self.W2, self.Yf, self.state, gamma=self.gamma, stream=st)
+                L.mlp_backward(X, self.W1, self.W2, self.state, self.dY, Y, self.dA, self.dB, self.ws,
+                               gamma=self.gamma, dgamma=self.dg, dbeta=self.db, stream=st)
+            self.run = train_step
         elif w.kind == "attn":
             S, H = w.S, w.H
             inp = synth.gen_attn(S, H, seed=w.seed + rank)
@@ -344,7 +379,7 @@ def run_ours(args, rank, world, local):
                 continue
             per_launch_ms = ms_k / n_timed
             launches_per_step = n_all / args.steps
-            tensor = kind != "reduce_residual_layernorm"
+            tensor = kind in ("gemm_tcgen05", "attention_fwd")
             work_per_launch = work / launches_per_step
             rate = work_per_launch / (per_launch_ms * 1e-3)
             if tensor:
@@ -374,10 +409,10 @@ def run_ours(args, rank, world, local):
         for key in ("S", "H", "F", "nh", "d", "M", "K", "N"):
             if getattr(w, key):
                 cfg[key] = getattr(w, key)
-        if w.kind == "mlp":
+        if w.kind in ("mlp", "mlp_train"):
             cfg["act"] = "gelu_tanh"
         result = {
-            "metric": METRIC,
+            "metric": metric_for(w),
             "value": round(value, 2),
             "unit": UNIT,
             "n_gpus": world,
@@ -425,6 +460,11 @@ def cpu_oracle_timing(w, rows_per_step: int, steps: int, warmup: int):
         inp = synth.gen_mlp(w.S, w.H, w.F, seed=w.seed)
         nrows = w.S
         call = lambda rows: O.mlp_block(inp.X, inp.A, inp.B, rows=rows)
+    elif w.kind == "mlp_train":
+        inp = synth.gen_mlp(w.S, w.H, w.F, seed=w.seed)
+        dY, gamma, _ = synth.gen_upstream(w.S, w.H, seed=w.seed + 2)
+        nrows = w.S
+        call = lambda rows: O.mlp_block_backward(inp.X[rows], inp.A, inp.B, dY[rows], gamma)
     elif w.kind == "attn":
         inp = synth.gen_attn(w.S, w.H, seed=w.seed)
         nrows = w.S
@@ -447,7 +487,8 @@ def cpu_oracle_timing(w, rows_per_step: int, steps: int, warmup: int):
     dt = time.perf_counter() - t0
     flops = w.flops * len(rows) / nrows * steps
     return {"value": round(flops / dt / 1e12, 5), "unit": UNIT, "cores": int(cores), "kind": "oracle",
-            "sample": (f"{len(rows)} of {nrows} output rows of {w.name} per step, {steps} step(s), "
+            "sample": (f"{len(rows)} of {nrows} {'batch' if w.kind == 'mlp_train' else 'output'} rows of {w.name} "
+                       f"per step, {steps} step(s), "
                        "fp64 numpy/OpenBLAS" + ("; every call also computes all K and V rows"
                                                 if w.kind == "attn" else "")),
             "seconds": round(dt, 3)}
@@ -463,7 +504,7 @@ def run_reference(args, rank, world):
     ms_step = cb["seconds"] / args.steps * 1e3
     return {
         "impl": "reference",
-        "metric": METRIC,
+        "metric": metric_for(w),
         "value": cb["value"],
         "unit": UNIT,
         "n_gpus": world,
@@ -494,7 +535,8 @@ def main():
         from megatron_tensor_transformer_gelu_b200.workloads import HEADLINE, WORKLOADS
         if not args.no_cpu_baseline:
             w = WORKLOADS[args.workload or HEADLINE]
-            rows = args.cpu_sample_rows if w.kind == "mlp" else min(args.cpu_sample_rows, 64)
+            rows = {"mlp": args.cpu_sample_rows, "mlp_train": min(args.cpu_sample_rows, 256)}.get(
+                w.kind, min(args.cpu_sample_rows, 64))
             res["cpu_baseline"] = cpu_oracle_timing(w, rows, 1, 0)
         print(json.dumps(res), flush=True)
 

@@ -48,32 +48,12 @@ __device__ __forceinline__ float lnb_block_sum(float v, float* red) {
   return t;
 }
 
-__device__ __forceinline__ void lnb_block_sum2(float& a, float& b, float* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    a += __shfl_xor_sync(0xffffffffu, a, o);
-    b += __shfl_xor_sync(0xffffffffu, b, o);
-  }
-  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) {
-    red[warp] = a;
-    red[lnb::MAX_WARPS + warp] = b;
-  }
-  __syncthreads();
-  float ta = 0.0f, tb = 0.0f;
-  for (int w = 0; w < nw; ++w) {
-    ta += red[w];
-    tb += red[lnb::MAX_WARPS + w];
-  }
-  a = ta;
-  b = tb;
-}
-
 // CH chunks of 8 consecutive elements per thread (CH = 1..4, up to 512
 // threads, so H <= 16384); chunk c of thread i covers elements
-// (c * blockDim.x + i) * 8 ...; chunks past H are masked.  dY is read twice
-// (the second time from cache) to keep registers for Z and the running
+// (c * blockDim.x + i) * 8 ...; chunks past H are masked.  A row takes two
+// CTA reductions: (sum z, sum g, sum g z), then sum (z - mean)^2, using
+// sum g xh = r (sum g z - mean sum g).  dY is read again (from cache) in the
+// last pass instead of being held, to keep registers for Z and the running
 // dgamma/dbeta column sums.
 __device__ __forceinline__ void lnb_load8_bf16(const __nv_bfloat16* src, float (&v)[8]) {
   const uint4 w = *reinterpret_cast<const uint4*>(src);
@@ -86,9 +66,36 @@ __device__ __forceinline__ void lnb_load8_bf16(const __nv_bfloat16* src, float (
   }
 }
 
+// Sum of three values over the CTA (fixed order), as lnb_block_sum.
+__device__ __forceinline__ void lnb_block_sum3(float& a, float& b, float& c, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    a += __shfl_xor_sync(0xffffffffu, a, o);
+    b += __shfl_xor_sync(0xffffffffu, b, o);
+    c += __shfl_xor_sync(0xffffffffu, c, o);
+  }
+  const int warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) {
+    red[warp] = a;
+    red[lnb::MAX_WARPS + warp] = b;
+    red[2 * lnb::MAX_WARPS + warp] = c;
+  }
+  __syncthreads();
+  float ta = 0.0f, tb = 0.0f, tc = 0.0f;
+  for (int w = 0; w < nw; ++w) {
+    ta += red[w];
+    tb += red[lnb::MAX_WARPS + w];
+    tc += red[2 * lnb::MAX_WARPS + w];
+  }
+  a = ta;
+  b = tb;
+  c = tc;
+}
+
 template <int CH>
 __global__ void __launch_bounds__(512) ln_backward_kernel(const LnBackArgs p) {
-  __shared__ float red[2 * lnb::MAX_WARPS];
+  __shared__ float red[3 * lnb::MAX_WARPS];
   const int nthr = blockDim.x;
   float z[CH][8], dg[CH][8], db[CH][8];
 #pragma unroll
@@ -99,12 +106,14 @@ __global__ void __launch_bounds__(512) ln_backward_kernel(const LnBackArgs p) {
 
   for (int row = blockIdx.x; row < p.S; row += gridDim.x) {
     const long long base = static_cast<long long>(row) * p.H;
-    float s = 0.0f;
+    float sz = 0.0f, sg = 0.0f, sgz = 0.0f;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int col = (c * nthr + threadIdx.x) * 8;
       if (col < p.H) {
+        float dy[8];
         lnb_load8_bf16(p.X + base + col, z[c]);
+        lnb_load8_bf16(p.dY + base + col, dy);
         for (int q = 0; q < p.nparts; ++q) {
           const float4* pp = reinterpret_cast<const float4*>(p.parts + q * p.part_stride + base + col);
           const float4 a = __ldcs(pp), b = __ldcs(pp + 1);
@@ -112,10 +121,16 @@ __global__ void __launch_bounds__(512) ln_backward_kernel(const LnBackArgs p) {
           z[c][4] += b.x; z[c][5] += b.y; z[c][6] += b.z; z[c][7] += b.w;
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) s += z[c][e];
+        for (int e = 0; e < 8; ++e) {
+          const float g = p.gamma ? dy[e] * __ldg(p.gamma + col + e) : dy[e];
+          sz += z[c][e];
+          sg += g;
+          sgz = fmaf(g, z[c][e], sgz);
+        }
       }
     }
-    const float mean = lnb_block_sum(s, red) * inv_h;
+    lnb_block_sum3(sz, sg, sgz, red);
+    const float mean = sz * inv_h;
     float v = 0.0f;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
@@ -130,27 +145,8 @@ __global__ void __launch_bounds__(512) ln_backward_kernel(const LnBackArgs p) {
     }
     const float var = lnb_block_sum(v, red) * inv_h;
     const float r = rsqrtf(var + p.eps);
-    float sg = 0.0f, sgx = 0.0f;
-#pragma unroll
-    for (int c = 0; c < CH; ++c) {
-      const int col = (c * nthr + threadIdx.x) * 8;
-      if (col < p.H) {
-        float dy[8];
-        lnb_load8_bf16(p.dY + base + col, dy);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float xh = (z[c][e] - mean) * r;
-          const float g = p.gamma ? dy[e] * __ldg(p.gamma + col + e) : dy[e];
-          z[c][e] = xh;  // z now holds the normalised row
-          sg += g;
-          sgx = fmaf(g, xh, sgx);
-          dg[c][e] = fmaf(dy[e], xh, dg[c][e]);
-          db[c][e] += dy[e];
-        }
-      }
-    }
-    lnb_block_sum2(sg, sgx, red);
-    const float mg = sg * inv_h, mgx = sgx * inv_h;
+    const float mg = sg * inv_h;
+    const float mgx = r * (sgz - mean * sg) * inv_h;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int col = (c * nthr + threadIdx.x) * 8;
@@ -164,8 +160,11 @@ __global__ void __launch_bounds__(512) ln_backward_kernel(const LnBackArgs p) {
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
             const int i = 2 * e + k;
+            const float xh = (z[c][i] - mean) * r;
             const float g = p.gamma ? dy[i] * __ldg(p.gamma + col + i) : dy[i];
-            o[k] = r * (g - mg - z[c][i] * mgx);
+            o[k] = r * (g - mg - xh * mgx);
+            dg[c][i] = fmaf(dy[i], xh, dg[c][i]);
+            db[c][i] += dy[i];
           }
           __nv_bfloat162 h = __floats2bfloat162_rn(o[0], o[1]);
           w[e] = *reinterpret_cast<uint32_t*>(&h);
@@ -190,19 +189,47 @@ __global__ void __launch_bounds__(512) ln_backward_kernel(const LnBackArgs p) {
   }
 }
 
-// dgamma[j] = sum_b partial[b][0][j], dbeta[j] = sum_b partial[b][1][j], in
-// CTA order (deterministic).  One thread per column; consecutive threads read
-// consecutive columns.
-__global__ void ln_grad_params_kernel(const float* partial, int nblk, int H, float* dgamma, float* dbeta) {
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= H) return;
-  float a = 0.0f, b = 0.0f;
-  for (int k = 0; k < nblk; ++k) {
-    a += partial[static_cast<long long>(k) * 2 * H + j];
-    b += partial[static_cast<long long>(k) * 2 * H + H + j];
+// dgamma[j] = sum_b partial[b][0][j], dbeta[j] = sum_b partial[b][1][j].
+// A CTA takes 32 columns with 32 warps: warp w sums the partial rows
+// b = w, w + 32, ... (each load a 128-byte row segment, four rows in flight
+// in separate accumulators added in a fixed order), then warp 0 adds the 32
+// warps' sums in warp order, so the result is deterministic.
+constexpr int LNB_PARAM_SLICES = 32;
+__global__ void __launch_bounds__(32 * LNB_PARAM_SLICES)
+    ln_grad_params_kernel(const float* partial, int nblk, int H, float* dgamma, float* dbeta) {
+  __shared__ float sa[LNB_PARAM_SLICES][33], sb[LNB_PARAM_SLICES][33];
+  const int lane = threadIdx.x & 31, slice = threadIdx.x >> 5;
+  const int j = blockIdx.x * 32 + lane;
+  float a[4] = {0.0f, 0.0f, 0.0f, 0.0f}, b[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  if (j < H) {
+    const long long step = 2LL * H;
+    int k = slice;
+    for (; k + 3 * LNB_PARAM_SLICES < nblk; k += 4 * LNB_PARAM_SLICES) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float* row = partial + (k + u * LNB_PARAM_SLICES) * step;
+        a[u] += row[j];
+        b[u] += row[H + j];
+      }
+    }
+    for (; k < nblk; k += LNB_PARAM_SLICES) {
+      a[0] += partial[k * step + j];
+      b[0] += partial[k * step + H + j];
+    }
   }
-  if (dgamma) dgamma[j] = a;
-  if (dbeta) dbeta[j] = b;
+  sa[slice][lane] = (a[0] + a[1]) + (a[2] + a[3]);
+  sb[slice][lane] = (b[0] + b[1]) + (b[2] + b[3]);
+  __syncthreads();
+  if (slice == 0 && j < H) {
+    float ta = 0.0f, tb = 0.0f;
+#pragma unroll 8
+    for (int w = 0; w < LNB_PARAM_SLICES; ++w) {
+      ta += sa[w][lane];
+      tb += sb[w][lane];
+    }
+    if (dgamma) dgamma[j] = ta;
+    if (dbeta) dbeta[j] = tb;
+  }
 }
 
 }  // namespace tp

@@ -530,7 +530,7 @@ int run_ln_backward(int S, int H, const float* V, const void* X, const void* dY,
   }
   if (dgamma || dbeta) {
     ProfScope ps(K_LN_BACK, st);
-    tp::ln_grad_params_kernel<<<ceil_div(H, 256), 256, 0, st>>>(partial, grid, H, dgamma, dbeta);
+    tp::ln_grad_params_kernel<<<ceil_div(H, 32), 32 * tp::LNB_PARAM_SLICES, 0, st>>>(partial, grid, H, dgamma, dbeta);
     return launch_status();
   }
   return TP_OK;

@@ -10,7 +10,7 @@ from dataclasses import dataclass, field
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str            # "mlp" | "attn" | "linear_col" | "linear_row"
+    kind: str            # "mlp" | "mlp_train" | "attn" | "linear_col" | "linear_row"
     dtype: str           # "f32" | "bf16"  (storage of X and weights)
     t: int               # shard count
     seed: int = 0
@@ -29,6 +29,9 @@ class Workload:
     def flops(self) -> int:
         if self.kind == "mlp":
             return 2 * 2 * self.S * self.H * self.F
+        if self.kind == "mlp_train":
+            # forward (X A, G B) + backward (dZ B^T, dU A^T, X^T dU, G^T dZ)
+            return 6 * 2 * self.S * self.H * self.F
         if self.kind == "attn":
             S, H = self.S, self.H
             qkv = 2 * S * H * 3 * H
@@ -53,6 +56,10 @@ WORKLOADS = {
                  S=2048, H=8192, nh=64, d=128, act="none", t_sweep=(1, 2, 4, 8)),
         Workload("mlp_s4096_h12288_f49152", "mlp", "bf16", t=8, seed=7,
                  S=4096, H=12288, F=49152, t_sweep=(8,)),
+        # One training step of the headline sublayer: forward keeping U/G/V,
+        # then the backward pass (all gradients).
+        Workload("mlp_train_s2048_h4096_f16384", "mlp_train", "bf16", t=4, seed=0,
+                 S=2048, H=4096, F=16384, t_sweep=(4,)),
     ]
 }
 

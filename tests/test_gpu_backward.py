@@ -64,6 +64,9 @@ def check(out, inp, dY, gamma, beta, act="gelu_tanh"):
     (300, 264, 1200, 3),     # ragged rows (also the K of the weight-gradient GEMMs), ragged K, shard width 400
     (129, 512, 2048, 8),
     (520, 1000, 2016, 2),
+    (72, 6144, 1024, 2),     # LayerNorm backward with 2 chunks per thread
+    (40, 12288, 512, 1),     # 3 chunks per thread (one row in flight)
+    (24, 16384, 256, 1),     # 4 chunks per thread, the largest row
 ])
 def test_backward_small(cuda_device, S, H, F, t):
     inp = synth.gen_mlp(S, H, F, seed=S + F, dtype=torch.bfloat16)

@@ -122,6 +122,11 @@ struct GemmArgs {
   // C = acc * Act'(U), with U read from `aux` (bf16, row stride ld_aux, same
   // columns as C) — the backward of the activation fused into the GEMM.
   int epi_mode;
+  // Output rows split into shards of m_split_rows rows (0: off; a multiple
+  // of the tile height): rows [s m_split_rows, (s+1) m_split_rows) go through
+  // tmC[s] (its own buffer) at row offset 0 — the weight gradients G^T dZ of
+  // all shards in one launch.
+  int m_split_rows;
   CUtensorMap tmAux[MAX_SHARDS];
   const void* aux;
   long long ld_aux;
@@ -569,9 +574,11 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
     for (int unit = cluster_id; unit < num_units; unit += num_clusters) {
       const TileCoord tc = tile_coord<CG>(p, unit % num_tiles);
       const int split = unit / num_tiles;
-      const CUtensorMap* tmC = &p.tmC[p.row_mode ? 0 : tc.shard];
-      const CUtensorMap* tmAux = &p.tmAux[p.row_mode ? 0 : tc.shard];
       const int y0 = tc.m0 + static_cast<int>(rank) * C::BM;
+      const int mshard = p.m_split_rows ? tc.m0 / p.m_split_rows : 0;
+      const int ystore = y0 - mshard * p.m_split_rows;
+      const CUtensorMap* tmC = &p.tmC[p.m_split_rows ? mshard : (p.row_mode ? 0 : tc.shard)];
+      const CUtensorMap* tmAux = &p.tmAux[p.row_mode ? 0 : tc.shard];
       // All 128 epilogue threads take the same decision (they meet at named
       // barriers below).
       if (!named_barrier_and(1, 128, mbar_wait(&tfull[acc], acc_phase))) break;
@@ -624,7 +631,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
           named_barrier_sync(1, 128);
           if (elected && y0 < p.M) {
             const CUtensorMap* map = part < parts - 1 ? tmAux : tmC;
-            tma_store_3d(map, sEpi + buf * C::EPI_BUF_BYTES, tc.n_in + c * cw, y0, split);
+            tma_store_3d(map, sEpi + buf * C::EPI_BUF_BYTES, tc.n_in + c * cw, ystore, split);
             bulk_commit_group();
           }
           buf ^= 1;

@@ -263,6 +263,8 @@ struct GemmExtra {
   int epi_mode = tp::EPI_PLAIN;
   const void* aux = nullptr;         // EPI_AUX_PRE: bf16 output laid out like C; EPI_GRAD: bf16 U
   long long ld_aux = 0;
+  int m_split = 0;                   // column mode, t = 1: output rows split into m_split buffers
+                                     // C_shards[s] of M / m_split rows each (a multiple of 256)
 };
 
 template <int CG, bool WIDE>
@@ -279,7 +281,12 @@ int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, const TilePlan& plan,
   const int slots = CG == 2 ? dev.max_pairs : dev.sm_count;
   p.splits = plan.splits;
   const long long es = p.out_f32 ? 4 : 2;
-  if (p.row_mode) {
+  if (ex.m_split > 0) {
+    p.m_split_rows = p.M / ex.m_split;
+    for (int s = 0; s < ex.m_split; ++s)
+      if (!tmap_out(&p.tmC[s], ex.C_shards[s], p.out_f32, p.shard_n, p.m_split_rows, 1, ex.ldc_shard, 0))
+        return TP_ERR_CUDA;
+  } else if (p.row_mode) {
     if (!tmap_out(&p.tmC[0], p.C, p.out_f32, p.shard_n, p.M, p.splits, p.ldc, p.slot_stride)) return TP_ERR_CUDA;
   } else {
     for (int s = 0; s < p.t; ++s) {
@@ -824,9 +831,20 @@ int tp_mlp_backward(int S, int H, int F, int t, int dtype, const void* X, const 
     st = run_gemm_tc(*dev, X, H, H, dU_sh, t, 0, S, Fs, nullptr, Fs, 1, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
     if (st != TP_OK) return st;
   }
-  //    dB_i = G_i^T dZ: A operand the column slice i of G read M-major.
+  //    dB_i = G_i^T dZ: G read M-major.  When every shard's F/t rows are whole
+  //    256-row tiles, all shards go in one launch of G^T dZ [F, H] whose
+  //    epilogue sends rows of shard i to dB_i; otherwise one launch per shard
+  //    on G's column slice i.
+  const void* dz1[1] = {dZ};
+  if (t > 1 && Fs % 256 == 0) {  // F >= 512 rows: the CTA-pair GEMM with 256-row tiles
+    GemmExtra ex;
+    ex.a_mnmajor = 1;
+    ex.m_split = t;
+    ex.C_shards = dB_shards;
+    ex.ldc_shard = H;
+    return run_gemm_tc(*dev, G, F, F, dz1, 1, 0, S, H, nullptr, H, 1, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
+  }
   for (int i = 0; i < t; ++i) {
-    const void* dz1[1] = {dZ};
     GemmExtra ex;
     ex.a_mnmajor = 1;
     st = run_gemm_tc(*dev, G + static_cast<size_t>(i) * Fs * 2, F, Fs, dz1, 1, 0, S, H, dB_shards[i], H, 1,

@@ -39,6 +39,7 @@ def metric_for(w) -> str:
     return METRIC_TRAIN if w.kind == "mlp_train" else METRIC
 UNIT = "TFLOP/s"
 L2_BYTES = 126 * 2**20
+PROFILE_EVERY = 8  # steps between the timed region's per-kernel event samples
 
 
 def parse():
@@ -297,12 +298,17 @@ def run_ours(args, rank, world, local):
         step()
     barrier()
     # ---- timed region: K steps, device time on the launching stream
+    # Per-kernel durations come from CUDA events the library records around its
+    # launches on every PROFILE_EVERY-th step of the timed region; the other
+    # steps run without events between their kernels (which would break the
+    # programmatic dependent launch between them).  Every launch is counted.
     L.profile_enable(True)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     t_wall0 = time.time()
     e0.record(stream)
-    for _ in range(args.steps):
+    for i in range(args.steps):
+        L.profile_sample(i % PROFILE_EVERY == 0)
         step()
     e1.record(stream)
     barrier()

@@ -296,6 +296,12 @@ int tp_selftest_wait_timeout(long long limit_cycles, void* stream);
  * launch and collect from one host thread. */
 int tp_profile_enable(int on);
 int tp_profile_collect(int* launches, int* timed, double* ms, int max_kinds);
+/* While profiling is enabled: on = 0 stops recording events for the
+ * following launches (they are still counted), on = 1 resumes.  Events sit in
+ * the stream between launches, so sampling a subset of launches leaves the
+ * others running back to back (programmatic dependent launch).  Enabling
+ * profiling resumes recording. */
+int tp_profile_sample(int on);
 const char* tp_kernel_kind_name(int kind);
 
 #ifdef __cplusplus

@@ -57,6 +57,7 @@ SIGNATURES = {
     "tp_set_gemm_tile_n": (_c_int, [_c_int]),
     "tp_selftest_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
     "tp_profile_enable": (_c_int, [_c_int]),
+    "tp_profile_sample": (_c_int, [_c_int]),
     "tp_profile_collect": (_c_int, [ctypes.POINTER(_c_int), ctypes.POINTER(_c_int), ctypes.POINTER(ctypes.c_double),
                                     _c_int]),
     "tp_kernel_kind_name": (ctypes.c_char_p, [_c_int]),
@@ -267,6 +268,10 @@ def device_error() -> int:
 
 def profile_enable(on: bool):
     _check(lib().tp_profile_enable(1 if on else 0), "tp_profile_enable")
+
+
+def profile_sample(on: bool):
+    _check(lib().tp_profile_sample(1 if on else 0), "tp_profile_sample")
 
 
 def profile_collect(nkinds: int = 5):

@@ -391,6 +391,11 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
   else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // The prologue above touched no global memory: only now wait for the
+  // preceding kernel (whose output may be A, or whose inputs C may overwrite),
+  // and let the next kernel start its own prologue as SMs free up.
+  griddep_wait();
+  griddep_launch_dependents();
 
   const int num_tiles = p.m_blocks * p.n_blocks;
   const int num_units = num_tiles * p.splits;

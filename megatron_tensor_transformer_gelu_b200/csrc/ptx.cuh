@@ -184,6 +184,15 @@ __device__ __forceinline__ bool named_barrier_and(int id, int count, bool v) {
 }
 
 // Barrier among `count` threads (multiple of 32) on hardware barrier `id`.
+// Programmatic dependent launch.  griddep_wait: block until the preceding
+// kernel in the stream has completed and its memory is visible (a no-op when
+// this kernel was launched without programmatic stream serialization);
+// griddep_launch_dependents: let the next kernel in the stream be scheduled
+// before this one ends (it still waits for this kernel's completion in its
+// own griddep_wait before touching its inputs).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 __device__ __forceinline__ void named_barrier_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }

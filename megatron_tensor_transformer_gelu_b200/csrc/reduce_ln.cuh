@@ -17,6 +17,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "ptx.cuh"
+
 namespace tp {
 
 namespace rln {
@@ -105,6 +107,8 @@ __global__ void __launch_bounds__(rln::cta_threads(WPR)) reduce_residual_ln_kern
   __shared__ float red[2][RPC][WPR];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rloc = warp / WPR, wr = warp % WPR;
+  griddep_wait();  // the partial sums come from the preceding kernel
+  griddep_launch_dependents();
   const int groups = (p.S + RPC - 1) / RPC;
   for (int g = blockIdx.x; g < groups; g += gridDim.x) {
     const long long row = static_cast<long long>(g) * RPC + rloc;

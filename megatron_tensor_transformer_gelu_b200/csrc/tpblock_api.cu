@@ -51,6 +51,7 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 constexpr int PROF_CAP = 16384;  // launches timed between two collects
 constexpr int PROF_KINDS = 5;
 bool g_prof_on = false;
+bool g_prof_sampling = true;  // record events for the launches made while set
 bool g_prof_events_made = false;
 cudaEvent_t g_ev_start[PROF_CAP];
 cudaEvent_t g_ev_stop[PROF_CAP];
@@ -66,7 +67,7 @@ struct ProfScope {
   ProfScope(int kind, cudaStream_t s) : st(s) {
     if (!g_prof_on) return;
     ++g_prof_launches[kind];
-    if (g_prof_n >= PROF_CAP) return;
+    if (!g_prof_sampling || g_prof_n >= PROF_CAP) return;
     slot = g_prof_n++;
     g_prof_kind[slot] = kind;
     cudaEventRecord(g_ev_start[slot], st);
@@ -302,17 +303,19 @@ int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, const TilePlan& plan,
   const long long units = tiles * p.splits;
   const int clusters = static_cast<int>(units < slots ? units : slots);
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = CG;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see griddep_wait in the kernel
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;
+  at[1].val.clusterDim.x = CG;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = 1;
   cfg.gridDim = dim3(clusters * CG, 1, 1);
   cfg.blockDim = dim3(C::NUM_THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = st;
   cfg.attrs = at;
-  cfg.numAttrs = CG == 2 ? 1 : 0;
+  cfg.numAttrs = CG == 2 ? 2 : 1;
   ProfScope ps(K_GEMM_TC, st);
   if (cudaLaunchKernelEx(&cfg, tp::gemm_tcgen05_kernel<CG, WIDE>, p) != cudaSuccess) return TP_ERR_CUDA;
   return launch_status();
@@ -435,7 +438,16 @@ int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, i
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, threads, 0) != cudaSuccess || per_sm < 1)
       per_sm = 1;
     const int grid = groups < per_sm * dev_sms ? groups : per_sm * dev_sms;
-    kern<<<grid, threads, 0, st>>>(p);
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see griddep_wait in the kernel
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(threads, 1, 1);
+    cfg.stream = st;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kern, p);
   };
   using namespace tp;
   if (H <= 512) np1 ? go(reduce_residual_ln_kernel<1, 2, true>, 1, 8) : go(reduce_residual_ln_kernel<1, 2, false>, 1, 8);
@@ -1042,8 +1054,14 @@ int tp_profile_enable(int on) {
     g_prof_events_made = true;
   }
   g_prof_on = on != 0;
+  g_prof_sampling = true;
   g_prof_n = 0;
   for (int k = 0; k < PROF_KINDS; ++k) g_prof_launches[k] = 0;
+  return TP_OK;
+}
+
+int tp_profile_sample(int on) {
+  g_prof_sampling = on != 0;
   return TP_OK;
 }
 

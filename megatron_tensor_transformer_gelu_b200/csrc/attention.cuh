@@ -118,6 +118,8 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  griddep_wait();  // Q, K and V come from the preceding kernel
+  griddep_launch_dependents();
 
   if (warp == 0 || warp == 10) {
     // ---------------------------------------------- producers (Q + K, V)

@@ -15,6 +15,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include "ptx.cuh"
+
 namespace tp {
 
 namespace lnb {
@@ -96,6 +98,8 @@ __device__ __forceinline__ void lnb_block_sum3(float& a, float& b, float& c, flo
 template <int CH>
 __global__ void __launch_bounds__(512) ln_backward_kernel(const LnBackArgs p) {
   __shared__ float red[3 * lnb::MAX_WARPS];
+  griddep_wait();  // V and dY come from preceding kernels
+  griddep_launch_dependents();
   const int nthr = blockDim.x;
   float z[CH][8], dg[CH][8], db[CH][8];
 #pragma unroll
@@ -199,6 +203,8 @@ __global__ void __launch_bounds__(32 * LNB_PARAM_SLICES)
     ln_grad_params_kernel(const float* partial, int nblk, int H, float* dgamma, float* dbeta) {
   __shared__ float sa[LNB_PARAM_SLICES][33], sb[LNB_PARAM_SLICES][33];
   const int lane = threadIdx.x & 31, slice = threadIdx.x >> 5;
+  griddep_wait();  // the partial rows come from the preceding kernel
+  griddep_launch_dependents();
   const int j = blockIdx.x * 32 + lane;
   float a[4] = {0.0f, 0.0f, 0.0f, 0.0f}, b[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   if (j < H) {

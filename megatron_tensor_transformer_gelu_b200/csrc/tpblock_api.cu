@@ -11,6 +11,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "../../include/tpblock.h"
 #include "attention.cuh"
@@ -174,6 +175,24 @@ bool tmap_out(CUtensorMap* m, void* base, int f32, long long cols, long long row
 }
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_CUDA; }
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// before the preceding kernel in the stream ends and waits for it itself
+// (griddep_wait) before touching data that kernel produced.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Tile plan of a tensor-core GEMM: tile width (256, or 288..512 for wide
 // tiles) and number of K splits, from a small cost model of a persistent
@@ -540,16 +559,17 @@ int run_ln_backward(int S, int H, const float* V, const void* X, const void* dY,
   {
     ProfScope ps(K_LN_BACK, st);
     switch (ch) {
-      case 1: tp::ln_backward_kernel<1><<<grid, threads, 0, st>>>(p); break;
-      case 2: tp::ln_backward_kernel<2><<<grid, threads, 0, st>>>(p); break;
-      case 3: tp::ln_backward_kernel<3><<<grid, threads, 0, st>>>(p); break;
-      default: tp::ln_backward_kernel<4><<<grid, threads, 0, st>>>(p); break;
+      case 1: launch_pdl(tp::ln_backward_kernel<1>, dim3(grid), dim3(threads), 0, st, p); break;
+      case 2: launch_pdl(tp::ln_backward_kernel<2>, dim3(grid), dim3(threads), 0, st, p); break;
+      case 3: launch_pdl(tp::ln_backward_kernel<3>, dim3(grid), dim3(threads), 0, st, p); break;
+      default: launch_pdl(tp::ln_backward_kernel<4>, dim3(grid), dim3(threads), 0, st, p); break;
     }
     if (launch_status() != TP_OK) return TP_ERR_CUDA;
   }
   if (dgamma || dbeta) {
     ProfScope ps(K_LN_BACK, st);
-    tp::ln_grad_params_kernel<<<ceil_div(H, 32), 32 * tp::LNB_PARAM_SLICES, 0, st>>>(partial, grid, H, dgamma, dbeta);
+    launch_pdl(tp::ln_grad_params_kernel, dim3(ceil_div(H, 32)), dim3(32 * tp::LNB_PARAM_SLICES), 0, st,
+               static_cast<const float*>(partial), grid, H, dgamma, dbeta);
     return launch_status();
   }
   return TP_OK;
@@ -665,7 +685,7 @@ int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
     dim3 grid((S + tp::attn::TILES * tp::attn::BQ - 1) / (tp::attn::TILES * tp::attn::BQ), nh);
     ProfScope ps(K_ATTN, s);
-    tp::attn_fwd_kernel<<<grid, tp::attn::NUM_THREADS, tp::attn::SMEM_BYTES, s>>>(a);
+    launch_pdl(tp::attn_fwd_kernel, grid, dim3(tp::attn::NUM_THREADS), tp::attn::SMEM_BYTES, s, a);
     st = launch_status();
     if (st != TP_OK) return st;
   }

@@ -180,7 +180,8 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? TP_OK : TP_ERR_
 // before the preceding kernel in the stream ends and waits for it itself
 // (griddep_wait) before touching data that kernel produced.
 template <typename... KArgs, typename... Args>
-void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute at[1];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -191,7 +192,7 @@ void launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cuda
   cfg.stream = st;
   cfg.attrs = at;
   cfg.numAttrs = 1;
-  cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // Tile plan of a tensor-core GEMM: tile width (256, or 288..512 for wide
@@ -446,6 +447,7 @@ int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, i
   p.eps = eps;
   p.Y = Y;
   p.y_bf16 = y_bf16;
+  bool launched = true;
   // WPR warps per row (each lane holds CH chunks of 8 values); max(1, 8 / WPR)
   // rows per CTA; a grid of the resident CTA count walks the row groups.
   ProfScope ps(K_REDUCE_LN, st);
@@ -466,7 +468,7 @@ int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, i
     cfg.stream = st;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, kern, p);
+    if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) launched = false;
   };
   using namespace tp;
   if (H <= 512) np1 ? go(reduce_residual_ln_kernel<1, 2, true>, 1, 8) : go(reduce_residual_ln_kernel<1, 2, false>, 1, 8);
@@ -477,7 +479,8 @@ int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, i
   // (one-row CTAs of 12 or 16 warps keep the generic loop: fewer registers, two CTAs per SM)
   else if (H <= 12288) go(reduce_residual_ln_kernel<12, 4, false>, 12, 1);
   else go(reduce_residual_ln_kernel<16, 4, false>, 16, 1);
-  return launch_status();
+  const int ls = launch_status();
+  return launched ? ls : TP_ERR_CUDA;
 }
 
 bool valid_dtype(int d) { return d == TP_DTYPE_F32 || d == TP_DTYPE_BF16; }
@@ -558,19 +561,21 @@ int run_ln_backward(int S, int H, const float* V, const void* X, const void* dY,
   if (grid < 1) grid = 1;
   {
     ProfScope ps(K_LN_BACK, st);
+    cudaError_t le;
     switch (ch) {
-      case 1: launch_pdl(tp::ln_backward_kernel<1>, dim3(grid), dim3(threads), 0, st, p); break;
-      case 2: launch_pdl(tp::ln_backward_kernel<2>, dim3(grid), dim3(threads), 0, st, p); break;
-      case 3: launch_pdl(tp::ln_backward_kernel<3>, dim3(grid), dim3(threads), 0, st, p); break;
-      default: launch_pdl(tp::ln_backward_kernel<4>, dim3(grid), dim3(threads), 0, st, p); break;
+      case 1: le = launch_pdl(tp::ln_backward_kernel<1>, dim3(grid), dim3(threads), 0, st, p); break;
+      case 2: le = launch_pdl(tp::ln_backward_kernel<2>, dim3(grid), dim3(threads), 0, st, p); break;
+      case 3: le = launch_pdl(tp::ln_backward_kernel<3>, dim3(grid), dim3(threads), 0, st, p); break;
+      default: le = launch_pdl(tp::ln_backward_kernel<4>, dim3(grid), dim3(threads), 0, st, p); break;
     }
-    if (launch_status() != TP_OK) return TP_ERR_CUDA;
+    if (le != cudaSuccess || launch_status() != TP_OK) return TP_ERR_CUDA;
   }
   if (dgamma || dbeta) {
     ProfScope ps(K_LN_BACK, st);
-    launch_pdl(tp::ln_grad_params_kernel, dim3(ceil_div(H, 32)), dim3(32 * tp::LNB_PARAM_SLICES), 0, st,
-               static_cast<const float*>(partial), grid, H, dgamma, dbeta);
-    return launch_status();
+    const cudaError_t le = launch_pdl(tp::ln_grad_params_kernel, dim3(ceil_div(H, 32)),
+                                      dim3(32 * tp::LNB_PARAM_SLICES), 0, st, static_cast<const float*>(partial),
+                                      grid, H, dgamma, dbeta);
+    return le != cudaSuccess ? TP_ERR_CUDA : launch_status();
   }
   return TP_OK;
 }
@@ -685,8 +690,9 @@ int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
     dim3 grid((S + tp::attn::TILES * tp::attn::BQ - 1) / (tp::attn::TILES * tp::attn::BQ), nh);
     ProfScope ps(K_ATTN, s);
-    launch_pdl(tp::attn_fwd_kernel, grid, dim3(tp::attn::NUM_THREADS), tp::attn::SMEM_BYTES, s, a);
-    st = launch_status();
+    st = launch_pdl(tp::attn_fwd_kernel, grid, dim3(tp::attn::NUM_THREADS), tp::attn::SMEM_BYTES, s, a) != cudaSuccess
+             ? TP_ERR_CUDA
+             : launch_status();
     if (st != TP_OK) return st;
   }
   // sum_s O_s Wo_s, the O projection row-split by head, summed in TMEM.

@@ -67,6 +67,8 @@ def check(out, inp, dY, gamma, beta, act="gelu_tanh"):
     (72, 6144, 1024, 2),     # LayerNorm backward with 2 chunks per thread
     (40, 12288, 512, 1),     # 3 chunks per thread (one row in flight)
     (24, 16384, 256, 1),     # 4 chunks per thread, the largest row
+    (64, 64, 256, 2),        # every GEMM in single-CTA form (M <= 128), M-major A included
+    (130, 64, 512, 2),       # weight gradients single-CTA, dU / dX in CTA pairs with a ragged tile
 ])
 def test_backward_small(cuda_device, S, H, F, t):
     inp = synth.gen_mlp(S, H, F, seed=S + F, dtype=torch.bfloat16)

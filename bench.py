@@ -448,7 +448,7 @@ def run_ours(args, rank, world, local):
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
-    return result
+    return result, (Y if rank == 0 else None)
 
 
 # -------------------------------------------------- oracle on host cores
@@ -489,7 +489,7 @@ def cpu_oracle_timing(w, rows_per_step: int, steps: int, warmup: int):
         call(rows)
     t0 = time.perf_counter()
     for _ in range(steps):
-        call(rows)
+        out = call(rows)
     dt = time.perf_counter() - t0
     flops = w.flops * len(rows) / nrows * steps
     return {"value": round(flops / dt / 1e12, 5), "unit": UNIT, "cores": int(cores), "kind": "oracle",
@@ -497,7 +497,19 @@ def cpu_oracle_timing(w, rows_per_step: int, steps: int, warmup: int):
                        f"per step, {steps} step(s), "
                        "fp64 numpy/OpenBLAS" + ("; every call also computes all K and V rows"
                                                 if w.kind == "attn" else "")),
-            "seconds": round(dt, 3)}
+            "seconds": round(dt, 3), "_rows": rows, "_out": out}
+
+
+def parity_vs_oracle(w, Y, rows, ref, tol: float = 2e-2):
+    """max|GPU - oracle| / max|oracle| over the oracle's sample rows: the
+    output the timed loop left (Y; dX for the training step) against the
+    baseline run's fp64 result on the same seeded inputs."""
+    import numpy as np
+    ref = np.asarray(ref["dX"] if isinstance(ref, dict) else ref, dtype=np.float64)
+    got = Y[list(rows)].double().cpu().numpy()
+    err = float(np.abs(got - ref).max() / np.abs(ref).max())
+    return {"rows": len(rows), "max_rel_err": err, "tol": tol, "pass": err <= tol,
+            "compared": "dX" if w.kind == "mlp_train" else "Y"}
 
 
 def run_reference(args, rank, world):
@@ -536,14 +548,16 @@ def main():
         if res is not None:
             print(json.dumps(res), flush=True)
         return
-    res = run_ours(args, rank, world, local)
+    res, Y = run_ours(args, rank, world, local)
     if rank == 0 and res is not None:
         from megatron_tensor_transformer_gelu_b200.workloads import HEADLINE, WORKLOADS
         if not args.no_cpu_baseline:
             w = WORKLOADS[args.workload or HEADLINE]
             rows = {"mlp": args.cpu_sample_rows, "mlp_train": min(args.cpu_sample_rows, 256)}.get(
                 w.kind, min(args.cpu_sample_rows, 64))
-            res["cpu_baseline"] = cpu_oracle_timing(w, rows, 1, 0)
+            cb = cpu_oracle_timing(w, rows, 1, 0)
+            res["parity"] = parity_vs_oracle(w, Y, cb.pop("_rows"), cb.pop("_out"))
+            res["cpu_baseline"] = cb
         print(json.dumps(res), flush=True)
 
 

@@ -159,6 +159,19 @@ int tp_mlp_backward(int S, int H, int F, int t, int dtype, const void* X,
                     const float* gamma, float eps, int act, const void* state, size_t state_bytes,
                     const void* dY, void* dX, void* const* dA_shards, void* const* dB_shards,
                     float* dgamma, float* dbeta, void* workspace, size_t workspace_bytes, void* stream);
+/* The same with a weight layout.  For TP_W_OUT_IN the weight shards are
+ * [out, in] (A_shards[i] [F/t, H], B_shards[i] [H, F/t]) and so are their
+ * gradients (dA_shards[i] [F/t, H], dB_shards[i] [H, F/t]); the state of a
+ * tp_mlp_forward_train_ex call with the same layout. */
+int tp_mlp_forward_train_ex(int S, int H, int F, int t, int dtype, int out_dtype, int w_layout, const void* X,
+                            const void* const* A_shards, const void* const* B_shards,
+                            const float* gamma, const float* beta, float eps, int act,
+                            void* Y, void* state, size_t state_bytes, void* stream);
+int tp_mlp_backward_ex(int S, int H, int F, int t, int dtype, int w_layout, const void* X,
+                       const void* const* A_shards, const void* const* B_shards,
+                       const float* gamma, float eps, int act, const void* state, size_t state_bytes,
+                       const void* dY, void* dX, void* const* dA_shards, void* const* dB_shards,
+                       float* dgamma, float* dbeta, void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------- MLP without allocation ----
  * The pages have no counterpart to this entry point: it exists for callers

@@ -51,6 +51,10 @@ SIGNATURES = {
     "tp_mlp_train_state_bytes": (_c_size, [_c_int] * 5),
     "tp_mlp_forward_train": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vpp, _vp, _vp, _c_float, _c_int, _vp, _vp, _c_size,
                                                       _vp]),
+    "tp_mlp_forward_train_ex": (_c_int, [_c_int] * 7 + [_vp, _vpp, _vpp, _vp, _vp, _c_float, _c_int, _vp, _vp,
+                                                         _c_size, _vp]),
+    "tp_mlp_backward_ex": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vpp, _vp, _c_float, _c_int, _vp, _c_size, _vp, _vp,
+                                                    _vpp, _vpp, _vp, _vp, _vp, _c_size, _vp]),
     "tp_mlp_backward_workspace_bytes": (_c_size, [_c_int] * 5),
     "tp_mlp_backward": (_c_int, [_c_int] * 5 + [_vp, _vpp, _vpp, _vp, _c_float, _c_int, _vp, _c_size, _vp, _vp, _vpp,
                                                  _vpp, _vp, _vp, _vp, _c_size, _vp]),
@@ -225,31 +229,32 @@ def mlp_backward_workspace_bytes(S, H, F, t, dtype=torch.bfloat16) -> int:
 
 
 def mlp_forward_train(X, A_shards, B_shards, Y, state, gamma=None, beta=None, eps=1e-5, act="gelu_tanh",
-                      stream=None):
+                      stream=None, layout="in_out"):
     S, H = X.shape
     t = len(A_shards)
-    F = sum(a.shape[1] for a in A_shards)
+    F = sum(a.shape[1 if layout == "in_out" else 0] for a in A_shards)
     pa, ka = _ptrs(A_shards)
     pb, kb = _ptrs(B_shards)
-    code = lib().tp_mlp_forward_train(S, H, F, t, DTYPE[X.dtype], DTYPE[Y.dtype], _ptr(X), pa, pb, _ptr(gamma),
-                                      _ptr(beta), float(eps), ACT[act], _ptr(Y), _ptr(state),
-                                      state.numel() * state.element_size(), _stream(stream))
+    code = lib().tp_mlp_forward_train_ex(S, H, F, t, DTYPE[X.dtype], DTYPE[Y.dtype], LAYOUT[layout], _ptr(X), pa, pb,
+                                         _ptr(gamma), _ptr(beta), float(eps), ACT[act], _ptr(Y), _ptr(state),
+                                         state.numel() * state.element_size(), _stream(stream))
     _check(code, "tp_mlp_forward_train")
 
 
 def mlp_backward(X, A_shards, B_shards, state, dY, dX, dA_shards, dB_shards, workspace, gamma=None, dgamma=None,
-                 dbeta=None, eps=1e-5, act="gelu_tanh", stream=None):
+                 dbeta=None, eps=1e-5, act="gelu_tanh", stream=None, layout="in_out"):
+    """Gradients of one tp_mlp_forward_train call; dA/dB shards have the weights' layout."""
     S, H = X.shape
     t = len(A_shards)
-    F = sum(a.shape[1] for a in A_shards)
+    F = sum(a.shape[1 if layout == "in_out" else 0] for a in A_shards)
     pa, ka = _ptrs(A_shards)
     pb, kb = _ptrs(B_shards)
     pda, kda = _ptrs(dA_shards)
     pdb, kdb = _ptrs(dB_shards)
-    code = lib().tp_mlp_backward(S, H, F, t, DTYPE[X.dtype], _ptr(X), pa, pb, _ptr(gamma), float(eps), ACT[act],
-                                 _ptr(state), state.numel() * state.element_size(), _ptr(dY), _ptr(dX), pda, pdb,
-                                 _ptr(dgamma), _ptr(dbeta), _ptr(workspace),
-                                 workspace.numel() * workspace.element_size(), _stream(stream))
+    code = lib().tp_mlp_backward_ex(S, H, F, t, DTYPE[X.dtype], LAYOUT[layout], _ptr(X), pa, pb, _ptr(gamma),
+                                    float(eps), ACT[act], _ptr(state), state.numel() * state.element_size(),
+                                    _ptr(dY), _ptr(dX), pda, pdb, _ptr(dgamma), _ptr(dbeta), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream))
     _check(code, "tp_mlp_backward")
 
 

@@ -772,6 +772,15 @@ int tp_mlp_forward_train(int S, int H, int F, int t, int dtype, int out_dtype, c
                          const void* const* A_shards, const void* const* B_shards, const float* gamma,
                          const float* beta, float eps, int act, void* Y, void* state, size_t state_bytes,
                          void* stream) {
+  return tp_mlp_forward_train_ex(S, H, F, t, dtype, out_dtype, TP_W_IN_OUT, X, A_shards, B_shards, gamma, beta, eps,
+                                 act, Y, state, state_bytes, stream);
+}
+
+int tp_mlp_forward_train_ex(int S, int H, int F, int t, int dtype, int out_dtype, int w_layout, const void* X,
+                            const void* const* A_shards, const void* const* B_shards, const float* gamma,
+                            const float* beta, float eps, int act, void* Y, void* state, size_t state_bytes,
+                            void* stream) {
+  if (w_layout != TP_W_IN_OUT && w_layout != TP_W_OUT_IN) return TP_ERR_INVALID_ARG;
   if (dtype != TP_DTYPE_BF16) return TP_ERR_UNSUPPORTED_SHAPE;
   int st = check_mlp_args(S, H, F, t, dtype, out_dtype, X, A_shards, B_shards, gamma, beta, eps, act, Y);
   if (st != TP_OK) return st;
@@ -794,10 +803,11 @@ int tp_mlp_forward_train(int S, int H, int F, int t, int dtype, int out_dtype, c
   ex.epi_mode = tp::EPI_AUX_PRE;
   ex.aux = U;
   ex.ld_aux = F;
-  st = run_gemm_tc(*dev, X, H, S, A_shards, t, 0, H, Fs, G, F, 0, act, s, 1, 0, nullptr, 0, &ex);
+  const int kmaj = w_layout == TP_W_OUT_IN;
+  st = run_gemm_tc(*dev, X, H, S, A_shards, t, 0, H, Fs, G, F, 0, act, s, 1, 0, nullptr, kmaj, &ex);
   if (st != TP_OK) return st;
   // V = sum_i G_i B_i in one f32 slot (no K split: the backward reads one).
-  st = run_gemm_tc(*dev, G, F, S, B_shards, t, 1, Fs, H, V, H, 1, TP_ACT_NONE, s, 1, 0, nullptr, 0);
+  st = run_gemm_tc(*dev, G, F, S, B_shards, t, 1, Fs, H, V, H, 1, TP_ACT_NONE, s, 1, 0, nullptr, kmaj);
   if (st != TP_OK) return st;
   return run_reduce_ln(S, H, 1, V, X, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s, dev->sm_count);
 }
@@ -811,6 +821,17 @@ int tp_mlp_backward(int S, int H, int F, int t, int dtype, const void* X, const 
                     const void* const* B_shards, const float* gamma, float eps, int act, const void* state,
                     size_t state_bytes, const void* dY, void* dX, void* const* dA_shards, void* const* dB_shards,
                     float* dgamma, float* dbeta, void* workspace, size_t workspace_bytes, void* stream) {
+  return tp_mlp_backward_ex(S, H, F, t, dtype, TP_W_IN_OUT, X, A_shards, B_shards, gamma, eps, act, state,
+                            state_bytes, dY, dX, dA_shards, dB_shards, dgamma, dbeta, workspace, workspace_bytes,
+                            stream);
+}
+
+int tp_mlp_backward_ex(int S, int H, int F, int t, int dtype, int w_layout, const void* X,
+                       const void* const* A_shards, const void* const* B_shards, const float* gamma, float eps,
+                       int act, const void* state, size_t state_bytes, const void* dY, void* dX,
+                       void* const* dA_shards, void* const* dB_shards, float* dgamma, float* dbeta, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  if (w_layout != TP_W_IN_OUT && w_layout != TP_W_OUT_IN) return TP_ERR_INVALID_ARG;
   if (dtype != TP_DTYPE_BF16) return TP_ERR_UNSUPPORTED_SHAPE;
   int st = check_mlp_args(S, H, F, t, dtype, TP_DTYPE_BF16, X, A_shards, B_shards, gamma, nullptr, eps, act, dX);
   if (st != TP_OK) return st;
@@ -840,52 +861,65 @@ int tp_mlp_backward(int S, int H, int F, int t, int dtype, const void* X, const 
   // 1. Through the LayerNorm: dZ, dgamma, dbeta.
   st = run_ln_backward(S, H, V, X, dY, gamma, eps, dZ, part, dgamma, dbeta, s, dev->sm_count);
   if (st != TP_OK) return st;
+  // In [out, in] storage (TP_W_OUT_IN) every weight is the transpose of its
+  // [in, out] form: the backward reads B_i and A_i with the other majorness,
+  // and each weight gradient is the transpose of the [in, out] one, computed
+  // with the operands' roles swapped (dA_i^T = dU_i^T X, dB_i^T = dZ^T G_i).
+  const bool oi = w_layout == TP_W_OUT_IN;
   // 2. Through V = G B and G = Act(U): dU_i = (dZ B_i^T) * Act'(U_i) into the
-  //    columns of shard i (B_i [Fs, H] is read K-major as B_i^T).
+  //    columns of shard i.
   {
     GemmExtra ex;
     ex.epi_mode = tp::EPI_GRAD;
     ex.aux = U;
     ex.ld_aux = F;
-    st = run_gemm_tc(*dev, dZ, H, S, B_shards, t, 0, H, Fs, dU, F, 0, act, s, 1, 0, nullptr, 1, &ex);
+    st = run_gemm_tc(*dev, dZ, H, S, B_shards, t, 0, H, Fs, dU, F, 0, act, s, 1, 0, nullptr, oi ? 0 : 1, &ex);
     if (st != TP_OK) return st;
   }
   // 3. Through U = X A and the residual: dX = dZ + sum_i dU_i A_i^T (row split
-  //    over the shards, A_i [H, Fs] read K-major), then the residual add.
-  st = run_gemm_tc(*dev, dU, F, S, A_shards, t, 1, Fs, H, dXp, H, 1, TP_ACT_NONE, s, 1, 0, nullptr, 1);
+  //    over the shards), then the residual add.
+  st = run_gemm_tc(*dev, dU, F, S, A_shards, t, 1, Fs, H, dXp, H, 1, TP_ACT_NONE, s, 1, 0, nullptr, oi ? 0 : 1);
   if (st != TP_OK) return st;
   st = run_reduce_ln(S, H, 1, dXp, dZ, 1, nullptr, nullptr, 1.0f, dX, 1, s, dev->sm_count, /*apply_ln=*/0);
   if (st != TP_OK) return st;
-  // 4. Weight gradients, each with its own shard.  dA_i = X^T dU_i: A operand
-  //    X read M-major, B operand the column slice i of dU (row stride F).
+  // 4. Weight gradients, each with its own shard.  A column-mode launch on an
+  //    M-major A operand with strided B shards, or an M-split launch (all
+  //    shards' rows in one GEMM) when F/t is a multiple of 256, else one
+  //    launch per shard.
+  //    [in, out]: dA_i = X^T dU_i (column mode over dU's slices),
+  //               dB_i = G_i^T dZ (M-split over G's columns).
+  //    [out, in]: dB_i^T = dZ^T G_i (column mode over G's slices),
+  //               dA_i^T = dU_i^T X (M-split over dU's columns).
+  const uint8_t* colsrc = oi ? G : dU;     // the column-mode launch's strided B shards
+  const void* colA = oi ? dZ : X;          // ... and its M-major A ([S, H])
+  void* const* colOut = oi ? dB_shards : dA_shards;
+  const uint8_t* splitA = oi ? dU : G;     // the M-split launch's M-major A ([S, F])
+  const void* splitB = oi ? X : dZ;        // ... and its B ([S, H])
+  void* const* splitOut = oi ? dA_shards : dB_shards;
   {
-    const void* dU_sh[TP_MAX_SHARDS];
-    for (int i = 0; i < t; ++i) dU_sh[i] = dU + static_cast<size_t>(i) * Fs * 2;
+    const void* sh[TP_MAX_SHARDS];
+    for (int i = 0; i < t; ++i) sh[i] = colsrc + static_cast<size_t>(i) * Fs * 2;
     GemmExtra ex;
     ex.a_mnmajor = 1;
     ex.ldb = F;
-    ex.C_shards = dA_shards;
+    ex.C_shards = colOut;
     ex.ldc_shard = Fs;
-    st = run_gemm_tc(*dev, X, H, H, dU_sh, t, 0, S, Fs, nullptr, Fs, 1, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
+    st = run_gemm_tc(*dev, colA, H, H, sh, t, 0, S, Fs, nullptr, Fs, 1, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
     if (st != TP_OK) return st;
   }
-  //    dB_i = G_i^T dZ: G read M-major.  When every shard's F/t rows are whole
-  //    256-row tiles, all shards go in one launch of G^T dZ [F, H] whose
-  //    epilogue sends rows of shard i to dB_i; otherwise one launch per shard
-  //    on G's column slice i.
-  const void* dz1[1] = {dZ};
+  const void* b1[1] = {splitB};
   if (t > 1 && Fs % 256 == 0) {  // F >= 512 rows: the CTA-pair GEMM with 256-row tiles
     GemmExtra ex;
     ex.a_mnmajor = 1;
     ex.m_split = t;
-    ex.C_shards = dB_shards;
+    ex.C_shards = splitOut;
     ex.ldc_shard = H;
-    return run_gemm_tc(*dev, G, F, F, dz1, 1, 0, S, H, nullptr, H, 1, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
+    return run_gemm_tc(*dev, splitA, F, F, b1, 1, 0, S, H, nullptr, H, 1, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
   }
   for (int i = 0; i < t; ++i) {
     GemmExtra ex;
     ex.a_mnmajor = 1;
-    st = run_gemm_tc(*dev, G + static_cast<size_t>(i) * Fs * 2, F, Fs, dz1, 1, 0, S, H, dB_shards[i], H, 1,
+    st = run_gemm_tc(*dev, splitA + static_cast<size_t>(i) * Fs * 2, F, Fs, b1, 1, 0, S, H, splitOut[i], H, 1,
                      TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
     if (st != TP_OK) return st;
   }

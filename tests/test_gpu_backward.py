@@ -29,25 +29,30 @@ def rel_err(got, ref) -> float:
     return float(np.abs(got - ref).max() / np.abs(ref).max())
 
 
-def run_train_step(inp, t, dY, gamma, beta, act="gelu_tanh"):
+def run_train_step(inp, t, dY, gamma, beta, act="gelu_tanh", layout="in_out"):
     X = inp.X.cuda()
     S, H = X.shape
     F = inp.A.shape[1]
-    As = [a.cuda() for a in synth.split_columns(inp.A, t)]
-    Bs = [b.cuda() for b in synth.split_rows(inp.B, t)]
+    oi = layout == "out_in"
+    As = [(a.t().contiguous() if oi else a).cuda() for a in synth.split_columns(inp.A, t)]
+    Bs = [(b.t().contiguous() if oi else b).cuda() for b in synth.split_rows(inp.B, t)]
     g, b = gamma.cuda(), beta.cuda()
     Y = torch.empty(S, H, dtype=torch.bfloat16, device="cuda")
     state = torch.empty(L.mlp_train_state_bytes(S, H, F, t), dtype=torch.uint8, device="cuda")
-    L.mlp_forward_train(X, As, Bs, Y, state, gamma=g, beta=b, act=act)
+    L.mlp_forward_train(X, As, Bs, Y, state, gamma=g, beta=b, act=act, layout=layout)
     dX = torch.empty(S, H, dtype=torch.bfloat16, device="cuda")
-    dAs = [torch.empty(H, F // t, dtype=torch.float32, device="cuda") for _ in range(t)]
-    dBs = [torch.empty(F // t, H, dtype=torch.float32, device="cuda") for _ in range(t)]
+    dAs = [torch.empty(*(a.shape), dtype=torch.float32, device="cuda") for a in As]
+    dBs = [torch.empty(*(b.shape), dtype=torch.float32, device="cuda") for b in Bs]
     dg = torch.empty(H, dtype=torch.float32, device="cuda")
     db = torch.empty(H, dtype=torch.float32, device="cuda")
     ws = torch.empty(L.mlp_backward_workspace_bytes(S, H, F, t), dtype=torch.uint8, device="cuda")
-    L.mlp_backward(X, As, Bs, state, dY.cuda(), dX, dAs, dBs, ws, gamma=g, dgamma=dg, dbeta=db, act=act)
+    L.mlp_backward(X, As, Bs, state, dY.cuda(), dX, dAs, dBs, ws, gamma=g, dgamma=dg, dbeta=db, act=act,
+                   layout=layout)
     torch.cuda.synchronize()
     assert L.device_error() == 0
+    if oi:  # back to the [in, out] orientation the oracle uses
+        dAs = [d.t() for d in dAs]
+        dBs = [d.t() for d in dBs]
     return {"Y": Y, "dX": dX, "dA": torch.cat(dAs, dim=1), "dB": torch.cat(dBs, dim=0), "dgamma": dg, "dbeta": db}
 
 
@@ -74,6 +79,15 @@ def test_backward_small(cuda_device, S, H, F, t):
     inp = synth.gen_mlp(S, H, F, seed=S + F, dtype=torch.bfloat16)
     dY, g, b = synth.gen_upstream(S, H, seed=S)
     check(run_train_step(inp, t, dY, g, b), inp, dY, g, b)
+
+
+@pytest.mark.parametrize("S,H,F,t", [(256, 256, 1024, 2), (300, 264, 1200, 3), (64, 64, 256, 2)])
+def test_backward_out_in_layout(cuda_device, S, H, F, t):
+    """nn.Linear [out, in] weights and gradients: the M-split and per-shard
+    weight-gradient paths with the operands' roles swapped."""
+    inp = synth.gen_mlp(S, H, F, seed=S + 7, dtype=torch.bfloat16)
+    dY, g, b = synth.gen_upstream(S, H, seed=S + 8)
+    check(run_train_step(inp, t, dY, g, b, layout="out_in"), inp, dY, g, b)
 
 
 @pytest.mark.parametrize("act", ["gelu_erf", "relu", "none"])

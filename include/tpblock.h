@@ -242,6 +242,14 @@ int tp_transformer_block_forward(int S, int H, int F, int nh, int d, int t, int 
                                  const float* ln1_gamma, const float* ln1_beta,
                                  const float* ln2_gamma, const float* ln2_beta, float eps, int act,
                                  void* Y, void* workspace, size_t workspace_bytes, void* stream);
+/* The same with a weight layout (TP_W_OUT_IN: every shard [out, in], as in
+ * tp_qkv_attn_oproj_forward_ex and tp_mlp_forward_ex). */
+int tp_transformer_block_forward_ex(int S, int H, int F, int nh, int d, int t, int dtype, int out_dtype, int pre_ln,
+                                    int w_layout, const void* X, const void* const* Wqkv_shards,
+                                    const void* const* Wo_shards, const void* const* A_shards,
+                                    const void* const* B_shards, const float* ln1_gamma, const float* ln1_beta,
+                                    const float* ln2_gamma, const float* ln2_beta, float eps, int act, void* Y,
+                                    void* workspace, size_t workspace_bytes, void* stream);
 
 /* ------------------------------------------------------ single linears ----
  * Column-split linear ([TYPC] §2.1; [PWWT] §1.1 figure 1; [0539] §1.1 列切分):

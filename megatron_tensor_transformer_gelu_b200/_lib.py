@@ -39,6 +39,8 @@ SIGNATURES = {
     "tp_block_workspace_bytes": (_c_size, [_c_int] * 7),
     "tp_transformer_block_forward": (_c_int, [_c_int] * 9 + [_vp, _vpp, _vpp, _vpp, _vpp, _vp, _vp, _vp, _vp, _c_float,
                                                               _c_int, _vp, _vp, _c_size, _vp]),
+    "tp_transformer_block_forward_ex": (_c_int, [_c_int] * 10 + [_vp, _vpp, _vpp, _vpp, _vpp, _vp, _vp, _vp, _vp,
+                                                                  _c_float, _c_int, _vp, _vp, _c_size, _vp]),
     "tp_linear_column_forward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _c_int, _vp, _vp]),
     "tp_linear_column_forward_ex": (_c_int, [_c_int] * 7 + [_vp, _vpp, _c_int, _vp, _vp]),
     "tp_linear_row_forward_ex": (_c_int, [_c_int] * 7 + [_vp, _vpp, _vp, _vp, _c_size, _vp]),
@@ -175,17 +177,17 @@ def block_workspace_bytes(S, H, F, nh, d, t, dtype=torch.bfloat16) -> int:
 
 
 def block_forward(X, Wqkv_shards, Wo_shards, A_shards, B_shards, nh, d, Y, workspace, pre_ln=False,
-                  ln1=(None, None), ln2=(None, None), eps=1e-5, act="gelu_tanh", stream=None):
+                  ln1=(None, None), ln2=(None, None), eps=1e-5, act="gelu_tanh", stream=None, layout="in_out"):
     """Attention sublayer then MLP sublayer (post-LN, or pre-LN with pre_ln=True)."""
     S, H = X.shape
     t = len(Wqkv_shards)
-    F = sum(a.shape[1] for a in A_shards)
+    F = sum(a.shape[1 if layout == "in_out" else 0] for a in A_shards)
     pq, kq = _ptrs(Wqkv_shards)
     po, ko = _ptrs(Wo_shards)
     pa, ka = _ptrs(A_shards)
     pb, kb = _ptrs(B_shards)
-    code = lib().tp_transformer_block_forward(
-        S, H, F, nh, d, t, DTYPE[X.dtype], DTYPE[Y.dtype], 1 if pre_ln else 0, _ptr(X), pq, po, pa, pb,
+    code = lib().tp_transformer_block_forward_ex(
+        S, H, F, nh, d, t, DTYPE[X.dtype], DTYPE[Y.dtype], 1 if pre_ln else 0, LAYOUT[layout], _ptr(X), pq, po, pa, pb,
         _ptr(ln1[0]), _ptr(ln1[1]), _ptr(ln2[0]), _ptr(ln2[1]), float(eps), ACT[act], _ptr(Y), _ptr(workspace),
         workspace.numel() * workspace.element_size() if workspace is not None else 0, _stream(stream))
     _check(code, "tp_transformer_block_forward")

@@ -973,7 +973,20 @@ int tp_transformer_block_forward(int S, int H, int F, int nh, int d, int t, int 
                                  const void* const* A_shards, const void* const* B_shards, const float* ln1_gamma,
                                  const float* ln1_beta, const float* ln2_gamma, const float* ln2_beta, float eps,
                                  int act, void* Y, void* workspace, size_t workspace_bytes, void* stream) {
+  return tp_transformer_block_forward_ex(S, H, F, nh, d, t, dtype, out_dtype, pre_ln, TP_W_IN_OUT, X, Wqkv_shards,
+                                         Wo_shards, A_shards, B_shards, ln1_gamma, ln1_beta, ln2_gamma, ln2_beta, eps,
+                                         act, Y, workspace, workspace_bytes, stream);
+}
+
+int tp_transformer_block_forward_ex(int S, int H, int F, int nh, int d, int t, int dtype, int out_dtype, int pre_ln,
+                                    int w_layout, const void* X, const void* const* Wqkv_shards,
+                                    const void* const* Wo_shards, const void* const* A_shards,
+                                    const void* const* B_shards, const float* ln1_gamma, const float* ln1_beta,
+                                    const float* ln2_gamma, const float* ln2_beta, float eps, int act, void* Y,
+                                    void* workspace, size_t workspace_bytes, void* stream) {
   if (pre_ln != 0 && pre_ln != 1) return TP_ERR_INVALID_ARG;
+  if (w_layout != TP_W_IN_OUT && w_layout != TP_W_OUT_IN) return TP_ERR_INVALID_ARG;
+  const int kmaj = w_layout == TP_W_OUT_IN;
   int st = check_attn_args(S, H, nh, d, t, dtype, TP_DTYPE_BF16, X, Wqkv_shards, Wo_shards, ln1_gamma, ln1_beta,
                            eps, Y);
   if (st != TP_OK) return st;
@@ -995,21 +1008,21 @@ int tp_transformer_block_forward(int S, int H, int F, int nh, int d, int t, int 
   if (!pre_ln) {
     // Y1 = LN1(X + Attn(X));  Y = LN2(Y1 + MLP(Y1))
     st = attn_core(*dev, S, H, nh, d, t, TP_DTYPE_BF16, X, X, Wqkv_shards, Wo_shards, ln1_gamma, ln1_beta, eps, 1,
-                   buf1, core, s);
+                   buf1, core, s, kmaj);
     if (st != TP_OK) return st;
     return mlp_core(*dev, S, H, F, t, dtype, out_dtype, buf1, buf1, A_shards, B_shards, ln2_gamma, ln2_beta, eps,
-                    act, 1, Y, core, s);
+                    act, 1, Y, core, s, kmaj);
   }
   // h1 = LN1(X);  Z1 = X + Attn(h1);  h2 = LN2(Z1);  Y = Z1 + MLP(h2)
   st = run_reduce_ln(S, H, 0, nullptr, X, 1, ln1_gamma, ln1_beta, eps, buf1, 1, s, dev->sm_count, 1);
   if (st != TP_OK) return st;
   st = attn_core(*dev, S, H, nh, d, t, TP_DTYPE_BF16, buf1, X, Wqkv_shards, Wo_shards, nullptr, nullptr, eps, 0,
-                 buf2, core, s);
+                 buf2, core, s, kmaj);
   if (st != TP_OK) return st;
   st = run_reduce_ln(S, H, 0, nullptr, buf2, 1, ln2_gamma, ln2_beta, eps, buf1, 1, s, dev->sm_count, 1);
   if (st != TP_OK) return st;
   return mlp_core(*dev, S, H, F, t, dtype, out_dtype, buf1, buf2, A_shards, B_shards, nullptr, nullptr, eps, act, 0,
-                  Y, core, s);
+                  Y, core, s, kmaj);
 }
 
 // ---------------------------------------------------------------- linears

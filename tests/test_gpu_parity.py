@@ -250,7 +250,7 @@ def test_mlp_s2048_h4096_f16384(cuda_device, t):
 
 
 @pytest.mark.slow
-@pytest.mark.parametrize("t", [4, 8])
+@pytest.mark.parametrize("t", [4, 1, 2, 8])
 def test_attn_s2048_h8192(cuda_device, t):
     w = WORKLOADS["attn_s2048_h8192_64x128"]
     inp = synth.gen_attn(w.S, w.H, seed=w.seed)
@@ -282,8 +282,10 @@ def _cached_mlp(w):
 
 @pytest.mark.parametrize("pre_ln", [False, True])
 @pytest.mark.parametrize("S,nh,F,t", [(256, 2, 1024, 2), (384, 4, 2048, 4)])
-def test_transformer_block(cuda_device, pre_ln, S, nh, F, t):
+@pytest.mark.parametrize("layout", ["in_out", "out_in"])
+def test_transformer_block(cuda_device, pre_ln, S, nh, F, t, layout):
     d = 128
+    tr = (lambda ws: [w.t().contiguous() for w in ws]) if layout == "out_in" else (lambda ws: ws)
     H = nh * d
     a = synth.gen_attn(S, H, seed=S + 1)
     m = synth.gen_mlp(S, H, F, seed=S + 2)
@@ -293,9 +295,10 @@ def test_transformer_block(cuda_device, pre_ln, S, nh, F, t):
     X = a.X.cuda()
     Y = torch.empty(S, H, dtype=torch.float32, device="cuda")
     ws = torch.empty(L.block_workspace_bytes(S, H, F, nh, d, t), dtype=torch.uint8, device="cuda")
-    L.block_forward(X, _dev(synth.split_qkv_by_head(a.Wqkv, nh, d, t)), _dev(synth.split_rows_by_head(a.Wo, nh, d, t)),
-                    _dev(synth.split_columns(m.A, t)), _dev(synth.split_rows(m.B, t)), nh, d, Y, ws, pre_ln=pre_ln,
-                    ln1=(ln1[0].cuda(), ln1[1].cuda()), ln2=(ln2[0].cuda(), ln2[1].cuda()))
+    L.block_forward(X, _dev(tr(synth.split_qkv_by_head(a.Wqkv, nh, d, t))),
+                    _dev(tr(synth.split_rows_by_head(a.Wo, nh, d, t))), _dev(tr(synth.split_columns(m.A, t))),
+                    _dev(tr(synth.split_rows(m.B, t))), nh, d, Y, ws, pre_ln=pre_ln,
+                    ln1=(ln1[0].cuda(), ln1[1].cuda()), ln2=(ln2[0].cuda(), ln2[1].cuda()), layout=layout)
     torch.cuda.synchronize()
     assert L.device_error() == 0
     ref = O.transformer_block(a.X, a.Wqkv, a.Wo, m.A, m.B, nh, d, ln1=ln1, ln2=ln2, pre_ln=pre_ln)

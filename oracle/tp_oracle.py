@@ -52,7 +52,7 @@ __all__ = [
     "layernorm", "mlp_block", "mlp_block_sharded",
     "linear_column", "linear_row",
     "attention_heads", "attention_sublayer", "attention_out", "mlp_out", "transformer_block",
-    "activation_grad", "layernorm_backward", "mlp_block_backward",
+    "activation_grad", "layernorm_backward", "mlp_block_backward", "attention_sublayer_backward",
 ]
 
 _COL_BLOCK = 2048  # output-column block for products whose fp64 weight copy is large
@@ -309,6 +309,60 @@ def mlp_block_backward(X, A, B, dY, gamma=None, beta=None, eps: float = 1e-5,
         "dX": dZ + dU @ A64.T,             # residual path + through step 1
         "dA": X64.T @ dU,
         "dB": G.T @ dZ,
+        "dgamma": dgamma,
+        "dbeta": dbeta,
+    }
+
+
+# Backward of the post-LN attention sublayer for an upstream gradient dY, by
+# the chain rule through attention_sublayer's steps:
+#   Q, K, V = X W_Q, X W_K, X W_V;  per head h: S_h = Q_h K_h^T / sqrt(d),
+#   P_h = softmax(S_h) (rows), O_h = P_h V_h;  Z = X + O W_O;  Y = LN(Z).
+# The softmax backward of a row p with upstream g is p * (g - sum(g * p)).
+# Splitting Wqkv by head and W_O by the matching rows splits their gradients
+# the same way ("TP到底在切什么" §4): dWqkv = X^T dQKV, dW_O = O^T dZ.
+
+def attention_sublayer_backward(X, Wqkv, Wo, nh: int, d: int, dY, gamma=None, beta=None,
+                                eps: float = 1e-5) -> dict:
+    """Gradients of attention_sublayer's output with respect to X, Wqkv, Wo,
+    gamma and beta, contracted with dY: {"dX", "dWqkv", "dWo", "dgamma", "dbeta"}."""
+    del beta
+    X64 = _f64(X)
+    W = _f64(Wqkv)
+    Wo64 = _f64(Wo)
+    H = X64.shape[1]
+    assert nh * d == H
+    QKV = X64 @ W
+    Q, K, V = QKV[:, :H], QKV[:, H:2 * H], QKV[:, 2 * H:]
+    scale = 1.0 / math.sqrt(d)
+    O = np.empty_like(Q)
+    P = []
+    for h in range(nh):
+        c = slice(h * d, (h + 1) * d)
+        s = (Q[:, c] @ K[:, c].T) * scale
+        s = s - s.max(axis=1, keepdims=True)
+        p = np.exp(s)
+        p = p / p.sum(axis=1, keepdims=True)
+        P.append(p)
+        O[:, c] = p @ V[:, c]
+    Z = X64 + O @ Wo64
+    dZ, dgamma, dbeta = layernorm_backward(Z, dY, gamma, eps)
+    dO = dZ @ Wo64.T
+    dWo = O.T @ dZ
+    dQKV = np.empty_like(QKV)
+    for h in range(nh):
+        c = slice(h * d, (h + 1) * d)
+        p = P[h]
+        dV = p.T @ dO[:, c]
+        dP = dO[:, c] @ V[:, c].T
+        dS = p * (dP - (dP * p).sum(axis=1, keepdims=True)) * scale
+        dQKV[:, c] = dS @ K[:, c]
+        dQKV[:, H + h * d:H + (h + 1) * d] = dS.T @ Q[:, c]
+        dQKV[:, 2 * H + h * d:2 * H + (h + 1) * d] = dV
+    return {
+        "dX": dZ + dQKV @ W.T,
+        "dWqkv": X64.T @ dQKV,
+        "dWo": dWo,
         "dgamma": dgamma,
         "dbeta": dbeta,
     }

@@ -345,13 +345,69 @@ def check_backward_invariants():
         np.testing.assert_allclose(O.gelu_tanh(Ui).T @ dZ, full["dB"][i * 4:(i + 1) * 4], atol=1e-12)
 
 
+def _attn_backward_case(S, nh, d, seed):
+    rng = np.random.default_rng(seed)
+    H = nh * d
+    X = rng.standard_normal((S, H))
+    Wqkv = rng.standard_normal((H, 3 * H)) / math.sqrt(H)
+    Wo = rng.standard_normal((H, H)) / math.sqrt(H)
+    g = 1.0 + 0.5 * rng.standard_normal(H)
+    b = 0.3 * rng.standard_normal(H)
+    dY = rng.standard_normal((S, H))
+    return X, Wqkv, Wo, g, b, dY
+
+
+def check_attention_backward_finite_differences():
+    """Brute force: every gradient entry of the attention sublayer against a
+    central difference of the (separately pinned) forward, L = sum(dY * Y)."""
+    S, nh, d = 4, 2, 3
+    h = 1e-5
+    X, Wqkv, Wo, g, b, dY = _attn_backward_case(S, nh, d, seed=21)
+    grads = O.attention_sublayer_backward(X, Wqkv, Wo, nh, d, dY, g, b)
+    params = {"dX": X, "dWqkv": Wqkv, "dWo": Wo, "dgamma": g, "dbeta": b}
+
+    def loss():
+        return float((dY * O.attention_sublayer(X, Wqkv, Wo, nh, d, g, b)).sum())
+
+    for key, P in params.items():
+        assert grads[key].shape == P.shape, key
+        for idx in np.ndindex(*P.shape):
+            old = P[idx]
+            P[idx] = old + h
+            lp = loss()
+            P[idx] = old - h
+            lm = loss()
+            P[idx] = old
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - grads[key][idx]) <= 1e-7 * max(1.0, abs(fd)), (key, idx, fd, grads[key][idx])
+
+
+def check_attention_backward_autograd():
+    """Library route: torch autograd (fp64) through torch's multi-head attention
+    functional and layer_norm gives the same gradients."""
+    S, nh, d = 8, 2, 4
+    H = nh * d
+    X, Wqkv, Wo, g, b, dY = _attn_backward_case(S, nh, d, seed=22)
+    ts = [torch.tensor(v, dtype=torch.float64, requires_grad=True) for v in (X, Wqkv, Wo, g, b)]
+    Xt, Wt, Wot, gt, bt = ts
+    x = Xt.unsqueeze(1)  # [S, batch 1, H]
+    att, _ = torch.nn.functional.multi_head_attention_forward(
+        x, x, x, H, nh, Wt.T.contiguous(), None, None, None, False, 0.0, Wot.T.contiguous(), None,
+        training=False, need_weights=False)
+    Y = torch.nn.functional.layer_norm(Xt + att.squeeze(1), (H,), gt, bt, eps=1e-5)
+    (Y * torch.tensor(dY)).sum().backward()
+    ref = O.attention_sublayer_backward(X, Wqkv, Wo, nh, d, dY, g, b)
+    for key, t in zip(("dX", "dWqkv", "dWo", "dgamma", "dbeta"), ts):
+        np.testing.assert_allclose(ref[key], t.grad.numpy(), rtol=1e-9, atol=1e-11, err_msg=key)
+
+
 ALL_CHECKS = [
     check_gelu_library, check_gelu_identities, check_layernorm_hand, check_layernorm_invariants,
     check_mlp_exact_bruteforce, check_mlp_closed_forms, check_mlp_block_identities,
     check_mlp_symmetries, check_linears_exact, check_attention_hand,
     check_attention_uniform_keys, check_attention_library, check_attention_row_equivariance,
     check_block_composition, check_backward_finite_differences, check_backward_autograd,
-    check_backward_invariants,
+    check_backward_invariants, check_attention_backward_finite_differences, check_attention_backward_autograd,
 ]
 
 
@@ -473,6 +529,34 @@ def _bad_backward_db_from_u(X, A, B, dY, gamma=None, beta=None, eps=1e-5, act="g
     return {"dX": dZ + dU @ A64.T, "dA": X64.T @ dU, "dB": U.T @ dZ, "dgamma": dg, "dbeta": db}
 
 
+def _bad_attention_backward_no_softmax_projection(X, Wqkv, Wo, nh, d, dY, gamma=None, beta=None, eps=1e-5):
+    X64, W, Wo64 = O._f64(X), O._f64(Wqkv), O._f64(Wo)
+    H = X64.shape[1]
+    QKV = X64 @ W
+    Q, K, V = QKV[:, :H], QKV[:, H:2 * H], QKV[:, 2 * H:]
+    sc = 1.0 / math.sqrt(d)
+    Oo = np.empty_like(Q)
+    Ps = []
+    for hh in range(nh):
+        c = slice(hh * d, (hh + 1) * d)
+        s_ = Q[:, c] @ K[:, c].T * sc
+        p = np.exp(s_ - s_.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        Ps.append(p)
+        Oo[:, c] = p @ V[:, c]
+    dZ, dg, db = O.layernorm_backward(X64 + Oo @ Wo64, dY, gamma, eps)
+    dO = dZ @ Wo64.T
+    dQKV = np.empty_like(QKV)
+    for hh in range(nh):
+        c = slice(hh * d, (hh + 1) * d)
+        p = Ps[hh]
+        dS = p * (dO[:, c] @ V[:, c].T) * sc          # the row projection term dropped
+        dQKV[:, c] = dS @ K[:, c]
+        dQKV[:, H + hh * d:H + (hh + 1) * d] = dS.T @ Q[:, c]
+        dQKV[:, 2 * H + hh * d:2 * H + (hh + 1) * d] = p.T @ dO[:, c]
+    return {"dX": dZ + dQKV @ W.T, "dWqkv": X64.T @ dQKV, "dWo": Oo.T @ dZ, "dgamma": dg, "dbeta": db}
+
+
 _PLANTED = [
     ("layernorm", _bad_layernorm_unbiased),
     ("layernorm", _bad_layernorm_eps_outside),
@@ -487,6 +571,7 @@ _PLANTED = [
     ("activation_grad", _bad_activation_grad_is_activation),
     ("mlp_block_backward", _bad_backward_no_residual),
     ("mlp_block_backward", _bad_backward_db_from_u),
+    ("attention_sublayer_backward", _bad_attention_backward_no_softmax_projection),
 ]
 
 

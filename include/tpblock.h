@@ -222,6 +222,39 @@ int tp_qkv_attn_oproj_forward_ex(int S, int H, int nh, int d, int t, int dtype, 
                                  const float* gamma, const float* beta, float eps,
                                  void* Y, void* workspace, size_t workspace_bytes, void* stream);
 
+/* -------------------------------------------- attention training step ----
+ * Backward pass of the attention sublayer (post-LN, [in, out] weights, bf16),
+ * the chain rule through QKV = X Wqkv, S_h = Q_h K_h^T / sqrt d,
+ * P_h = softmax(S_h), O_h = P_h V_h, Z = X + O Wo, Y = LN(Z):
+ *   dZ = LayerNorm backward of dY;  dO = dZ Wo^T;  dWo = O^T dZ;
+ *   per head: dV_h = P_h^T dO_h, dS_h = P_h * (dO_h V_h^T - rowsum(dO_h * O_h)) / sqrt d,
+ *             dQ_h = dS_h K_h, dK_h = dS_h^T Q_h;
+ *   dX = dZ + dQKV Wqkv^T;  dWqkv = X^T dQKV.
+ * Each shard's weight gradients stay with the shard ([PWWT] §4).
+ *
+ * tp_attn_forward_train: tp_qkv_attn_oproj_forward that also keeps, in the
+ * caller's `state` (>= tp_attn_train_state_bytes()), QKV [S, 3H] bf16, O
+ * [S, H] bf16, O Wo [S, H] f32 and each row's log2 softmax denominator per
+ * head [nh, S] f32 (P is rebuilt from it in the backward).
+ *
+ * tp_attn_backward: from the same X, shards, gamma, eps and the state of one
+ * tp_attn_forward_train call, and dY [S, H] bf16, writes dX [S, H] bf16,
+ * dWqkv_shards[s] [H, 3 (nh/t) d] and dWo_shards[s] [(nh/t) d, H] f32 (the
+ * shards' layout), dgamma and dbeta [H] f32 (either may be NULL).
+ * workspace >= tp_attn_backward_workspace_bytes() (it holds one head's
+ * [S, S] score, P, dP and dS matrices).  Shapes as tp_qkv_attn_oproj_forward. */
+size_t tp_attn_train_state_bytes(int S, int H, int nh, int d, int t, int dtype);
+int tp_attn_forward_train(int S, int H, int nh, int d, int t, int dtype, int out_dtype, const void* X,
+                          const void* const* Wqkv_shards, const void* const* Wo_shards,
+                          const float* gamma, const float* beta, float eps,
+                          void* Y, void* state, size_t state_bytes, void* stream);
+size_t tp_attn_backward_workspace_bytes(int S, int H, int nh, int d, int t, int dtype);
+int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* X,
+                     const void* const* Wqkv_shards, const void* const* Wo_shards,
+                     const float* gamma, float eps, const void* state, size_t state_bytes,
+                     const void* dY, void* dX, void* const* dWqkv_shards, void* const* dWo_shards,
+                     float* dgamma, float* dbeta, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---------------------------------------------------- Transformer block ----
  * The attention sublayer followed by the MLP sublayer, the two TP pairs of one
  * Transformer block ([PWWT] §2.1 figure 3: QKV/O one pair, the two MLP

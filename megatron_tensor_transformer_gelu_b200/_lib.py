@@ -60,6 +60,11 @@ SIGNATURES = {
     "tp_mlp_backward_workspace_bytes": (_c_size, [_c_int] * 5),
     "tp_mlp_backward": (_c_int, [_c_int] * 5 + [_vp, _vpp, _vpp, _vp, _c_float, _c_int, _vp, _c_size, _vp, _vp, _vpp,
                                                  _vpp, _vp, _vp, _vp, _c_size, _vp]),
+    "tp_attn_train_state_bytes": (_c_size, [_c_int] * 6),
+    "tp_attn_forward_train": (_c_int, [_c_int] * 7 + [_vp, _vpp, _vpp, _vp, _vp, _c_float, _vp, _vp, _c_size, _vp]),
+    "tp_attn_backward_workspace_bytes": (_c_size, [_c_int] * 6),
+    "tp_attn_backward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vpp, _vp, _c_float, _vp, _c_size, _vp, _vp, _vpp, _vpp,
+                                                  _vp, _vp, _vp, _c_size, _vp]),
     "tp_set_gemm_tile_n": (_c_int, [_c_int]),
     "tp_selftest_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
     "tp_profile_enable": (_c_int, [_c_int]),
@@ -258,6 +263,40 @@ def mlp_backward(X, A_shards, B_shards, state, dY, dX, dA_shards, dB_shards, wor
                                     _ptr(dY), _ptr(dX), pda, pdb, _ptr(dgamma), _ptr(dbeta), _ptr(workspace),
                                     workspace.numel() * workspace.element_size(), _stream(stream))
     _check(code, "tp_mlp_backward")
+
+
+def attn_train_state_bytes(S, H, nh, d, t, dtype=torch.bfloat16) -> int:
+    return int(lib().tp_attn_train_state_bytes(S, H, nh, d, t, DTYPE[dtype]))
+
+
+def attn_backward_workspace_bytes(S, H, nh, d, t, dtype=torch.bfloat16) -> int:
+    return int(lib().tp_attn_backward_workspace_bytes(S, H, nh, d, t, DTYPE[dtype]))
+
+
+def attn_forward_train(X, Wqkv_shards, Wo_shards, nh, d, Y, state, gamma=None, beta=None, eps=1e-5, stream=None):
+    S, H = X.shape
+    t = len(Wqkv_shards)
+    pq, kq = _ptrs(Wqkv_shards)
+    po, ko = _ptrs(Wo_shards)
+    code = lib().tp_attn_forward_train(S, H, nh, d, t, DTYPE[X.dtype], DTYPE[Y.dtype], _ptr(X), pq, po, _ptr(gamma),
+                                       _ptr(beta), float(eps), _ptr(Y), _ptr(state),
+                                       state.numel() * state.element_size(), _stream(stream))
+    _check(code, "tp_attn_forward_train")
+
+
+def attn_backward(X, Wqkv_shards, Wo_shards, nh, d, state, dY, dX, dWqkv_shards, dWo_shards, workspace, gamma=None,
+                  dgamma=None, dbeta=None, eps=1e-5, stream=None):
+    S, H = X.shape
+    t = len(Wqkv_shards)
+    pq, kq = _ptrs(Wqkv_shards)
+    po, ko = _ptrs(Wo_shards)
+    pdq, kdq = _ptrs(dWqkv_shards)
+    pdo, kdo = _ptrs(dWo_shards)
+    code = lib().tp_attn_backward(S, H, nh, d, t, DTYPE[X.dtype], _ptr(X), pq, po, _ptr(gamma), float(eps),
+                                  _ptr(state), state.numel() * state.element_size(), _ptr(dY), _ptr(dX), pdq, pdo,
+                                  _ptr(dgamma), _ptr(dbeta), _ptr(workspace),
+                                  workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(code, "tp_attn_backward")
 
 
 def set_gemm_tile_n(tile_n: int) -> None:

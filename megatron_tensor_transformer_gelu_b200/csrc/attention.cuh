@@ -58,6 +58,9 @@ struct AttnArgs {
   int heads_per_shard;
   int shard_cols;      // 3 * heads_per_shard * D: width of one shard's [Q|K|V] block
   float scale_log2;    // log2(e) / sqrt(D)
+  float* lse2;         // optional [nh, S]: log2 of each row's softmax denominator, in the
+                       // units of the scores times scale_log2 (what a backward pass
+                       // needs to rebuild P = 2^(s scale_log2 - lse2))
 };
 
 __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __grid_constant__ AttnArgs a) {
@@ -306,6 +309,7 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
       tc_fence_after();
       const float inv = 1.0f / l_run;
       const int grow = q0 + tile * BQ + r;
+      if (a.lse2) a.lse2[static_cast<long long>(h) * a.S + grow] = m_run + __log2f(l_run);
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.O) + static_cast<long long>(grow) * a.H + h * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {

@@ -15,6 +15,7 @@
 
 #include "../../include/tpblock.h"
 #include "attention.cuh"
+#include "attn_backward.cuh"
 #include "gemm_tcgen05.cuh"
 #include "ln_backward.cuh"
 #include "reduce_ln.cuh"
@@ -660,16 +661,27 @@ int mlp_core(const DeviceInfo& dev, int S, int H, int F, int t, int dtype, int o
 
 // Attention sublayer on `in` with residual `res` (bf16): Y = LN(res + O Wo)
 // or Y = res + O Wo (apply_ln = 0).  Arguments are already checked.
+// Kept by a training forward of the attention sublayer: the buffers it writes
+// anyway (QKV, O, the O projection's f32 output) and each row's log2 softmax
+// denominator per head.
+struct AttnKeep {
+  void* qkv = nullptr;
+  void* o = nullptr;
+  float* zsum = nullptr;
+  float* lse2 = nullptr;
+};
+
 int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out_dtype, const void* in,
               const void* res, const void* const* Wqkv_shards, const void* const* Wo_shards, const float* gamma,
               const float* beta, float eps, int apply_ln, void* Y, void* workspace, cudaStream_t s,
-              int kmaj = 0) {
+              int kmaj = 0, const AttnKeep* keep = nullptr) {
   if (S == 0) return TP_OK;
   const int Hs = H / t;  // columns of one shard's heads
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  void* QKV = ws;                                                            // [S, 3H] bf16
-  void* Obuf = ws + align256(static_cast<size_t>(S) * 3 * H * 2);            // [S, H]  bf16
-  float* Zsum = reinterpret_cast<float*>(static_cast<uint8_t*>(Obuf) + align256(static_cast<size_t>(S) * H * 2));
+  void* QKV = keep ? keep->qkv : ws;                                         // [S, 3H] bf16
+  void* Obuf = keep ? keep->o : ws + align256(static_cast<size_t>(S) * 3 * H * 2);   // [S, H] bf16
+  float* Zsum = keep ? keep->zsum
+                     : reinterpret_cast<float*>(static_cast<uint8_t*>(Obuf) + align256(static_cast<size_t>(S) * H * 2));
   // [Q_s | K_s | V_s] = in Wqkv_s into columns [3 s Hs, 3 (s+1) Hs) of QKV.
   int st = run_gemm_tc(dev, in, H, S, Wqkv_shards, t, 0, H, 3 * Hs, QKV, 3LL * H, 0, TP_ACT_NONE, s, 1, 0, nullptr,
                        kmaj);
@@ -688,6 +700,7 @@ int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out
     a.heads_per_shard = nhs;
     a.shard_cols = 3 * Hs;
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+    a.lse2 = keep ? keep->lse2 : nullptr;
     dim3 grid((S + tp::attn::TILES * tp::attn::BQ - 1) / (tp::attn::TILES * tp::attn::BQ), nh);
     ProfScope ps(K_ATTN, s);
     st = launch_pdl(tp::attn_fwd_kernel, grid, dim3(tp::attn::NUM_THREADS), tp::attn::SMEM_BYTES, s, a) != cudaSuccess
@@ -697,7 +710,7 @@ int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out
   }
   // sum_s O_s Wo_s, the O projection row-split by head, summed in TMEM.
   int nparts = 1;
-  st = run_gemm_tc(dev, Obuf, H, S, Wo_shards, t, 1, Hs, H, Zsum, H, 1, TP_ACT_NONE, s, TP_MAX_K_SPLITS,
+  st = run_gemm_tc(dev, Obuf, H, S, Wo_shards, t, 1, Hs, H, Zsum, H, 1, TP_ACT_NONE, s, keep ? 1 : TP_MAX_K_SPLITS,
                    static_cast<long long>(S) * H, &nparts, kmaj);
   if (st != TP_OK) return st;
   return run_reduce_ln(S, H, nparts, Zsum, res, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s, dev.sm_count,
@@ -959,6 +972,238 @@ int tp_qkv_attn_oproj_forward_ex(int S, int H, int nh, int d, int t, int dtype, 
 }
 
 // ---------------------------------------------------------- Transformer block
+// ------------------------------------------------- attention training step
+namespace {
+struct AttnState {
+  size_t off_qkv, off_o, off_z, off_lse, bytes;
+};
+AttnState attn_state_layout(int S, int H, int nh) {
+  AttnState a;
+  const size_t s = static_cast<size_t>(S), h = static_cast<size_t>(H);
+  a.off_qkv = 0;
+  a.off_o = align256(s * 3 * h * 2);
+  a.off_z = a.off_o + align256(s * h * 2);
+  a.off_lse = a.off_z + align256(s * h * 4);
+  a.bytes = a.off_lse + align256(static_cast<size_t>(nh) * s * 4);
+  return a;
+}
+struct AttnBackWs {
+  size_t off_dz, off_do, off_dqkv, off_dxp, off_sc, off_p, off_dp, off_ds, off_d, off_part, bytes;
+};
+AttnBackWs attn_back_layout(int S, int H, int nh) {
+  AttnBackWs w;
+  const size_t s = static_cast<size_t>(S), h = static_cast<size_t>(H);
+  w.off_dz = 0;
+  w.off_do = align256(s * h * 2);
+  w.off_dqkv = w.off_do + align256(s * h * 2);
+  w.off_dxp = w.off_dqkv + align256(s * 3 * h * 2);
+  w.off_sc = w.off_dxp + align256(s * h * 4);
+  w.off_p = w.off_sc + align256(s * s * 4);
+  w.off_dp = w.off_p + align256(s * s * 2);
+  w.off_ds = w.off_dp + align256(s * s * 4);
+  w.off_d = w.off_ds + align256(s * s * 2);
+  w.off_part = w.off_d + align256(static_cast<size_t>(nh) * s * 4);
+  w.bytes = w.off_part + align256(static_cast<size_t>(LNB_MAX_CTAS) * 2 * h * 4);
+  return w;
+}
+int grid_for(long long n8, int sms) {
+  const long long b = (n8 + 255) / 256;
+  const long long cap = 8LL * sms;
+  return static_cast<int>(b < cap ? (b < 1 ? 1 : b) : cap);
+}
+}  // namespace
+
+size_t tp_attn_train_state_bytes(int S, int H, int nh, int d, int t, int dtype) {
+  if (S < 0 || H <= 0 || nh <= 0 || d <= 0 || t < 1 || dtype != TP_DTYPE_BF16) return 0;
+  return attn_state_layout(S, H, nh).bytes;
+}
+
+int tp_attn_forward_train(int S, int H, int nh, int d, int t, int dtype, int out_dtype, const void* X,
+                          const void* const* Wqkv_shards, const void* const* Wo_shards, const float* gamma,
+                          const float* beta, float eps, void* Y, void* state, size_t state_bytes, void* stream) {
+  int st = check_attn_args(S, H, nh, d, t, dtype, out_dtype, X, Wqkv_shards, Wo_shards, gamma, beta, eps, Y);
+  if (st != TP_OK) return st;
+  if (!opt_ptr_ok(state)) return TP_ERR_INVALID_ARG;
+  if (S == 0) return TP_OK;
+  const AttnState L = attn_state_layout(S, H, nh);
+  if (!state || state_bytes < L.bytes) return TP_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  uint8_t* b = static_cast<uint8_t*>(state);
+  AttnKeep keep;
+  keep.qkv = b + L.off_qkv;
+  keep.o = b + L.off_o;
+  keep.zsum = reinterpret_cast<float*>(b + L.off_z);
+  keep.lse2 = reinterpret_cast<float*>(b + L.off_lse);
+  return attn_core(*dev, S, H, nh, d, t, out_dtype, X, X, Wqkv_shards, Wo_shards, gamma, beta, eps, 1, Y, nullptr,
+                   static_cast<cudaStream_t>(stream), 0, &keep);
+}
+
+size_t tp_attn_backward_workspace_bytes(int S, int H, int nh, int d, int t, int dtype) {
+  if (S < 0 || H <= 0 || nh <= 0 || d <= 0 || t < 1 || dtype != TP_DTYPE_BF16) return 0;
+  return attn_back_layout(S, H, nh).bytes;
+}
+
+int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* X,
+                     const void* const* Wqkv_shards, const void* const* Wo_shards, const float* gamma, float eps,
+                     const void* state, size_t state_bytes, const void* dY, void* dX, void* const* dWqkv_shards,
+                     void* const* dWo_shards, float* dgamma, float* dbeta, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  int st = check_attn_args(S, H, nh, d, t, dtype, TP_DTYPE_BF16, X, Wqkv_shards, Wo_shards, gamma, nullptr, eps, dX);
+  if (st != TP_OK) return st;
+  if ((S > 0 && (!ptr_ok(dY) || !ptr_ok(state))) || !opt_ptr_ok(dY) || !opt_ptr_ok(state) ||
+      !shards_ok(dWqkv_shards, t) || !shards_ok(dWo_shards, t) || !opt_ptr_ok(dgamma) || !opt_ptr_ok(dbeta) ||
+      !opt_ptr_ok(workspace))
+    return TP_ERR_INVALID_ARG;
+  if (S == 0) return TP_OK;
+  const AttnState L = attn_state_layout(S, H, nh);
+  if (state_bytes < L.bytes) return TP_ERR_WORKSPACE_TOO_SMALL;
+  const AttnBackWs W = attn_back_layout(S, H, nh);
+  if (!workspace || workspace_bytes < W.bytes) return TP_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int Hs = H / t, hps = nh / t;
+  const long long H3 = 3LL * H;
+  const uint8_t* sb = static_cast<const uint8_t*>(state);
+  const uint8_t* QKV = sb + L.off_qkv;
+  const uint8_t* Ob = sb + L.off_o;
+  const float* Vo = reinterpret_cast<const float*>(sb + L.off_z);
+  const float* lse2 = reinterpret_cast<const float*>(sb + L.off_lse);
+  uint8_t* wb = static_cast<uint8_t*>(workspace);
+  void* dZ = wb + W.off_dz;
+  uint8_t* dO = wb + W.off_do;
+  uint8_t* dQKV = wb + W.off_dqkv;
+  float* dXp = reinterpret_cast<float*>(wb + W.off_dxp);
+  float* Sc = reinterpret_cast<float*>(wb + W.off_sc);
+  __nv_bfloat16* P = reinterpret_cast<__nv_bfloat16*>(wb + W.off_p);
+  float* dP = reinterpret_cast<float*>(wb + W.off_dp);
+  __nv_bfloat16* dS = reinterpret_cast<__nv_bfloat16*>(wb + W.off_ds);
+  float* D = reinterpret_cast<float*>(wb + W.off_d);
+  float* part = reinterpret_cast<float*>(wb + W.off_part);
+  // 1. Through the LayerNorm: dZ, dgamma, dbeta (Z = X + the O projection's output).
+  st = run_ln_backward(S, H, Vo, X, dY, gamma, eps, dZ, part, dgamma, dbeta, s, dev->sm_count);
+  if (st != TP_OK) return st;
+  // 2. Through the O projection: dO_s = dZ Wo_s^T (Wo_s [Hs, H] read K-major)
+  //    into shard s's head columns of dO, and dWo_s = O_s^T dZ.
+  st = run_gemm_tc(*dev, dZ, H, S, Wo_shards, t, 0, H, Hs, dO, H, 0, TP_ACT_NONE, s, 1, 0, nullptr, 1);
+  if (st != TP_OK) return st;
+  {
+    const void* b1[1] = {dZ};
+    if (t > 1 && Hs % 256 == 0) {
+      GemmExtra ex;
+      ex.a_mnmajor = 1;
+      ex.m_split = t;
+      ex.C_shards = dWo_shards;
+      ex.ldc_shard = H;
+      st = run_gemm_tc(*dev, Ob, H, H, b1, 1, 0, S, H, nullptr, H, 1, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
+      if (st != TP_OK) return st;
+    } else {
+      for (int i = 0; i < t; ++i) {
+        GemmExtra ex;
+        ex.a_mnmajor = 1;
+        st = run_gemm_tc(*dev, Ob + static_cast<size_t>(i) * Hs * 2, H, Hs, b1, 1, 0, S, H, dWo_shards[i], H, 1,
+                         TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
+        if (st != TP_OK) return st;
+      }
+    }
+  }
+  // 3. Per head, through the softmax attention (P rebuilt from the scores and
+  //    the forward's log2 denominators).
+  const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
+  const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+  st = launch_pdl(tp::rowdot_kernel, dim3(ceil_div(static_cast<long long>(S) * nh * 32, 256)), dim3(256), 0, s,
+                  reinterpret_cast<const __nv_bfloat16*>(dO), reinterpret_cast<const __nv_bfloat16*>(Ob), D, S, H,
+                  nh) != cudaSuccess
+           ? TP_ERR_CUDA
+           : launch_status();
+  if (st != TP_OK) return st;
+  const int eg = grid_for(static_cast<long long>(S) * S / 8, dev->sm_count);
+  for (int h = 0; h < nh; ++h) {
+    const int sh = h / hps, hj = h % hps;
+    const long long qcol = static_cast<long long>(sh) * 3 * Hs + static_cast<long long>(hj) * d;
+    const uint8_t* Qh = QKV + qcol * 2;
+    const uint8_t* Kh = QKV + (qcol + Hs) * 2;
+    const uint8_t* Vh = QKV + (qcol + 2LL * Hs) * 2;
+    const uint8_t* dOh = dO + static_cast<long long>(h) * d * 2;
+    // raw scores S = Q_h K_h^T (K_h [keys, d] is the K-major B operand)
+    {
+      const void* b1[1] = {Kh};
+      GemmExtra ex;
+      ex.ldb = H3;
+      st = run_gemm_tc(*dev, Qh, H3, S, b1, 1, 0, d, S, Sc, S, 1, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
+      if (st != TP_OK) return st;
+    }
+    st = launch_pdl(tp::softmax_rebuild_kernel, dim3(eg), dim3(256), 0, s, static_cast<const float*>(Sc),
+                    lse2 + static_cast<long long>(h) * S, scale_log2, P, S) != cudaSuccess
+             ? TP_ERR_CUDA
+             : launch_status();
+    if (st != TP_OK) return st;
+    // dV_h = P^T dO_h into V_h's columns of dQKV (P read M-major)
+    {
+      const void* b1[1] = {dOh};
+      GemmExtra ex;
+      ex.a_mnmajor = 1;
+      ex.ldb = H;
+      st = run_gemm_tc(*dev, P, S, S, b1, 1, 0, S, d, dQKV + (qcol + 2LL * Hs) * 2, H3, 0, TP_ACT_NONE, s, 1, 0,
+                       nullptr, 0, &ex);
+      if (st != TP_OK) return st;
+    }
+    // dP = dO_h V_h^T (V_h [keys, d] is the K-major B operand)
+    {
+      const void* b1[1] = {Vh};
+      GemmExtra ex;
+      ex.ldb = H3;
+      st = run_gemm_tc(*dev, dOh, H, S, b1, 1, 0, d, S, dP, S, 1, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
+      if (st != TP_OK) return st;
+    }
+    st = launch_pdl(tp::softmax_backward_kernel, dim3(eg), dim3(256), 0, s, static_cast<const __nv_bfloat16*>(P),
+                    static_cast<const float*>(dP), static_cast<const float*>(D + static_cast<long long>(h) * S),
+                    scale, dS, S) != cudaSuccess
+             ? TP_ERR_CUDA
+             : launch_status();
+    if (st != TP_OK) return st;
+    // dQ_h = dS K_h and dK_h = dS^T Q_h into their columns of dQKV
+    {
+      const void* b1[1] = {Kh};
+      GemmExtra ex;
+      ex.ldb = H3;
+      st = run_gemm_tc(*dev, dS, S, S, b1, 1, 0, S, d, dQKV + qcol * 2, H3, 0, TP_ACT_NONE, s, 1, 0, nullptr, 0,
+                       &ex);
+      if (st != TP_OK) return st;
+    }
+    {
+      const void* b1[1] = {Qh};
+      GemmExtra ex;
+      ex.a_mnmajor = 1;
+      ex.ldb = H3;
+      st = run_gemm_tc(*dev, dS, S, S, b1, 1, 0, S, d, dQKV + (qcol + Hs) * 2, H3, 0, TP_ACT_NONE, s, 1, 0,
+                       nullptr, 0, &ex);
+      if (st != TP_OK) return st;
+    }
+  }
+  // 4. Through the QKV projection and the residual: dX = dZ + sum_s dQKV_s
+  //    Wqkv_s^T (row split over the shards, Wqkv_s [H, 3 Hs] read K-major),
+  //    then dWqkv_s = X^T dQKV_s.
+  st = run_gemm_tc(*dev, dQKV, H3, S, Wqkv_shards, t, 1, 3 * Hs, H, dXp, H, 1, TP_ACT_NONE, s, 1, 0, nullptr, 1);
+  if (st != TP_OK) return st;
+  st = run_reduce_ln(S, H, 1, dXp, dZ, 1, nullptr, nullptr, 1.0f, dX, 1, s, dev->sm_count, /*apply_ln=*/0);
+  if (st != TP_OK) return st;
+  {
+    const void* sh[TP_MAX_SHARDS];
+    for (int i = 0; i < t; ++i) sh[i] = dQKV + static_cast<size_t>(i) * 3 * Hs * 2;
+    GemmExtra ex;
+    ex.a_mnmajor = 1;
+    ex.ldb = H3;
+    ex.C_shards = dWqkv_shards;
+    ex.ldc_shard = 3 * Hs;
+    return run_gemm_tc(*dev, X, H, H, sh, t, 0, S, 3 * Hs, nullptr, 3 * Hs, 1, TP_ACT_NONE, s, 1, 0, nullptr, 0,
+                       &ex);
+  }
+}
+
 size_t tp_block_workspace_bytes(int S, int H, int F, int nh, int d, int t, int dtype) {
   if (S < 0 || H <= 0 || F <= 0 || nh <= 0 || d <= 0 || t < 1 || dtype != TP_DTYPE_BF16) return 0;
   const size_t a = tp_attn_workspace_bytes(S, H, nh, d, t, dtype);

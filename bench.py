@@ -33,10 +33,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "TP MLP block fwd TFLOP/s (bf16, 1 B200) and % of dense bf16 tensor peak"
 METRIC_TRAIN = "TP MLP block training step (fwd + bwd) TFLOP/s (bf16, 1 B200) and % of dense bf16 tensor peak"
+METRIC_ATTN_TRAIN = ("TP attention sublayer training step (fwd + bwd) TFLOP/s (bf16, 1 B200) "
+                     "and % of dense bf16 tensor peak")
 
 
 def metric_for(w) -> str:
-    return METRIC_TRAIN if w.kind == "mlp_train" else METRIC
+    return {"mlp_train": METRIC_TRAIN, "attn_train": METRIC_ATTN_TRAIN}.get(w.kind, METRIC)
 UNIT = "TFLOP/s"
 L2_BYTES = 126 * 2**20
 PROFILE_EVERY = 8  # steps between the timed region's per-kernel event samples
@@ -226,6 +228,41 @@ class Problem:
                 L.mlp_backward(X, self.W1, self.W2, self.state, self.dY, Y, self.dA, self.dB, self.ws,
                                gamma=self.gamma, dgamma=self.dg, dbeta=self.db, stream=st)
             self.run = train_step
+        elif w.kind == "attn_train":
+            S, H = w.S, w.H
+            inp = synth.gen_attn(S, H, seed=w.seed + rank)
+            dY, gamma, _ = synth.gen_upstream(S, H, seed=w.seed + rank + 2)
+            self.X = inp.X.to(dev)
+            self.W1 = [q.to(dev) for q in synth.split_qkv_by_head(inp.Wqkv, w.nh, w.d, t)]
+            self.W2 = [o.to(dev) for o in synth.split_rows_by_head(inp.Wo, w.nh, w.d, t)]
+            self.dY = dY.to(dev)
+            self.gamma = gamma.to(dev)
+            self.Yf = torch.empty(S, H, dtype=bf, device=dev)
+            self.Y = torch.empty(S, H, dtype=bf, device=dev)            # the step's result: dX
+            self.state = torch.empty(L.attn_train_state_bytes(S, H, w.nh, w.d, t), dtype=torch.uint8, device=dev)
+            self.ws = torch.empty(L.attn_backward_workspace_bytes(S, H, w.nh, w.d, t), dtype=torch.uint8,
+                                  device=dev)
+            self.dWq = [torch.empty(*q.shape, dtype=torch.float32, device=dev) for q in self.W1]
+            self.dWo = [torch.empty(*o.shape, dtype=torch.float32, device=dev) for o in self.W2]
+            self.dg = torch.empty(H, dtype=torch.float32, device=dev)
+            self.db = torch.empty(H, dtype=torch.float32, device=dev)
+            att = 2 * 2 * S * S * w.d * w.nh
+            # Bytes of the elementwise backward kernels: per head the rebuilt P
+            # (scores f32 in, P bf16 out) and dS (P bf16 + dP f32 in, dS bf16
+            # out); D = rowsum(dO * O) reads dO and O once.
+            self.work = {"gemm_tcgen05": w.flops - att,          # every product but the fused forward attention
+                         "attention_fwd": att,
+                         "reduce_residual_layernorm": 2 * (S * H * 8 + H * 8),
+                         "layernorm_backward": S * H * (4 + 2 + 2 + 2),
+                         "attention_backward_elementwise": w.nh * S * S * (4 + 2 + 2 + 4 + 2) + S * H * 4}
+            self.Xh_src = inp.X
+
+            def attn_train_step(X, Y, st):
+                L.attn_forward_train(X, self.W1, self.W2, w.nh, w.d, self.Yf, self.state, gamma=self.gamma,
+                                     stream=st)
+                L.attn_backward(X, self.W1, self.W2, w.nh, w.d, self.state, self.dY, Y, self.dWq, self.dWo,
+                                self.ws, gamma=self.gamma, dgamma=self.dg, dbeta=self.db, stream=st)
+            self.run = attn_train_step
         elif w.kind == "attn":
             S, H = w.S, w.H
             inp = synth.gen_attn(S, H, seed=w.seed + rank)
@@ -475,6 +512,13 @@ def cpu_oracle_timing(w, rows_per_step: int, steps: int, warmup: int):
         inp = synth.gen_attn(w.S, w.H, seed=w.seed)
         nrows = w.S
         call = lambda rows: O.attention_sublayer(inp.X, inp.Wqkv, inp.Wo, w.nh, w.d, rows=rows)
+    elif w.kind == "attn_train":
+        # The backward of a row sample needs every key row: the oracle runs on
+        # the first `rows` rows as a shorter sequence (its own attention).
+        inp = synth.gen_attn(w.S, w.H, seed=w.seed)
+        dY, gamma, _ = synth.gen_upstream(w.S, w.H, seed=w.seed + 2)
+        nrows = w.S
+        call = lambda rows: O.attention_sublayer_backward(inp.X[rows], inp.Wqkv, inp.Wo, w.nh, w.d, dY[rows], gamma)
     else:
         inp = synth.gen_linear(w.M, w.K, w.N, seed=w.seed)
         nrows = w.M
@@ -492,6 +536,9 @@ def cpu_oracle_timing(w, rows_per_step: int, steps: int, warmup: int):
         out = call(rows)
     dt = time.perf_counter() - t0
     flops = w.flops * len(rows) / nrows * steps
+    if w.kind == "attn_train":  # a shorter sequence: the attention terms scale with rows^2
+        from dataclasses import replace
+        flops = replace(w, S=len(rows)).flops * steps
     return {"value": round(flops / dt / 1e12, 5), "unit": UNIT, "cores": int(cores), "kind": "oracle",
             "sample": (f"{len(rows)} of {nrows} {'batch' if w.kind == 'mlp_train' else 'output'} rows of {w.name} "
                        f"per step, {steps} step(s), "
@@ -505,6 +552,9 @@ def parity_vs_oracle(w, Y, rows, ref, tol: float = 2e-2):
     output the timed loop left (Y; dX for the training step) against the
     baseline run's fp64 result on the same seeded inputs."""
     import numpy as np
+    if w.kind == "attn_train":
+        return {"compared": None, "note": ("the oracle's row sample is a shorter sequence, whose gradients differ "
+                                           "from the full sequence's; full-size parity is a GPU test")}
     ref = np.asarray(ref["dX"] if isinstance(ref, dict) else ref, dtype=np.float64)
     got = Y[list(rows)].double().cpu().numpy()
     err = float(np.abs(got - ref).max() / np.abs(ref).max())

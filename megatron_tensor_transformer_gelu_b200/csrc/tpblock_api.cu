@@ -51,7 +51,7 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 // ------------------------------------------------------------ event timing
 constexpr int PROF_CAP = 16384;  // launches timed between two collects
-constexpr int PROF_KINDS = 5;
+constexpr int PROF_KINDS = 6;
 bool g_prof_on = false;
 bool g_prof_sampling = true;  // record events for the launches made while set
 bool g_prof_events_made = false;
@@ -61,7 +61,7 @@ int g_prof_kind[PROF_CAP];
 int g_prof_n = 0;
 long long g_prof_launches[PROF_KINDS];  // every launch while enabled, timed or not
 
-enum Kind { K_GEMM_TC = 0, K_REDUCE_LN = 1, K_GEMM_SIMT = 2, K_ATTN = 3, K_LN_BACK = 4 };
+enum Kind { K_GEMM_TC = 0, K_REDUCE_LN = 1, K_GEMM_SIMT = 2, K_ATTN = 3, K_LN_BACK = 4, K_ATTN_BACK = 5 };
 
 struct ProfScope {
   int slot = -1;
@@ -1114,11 +1114,14 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
   //    the forward's log2 denominators).
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
+  {
+  ProfScope ps(K_ATTN_BACK, s);
   st = launch_pdl(tp::rowdot_kernel, dim3(ceil_div(static_cast<long long>(S) * nh * 32, 256)), dim3(256), 0, s,
                   reinterpret_cast<const __nv_bfloat16*>(dO), reinterpret_cast<const __nv_bfloat16*>(Ob), D, S, H,
                   nh) != cudaSuccess
            ? TP_ERR_CUDA
            : launch_status();
+  }
   if (st != TP_OK) return st;
   const int eg = grid_for(static_cast<long long>(S) * S / 8, dev->sm_count);
   for (int h = 0; h < nh; ++h) {
@@ -1136,10 +1139,13 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
       st = run_gemm_tc(*dev, Qh, H3, S, b1, 1, 0, d, S, Sc, S, 1, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
       if (st != TP_OK) return st;
     }
+    {
+    ProfScope ps(K_ATTN_BACK, s);
     st = launch_pdl(tp::softmax_rebuild_kernel, dim3(eg), dim3(256), 0, s, static_cast<const float*>(Sc),
                     lse2 + static_cast<long long>(h) * S, scale_log2, P, S) != cudaSuccess
              ? TP_ERR_CUDA
              : launch_status();
+    }
     if (st != TP_OK) return st;
     // dV_h = P^T dO_h into V_h's columns of dQKV (P read M-major)
     {
@@ -1159,11 +1165,14 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
       st = run_gemm_tc(*dev, dOh, H, S, b1, 1, 0, d, S, dP, S, 1, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
       if (st != TP_OK) return st;
     }
+    {
+    ProfScope ps(K_ATTN_BACK, s);
     st = launch_pdl(tp::softmax_backward_kernel, dim3(eg), dim3(256), 0, s, static_cast<const __nv_bfloat16*>(P),
                     static_cast<const float*>(dP), static_cast<const float*>(D + static_cast<long long>(h) * S),
                     scale, dS, S) != cudaSuccess
              ? TP_ERR_CUDA
              : launch_status();
+    }
     if (st != TP_OK) return st;
     // dQ_h = dS K_h and dK_h = dS^T Q_h into their columns of dQKV
     {
@@ -1412,6 +1421,7 @@ const char* tp_kernel_kind_name(int kind) {
     case K_GEMM_SIMT: return "gemm_simt_f32";
     case K_ATTN: return "attention_fwd";
     case K_LN_BACK: return "layernorm_backward";
+    case K_ATTN_BACK: return "attention_backward_elementwise";
     default: return "unknown";
   }
 }

@@ -10,7 +10,7 @@ from dataclasses import dataclass, field
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str            # "mlp" | "mlp_train" | "attn" | "linear_col" | "linear_row"
+    kind: str            # "mlp" | "mlp_train" | "attn" | "attn_train" | "linear_col" | "linear_row"
     dtype: str           # "f32" | "bf16"  (storage of X and weights)
     t: int               # shard count
     seed: int = 0
@@ -32,12 +32,16 @@ class Workload:
         if self.kind == "mlp_train":
             # forward (X A, G B) + backward (dZ B^T, dU A^T, X^T dU, G^T dZ)
             return 6 * 2 * self.S * self.H * self.F
-        if self.kind == "attn":
+        if self.kind in ("attn", "attn_train"):
             S, H = self.S, self.H
             qkv = 2 * S * H * 3 * H
             att = 2 * 2 * S * S * self.d * self.nh
             oproj = 2 * S * H * H
-            return qkv + att + oproj
+            if self.kind == "attn":
+                return qkv + att + oproj
+            # + backward: dO and dWo (2 x oproj), per head the rebuilt scores,
+            # dV, dP, dQ and dK (5 x att / 2), dX and dWqkv (2 x qkv)
+            return qkv + att + oproj + 2 * oproj + 5 * att // 2 + 2 * qkv
         return 2 * self.M * self.K * self.N
 
 
@@ -60,6 +64,10 @@ WORKLOADS = {
         # then the backward pass (all gradients).
         Workload("mlp_train_s2048_h4096_f16384", "mlp_train", "bf16", t=4, seed=0,
                  S=2048, H=4096, F=16384, t_sweep=(4,)),
+        # One training step of the attention sublayer: forward keeping state,
+        # then the backward pass.
+        Workload("attn_train_s2048_h8192_64x128", "attn_train", "bf16", t=4, seed=0,
+                 S=2048, H=8192, nh=64, d=128, act="none", t_sweep=(4,)),
     ]
 }
 

@@ -529,32 +529,44 @@ def _bad_backward_db_from_u(X, A, B, dY, gamma=None, beta=None, eps=1e-5, act="g
     return {"dX": dZ + dU @ A64.T, "dA": X64.T @ dU, "dB": U.T @ dZ, "dgamma": dg, "dbeta": db}
 
 
-def _bad_attention_backward_no_softmax_projection(X, Wqkv, Wo, nh, d, dY, gamma=None, beta=None, eps=1e-5):
-    X64, W, Wo64 = O._f64(X), O._f64(Wqkv), O._f64(Wo)
-    H = X64.shape[1]
-    QKV = X64 @ W
-    Q, K, V = QKV[:, :H], QKV[:, H:2 * H], QKV[:, 2 * H:]
-    sc = 1.0 / math.sqrt(d)
-    Oo = np.empty_like(Q)
-    Ps = []
-    for hh in range(nh):
-        c = slice(hh * d, (hh + 1) * d)
-        s_ = Q[:, c] @ K[:, c].T * sc
-        p = np.exp(s_ - s_.max(axis=1, keepdims=True))
-        p /= p.sum(axis=1, keepdims=True)
-        Ps.append(p)
-        Oo[:, c] = p @ V[:, c]
-    dZ, dg, db = O.layernorm_backward(X64 + Oo @ Wo64, dY, gamma, eps)
-    dO = dZ @ Wo64.T
-    dQKV = np.empty_like(QKV)
-    for hh in range(nh):
-        c = slice(hh * d, (hh + 1) * d)
-        p = Ps[hh]
-        dS = p * (dO[:, c] @ V[:, c].T) * sc          # the row projection term dropped
-        dQKV[:, c] = dS @ K[:, c]
-        dQKV[:, H + hh * d:H + (hh + 1) * d] = dS.T @ Q[:, c]
-        dQKV[:, 2 * H + hh * d:2 * H + (hh + 1) * d] = p.T @ dO[:, c]
-    return {"dX": dZ + dQKV @ W.T, "dWqkv": X64.T @ dQKV, "dWo": Oo.T @ dZ, "dgamma": dg, "dbeta": db}
+def _attention_backward_with(mistake: str):
+    """The attention sublayer's chain rule with one plausible mistake in it."""
+    def bad(X, Wqkv, Wo, nh, d, dY, gamma=None, beta=None, eps=1e-5):
+        X64, W, Wo64 = O._f64(X), O._f64(Wqkv), O._f64(Wo)
+        H = X64.shape[1]
+        QKV = X64 @ W
+        Q, K, V = QKV[:, :H], QKV[:, H:2 * H], QKV[:, 2 * H:]
+        sc = 1.0 / math.sqrt(d)
+        Oo = np.empty_like(Q)
+        Ps = []
+        for hh in range(nh):
+            c = slice(hh * d, (hh + 1) * d)
+            s_ = Q[:, c] @ K[:, c].T * sc
+            p = np.exp(s_ - s_.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            Ps.append(p)
+            Oo[:, c] = p @ V[:, c]
+        dZ, dg, db = O.layernorm_backward(X64 + Oo @ Wo64, dY, gamma, eps)
+        dO = dZ @ Wo64.T
+        dQKV = np.empty_like(QKV)
+        for hh in range(nh):
+            c = slice(hh * d, (hh + 1) * d)
+            p = Ps[hh]
+            dP = dO[:, c] @ V[:, c].T
+            if mistake == "no_softmax_projection":
+                dS = p * dP * sc
+            else:
+                dS = p * (dP - (p * dP).sum(axis=1, keepdims=True))
+                if mistake != "no_scale":
+                    dS = dS * sc
+            dQKV[:, c] = dS @ K[:, c]
+            dQKV[:, H + hh * d:H + (hh + 1) * d] = (dS if mistake == "dk_untransposed" else dS.T) @ Q[:, c]
+            dQKV[:, 2 * H + hh * d:2 * H + (hh + 1) * d] = (p if mistake == "dv_untransposed" else p.T) @ dO[:, c]
+        dX = dQKV @ W.T if mistake == "no_residual" else dZ + dQKV @ W.T
+        dWo = dZ.T @ Oo if mistake == "dwo_transposed" else Oo.T @ dZ
+        return {"dX": dX, "dWqkv": X64.T @ dQKV, "dWo": dWo, "dgamma": dg, "dbeta": db}
+    bad.__name__ = f"_bad_attention_backward_{mistake}"
+    return bad
 
 
 _PLANTED = [
@@ -571,8 +583,9 @@ _PLANTED = [
     ("activation_grad", _bad_activation_grad_is_activation),
     ("mlp_block_backward", _bad_backward_no_residual),
     ("mlp_block_backward", _bad_backward_db_from_u),
-    ("attention_sublayer_backward", _bad_attention_backward_no_softmax_projection),
-]
+] + [("attention_sublayer_backward", _attention_backward_with(m))
+      for m in ("no_softmax_projection", "no_scale", "dk_untransposed", "dv_untransposed", "dwo_transposed",
+                "no_residual")]
 
 
 @pytest.mark.parametrize("name,bad", _PLANTED, ids=lambda x: getattr(x, "__name__", x))

@@ -1,5 +1,5 @@
-// Elementwise steps of the attention backward, per head h, between GEMMs that
-// run on the tensor cores:
+// Elementwise steps of the attention backward, per head h (a launch covers a
+// group of heads), between GEMMs that run on the tensor cores:
 //
 //   D_h[r]   = sum_c dO[r, h d + c] * O[r, h d + c]              (rowdot_kernel)
 //   P[r, k]  = 2^(S[r, k] * scale_log2 - lse2_h[r])              (softmax_rebuild_kernel)
@@ -43,12 +43,14 @@ __global__ void __launch_bounds__(256) rowdot_kernel(const __nv_bfloat16* dO, co
   if (lane == 0) D[static_cast<long long>(h) * S + r] = v;
 }
 
-// 8 consecutive elements of an [S, S] matrix per thread (S % 8 == 0), grid-stride.
+// 8 consecutive elements of a [rows, S] matrix per thread (S % 8 == 0),
+// grid-stride.  rows = g S for a group of g heads stored one [S, S] matrix
+// after another; their per-row vectors (lse2, D) are then consecutive too.
 __global__ void __launch_bounds__(256) softmax_rebuild_kernel(const float* Sc, const float* lse2, float scale_log2,
-                                                              __nv_bfloat16* P, int S) {
+                                                              __nv_bfloat16* P, int rows, int S) {
   griddep_wait();
   griddep_launch_dependents();
-  const long long n8 = static_cast<long long>(S) * S / 8;
+  const long long n8 = static_cast<long long>(rows) * S / 8;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long e = i * 8;
@@ -68,10 +70,10 @@ __global__ void __launch_bounds__(256) softmax_rebuild_kernel(const float* Sc, c
 }
 
 __global__ void __launch_bounds__(256) softmax_backward_kernel(const __nv_bfloat16* P, const float* dP, const float* D,
-                                                               float scale, __nv_bfloat16* dS, int S) {
+                                                               float scale, __nv_bfloat16* dS, int rows, int S) {
   griddep_wait();
   griddep_launch_dependents();
-  const long long n8 = static_cast<long long>(S) * S / 8;
+  const long long n8 = static_cast<long long>(rows) * S / 8;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < n8;
        i += static_cast<long long>(gridDim.x) * blockDim.x) {
     const long long e = i * 8;

@@ -87,7 +87,9 @@ struct GemmCfg {
 };
 
 struct GemmArgs {
-  CUtensorMap tmA;               // A [M, K] bf16 row-major, box {64, 128}
+  // A [M, K] bf16 row-major, box {64, 128}: one map, or (a_per_shard, column
+  // mode) one per shard, so that t independent products A_s B_s run in one launch.
+  CUtensorMap tmA[MAX_SHARDS];
   CUtensorMap tmB[MAX_SHARDS];   // B shard s: [k rows, n cols] box {64, 64}, or K-major [n rows, k cols] box {64, BN/CG}
   // Output maps, 3-D {cols, M, splits}, box {128 B of columns, 128, 1}, 128-byte
   // swizzle: column mode one per shard (its column slice of C), row mode one.
@@ -130,6 +132,7 @@ struct GemmArgs {
   CUtensorMap tmAux[MAX_SHARDS];
   const void* aux;
   long long ld_aux;
+  int a_per_shard;
 };
 
 enum : int { EPI_PLAIN = 0, EPI_AUX_PRE = 1, EPI_GRAD = 2 };
@@ -376,7 +379,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
     mbar_fence_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&p.tmA);
+    for (int s = 0; s < (p.a_per_shard ? p.t : 1); ++s) tma_prefetch_desc(&p.tmA[s]);
     for (int s = 0; s < p.t; ++s) tma_prefetch_desc(&p.tmB[s]);
   }
   if (warp == 2 && lane == 0) {
@@ -416,6 +419,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         int kb_begin, kb_end;
         split_range(p, unit / num_tiles, kb_begin, kb_end);
         const TileCoord tc = tile_coord<CG>(p, tile);
+        const CUtensorMap* mA = &p.tmA[p.a_per_shard ? tc.shard : 0];
         const int my_row0 = tc.m0 + static_cast<int>(rank) * C::BM;
         const bool my_a = my_row0 < p.M;
         const int my_aboxes = a_mn_boxes(p, my_row0);  // M-major A: 64-row boxes this CTA loads
@@ -434,7 +438,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
             if (kp < kb_end && !p.a_mnmajor) {
               int ps, pa, pb;
               kblock_coords(p, tc, kp, ps, pa, pb);
-              if (my_a) tma_prefetch_l2_2d(&p.tmA, pa, my_row0);
+              if (my_a) tma_prefetch_l2_2d(mA, pa, my_row0);
               for (int j = 0; j < my_boxes; ++j) tma_prefetch_l2_2d(&p.tmB[ps], b_x0 + j * C::B_BOX_N, pb);
             }
           }
@@ -448,9 +452,9 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
             armed[stage] = static_cast<int>(phase);
             if (p.a_mnmajor) {
               for (int j = 0; j < my_aboxes; ++j)
-                tma_load_2d(dA + j * C::B_BOX_BYTES, &p.tmA, my_row0 + j * 64, a_x, &full[stage]);
+                tma_load_2d(dA + j * C::B_BOX_BYTES, mA, my_row0 + j * 64, a_x, &full[stage]);
             } else {
-              tma_load_2d(dA, &p.tmA, a_x, my_row0, &full[stage]);
+              tma_load_2d(dA, mA, a_x, my_row0, &full[stage]);
             }
             if (p.b_kmajor) {
               if (my_boxes) tma_load_2d(dB, &p.tmB[shard], b_y, b_x0, &full[stage]);
@@ -466,9 +470,9 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
             }
             if (p.a_mnmajor) {
               for (int j = 0; j < my_aboxes; ++j)
-                tma_load_2d_pair(dA + j * C::B_BOX_BYTES, &p.tmA, my_row0 + j * 64, a_x, bar);
+                tma_load_2d_pair(dA + j * C::B_BOX_BYTES, mA, my_row0 + j * 64, a_x, bar);
             } else if (my_a) {
-              tma_load_2d_pair(dA, &p.tmA, a_x, my_row0, bar);
+              tma_load_2d_pair(dA, mA, a_x, my_row0, bar);
             }
             if (p.b_kmajor) {
               if (my_boxes) tma_load_2d_pair(dB, &p.tmB[shard], b_y, b_x0, bar);

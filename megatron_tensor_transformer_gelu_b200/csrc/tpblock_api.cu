@@ -287,6 +287,8 @@ struct GemmExtra {
   long long ld_aux = 0;
   int m_split = 0;                   // column mode, t = 1: output rows split into m_split buffers
                                      // C_shards[s] of M / m_split rows each (a multiple of 256)
+  const void* const* A_shards = nullptr;  // column mode: shard s reads its own A_shards[s] (same
+                                          // shape and lda as A): t independent products in one launch
 };
 
 template <int CG, bool WIDE>
@@ -363,11 +365,17 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
   tp::GemmArgs p;
   std::memset(&p, 0, sizeof(p));
   const long long K_total = row_mode ? static_cast<long long>(shard_k) * t : shard_k;
-  if (ex.a_mnmajor) {  // stored [K, M]; box 64 m x 64 k
-    if (!tmap_bf16(&p.tmA, A, K_total, M, lda, 64, G::BK)) return TP_ERR_CUDA;
-  } else if (!tmap_bf16(&p.tmA, A, M, K_total, lda, G::BK, G::BM)) {
-    return TP_ERR_CUDA;
+  if (ex.A_shards && (row_mode || ex.m_split > 0)) return TP_ERR_INVALID_ARG;
+  const int na = ex.A_shards ? t : 1;
+  for (int s = 0; s < na; ++s) {
+    const void* a = ex.A_shards ? ex.A_shards[s] : A;
+    if (ex.a_mnmajor) {  // stored [K, M]; box 64 m x 64 k
+      if (!tmap_bf16(&p.tmA[s], a, K_total, M, lda, 64, G::BK)) return TP_ERR_CUDA;
+    } else if (!tmap_bf16(&p.tmA[s], a, M, K_total, lda, G::BK, G::BM)) {
+      return TP_ERR_CUDA;
+    }
   }
+  p.a_per_shard = ex.A_shards ? 1 : 0;
   for (int s = 0; s < t; ++s) {
     bool ok;
     if (b_kmajor)  // shard [shard_n rows, shard_k cols]; box 64 k x (BN / CG) rows
@@ -990,18 +998,28 @@ AttnState attn_state_layout(int S, int H, int nh) {
 struct AttnBackWs {
   size_t off_dz, off_do, off_dqkv, off_dxp, off_sc, off_p, off_dp, off_ds, off_d, off_part, bytes;
 };
+// Heads whose [S, S] score, P, dP and dS matrices (12 bytes an element) the
+// backward holds at once: as many as one GEMM launch takes (MAX_SHARDS), fewer
+// where that would pass 1 GiB.
+int attn_back_group(int S, int nh) {
+  int g = nh < MAX_SHARDS ? nh : MAX_SHARDS;
+  const size_t per_head = static_cast<size_t>(S) * S * 12;
+  while (g > 1 && per_head * g > (static_cast<size_t>(1) << 30)) --g;
+  return g;
+}
 AttnBackWs attn_back_layout(int S, int H, int nh) {
   AttnBackWs w;
   const size_t s = static_cast<size_t>(S), h = static_cast<size_t>(H);
+  const size_t ss = static_cast<size_t>(attn_back_group(S, nh)) * s * s;
   w.off_dz = 0;
   w.off_do = align256(s * h * 2);
   w.off_dqkv = w.off_do + align256(s * h * 2);
   w.off_dxp = w.off_dqkv + align256(s * 3 * h * 2);
   w.off_sc = w.off_dxp + align256(s * h * 4);
-  w.off_p = w.off_sc + align256(s * s * 4);
-  w.off_dp = w.off_p + align256(s * s * 2);
-  w.off_ds = w.off_dp + align256(s * s * 4);
-  w.off_d = w.off_ds + align256(s * s * 2);
+  w.off_p = w.off_sc + align256(ss * 4);
+  w.off_dp = w.off_p + align256(ss * 2);
+  w.off_ds = w.off_dp + align256(ss * 4);
+  w.off_d = w.off_ds + align256(ss * 2);
   w.off_part = w.off_d + align256(static_cast<size_t>(nh) * s * 4);
   w.bytes = w.off_part + align256(static_cast<size_t>(LNB_MAX_CTAS) * 2 * h * 4);
   return w;
@@ -1123,73 +1141,98 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
            : launch_status();
   }
   if (st != TP_OK) return st;
-  const int eg = grid_for(static_cast<long long>(S) * S / 8, dev->sm_count);
-  for (int h = 0; h < nh; ++h) {
-    const int sh = h / hps, hj = h % hps;
-    const long long qcol = static_cast<long long>(sh) * 3 * Hs + static_cast<long long>(hj) * d;
-    const uint8_t* Qh = QKV + qcol * 2;
-    const uint8_t* Kh = QKV + (qcol + Hs) * 2;
-    const uint8_t* Vh = QKV + (qcol + 2LL * Hs) * 2;
-    const uint8_t* dOh = dO + static_cast<long long>(h) * d * 2;
-    // raw scores S = Q_h K_h^T (K_h [keys, d] is the K-major B operand)
+  // The heads go through in groups of G: each GEMM below is one launch over
+  // the group's heads (shard j of the launch = head h0 + j, with its own A, B
+  // and output), and the elementwise kernels cover the group's [G S, S] rows.
+  const int G = attn_back_group(S, nh);
+  const long long ss = static_cast<long long>(S) * S;
+  for (int h0 = 0; h0 < nh; h0 += G) {
+    const int g = nh - h0 < G ? nh - h0 : G;
+    const void *Qg[MAX_SHARDS], *Kg[MAX_SHARDS], *Vg[MAX_SHARDS], *dOg[MAX_SHARDS], *Pg[MAX_SHARDS],
+        *dSg[MAX_SHARDS];
+    void *Scg[MAX_SHARDS], *dPg[MAX_SHARDS], *dQg[MAX_SHARDS], *dKg[MAX_SHARDS], *dVg[MAX_SHARDS];
+    for (int j = 0; j < g; ++j) {
+      const int h = h0 + j, sh = h / hps, hj = h % hps;
+      const long long qcol = static_cast<long long>(sh) * 3 * Hs + static_cast<long long>(hj) * d;
+      Qg[j] = QKV + qcol * 2;
+      Kg[j] = QKV + (qcol + Hs) * 2;
+      Vg[j] = QKV + (qcol + 2LL * Hs) * 2;
+      dOg[j] = dO + static_cast<long long>(h) * d * 2;
+      Scg[j] = Sc + j * ss;
+      Pg[j] = P + j * ss;
+      dPg[j] = dP + j * ss;
+      dSg[j] = dS + j * ss;
+      dQg[j] = dQKV + qcol * 2;
+      dKg[j] = dQKV + (qcol + Hs) * 2;
+      dVg[j] = dQKV + (qcol + 2LL * Hs) * 2;
+    }
+    const int eg = grid_for(g * ss / 8, dev->sm_count);
+    // raw scores S_h = Q_h K_h^T (K_h [keys, d] is the K-major B operand)
     {
-      const void* b1[1] = {Kh};
       GemmExtra ex;
       ex.ldb = H3;
-      st = run_gemm_tc(*dev, Qh, H3, S, b1, 1, 0, d, S, Sc, S, 1, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
+      ex.A_shards = Qg;
+      ex.C_shards = Scg;
+      ex.ldc_shard = S;
+      st = run_gemm_tc(*dev, Qg[0], H3, S, Kg, g, 0, d, S, Scg[0], S, 1, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
       if (st != TP_OK) return st;
     }
     {
     ProfScope ps(K_ATTN_BACK, s);
     st = launch_pdl(tp::softmax_rebuild_kernel, dim3(eg), dim3(256), 0, s, static_cast<const float*>(Sc),
-                    lse2 + static_cast<long long>(h) * S, scale_log2, P, S) != cudaSuccess
+                    lse2 + static_cast<long long>(h0) * S, scale_log2, P, g * S, S) != cudaSuccess
              ? TP_ERR_CUDA
              : launch_status();
     }
     if (st != TP_OK) return st;
-    // dV_h = P^T dO_h into V_h's columns of dQKV (P read M-major)
+    // dV_h = P_h^T dO_h into V_h's columns of dQKV (P_h read M-major)
     {
-      const void* b1[1] = {dOh};
       GemmExtra ex;
       ex.a_mnmajor = 1;
       ex.ldb = H;
-      st = run_gemm_tc(*dev, P, S, S, b1, 1, 0, S, d, dQKV + (qcol + 2LL * Hs) * 2, H3, 0, TP_ACT_NONE, s, 1, 0,
-                       nullptr, 0, &ex);
+      ex.A_shards = Pg;
+      ex.C_shards = dVg;
+      ex.ldc_shard = H3;
+      st = run_gemm_tc(*dev, Pg[0], S, S, dOg, g, 0, S, d, dVg[0], H3, 0, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
       if (st != TP_OK) return st;
     }
-    // dP = dO_h V_h^T (V_h [keys, d] is the K-major B operand)
+    // dP_h = dO_h V_h^T (V_h [keys, d] is the K-major B operand)
     {
-      const void* b1[1] = {Vh};
       GemmExtra ex;
       ex.ldb = H3;
-      st = run_gemm_tc(*dev, dOh, H, S, b1, 1, 0, d, S, dP, S, 1, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
+      ex.A_shards = dOg;
+      ex.C_shards = dPg;
+      ex.ldc_shard = S;
+      st = run_gemm_tc(*dev, dOg[0], H, S, Vg, g, 0, d, S, dPg[0], S, 1, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
       if (st != TP_OK) return st;
     }
     {
     ProfScope ps(K_ATTN_BACK, s);
     st = launch_pdl(tp::softmax_backward_kernel, dim3(eg), dim3(256), 0, s, static_cast<const __nv_bfloat16*>(P),
-                    static_cast<const float*>(dP), static_cast<const float*>(D + static_cast<long long>(h) * S),
-                    scale, dS, S) != cudaSuccess
+                    static_cast<const float*>(dP), static_cast<const float*>(D + static_cast<long long>(h0) * S),
+                    scale, dS, g * S, S) != cudaSuccess
              ? TP_ERR_CUDA
              : launch_status();
     }
     if (st != TP_OK) return st;
-    // dQ_h = dS K_h and dK_h = dS^T Q_h into their columns of dQKV
+    // dQ_h = dS_h K_h and dK_h = dS_h^T Q_h into their columns of dQKV
     {
-      const void* b1[1] = {Kh};
       GemmExtra ex;
       ex.ldb = H3;
-      st = run_gemm_tc(*dev, dS, S, S, b1, 1, 0, S, d, dQKV + qcol * 2, H3, 0, TP_ACT_NONE, s, 1, 0, nullptr, 0,
-                       &ex);
+      ex.A_shards = dSg;
+      ex.C_shards = dQg;
+      ex.ldc_shard = H3;
+      st = run_gemm_tc(*dev, dSg[0], S, S, Kg, g, 0, S, d, dQg[0], H3, 0, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
       if (st != TP_OK) return st;
     }
     {
-      const void* b1[1] = {Qh};
       GemmExtra ex;
       ex.a_mnmajor = 1;
       ex.ldb = H3;
-      st = run_gemm_tc(*dev, dS, S, S, b1, 1, 0, S, d, dQKV + (qcol + Hs) * 2, H3, 0, TP_ACT_NONE, s, 1, 0,
-                       nullptr, 0, &ex);
+      ex.A_shards = dSg;
+      ex.C_shards = dKg;
+      ex.ldc_shard = H3;
+      st = run_gemm_tc(*dev, dSg[0], S, S, Qg, g, 0, S, d, dKg[0], H3, 0, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
       if (st != TP_OK) return st;
     }
   }

@@ -57,9 +57,19 @@ def run_and_check(S, nh, t, seed, d=128):
     assert all(e <= TOL for e in errs.values()), errs
 
 
-@pytest.mark.parametrize("S,nh,t", [(256, 2, 1), (384, 4, 2), (256, 4, 4), (512, 8, 2)])
+# The per-head GEMMs run over groups of up to 8 heads per launch: (256, 12, 4)
+# and (512, 10, 2) end on a partial group, with the group's heads spread over
+# several shards.
+@pytest.mark.parametrize("S,nh,t", [(256, 2, 1), (384, 4, 2), (256, 4, 4), (512, 8, 2), (256, 12, 4),
+                                    (512, 10, 2)])
 def test_attention_backward_small(cuda_device, S, nh, t):
     run_and_check(S, nh, t, seed=S + nh + t)
+
+
+def test_attention_backward_group_of_seven(cuda_device):
+    """S = 3456: eight heads' [S, S] matrices would pass 1 GiB, so the heads go
+    through as a group of 7 and a group of 1."""
+    run_and_check(3456, 8, 2, seed=11)
 
 
 @pytest.mark.slow

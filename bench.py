@@ -247,14 +247,14 @@ class Problem:
             self.dg = torch.empty(H, dtype=torch.float32, device=dev)
             self.db = torch.empty(H, dtype=torch.float32, device=dev)
             att = 2 * 2 * S * S * w.d * w.nh
-            # Bytes of the elementwise backward kernels: per head the rebuilt P
-            # (scores f32 in, P bf16 out) and dS (P bf16 + dP f32 in, dS bf16
-            # out); D = rowsum(dO * O) reads dO and O once.
+            # Bytes of the backward's elementwise kernel: D = rowsum(dO * O) per
+            # head reads dO and O once and writes D [nh, S] f32 (P and dS are
+            # made in GEMM epilogues).
             self.work = {"gemm_tcgen05": w.flops - att,          # every product but the fused forward attention
                          "attention_fwd": att,
                          "reduce_residual_layernorm": 2 * (S * H * 8 + H * 8),
                          "layernorm_backward": S * H * (4 + 2 + 2 + 2),
-                         "attention_backward_elementwise": w.nh * S * S * (4 + 2 + 2 + 4 + 2) + S * H * 4}
+                         "attention_backward_elementwise": S * H * 4 + w.nh * S * 4}
             self.Xh_src = inp.X
 
             def attn_train_step(X, Y, st):

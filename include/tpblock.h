@@ -346,7 +346,7 @@ int tp_selftest_wait_timeout(long long limit_cycles, void* stream);
  * the launch's stream.  tp_profile_collect synchronises those events and
  * writes per kernel kind (0 tensor-core GEMM, 1 reduce+residual+LayerNorm,
  * 2 f32 CUDA-core GEMM, 3 attention, 4 LayerNorm backward, 5 the attention
- * backward's elementwise kernels): `launches` = all launches, `timed` = the
+ * backward's elementwise row-dot kernel): `launches` = all launches, `timed` = the
  * launches with events, `ms` = their summed device milliseconds; then it
  * clears the record.  Any output array may be NULL.  Returns the number of
  * kinds written (<= max_kinds), or -TP_ERR_CUDA.  Not thread-safe: enable,

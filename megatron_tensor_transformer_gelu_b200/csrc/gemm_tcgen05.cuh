@@ -123,6 +123,11 @@ struct GemmArgs {
   // pre-activation acc (bf16) through tmAux (same tiling as C).  EPI_GRAD: bf16
   // C = acc * Act'(U), with U read from `aux` (bf16, row stride ld_aux, same
   // columns as C) — the backward of the activation fused into the GEMM.
+  // EPI_SOFTMAX: bf16 C = 2^(acc * epi_scale - r), and EPI_DSOFTMAX: bf16
+  // C = P (acc - r) epi_scale with P read from `aux` like U, where
+  // r = rowvec[shard * rowvec_ld + row] (the softmax rebuilt from its log2
+  // denominators, and its backward, fused into the attention backward's score
+  // and dP GEMMs).
   int epi_mode;
   // Output rows split into shards of m_split_rows rows (0: off; a multiple
   // of the tile height): rows [s m_split_rows, (s+1) m_split_rows) go through
@@ -133,9 +138,12 @@ struct GemmArgs {
   const void* aux;
   long long ld_aux;
   int a_per_shard;
+  const float* rowvec;
+  long long rowvec_ld;
+  float epi_scale;
 };
 
-enum : int { EPI_PLAIN = 0, EPI_AUX_PRE = 1, EPI_GRAD = 2 };
+enum : int { EPI_PLAIN = 0, EPI_AUX_PRE = 1, EPI_GRAD = 2, EPI_SOFTMAX = 3, EPI_DSOFTMAX = 4 };
 
 __device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& kb0, int& kb1) {
   kb0 = static_cast<int>(static_cast<long long>(split) * p.k_blocks / p.splits);
@@ -219,6 +227,72 @@ __device__ __forceinline__ void epi_chunk_grad(uint32_t taddr, uint8_t* stage_ro
         const int i0 = 8 * j + 2 * e;
         w4[e] = pack_bf16x2(__uint_as_float(r[i0]) * act_grad_t<ACT>(u[i0]),
                             __uint_as_float(r[i0 + 1]) * act_grad_t<ACT>(u[i0 + 1]));
+      }
+      *reinterpret_cast<uint4*>(stage_row + (((4 * h + j) ^ (row_local & 7)) << 4)) =
+          make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+  }
+}
+
+// Softmax epilogue chunk (bf16 out, 64 columns): 2^(acc * scale - r).
+__device__ __forceinline__ void epi_chunk_softmax(uint32_t taddr, uint8_t* stage_row, int row_local, float r,
+                                                  float scale) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(taddr + h * 32, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i0 = 8 * j + 2 * e;
+        w4[e] = pack_bf16x2(exp2f(fmaf(__uint_as_float(v[i0]), scale, -r)),
+                            exp2f(fmaf(__uint_as_float(v[i0 + 1]), scale, -r)));
+      }
+      *reinterpret_cast<uint4*>(stage_row + (((4 * h + j) ^ (row_local & 7)) << 4)) =
+          make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
+  }
+}
+
+// Softmax-backward epilogue chunk (bf16 out, 64 columns): P (acc - r) scale,
+// with this thread's P values read from global memory 32 at a time as in
+// epi_chunk_grad (columns past `nvalid` and rows past M use P = 0).
+__device__ __forceinline__ void epi_chunk_dsoftmax(uint32_t taddr, uint8_t* stage_row, int row_local,
+                                                   const __nv_bfloat16* prow, int nvalid, float r, float scale) {
+#pragma unroll 1
+  for (int h = 0; h < 2; ++h) {
+    float pv[32];
+    const int nv = nvalid - 32 * h;
+    if (prow != nullptr && nv >= 32) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4*>(prow + 32 * h) + j);
+        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = __bfloat1622float2(hv[e]);
+          pv[8 * j + 2 * e] = f.x;
+          pv[8 * j + 2 * e + 1] = f.y;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int j = 0; j < 32; ++j) pv[j] = (prow != nullptr && j < nv) ? __bfloat162float(prow[32 * h + j]) : 0.0f;
+    }
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(taddr + h * 32, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t w4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i0 = 8 * j + 2 * e;
+        w4[e] = pack_bf16x2(pv[i0] * (__uint_as_float(v[i0]) - r) * scale,
+                            pv[i0 + 1] * (__uint_as_float(v[i0 + 1]) - r) * scale);
       }
       *reinterpret_cast<uint4*>(stage_row + (((4 * h + j) ^ (row_local & 7)) << 4)) =
           make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -596,6 +670,9 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       const int nchunks = (tc.n_valid + cw - 1) / cw;
       const int parts = p.epi_mode == EPI_AUX_PRE ? 2 : 1;  // aux (pre-activation) store first
       const int grow = y0 + row_local;
+      const float rv = (p.rowvec != nullptr && grow < p.M)
+                           ? __ldg(p.rowvec + static_cast<long long>(tc.shard) * p.rowvec_ld + grow)
+                           : 0.0f;
       for (int c = 0; c < nchunks; ++c) {
         for (int part = 0; part < parts; ++part) {
           // The TMA store that last read this staging buffer must be done with it.
@@ -603,7 +680,15 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
           named_barrier_sync(1, 128);
           uint8_t* stage_row = sEpi + buf * C::EPI_BUF_BYTES + row_local * 128;
           const uint32_t taddr = t_row + c * (p.out_f32 ? 32 : 64);
-          if (p.epi_mode == EPI_GRAD) {
+          if (p.epi_mode == EPI_SOFTMAX) {
+            epi_chunk_softmax(taddr, stage_row, row_local, rv, p.epi_scale);
+          } else if (p.epi_mode == EPI_DSOFTMAX) {
+            const __nv_bfloat16* prow =
+                grow < p.M ? static_cast<const __nv_bfloat16*>(p.aux) + static_cast<long long>(grow) * p.ld_aux +
+                                 tc.out_col0 + c * 64
+                           : nullptr;
+            epi_chunk_dsoftmax(taddr, stage_row, row_local, prow, tc.n_valid - c * 64, rv, p.epi_scale);
+          } else if (p.epi_mode == EPI_GRAD) {
             const __nv_bfloat16* urow =
                 grow < p.M ? static_cast<const __nv_bfloat16*>(p.aux) + static_cast<long long>(grow) * p.ld_aux +
                                  tc.out_col0 + c * 64

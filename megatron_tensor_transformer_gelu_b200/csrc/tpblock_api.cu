@@ -289,6 +289,9 @@ struct GemmExtra {
                                      // C_shards[s] of M / m_split rows each (a multiple of 256)
   const void* const* A_shards = nullptr;  // column mode: shard s reads its own A_shards[s] (same
                                           // shape and lda as A): t independent products in one launch
+  const float* rowvec = nullptr;     // EPI_SOFTMAX / EPI_DSOFTMAX: row values r, shard s at
+  long long rowvec_ld = 0;           //   rowvec + s * rowvec_ld
+  float epi_scale = 1.0f;
 };
 
 template <int CG, bool WIDE>
@@ -385,8 +388,14 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
       ok = tmap_bf16(&p.tmB[s], B[s], shard_k, shard_n, ex.ldb ? ex.ldb : shard_n, G::B_BOX_N, G::BK);
     if (!ok) return TP_ERR_CUDA;
   }
+  const bool softmax_epi = ex.epi_mode == tp::EPI_SOFTMAX || ex.epi_mode == tp::EPI_DSOFTMAX;
+  if (softmax_epi && (out_f32 || row_mode || !ex.rowvec || (ex.epi_mode == tp::EPI_DSOFTMAX && !ex.aux)))
+    return TP_ERR_INVALID_ARG;
   p.a_mnmajor = ex.a_mnmajor;
   p.epi_mode = ex.epi_mode;
+  p.rowvec = ex.rowvec;
+  p.rowvec_ld = ex.rowvec_ld;
+  p.epi_scale = ex.epi_scale;
   p.aux = ex.aux;
   p.ld_aux = ex.ld_aux;
   p.C = C;
@@ -996,14 +1005,14 @@ AttnState attn_state_layout(int S, int H, int nh) {
   return a;
 }
 struct AttnBackWs {
-  size_t off_dz, off_do, off_dqkv, off_dxp, off_sc, off_p, off_dp, off_ds, off_d, off_part, bytes;
+  size_t off_dz, off_do, off_dqkv, off_dxp, off_p, off_ds, off_d, off_part, bytes;
 };
-// Heads whose [S, S] score, P, dP and dS matrices (12 bytes an element) the
-// backward holds at once: as many as one GEMM launch takes (MAX_SHARDS), fewer
-// where that would pass 1 GiB.
+// Heads whose [S, S] P and dS matrices (bf16, 4 bytes an element for the
+// two) the backward holds at once: as many as one GEMM launch takes
+// (MAX_SHARDS), fewer where that would pass 1 GiB.
 int attn_back_group(int S, int nh) {
   int g = nh < MAX_SHARDS ? nh : MAX_SHARDS;
-  const size_t per_head = static_cast<size_t>(S) * S * 12;
+  const size_t per_head = static_cast<size_t>(S) * S * 4;
   while (g > 1 && per_head * g > (static_cast<size_t>(1) << 30)) --g;
   return g;
 }
@@ -1015,19 +1024,12 @@ AttnBackWs attn_back_layout(int S, int H, int nh) {
   w.off_do = align256(s * h * 2);
   w.off_dqkv = w.off_do + align256(s * h * 2);
   w.off_dxp = w.off_dqkv + align256(s * 3 * h * 2);
-  w.off_sc = w.off_dxp + align256(s * h * 4);
-  w.off_p = w.off_sc + align256(ss * 4);
-  w.off_dp = w.off_p + align256(ss * 2);
-  w.off_ds = w.off_dp + align256(ss * 4);
+  w.off_p = w.off_dxp + align256(s * h * 4);
+  w.off_ds = w.off_p + align256(ss * 2);
   w.off_d = w.off_ds + align256(ss * 2);
   w.off_part = w.off_d + align256(static_cast<size_t>(nh) * s * 4);
   w.bytes = w.off_part + align256(static_cast<size_t>(LNB_MAX_CTAS) * 2 * h * 4);
   return w;
-}
-int grid_for(long long n8, int sms) {
-  const long long b = (n8 + 255) / 256;
-  const long long cap = 8LL * sms;
-  return static_cast<int>(b < cap ? (b < 1 ? 1 : b) : cap);
 }
 }  // namespace
 
@@ -1095,9 +1097,7 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
   uint8_t* dO = wb + W.off_do;
   uint8_t* dQKV = wb + W.off_dqkv;
   float* dXp = reinterpret_cast<float*>(wb + W.off_dxp);
-  float* Sc = reinterpret_cast<float*>(wb + W.off_sc);
   __nv_bfloat16* P = reinterpret_cast<__nv_bfloat16*>(wb + W.off_p);
-  float* dP = reinterpret_cast<float*>(wb + W.off_dp);
   __nv_bfloat16* dS = reinterpret_cast<__nv_bfloat16*>(wb + W.off_ds);
   float* D = reinterpret_cast<float*>(wb + W.off_d);
   float* part = reinterpret_cast<float*>(wb + W.off_part);
@@ -1143,14 +1143,16 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
   if (st != TP_OK) return st;
   // The heads go through in groups of G: each GEMM below is one launch over
   // the group's heads (shard j of the launch = head h0 + j, with its own A, B
-  // and output), and the elementwise kernels cover the group's [G S, S] rows.
+  // and output).  P and dS are [S, G S] with head j in columns [j S, (j+1) S);
+  // the softmax and its backward run in the epilogues of the GEMMs that make
+  // the scores and dP, so neither f32 matrix reaches memory.
   const int G = attn_back_group(S, nh);
-  const long long ss = static_cast<long long>(S) * S;
+  const long long GS = static_cast<long long>(G) * S;
   for (int h0 = 0; h0 < nh; h0 += G) {
     const int g = nh - h0 < G ? nh - h0 : G;
     const void *Qg[MAX_SHARDS], *Kg[MAX_SHARDS], *Vg[MAX_SHARDS], *dOg[MAX_SHARDS], *Pg[MAX_SHARDS],
         *dSg[MAX_SHARDS];
-    void *Scg[MAX_SHARDS], *dPg[MAX_SHARDS], *dQg[MAX_SHARDS], *dKg[MAX_SHARDS], *dVg[MAX_SHARDS];
+    void *dQg[MAX_SHARDS], *dKg[MAX_SHARDS], *dVg[MAX_SHARDS];
     for (int j = 0; j < g; ++j) {
       const int h = h0 + j, sh = h / hps, hj = h % hps;
       const long long qcol = static_cast<long long>(sh) * 3 * Hs + static_cast<long long>(hj) * d;
@@ -1158,33 +1160,24 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
       Kg[j] = QKV + (qcol + Hs) * 2;
       Vg[j] = QKV + (qcol + 2LL * Hs) * 2;
       dOg[j] = dO + static_cast<long long>(h) * d * 2;
-      Scg[j] = Sc + j * ss;
-      Pg[j] = P + j * ss;
-      dPg[j] = dP + j * ss;
-      dSg[j] = dS + j * ss;
+      Pg[j] = P + static_cast<long long>(j) * S;
+      dSg[j] = dS + static_cast<long long>(j) * S;
       dQg[j] = dQKV + qcol * 2;
       dKg[j] = dQKV + (qcol + Hs) * 2;
       dVg[j] = dQKV + (qcol + 2LL * Hs) * 2;
     }
-    const int eg = grid_for(g * ss / 8, dev->sm_count);
-    // raw scores S_h = Q_h K_h^T (K_h [keys, d] is the K-major B operand)
+    // P_h = 2^(Q_h K_h^T scale_log2 - lse2_h) (K_h [keys, d] is the K-major B operand)
     {
       GemmExtra ex;
       ex.ldb = H3;
       ex.A_shards = Qg;
-      ex.C_shards = Scg;
-      ex.ldc_shard = S;
-      st = run_gemm_tc(*dev, Qg[0], H3, S, Kg, g, 0, d, S, Scg[0], S, 1, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
+      ex.epi_mode = tp::EPI_SOFTMAX;
+      ex.rowvec = lse2 + static_cast<long long>(h0) * S;
+      ex.rowvec_ld = S;
+      ex.epi_scale = scale_log2;
+      st = run_gemm_tc(*dev, Qg[0], H3, S, Kg, g, 0, d, S, P, GS, 0, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
       if (st != TP_OK) return st;
     }
-    {
-    ProfScope ps(K_ATTN_BACK, s);
-    st = launch_pdl(tp::softmax_rebuild_kernel, dim3(eg), dim3(256), 0, s, static_cast<const float*>(Sc),
-                    lse2 + static_cast<long long>(h0) * S, scale_log2, P, g * S, S) != cudaSuccess
-             ? TP_ERR_CUDA
-             : launch_status();
-    }
-    if (st != TP_OK) return st;
     // dV_h = P_h^T dO_h into V_h's columns of dQKV (P_h read M-major)
     {
       GemmExtra ex;
@@ -1193,28 +1186,23 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
       ex.A_shards = Pg;
       ex.C_shards = dVg;
       ex.ldc_shard = H3;
-      st = run_gemm_tc(*dev, Pg[0], S, S, dOg, g, 0, S, d, dVg[0], H3, 0, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
+      st = run_gemm_tc(*dev, Pg[0], GS, S, dOg, g, 0, S, d, dVg[0], H3, 0, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
       if (st != TP_OK) return st;
     }
-    // dP_h = dO_h V_h^T (V_h [keys, d] is the K-major B operand)
+    // dS_h = P_h (dO_h V_h^T - D_h) / sqrt d (V_h [keys, d] is the K-major B operand)
     {
       GemmExtra ex;
       ex.ldb = H3;
       ex.A_shards = dOg;
-      ex.C_shards = dPg;
-      ex.ldc_shard = S;
-      st = run_gemm_tc(*dev, dOg[0], H, S, Vg, g, 0, d, S, dPg[0], S, 1, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
+      ex.epi_mode = tp::EPI_DSOFTMAX;
+      ex.aux = P;
+      ex.ld_aux = GS;
+      ex.rowvec = D + static_cast<long long>(h0) * S;
+      ex.rowvec_ld = S;
+      ex.epi_scale = scale;
+      st = run_gemm_tc(*dev, dOg[0], H, S, Vg, g, 0, d, S, dS, GS, 0, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
       if (st != TP_OK) return st;
     }
-    {
-    ProfScope ps(K_ATTN_BACK, s);
-    st = launch_pdl(tp::softmax_backward_kernel, dim3(eg), dim3(256), 0, s, static_cast<const __nv_bfloat16*>(P),
-                    static_cast<const float*>(dP), static_cast<const float*>(D + static_cast<long long>(h0) * S),
-                    scale, dS, g * S, S) != cudaSuccess
-             ? TP_ERR_CUDA
-             : launch_status();
-    }
-    if (st != TP_OK) return st;
     // dQ_h = dS_h K_h and dK_h = dS_h^T Q_h into their columns of dQKV
     {
       GemmExtra ex;
@@ -1222,7 +1210,7 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
       ex.A_shards = dSg;
       ex.C_shards = dQg;
       ex.ldc_shard = H3;
-      st = run_gemm_tc(*dev, dSg[0], S, S, Kg, g, 0, S, d, dQg[0], H3, 0, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
+      st = run_gemm_tc(*dev, dSg[0], GS, S, Kg, g, 0, S, d, dQg[0], H3, 0, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
       if (st != TP_OK) return st;
     }
     {
@@ -1232,7 +1220,7 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
       ex.A_shards = dSg;
       ex.C_shards = dKg;
       ex.ldc_shard = H3;
-      st = run_gemm_tc(*dev, dSg[0], S, S, Qg, g, 0, S, d, dKg[0], H3, 0, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
+      st = run_gemm_tc(*dev, dSg[0], GS, S, Qg, g, 0, S, d, dKg[0], H3, 0, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
       if (st != TP_OK) return st;
     }
   }

@@ -67,9 +67,9 @@ def test_attention_backward_small(cuda_device, S, nh, t):
 
 
 def test_attention_backward_group_of_seven(cuda_device):
-    """S = 3456: eight heads' [S, S] matrices would pass 1 GiB, so the heads go
-    through as a group of 7 and a group of 1."""
-    run_and_check(3456, 8, 2, seed=11)
+    """S = 5888: eight heads' [S, S] P and dS matrices would pass 1 GiB, so the
+    heads go through as a group of 7 and a group of 1."""
+    run_and_check(5888, 8, 2, seed=11)
 
 
 @pytest.mark.slow

@@ -324,9 +324,12 @@ int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts,
  * tile_n == 0 (the default): a cost model picks, per launch, 256-column tiles
  * (with an optional K split for f32 partial sums) or wide tiles of up to 512
  * columns (two MMAs per K step filling TMEM) where they give fuller waves on
- * the SM pairs.  tile_n in [256, 512], a multiple of 32: every GEMM of at
- * least 129 rows uses that tile width (rounded up to a multiple of 64 for
- * bf16 output) and no K split.  Results are the same to rounding either way.
+ * the SM pairs, or 128-column tiles with an N = 128 MMA where a shard has at
+ * most 128 columns and B is N-major.  tile_n in [256, 512], a multiple of 32:
+ * every GEMM of at least 129 rows uses that tile width (rounded up to a
+ * multiple of 64 for bf16 output) and no K split.  tile_n = 128: every GEMM
+ * uses 128-column tiles (an N = 128 MMA where B is N-major) and no K split.
+ * Results are the same to rounding either way.
  * Process-wide, not thread-safe against concurrent launches.  Returns
  * TP_ERR_INVALID_ARG for other values. */
 int tp_set_gemm_tile_n(int tile_n);

@@ -84,6 +84,10 @@ struct GemmCfg {
   static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN, /*a_mn=*/false, /*b_mn=*/true);
   // B given K-major ([out, in] weights): one box of B_COLS_CTA rows x 64 k.
   static constexpr uint32_t IDESC_BK = idesc_bf16_f32(TILE_M, BN, /*a_mn=*/false, /*b_mn=*/false);
+  // Narrow tiles (tile_n == 128, N-major B, not wide): one MMA of N = 128, for
+  // which each CTA of a pair holds 64 B columns (one box).
+  static constexpr int NARROW_N = 128;
+  static constexpr uint32_t IDESC_N128 = idesc_bf16_f32(TILE_M, NARROW_N, /*a_mn=*/false, /*b_mn=*/true);
 };
 
 struct GemmArgs {
@@ -257,31 +261,33 @@ __device__ __forceinline__ void epi_chunk_softmax(uint32_t taddr, uint8_t* stage
   }
 }
 
-// Softmax-backward epilogue chunk (bf16 out, 64 columns): P (acc - r) scale,
-// with this thread's P values read from global memory 32 at a time as in
-// epi_chunk_grad (columns past `nvalid` and rows past M use P = 0).
-__device__ __forceinline__ void epi_chunk_dsoftmax(uint32_t taddr, uint8_t* stage_row, int row_local,
-                                                   const __nv_bfloat16* prow, int nvalid, float r, float scale) {
-#pragma unroll 1
-  for (int h = 0; h < 2; ++h) {
-    float pv[32];
-    const int nv = nvalid - 32 * h;
-    if (prow != nullptr && nv >= 32) {
+// Softmax-backward epilogue chunk (bf16 out, 64 columns): P (acc - r) scale.
+// The chunk's 64 P values (bf16 pairs) are loaded first, all eight 16-byte
+// loads in flight at once (columns past `nvalid` and rows past M use P = 0).
+__device__ __forceinline__ void epi_load_p64(const __nv_bfloat16* prow, int nvalid, uint32_t (&pw)[32]) {
+  if (prow != nullptr && nvalid >= 64) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(prow + 32 * h) + j);
-        const __nv_bfloat162* hv = reinterpret_cast<const __nv_bfloat162*>(&w);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = __bfloat1622float2(hv[e]);
-          pv[8 * j + 2 * e] = f.x;
-          pv[8 * j + 2 * e + 1] = f.y;
-        }
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) pv[j] = (prow != nullptr && j < nv) ? __bfloat162float(prow[32 * h + j]) : 0.0f;
+    for (int j = 0; j < 8; ++j) {
+      const uint4 w = __ldg(reinterpret_cast<const uint4*>(prow) + j);
+      pw[4 * j] = w.x;
+      pw[4 * j + 1] = w.y;
+      pw[4 * j + 2] = w.z;
+      pw[4 * j + 3] = w.w;
     }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float lo = (prow != nullptr && 2 * j < nvalid) ? __bfloat162float(prow[2 * j]) : 0.0f;
+      const float hi = (prow != nullptr && 2 * j + 1 < nvalid) ? __bfloat162float(prow[2 * j + 1]) : 0.0f;
+      pw[j] = pack_bf16x2(lo, hi);
+    }
+  }
+}
+
+__device__ __forceinline__ void epi_chunk_dsoftmax(uint32_t taddr, uint8_t* stage_row, int row_local,
+                                                   const uint32_t (&pw)[32], float r, float scale) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
     uint32_t v[32];
     tmem_ld_32x32b_x32(taddr + h * 32, v);
     tmem_wait_ld();
@@ -290,9 +296,11 @@ __device__ __forceinline__ void epi_chunk_dsoftmax(uint32_t taddr, uint8_t* stag
       uint32_t w4[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int i0 = 8 * j + 2 * e;
-        w4[e] = pack_bf16x2(pv[i0] * (__uint_as_float(v[i0]) - r) * scale,
-                            pv[i0 + 1] * (__uint_as_float(v[i0 + 1]) - r) * scale);
+        const int i0 = 8 * j + 2 * e;  // columns 32 h + i0, i0 + 1 = bf16 pair 16 h + 4 j + e
+        const uint32_t pp = pw[16 * h + 4 * j + e];
+        const float2 pf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&pp));
+        w4[e] = pack_bf16x2(pf.x * (__uint_as_float(v[i0]) - r) * scale,
+                            pf.y * (__uint_as_float(v[i0 + 1]) - r) * scale);
       }
       *reinterpret_cast<uint4*>(stage_row + (((4 * h + j) ^ (row_local & 7)) << 4)) =
           make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -387,13 +395,21 @@ __device__ __forceinline__ void kblock_coords(const GemmArgs& p, const TileCoord
 
 // Number of 64-column B boxes CTA `rank` of the pair loads for a tile (N-major
 // B); a K-major B is one box of B_COLS_CTA rows, counted here as B_BOXES.
+// Narrow tiles: B columns per CTA are NARROW_N / CG (a pair: one box each).
 template <int CG>
-__device__ __forceinline__ int b_boxes_for(int n_valid, int rank, int b_kmajor) {
+__device__ __forceinline__ int b_boxes_for(int n_valid, int rank, int b_kmajor, bool narrow = false) {
   using C = GemmCfg<CG>;
-  const int cols = min(n_valid, C::BN) - rank * C::B_COLS_CTA;
+  const int per_cta = narrow ? C::NARROW_N / CG : C::B_COLS_CTA;
+  const int cols = min(n_valid, narrow ? C::NARROW_N : C::BN) - rank * per_cta;
   if (cols <= 0) return 0;
   if (b_kmajor) return C::B_BOXES;
-  return min(C::B_BOXES, (cols + C::B_BOX_N - 1) / C::B_BOX_N);
+  return min(per_cta / C::B_BOX_N, (cols + C::B_BOX_N - 1) / C::B_BOX_N);
+}
+
+// Narrow tiles: 128-column tiles with an N-major B run one N = 128 MMA.
+template <bool WIDE>
+__device__ __forceinline__ bool narrow_tiles(const GemmArgs& p) {
+  return !WIDE && p.tile_n == 128 && !p.b_kmajor;
 }
 
 // A bytes a CTA whose rows start at row0 brings into a stage: one 128 x 64
@@ -475,6 +491,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
   griddep_launch_dependents();
 
   const int num_tiles = p.m_blocks * p.n_blocks;
+  const bool narrow = narrow_tiles<WIDE>(p);
   const int num_units = num_tiles * p.splits;
   const int cluster_id = blockIdx.x / CG;
   const int num_clusters = gridDim.x / CG;
@@ -497,14 +514,14 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         const int my_row0 = tc.m0 + static_cast<int>(rank) * C::BM;
         const bool my_a = my_row0 < p.M;
         const int my_aboxes = a_mn_boxes(p, my_row0);  // M-major A: 64-row boxes this CTA loads
-        const int my_boxes = b_boxes_for<CG>(tc.n_valid, rank, p.b_kmajor);
+        const int my_boxes = b_boxes_for<CG>(tc.n_valid, rank, p.b_kmajor, narrow);
         const int my_boxes2 = WIDE ? b2_boxes_for(tc.n_valid, p.n2, rank, p.b_kmajor) : 0;
         uint32_t bytes = 0;  // leader: bytes the whole tile stage brings in
         for (int r = 0; r < CG; ++r) {
-          bytes += a_bytes_for(p, tc.m0 + r * C::BM) + b_boxes_for<CG>(tc.n_valid, r, p.b_kmajor) * C::B_BOX_BYTES;
+          bytes += a_bytes_for(p, tc.m0 + r * C::BM) + b_boxes_for<CG>(tc.n_valid, r, p.b_kmajor, narrow) * C::B_BOX_BYTES;
           if constexpr (WIDE) bytes += b2_boxes_for(tc.n_valid, p.n2, r, p.b_kmajor) * C::B_BOX_BYTES;
         }
-        const int b_x0 = tc.n_in + static_cast<int>(rank) * C::B_COLS_CTA;
+        const int b_x0 = tc.n_in + static_cast<int>(rank) * (narrow ? C::NARROW_N / CG : C::B_COLS_CTA);
         const int b_x2 = tc.n_in + C::BN + static_cast<int>(rank) * (p.n2 / 2);  // wide: second region
         for (int kb = kb_begin; kb < kb_end; ++kb) {
           if constexpr (C::PREFETCH > 0) {
@@ -598,7 +615,8 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
           tc_fence_after();
           const uint32_t a0 = smem_u32(sA + stage * C::A_BYTES);
           const uint32_t b0 = smem_u32(sB + stage * C::B_BYTES);
-          const uint32_t idesc = (p.b_kmajor ? C::IDESC_BK : C::IDESC) | (p.a_mnmajor ? (1u << 15) : 0u);
+          const uint32_t idesc = (narrow ? C::IDESC_N128 : (p.b_kmajor ? C::IDESC_BK : C::IDESC)) |
+                                 (p.a_mnmajor ? (1u << 15) : 0u);
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk) {
             // A K-major: 16 k-elements = 32 bytes further along the swizzled row.
@@ -687,7 +705,9 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
                 grow < p.M ? static_cast<const __nv_bfloat16*>(p.aux) + static_cast<long long>(grow) * p.ld_aux +
                                  tc.out_col0 + c * 64
                            : nullptr;
-            epi_chunk_dsoftmax(taddr, stage_row, row_local, prow, tc.n_valid - c * 64, rv, p.epi_scale);
+            uint32_t pw[32];
+            epi_load_p64(prow, tc.n_valid - c * 64, pw);
+            epi_chunk_dsoftmax(taddr, stage_row, row_local, pw, rv, p.epi_scale);
           } else if (p.epi_mode == EPI_GRAD) {
             const __nv_bfloat16* urow =
                 grow < p.M ? static_cast<const __nv_bfloat16*>(p.aux) + static_cast<long long>(grow) * p.ld_aux +

@@ -253,10 +253,20 @@ TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits)
   }
   const int step = p.out_f32 ? 32 : 64;  // a 128-byte output chunk must not cross a tile edge
   if (g_force_tile_n) {
-    if (!pair) return best;
     best.splits = 1;
+    if (g_force_tile_n == 128) {  // narrow tiles, single CTAs included
+      best.tile_n = 128;
+      return best;
+    }
+    if (!pair) return best;
     best.tile_n = (g_force_tile_n + step - 1) / step * step;
     if (best.tile_n > 512) best.tile_n = 512;
+    return best;
+  }
+  // Shards of at most 128 columns with an N-major B: 128-column tiles, whose
+  // N = 128 MMA does no work on columns past the shard (same tile count).
+  if (p.shard_n <= 128 && !p.b_kmajor) {
+    best.tile_n = 128;
     return best;
   }
   if (!pair) return best;
@@ -1386,7 +1396,8 @@ int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts, c
 
 // ------------------------------------------------------------- GEMM tiling
 int tp_set_gemm_tile_n(int tile_n) {
-  if (tile_n != 0 && (tile_n < 256 || tile_n > 512 || tile_n % 32 != 0)) return TP_ERR_INVALID_ARG;
+  if (tile_n != 0 && tile_n != 128 && (tile_n < 256 || tile_n > 512 || tile_n % 32 != 0))
+    return TP_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lk(g_mu);
   g_force_tile_n = tile_n;
   return TP_OK;

@@ -187,9 +187,9 @@ def test_training_argument_checks(lib):
 
 def test_gemm_tile_override_checks(lib):
     try:
-        for bad in (-32, 100, 224, 300, 544):
+        for bad in (-32, 64, 100, 160, 224, 300, 544):
             assert lib.tp_set_gemm_tile_n(bad) == INVALID
-        for good in (256, 288, 480, 512, 0):
+        for good in (128, 256, 288, 480, 512, 0):
             assert lib.tp_set_gemm_tile_n(good) == OK
     finally:
         lib.tp_set_gemm_tile_n(0)

@@ -205,12 +205,17 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 //    that MMA work, at a lower time per MAC because every operand byte feeds
 //    more MACs (the main loop is bound by operand traffic from L2): relative
 //    time per MAC 1.0 at w = 256, 0.95 at 384, 0.88 at 448, 0.82 at 480 and
-//    0.78 at 512 (linear in between).
+//    0.75 at 512 (linear in between).  The 512 figure is the sustained one:
+//    0.78 on a cool GPU, but moving fewer operand bytes per MAC also draws
+//    less power, and under the power cap the clock stays higher (the MLP
+//    sublayer step at S2048 H4096 F16384 ran 2.1 % faster over 2000 steps
+//    with both GEMMs at 512 than with 256 and 480).
 //  * Every extra f32 partial slot of a K split costs one write and one read of
 //    M x N x 4 bytes at HBM speed (the reduce + LayerNorm kernel adds slots).
 //  * A wide tile fills TMEM, so its epilogue no longer overlaps the next
 //    tile's main loop: each wave but the last pays it (about 3.5 us per 256
-//    columns).
+//    columns, twice that for an epilogue that also stores the pre-activation
+//    or reads a second operand: U, P).
 struct TilePlan {
   int tile_n = 256;
   int splits = 1;
@@ -221,7 +226,7 @@ constexpr double T_EPI_256 = 3.5e-6;
 
 double per_mac_factor(int w) {
   static const int xs[] = {256, 384, 448, 480, 512};
-  static const double ys[] = {1.0, 0.95, 0.88, 0.82, 0.78};
+  static const double ys[] = {1.0, 0.95, 0.88, 0.82, 0.75};
   if (w <= xs[0]) return ys[0];
   for (int i = 1; i < 5; ++i)
     if (w <= xs[i]) return ys[i - 1] + (ys[i] - ys[i - 1]) * (w - xs[i - 1]) / double(xs[i] - xs[i - 1]);
@@ -270,12 +275,13 @@ TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits)
     return best;
   }
   if (!pair) return best;
+  const double epi_weight = p.epi_mode == tp::EPI_PLAIN ? 1.0 : 2.0;
   for (int w = 256 + step; w <= 512; w += step) {
     const long long wt = m_blocks * n_blocks_for(p, w);
     const long long waves = (wt + slots - 1) / slots;
     const double t = static_cast<double>(waves * p.k_blocks) * kb_cost(w) * T_KB +
-                     static_cast<double>(waves - 1) * (w / 256.0) * T_EPI_256;
-    if (t < best_t * 0.97) {  // wide tiles must buy at least 3%
+                     static_cast<double>(waves - 1) * (w / 256.0) * T_EPI_256 * epi_weight;
+    if (t < best_t * 0.98) {  // wide tiles must buy at least 2%
       best_t = t;
       best.tile_n = w;
       best.splits = 1;

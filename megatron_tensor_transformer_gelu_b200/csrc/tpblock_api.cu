@@ -1144,7 +1144,8 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
       }
     }
   }
-  // 3. Per head, through the softmax attention (P rebuilt from the scores and
+  // 3. Through the softmax attention of every head: D_h = rowsum(dO_h * O_h)
+  //    for all heads, then the heads in groups (P rebuilt from the scores and
   //    the forward's log2 denominators).
   const float scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(d)));
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));

@@ -2,7 +2,8 @@
 larger allocation whose guard regions before and after it are filled with a
 byte pattern; after the call the guards must be unchanged.  Ragged shapes put
 partial tiles at every edge the kernels clip (rows past M, columns past a
-shard or the output width), in both GEMM tile shapes."""
+shard or the output width), in every GEMM tile shape (narrow 128-column
+tiles, the cost model's choice, wide tiles)."""
 from __future__ import annotations
 
 import pytest
@@ -39,7 +40,7 @@ def _cuda(ts):
     return [x.cuda() for x in ts]
 
 
-@pytest.mark.parametrize("tile_n", [0, 480])
+@pytest.mark.parametrize("tile_n", [0, 128, 480])
 @pytest.mark.parametrize("S,H,F,t", [(200, 264, 1200, 3), (129, 1000, 2016, 2), (72, 72, 144, 1)])
 def test_mlp_forward_and_training_writes_stay_in_bounds(cuda_device, tile_n, S, H, F, t):
     inp = synth.gen_mlp(S, H, F, seed=S)
@@ -91,3 +92,37 @@ def test_attention_writes_stay_in_bounds(cuda_device):
                    _cuda(synth.split_rows_by_head(inp.Wo, nh, d, t)), nh, d, Y.t, ws.t)
     torch.cuda.synchronize()
     assert Y.intact() and ws.intact()
+
+
+@pytest.mark.parametrize("tile_n", [0, 128])
+def test_attention_training_writes_stay_in_bounds(cuda_device, tile_n):
+    """10 heads: a group of 8 and a group of 2 through the head-grouped GEMMs
+    (the second group writes only part of the P / dS workspace), 384 rows (a
+    partial 256-row tile)."""
+    S, nh, d, t = 384, 10, 128, 2
+    H = nh * d
+    inp = synth.gen_attn(S, H, seed=5)
+    dY, g, b = synth.gen_upstream(S, H, seed=6)
+    X = inp.X.cuda()
+    Wq = _cuda(synth.split_qkv_by_head(inp.Wqkv, nh, d, t))
+    Wo = _cuda(synth.split_rows_by_head(inp.Wo, nh, d, t))
+    Y = Guarded((S, H), torch.bfloat16)
+    state = Guarded((L.attn_train_state_bytes(S, H, nh, d, t),), torch.uint8)
+    bws = Guarded((L.attn_backward_workspace_bytes(S, H, nh, d, t),), torch.uint8)
+    dX = Guarded((S, H), torch.bfloat16)
+    dWq = [Guarded(tuple(w.shape), torch.float32) for w in Wq]
+    dWo = [Guarded(tuple(w.shape), torch.float32) for w in Wo]
+    dg, db = Guarded((H,), torch.float32), Guarded((H,), torch.float32)
+    try:
+        L.set_gemm_tile_n(tile_n)
+        L.attn_forward_train(X, Wq, Wo, nh, d, Y.t, state.t, gamma=g.cuda(), beta=b.cuda())
+        L.attn_backward(X, Wq, Wo, nh, d, state.t, dY.cuda(), dX.t, [w.t for w in dWq], [w.t for w in dWo], bws.t,
+                        gamma=g.cuda(), dgamma=dg.t, dbeta=db.t)
+        torch.cuda.synchronize()
+    finally:
+        L.set_gemm_tile_n(0)
+    assert L.device_error() == 0
+    for name, buf in [("Y", Y), ("state", state), ("backward workspace", bws), ("dX", dX), ("dgamma", dg),
+                      ("dbeta", db)] + [(f"dWqkv{i}", w) for i, w in enumerate(dWq)] + \
+            [(f"dWo{i}", w) for i, w in enumerate(dWo)]:
+        assert buf.intact(), name

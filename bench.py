@@ -74,12 +74,16 @@ def load_peaks():
 
 
 def source_digest() -> str:
-    """Hash of the GEMM kernel sources, to tie stored ncu counters to the code."""
+    """Hash of the GEMM kernel sources' code (line comments and blank lines
+    dropped, whitespace stripped), to tie stored ncu counters to the code."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "megatron_tensor_transformer_gelu_b200", "csrc")
     for name in ("gemm_tcgen05.cuh", "ptx.cuh"):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            for line in f:
+                code = line.split("//", 1)[0].strip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

@@ -25,7 +25,8 @@
 //               accumulator in TMEM and commits stage/accumulator releases
 //               to both CTAs.
 //   warps 2..5  epilogue: tcgen05.ld of this CTA's 128 accumulator rows,
-//               activation, 16-byte stores.
+//               activation (or another epilogue mode, see GemmArgs), a
+//               swizzled staging write, and a TMA store per 128-byte chunk.
 // The accumulator is double-buffered in TMEM (2 x 256 of the 512 columns), so
 // the epilogue of tile i overlaps the main loop of tile i+1.  No load uses
 // cluster multicast: every CTA fetches its own operand boxes.
@@ -35,6 +36,13 @@
 // [0, 256), N = n2 into [256, 256 + n2)).  The accumulator then fills TMEM and
 // is single-buffered, but every operand byte feeds more MACs and the tile
 // count can be matched to the number of SM pairs (fewer, fuller waves).
+//
+// Narrow tiles (tile_n == 128, N-major B, not wide): one MMA of N = 128 per K
+// step, each CTA of a pair holding 64 B columns, for shards of at most 128
+// columns (no MMA work on columns past the shard).
+//
+// Column mode can give each shard its own A (a_per_shard): t independent
+// products A_s B_s in one persistent launch (the attention backward's heads).
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>

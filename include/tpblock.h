@@ -334,6 +334,21 @@ int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts,
  * TP_ERR_INVALID_ARG for other values. */
 int tp_set_gemm_tile_n(int tile_n);
 
+/* The tile plan the next tensor-core GEMM launch of this shape would get (the
+ * cost model above, or the tp_set_gemm_tile_n override): host logic only, no
+ * device is touched.  M output rows; t shards, each shard_n columns of B
+ * (column mode, row_mode = 0) or shard_k rows of K (row mode, the shards
+ * summed); K = shard_k in column mode.  out_f32: f32 output (only then may the
+ * K loop be split, into at most max_splits ranges).  b_kmajor: B stored
+ * [n, k].  heavy_epilogue: the epilogue also stores the pre-activation or
+ * reads a second operand (the training step's GEMMs).  slots: co-resident
+ * CTA pairs (74 on a 148-SM B200), or SMs where M < 129 (single CTAs).
+ * Writes *tile_n (128, 256 or a wide width up to 512) and *splits.  Returns
+ * TP_ERR_INVALID_ARG for non-positive sizes, t outside [1, TP_MAX_SHARDS] or
+ * NULL outputs. */
+int tp_gemm_plan(int M, int t, int row_mode, int shard_k, int shard_n, int out_f32, int b_kmajor,
+                 int heavy_epilogue, int slots, int max_splits, int* tile_n, int* splits);
+
 /* ------------------------------------------------------------ self-test ----
  * Diagnostic for the bounded-wait path every kernel here takes when one of its
  * device-side waits gives up: launches one CTA whose mbarrier wait nothing can

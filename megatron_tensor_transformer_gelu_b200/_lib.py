@@ -66,6 +66,7 @@ SIGNATURES = {
     "tp_attn_backward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vpp, _vp, _c_float, _vp, _c_size, _vp, _vp, _vpp, _vpp,
                                                   _vp, _vp, _vp, _c_size, _vp]),
     "tp_set_gemm_tile_n": (_c_int, [_c_int]),
+    "tp_gemm_plan": (_c_int, [_c_int] * 10 + [ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
     "tp_selftest_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
     "tp_profile_enable": (_c_int, [_c_int]),
     "tp_profile_sample": (_c_int, [_c_int]),
@@ -300,8 +301,19 @@ def attn_backward(X, Wqkv_shards, Wo_shards, nh, d, state, dY, dX, dWqkv_shards,
 
 
 def set_gemm_tile_n(tile_n: int) -> None:
-    """0: the library's cost model picks GEMM tiles; 256..512: force that tile width."""
+    """0: the library's cost model picks GEMM tiles; 128: narrow tiles; 256..512:
+    force that tile width."""
     _check(lib().tp_set_gemm_tile_n(int(tile_n)), "tp_set_gemm_tile_n")
+
+
+def gemm_plan(M, t, row_mode, shard_k, shard_n, out_f32, b_kmajor=False, heavy_epilogue=False, slots=74,
+              max_splits=1):
+    """(tile_n, splits) the next GEMM launch of this shape would get (host logic only)."""
+    tn, sp = ctypes.c_int(0), ctypes.c_int(0)
+    _check(lib().tp_gemm_plan(int(M), int(t), int(bool(row_mode)), int(shard_k), int(shard_n), int(bool(out_f32)),
+                              int(bool(b_kmajor)), int(bool(heavy_epilogue)), int(slots), int(max_splits),
+                              ctypes.byref(tn), ctypes.byref(sp)), "tp_gemm_plan")
+    return tn.value, sp.value
 
 
 def selftest_wait_timeout(limit_cycles: int, stream=None):

@@ -1410,6 +1410,28 @@ int tp_set_gemm_tile_n(int tile_n) {
   return TP_OK;
 }
 
+int tp_gemm_plan(int M, int t, int row_mode, int shard_k, int shard_n, int out_f32, int b_kmajor,
+                 int heavy_epilogue, int slots, int max_splits, int* tile_n, int* splits) {
+  if (M < 1 || t < 1 || t > TP_MAX_SHARDS || shard_k < 1 || shard_n < 1 || slots < 1 || max_splits < 1 ||
+      !tile_n || !splits)
+    return TP_ERR_INVALID_ARG;
+  tp::GemmArgs p;
+  std::memset(&p, 0, sizeof(p));
+  p.M = M;
+  p.t = t;
+  p.row_mode = row_mode ? 1 : 0;
+  p.shard_k = shard_k;
+  p.shard_n = shard_n;
+  p.k_blocks = ceil_div(shard_k, tp::GemmCfg<1>::BK) * (row_mode ? t : 1);
+  p.out_f32 = out_f32 ? 1 : 0;
+  p.b_kmajor = b_kmajor ? 1 : 0;
+  p.epi_mode = heavy_epilogue ? tp::EPI_GRAD : tp::EPI_PLAIN;
+  const TilePlan plan = plan_tiles(p, M >= TP_GEMM_PAIR_MIN_ROWS, slots, out_f32 ? max_splits : 1);
+  *tile_n = plan.tile_n;
+  *splits = plan.splits;
+  return TP_OK;
+}
+
 // ------------------------------------------------------------- self-test
 int tp_selftest_wait_timeout(long long limit_cycles, void* stream) {
   if (limit_cycles < 1) return TP_ERR_INVALID_ARG;

@@ -1,0 +1,89 @@
+"""Host logic of the GEMM tile plan (tp_gemm_plan: the choice the next launch
+of a shape gets), pinned on the GEMM shapes of the workloads.  No device is
+touched.  The expected picks follow from the cost model the header documents:
+waves x k-blocks x time per k-block (relative time per MAC 1.0 at 256 columns
+down to 0.75 at 512), plus the epilogue each wave but the last exposes for
+wide tiles (doubled for epilogues that store or read a second operand), plus
+the f32 slot traffic of a K split; a wide tile must buy 2 %."""
+from __future__ import annotations
+
+import pytest
+
+from megatron_tensor_transformer_gelu_b200 import _lib as L
+from megatron_tensor_transformer_gelu_b200 import build as B
+
+PAIRS = 74  # co-resident CTA pairs on a 148-SM B200
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    B.build()
+    L.lib()
+    L.set_gemm_tile_n(0)
+
+
+# (name, M, t, row_mode, shard_k, shard_n, out_f32, b_kmajor, heavy_epilogue, max_splits) -> (tile_n, splits)
+CASES = [
+    # MLP S2048 H4096 F16384 t4: 256 tiles of 512 columns in 3.46 waves beat 512 tiles of 256 in 7
+    ("mlp GEMM1", 2048, 4, 0, 4096, 4096, 0, 0, 0, 1, (512, 1)),
+    # row split over 4 shards: 64 tiles of 512 columns, one wave, no K split
+    ("mlp GEMM2", 2048, 4, 1, 4096, 4096, 1, 0, 0, 4, (512, 1)),
+    # attention S2048 H8192 t4: QKV (3 x 2048 columns per shard) and O projection
+    ("QKV", 2048, 4, 0, 8192, 6144, 0, 0, 0, 1, (512, 1)),
+    ("O projection", 2048, 4, 1, 2048, 8192, 1, 0, 0, 4, (512, 1)),
+    # large MLP S4096 H12288 F49152 t8
+    ("large GEMM1", 4096, 8, 0, 12288, 6144, 0, 0, 0, 1, (512, 1)),
+    ("large GEMM2", 4096, 8, 1, 6144, 12288, 1, 0, 0, 4, (512, 1)),
+    # training forward GEMM1 also stores U: its exposed epilogue doubles, 256 stays
+    ("train GEMM1 + U store", 2048, 4, 0, 4096, 4096, 0, 0, 1, 1, (256, 1)),
+    # dU = (dZ B^T) * Act'(U): K-major B, reads U in the epilogue
+    ("train dU", 2048, 4, 0, 4096, 4096, 0, 1, 1, 1, (256, 1)),
+    # attention backward: dV/dQ/dK of a group of 8 heads (N = d = 128, N-major B): narrow tiles
+    ("attn dV (8 heads)", 2048, 8, 0, 2048, 128, 0, 0, 0, 1, (128, 1)),
+    # the score GEMM of a group (K = 128, K-major B, softmax epilogue): 256
+    ("attn P (8 heads)", 2048, 8, 0, 128, 2048, 0, 1, 1, 1, (256, 1)),
+    # a K-major B never gets narrow tiles (its box is 128 rows per CTA)
+    ("K-major 128 columns", 2048, 1, 0, 2048, 128, 0, 1, 0, 1, (256, 1)),
+    # single CTAs (M < 129): 256 unless narrow
+    ("single-CTA", 100, 2, 0, 512, 1024, 0, 0, 0, 1, (256, 1)),
+    ("single-CTA narrow", 100, 2, 0, 512, 64, 0, 0, 0, 1, (128, 1)),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=[c[0] for c in CASES])
+def test_plan_of_workload_gemms(case):
+    _, M, t, row, sk, sn, f32, bk, heavy, ms, want = case
+    assert L.gemm_plan(M, t, row, sk, sn, f32, bk, heavy, PAIRS, ms) == want
+
+
+def test_k_split_fills_idle_pairs():
+    """A row-split GEMM with few tiles and a long K loop (f32 out): splitting K
+    puts the idle pairs to work; never with bf16 output or max_splits = 1."""
+    tn, sp = L.gemm_plan(512, 4, 1, 4096, 1024, 1, 0, 0, PAIRS, 4)
+    assert sp > 1 and tn == 256
+    assert L.gemm_plan(512, 4, 1, 4096, 1024, 0, 0, 0, PAIRS, 4)[1] == 1
+    assert L.gemm_plan(512, 4, 1, 4096, 1024, 1, 0, 0, PAIRS, 1)[1] == 1
+
+
+def test_override_is_what_the_next_launch_gets():
+    try:
+        L.set_gemm_tile_n(480)
+        assert L.gemm_plan(2048, 4, 1, 4096, 4096, 1, 0, 0, PAIRS, 4) == (480, 1)  # f32: 32-column steps
+        assert L.gemm_plan(2048, 4, 0, 4096, 4096, 0, 0, 0, PAIRS, 1) == (512, 1)  # bf16: rounded up to 64
+        assert L.gemm_plan(100, 2, 0, 512, 1024, 0, 0, 0, PAIRS, 1) == (256, 1)    # single CTAs: no wide tiles
+        L.set_gemm_tile_n(128)
+        assert L.gemm_plan(2048, 4, 0, 4096, 4096, 0, 0, 0, PAIRS, 1) == (128, 1)
+        assert L.gemm_plan(100, 2, 0, 512, 1024, 0, 0, 0, PAIRS, 1) == (128, 1)
+    finally:
+        L.set_gemm_tile_n(0)
+    assert L.gemm_plan(2048, 4, 0, 4096, 4096, 0, 0, 0, PAIRS, 1) == (512, 1)
+
+
+def test_bad_arguments():
+    import ctypes
+    tn, sp = ctypes.c_int(), ctypes.c_int()
+    lib = L.lib()
+    for args in [(0, 4, 0, 64, 64), (64, 0, 0, 64, 64), (64, 9, 0, 64, 64), (64, 4, 0, 0, 64), (64, 4, 0, 64, 0)]:
+        assert lib.tp_gemm_plan(*args, 0, 0, 0, PAIRS, 1, ctypes.byref(tn), ctypes.byref(sp)) == 1
+    assert lib.tp_gemm_plan(64, 4, 0, 64, 64, 0, 0, 0, 0, 1, ctypes.byref(tn), ctypes.byref(sp)) == 1
+    assert lib.tp_gemm_plan(64, 4, 0, 64, 64, 0, 0, 0, PAIRS, 1, None, ctypes.byref(sp)) == 1

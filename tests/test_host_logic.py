@@ -65,6 +65,21 @@ def test_workload_flops():
     assert a.flops == 2 * 2048 * 8192 * 3 * 8192 + 4 * 2048 * 2048 * 128 * 64 + 2 * 2048 * 8192 * 8192
 
 
+def test_training_workload_flops():
+    """A training step counts every product of the forward and the backward:
+    the MLP's 2 forward GEMMs plus dU, dX, dA, dB (each 2 S H F); the attention
+    sublayer's forward plus dO, dWo, the five per-head products of the softmax
+    attention's backward (each 2 S^2 d per head) and dX, dWqkv."""
+    S, H, F = 2048, 4096, 16384
+    assert WORKLOADS["mlp_train_s2048_h4096_f16384"].flops == 6 * 2 * S * H * F
+    S, H, nh, d = 2048, 8192, 64, 128
+    qkv, oproj = 2 * S * H * 3 * H, 2 * S * H * H
+    fwd = qkv + 4 * S * S * d * nh + oproj
+    bwd = 2 * oproj + 5 * 2 * S * S * d * nh + 2 * qkv
+    assert WORKLOADS["attn_train_s2048_h8192_64x128"].flops == fwd + bwd
+    assert round((fwd + bwd) / 1e9, 1) == 3779.5
+
+
 def test_row_sample_deterministic_and_bounded():
     r1 = synth.row_sample(2048, 1)
     r2 = synth.row_sample(2048, 1)

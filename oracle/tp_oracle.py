@@ -17,7 +17,7 @@ Pages cited (by title and section):
   [0539]  "1. 张量并行：Tensor Parallelism" (0539edu.com news 288531)
   [PWWT]  "TP到底在切什么——从一次矩阵乘法说起" (pwwt.cn news 5934571)
 
-Readings where the pages are silent or garbled (each is listed in the design doc):
+Readings adopted where the pages are silent, garbled or contradict each other:
   * A is split by columns and B by rows ([TYPC] §3 MLP bullet; [0539] §1.2.1);
     the [PWWT] §2.3 labels are swapped and are not followed.
   * Post-LN: Y = LN(X + sum_i Act(X A_i) B_i); no LayerNorm on the input.

@@ -164,6 +164,24 @@ def check_linears_exact():
     np.testing.assert_array_equal(O.linear_column(X, W, act="relu"), np.maximum(ref, 0))
 
 
+def check_column_blocking():
+    """The oracle forms wide products one block of output columns at a time.
+    With a block of a few columns every product in the exact brute-force,
+    closed-form and library pins crosses several blocks and ends in a ragged
+    one, so a slice error in the block loop shows up against values computed
+    without it."""
+    saved = O._COL_BLOCK
+    try:
+        for blk in (1, 2, 3, 5):
+            O._COL_BLOCK = blk
+            check_mlp_exact_bruteforce()
+            check_linears_exact()
+            check_mlp_closed_forms()
+            check_attention_library()
+    finally:
+        O._COL_BLOCK = saved
+
+
 def check_attention_hand():
     # one head, d = 1, two keys: scores [0, ln 3] -> softmax [1/4, 3/4]
     Q = np.array([[1.0]])
@@ -404,7 +422,7 @@ def check_attention_backward_autograd():
 ALL_CHECKS = [
     check_gelu_library, check_gelu_identities, check_layernorm_hand, check_layernorm_invariants,
     check_mlp_exact_bruteforce, check_mlp_closed_forms, check_mlp_block_identities,
-    check_mlp_symmetries, check_linears_exact, check_attention_hand,
+    check_mlp_symmetries, check_linears_exact, check_column_blocking, check_attention_hand,
     check_attention_uniform_keys, check_attention_library, check_attention_row_equivariance,
     check_block_composition, check_backward_finite_differences, check_backward_autograd,
     check_backward_invariants, check_attention_backward_finite_differences, check_attention_backward_autograd,
@@ -569,6 +587,26 @@ def _attention_backward_with(mistake: str):
     return bad
 
 
+def _bad_matmul_cols_short_block(Xr, W, act="none"):
+    # each block stops one column short of the next block's start
+    n = W.shape[1]
+    out = np.zeros((Xr.shape[0], n), dtype=np.float64)
+    for c0 in range(0, n, O._COL_BLOCK):
+        c1 = min(n, c0 + O._COL_BLOCK - 1)
+        out[:, c0:c1] = O.activation(Xr @ O._f64(W[:, c0:c1]), act)
+    return out
+
+
+def _bad_matmul_cols_ragged_tail_dropped(Xr, W, act="none"):
+    # the last, partial block is never formed
+    n = W.shape[1]
+    out = np.zeros((Xr.shape[0], n), dtype=np.float64)
+    for c0 in range(0, n - n % O._COL_BLOCK, O._COL_BLOCK):
+        c1 = c0 + O._COL_BLOCK
+        out[:, c0:c1] = O.activation(Xr @ O._f64(W[:, c0:c1]), act)
+    return out
+
+
 _PLANTED = [
     ("layernorm", _bad_layernorm_unbiased),
     ("layernorm", _bad_layernorm_eps_outside),
@@ -583,6 +621,8 @@ _PLANTED = [
     ("activation_grad", _bad_activation_grad_is_activation),
     ("mlp_block_backward", _bad_backward_no_residual),
     ("mlp_block_backward", _bad_backward_db_from_u),
+    ("_matmul_cols", _bad_matmul_cols_short_block),
+    ("_matmul_cols", _bad_matmul_cols_ragged_tail_dropped),
 ] + [("attention_sublayer_backward", _attention_backward_with(m))
       for m in ("no_softmax_projection", "no_scale", "dk_untransposed", "dv_untransposed", "dwo_transposed",
                 "no_residual")]

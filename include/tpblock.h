@@ -182,11 +182,14 @@ int tp_mlp_backward_ex(int S, int H, int F, int t, int dtype, int w_layout, cons
  * the scratch is a fixed device array inside the library, of
  * tp_noalloc_scratch_bytes() bytes (32 MiB), held on every GPU that loads the
  * library until the process exits.
- *  - Sizes whose tp_mlp_workspace_bytes() exceeds that maximum are rejected
- *    with TP_ERR_WORKSPACE_TOO_SMALL before anything is launched.
- *  - The call allocates nothing.  Its first call on a device looks up the
- *    array's device address (with that device current); make that first call
- *    before any stream capture.
+ *  - Arguments are checked first, exactly as tp_mlp_forward checks them
+ *    (same statuses).  Then sizes whose tp_mlp_workspace_bytes() exceeds the
+ *    maximum are rejected with TP_ERR_WORKSPACE_TOO_SMALL before anything is
+ *    launched.
+ *  - The call allocates nothing.  Its first call on a device whose arguments
+ *    pass the checks looks up the array's device address (with that device
+ *    current); an empty call (S == 0, X and Y may be NULL) is enough.  Make
+ *    that first call before any stream capture.
  *  - Every call on a device shares the array: calls whose kernels may overlap
  *    on the GPU race on it; order them on one stream.  Nothing in it needs to
  *    start at zero. */

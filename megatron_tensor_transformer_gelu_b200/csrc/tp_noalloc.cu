@@ -21,13 +21,17 @@
 //  * In host code `g_tp_noalloc_scratch` names a host-side stand-in, not a
 //    device address.  Its device address is looked up once per device with
 //    cudaGetSymbolAddress, with that device current, during the first call
-//    on that device.  Make that first call before any stream capture.
+//    on that device whose arguments pass the checks (an empty call with
+//    S == 0 is enough).  Make that first call before any stream capture.
+//  * Order of checks: the arguments (as tp_mlp_forward checks them), then
+//    the address lookup, then the size limit.
 #include <cuda_runtime.h>
 
 #include <cstdint>
 #include <mutex>
 
 #include "../../include/tpblock.h"
+#include "tp_internal.h"
 
 namespace {
 
@@ -63,14 +67,16 @@ size_t tp_noalloc_scratch_bytes(void) { return TP_NOALLOC_SCRATCH_BYTES; }
 int tp_mlp_forward_noalloc(int S, int H, int F, int t, int dtype, int out_dtype, const void* X,
                            const void* const* A_shards, const void* const* B_shards, const float* gamma,
                            const float* beta, float eps, int act, void* Y, void* stream) {
-  const size_t need = tp_mlp_workspace_bytes(S, H, F, t, dtype);
-  if (need > TP_NOALLOC_SCRATCH_BYTES) return TP_ERR_WORKSPACE_TOO_SMALL;
-  if (need == 0)  // empty or invalid sizes: the regular entry point answers
-    return tp_mlp_forward(S, H, F, t, dtype, out_dtype, X, A_shards, B_shards, gamma, beta, eps, act, Y, nullptr, 0,
-                          stream);
-  void* scratch = nullptr;
-  const int st = noalloc_scratch(&scratch);
+  // 1. The same argument checks as tp_mlp_forward, in the same order.
+  int st = tp_internal_check_mlp_args(S, H, F, t, dtype, out_dtype, X, A_shards, B_shards, gamma, beta, eps, act, Y);
   if (st != TP_OK) return st;
+  // 2. The scratch array's device address on the current device, looked up on
+  //    the first call there (an empty call, S == 0, does it too).
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != TP_OK) return st;
+  // 3. The size limit: nothing is launched for sizes the array cannot hold.
+  if (tp_mlp_workspace_bytes(S, H, F, t, dtype) > TP_NOALLOC_SCRATCH_BYTES) return TP_ERR_WORKSPACE_TOO_SMALL;
   return tp_mlp_forward(S, H, F, t, dtype, out_dtype, X, A_shards, B_shards, gamma, beta, eps, act, Y, scratch,
                         TP_NOALLOC_SCRATCH_BYTES, stream);
 }

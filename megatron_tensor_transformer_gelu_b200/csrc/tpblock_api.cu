@@ -20,6 +20,7 @@
 #include "ln_backward.cuh"
 #include "reduce_ln.cuh"
 #include "simt_f32.cuh"
+#include "tp_internal.h"
 
 namespace {
 
@@ -780,6 +781,12 @@ int check_attn_args(int S, int H, int nh, int d, int t, int dtype, int out_dtype
 }
 
 }  // namespace
+
+int tp_internal_check_mlp_args(int S, int H, int F, int t, int dtype, int out_dtype, const void* X,
+                               const void* const* A_shards, const void* const* B_shards, const float* gamma,
+                               const float* beta, float eps, int act, const void* Y) {
+  return check_mlp_args(S, H, F, t, dtype, out_dtype, X, A_shards, B_shards, gamma, beta, eps, act, Y);
+}
 
 extern "C" {
 

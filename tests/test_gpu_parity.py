@@ -253,10 +253,13 @@ def test_mlp_s2048_h4096_f16384(cuda_device, t):
 @pytest.mark.parametrize("t", [4, 1, 2, 8])
 def test_attn_s2048_h8192(cuda_device, t):
     w = WORKLOADS["attn_s2048_h8192_64x128"]
-    inp = synth.gen_attn(w.S, w.H, seed=w.seed)
+    if w.name not in _CACHE:  # inputs and the oracle's 64 sampled rows, shared by every t
+        inp = synth.gen_attn(w.S, w.H, seed=w.seed)
+        rows = synth.row_sample(w.S, w.seed + 1)
+        _CACHE[w.name] = (inp, rows, O.attention_sublayer(inp.X, inp.Wqkv, inp.Wo, w.nh, w.d, rows=rows))
+    inp, rows, ref = _CACHE[w.name]
     Y = run_attn(inp, w.nh, w.d, t)
-    rows = synth.row_sample(w.S, w.seed + 1, n=16)
-    ref = O.attention_sublayer(inp.X, inp.Wqkv, inp.Wo, w.nh, w.d, rows=rows)
+    assert len(rows) == 64
     assert rel_err(Y[rows], ref) <= TOL_BF16
 
 
@@ -265,7 +268,8 @@ def test_mlp_s4096_h12288_f49152(cuda_device):
     w = WORKLOADS["mlp_s4096_h12288_f49152"]
     inp = synth.gen_mlp(w.S, w.H, w.F, seed=w.seed)
     Y = run_mlp(inp, w.t)
-    rows = synth.row_sample(w.S, w.seed + 1, n=8)
+    rows = synth.row_sample(w.S, w.seed + 1)
+    assert len(rows) == 64  # rows 0 and S-1 and 62 drawn; they fall in all 16 of the 256-row tiles
     assert rel_err(Y[rows], O.mlp_block(inp.X, inp.A, inp.B, rows=rows)) <= TOL_BF16
 
 

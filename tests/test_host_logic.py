@@ -104,3 +104,29 @@ def test_bf16_storage_is_rounded_fp32_draw():
     h = synth.gen_mlp(8, 16, 32, seed=5, dtype=torch.bfloat16)
     assert torch.equal(f.X.to(torch.bfloat16), h.X)
     assert torch.equal(f.A.to(torch.bfloat16), h.A)
+
+
+def test_bench_kernel_table_roofline_arithmetic():
+    """bench.py's per-kernel roofline: algorithmic work per launch (work per
+    step / launches per step) over the mean event-timed launch duration; the
+    f32 CUDA-core kind against SMs x 128 FMA x 2 x clock."""
+    import bench
+    peaks = {"bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6500.0, "source": "measured"}
+    steps = 4
+    # 2 GEMM launches per step of 1e12 FLOP each, 2 ms each; 1 LayerNorm launch of 6.5e9 B taking 1 ms
+    prof = {"gemm_tcgen05": (8, 8, 16.0), "reduce_residual_layernorm": (4, 4, 4.0), "attention_fwd": (0, 0, 0.0)}
+    work = {"gemm_tcgen05": 2e12, "reduce_residual_layernorm": 6.5e9}
+    k = bench.kernel_table(prof, work, steps, peaks)
+    assert k["gemm_tcgen05"]["achieved"] == pytest.approx(500.0)
+    assert k["gemm_tcgen05"]["frac"] == pytest.approx(500.0 / 1600.0, abs=1e-4)
+    assert k["gemm_tcgen05"]["flops_per_launch"] == 1e12
+    assert k["reduce_residual_layernorm"]["achieved"] == pytest.approx(6500.0)
+    assert k["reduce_residual_layernorm"]["frac"] == pytest.approx(1.0)
+    assert k["gemm_tcgen05"]["share_of_step"] == pytest.approx(0.8)
+    dom, roof = bench.dominant(k, peaks, "none")
+    assert dom == "gemm_tcgen05" and roof["frac_of_sustained"] == pytest.approx(500.0 / 1400.0, abs=1e-4)
+    # f32 FMA peak of 148 SMs at 1965 MHz: 148 * 128 * 2 * 1.965e9 = 74.45 TFLOP/s
+    assert bench.alu_peak(148, 1965.0) == pytest.approx(74.449, abs=1e-3)
+    ka = bench.kernel_table({"gemm_simt_f32": (2, 2, 0.004)}, {"gemm_simt_f32": 1.34e8}, 1, peaks, 74.449)
+    assert ka["gemm_simt_f32"]["bound"] == "alu"
+    assert ka["gemm_simt_f32"]["achieved"] == pytest.approx(1.34e8 / 2 / 2e-6 / 1e12, abs=0.01)

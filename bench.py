@@ -24,6 +24,12 @@ roofline and its parity against the fp64 oracle on 64 sampled rows; and a
 `sustained` figure, the headline step run back to back for a few seconds
 under the GPU's power cap.
 
+`--tp allreduce|rs_ag` (torchrun, N ranks) splits one sublayer over the GPUs
+instead: rank r holds shard r of the weights, computes its partial sum, and
+the partials are reduced by an NCCL AllReduce, or by ReduceScatter ->
+LayerNorm on S/N rows -> AllGather (strong scaling: `value` is the one
+sublayer's FLOPs over the slowest rank's time).
+
 `--impl reference` times the fp64 CPU oracle on the host cores instead (rows
 sampled from the same workload each step); see the JSON's cpu_baseline.
 """
@@ -72,6 +78,9 @@ def parse():
     ap.add_argument("--sustained-seconds", type=float, default=3.0,
                     help="length of the back-to-back headline run (0: skip)")
     ap.add_argument("--no-other-workloads", action="store_true")
+    ap.add_argument("--tp", choices=["none", "allreduce", "rs_ag"], default="none",
+                    help="split the sublayer over the GPUs (tensor parallelism across ranks, strong scaling) "
+                         "instead of running one replica per GPU")
     return ap.parse_args()
 
 
@@ -376,6 +385,46 @@ class Problem:
         self.input_bytes = sum(x.numel() * x.element_size() for x in [self.X, *self.W1, *self.W2])
 
 
+class TPProblem:
+    """One rank's part of the sublayer split over `world` GPUs: the whole
+    sublayer's inputs are drawn identically on every rank and rank r keeps
+    shard r of the weights (1/world of A's columns and B's rows, or of the
+    heads); the partial sums are reduced with the collective `mode`."""
+
+    def __init__(self, w, dev, rank, world, mode, L, synth, torch):
+        from megatron_tensor_transformer_gelu_b200 import tp_dist
+        bf = torch.bfloat16
+        S, H = w.S, w.H
+        if w.kind == "mlp":
+            inp = synth.gen_mlp(S, H, w.F, seed=w.seed)
+            self.W1 = [synth.split_columns(inp.A, world)[rank].to(dev)]
+            self.W2 = [synth.split_rows(inp.B, world)[rank].to(dev)]
+            self.ws = torch.empty(L.mlp_partial_workspace_bytes(S, H, w.F // world, 1), dtype=torch.uint8, device=dev)
+            partial = tp_dist.mlp_partial_fn(self.W1, self.W2, self.ws)
+            self.work = {"gemm_tcgen05": 2 * 2 * S * H * w.F // world}
+            self.oracle = lambda O, rows: O.mlp_block(inp.X, inp.A, inp.B, rows=rows)
+        elif w.kind == "attn":
+            inp = synth.gen_attn(S, H, seed=w.seed)
+            nh_r = w.nh // world
+            self.W1 = [synth.split_qkv_by_head(inp.Wqkv, w.nh, w.d, world)[rank].to(dev)]
+            self.W2 = [synth.split_rows_by_head(inp.Wo, w.nh, w.d, world)[rank].to(dev)]
+            self.ws = torch.empty(L.attn_partial_workspace_bytes(S, H, nh_r, w.d, 1), dtype=torch.uint8, device=dev)
+            partial = tp_dist.attn_partial_fn(self.W1, self.W2, nh_r, w.d, self.ws)
+            self.work = {"gemm_tcgen05": (2 * S * H * 3 * H + 2 * S * H * H) // world,
+                         "attention_fwd": 4 * S * S * w.d * w.nh // world}
+            self.oracle = lambda O, rows: O.attention_sublayer(inp.X, inp.Wqkv, inp.Wo, w.nh, w.d, rows=rows)
+        else:
+            raise SystemExit(f"--tp takes an MLP or attention workload, not {w.name}")
+        rows = S if mode == "allreduce" else S // world
+        self.work["reduce_residual_layernorm"] = rows * H * (4 + 2 + 2) + H * 8
+        self.X = inp.X.to(dev)
+        self.Y = torch.empty(S, H, dtype=bf, device=dev)
+        self.sub = tp_dist.TPSublayer(partial, S, H, bf, bf, mode=mode, device=dev, world=world, rank=rank)
+        self.run = lambda X, Y, st: self.sub.forward(X, Y, st)
+        self.Xh_src = inp.X
+        self.input_bytes = sum(x.numel() * x.element_size() for x in [self.X, *self.W1, *self.W2])
+
+
 def time_steps(step, stream, steps, torch):
     """Device milliseconds of `steps` steps, CUDA events on the launching stream."""
     e0 = torch.cuda.Event(enable_timing=True)
@@ -427,7 +476,8 @@ def run_ours(args, rank, world, local):
     if world > 1:
         dist.barrier()
     L.lib()  # load the CUDA library (raises if it is not built)
-    P = Problem(w, dev, rank, L, synth, torch)
+    tp_mode = args.tp != "none"
+    P = TPProblem(w, dev, rank, world, args.tp, L, synth, torch) if tp_mode else Problem(w, dev, rank, L, synth, torch)
     X, Y = P.X, P.Y
     stream = torch.cuda.Stream(device=dev)
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
@@ -536,15 +586,21 @@ def run_ours(args, rank, world, local):
     if rank == 0:
         peaks = load_peaks()
         ms_step = ms_total / args.steps
-        value = whole_job_tflops(w.flops, args.steps, world, ms_total)
-        e2e_value = whole_job_tflops(w.flops, e2e_steps, world, e2e_ms)
+        # replicas: every rank runs the whole workload (weak scaling); --tp: the
+        # ranks run one workload together (strong scaling)
+        units = 1 if tp_mode else world
+        value = whole_job_tflops(w.flops, args.steps, units, ms_total)
+        e2e_value = whole_job_tflops(w.flops, e2e_steps, units, e2e_ms)
         launches = sum(v[0] for v in counted.values())
         clocks = sampler.summary(t_wall0, t_wall1)
         kinds = kernel_table(prof, P.work, kernel_steps, peaks, alu_peak(sms, clocks.get("sm_mhz")))
         dom, roof = dominant(kinds, peaks, w.name)
         others = {k: v for k, v in kinds.items() if k != dom}
-        cfg = {"workload": w.name, "t": w.t, "flops_per_step": w.flops,
-               "parallelism": f"{w.t} logical TP shards per GPU; {world} independent replica(s)",
+        parallelism = (f"tensor parallel over {world} GPU(s), one shard of A's columns and B's rows (or of the "
+                       f"heads) per GPU, partial sums reduced by {args.tp}" if tp_mode else
+                       f"{w.t} logical TP shards per GPU; {world} independent replica(s)")
+        cfg = {"workload": w.name, "t": world if tp_mode else w.t, "flops_per_step": w.flops,
+               "parallelism": parallelism,
                "l2": f"inputs larger than L2 ({P.input_bytes / 2**20:.0f} MiB resident vs {L2_BYTES // 2**20} MiB L2)"}
         for key in ("S", "H", "F", "nh", "d", "M", "K", "N"):
             if getattr(w, key):
@@ -560,7 +616,7 @@ def run_ours(args, rank, world, local):
             "warmup": args.warmup,
             "ms_per_step": round(ms_step, 5),
             "higher_is_better": True,
-            "scaling": "weak",
+            "scaling": "strong" if tp_mode else "weak",
             "vs_baseline": None,
             "dtype": w.dtype,
             "data": "synthetic (seeded torch.randn; X~N(0,1), weights~N(0,1/fan_in))",
@@ -586,6 +642,11 @@ def run_ours(args, rank, world, local):
         if sustained is not None:
             sustained["frac_of_burst_peak"] = round(sustained["value"] / peaks["bf16_tflops"], 4)
             result["sustained"] = sustained
+        if tp_mode:
+            kernel_ms = sum(k["avg_launch_ms"] * k["launches"] for k in kinds.values()) / kernel_steps
+            result["tp"] = {"mode": args.tp, "ranks": world,
+                            "collective_ms_per_step_estimate": round(max(0.0, ms_step - kernel_ms), 5),
+                            "note": "the step time less the library kernels' event-timed time per step"}
     sampler.stop()
     if world > 1:
         dist.barrier()
@@ -760,8 +821,10 @@ def main():
             cb = cpu_oracle_timing(w, rows, 1, 0)
             res["parity"] = parity_vs_oracle(w, P.Y, cb.pop("_rows"), cb.pop("_out"),
                                              tol=1e-4 if w.dtype == "f32" else 2e-2)
+            if args.tp != "none":
+                res["parity"]["note"] = "rank 0's Y, the sublayer computed by all ranks together"
             res["cpu_baseline"] = cb
-        if world == 1 and args.workload in (None, HEADLINE) and not args.no_other_workloads:
+        if world == 1 and args.workload in (None, HEADLINE) and args.tp == "none" and not args.no_other_workloads:
             import torch
 
             from megatron_tensor_transformer_gelu_b200 import _lib as L

@@ -322,6 +322,54 @@ int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts,
                                  const void* X, int x_dtype, const float* gamma, const float* beta,
                                  float eps, void* Y, int out_dtype, void* stream);
 
+/* ------------------------------------ tensor parallelism across GPUs ----
+ * The multi-GPU form of the sublayers: each rank (GPU) holds its own weight
+ * shards, computes its partial sum of the row-split product, and the partial
+ * sums of all ranks are reduced before the residual add and the LayerNorm
+ * ([TYPC] §2.2 and §3; [PWWT] §3.3 RowParallelLinear's all_reduce, and §5.1:
+ * an AllReduce is a ReduceScatter followed by an AllGather, and the
+ * ReduceScatter's output can be used as it is, split by rows, which is what
+ * sequence parallelism does).  The exchange itself is either a collective
+ * library call made by the caller between these entry points, or the pointer
+ * lists of tp_reduce_residual_layernorm_multi below, which read other GPUs'
+ * partials and write other GPUs' outputs directly (peer access).
+ *
+ * tp_mlp_partial_forward: P = sum_{i < t} Act(X A_i) B_i over the t shards
+ *   this rank holds (F = the FFN width they cover; A_i [H, F/t], B_i [F/t, H]),
+ *   f32 [S, H], no residual and no LayerNorm.  dtype bf16 (tensor cores) or
+ *   f32 (CUDA cores).  workspace >= tp_mlp_partial_workspace_bytes(): the
+ *   [S, F] activation buffer.  Supported: H % 8 == 0, (F/t) % 8 == 0.
+ * tp_attn_partial_forward: P = sum_{s < t} O_s Wo_s for the nh heads this
+ *   rank holds (t shards of nh/t heads; X [S, H] with H the model's hidden
+ *   size, nh d <= H; Wqkv_shards[s] [H, 3 (nh/t) d] = [Q | K | V] columns of
+ *   shard s's heads; Wo_shards[s] [(nh/t) d, H]), f32 [S, H].  dtype bf16;
+ *   d == 128; nh % t == 0; S % 128 == 0; H % 8 == 0.  workspace >=
+ *   tp_attn_partial_workspace_bytes(): QKV [S, 3 nh d] and O [S, nh d] bf16.
+ * tp_reduce_residual_layernorm_multi: for `rows` rows,
+ *   Y = LN(X + sum_{q < nparts} parts[q]) (mean, biased variance, eps inside
+ *   the square root, gamma/beta [H] f32 or NULL), written to every one of the
+ *   nout outputs Y_outs[0..nout).  parts (nparts f32 buffers), X (x_dtype) and
+ *   each Y_outs[o] (out_dtype) are host arrays of device pointers to the first
+ *   of the `rows` rows, rows of H contiguous elements.  A pointer may address
+ *   another GPU's memory that this device can reach (peer access, CUDA IPC):
+ *   rank r then reduces its 1/N slice of the rows from every rank's partial
+ *   and stores the normalised rows into every rank's output, the
+ *   ReduceScatter -> LayerNorm on S/N rows -> AllGather of [PWWT] §5.1 in one
+ *   kernel.  The caller orders it after the partials are complete on every
+ *   rank and before the outputs are read.  0 <= nparts <= 8; 1 <= nout <= 8;
+ *   H % 8 == 0, 8 <= H <= 16384. */
+size_t tp_mlp_partial_workspace_bytes(int S, int H, int F, int t, int dtype);
+int tp_mlp_partial_forward(int S, int H, int F, int t, int dtype, const void* X, const void* const* A_shards,
+                           const void* const* B_shards, int act, float* P, void* workspace, size_t workspace_bytes,
+                           void* stream);
+size_t tp_attn_partial_workspace_bytes(int S, int H, int nh, int d, int t, int dtype);
+int tp_attn_partial_forward(int S, int H, int nh, int d, int t, int dtype, const void* X,
+                            const void* const* Wqkv_shards, const void* const* Wo_shards, float* P, void* workspace,
+                            size_t workspace_bytes, void* stream);
+int tp_reduce_residual_layernorm_multi(int rows, int H, int nparts, const float* const* parts, const void* X,
+                                       int x_dtype, const float* gamma, const float* beta, float eps, int nout,
+                                       void* const* Y_outs, int out_dtype, void* stream);
+
 /* -------------------------------------------------------- GEMM tiling ----
  * Tuning override for the tensor-core GEMMs (every sublayer and linear here).
  * tile_n == 0 (the default): a cost model picks, per launch, 256-column tiles

@@ -65,6 +65,12 @@ SIGNATURES = {
     "tp_attn_backward_workspace_bytes": (_c_size, [_c_int] * 6),
     "tp_attn_backward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vpp, _vp, _c_float, _vp, _c_size, _vp, _vp, _vpp, _vpp,
                                                   _vp, _vp, _vp, _c_size, _vp]),
+    "tp_mlp_partial_workspace_bytes": (_c_size, [_c_int] * 5),
+    "tp_mlp_partial_forward": (_c_int, [_c_int] * 5 + [_vp, _vpp, _vpp, _c_int, _vp, _vp, _c_size, _vp]),
+    "tp_attn_partial_workspace_bytes": (_c_size, [_c_int] * 6),
+    "tp_attn_partial_forward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vpp, _vp, _vp, _c_size, _vp]),
+    "tp_reduce_residual_layernorm_multi": (_c_int, [_c_int] * 3 + [_vpp, _vp, _c_int, _vp, _vp, _c_float, _c_int,
+                                                                   _vpp, _c_int, _vp]),
     "tp_set_gemm_tile_n": (_c_int, [_c_int]),
     "tp_gemm_plan": (_c_int, [_c_int] * 10 + [ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
     "tp_selftest_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
@@ -226,6 +232,62 @@ def reduce_residual_layernorm(parts, X, Y, gamma=None, beta=None, eps=1e-5, stre
     code = lib().tp_reduce_residual_layernorm(S, H, nparts, _ptr(parts), _ptr(X), DTYPE[X.dtype], _ptr(gamma),
                                               _ptr(beta), float(eps), _ptr(Y), DTYPE[Y.dtype], _stream(stream))
     _check(code, "tp_reduce_residual_layernorm")
+
+
+def _addr(x) -> int:
+    """Device address of a tensor, or an address given as an int (for example
+    another GPU's buffer opened through CUDA IPC)."""
+    return int(x) if isinstance(x, int) else x.data_ptr()
+
+
+def _addrs(xs):
+    arr = (ctypes.c_void_p * max(1, len(xs)))(*[_addr(x) for x in xs])
+    return ctypes.cast(arr, _vpp), arr
+
+
+def mlp_partial_workspace_bytes(S, H, F, t, dtype=torch.bfloat16) -> int:
+    return int(lib().tp_mlp_partial_workspace_bytes(S, H, F, t, DTYPE[dtype]))
+
+
+def mlp_partial_forward(X, A_shards, B_shards, P, workspace, act="gelu_tanh", stream=None):
+    """One rank's partial sum P = sum_i Act(X A_i) B_i (f32 [S, H]) over its shards."""
+    S, H = X.shape
+    t = len(A_shards)
+    F = sum(a.shape[1] for a in A_shards)
+    pa, ka = _ptrs(A_shards)
+    pb, kb = _ptrs(B_shards)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    code = lib().tp_mlp_partial_forward(S, H, F, t, DTYPE[X.dtype], _ptr(X), pa, pb, ACT[act], _ptr(P),
+                                        _ptr(workspace), ws_bytes, _stream(stream))
+    _check(code, "tp_mlp_partial_forward")
+
+
+def attn_partial_workspace_bytes(S, H, nh, d, t, dtype=torch.bfloat16) -> int:
+    return int(lib().tp_attn_partial_workspace_bytes(S, H, nh, d, t, DTYPE[dtype]))
+
+
+def attn_partial_forward(X, Wqkv_shards, Wo_shards, nh, d, P, workspace, stream=None):
+    """One rank's partial sum P = sum_s O_s Wo_s (f32 [S, H]) over the nh heads its shards hold."""
+    S, H = X.shape
+    t = len(Wqkv_shards)
+    pq, kq = _ptrs(Wqkv_shards)
+    po, ko = _ptrs(Wo_shards)
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    code = lib().tp_attn_partial_forward(S, H, nh, d, t, DTYPE[X.dtype], _ptr(X), pq, po, _ptr(P), _ptr(workspace),
+                                         ws_bytes, _stream(stream))
+    _check(code, "tp_attn_partial_forward")
+
+
+def reduce_residual_layernorm_multi(rows, H, parts, X, Y_outs, x_dtype, out_dtype, gamma=None, beta=None, eps=1e-5,
+                                    stream=None):
+    """Y = LN(X + sum of the partials) for `rows` rows, into every output.
+    parts, X, Y_outs: tensors or device addresses, each at the first of the rows."""
+    pp, kp = _addrs(parts)
+    py, ky = _addrs(Y_outs)
+    code = lib().tp_reduce_residual_layernorm_multi(int(rows), int(H), len(parts), pp, ctypes.c_void_p(_addr(X)),
+                                                    DTYPE[x_dtype], _ptr(gamma), _ptr(beta), float(eps),
+                                                    len(Y_outs), py, DTYPE[out_dtype], _stream(stream))
+    _check(code, "tp_reduce_residual_layernorm_multi")
 
 
 def mlp_train_state_bytes(S, H, F, t, dtype=torch.bfloat16) -> int:

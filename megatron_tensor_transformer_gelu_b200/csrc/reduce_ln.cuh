@@ -30,11 +30,15 @@ constexpr int MAX_H = MAX_WPR * 32 * MAX_CH * 8;  // 16384
 __host__ __device__ constexpr int cta_threads(int wpr) { return wpr > 8 ? wpr * 32 : THREADS; }
 }
 
+constexpr int RLN_MAX_PTRS = 8;  // partial sources / output copies given as pointer lists
+
 struct ReduceLnArgs {
   int S, H;
   int nparts;                 // number of f32 partial-sum buffers (0 = none)
-  const float* parts;         // nparts x [S, H], contiguous, part_stride elements apart
+  const float* parts;         // nparts x [S, H], contiguous, part_stride elements apart; or null:
   long long part_stride;
+  const float* part_ptr[RLN_MAX_PTRS];  // ... partial q at part_ptr[q] ([S, H] each; on this GPU or,
+                                        // through peer access, on another: the reduce-scatter's loads)
   const void* X;              // [S, H] residual, bf16 or f32
   int x_bf16;
   const float* gamma;         // [H] or null (= 1)
@@ -42,6 +46,8 @@ struct ReduceLnArgs {
   float eps;
   void* Y;                    // [S, H], bf16 or f32
   int y_bf16;
+  int ny_extra;               // further copies of Y written (the all-gather's stores), 0..RLN_MAX_PTRS-1
+  void* y_extra[RLN_MAX_PTRS];
   int apply_ln;               // 0: Y = X + sum_p P_p only (pre-LN residual stream)
 };
 
@@ -72,10 +78,21 @@ __device__ __forceinline__ void load8_f32_keep(const float* src, float* v) {
   v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
 }
 
-// 8 consecutive output values, bf16 (one 16-byte store) or f32 (two).
+// 8 consecutive output values, bf16 (one 16-byte store) or f32 (two), into Y
+// and into each extra copy.
+__device__ __forceinline__ void store8_to(void* Y, int y_bf16, long long off, const uint4& u, const float* y) {
+  if (y_bf16) {
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(Y) + off) = u;
+  } else {
+    float4* d = reinterpret_cast<float4*>(static_cast<float*>(Y) + off);
+    d[0] = make_float4(y[0], y[1], y[2], y[3]);
+    d[1] = make_float4(y[4], y[5], y[6], y[7]);
+  }
+}
+
 __device__ __forceinline__ void store8(const ReduceLnArgs& p, long long off, const float* y) {
+  uint4 u = make_uint4(0u, 0u, 0u, 0u);
   if (p.y_bf16) {
-    uint4 u;
     __nv_bfloat162 h0 = __floats2bfloat162_rn(y[0], y[1]);
     __nv_bfloat162 h1 = __floats2bfloat162_rn(y[2], y[3]);
     __nv_bfloat162 h2 = __floats2bfloat162_rn(y[4], y[5]);
@@ -84,12 +101,9 @@ __device__ __forceinline__ void store8(const ReduceLnArgs& p, long long off, con
     u.y = *reinterpret_cast<uint32_t*>(&h1);
     u.z = *reinterpret_cast<uint32_t*>(&h2);
     u.w = *reinterpret_cast<uint32_t*>(&h3);
-    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + off) = u;
-  } else {
-    float4* d = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + off);
-    d[0] = make_float4(y[0], y[1], y[2], y[3]);
-    d[1] = make_float4(y[4], y[5], y[6], y[7]);
   }
+  store8_to(p.Y, p.y_bf16, off, u, y);
+  for (int o = 0; o < p.ny_extra; ++o) store8_to(p.y_extra[o], p.y_bf16, off, u, y);
 }
 
 // One row is handled by WPR consecutive warps; a CTA holds max(1, 8 / WPR)
@@ -145,7 +159,8 @@ __global__ void __launch_bounds__(rln::cta_threads(WPR)) reduce_residual_ln_kern
           const int col = ((c * WPR + wr) * 32 + lane) * 8;
           if (live && col < p.H) {
             float w[8];
-            load8_f32(p.parts + q * p.part_stride + base + col, w);
+            const float* src = p.parts ? p.parts + q * p.part_stride : p.part_ptr[q];
+            load8_f32(src + base + col, w);
 #pragma unroll
             for (int e = 0; e < 8; ++e) v[c][e] += w[e];
           }

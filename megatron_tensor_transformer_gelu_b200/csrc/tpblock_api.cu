@@ -464,17 +464,29 @@ int run_gemm_simt(const float* A, long long lda, int M, const void* const* B, in
   return launch_status();
 }
 
+// Y = LN(X + sum of the partials) (or the residual add alone).  The partials
+// are `nparts` contiguous [S, H] slots starting at `parts`, or (parts == NULL)
+// the list part_list[0..nparts); `ny_extra` further outputs y_extra[] receive
+// the same values as Y.
 int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, int x_bf16, const float* gamma,
                   const float* beta, float eps, void* Y, int y_bf16, cudaStream_t st, int dev_sms,
-                  int apply_ln = 1) {
+                  int apply_ln = 1, const float* const* part_list = nullptr, int ny_extra = 0,
+                  void* const* y_extra = nullptr) {
   if (S == 0) return TP_OK;
   tp::ReduceLnArgs p;
+  std::memset(&p, 0, sizeof(p));
   p.apply_ln = apply_ln;
   p.S = S;
   p.H = H;
   p.nparts = nparts;
   p.parts = parts;
   p.part_stride = static_cast<long long>(S) * H;
+  if (!parts && part_list) {
+    for (int q = 0; q < nparts; ++q) p.part_ptr[q] = part_list[q];
+    if (nparts == 1) p.parts = part_list[0];  // the single-partial kernel reads `parts`
+  }
+  p.ny_extra = ny_extra;
+  for (int o = 0; o < ny_extra; ++o) p.y_extra[o] = y_extra[o];
   p.X = X;
   p.x_bf16 = x_bf16;
   p.gamma = gamma;
@@ -657,6 +669,32 @@ size_t tp_mlp_workspace_bytes(int S, int H, int F, int t, int dtype) {
 
 namespace {
 
+// The two products of the MLP sublayer on `in` ([S, H]): Hbuf = Act(in A_i) in
+// the column slices of an [S, F] buffer, then Zsum = sum_i Hbuf_i B_i (f32
+// [S, H]; the K loop may be cut into up to max_splits ranges, *nparts of them
+// used, one slot of S*H floats each).  Arguments are already checked.
+int mlp_products(const DeviceInfo& dev, int S, int H, int F, int t, int dtype, const void* in,
+                 const void* const* A_shards, const void* const* B_shards, int act, void* Hbuf, float* Zsum,
+                 int max_splits, int* nparts, cudaStream_t s, int kmaj) {
+  *nparts = 1;
+  if (S == 0) return TP_OK;
+  const int Fs = F / t;
+  int st;
+  if (dtype == TP_DTYPE_BF16) {
+    // H_i = Act(in A_i) into columns [i Fs, (i+1) Fs) of Hbuf [S, F] (bf16).
+    st = run_gemm_tc(dev, in, H, S, A_shards, t, /*row_mode=*/0, /*shard_k=*/H, /*shard_n=*/Fs, Hbuf, F,
+                     /*out_f32=*/0, act, s, 1, 0, nullptr, kmaj);
+    if (st != TP_OK) return st;
+    // Zsum = sum_i H_i B_i, accumulated in TMEM across the shards (f32).
+    return run_gemm_tc(dev, Hbuf, F, S, B_shards, t, /*row_mode=*/1, /*shard_k=*/Fs, /*shard_n=*/H, Zsum, H,
+                       /*out_f32=*/1, TP_ACT_NONE, s, max_splits, static_cast<long long>(S) * H, nparts, kmaj);
+  }
+  st = run_gemm_simt(static_cast<const float*>(in), H, S, A_shards, t, 0, H, Fs, static_cast<float*>(Hbuf), F, act,
+                     s, kmaj);
+  if (st != TP_OK) return st;
+  return run_gemm_simt(static_cast<const float*>(Hbuf), F, S, B_shards, t, 1, Fs, H, Zsum, H, TP_ACT_NONE, s, kmaj);
+}
+
 // MLP sublayer on `in` with residual `res`: Y = LN(res + sum_i Act(in A_i) B_i),
 // or Y = res + sum_i Act(in A_i) B_i without the LayerNorm (apply_ln = 0).
 // Arguments are already checked.
@@ -665,30 +703,14 @@ int mlp_core(const DeviceInfo& dev, int S, int H, int F, int t, int dtype, int o
              const float* beta, float eps, int act, int apply_ln, void* Y, void* workspace, cudaStream_t s,
              int kmaj = 0) {
   if (S == 0) return TP_OK;
-  const int Fs = F / t;
-  int nparts = 1;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t eh = dtype == TP_DTYPE_BF16 ? 2 : 4;
   void* Hbuf = ws;
   float* Zsum = reinterpret_cast<float*>(ws + align256(static_cast<size_t>(S) * F * eh));
-  int st;
-  if (dtype == TP_DTYPE_BF16) {
-    // H_i = Act(in A_i) into columns [i Fs, (i+1) Fs) of Hbuf [S, F] (bf16).
-    st = run_gemm_tc(dev, in, H, S, A_shards, t, /*row_mode=*/0, /*shard_k=*/H, /*shard_n=*/Fs, Hbuf, F,
-                     /*out_f32=*/0, act, s, 1, 0, nullptr, kmaj);
-    if (st != TP_OK) return st;
-    // Zsum = sum_i H_i B_i, accumulated in TMEM across the shards (f32); the K
-    // loop may be cut into `nparts` ranges (partial-sum slots) to fill the GPU.
-    st = run_gemm_tc(dev, Hbuf, F, S, B_shards, t, /*row_mode=*/1, /*shard_k=*/Fs, /*shard_n=*/H, Zsum, H,
-                     /*out_f32=*/1, TP_ACT_NONE, s, TP_MAX_K_SPLITS, static_cast<long long>(S) * H, &nparts, kmaj);
-    if (st != TP_OK) return st;
-  } else {
-    st = run_gemm_simt(static_cast<const float*>(in), H, S, A_shards, t, 0, H, Fs, static_cast<float*>(Hbuf), F,
-                       act, s, kmaj);
-    if (st != TP_OK) return st;
-    st = run_gemm_simt(static_cast<const float*>(Hbuf), F, S, B_shards, t, 1, Fs, H, Zsum, H, TP_ACT_NONE, s, kmaj);
-    if (st != TP_OK) return st;
-  }
+  int nparts = 1;
+  int st = mlp_products(dev, S, H, F, t, dtype, in, A_shards, B_shards, act, Hbuf, Zsum,
+                        dtype == TP_DTYPE_BF16 ? TP_MAX_K_SPLITS : 1, &nparts, s, kmaj);
+  if (st != TP_OK) return st;
   return run_reduce_ln(S, H, nparts, Zsum, res, dtype == TP_DTYPE_BF16, gamma, beta, eps, Y,
                        out_dtype == TP_DTYPE_BF16, s, dev.sm_count, apply_ln);
 }
@@ -705,19 +727,19 @@ struct AttnKeep {
   float* lse2 = nullptr;
 };
 
-int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out_dtype, const void* in,
-              const void* res, const void* const* Wqkv_shards, const void* const* Wo_shards, const float* gamma,
-              const float* beta, float eps, int apply_ln, void* Y, void* workspace, cudaStream_t s,
-              int kmaj = 0, const AttnKeep* keep = nullptr) {
+// QKV, per-head attention and the row-split O projection of the nh heads held
+// by t shards (nh / t each) of a model of hidden size H: QKV [S, 3 nh d] and O
+// [S, nh d] bf16 in the given buffers, Zsum = sum_s O_s Wo_s (f32 [S, H]; up to
+// max_splits K-split slots, *nparts used).  Arguments are already checked.
+int attn_products(const DeviceInfo& dev, int S, int H, int nh, int d, int t, const void* in,
+                  const void* const* Wqkv_shards, const void* const* Wo_shards, void* QKV, void* Obuf, float* Zsum,
+                  int max_splits, int* nparts, cudaStream_t s, int kmaj, float* lse2) {
+  *nparts = 1;
   if (S == 0) return TP_OK;
-  const int Hs = H / t;  // columns of one shard's heads
-  uint8_t* ws = static_cast<uint8_t*>(workspace);
-  void* QKV = keep ? keep->qkv : ws;                                         // [S, 3H] bf16
-  void* Obuf = keep ? keep->o : ws + align256(static_cast<size_t>(S) * 3 * H * 2);   // [S, H] bf16
-  float* Zsum = keep ? keep->zsum
-                     : reinterpret_cast<float*>(static_cast<uint8_t*>(Obuf) + align256(static_cast<size_t>(S) * H * 2));
+  const int Hl = nh * d;    // columns of the heads held here
+  const int Hs = Hl / t;    // columns of one shard's heads
   // [Q_s | K_s | V_s] = in Wqkv_s into columns [3 s Hs, 3 (s+1) Hs) of QKV.
-  int st = run_gemm_tc(dev, in, H, S, Wqkv_shards, t, 0, H, 3 * Hs, QKV, 3LL * H, 0, TP_ACT_NONE, s, 1, 0, nullptr,
+  int st = run_gemm_tc(dev, in, H, S, Wqkv_shards, t, 0, H, 3 * Hs, QKV, 3LL * Hl, 0, TP_ACT_NONE, s, 1, 0, nullptr,
                        kmaj);
   if (st != TP_OK) return st;
   // O_h = softmax(Q_h K_h^T / sqrt d) V_h, written to columns [h d, (h+1) d) of O.
@@ -725,16 +747,16 @@ int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out
     tp::AttnArgs a;
     std::memset(&a, 0, sizeof(a));
     const int nhs = nh / t;
-    // Q/K/V boxes: 64 columns (128 B) x 128 rows of the [S, 3H] buffer.
-    if (!tmap_bf16(&a.tmQKV, QKV, S, 3LL * H, 3LL * H, 64, tp::attn::BQ)) return TP_ERR_CUDA;
+    // Q/K/V boxes: 64 columns (128 B) x 128 rows of the [S, 3 Hl] buffer.
+    if (!tmap_bf16(&a.tmQKV, QKV, S, 3LL * Hl, 3LL * Hl, 64, tp::attn::BQ)) return TP_ERR_CUDA;
     a.O = Obuf;
     a.S = S;
-    a.H = H;
+    a.H = Hl;
     a.nh = nh;
     a.heads_per_shard = nhs;
     a.shard_cols = 3 * Hs;
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
-    a.lse2 = keep ? keep->lse2 : nullptr;
+    a.lse2 = lse2;
     dim3 grid((S + tp::attn::TILES * tp::attn::BQ - 1) / (tp::attn::TILES * tp::attn::BQ), nh);
     ProfScope ps(K_ATTN, s);
     st = launch_pdl(tp::attn_fwd_kernel, grid, dim3(tp::attn::NUM_THREADS), tp::attn::SMEM_BYTES, s, a) != cudaSuccess
@@ -743,9 +765,23 @@ int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out
     if (st != TP_OK) return st;
   }
   // sum_s O_s Wo_s, the O projection row-split by head, summed in TMEM.
+  return run_gemm_tc(dev, Obuf, Hl, S, Wo_shards, t, 1, Hs, H, Zsum, H, 1, TP_ACT_NONE, s, max_splits,
+                     static_cast<long long>(S) * H, nparts, kmaj);
+}
+
+int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out_dtype, const void* in,
+              const void* res, const void* const* Wqkv_shards, const void* const* Wo_shards, const float* gamma,
+              const float* beta, float eps, int apply_ln, void* Y, void* workspace, cudaStream_t s,
+              int kmaj = 0, const AttnKeep* keep = nullptr) {
+  if (S == 0) return TP_OK;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* QKV = keep ? keep->qkv : ws;                                         // [S, 3H] bf16
+  void* Obuf = keep ? keep->o : ws + align256(static_cast<size_t>(S) * 3 * H * 2);   // [S, H] bf16
+  float* Zsum = keep ? keep->zsum
+                     : reinterpret_cast<float*>(static_cast<uint8_t*>(Obuf) + align256(static_cast<size_t>(S) * H * 2));
   int nparts = 1;
-  st = run_gemm_tc(dev, Obuf, H, S, Wo_shards, t, 1, Hs, H, Zsum, H, 1, TP_ACT_NONE, s, keep ? 1 : TP_MAX_K_SPLITS,
-                   static_cast<long long>(S) * H, &nparts, kmaj);
+  int st = attn_products(dev, S, H, nh, d, t, in, Wqkv_shards, Wo_shards, QKV, Obuf, Zsum,
+                         keep ? 1 : TP_MAX_K_SPLITS, &nparts, s, kmaj, keep ? keep->lse2 : nullptr);
   if (st != TP_OK) return st;
   return run_reduce_ln(S, H, nparts, Zsum, res, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s, dev.sm_count,
                        apply_ln);
@@ -1409,6 +1445,86 @@ int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts, c
 }
 
 // ------------------------------------------------------------- GEMM tiling
+int tp_reduce_residual_layernorm_multi(int rows, int H, int nparts, const float* const* parts, const void* X,
+                                       int x_dtype, const float* gamma, const float* beta, float eps, int nout,
+                                       void* const* Y_outs, int out_dtype, void* stream) {
+  if (rows < 0 || nparts < 0 || nparts > TP_MAX_SHARDS || nout < 1 || nout > TP_MAX_SHARDS ||
+      !valid_dtype(x_dtype) || !valid_dtype(out_dtype) || !(eps > 0.0f) || !std::isfinite(eps))
+    return TP_ERR_INVALID_ARG;
+  if ((nparts > 0 && !parts) || !Y_outs || !opt_ptr_ok(gamma) || !opt_ptr_ok(beta) || !opt_ptr_ok(X))
+    return TP_ERR_INVALID_ARG;
+  if (rows > 0) {
+    if (!ptr_ok(X)) return TP_ERR_INVALID_ARG;
+    for (int q = 0; q < nparts; ++q)
+      if (!ptr_ok(parts[q])) return TP_ERR_INVALID_ARG;
+    for (int o = 0; o < nout; ++o)
+      if (!ptr_ok(Y_outs[o])) return TP_ERR_INVALID_ARG;
+  }
+  if (!hidden_ok(H)) return TP_ERR_UNSUPPORTED_SHAPE;
+  DeviceInfo* dev = nullptr;
+  int st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  if (rows == 0) return TP_OK;
+  return run_reduce_ln(rows, H, nparts, nullptr, X, x_dtype == TP_DTYPE_BF16, gamma, beta, eps, Y_outs[0],
+                       out_dtype == TP_DTYPE_BF16, static_cast<cudaStream_t>(stream), dev->sm_count, 1, parts,
+                       nout - 1, Y_outs + 1);
+}
+
+// ------------------------------------------------- one rank's partial sum
+size_t tp_mlp_partial_workspace_bytes(int S, int H, int F, int t, int dtype) {
+  if (S < 0 || H <= 0 || F <= 0 || t < 1 || !valid_dtype(dtype)) return 0;
+  const size_t eh = dtype == TP_DTYPE_BF16 ? 2 : 4;
+  return align256(static_cast<size_t>(S) * F * eh);
+}
+
+int tp_mlp_partial_forward(int S, int H, int F, int t, int dtype, const void* X, const void* const* A_shards,
+                           const void* const* B_shards, int act, float* P, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  if (t < 1 || t > TP_MAX_SHARDS || S < 0 || H <= 0 || F <= 0 || !valid_dtype(dtype) || !valid_act(act))
+    return TP_ERR_INVALID_ARG;
+  if ((S > 0 && (!ptr_ok(X) || !ptr_ok(P))) || !opt_ptr_ok(X) || !opt_ptr_ok(P) || !shards_ok(A_shards, t) ||
+      !shards_ok(B_shards, t) || !opt_ptr_ok(workspace))
+    return TP_ERR_INVALID_ARG;
+  if (F % t != 0 || (F / t) % 8 != 0 || H % 8 != 0) return TP_ERR_UNSUPPORTED_SHAPE;
+  const size_t need = tp_mlp_partial_workspace_bytes(S, H, F, t, dtype);
+  if (workspace_bytes < need || (need > 0 && !workspace)) return TP_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  int st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  int nparts = 1;
+  return mlp_products(*dev, S, H, F, t, dtype, X, A_shards, B_shards, act, workspace, P, 1, &nparts,
+                      static_cast<cudaStream_t>(stream), 0);
+}
+
+size_t tp_attn_partial_workspace_bytes(int S, int H, int nh, int d, int t, int dtype) {
+  if (S < 0 || H <= 0 || nh <= 0 || d <= 0 || t < 1 || dtype != TP_DTYPE_BF16) return 0;
+  const size_t s = static_cast<size_t>(S), hl = static_cast<size_t>(nh) * d;
+  return align256(s * 3 * hl * 2) + align256(s * hl * 2);
+}
+
+int tp_attn_partial_forward(int S, int H, int nh, int d, int t, int dtype, const void* X,
+                            const void* const* Wqkv_shards, const void* const* Wo_shards, float* P, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (t < 1 || t > TP_MAX_SHARDS || S < 0 || H <= 0 || nh <= 0 || d <= 0 || dtype != TP_DTYPE_BF16)
+    return TP_ERR_INVALID_ARG;
+  if ((S > 0 && (!ptr_ok(X) || !ptr_ok(P))) || !opt_ptr_ok(X) || !opt_ptr_ok(P) || !shards_ok(Wqkv_shards, t) ||
+      !shards_ok(Wo_shards, t) || !opt_ptr_ok(workspace))
+    return TP_ERR_INVALID_ARG;
+  if (d != tp::attn::D || nh % t != 0 || static_cast<long long>(nh) * d > H || H % 8 != 0 ||
+      S % tp::attn::BQ != 0)
+    return TP_ERR_UNSUPPORTED_SHAPE;
+  const size_t need = tp_attn_partial_workspace_bytes(S, H, nh, d, t, dtype);
+  if (workspace_bytes < need || (need > 0 && !workspace)) return TP_ERR_WORKSPACE_TOO_SMALL;
+  DeviceInfo* dev = nullptr;
+  int st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t hl = static_cast<size_t>(nh) * d;
+  int nparts = 1;
+  return attn_products(*dev, S, H, nh, d, t, X, Wqkv_shards, Wo_shards, ws, ws + align256(static_cast<size_t>(S) * 3 * hl * 2),
+                       P, 1, &nparts, static_cast<cudaStream_t>(stream), 0, nullptr);
+}
+
 int tp_set_gemm_tile_n(int tile_n) {
   if (tile_n != 0 && tile_n != 128 && (tile_n < 256 || tile_n > 512 || tile_n % 32 != 0))
     return TP_ERR_INVALID_ARG;

@@ -440,8 +440,14 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
   return r;
 }
 
+// f32 CUDA-core GEMM (same shard modes as run_gemm_tc).  With max_splits > 1
+// (row mode, no activation) the K range may be cut over up to max_splits
+// CTAs per tile, split z writing slot z at C + z * slot_stride; *splits_out
+// tells the caller how many slots to add.
 int run_gemm_simt(const float* A, long long lda, int M, const void* const* B, int t, int row_mode, int shard_k,
-                  int shard_n, float* C, long long ldc, int act, cudaStream_t st, int b_kmajor = 0) {
+                  int shard_n, float* C, long long ldc, int act, cudaStream_t st, int b_kmajor = 0, int dev_sms = 148,
+                  int max_splits = 1, long long slot_stride = 0, int* splits_out = nullptr) {
+  if (splits_out) *splits_out = 1;
   if (M == 0) return TP_OK;
   tp::SimtArgs p;
   std::memset(&p, 0, sizeof(p));
@@ -450,6 +456,7 @@ int run_gemm_simt(const float* A, long long lda, int M, const void* const* B, in
   for (int s = 0; s < t; ++s) p.B[s] = static_cast<const float*>(B[s]);
   p.C = C;
   p.ldc = ldc;
+  p.slot_stride = slot_stride;
   p.M = M;
   p.row_mode = row_mode;
   p.shard_n = shard_n;
@@ -458,7 +465,17 @@ int run_gemm_simt(const float* A, long long lda, int M, const void* const* B, in
   p.K = row_mode ? shard_k * t : shard_k;
   p.act = act;
   p.b_kmajor = b_kmajor;
-  dim3 grid(ceil_div(p.N, tp::simt::TN), ceil_div(M, tp::simt::TM));
+  // Enough CTAs for two per SM where the K range allows it (each split keeps
+  // at least two K chunks).
+  const long long tiles = static_cast<long long>(ceil_div(p.N, tp::simt::TN)) * ceil_div(M, tp::simt::TM);
+  const int chunks = ceil_div(p.K, tp::simt::TK);
+  int splits = 1;
+  if (act == TP_ACT_NONE && max_splits > 1) {
+    while (splits < max_splits && tiles * splits < 2LL * dev_sms && chunks / (splits + 1) >= 2) ++splits;
+  }
+  p.splits = splits;
+  if (splits_out) *splits_out = splits;
+  dim3 grid(ceil_div(p.N, tp::simt::TN), ceil_div(M, tp::simt::TM), splits);
   ProfScope ps(K_GEMM_SIMT, st);
   tp::simt_gemm_f32_kernel<<<grid, tp::simt::THREADS, 0, st>>>(p);
   return launch_status();
@@ -661,8 +678,7 @@ size_t tp_mlp_workspace_bytes(int S, int H, int F, int t, int dtype) {
   if (S < 0 || H <= 0 || F <= 0 || t < 1 || !valid_dtype(dtype)) return 0;
   (void)t;
   const size_t eh = dtype == TP_DTYPE_BF16 ? 2 : 4;
-  const size_t slots = dtype == TP_DTYPE_BF16 ? TP_MAX_K_SPLITS : 1;
-  return align256(static_cast<size_t>(S) * F * eh) + slots * static_cast<size_t>(S) * H * 4;
+  return align256(static_cast<size_t>(S) * F * eh) + TP_MAX_K_SPLITS * static_cast<size_t>(S) * H * 4;
 }
 
 }  // extern "C"
@@ -690,9 +706,10 @@ int mlp_products(const DeviceInfo& dev, int S, int H, int F, int t, int dtype, c
                        /*out_f32=*/1, TP_ACT_NONE, s, max_splits, static_cast<long long>(S) * H, nparts, kmaj);
   }
   st = run_gemm_simt(static_cast<const float*>(in), H, S, A_shards, t, 0, H, Fs, static_cast<float*>(Hbuf), F, act,
-                     s, kmaj);
+                     s, kmaj, dev.sm_count);
   if (st != TP_OK) return st;
-  return run_gemm_simt(static_cast<const float*>(Hbuf), F, S, B_shards, t, 1, Fs, H, Zsum, H, TP_ACT_NONE, s, kmaj);
+  return run_gemm_simt(static_cast<const float*>(Hbuf), F, S, B_shards, t, 1, Fs, H, Zsum, H, TP_ACT_NONE, s, kmaj,
+                       dev.sm_count, max_splits, static_cast<long long>(S) * H, nparts);
 }
 
 // MLP sublayer on `in` with residual `res`: Y = LN(res + sum_i Act(in A_i) B_i),
@@ -708,8 +725,8 @@ int mlp_core(const DeviceInfo& dev, int S, int H, int F, int t, int dtype, int o
   void* Hbuf = ws;
   float* Zsum = reinterpret_cast<float*>(ws + align256(static_cast<size_t>(S) * F * eh));
   int nparts = 1;
-  int st = mlp_products(dev, S, H, F, t, dtype, in, A_shards, B_shards, act, Hbuf, Zsum,
-                        dtype == TP_DTYPE_BF16 ? TP_MAX_K_SPLITS : 1, &nparts, s, kmaj);
+  int st = mlp_products(dev, S, H, F, t, dtype, in, A_shards, B_shards, act, Hbuf, Zsum, TP_MAX_K_SPLITS, &nparts, s,
+                        kmaj);
   if (st != TP_OK) return st;
   return run_reduce_ln(S, H, nparts, Zsum, res, dtype == TP_DTYPE_BF16, gamma, beta, eps, Y,
                        out_dtype == TP_DTYPE_BF16, s, dev.sm_count, apply_ln);

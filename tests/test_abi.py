@@ -68,7 +68,7 @@ def test_version_and_status_strings(lib):
 def test_workspace_sizes(lib):
     S, H, F = 2048, 4096, 16384
     assert lib.tp_mlp_workspace_bytes(S, H, F, 4, 1) == S * F * 2 + 4 * S * H * 4
-    assert lib.tp_mlp_workspace_bytes(S, H, F, 4, 0) == S * F * 4 + S * H * 4
+    assert lib.tp_mlp_workspace_bytes(S, H, F, 4, 0) == S * F * 4 + 4 * S * H * 4
     assert lib.tp_mlp_workspace_bytes(-1, H, F, 4, 1) == 0
     assert lib.tp_attn_workspace_bytes(2048, 8192, 64, 128, 4, 1) == 2048 * 8192 * (6 + 2 + 16)
     assert lib.tp_attn_workspace_bytes(2048, 8192, 64, 128, 4, 0) == 0

@@ -126,3 +126,40 @@ def test_attention_training_writes_stay_in_bounds(cuda_device, tile_n):
                       ("dbeta", db)] + [(f"dWqkv{i}", w) for i, w in enumerate(dWq)] + \
             [(f"dWo{i}", w) for i, w in enumerate(dWo)]:
         assert buf.intact(), name
+
+
+@pytest.mark.parametrize("S,H,F,t", [(77, 136, 312, 3), (128, 256, 1024, 2), (33, 40, 1040, 2)])
+def test_mlp_f32_writes_stay_in_bounds(cuda_device, S, H, F, t):
+    """The f32 CUDA-core path: ragged 32 x 32 tiles, and the row-split GEMM's
+    K range cut over several f32 slots."""
+    inp = synth.gen_mlp(S, H, F, seed=S + 1, dtype=torch.float32)
+    X = inp.X.cuda()
+    Y = Guarded((S, H), torch.float32)
+    ws = Guarded((L.mlp_workspace_bytes(S, H, F, t, torch.float32),), torch.uint8)
+    L.mlp_forward(X, _cuda(synth.split_columns(inp.A, t)), _cuda(synth.split_rows(inp.B, t)), Y.t, ws.t)
+    torch.cuda.synchronize()
+    assert Y.intact() and ws.intact()
+
+
+def test_tp_partials_and_multi_output_reduce_stay_in_bounds(cuda_device):
+    """Per-rank partial sums and the reduce + LayerNorm over pointer lists
+    (row slices written into every output copy)."""
+    S, H, F, N = 200, 264, 1200, 3
+    inp = synth.gen_mlp(S, H, F, seed=9)
+    X = inp.X.cuda()
+    A, B = _cuda(synth.split_columns(inp.A, N)), _cuda(synth.split_rows(inp.B, N))
+    parts, wss = [], []
+    for r in range(N):
+        P = Guarded((S, H), torch.float32)
+        ws = Guarded((L.mlp_partial_workspace_bytes(S, H, F // N, 1),), torch.uint8)
+        L.mlp_partial_forward(X, A[r:r + 1], B[r:r + 1], P.t, ws.t)
+        parts.append(P)
+        wss.append(ws)
+    Ys = [Guarded((S, H), torch.bfloat16) for _ in range(N)]
+    S_ = S - S % N
+    for r in range(N):
+        r0, n = r * (S_ // N), S_ // N
+        L.reduce_residual_layernorm_multi(n, H, [p.t[r0:] for p in parts], X[r0:], [y.t[r0:] for y in Ys],
+                                          torch.bfloat16, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert all(b.intact() for b in parts + wss + Ys)

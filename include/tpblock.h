@@ -400,6 +400,30 @@ int tp_set_gemm_tile_n(int tile_n);
 int tp_gemm_plan(int M, int t, int row_mode, int shard_k, int shard_n, int out_f32, int b_kmajor,
                  int heavy_epilogue, int slots, int max_splits, int* tile_n, int* splits);
 
+/* Stream-K scheduling of the tensor-core GEMMs.  Where a sublayer has
+ * scratch to spare for it (the partial-sum slots past the first of the MLP
+ * and attention workspaces) and the epilogue is the plain one, a GEMM may cut
+ * the k-blocks of all its tiles, laid end to end, into one contiguous range
+ * per CTA pair instead of dealing whole tiles out in waves, so that no pair
+ * idles in a partly filled last wave.  A tile cut between pairs is summed by
+ * the pair holding its last k-block, after a bounded wait for the others' f32
+ * partials (TP_ERR_TIMEOUT through tp_device_error() if it gives up); the
+ * partials are added in a fixed order, so results are run-to-run repeatable.
+ * mode 0 (the default): the tile cost model chooses, per launch, between
+ * whole-tile waves and stream-K; 1: every GEMM that has the scratch uses
+ * stream-K (over as many pairs as the scratch holds partial blocks for); -1:
+ * never.  Process-wide, not thread-safe against concurrent launches.  Returns
+ * TP_ERR_INVALID_ARG for other values. */
+int tp_set_gemm_stream_k(int mode);
+
+/* tp_gemm_plan with the stream-K option: sk_area_bytes of scratch available
+ * to the launch (0: none).  Also writes *stream_k (1 if the launch would use
+ * stream-K) and *sk_clusters (the CTA pairs, or single CTAs, it would run
+ * on); either may be NULL. */
+int tp_gemm_plan_sk(int M, int t, int row_mode, int shard_k, int shard_n, int out_f32, int b_kmajor,
+                    int heavy_epilogue, int slots, int max_splits, size_t sk_area_bytes, int* tile_n, int* splits,
+                    int* stream_k, int* sk_clusters);
+
 /* ------------------------------------------------------------ self-test ----
  * Diagnostic for the bounded-wait path every kernel here takes when one of its
  * device-side waits gives up: launches one CTA whose mbarrier wait nothing can
@@ -408,6 +432,18 @@ int tp_gemm_plan(int M, int t, int row_mode, int shard_k, int shard_n, int out_f
  * tp_device_error() returns TP_ERR_TIMEOUT (and clears the word); the context
  * stays usable.  Returns TP_ERR_INVALID_ARG for limit_cycles < 1. */
 int tp_selftest_wait_timeout(long long limit_cycles, void* stream);
+/* The same for the other kind of bounded wait the kernels make: one thread
+ * waits for a flag in global memory that nothing sets (what a stream-K GEMM's
+ * finishing CTA pair does for the pairs whose partial sums it adds), so the
+ * wait ends after `limit_cycles` SM cycles and raises the device error word;
+ * tp_device_error() then returns TP_ERR_TIMEOUT and clears it. */
+int tp_selftest_flag_wait_timeout(long long limit_cycles, void* stream);
+
+/* Diagnostic for the attention kernel's exponentials: part of the softmax's
+ * 2^x terms are evaluated on the FMA pipe by a polynomial instead of the MUFU
+ * unit.  Writes, for the n f32 inputs x (device), that evaluation into y_poly
+ * and CUDA's exp2f(x) into y_exp2f (device, n each). */
+int tp_selftest_exp2(const float* x, float* y_poly, float* y_exp2f, int n, void* stream);
 
 /* ----------------------------------------------------- kernel timing ----
  * When enabled, every kernel the library launches is counted, and the first

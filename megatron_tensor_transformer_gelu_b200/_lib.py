@@ -73,7 +73,11 @@ SIGNATURES = {
                                                                    _vpp, _c_int, _vp]),
     "tp_set_gemm_tile_n": (_c_int, [_c_int]),
     "tp_gemm_plan": (_c_int, [_c_int] * 10 + [ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
+    "tp_set_gemm_stream_k": (_c_int, [_c_int]),
+    "tp_gemm_plan_sk": (_c_int, [_c_int] * 10 + [_c_size] + [ctypes.POINTER(_c_int)] * 4),
     "tp_selftest_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
+    "tp_selftest_flag_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
+    "tp_selftest_exp2": (_c_int, [_vp, _vp, _vp, _c_int, _vp]),
     "tp_profile_enable": (_c_int, [_c_int]),
     "tp_profile_sample": (_c_int, [_c_int]),
     "tp_profile_collect": (_c_int, [ctypes.POINTER(_c_int), ctypes.POINTER(_c_int), ctypes.POINTER(ctypes.c_double),
@@ -378,8 +382,38 @@ def gemm_plan(M, t, row_mode, shard_k, shard_n, out_f32, b_kmajor=False, heavy_e
     return tn.value, sp.value
 
 
+def set_gemm_stream_k(mode: int) -> None:
+    """0: the cost model decides per GEMM launch; 1: stream-K wherever a
+    launch has scratch for it; -1: never."""
+    _check(lib().tp_set_gemm_stream_k(int(mode)), "tp_set_gemm_stream_k")
+
+
+def gemm_plan_sk(M, t, row_mode, shard_k, shard_n, out_f32, b_kmajor=False, heavy_epilogue=False, slots=74,
+                 max_splits=1, sk_area_bytes=0):
+    """(tile_n, splits, stream_k, sk_clusters) of the next GEMM launch of this
+    shape with sk_area_bytes of stream-K scratch (host logic only)."""
+    out = [ctypes.c_int(0) for _ in range(4)]
+    _check(lib().tp_gemm_plan_sk(int(M), int(t), int(bool(row_mode)), int(shard_k), int(shard_n),
+                                 int(bool(out_f32)), int(bool(b_kmajor)), int(bool(heavy_epilogue)), int(slots),
+                                 int(max_splits), int(sk_area_bytes), *[ctypes.byref(o) for o in out]),
+           "tp_gemm_plan_sk")
+    return tuple(o.value for o in out)
+
+
 def selftest_wait_timeout(limit_cycles: int, stream=None):
     _check(lib().tp_selftest_wait_timeout(int(limit_cycles), _stream(stream)), "tp_selftest_wait_timeout")
+
+
+def selftest_flag_wait_timeout(limit_cycles: int, stream=None):
+    _check(lib().tp_selftest_flag_wait_timeout(int(limit_cycles), _stream(stream)), "tp_selftest_flag_wait_timeout")
+
+
+def selftest_exp2(x, stream=None):
+    """(the attention kernel's polynomial 2^x, CUDA's exp2f(x)) for a device f32 tensor x."""
+    yp = torch.empty_like(x)
+    yr = torch.empty_like(x)
+    _check(lib().tp_selftest_exp2(_ptr(x), _ptr(yp), _ptr(yr), x.numel(), _stream(stream)), "tp_selftest_exp2")
+    return yp, yr
 
 
 def device_error() -> int:

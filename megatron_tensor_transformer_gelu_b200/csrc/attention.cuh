@@ -49,6 +49,10 @@ constexpr uint32_t IDESC_QK = idesc_bf16_f32(BQ, BKV, false, false);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(BQ, D, false, true);
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;
+#ifndef TP_ATTN_EXP2_POLY_EVERY
+#define TP_ATTN_EXP2_POLY_EVERY 4
+#endif
+constexpr int EXP2_POLY_EVERY = TP_ATTN_EXP2_POLY_EVERY;  // 0: every exponential on the MUFU unit
 }  // namespace attn
 
 struct AttnArgs {
@@ -268,12 +272,17 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
       }
       // p = 2^(s * scale_log2 - m) in f32, kept as bf16 pairs for the P V
       // product; the row sum adds the f32 values in 8 independent chains.
+      // One pair in EXP2_POLY_EVERY is evaluated on the FMA pipe (exp2_poly)
+      // instead of the MUFU unit, whose exponentials bound this loop.
       float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       uint32_t pk0[32], pk1[32];
 #pragma unroll
       for (int e = 0; e < BKV; e += 2) {
-        const float p0 = exp2_fast(fmaf(s[e], a.scale_log2, -m_run));
-        const float p1 = exp2_fast(fmaf(s[e + 1], a.scale_log2, -m_run));
+        const bool poly = EXP2_POLY_EVERY > 0 && (e / 2) % EXP2_POLY_EVERY == EXP2_POLY_EVERY - 1;
+        const float x0 = fmaf(s[e], a.scale_log2, -m_run);
+        const float x1 = fmaf(s[e + 1], a.scale_log2, -m_run);
+        const float p0 = poly ? exp2_poly(x0) : exp2_fast(x0);
+        const float p1 = poly ? exp2_poly(x1) : exp2_fast(x1);
         sum8[(e / 2) & 7] += p0 + p1;
         if (e < 64) pk0[e / 2] = pack_bf16x2(p0, p1);
         else pk1[(e - 64) / 2] = pack_bf16x2(p0, p1);

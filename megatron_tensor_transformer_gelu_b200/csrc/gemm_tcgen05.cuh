@@ -43,6 +43,20 @@
 //
 // Column mode can give each shard its own A (a_per_shard): t independent
 // products A_s B_s in one persistent launch (the attention backward's heads).
+//
+// Stream-K (sk = 1): instead of whole tiles dealt round-robin to the clusters
+// (the last wave partly idle when the tile count is not a multiple of the
+// cluster count), the k-blocks of all tiles, laid end to end, are cut into
+// one contiguous range per cluster.  A tile whose k-blocks are cut between
+// clusters is summed by the cluster holding its last k-block (the finisher):
+// each other cluster (a producer) stores its f32 partial accumulator to a
+// workspace and publishes a flag; the finisher waits for those flags (bounded
+// wait), adds the partials into its TMEM accumulator and runs the normal
+// epilogue.  Every cluster processes its producer piece first and its
+// finisher piece last, and a finisher waits only on lower-numbered clusters'
+// producer pieces, so no wait can form a cycle; the grid is never larger than
+// the clusters resident at once.  The partials are added in a fixed order, so
+// results are run-to-run repeatable.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -153,9 +167,73 @@ struct GemmArgs {
   const float* rowvec;
   long long rowvec_ld;
   float epi_scale;
+  // Stream-K (see the top of this file).  sk_ws holds, per cluster c and CTA
+  // rank r, a 128 x tile_n f32 block at ((c CG + r) 128 tile_n) (the partial a
+  // producer piece leaves, float4 chunk j of row l at (j 128 + l)); sk_flags
+  // [clusters x CG] hold the epoch of the last partial each one published.
+  int sk;
+  float* sk_ws;
+  unsigned long long* sk_flags;
+  unsigned long long sk_epoch;
 };
 
 enum : int { EPI_PLAIN = 0, EPI_AUX_PRE = 1, EPI_GRAD = 2, EPI_SOFTMAX = 3, EPI_DSOFTMAX = 4 };
+
+// One piece of work of a cluster: the k-blocks [kb0, kb1) of a tile (of K
+// split `split` in the K-split mode), and what its epilogue does with them.
+enum : int { ROLE_FULL = 0, ROLE_PRODUCER = 1, ROLE_FINISHER = 2 };
+struct WorkItem {
+  int tile, split, kb0, kb1, role;
+};
+
+// Stream-K: cluster c's range of the k-blocks of all tiles laid end to end.
+__device__ __forceinline__ void sk_range(const GemmArgs& p, int c, int nclusters, long long& k0, long long& k1) {
+  const long long total = static_cast<long long>(p.m_blocks) * p.n_blocks * p.k_blocks;
+  k0 = total * c / nclusters;
+  k1 = total * (c + 1) / nclusters;
+}
+
+__device__ __forceinline__ int num_work_items(const GemmArgs& p, int c, int nclusters) {
+  if (!p.sk) {
+    const int units = p.m_blocks * p.n_blocks * p.splits;
+    return c < units ? (units - 1 - c) / nclusters + 1 : 0;
+  }
+  long long k0, k1;
+  sk_range(p, c, nclusters, k0, k1);
+  if (k1 <= k0) return 0;
+  return static_cast<int>((k1 - 1) / p.k_blocks - k0 / p.k_blocks + 1);
+}
+
+__device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& kb0, int& kb1);
+
+// The idx-th of cluster c's n work items, in processing order.  Stream-K
+// order: the range's last piece (a producer when it ends inside a tile)
+// first, the whole tiles between, the first piece (a finisher when it starts
+// inside a tile) last.
+__device__ __forceinline__ WorkItem work_item(const GemmArgs& p, int c, int nclusters, int idx, int n) {
+  WorkItem w;
+  if (!p.sk) {
+    const int num_tiles = p.m_blocks * p.n_blocks;
+    const int unit = c + idx * nclusters;
+    w.tile = unit % num_tiles;
+    w.split = unit / num_tiles;
+    split_range(p, w.split, w.kb0, w.kb1);
+    w.role = ROLE_FULL;
+    return w;
+  }
+  long long k0, k1;
+  sk_range(p, c, nclusters, k0, k1);
+  const int seg = n == 1 ? 0 : (idx == 0 ? n - 1 : (idx == n - 1 ? 0 : idx));
+  const long long kbt = p.k_blocks;
+  const long long ti = k0 / kbt + seg;
+  const long long ts = ti * kbt;
+  w.tile = static_cast<int>(ti);
+  w.split = 0;
+  w.kb0 = static_cast<int>((k0 > ts ? k0 : ts) - ts);
+  w.kb1 = static_cast<int>((k1 < ts + kbt ? k1 : ts + kbt) - ts);
+  w.role = w.kb1 < kbt ? ROLE_PRODUCER : (w.kb0 > 0 ? ROLE_FINISHER : ROLE_FULL);
+  return w;
+}
 
 __device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& kb0, int& kb1) {
   kb0 = static_cast<int>(static_cast<long long>(split) * p.k_blocks / p.splits);
@@ -498,11 +576,10 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
   griddep_wait();
   griddep_launch_dependents();
 
-  const int num_tiles = p.m_blocks * p.n_blocks;
   const bool narrow = narrow_tiles<WIDE>(p);
-  const int num_units = num_tiles * p.splits;
   const int cluster_id = blockIdx.x / CG;
   const int num_clusters = gridDim.x / CG;
+  const int num_items = num_work_items(p, cluster_id, num_clusters);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -513,11 +590,10 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       int armed[STAGES];  // parity of the last phase this thread armed per stage (leader)
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) armed[s] = -1;
-      for (int unit = cluster_id; unit < num_units && ok; unit += num_clusters) {
-        const int tile = unit % num_tiles;
-        int kb_begin, kb_end;
-        split_range(p, unit / num_tiles, kb_begin, kb_end);
-        const TileCoord tc = tile_coord<CG>(p, tile);
+      for (int idx = 0; idx < num_items && ok; ++idx) {
+        const WorkItem wi = work_item(p, cluster_id, num_clusters, idx, num_items);
+        const int kb_begin = wi.kb0, kb_end = wi.kb1;
+        const TileCoord tc = tile_coord<CG>(p, wi.tile);
         const CUtensorMap* mA = &p.tmA[p.a_per_shard ? tc.shard : 0];
         const int my_row0 = tc.m0 + static_cast<int>(rank) * C::BM;
         const bool my_a = my_row0 < p.M;
@@ -610,14 +686,14 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int unit = cluster_id; unit < num_units && ok; unit += num_clusters) {
-        int kb_begin, kb_end;
-        split_range(p, unit / num_tiles, kb_begin, kb_end);
+      for (int idx = 0; idx < num_items && ok; ++idx) {
+        const WorkItem wi = work_item(p, cluster_id, num_clusters, idx, num_items);
+        const int kb_begin = wi.kb0, kb_end = wi.kb1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * C::BN);
         // Wide tiles: the second MMA only where the tile has columns past BN.
-        const bool two = WIDE && tile_coord<CG>(p, unit % num_tiles).n_valid > C::BN;
+        const bool two = WIDE && tile_coord<CG>(p, wi.tile).n_valid > C::BN;
         for (int kb = kb_begin; kb < kb_end; ++kb) {
           if (!mbar_wait(&full[stage], phase)) { ok = false; break; }
           tc_fence_after();
@@ -680,9 +756,10 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
     uint32_t acc_phase = 0;
     int buf = 0;
     const uint32_t tempty_leader0 = CG == 2 ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
-    for (int unit = cluster_id; unit < num_units; unit += num_clusters) {
-      const TileCoord tc = tile_coord<CG>(p, unit % num_tiles);
-      const int split = unit / num_tiles;
+    for (int idx = 0; idx < num_items; ++idx) {
+      const WorkItem wi = work_item(p, cluster_id, num_clusters, idx, num_items);
+      const TileCoord tc = tile_coord<CG>(p, wi.tile);
+      const int split = wi.split;
       const int y0 = tc.m0 + static_cast<int>(rank) * C::BM;
       const int mshard = p.m_split_rows ? tc.m0 / p.m_split_rows : 0;
       const int ystore = y0 - mshard * p.m_split_rows;
@@ -693,6 +770,75 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       if (!named_barrier_and(1, 128, mbar_wait(&tfull[acc], acc_phase))) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
+      if (wi.role == ROLE_PRODUCER) {
+        // Stream-K producer piece: the raw f32 accumulator goes to this CTA's
+        // block of the workspace (coalesced: float4 chunk j of row l at
+        // j * 128 + l), then the TMEM buffer is handed back and the flag
+        // published once every thread's stores are visible.
+        float4* dst = reinterpret_cast<float4*>(p.sk_ws + static_cast<long long>(cluster_id * CG + rank) * C::BM *
+                                                              p.tile_n) + row_local;
+        for (int c32 = 0; c32 < p.tile_n / 32; ++c32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + c32 * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            __stcg(dst + static_cast<long long>(c32 * 8 + j) * C::BM,
+                   make_float4(__uint_as_float(r[4 * j]), __uint_as_float(r[4 * j + 1]),
+                               __uint_as_float(r[4 * j + 2]), __uint_as_float(r[4 * j + 3])));
+        }
+        tc_fence_before();
+        if constexpr (CG == 1) {
+          mbar_arrive(&tempty[acc]);
+        } else {
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tempty_leader0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+        }
+        __threadfence();
+        named_barrier_sync(1, 128);
+        if (elected) flag_publish(p.sk_flags + cluster_id * CG + rank, p.sk_epoch);
+        if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
+        continue;
+      }
+      if (wi.role == ROLE_FINISHER) {
+        // Stream-K finisher piece: wait for every producer of this tile (the
+        // lower-numbered clusters whose ranges reach into it), then add their
+        // partials into the TMEM accumulator, highest cluster first.
+        const long long tile_k0 = static_cast<long long>(wi.tile) * p.k_blocks;
+        if (elected) {
+          for (int pc = cluster_id - 1; pc >= 0; --pc) {
+            long long q0, q1;
+            sk_range(p, pc, num_clusters, q0, q1);
+            if (q1 <= tile_k0) break;
+            if (q1 <= q0) continue;  // an empty range publishes nothing
+            if (!flag_wait_eq(p.sk_flags + pc * CG + rank, p.sk_epoch)) break;
+          }
+        }
+        named_barrier_sync(1, 128);
+        for (int c32 = 0; c32 < p.tile_n / 32; ++c32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(t_row + c32 * 32, r);
+          tmem_wait_ld();
+          for (int pc = cluster_id - 1; pc >= 0; --pc) {
+            long long q0, q1;
+            sk_range(p, pc, num_clusters, q0, q1);
+            if (q1 <= tile_k0) break;
+            if (q1 <= q0) continue;
+            const float4* src = reinterpret_cast<const float4*>(p.sk_ws + static_cast<long long>(pc * CG + rank) *
+                                                                              C::BM * p.tile_n) + row_local;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const float4 a = __ldcg(src + static_cast<long long>(c32 * 8 + j) * C::BM);
+              r[4 * j] = __float_as_uint(__uint_as_float(r[4 * j]) + a.x);
+              r[4 * j + 1] = __float_as_uint(__uint_as_float(r[4 * j + 1]) + a.y);
+              r[4 * j + 2] = __float_as_uint(__uint_as_float(r[4 * j + 2]) + a.z);
+              r[4 * j + 3] = __float_as_uint(__uint_as_float(r[4 * j + 3]) + a.w);
+            }
+          }
+          tmem_st_32x32b_x32(t_row + c32 * 32, r);
+        }
+        tmem_wait_st();
+      }
       const int nchunks = (tc.n_valid + cw - 1) / cw;
       const int parts = p.epi_mode == EPI_AUX_PRE ? 2 : 1;  // aux (pre-activation) store first
       const int grow = y0 + row_local;

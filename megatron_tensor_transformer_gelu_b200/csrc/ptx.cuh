@@ -80,6 +80,39 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
   }
 }
 
+// ------------------------------------------------- flags in global memory
+// Publish `v` after this thread's earlier global writes (release, GPU scope).
+__device__ __forceinline__ void flag_publish(unsigned long long* addr, unsigned long long v) {
+  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(addr), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long flag_read(const unsigned long long* addr) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(addr) : "memory");
+  return v;
+}
+
+// Wait until *addr == v (acquire).  Returns false (and raises the device
+// error word) if that did not happen within `limit` SM cycles, or if another
+// wait already raised it.
+__device__ __forceinline__ bool flag_wait_eq(const unsigned long long* addr, unsigned long long v,
+                                             long long limit = WAIT_LIMIT_CYCLES) {
+  if (flag_read(addr) == v) return true;
+  const long long t0 = clock64();
+  uint32_t n = 0;
+  while (true) {
+    __nanosleep(64);
+    if (flag_read(addr) == v) return true;
+    if ((++n & 63u) == 0u) {
+      if (error_raised()) return false;
+      if (clock64() - t0 > limit) {
+        flag_error(DEV_ERR_TIMEOUT);
+        return false;
+      }
+    }
+  }
+}
+
 // Diagnostic: one thread waits on an mbarrier that nothing completes, so the
 // bounded wait above gives up after `limit` cycles and raises the error word.
 __global__ void selftest_wait_timeout_kernel(long long limit) {
@@ -91,7 +124,25 @@ __global__ void selftest_wait_timeout_kernel(long long limit) {
   }
 }
 
+// Diagnostic: one thread waits for a global flag that nothing sets (the wait
+// a stream-K finisher makes for its producers), so the bounded wait gives up
+// after `limit` cycles and raises the error word.
+__device__ unsigned long long g_tp_selftest_flag = 0;
+
+__global__ void selftest_flag_wait_kernel(long long limit) {
+  if (threadIdx.x == 0) (void)flag_wait_eq(&g_tp_selftest_flag, 1ull, limit);
+}
+
 // ----------------------------------------------------------------------- TMA
+// Untiled bulk copy global -> this CTA's shared memory, completing `bytes` on
+// the mbarrier.  Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load_1d(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
@@ -330,6 +381,36 @@ __device__ __forceinline__ float exp2_fast(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe instead of the MUFU unit, for the share of a softmax's
+// exponentials that would otherwise queue behind the MUFU: x = n + f with
+// n = round(x) (adding 1.5 * 2^23 leaves round(x) in the low mantissa bits)
+// and f in [-1/2, 1/2]; 2^f from a degree-4 polynomial whose coefficients were
+// fitted for minimax relative error on [-1/2, 1/2] by the Remez exchange
+// (max relative error 2.6e-6, 2.7e-6 evaluated in f32); 2^n goes into the
+// exponent field with an integer add.  x is clamped at -125 (smaller values
+// give 2^-125, not 0: nothing a sum of softmax terms can see).  For x <= 64.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -125.0f);
+  const float magic = 12582912.0f;  // 1.5 * 2^23
+  const float t = x + magic;
+  const float f = x - (t - magic);
+  float p = 0.009570102f;
+  p = fmaf(p, f, 0.055917859f);
+  p = fmaf(p, f, 0.24024744f);
+  p = fmaf(p, f, 0.69312179f);
+  p = fmaf(p, f, 0.99999928f);
+  const int n = __float_as_int(t) - __float_as_int(magic);
+  return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
+// Diagnostic: exp2_poly and CUDA's exp2f side by side on n inputs.
+__global__ void selftest_exp2_kernel(const float* x, float* y_poly, float* y_ref, int n) {
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
+    y_poly[i] = exp2_poly(x[i]);
+    y_ref[i] = exp2f(x[i]);
+  }
 }
 
 // Shared-memory matrix descriptor (sm_100 format): start address, leading and

@@ -244,4 +244,178 @@ __global__ void __launch_bounds__(rln::cta_threads(WPR)) reduce_residual_ln_kern
   }
 }
 
+// ------------------------------------------------ rows staged by bulk copies
+// The same operation with each row's inputs (X and the f32 partials) brought
+// into shared memory by untiled bulk copies (cp.async.bulk) instead of loaded
+// by the threads: one thread issues a row's copies `nst` rows ahead of the
+// row the CTA is reducing, so several rows per CTA are in flight from HBM
+// while the CTA runs a row's two reductions, and the threads hold only their
+// own 8-element chunks in registers.  One CTA of 256 threads walks rows
+// blockIdx.x, blockIdx.x + gridDim.x, ...; thread i's chunk c covers columns
+// (c * 256 + i) * 8 .. + 7.  The statistics are the two-pass ones of the
+// register kernel (mean, then the variance of the centred values; warp
+// shuffles, then the warps' sums in warp order), so results are repeatable.
+// Stage layout: [X row][partial 0 row][partial 1 row]..., each a multiple of
+// 16 bytes (H % 8 == 0).
+namespace rlb {
+constexpr int THREADS = 256;
+constexpr int WARPS = THREADS / 32;
+constexpr int MAX_STAGE_SMEM = 200 * 1024;  // stages x stage bytes of one CTA
+}
+
+__device__ __forceinline__ void rlb_issue_row(const ReduceLnArgs& p, long long row, uint8_t* dst, uint64_t* bar,
+                                              uint32_t xbytes, uint32_t pbytes) {
+  mbar_arrive_expect_tx(bar, xbytes + static_cast<uint32_t>(p.nparts) * pbytes);
+  const uint8_t* xsrc = static_cast<const uint8_t*>(p.X) + row * xbytes;
+  bulk_load_1d(dst, xsrc, xbytes, bar);
+  for (int q = 0; q < p.nparts; ++q) {
+    const float* src = p.parts ? p.parts + q * p.part_stride : p.part_ptr[q];
+    bulk_load_1d(dst + xbytes + q * pbytes, src + row * p.H, pbytes, bar);
+  }
+}
+
+template <int CH>
+__global__ void __launch_bounds__(rlb::THREADS) reduce_residual_ln_bulk_kernel(const ReduceLnArgs p, int nst,
+                                                                              int stage_bytes) {
+  extern __shared__ __align__(128) uint8_t rlb_smem[];
+  __shared__ uint64_t full[4];
+  __shared__ float red[2][2][rlb::WARPS];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t xbytes = static_cast<uint32_t>(p.H) * (p.x_bf16 ? 2u : 4u);
+  const uint32_t pbytes = static_cast<uint32_t>(p.H) * 4u;
+  if (tid == 0) {
+    for (int s = 0; s < nst; ++s) mbar_init(&full[s], 1);
+    mbar_fence_init();
+  }
+  __syncthreads();
+  griddep_wait();  // the partial sums come from the preceding kernel
+  griddep_launch_dependents();
+  const int n_my = blockIdx.x < p.S ? (p.S - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x) + 1 : 0;
+  int issued = 0;  // rows whose copies thread 0 has issued
+  if (tid == 0) {
+    for (; issued < nst && issued < n_my; ++issued)
+      rlb_issue_row(p, blockIdx.x + static_cast<long long>(issued) * gridDim.x, rlb_smem + issued * stage_bytes,
+                    &full[issued], xbytes, pbytes);
+  }
+  const float inv_h = 1.0f / static_cast<float>(p.H);
+  int i = 0;
+  for (; i < n_my; ++i) {
+    const int s = i % nst;
+    const long long row = blockIdx.x + static_cast<long long>(i) * gridDim.x;
+    const uint8_t* st = rlb_smem + s * stage_bytes;
+    // Every thread waits for the row's copies; all take the same exit.
+    const bool ok = mbar_wait(&full[s], static_cast<uint32_t>((i / nst) & 1));
+    if (!__syncthreads_and(ok)) break;
+    float v[CH][8];
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = (c * rlb::THREADS + tid) * 8;
+      if (col < p.H) {
+        if (p.x_bf16) {
+          load8_bf16(reinterpret_cast<const __nv_bfloat16*>(st) + col, v[c]);
+        } else {
+          const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(st) + col);
+          const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(st) + col + 4);
+          v[c][0] = a.x; v[c][1] = a.y; v[c][2] = a.z; v[c][3] = a.w;
+          v[c][4] = b.x; v[c][5] = b.y; v[c][6] = b.z; v[c][7] = b.w;
+        }
+        for (int q = 0; q < p.nparts; ++q) {
+          const float* pr = reinterpret_cast<const float*>(st + xbytes + q * pbytes) + col;
+          const float4 a = *reinterpret_cast<const float4*>(pr);
+          const float4 b = *reinterpret_cast<const float4*>(pr + 4);
+          v[c][0] += a.x; v[c][1] += a.y; v[c][2] += a.z; v[c][3] += a.w;
+          v[c][4] += b.x; v[c][5] += b.y; v[c][6] += b.z; v[c][7] += b.w;
+        }
+      }
+    }
+    if (!p.apply_ln) {
+      __syncthreads();  // every thread has its values: the stage may be refilled
+      if (tid == 0 && i + nst < n_my) {
+        fence_proxy_async_smem();
+        rlb_issue_row(p, row + static_cast<long long>(nst) * gridDim.x, rlb_smem + s * stage_bytes, &full[s], xbytes,
+                      pbytes);
+        ++issued;
+      }
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int col = (c * rlb::THREADS + tid) * 8;
+        if (col < p.H) store8(p, row * p.H + col, v[c]);
+      }
+      continue;
+    }
+    float sum = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      if ((c * rlb::THREADS + tid) * 8 < p.H) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sum += v[c][e];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) red[i & 1][0][warp] = sum;
+    __syncthreads();
+    // Every thread has read the stage: refill it with the row nst rows ahead.
+    if (tid == 0 && i + nst < n_my) {
+      fence_proxy_async_smem();
+      rlb_issue_row(p, row + static_cast<long long>(nst) * gridDim.x, rlb_smem + s * stage_bytes, &full[s], xbytes,
+                    pbytes);
+      ++issued;
+    }
+    float tot = 0.0f;
+#pragma unroll
+    for (int w = 0; w < rlb::WARPS; ++w) tot += red[i & 1][0][w];
+    const float mean = tot * inv_h;
+    float s2 = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      if ((c * rlb::THREADS + tid) * 8 < p.H) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float d = v[c][e] - mean;
+          s2 = fmaf(d, d, s2);
+        }
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    if (lane == 0) red[i & 1][1][warp] = s2;
+    __syncthreads();
+    float tot2 = 0.0f;
+#pragma unroll
+    for (int w = 0; w < rlb::WARPS; ++w) tot2 += red[i & 1][1][w];
+    const float rstd = 1.0f / sqrtf(tot2 * inv_h + p.eps);
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = (c * rlb::THREADS + tid) * 8;
+      if (col < p.H) {
+        float gm[8], bt[8];
+        if (p.gamma) load8_f32_keep(p.gamma + col, gm);
+        else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) gm[e] = 1.0f;
+        }
+        if (p.beta) load8_f32_keep(p.beta + col, bt);
+        else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) bt[e] = 0.0f;
+        }
+        float y[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = fmaf((v[c][e] - mean) * rstd, gm[e], bt[e]);
+        store8(p, row * p.H + col, y);
+      }
+    }
+  }
+  // After an error exit, rows issued but not consumed may still have copies in
+  // flight: let them land (bounded) before the CTA's shared memory is released.
+  if (tid == 0) {
+    for (int j = i; j < issued; ++j) {
+      const uint32_t a = smem_u32(&full[j % nst]);
+      const long long t0 = clock64();
+      while (!mbar_try_wait(a, static_cast<uint32_t>((j / nst) & 1)) && clock64() - t0 < WAIT_LIMIT_CYCLES) {}
+    }
+  }
+}
+
 }  // namespace tp

@@ -10,6 +10,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <chrono>
 #include <mutex>
 #include <utility>
 
@@ -36,6 +37,12 @@ struct DeviceInfo {
   int max_pairs = 0;  // co-resident CTA pairs of the cta_group::2 GEMM
 };
 
+// The reduce + residual + LayerNorm stages rows in shared memory with bulk
+// copies (1) or loads them into registers (0).
+#ifndef TP_RLN_BULK
+#define TP_RLN_BULK 1
+#endif
+
 // Most K-split partial-sum slots a row-split GEMM feeding the LayerNorm may use.
 #define TP_MAX_K_SPLITS 4
 
@@ -48,6 +55,8 @@ struct DeviceInfo {
 std::mutex g_mu;
 DeviceInfo g_dev[MAX_DEVICES];
 int g_force_tile_n = 0;  // tp_set_gemm_tile_n: 0 = cost model
+int g_stream_k = 0;      // tp_set_gemm_stream_k: 0 = cost model, 1 = wherever a workspace allows, -1 = never
+unsigned long long g_sk_epoch = 0;  // last stream-K launch's epoch (see next_sk_epoch)
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 // ------------------------------------------------------------ event timing
@@ -220,7 +229,30 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 struct TilePlan {
   int tile_n = 256;
   int splits = 1;
+  int stream_k = 0;   // 1: stream-K over `sk_clusters` clusters
+  int sk_clusters = 0;
 };
+
+// Workspace a stream-K launch needs: a 128 x w f32 partial block per CTA of
+// each of `clusters` clusters of cg CTAs, then one 8-byte flag per CTA.
+size_t sk_bytes(long long clusters, int cg, int w) {
+  return align256(static_cast<size_t>(clusters) * cg * 128 * w * 4) + static_cast<size_t>(clusters) * cg * 8;
+}
+
+// Flags of stream-K launches carry the launch's epoch, so a flag left by an
+// earlier launch never matches.  The epochs start from a process-specific
+// salt in the high half, so stale workspace contents from another process
+// are not mistaken for this one's either.
+unsigned long long next_sk_epoch() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_sk_epoch == 0) {
+    const unsigned long long salt =
+        (static_cast<unsigned long long>(reinterpret_cast<uintptr_t>(&g_sk_epoch)) >> 4) ^
+        static_cast<unsigned long long>(std::chrono::steady_clock::now().time_since_epoch().count());
+    g_sk_epoch = (salt | 1ull) << 32;
+  }
+  return ++g_sk_epoch;
+}
 
 constexpr double T_KB = 0.40e-6;
 constexpr double T_EPI_256 = 3.5e-6;
@@ -241,7 +273,9 @@ long long n_blocks_for(const tp::GemmArgs& p, int w) {
   return p.row_mode ? per_shard : per_shard * p.t;
 }
 
-TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits) {
+// The data-parallel plan: whole tiles dealt round-robin to the clusters,
+// optionally with the K loop split into f32 slots.
+TilePlan plan_tiles_dp(const tp::GemmArgs& p, bool pair, int slots, int max_splits, double* cost) {
   TilePlan best;
   const long long m_blocks = (p.M + (pair ? 255 : 127)) / (pair ? 256 : 128);
   const long long out_elems = static_cast<long long>(p.M) * (p.row_mode ? p.shard_n : p.shard_n * p.t);
@@ -258,6 +292,7 @@ TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits)
     }
   }
   const int step = p.out_f32 ? 32 : 64;  // a 128-byte output chunk must not cross a tile edge
+  *cost = best_t;
   if (g_force_tile_n) {
     best.splits = 1;
     if (g_force_tile_n == 128) {  // narrow tiles, single CTAs included
@@ -288,6 +323,63 @@ TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits)
       best.splits = 1;
     }
   }
+  *cost = best_t;
+  return best;
+}
+
+// Stream-K: one contiguous range of (tile, k-block) steps per cluster, so the
+// time is the steps per cluster rather than whole waves, plus the exposed
+// epilogue of every piece but the last with wide tiles, plus the fixed cost
+// of the split tiles' partials (a producer's store, its finisher's wait and
+// reads: about 3 us).
+constexpr double T_SK_FIX = 3.0e-6;
+
+double sk_cost(const tp::GemmArgs& p, bool pair, int clusters, int w) {
+  const long long m_blocks = (p.M + (pair ? 255 : 127)) / (pair ? 256 : 128);
+  const long long tiles = m_blocks * n_blocks_for(p, w);
+  const long long steps = (tiles * p.k_blocks + clusters - 1) / clusters;
+  const double epi_weight = p.epi_mode == tp::EPI_PLAIN ? 1.0 : 2.0;
+  const long long exposed = w > 256 ? (tiles + clusters - 1) / clusters : 0;
+  return static_cast<double>(steps) * kb_cost(w) * T_KB + T_SK_FIX +
+         static_cast<double>(exposed) * (w / 256.0) * T_EPI_256 * epi_weight;
+}
+
+// The tile plan: the data-parallel one, or stream-K where the caller gives a
+// workspace of `sk_area` bytes for the partials (0: none), the epilogue is the
+// plain one, and it is at least 2 % faster by the cost model.
+TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits, size_t sk_area = 0) {
+  double best_t = 0.0;
+  TilePlan best = plan_tiles_dp(p, pair, slots, max_splits, &best_t);
+  if (g_stream_k < 0 || sk_area == 0 || p.epi_mode != tp::EPI_PLAIN) return best;
+  const int cg = pair ? 2 : 1;
+  const int step = p.out_f32 ? 32 : 64;
+  const long long m_blocks = (p.M + (pair ? 255 : 127)) / (pair ? 256 : 128);
+  if (g_stream_k > 0) {
+    // Forced (tests): the data-parallel plan's width (or the forced width),
+    // over as many clusters as the workspace holds partial blocks for.
+    long long clusters = slots;
+    while (clusters >= 2 && sk_bytes(clusters, cg, best.tile_n) > sk_area) --clusters;
+    const long long steps = m_blocks * n_blocks_for(p, best.tile_n) * p.k_blocks;
+    if (clusters >= 2 && steps >= clusters) {
+      best.stream_k = 1;
+      best.sk_clusters = static_cast<int>(clusters);
+      best.splits = 1;
+    }
+    return best;
+  }
+  if (g_force_tile_n || best.tile_n == 128) return best;  // a forced width, or narrow shards: as planned
+  for (int w = 256; w <= (pair ? 512 : 256); w += step) {
+    if (sk_bytes(slots, cg, w) > sk_area) continue;
+    if (m_blocks * n_blocks_for(p, w) * p.k_blocks < 4LL * slots) continue;  // too little work to split
+    const double t = sk_cost(p, pair, slots, w);
+    if (t < best_t * 0.98) {
+      best_t = t;
+      best.tile_n = w;
+      best.splits = 1;
+      best.stream_k = 1;
+      best.sk_clusters = slots;
+    }
+  }
   return best;
 }
 
@@ -309,6 +401,8 @@ struct GemmExtra {
   const float* rowvec = nullptr;     // EPI_SOFTMAX / EPI_DSOFTMAX: row values r, shard s at
   long long rowvec_ld = 0;           //   rowvec + s * rowvec_ld
   float epi_scale = 1.0f;
+  void* sk_ws = nullptr;             // scratch the launch may use for stream-K partials and flags
+  size_t sk_ws_bytes = 0;            //   (256-byte aligned; 0: no stream-K)
 };
 
 template <int CG, bool WIDE>
@@ -344,7 +438,16 @@ int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, const TilePlan& plan,
     }
   }
   const long long units = tiles * p.splits;
-  const int clusters = static_cast<int>(units < slots ? units : slots);
+  int clusters = static_cast<int>(units < slots ? units : slots);
+  if (plan.stream_k) {
+    clusters = plan.sk_clusters;
+    p.sk = 1;
+    p.splits = 1;
+    p.sk_ws = static_cast<float*>(ex.sk_ws);
+    p.sk_flags = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(ex.sk_ws) +
+                                                       align256(static_cast<size_t>(clusters) * CG * 128 * p.tile_n * 4));
+    p.sk_epoch = next_sk_epoch();
+  }
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see griddep_wait in the kernel
@@ -431,7 +534,8 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
   p.slot_stride = slot_stride;
   p.b_kmajor = b_kmajor;
   if (!out_f32) max_splits = 1;
-  const TilePlan plan = plan_tiles(p, pair, pair ? dev.max_pairs : dev.sm_count, max_splits);
+  const TilePlan plan = plan_tiles(p, pair, pair ? dev.max_pairs : dev.sm_count, max_splits,
+                                   (ex.sk_ws && ex.m_split == 0) ? ex.sk_ws_bytes : 0);
   int r;
   if (!pair) r = launch_gemm_tc<1, false>(dev, p, plan, ex, st);
   else if (plan.tile_n > tp::GemmCfg<2>::BN) r = launch_gemm_tc<2, true>(dev, p, plan, ex, st);
@@ -512,9 +616,49 @@ int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, i
   p.Y = Y;
   p.y_bf16 = y_bf16;
   bool launched = true;
+  ProfScope ps(K_REDUCE_LN, st);
+#if TP_RLN_BULK
+  // Rows staged in shared memory by bulk copies, `nst` rows ahead per CTA:
+  // stages of up to 48 KiB are sized for two CTAs per SM (4 stages at most),
+  // larger ones for one; rows too wide for two stages take the register
+  // kernel below.
+  {
+    const size_t xb = x_bf16 ? 2 : 4;
+    const size_t stage = ((static_cast<size_t>(H) * (xb + 4 * nparts)) + 127) & ~size_t(127);
+    if (2 * stage <= static_cast<size_t>(tp::rlb::MAX_STAGE_SMEM)) {
+      const size_t budget = stage <= 48 * 1024 ? 96 * 1024 : tp::rlb::MAX_STAGE_SMEM;
+      int nst = static_cast<int>(budget / stage);
+      nst = nst < 2 ? 2 : (nst > 4 ? 4 : nst);
+      const size_t smem = static_cast<size_t>(nst) * stage;
+      auto go_bulk = [&](auto kern) {
+        int per_sm = 1;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+                cudaSuccess ||
+            cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, tp::rlb::THREADS, smem) != cudaSuccess ||
+            per_sm < 1)
+          per_sm = 1;
+        const int grid = S < per_sm * dev_sms ? S : per_sm * dev_sms;
+        if (launch_pdl(kern, dim3(grid), dim3(tp::rlb::THREADS), smem, st, p, nst, static_cast<int>(stage)) !=
+            cudaSuccess)
+          launched = false;
+      };
+      const int ch = (H + 2047) / 2048;
+      using namespace tp;
+      switch (ch) {
+        case 1: go_bulk(reduce_residual_ln_bulk_kernel<1>); break;
+        case 2: go_bulk(reduce_residual_ln_bulk_kernel<2>); break;
+        case 3: go_bulk(reduce_residual_ln_bulk_kernel<3>); break;
+        case 4: go_bulk(reduce_residual_ln_bulk_kernel<4>); break;
+        case 5: case 6: go_bulk(reduce_residual_ln_bulk_kernel<6>); break;
+        default: go_bulk(reduce_residual_ln_bulk_kernel<8>); break;
+      }
+      const int ls = launch_status();
+      return launched ? ls : TP_ERR_CUDA;
+    }
+  }
+#endif
   // WPR warps per row (each lane holds CH chunks of 8 values); max(1, 8 / WPR)
   // rows per CTA; a grid of the resident CTA count walks the row groups.
-  ProfScope ps(K_REDUCE_LN, st);
   const bool np1 = nparts == 1;
   auto go = [&](auto kern, int wpr, int rows_per_cta) {
     const int threads = tp::rln::cta_threads(wpr);
@@ -691,19 +835,23 @@ namespace {
 // used, one slot of S*H floats each).  Arguments are already checked.
 int mlp_products(const DeviceInfo& dev, int S, int H, int F, int t, int dtype, const void* in,
                  const void* const* A_shards, const void* const* B_shards, int act, void* Hbuf, float* Zsum,
-                 int max_splits, int* nparts, cudaStream_t s, int kmaj) {
+                 int max_splits, int* nparts, cudaStream_t s, int kmaj, void* sk_ws = nullptr,
+                 size_t sk_bytes = 0) {
   *nparts = 1;
   if (S == 0) return TP_OK;
   const int Fs = F / t;
   int st;
   if (dtype == TP_DTYPE_BF16) {
+    GemmExtra ex;  // scratch for stream-K partials (its plan never also splits K into slots)
+    ex.sk_ws = sk_ws;
+    ex.sk_ws_bytes = sk_bytes;
     // H_i = Act(in A_i) into columns [i Fs, (i+1) Fs) of Hbuf [S, F] (bf16).
     st = run_gemm_tc(dev, in, H, S, A_shards, t, /*row_mode=*/0, /*shard_k=*/H, /*shard_n=*/Fs, Hbuf, F,
-                     /*out_f32=*/0, act, s, 1, 0, nullptr, kmaj);
+                     /*out_f32=*/0, act, s, 1, 0, nullptr, kmaj, &ex);
     if (st != TP_OK) return st;
     // Zsum = sum_i H_i B_i, accumulated in TMEM across the shards (f32).
     return run_gemm_tc(dev, Hbuf, F, S, B_shards, t, /*row_mode=*/1, /*shard_k=*/Fs, /*shard_n=*/H, Zsum, H,
-                       /*out_f32=*/1, TP_ACT_NONE, s, max_splits, static_cast<long long>(S) * H, nparts, kmaj);
+                       /*out_f32=*/1, TP_ACT_NONE, s, max_splits, static_cast<long long>(S) * H, nparts, kmaj, &ex);
   }
   st = run_gemm_simt(static_cast<const float*>(in), H, S, A_shards, t, 0, H, Fs, static_cast<float*>(Hbuf), F, act,
                      s, kmaj, dev.sm_count);
@@ -725,8 +873,11 @@ int mlp_core(const DeviceInfo& dev, int S, int H, int F, int t, int dtype, int o
   void* Hbuf = ws;
   float* Zsum = reinterpret_cast<float*>(ws + align256(static_cast<size_t>(S) * F * eh));
   int nparts = 1;
+  // Slots 1.. of the partial-sum area double as stream-K scratch: a stream-K
+  // plan writes slot 0 only.
+  const size_t sh4 = static_cast<size_t>(S) * H * 4;
   int st = mlp_products(dev, S, H, F, t, dtype, in, A_shards, B_shards, act, Hbuf, Zsum, TP_MAX_K_SPLITS, &nparts, s,
-                        kmaj);
+                        kmaj, reinterpret_cast<uint8_t*>(Zsum) + sh4, (TP_MAX_K_SPLITS - 1) * sh4);
   if (st != TP_OK) return st;
   return run_reduce_ln(S, H, nparts, Zsum, res, dtype == TP_DTYPE_BF16, gamma, beta, eps, Y,
                        out_dtype == TP_DTYPE_BF16, s, dev.sm_count, apply_ln);
@@ -750,14 +901,18 @@ struct AttnKeep {
 // max_splits K-split slots, *nparts used).  Arguments are already checked.
 int attn_products(const DeviceInfo& dev, int S, int H, int nh, int d, int t, const void* in,
                   const void* const* Wqkv_shards, const void* const* Wo_shards, void* QKV, void* Obuf, float* Zsum,
-                  int max_splits, int* nparts, cudaStream_t s, int kmaj, float* lse2) {
+                  int max_splits, int* nparts, cudaStream_t s, int kmaj, float* lse2, void* sk_ws = nullptr,
+                  size_t sk_bytes = 0) {
   *nparts = 1;
   if (S == 0) return TP_OK;
   const int Hl = nh * d;    // columns of the heads held here
   const int Hs = Hl / t;    // columns of one shard's heads
+  GemmExtra ex;  // scratch for stream-K partials (its plan never also splits K into slots)
+  ex.sk_ws = sk_ws;
+  ex.sk_ws_bytes = sk_bytes;
   // [Q_s | K_s | V_s] = in Wqkv_s into columns [3 s Hs, 3 (s+1) Hs) of QKV.
   int st = run_gemm_tc(dev, in, H, S, Wqkv_shards, t, 0, H, 3 * Hs, QKV, 3LL * Hl, 0, TP_ACT_NONE, s, 1, 0, nullptr,
-                       kmaj);
+                       kmaj, &ex);
   if (st != TP_OK) return st;
   // O_h = softmax(Q_h K_h^T / sqrt d) V_h, written to columns [h d, (h+1) d) of O.
   {
@@ -783,7 +938,7 @@ int attn_products(const DeviceInfo& dev, int S, int H, int nh, int d, int t, con
   }
   // sum_s O_s Wo_s, the O projection row-split by head, summed in TMEM.
   return run_gemm_tc(dev, Obuf, Hl, S, Wo_shards, t, 1, Hs, H, Zsum, H, 1, TP_ACT_NONE, s, max_splits,
-                     static_cast<long long>(S) * H, nparts, kmaj);
+                     static_cast<long long>(S) * H, nparts, kmaj, &ex);
 }
 
 int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out_dtype, const void* in,
@@ -797,8 +952,12 @@ int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out
   float* Zsum = keep ? keep->zsum
                      : reinterpret_cast<float*>(static_cast<uint8_t*>(Obuf) + align256(static_cast<size_t>(S) * H * 2));
   int nparts = 1;
+  // Slots 1.. of the partial-sum area double as stream-K scratch (not when a
+  // training forward keeps a single slot in its state).
+  const size_t sh4 = static_cast<size_t>(S) * H * 4;
   int st = attn_products(dev, S, H, nh, d, t, in, Wqkv_shards, Wo_shards, QKV, Obuf, Zsum,
-                         keep ? 1 : TP_MAX_K_SPLITS, &nparts, s, kmaj, keep ? keep->lse2 : nullptr);
+                         keep ? 1 : TP_MAX_K_SPLITS, &nparts, s, kmaj, keep ? keep->lse2 : nullptr,
+                         keep ? nullptr : reinterpret_cast<uint8_t*>(Zsum) + sh4, keep ? 0 : (TP_MAX_K_SPLITS - 1) * sh4);
   if (st != TP_OK) return st;
   return run_reduce_ln(S, H, nparts, Zsum, res, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s, dev.sm_count,
                        apply_ln);
@@ -1550,8 +1709,16 @@ int tp_set_gemm_tile_n(int tile_n) {
   return TP_OK;
 }
 
-int tp_gemm_plan(int M, int t, int row_mode, int shard_k, int shard_n, int out_f32, int b_kmajor,
-                 int heavy_epilogue, int slots, int max_splits, int* tile_n, int* splits) {
+int tp_set_gemm_stream_k(int mode) {
+  if (mode < -1 || mode > 1) return TP_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_stream_k = mode;
+  return TP_OK;
+}
+
+int tp_gemm_plan_sk(int M, int t, int row_mode, int shard_k, int shard_n, int out_f32, int b_kmajor,
+                    int heavy_epilogue, int slots, int max_splits, size_t sk_area_bytes, int* tile_n, int* splits,
+                    int* stream_k, int* sk_clusters) {
   if (M < 1 || t < 1 || t > TP_MAX_SHARDS || shard_k < 1 || shard_n < 1 || slots < 1 || max_splits < 1 ||
       !tile_n || !splits)
     return TP_ERR_INVALID_ARG;
@@ -1566,13 +1733,41 @@ int tp_gemm_plan(int M, int t, int row_mode, int shard_k, int shard_n, int out_f
   p.out_f32 = out_f32 ? 1 : 0;
   p.b_kmajor = b_kmajor ? 1 : 0;
   p.epi_mode = heavy_epilogue ? tp::EPI_GRAD : tp::EPI_PLAIN;
-  const TilePlan plan = plan_tiles(p, M >= TP_GEMM_PAIR_MIN_ROWS, slots, out_f32 ? max_splits : 1);
+  const TilePlan plan = plan_tiles(p, M >= TP_GEMM_PAIR_MIN_ROWS, slots, out_f32 ? max_splits : 1, sk_area_bytes);
   *tile_n = plan.tile_n;
   *splits = plan.splits;
+  if (stream_k) *stream_k = plan.stream_k;
+  if (sk_clusters) *sk_clusters = plan.sk_clusters;
   return TP_OK;
 }
 
+int tp_gemm_plan(int M, int t, int row_mode, int shard_k, int shard_n, int out_f32, int b_kmajor,
+                 int heavy_epilogue, int slots, int max_splits, int* tile_n, int* splits) {
+  return tp_gemm_plan_sk(M, t, row_mode, shard_k, shard_n, out_f32, b_kmajor, heavy_epilogue, slots, max_splits, 0,
+                         tile_n, splits, nullptr, nullptr);
+}
+
 // ------------------------------------------------------------- self-test
+int tp_selftest_flag_wait_timeout(long long limit_cycles, void* stream) {
+  if (limit_cycles < 1) return TP_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  int st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  tp::selftest_flag_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles);
+  return launch_status();
+}
+
+int tp_selftest_exp2(const float* x, float* y_poly, float* y_exp2f, int n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y_poly || !y_exp2f))) return TP_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  int st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  if (n == 0) return TP_OK;
+  const int blocks = ceil_div(n, 256) < 4 * dev->sm_count ? ceil_div(n, 256) : 4 * dev->sm_count;
+  tp::selftest_exp2_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_exp2f, n);
+  return launch_status();
+}
+
 int tp_selftest_wait_timeout(long long limit_cycles, void* stream) {
   if (limit_cycles < 1) return TP_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;

@@ -38,3 +38,15 @@ def test_bounded_wait_times_out_and_context_survives(cuda_device):
 def test_selftest_rejects_bad_limit(cuda_device):
     with pytest.raises(L.TPError):
         L.selftest_wait_timeout(0)
+
+
+def test_bounded_flag_wait_times_out_and_context_survives(cuda_device):
+    """The stream-K finisher's kind of wait (a global flag another CTA pair
+    publishes): a flag nothing sets makes it give up with TP_ERR_TIMEOUT."""
+    assert L.device_error() == 0
+    L.selftest_flag_wait_timeout(20_000_000)
+    torch.cuda.synchronize()
+    assert L.device_error() == TP_ERR_TIMEOUT
+    assert L.device_error() == 0
+    with pytest.raises(L.TPError):
+        L.selftest_flag_wait_timeout(0)

@@ -307,3 +307,21 @@ def test_transformer_block(cuda_device, pre_ln, S, nh, F, t, layout):
     assert L.device_error() == 0
     ref = O.transformer_block(a.X, a.Wqkv, a.Wo, m.A, m.B, nh, d, ln1=ln1, ln2=ln2, pre_ln=pre_ln)
     assert rel_err(Y, ref) <= TOL_BF16
+
+
+def test_attention_polynomial_exp2_against_exp2f(cuda_device):
+    """The attention kernel evaluates one exponential pair in four on the FMA
+    pipe.  Over the range its softmax arguments take (s * log2(e)/sqrt(d) - m,
+    at most 2^8 above the running max, far below it for small scores), its
+    relative error against CUDA's exp2f stays within the polynomial's fitted
+    bound (2.7e-6) plus exp2f's own few ulp."""
+    x = torch.cat([torch.linspace(-125.0, 8.0, 1_000_001), torch.linspace(-1.0, 1.0, 200_001),
+                   torch.tensor([0.0, -0.5, 0.5, -1.0, 8.0, -125.0])]).cuda()
+    yp, yr = L.selftest_exp2(x)
+    torch.cuda.synchronize()
+    rel = ((yp.double() - yr.double()).abs() / yr.double()).max().item()
+    assert rel <= 3.0e-6, rel
+    # integer arguments: 2^n exactly up to the polynomial's value at f = 0
+    yi, _ = L.selftest_exp2(torch.tensor([0.0, 1.0, -3.0, 7.0]).cuda())
+    torch.cuda.synchronize()
+    np.testing.assert_allclose(yi.cpu().numpy(), [1.0, 2.0, 0.125, 128.0], rtol=1e-6)

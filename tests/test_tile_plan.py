@@ -87,3 +87,43 @@ def test_bad_arguments():
         assert lib.tp_gemm_plan(*args, 0, 0, 0, PAIRS, 1, ctypes.byref(tn), ctypes.byref(sp)) == 1
     assert lib.tp_gemm_plan(64, 4, 0, 64, 64, 0, 0, 0, 0, 1, ctypes.byref(tn), ctypes.byref(sp)) == 1
     assert lib.tp_gemm_plan(64, 4, 0, 64, 64, 0, 0, 0, PAIRS, 1, None, ctypes.byref(sp)) == 1
+
+
+# With the sublayers' spare partial-sum slots (3 x S x H x 4 bytes) as stream-K
+# scratch: (tile_n, splits, stream_k, pairs).  Stream-K wins where whole-tile
+# waves leave pairs idle: 64 or 128 tiles of 512 columns on 74 pairs, 256 or
+# 384 in 3.46 / 5.19 waves.  The large MLP's first GEMM (1536 tiles, 20.75
+# waves) gains under 2 % and keeps whole tiles.
+SK_CASES = [
+    ("mlp GEMM1", 2048, 4, 0, 4096, 4096, 0, 1, 2048 * 4096, (512, 1, 1, 74)),
+    ("mlp GEMM2", 2048, 4, 1, 4096, 4096, 1, 4, 2048 * 4096, (512, 1, 1, 74)),
+    ("QKV", 2048, 4, 0, 8192, 6144, 0, 1, 2048 * 8192, (512, 1, 1, 74)),
+    ("O projection", 2048, 4, 1, 2048, 8192, 1, 4, 2048 * 8192, (512, 1, 1, 74)),
+    ("large GEMM1", 4096, 8, 0, 12288, 6144, 0, 1, 4096 * 12288, (512, 1, 0, 0)),
+    ("large GEMM2", 4096, 8, 1, 6144, 12288, 1, 4, 4096 * 12288, (512, 1, 1, 74)),
+    # too little scratch for 74 partial blocks of 256 x 256: the K split stays
+    ("small row split", 1024, 4, 1, 1024, 1024, 1, 4, 1024 * 1024, (256, 4, 0, 0)),
+]
+
+
+@pytest.mark.parametrize("case", SK_CASES, ids=[c[0] for c in SK_CASES])
+def test_stream_k_plan_of_workload_gemms(case):
+    _, M, t, row, sk, sn, f32, ms, sh, want = case
+    assert L.gemm_plan_sk(M, t, row, sk, sn, f32, max_splits=ms, sk_area_bytes=3 * sh * 4) == want
+
+
+def test_stream_k_switch():
+    try:
+        L.set_gemm_stream_k(-1)
+        assert L.gemm_plan_sk(2048, 4, 1, 4096, 4096, 1, max_splits=4, sk_area_bytes=3 * 2048 * 4096 * 4)[2] == 0
+        # forced: as many pairs as the scratch holds 256 x 256 f32 blocks for (+ one flag each)
+        L.set_gemm_stream_k(1)
+        area = 10 * 2 * 128 * 256 * 4 + 256 + 10 * 2 * 8
+        tn, sp, on, pairs = L.gemm_plan_sk(600, 2, 0, 520, 1120, 0, sk_area_bytes=area)
+        assert (tn, sp, on, pairs) == (256, 1, 1, 10)
+        # no scratch, no stream-K
+        assert L.gemm_plan_sk(600, 2, 0, 520, 1120, 0, sk_area_bytes=0)[2] == 0
+        with pytest.raises(L.TPError):
+            L.set_gemm_stream_k(2)
+    finally:
+        L.set_gemm_stream_k(0)

@@ -44,6 +44,12 @@
 // Column mode can give each shard its own A (a_per_shard): t independent
 // products A_s B_s in one persistent launch (the attention backward's heads).
 //
+// Dual accumulators (dual = 1, column mode, 256-column tiles): each tile runs
+// two products of the same shape, A B (k-blocks [0, k/2)) into TMEM columns
+// [0, 256) and A2 B2 (k-blocks [k/2, k)) into [256, 512), and the epilogue
+// reads both: the attention backward's scores Q K^T and dP = dO V^T for the
+// same block, from which it makes P and dS together (EPI_DUAL_SOFTMAX).
+//
 // Stream-K (sk = 1): instead of whole tiles dealt round-robin to the clusters
 // (the last wave partly idle when the tile count is not a multiple of the
 // cluster count), the k-blocks of all tiles, laid end to end, are cut into
@@ -83,6 +89,11 @@ struct GemmCfg {
 #endif
 #ifndef TP_GEMM_WIDE_STAGES
 #define TP_GEMM_WIDE_STAGES 4
+#endif
+// Epilogue stores: each epilogue warp issues the TMA store of its own 32 rows
+// (1), or one thread stores all 128 rows after a barrier of the four warps (0).
+#ifndef TP_GEMM_WARP_STORES
+#define TP_GEMM_WARP_STORES 0
 #endif
   static_assert(!WIDE || CG == 2, "wide tiles need a CTA pair");
   static constexpr int STAGES = WIDE ? TP_GEMM_WIDE_STAGES : (CG == 2 ? TP_GEMM_PAIR_STAGES : 4);
@@ -175,9 +186,16 @@ struct GemmArgs {
   float* sk_ws;
   unsigned long long* sk_flags;
   unsigned long long sk_epoch;
+  // Dual accumulators (see the top of this file): the second product's A and
+  // B maps per shard, and its epilogue row vector and scale.
+  int dual;
+  CUtensorMap tmA2[MAX_SHARDS];
+  CUtensorMap tmB2[MAX_SHARDS];
+  const float* rowvec2;
+  float epi_scale2;
 };
 
-enum : int { EPI_PLAIN = 0, EPI_AUX_PRE = 1, EPI_GRAD = 2, EPI_SOFTMAX = 3, EPI_DSOFTMAX = 4 };
+enum : int { EPI_PLAIN = 0, EPI_AUX_PRE = 1, EPI_GRAD = 2, EPI_SOFTMAX = 3, EPI_DSOFTMAX = 4, EPI_DUAL_SOFTMAX = 5 };
 
 // One piece of work of a cluster: the k-blocks [kb0, kb1) of a tile (of K
 // split `split` in the K-split mode), and what its epilogue does with them.
@@ -394,6 +412,39 @@ __device__ __forceinline__ void epi_chunk_dsoftmax(uint32_t taddr, uint8_t* stag
   }
 }
 
+// Dual softmax epilogue chunk (bf16 out, 64 columns): from the scores s (TMEM
+// columns taddr ..) and dP (taddr + 256 ..) of the same row,
+//   P  = 2^(s * scale1 - r1)                 into stage_p,
+//   dS = P (dP - r2) scale2                  into stage_ds,
+// with P in f32 for dS (its bf16 rounding only for the stored copy).
+__device__ __forceinline__ void epi_chunk_dual_softmax(uint32_t taddr, uint8_t* stage_p, uint8_t* stage_ds,
+                                                       int row_local, float r1, float scale1, float r2,
+                                                       float scale2) {
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    uint32_t sv[32], dv[32];
+    tmem_ld_32x32b_x32(taddr + h * 32, sv);
+    tmem_ld_32x32b_x32(taddr + 256 + h * 32, dv);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t wp[4], wd[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i0 = 8 * j + 2 * e;
+        const float p0 = exp2f(fmaf(__uint_as_float(sv[i0]), scale1, -r1));
+        const float p1 = exp2f(fmaf(__uint_as_float(sv[i0 + 1]), scale1, -r1));
+        wp[e] = pack_bf16x2(p0, p1);
+        wd[e] = pack_bf16x2(p0 * (__uint_as_float(dv[i0]) - r2) * scale2,
+                            p1 * (__uint_as_float(dv[i0 + 1]) - r2) * scale2);
+      }
+      const int off = ((4 * h + j) ^ (row_local & 7)) << 4;
+      *reinterpret_cast<uint4*>(stage_p + off) = make_uint4(wp[0], wp[1], wp[2], wp[3]);
+      *reinterpret_cast<uint4*>(stage_ds + off) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+    }
+  }
+}
+
 template <int ACT>
 __device__ __forceinline__ void epi_chunk_f32(uint32_t taddr, uint8_t* stage_row, int row_local) {
   uint32_t r[32];
@@ -468,6 +519,13 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& p, int tile) {
 __device__ __forceinline__ void kblock_coords(const GemmArgs& p, const TileCoord& tc, int kb, int& shard, int& a_x,
                                               int& b_y) {
   constexpr int BK = 64;
+  if (p.dual) {  // k-blocks [k/2, k) are the second product's, from its own k = 0
+    const int half = p.k_blocks / 2;
+    shard = tc.shard;
+    b_y = (kb < half ? kb : kb - half) * BK;
+    a_x = b_y;
+    return;
+  }
   if (p.row_mode) {
     shard = kb / p.k_blocks_per_shard;
     b_y = (kb % p.k_blocks_per_shard) * BK;
@@ -622,20 +680,24 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
           kblock_coords(p, tc, kb, shard, a_x, b_y);
           uint8_t* dA = sA + stage * C::A_BYTES;
           uint8_t* dB = sB + stage * C::B_BYTES;
+          // Dual accumulators: the second half of the k-blocks is the second product's.
+          const bool second = p.dual && kb >= p.k_blocks / 2;
+          const CUtensorMap* mAk = second ? &p.tmA2[p.a_per_shard ? tc.shard : 0] : mA;
+          const CUtensorMap* mBk = second ? &p.tmB2[shard] : &p.tmB[shard];
           if constexpr (CG == 1) {
             mbar_arrive_expect_tx(&full[stage], bytes);
             armed[stage] = static_cast<int>(phase);
             if (p.a_mnmajor) {
               for (int j = 0; j < my_aboxes; ++j)
-                tma_load_2d(dA + j * C::B_BOX_BYTES, mA, my_row0 + j * 64, a_x, &full[stage]);
+                tma_load_2d(dA + j * C::B_BOX_BYTES, mAk, my_row0 + j * 64, a_x, &full[stage]);
             } else {
-              tma_load_2d(dA, mA, a_x, my_row0, &full[stage]);
+              tma_load_2d(dA, mAk, a_x, my_row0, &full[stage]);
             }
             if (p.b_kmajor) {
-              if (my_boxes) tma_load_2d(dB, &p.tmB[shard], b_y, b_x0, &full[stage]);
+              if (my_boxes) tma_load_2d(dB, mBk, b_y, b_x0, &full[stage]);
             } else {
               for (int j = 0; j < my_boxes; ++j)
-                tma_load_2d(dB + j * C::B_BOX_BYTES, &p.tmB[shard], b_x0 + j * C::B_BOX_N, b_y, &full[stage]);
+                tma_load_2d(dB + j * C::B_BOX_BYTES, mBk, b_x0 + j * C::B_BOX_N, b_y, &full[stage]);
             }
           } else {
             const uint32_t bar = mapa_shared(smem_u32(&full[stage]), 0);
@@ -645,23 +707,23 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
             }
             if (p.a_mnmajor) {
               for (int j = 0; j < my_aboxes; ++j)
-                tma_load_2d_pair(dA + j * C::B_BOX_BYTES, mA, my_row0 + j * 64, a_x, bar);
+                tma_load_2d_pair(dA + j * C::B_BOX_BYTES, mAk, my_row0 + j * 64, a_x, bar);
             } else if (my_a) {
-              tma_load_2d_pair(dA, mA, a_x, my_row0, bar);
+              tma_load_2d_pair(dA, mAk, a_x, my_row0, bar);
             }
             if (p.b_kmajor) {
-              if (my_boxes) tma_load_2d_pair(dB, &p.tmB[shard], b_y, b_x0, bar);
+              if (my_boxes) tma_load_2d_pair(dB, mBk, b_y, b_x0, bar);
             } else {
               for (int j = 0; j < my_boxes; ++j)
-                tma_load_2d_pair(dB + j * C::B_BOX_BYTES, &p.tmB[shard], b_x0 + j * C::B_BOX_N, b_y, bar);
+                tma_load_2d_pair(dB + j * C::B_BOX_BYTES, mBk, b_x0 + j * C::B_BOX_N, b_y, bar);
             }
             if constexpr (WIDE) {
               uint8_t* dB2 = dB + C::B_REGION_BYTES;
               if (p.b_kmajor) {
-                if (my_boxes2) tma_load_2d_pair(dB2, &p.tmB[shard], b_y, b_x2, bar);
+                if (my_boxes2) tma_load_2d_pair(dB2, mBk, b_y, b_x2, bar);
               } else {
                 for (int j = 0; j < my_boxes2; ++j)
-                  tma_load_2d_pair(dB2 + j * C::B_BOX_BYTES, &p.tmB[shard], b_x2 + j * C::B_BOX_N, b_y, bar);
+                  tma_load_2d_pair(dB2 + j * C::B_BOX_BYTES, mBk, b_x2 + j * C::B_BOX_N, b_y, bar);
               }
             }
           }
@@ -686,6 +748,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
+      const int acc_bufs = p.dual ? 1 : C::ACC_BUFS;  // dual: both 256-column halves per tile
       for (int idx = 0; idx < num_items && ok; ++idx) {
         const WorkItem wi = work_item(p, cluster_id, num_clusters, idx, num_items);
         const int kb_begin = wi.kb0, kb_end = wi.kb1;
@@ -712,9 +775,11 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
             // B K-major: like A.
             const uint64_t bd = p.b_kmajor ? sdesc_sw128(b0 + kk * 32, 16, 1024)
                                            : sdesc_sw128(b0 + kk * 2048, C::B_BOX_BYTES, 1024);
-            const uint32_t accum = (kb != kb_begin || kk != 0) ? 1u : 0u;
-            if constexpr (CG == 1) umma_bf16(d_tmem, ad, bd, idesc, accum);
-            else umma_bf16_pair(d_tmem, ad, bd, idesc, accum);
+            const bool second = p.dual && kb >= p.k_blocks / 2;
+            const uint32_t accum = ((kb != kb_begin && !(p.dual && kb == p.k_blocks / 2)) || kk != 0) ? 1u : 0u;
+            const uint32_t dt = d_tmem + (second ? static_cast<uint32_t>(C::BN) : 0u);
+            if constexpr (CG == 1) umma_bf16(dt, ad, bd, idesc, accum);
+            else umma_bf16_pair(dt, ad, bd, idesc, accum);
             if constexpr (WIDE) {
               if (two) {
                 const uint32_t b2 = b0 + C::B_REGION_BYTES;
@@ -731,7 +796,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         if (!ok) break;
         if constexpr (CG == 1) umma_commit(&tfull[acc]);
         else umma_commit_pair_mc(&tfull[acc], 0x3);
-        if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
+        if (++acc == acc_bufs) { acc = 0; acc_phase ^= 1; }
       }
       if (!ok) {
         // Wait (bounded) for every MMA already issued before TMEM is freed.
@@ -756,6 +821,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
     uint32_t acc_phase = 0;
     int buf = 0;
     const uint32_t tempty_leader0 = CG == 2 ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
+    const int acc_bufs = p.dual ? 1 : C::ACC_BUFS;
     for (int idx = 0; idx < num_items; ++idx) {
       const WorkItem wi = work_item(p, cluster_id, num_clusters, idx, num_items);
       const TileCoord tc = tile_coord<CG>(p, wi.tile);
@@ -797,7 +863,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         __threadfence();
         named_barrier_sync(1, 128);
         if (elected) flag_publish(p.sk_flags + cluster_id * CG + rank, p.sk_epoch);
-        if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
+        if (++acc == acc_bufs) { acc = 0; acc_phase ^= 1; }
         continue;
       }
       if (wi.role == ROLE_FINISHER) {
@@ -845,11 +911,60 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       const float rv = (p.rowvec != nullptr && grow < p.M)
                            ? __ldg(p.rowvec + static_cast<long long>(tc.shard) * p.rowvec_ld + grow)
                            : 0.0f;
+      if (p.epi_mode == EPI_DUAL_SOFTMAX) {
+        // P into staging buffer 0 and dS into buffer 1, then one store of each.
+        const float rv2 = (p.rowvec2 != nullptr && grow < p.M)
+                              ? __ldg(p.rowvec2 + static_cast<long long>(tc.shard) * p.rowvec_ld + grow)
+                              : 0.0f;
+        for (int c = 0; c < nchunks; ++c) {
+#if TP_GEMM_WARP_STORES
+          if (lane == 0) bulk_wait_group_read<0>();
+          __syncwarp();
+#else
+          if (elected) bulk_wait_group_read<0>();
+          named_barrier_sync(1, 128);
+#endif
+          epi_chunk_dual_softmax(t_row + c * 64, sEpi + row_local * 128, sEpi + C::EPI_BUF_BYTES + row_local * 128,
+                                 row_local, rv, p.epi_scale, rv2, p.epi_scale2);
+          if (c == nchunks - 1) {
+            tc_fence_before();
+            if constexpr (CG == 1) {
+              mbar_arrive(&tempty[acc]);
+            } else {
+              __syncwarp();
+              if (lane == 0) mbar_arrive_cluster(tempty_leader0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+            }
+          }
+          fence_proxy_async_smem();
+#if TP_GEMM_WARP_STORES
+          __syncwarp();
+          if (lane == 0 && y0 + q * 32 < p.M) {
+            tma_store_3d(tmC, sEpi + q * 32 * 128, tc.n_in + c * 64, ystore + q * 32, 0);
+            tma_store_3d(tmAux, sEpi + C::EPI_BUF_BYTES + q * 32 * 128, tc.n_in + c * 64, ystore + q * 32, 0);
+            bulk_commit_group();
+          }
+#else
+          named_barrier_sync(1, 128);
+          if (elected && y0 < p.M) {
+            tma_store_3d(tmC, sEpi, tc.n_in + c * 64, ystore, 0);
+            tma_store_3d(tmAux, sEpi + C::EPI_BUF_BYTES, tc.n_in + c * 64, ystore, 0);
+            bulk_commit_group();
+          }
+#endif
+        }
+        if (++acc == acc_bufs) { acc = 0; acc_phase ^= 1; }
+        continue;
+      }
       for (int c = 0; c < nchunks; ++c) {
         for (int part = 0; part < parts; ++part) {
           // The TMA store that last read this staging buffer must be done with it.
+#if TP_GEMM_WARP_STORES
+          if (lane == 0) bulk_wait_group_read<1>();
+          __syncwarp();
+#else
           if (elected) bulk_wait_group_read<1>();
           named_barrier_sync(1, 128);
+#endif
           uint8_t* stage_row = sEpi + buf * C::EPI_BUF_BYTES + row_local * 128;
           const uint32_t taddr = t_row + c * (p.out_f32 ? 32 : 64);
           if (p.epi_mode == EPI_SOFTMAX) {
@@ -896,18 +1011,33 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
             }
           }
           fence_proxy_async_smem();
+#if TP_GEMM_WARP_STORES
+          // Each warp stores its own 32 rows (a 4 KiB, 1 KiB-aligned slice of the
+          // staging buffer, so the 128-byte swizzle pattern is the same).
+          __syncwarp();
+          if (lane == 0 && y0 + q * 32 < p.M) {
+            const CUtensorMap* map = part < parts - 1 ? tmAux : tmC;
+            tma_store_3d(map, sEpi + buf * C::EPI_BUF_BYTES + q * 32 * 128, tc.n_in + c * cw, ystore + q * 32, split);
+            bulk_commit_group();
+          }
+#else
           named_barrier_sync(1, 128);
           if (elected && y0 < p.M) {
             const CUtensorMap* map = part < parts - 1 ? tmAux : tmC;
             tma_store_3d(map, sEpi + buf * C::EPI_BUF_BYTES, tc.n_in + c * cw, ystore, split);
             bulk_commit_group();
           }
+#endif
           buf ^= 1;
         }
       }
-      if (++acc == C::ACC_BUFS) { acc = 0; acc_phase ^= 1; }
+      if (++acc == acc_bufs) { acc = 0; acc_phase ^= 1; }
     }
+#if TP_GEMM_WARP_STORES
+    if (lane == 0) bulk_wait_group_all();
+#else
     if (elected) bulk_wait_group_all();
+#endif
   }
 
   tc_fence_before();

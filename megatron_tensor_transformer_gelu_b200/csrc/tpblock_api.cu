@@ -43,6 +43,12 @@ struct DeviceInfo {
 #define TP_RLN_BULK 1
 #endif
 
+// The attention backward makes P and dS in one dual-accumulator GEMM (1) or in
+// a score GEMM and a dP GEMM that reads P back (0).
+#ifndef TP_ATTN_BACK_DUAL
+#define TP_ATTN_BACK_DUAL 1
+#endif
+
 // Most K-split partial-sum slots a row-split GEMM feeding the LayerNorm may use.
 #define TP_MAX_K_SPLITS 4
 
@@ -168,8 +174,9 @@ bool tmap_bf16(CUtensorMap* m, const void* base, long long rows, long long cols,
 }
 
 // 3-D output map {cols, rows, slots} over row-major [slots][rows][ld] (f32 or
-// bf16); box {128 bytes of columns, 128 rows, 1 slot}; 128-byte swizzle.  TMA
-// stores through it write nothing outside [cols] x [rows] x [slots].
+// bf16); box {128 bytes of columns, 128 rows (32 with per-warp epilogue
+// stores), 1 slot}; 128-byte swizzle.  TMA stores through it write nothing
+// outside [cols] x [rows] x [slots].
 bool tmap_out(CUtensorMap* m, void* base, int f32, long long cols, long long rows, long long slots, long long ld,
               long long slot_stride) {
   const cuuint64_t es = f32 ? 4u : 2u;
@@ -177,7 +184,7 @@ bool tmap_out(CUtensorMap* m, void* base, int f32, long long cols, long long row
                         static_cast<cuuint64_t>(slots)};
   const long long ss = slot_stride > 0 ? slot_stride : rows * ld;
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(ld) * es, static_cast<cuuint64_t>(ss) * es};
-  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), 128u, 1u};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / es), TP_GEMM_WARP_STORES ? 32u : 128u, 1u};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = g_encode(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -403,6 +410,15 @@ struct GemmExtra {
   float epi_scale = 1.0f;
   void* sk_ws = nullptr;             // scratch the launch may use for stream-K partials and flags
   size_t sk_ws_bytes = 0;            //   (256-byte aligned; 0: no stream-K)
+  // Dual accumulators (column mode, K-major B, EPI_DUAL_SOFTMAX): a second
+  // product A2_s B2_s of the same shape per shard, its A with row stride lda2
+  // and its B with row stride ldb2; the second output (dS) goes to `aux`.
+  const void* const* A2_shards = nullptr;
+  long long lda2 = 0;
+  const void* const* B2_shards = nullptr;
+  long long ldb2 = 0;
+  const float* rowvec2 = nullptr;
+  float epi_scale2 = 1.0f;
 };
 
 template <int CG, bool WIDE>
@@ -431,7 +447,7 @@ int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, const TilePlan& plan,
       void* base = ex.C_shards ? ex.C_shards[s] : static_cast<uint8_t*>(p.C) + static_cast<long long>(s) * p.shard_n * es;
       const long long ld = ex.C_shards ? ex.ldc_shard : p.ldc;
       if (!tmap_out(&p.tmC[s], base, p.out_f32, p.shard_n, p.M, 1, ld, 0)) return TP_ERR_CUDA;
-      if (ex.epi_mode == tp::EPI_AUX_PRE) {
+      if (ex.epi_mode == tp::EPI_AUX_PRE || ex.epi_mode == tp::EPI_DUAL_SOFTMAX) {
         void* abase = static_cast<uint8_t*>(const_cast<void*>(ex.aux)) + static_cast<long long>(s) * p.shard_n * 2;
         if (!tmap_out(&p.tmAux[s], abase, 0, p.shard_n, p.M, 1, ex.ld_aux, 0)) return TP_ERR_CUDA;
       }
@@ -508,9 +524,25 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
       ok = tmap_bf16(&p.tmB[s], B[s], shard_k, shard_n, ex.ldb ? ex.ldb : shard_n, G::B_BOX_N, G::BK);
     if (!ok) return TP_ERR_CUDA;
   }
-  const bool softmax_epi = ex.epi_mode == tp::EPI_SOFTMAX || ex.epi_mode == tp::EPI_DSOFTMAX;
+  const bool softmax_epi = ex.epi_mode == tp::EPI_SOFTMAX || ex.epi_mode == tp::EPI_DSOFTMAX ||
+                           ex.epi_mode == tp::EPI_DUAL_SOFTMAX;
   if (softmax_epi && (out_f32 || row_mode || !ex.rowvec || (ex.epi_mode == tp::EPI_DSOFTMAX && !ex.aux)))
     return TP_ERR_INVALID_ARG;
+  const bool dual = ex.epi_mode == tp::EPI_DUAL_SOFTMAX;
+  if (dual) {
+    // Dual accumulators: the second product's maps, shaped like the first's.
+    if (!ex.A2_shards || !ex.B2_shards || !ex.rowvec2 || !ex.aux || !b_kmajor || ex.a_mnmajor || ex.m_split)
+      return TP_ERR_INVALID_ARG;
+    for (int s = 0; s < t; ++s) {
+      if (!tmap_bf16(&p.tmA2[s], ex.A2_shards[s], M, K_total, ex.lda2, G::BK, G::BM) ||
+          !tmap_bf16(&p.tmB2[s], ex.B2_shards[s], shard_n, shard_k, ex.ldb2, G::BK,
+                     pair ? tp::GemmCfg<2>::B_COLS_CTA : G::BN))
+        return TP_ERR_CUDA;
+    }
+    p.dual = 1;
+    p.rowvec2 = ex.rowvec2;
+    p.epi_scale2 = ex.epi_scale2;
+  }
   p.a_mnmajor = ex.a_mnmajor;
   p.epi_mode = ex.epi_mode;
   p.rowvec = ex.rowvec;
@@ -528,14 +560,19 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
   p.N = row_mode ? shard_n : shard_n * t;
   p.k_blocks_per_shard = ceil_div(shard_k, G::BK);
   p.k_blocks = row_mode ? p.k_blocks_per_shard * t : p.k_blocks_per_shard;
+  if (dual) p.k_blocks *= 2;  // the second product's k-blocks follow the first's
   p.act = act;
   p.out_f32 = out_f32;
   p.splits = 1;
   p.slot_stride = slot_stride;
   p.b_kmajor = b_kmajor;
   if (!out_f32) max_splits = 1;
-  const TilePlan plan = plan_tiles(p, pair, pair ? dev.max_pairs : dev.sm_count, max_splits,
-                                   (ex.sk_ws && ex.m_split == 0) ? ex.sk_ws_bytes : 0);
+  TilePlan plan = plan_tiles(p, pair, pair ? dev.max_pairs : dev.sm_count, max_splits,
+                             (ex.sk_ws && ex.m_split == 0) ? ex.sk_ws_bytes : 0);
+  if (dual) {  // both accumulators fill TMEM: 256-column tiles, one tile at a time
+    plan = TilePlan();
+    plan.tile_n = 256;
+  }
   int r;
   if (!pair) r = launch_gemm_tc<1, false>(dev, p, plan, ex, st);
   else if (plan.tile_n > tp::GemmCfg<2>::BN) r = launch_gemm_tc<2, true>(dev, p, plan, ex, st);
@@ -1402,6 +1439,30 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
       dKg[j] = dQKV + (qcol + Hs) * 2;
       dVg[j] = dQKV + (qcol + 2LL * Hs) * 2;
     }
+#if TP_ATTN_BACK_DUAL
+    // P_h = 2^(Q_h K_h^T scale_log2 - lse2_h) and dS_h = P_h (dO_h V_h^T - D_h) / sqrt d
+    // from one tile: the scores and dP of the same 256 x 256 block in the two
+    // halves of TMEM (K_h and V_h [keys, d] are the K-major B operands).
+    {
+      GemmExtra ex;
+      ex.ldb = H3;
+      ex.A_shards = Qg;
+      ex.A2_shards = dOg;
+      ex.lda2 = H;
+      ex.B2_shards = Vg;
+      ex.ldb2 = H3;
+      ex.epi_mode = tp::EPI_DUAL_SOFTMAX;
+      ex.aux = dS;
+      ex.ld_aux = GS;
+      ex.rowvec = lse2 + static_cast<long long>(h0) * S;
+      ex.rowvec2 = D + static_cast<long long>(h0) * S;
+      ex.rowvec_ld = S;
+      ex.epi_scale = scale_log2;
+      ex.epi_scale2 = scale;
+      st = run_gemm_tc(*dev, Qg[0], H3, S, Kg, g, 0, d, S, P, GS, 0, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
+      if (st != TP_OK) return st;
+    }
+#else
     // P_h = 2^(Q_h K_h^T scale_log2 - lse2_h) (K_h [keys, d] is the K-major B operand)
     {
       GemmExtra ex;
@@ -1414,6 +1475,7 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
       st = run_gemm_tc(*dev, Qg[0], H3, S, Kg, g, 0, d, S, P, GS, 0, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
       if (st != TP_OK) return st;
     }
+#endif
     // dV_h = P_h^T dO_h into V_h's columns of dQKV (P_h read M-major)
     {
       GemmExtra ex;
@@ -1425,6 +1487,7 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
       st = run_gemm_tc(*dev, Pg[0], GS, S, dOg, g, 0, S, d, dVg[0], H3, 0, TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
       if (st != TP_OK) return st;
     }
+#if !TP_ATTN_BACK_DUAL
     // dS_h = P_h (dO_h V_h^T - D_h) / sqrt d (V_h [keys, d] is the K-major B operand)
     {
       GemmExtra ex;
@@ -1439,6 +1502,7 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
       st = run_gemm_tc(*dev, dOg[0], H, S, Vg, g, 0, d, S, dS, GS, 0, TP_ACT_NONE, s, 1, 0, nullptr, 1, &ex);
       if (st != TP_OK) return st;
     }
+#endif
     // dQ_h = dS_h K_h and dK_h = dS_h^T Q_h into their columns of dQKV
     {
       GemmExtra ex;

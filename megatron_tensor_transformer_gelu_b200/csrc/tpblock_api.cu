@@ -804,7 +804,43 @@ int run_ln_backward(int S, int H, const float* V, const void* X, const void* dY,
   if (grid > LNB_MAX_CTAS) grid = LNB_MAX_CTAS;
   if (grid > S) grid = S;
   if (grid < 1) grid = 1;
-  {
+#if TP_RLN_BULK
+  // Rows staged in shared memory by bulk copies (X, dY, V: 8 bytes a column),
+  // 2 to 4 stages; rows too wide for two stages take the register kernel.
+  const size_t stage = (static_cast<size_t>(H) * 8 + 127) & ~size_t(127);
+  const bool bulk = 2 * stage <= static_cast<size_t>(tp::rlb::MAX_STAGE_SMEM);
+#else
+  const bool bulk = false;
+#endif
+  if (bulk) {
+    const size_t budget = stage <= 32 * 1024 ? 96 * 1024 : tp::rlb::MAX_STAGE_SMEM;
+    int nst = static_cast<int>(budget / stage);
+    nst = nst < 2 ? 2 : (nst > 4 ? 4 : nst);
+    const size_t smem = static_cast<size_t>(nst) * stage;
+    cudaError_t le = cudaSuccess;
+    auto go = [&](auto kern) {
+      int per_sm = 1;
+      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+              cudaSuccess ||
+          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, tp::lnbb::THREADS, smem) != cudaSuccess ||
+          per_sm < 1)
+        per_sm = 1;
+      grid = per_sm * dev_sms;
+      if (grid > LNB_MAX_CTAS) grid = LNB_MAX_CTAS;
+      if (grid > S) grid = S;
+      le = launch_pdl(kern, dim3(grid), dim3(tp::lnbb::THREADS), smem, st, p, nst, static_cast<int>(stage));
+    };
+    ProfScope ps(K_LN_BACK, st);
+    switch ((H + 2047) / 2048) {
+      case 1: go(tp::ln_backward_bulk_kernel<1>); break;
+      case 2: go(tp::ln_backward_bulk_kernel<2>); break;
+      case 3: go(tp::ln_backward_bulk_kernel<3>); break;
+      case 4: go(tp::ln_backward_bulk_kernel<4>); break;
+      case 5: case 6: go(tp::ln_backward_bulk_kernel<6>); break;
+      default: go(tp::ln_backward_bulk_kernel<8>); break;
+    }
+    if (le != cudaSuccess || launch_status() != TP_OK) return TP_ERR_CUDA;
+  } else {
     ProfScope ps(K_LN_BACK, st);
     cudaError_t le;
     switch (ch) {

@@ -358,6 +358,30 @@ int tp_reduce_residual_layernorm(int S, int H, int nparts, const float* parts,
  *   kernel.  The caller orders it after the partials are complete on every
  *   rank and before the outputs are read.  0 <= nparts <= 8; 1 <= nout <= 8;
  *   H % 8 == 0, 8 <= H <= 16384. */
+/* Peer access for the fused form, between the ranks' processes (CUDA IPC).
+ * tp_ipc_export writes a TP_IPC_HANDLE_BYTES-byte handle (host memory) for a
+ * device address of this process (the allocation containing it, and the
+ * address's offset in it); tp_ipc_import maps that allocation in another
+ * process on its current device and returns the same address's counterpart
+ * there (peer access is enabled as needed); tp_ipc_close unmaps an address
+ * tp_ipc_import returned.  TP_ERR_CUDA when the
+ * runtime refuses (for example an import in the exporting process itself).
+ * tp_peer_barrier: rank `rank` of `nranks` (<= 8) stores `epoch` into its
+ * slot of every rank's flag array, then waits (bounded; TP_ERR_TIMEOUT
+ * through tp_device_error() if it gives up) until its own array holds `epoch`
+ * in every rank's slot.  flags[q] is rank q's array of nranks unsigned 64-bit
+ * words (this device's own array at flags[rank], the peers' through
+ * tp_ipc_import), zero when first used; every rank passes the same epoch,
+ * which must grow from call to call.  Enqueued on `stream` between the
+ * partial sums and tp_reduce_residual_layernorm_multi (every partial is
+ * complete before any rank reads it), and after it (every rank's rows have
+ * landed before any output is read). */
+#define TP_IPC_HANDLE_BYTES 72
+int tp_ipc_export(const void* dev_ptr, void* handle);
+int tp_ipc_import(const void* handle, void** dev_ptr);
+int tp_ipc_close(void* dev_ptr);
+int tp_peer_barrier(int nranks, int rank, unsigned long long* const* flags, unsigned long long epoch, void* stream);
+
 size_t tp_mlp_partial_workspace_bytes(int S, int H, int F, int t, int dtype);
 int tp_mlp_partial_forward(int S, int H, int F, int t, int dtype, const void* X, const void* const* A_shards,
                            const void* const* B_shards, int act, float* P, void* workspace, size_t workspace_bytes,

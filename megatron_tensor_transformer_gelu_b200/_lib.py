@@ -71,6 +71,10 @@ SIGNATURES = {
     "tp_attn_partial_forward": (_c_int, [_c_int] * 6 + [_vp, _vpp, _vpp, _vp, _vp, _c_size, _vp]),
     "tp_reduce_residual_layernorm_multi": (_c_int, [_c_int] * 3 + [_vpp, _vp, _c_int, _vp, _vp, _c_float, _c_int,
                                                                    _vpp, _c_int, _vp]),
+    "tp_ipc_export": (_c_int, [_vp, _vp]),
+    "tp_ipc_import": (_c_int, [_vp, ctypes.POINTER(_vp)]),
+    "tp_ipc_close": (_c_int, [_vp]),
+    "tp_peer_barrier": (_c_int, [_c_int, _c_int, _vpp, ctypes.c_ulonglong, _vp]),
     "tp_set_gemm_tile_n": (_c_int, [_c_int]),
     "tp_gemm_plan": (_c_int, [_c_int] * 10 + [ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
     "tp_set_gemm_stream_k": (_c_int, [_c_int]),
@@ -247,6 +251,37 @@ def _addr(x) -> int:
 def _addrs(xs):
     arr = (ctypes.c_void_p * max(1, len(xs)))(*[_addr(x) for x in xs])
     return ctypes.cast(arr, _vpp), arr
+
+
+IPC_HANDLE_BYTES = 72
+
+
+def ipc_export(t) -> bytes:
+    """CUDA IPC handle of a device tensor's allocation (to send to another rank's process)."""
+    buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    _check(lib().tp_ipc_export(ctypes.c_void_p(t.data_ptr()), buf), "tp_ipc_export")
+    return buf.raw
+
+
+def ipc_import(handle: bytes) -> int:
+    """Device address, on the current device, of another process's exported allocation."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError("bad IPC handle")
+    out = ctypes.c_void_p(0)
+    buf = ctypes.create_string_buffer(bytes(handle), IPC_HANDLE_BYTES)
+    _check(lib().tp_ipc_import(buf, ctypes.byref(out)), "tp_ipc_import")
+    return int(out.value)
+
+
+def ipc_close(addr: int) -> None:
+    _check(lib().tp_ipc_close(ctypes.c_void_p(addr)), "tp_ipc_close")
+
+
+def peer_barrier(nranks: int, rank: int, flag_arrays, epoch: int, stream=None) -> None:
+    """flag_arrays: rank q's flag array (tensor or device address) for every q."""
+    pf, kf = _addrs(flag_arrays)
+    _check(lib().tp_peer_barrier(int(nranks), int(rank), pf, ctypes.c_ulonglong(int(epoch)), _stream(stream)),
+           "tp_peer_barrier")
 
 
 def mlp_partial_workspace_bytes(S, H, F, t, dtype=torch.bfloat16) -> int:

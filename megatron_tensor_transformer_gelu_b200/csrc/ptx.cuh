@@ -113,6 +113,52 @@ __device__ __forceinline__ bool flag_wait_eq(const unsigned long long* addr, uns
   }
 }
 
+// Publish / read a flag at system scope (visible to, and written by, other
+// GPUs through peer mappings).
+__device__ __forceinline__ void flag_publish_sys(unsigned long long* addr, unsigned long long v) {
+  asm volatile("st.release.sys.global.u64 [%0], %1;" ::"l"(addr), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long flag_read_sys(const unsigned long long* addr) {
+  unsigned long long v;
+  asm volatile("ld.acquire.sys.global.u64 %0, [%1];" : "=l"(v) : "l"(addr) : "memory");
+  return v;
+}
+
+// Cross-rank barrier of the fused multi-GPU reduction: thread q < nranks
+// stores `epoch` into this rank's slot of rank q's flag array (a peer mapping
+// for q != rank), then waits (bounded, TP_ERR_TIMEOUT through the error word)
+// until this rank's own array holds `epoch` in rank q's slot.
+struct PeerBarrierArgs {
+  unsigned long long* flags[8];  // rank q's array of nranks flags
+  int nranks, rank;
+  unsigned long long epoch;
+  long long limit;
+};
+
+__global__ void peer_barrier_kernel(const PeerBarrierArgs a) {
+  const int q = threadIdx.x;
+  if (q < a.nranks) {
+    __threadfence_system();
+    flag_publish_sys(a.flags[q] + a.rank, a.epoch);
+  }
+  __syncwarp();
+  if (q < a.nranks) {
+    const unsigned long long* mine = a.flags[a.rank] + q;
+    const long long t0 = clock64();
+    uint32_t n = 0;
+    while (flag_read_sys(mine) < a.epoch) {
+      __nanosleep(128);
+      if ((++n & 63u) == 0u && (error_raised() || clock64() - t0 > a.limit)) {
+        flag_error(DEV_ERR_TIMEOUT);
+        break;
+      }
+    }
+  }
+  __syncwarp();
+  __threadfence_system();
+}
+
 // Diagnostic: one thread waits on an mbarrier that nothing completes, so the
 // bounded wait above gives up after `limit` cycles and raises the error word.
 __global__ void selftest_wait_timeout_kernel(long long limit) {

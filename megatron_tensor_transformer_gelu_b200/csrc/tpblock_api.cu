@@ -1801,6 +1801,91 @@ int tp_attn_partial_forward(int S, int H, int nh, int d, int t, int dtype, const
                        P, 1, &nparts, static_cast<cudaStream_t>(stream), 0, nullptr);
 }
 
+// --------------------------------------------- peer access between ranks
+// The handle is the CUDA IPC handle of the allocation that contains dev_ptr
+// (a caching allocator hands out pieces of larger allocations) followed by
+// dev_ptr's byte offset in it; an import maps the allocation and adds the
+// offset.  Imports are remembered so that close can unmap by the address it
+// returned.
+static_assert(sizeof(cudaIpcMemHandle_t) + sizeof(unsigned long long) == TP_IPC_HANDLE_BYTES, "IPC handle size");
+std::mutex g_ipc_mu;
+struct IpcImport {
+  void* addr;
+  void* base;
+};
+IpcImport g_ipc_imports[1024];
+int g_ipc_n = 0;
+
+int tp_ipc_export(const void* dev_ptr, void* handle) {
+  if (!dev_ptr || !handle) return TP_ERR_INVALID_ARG;
+  static PFN_cuMemGetAddressRange_v3020 range_fn = nullptr;
+  if (!range_fn) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+      return TP_ERR_CUDA;
+    range_fn = reinterpret_cast<PFN_cuMemGetAddressRange_v3020>(fn);
+  }
+  CUdeviceptr base = 0;
+  size_t size = 0;
+  if (range_fn(&base, &size, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS) return TP_ERR_CUDA;
+  cudaIpcMemHandle_t h;
+  if (cudaIpcGetMemHandle(&h, reinterpret_cast<void*>(base)) != cudaSuccess) return TP_ERR_CUDA;
+  const unsigned long long off = reinterpret_cast<CUdeviceptr>(dev_ptr) - base;
+  std::memcpy(handle, &h, sizeof(h));
+  std::memcpy(static_cast<uint8_t*>(handle) + sizeof(h), &off, sizeof(off));
+  return TP_OK;
+}
+
+int tp_ipc_import(const void* handle, void** dev_ptr) {
+  if (!handle || !dev_ptr) return TP_ERR_INVALID_ARG;
+  cudaIpcMemHandle_t h;
+  unsigned long long off = 0;
+  std::memcpy(&h, handle, sizeof(h));
+  std::memcpy(&off, static_cast<const uint8_t*>(handle) + sizeof(h), sizeof(off));
+  std::lock_guard<std::mutex> lk(g_ipc_mu);
+  if (g_ipc_n >= 1024) return TP_ERR_INVALID_ARG;
+  void* base = nullptr;
+  if (cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess) return TP_ERR_CUDA;
+  void* addr = static_cast<uint8_t*>(base) + off;
+  g_ipc_imports[g_ipc_n++] = {addr, base};
+  *dev_ptr = addr;
+  return TP_OK;
+}
+
+int tp_ipc_close(void* dev_ptr) {
+  if (!dev_ptr) return TP_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_ipc_mu);
+  for (int i = 0; i < g_ipc_n; ++i) {
+    if (g_ipc_imports[i].addr == dev_ptr) {
+      void* base = g_ipc_imports[i].base;
+      g_ipc_imports[i] = g_ipc_imports[--g_ipc_n];
+      return cudaIpcCloseMemHandle(base) == cudaSuccess ? TP_OK : TP_ERR_CUDA;
+    }
+  }
+  return TP_ERR_INVALID_ARG;
+}
+
+int tp_peer_barrier(int nranks, int rank, unsigned long long* const* flags, unsigned long long epoch, void* stream) {
+  if (nranks < 1 || nranks > TP_MAX_SHARDS || rank < 0 || rank >= nranks || !flags || epoch == 0)
+    return TP_ERR_INVALID_ARG;
+  for (int q = 0; q < nranks; ++q)
+    if (!flags[q] || (reinterpret_cast<uintptr_t>(flags[q]) & 7u)) return TP_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  int st = device_ready(&dev);
+  if (st != TP_OK) return st;
+  tp::PeerBarrierArgs a;
+  std::memset(&a, 0, sizeof(a));
+  for (int q = 0; q < nranks; ++q) a.flags[q] = flags[q];
+  a.nranks = nranks;
+  a.rank = rank;
+  a.epoch = epoch;
+  a.limit = tp::WAIT_LIMIT_CYCLES;
+  tp::peer_barrier_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(a);
+  return launch_status();
+}
+
 int tp_set_gemm_tile_n(int tile_n) {
   if (tile_n != 0 && tile_n != 128 && (tile_n < 256 || tile_n > 512 || tile_n % 32 != 0))
     return TP_ERR_INVALID_ARG;

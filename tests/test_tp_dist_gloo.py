@@ -62,7 +62,7 @@ def _worker(rank, world, port, mode, out):
 
 
 @pytest.mark.parametrize("world", [2, 4])
-@pytest.mark.parametrize("mode", list(tp_dist.MODES))
+@pytest.mark.parametrize("mode", ["allreduce", "rs_ag"])  # the collective modes (peer mode: below)
 def test_gloo_ranks_reduce_every_partial(world, mode):
     port = _free_port()
     mgr = mp.Manager()
@@ -94,7 +94,7 @@ def test_row_split():
 
 def test_single_rank_without_a_process_group():
     # world 1: no collective; both modes reduce the rank's own partial
-    for mode in tp_dist.MODES:
+    for mode in ("allreduce", "rs_ag"):
         def partial(X, P, stream):
             P.fill_(2.0)
 
@@ -105,3 +105,67 @@ def test_single_rank_without_a_process_group():
                                  world=1, rank=0)
         Y = sub.forward(torch.ones(8, 4), torch.zeros(8, 4))
         assert torch.equal(Y, torch.full((8, 4), 3.0))
+
+
+class _FakePeerOps:
+    """Stands in for CUDA IPC and the device barrier: handles are names,
+    imports are made-up addresses, calls are recorded."""
+
+    def __init__(self):
+        self.calls = []
+
+    def export(self, t):
+        return ("handle", t.data_ptr())
+
+    def import_(self, handle):
+        return 10_000_000 + handle[1] % 1_000_003
+
+    def close(self, addr):
+        self.calls.append(("close", addr))
+
+    def barrier(self, nranks, rank, flag_addrs, epoch, stream):
+        self.calls.append(("barrier", nranks, rank, tuple(flag_addrs), epoch))
+
+
+def test_peer_mode_bookkeeping():
+    """Rank 1 of 2: the fused reduction reads rows [S/2, S) of both ranks'
+    partials and writes them into both ranks' outputs, between two barriers
+    with growing epochs; the imports are closed on close()."""
+    S, H, world, rank = 8, 4, 2, 1
+    ops = _FakePeerOps()
+    theirs = {}
+
+    def exchange(mine):
+        other = tuple(("handle", 1000 + 64 * i) for i in range(3))  # rank 0's P, Ybuf, flags
+        theirs["imports"] = [ops.import_(h) for h in other]
+        return [other, mine]
+
+    seen = []
+
+    def partial(X, P, stream):
+        P.fill_(1.0)
+
+    def reduce_ln(rows, parts, X_rows, Y_outs, stream):
+        seen.append((rows, list(parts), X_rows.clone(), list(Y_outs)))
+
+    sub = tp_dist.TPSublayer(partial, S, H, torch.float32, torch.bfloat16, mode="peer", reduce_ln=reduce_ln,
+                             world=world, rank=rank, peer_ops=ops, exchange=exchange)
+    X = torch.arange(S * H, dtype=torch.float32).view(S, H)
+    Y = torch.empty(S, H, dtype=torch.bfloat16)
+    sub.Ybuf.fill_(3.0)
+    sub.forward(X, Y)
+    r0 = S // 2
+    P0, Y0, F0 = theirs["imports"]
+    assert sub.P_addr == [P0, sub.P.data_ptr()] and sub.Y_addr == [Y0, sub.Ybuf.data_ptr()]
+    assert sub.F_addr == [F0, sub.flags.data_ptr()]
+    (rows, parts, X_rows, outs), = seen
+    assert rows == S // 2 and torch.equal(X_rows, X[r0:])
+    assert parts == [P0 + r0 * H * 4, sub.P.data_ptr() + r0 * H * 4]
+    assert outs == [Y0 + r0 * H * 2, sub.Ybuf.data_ptr() + r0 * H * 2]
+    barriers = [c for c in ops.calls if c[0] == "barrier"]
+    assert [b[4] for b in barriers] == [1, 2] and all(b[1:4] == (2, 1, tuple(sub.F_addr)) for b in barriers)
+    assert torch.equal(Y, torch.full((S, H), 3.0, dtype=torch.bfloat16))  # copied from the shared output buffer
+    sub.forward(X, Y)
+    assert [c[4] for c in ops.calls if c[0] == "barrier"] == [1, 2, 3, 4]
+    sub.close()
+    assert sorted(c[1] for c in ops.calls if c[0] == "close") == sorted([P0, Y0, F0])

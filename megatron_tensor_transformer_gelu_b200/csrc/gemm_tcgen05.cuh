@@ -90,6 +90,11 @@ struct GemmCfg {
 #ifndef TP_GEMM_WIDE_STAGES
 #define TP_GEMM_WIDE_STAGES 4
 #endif
+// bf16 epilogue chunks: both 32-column TMEM loads issued before one wait (1),
+// or load-wait-convert per 32 columns (0).
+#ifndef TP_GEMM_EPI_LD64
+#define TP_GEMM_EPI_LD64 0
+#endif
 // Epilogue stores: each epilogue warp issues the TMA store of its own 32 rows
 // (1), or one thread stores all 128 rows after a barrier of the four warps (0).
 #ifndef TP_GEMM_WARP_STORES
@@ -463,11 +468,22 @@ __device__ __forceinline__ void epi_chunk_f32(uint32_t taddr, uint8_t* stage_row
 
 template <int ACT>
 __device__ __forceinline__ void epi_chunk_bf16(uint32_t taddr, uint8_t* stage_row, int row_local) {
+#if TP_GEMM_EPI_LD64
+  // Both 32-column loads in flight before one wait.
+  uint32_t r2[2][32];
+  tmem_ld_32x32b_x32(taddr, r2[0]);
+  tmem_ld_32x32b_x32(taddr + 32, r2[1]);
+  tmem_wait_ld();
+#endif
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
+#if TP_GEMM_EPI_LD64
+    const uint32_t (&r)[32] = r2[h];
+#else
     uint32_t r[32];
     tmem_ld_32x32b_x32(taddr + h * 32, r);
     tmem_wait_ld();
+#endif
 #pragma unroll
     for (int j = 0; j < 4; ++j) {  // 16-byte chunk 4h+j = 8 bf16
       uint4 w;

@@ -50,9 +50,10 @@ constexpr uint32_t IDESC_PV = idesc_bf16_f32(BQ, D, false, true);
 constexpr uint32_t TMEM_COLS = 512;
 constexpr float RESCALE_THRESHOLD = 8.0f;
 #ifndef TP_ATTN_EXP2_POLY_EVERY
-#define TP_ATTN_EXP2_POLY_EVERY 4
+#define TP_ATTN_EXP2_POLY_EVERY 0
 #endif
 constexpr int EXP2_POLY_EVERY = TP_ATTN_EXP2_POLY_EVERY;  // 0: every exponential on the MUFU unit
+constexpr int EXP2_POLY_MOD = EXP2_POLY_EVERY > 0 ? EXP2_POLY_EVERY : 1;
 }  // namespace attn
 
 struct AttnArgs {
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
       uint32_t pk0[32], pk1[32];
 #pragma unroll
       for (int e = 0; e < BKV; e += 2) {
-        const bool poly = EXP2_POLY_EVERY > 0 && (e / 2) % EXP2_POLY_EVERY == EXP2_POLY_EVERY - 1;
+        const bool poly = EXP2_POLY_EVERY > 0 && (e / 2) % EXP2_POLY_MOD == EXP2_POLY_MOD - 1;
         const float x0 = fmaf(s[e], a.scale_log2, -m_run);
         const float x1 = fmaf(s[e + 1], a.scale_log2, -m_run);
         const float p0 = poly ? exp2_poly(x0) : exp2_fast(x0);

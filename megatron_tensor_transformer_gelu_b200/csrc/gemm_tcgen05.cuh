@@ -50,19 +50,19 @@
 // reads both: the attention backward's scores Q K^T and dP = dO V^T for the
 // same block, from which it makes P and dS together (EPI_DUAL_SOFTMAX).
 //
-// Stream-K (sk = 1): instead of whole tiles dealt round-robin to the clusters
-// (the last wave partly idle when the tile count is not a multiple of the
-// cluster count), the k-blocks of all tiles, laid end to end, are cut into
-// one contiguous range per cluster.  A tile whose k-blocks are cut between
-// clusters is summed by the cluster holding its last k-block (the finisher):
-// each other cluster (a producer) stores its f32 partial accumulator to a
-// workspace and publishes a flag; the finisher waits for those flags (bounded
-// wait), adds the partials into its TMEM accumulator and runs the normal
-// epilogue.  Every cluster processes its producer piece first and its
-// finisher piece last, and a finisher waits only on lower-numbered clusters'
-// producer pieces, so no wait can form a cycle; the grid is never larger than
-// the clusters resident at once.  The partials are added in a fixed order, so
-// results are run-to-run repeatable.
+// Stream-K (sk = 1): whole tiles dealt round-robin leave clusters idle in the
+// last wave when the tile count is not a multiple of the cluster count.
+// Here the whole waves stay as they are (concurrently running clusters share
+// their operands in L2), and only the remainder tiles are split along K: the
+// first clusters each run the head of one remainder tile and finish it, and
+// the spare clusters run the remainder tiles' tails, laid end to end and cut
+// evenly (sk_split).  A tail piece (a producer) stores its f32 partial
+// accumulator to a workspace slot and publishes a flag; the head's cluster (the
+// finisher) waits for those flags (bounded wait), adds the partials into its
+// TMEM accumulator and runs the normal epilogue.  Producers never wait and a
+// finisher piece is its cluster's last, so no wait can form a cycle; the grid
+// is never larger than the clusters resident at once.  The partials are added
+// in a fixed order, so results are run-to-run repeatable.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -203,58 +203,108 @@ struct GemmArgs {
 enum : int { EPI_PLAIN = 0, EPI_AUX_PRE = 1, EPI_GRAD = 2, EPI_SOFTMAX = 3, EPI_DSOFTMAX = 4, EPI_DUAL_SOFTMAX = 5 };
 
 // One piece of work of a cluster: the k-blocks [kb0, kb1) of a tile (of K
-// split `split` in the K-split mode), and what its epilogue does with them.
+// split `split` in the K-split mode), and what its epilogue does with them;
+// a stream-K producer piece's partial goes to workspace slot `slot`.
 enum : int { ROLE_FULL = 0, ROLE_PRODUCER = 1, ROLE_FINISHER = 2 };
 struct WorkItem {
-  int tile, split, kb0, kb1, role;
+  int tile, split, kb0, kb1, role, slot;
 };
 
-// Stream-K: cluster c's range of the k-blocks of all tiles laid end to end.
-__device__ __forceinline__ void sk_range(const GemmArgs& p, int c, int nclusters, long long& k0, long long& k1) {
-  const long long total = static_cast<long long>(p.m_blocks) * p.n_blocks * p.k_blocks;
-  k0 = total * c / nclusters;
-  k1 = total * (c + 1) / nclusters;
+// Stream-K split of T tiles of kbt k-blocks over P clusters: W = T / P whole
+// waves of tiles (dealt round-robin, so concurrently running clusters share
+// operands in L2 as in the data-parallel schedule), then the R = T % P
+// remaining tiles split along K: cluster c < R runs k-blocks [0, m) of
+// remainder tile c (and finishes it), and the P - R spare clusters run the
+// tails [m, kbt) of all R remainder tiles, laid end to end and cut into
+// P - R equal ranges (producer pieces).  m = round(R kbt / P) balances the
+// two.  m = 0 when there is no split (R == 0, or m would be 0 or kbt): the
+// remainder tiles are then whole tiles too.
+struct SkSplit {
+  int W, R, m;
+};
+
+__host__ __device__ __forceinline__ SkSplit sk_split(long long T, int kbt, int P) {
+  SkSplit s;
+  s.W = static_cast<int>(T / P);
+  s.R = static_cast<int>(T % P);
+  const long long m = (2LL * s.R * kbt + P) / (2LL * P);
+  s.m = (s.R == 0 || m < 1 || m >= kbt) ? 0 : static_cast<int>(m);
+  return s;
+}
+
+// Spare cluster s's range of the remainder tiles' tail k-blocks laid end to end.
+__device__ __forceinline__ void sk_tail_range(const SkSplit& sp, int kbt, int P, int s, long long& a, long long& b) {
+  const long long tt = static_cast<long long>(sp.R) * (kbt - sp.m);
+  const int spare = P - sp.R;
+  a = tt * s / spare;
+  b = tt * (s + 1) / spare;
 }
 
 __device__ __forceinline__ int num_work_items(const GemmArgs& p, int c, int nclusters) {
+  const int num_tiles = p.m_blocks * p.n_blocks;
   if (!p.sk) {
-    const int units = p.m_blocks * p.n_blocks * p.splits;
+    const int units = num_tiles * p.splits;
     return c < units ? (units - 1 - c) / nclusters + 1 : 0;
   }
-  long long k0, k1;
-  sk_range(p, c, nclusters, k0, k1);
-  if (k1 <= k0) return 0;
-  return static_cast<int>((k1 - 1) / p.k_blocks - k0 / p.k_blocks + 1);
+  const SkSplit sp = sk_split(num_tiles, p.k_blocks, nclusters);
+  if (sp.R == 0) return sp.W;
+  if (sp.m == 0) return sp.W + (c < sp.R ? 1 : 0);
+  if (c < sp.R) return sp.W + 1;
+  long long a, b;
+  sk_tail_range(sp, p.k_blocks, nclusters, c - sp.R, a, b);
+  const int L = p.k_blocks - sp.m;
+  return sp.W + (b > a ? static_cast<int>((b - 1) / L - a / L + 1) : 0);
 }
 
 __device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& kb0, int& kb1);
 
-// The idx-th of cluster c's n work items, in processing order.  Stream-K
-// order: the range's last piece (a producer when it ends inside a tile)
-// first, the whole tiles between, the first piece (a finisher when it starts
-// inside a tile) last.
+// The idx-th of cluster c's n work items, in processing order: its whole
+// tiles first, then its remainder piece (a finisher, last) or its tail
+// pieces (producers).
 __device__ __forceinline__ WorkItem work_item(const GemmArgs& p, int c, int nclusters, int idx, int n) {
   WorkItem w;
+  w.split = 0;
+  w.slot = 0;
+  w.role = ROLE_FULL;
+  const int num_tiles = p.m_blocks * p.n_blocks;
   if (!p.sk) {
-    const int num_tiles = p.m_blocks * p.n_blocks;
     const int unit = c + idx * nclusters;
     w.tile = unit % num_tiles;
     w.split = unit / num_tiles;
     split_range(p, w.split, w.kb0, w.kb1);
-    w.role = ROLE_FULL;
     return w;
   }
-  long long k0, k1;
-  sk_range(p, c, nclusters, k0, k1);
-  const int seg = n == 1 ? 0 : (idx == 0 ? n - 1 : (idx == n - 1 ? 0 : idx));
-  const long long kbt = p.k_blocks;
-  const long long ti = k0 / kbt + seg;
-  const long long ts = ti * kbt;
-  w.tile = static_cast<int>(ti);
-  w.split = 0;
-  w.kb0 = static_cast<int>((k0 > ts ? k0 : ts) - ts);
-  w.kb1 = static_cast<int>((k1 < ts + kbt ? k1 : ts + kbt) - ts);
-  w.role = w.kb1 < kbt ? ROLE_PRODUCER : (w.kb0 > 0 ? ROLE_FINISHER : ROLE_FULL);
+  (void)n;
+  const SkSplit sp = sk_split(num_tiles, p.k_blocks, nclusters);
+  w.kb0 = 0;
+  w.kb1 = p.k_blocks;
+  if (idx < sp.W) {
+    w.tile = c + idx * nclusters;
+    return w;
+  }
+  const int base = sp.W * nclusters;  // first remainder tile
+  if (sp.m == 0) {
+    w.tile = base + c;
+    return w;
+  }
+  if (c < sp.R) {
+    w.tile = base + c;
+    w.kb1 = sp.m;
+    w.role = ROLE_FINISHER;
+    return w;
+  }
+  const int s = c - sp.R;
+  const int L = p.k_blocks - sp.m;
+  long long a, b;
+  sk_tail_range(sp, p.k_blocks, nclusters, s, a, b);
+  const int r = static_cast<int>(a / L) + (idx - sp.W);
+  const long long lo = a > static_cast<long long>(r) * L ? a : static_cast<long long>(r) * L;
+  const long long hi = b < static_cast<long long>(r + 1) * L ? b : static_cast<long long>(r + 1) * L;
+  w.tile = base + r;
+  w.kb0 = sp.m + static_cast<int>(lo - static_cast<long long>(r) * L);
+  w.kb1 = sp.m + static_cast<int>(hi - static_cast<long long>(r) * L);
+  w.role = ROLE_PRODUCER;
+  w.slot = r + s;
   return w;
 }
 
@@ -857,7 +907,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         // block of the workspace (coalesced: float4 chunk j of row l at
         // j * 128 + l), then the TMEM buffer is handed back and the flag
         // published once every thread's stores are visible.
-        float4* dst = reinterpret_cast<float4*>(p.sk_ws + static_cast<long long>(cluster_id * CG + rank) * C::BM *
+        float4* dst = reinterpret_cast<float4*>(p.sk_ws + static_cast<long long>(wi.slot * CG + rank) * C::BM *
                                                               p.tile_n) + row_local;
         for (int c32 = 0; c32 < p.tile_n / 32; ++c32) {
           uint32_t r[32];
@@ -878,46 +928,50 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         }
         __threadfence();
         named_barrier_sync(1, 128);
-        if (elected) flag_publish(p.sk_flags + cluster_id * CG + rank, p.sk_epoch);
+        if (elected) flag_publish(p.sk_flags + wi.slot * CG + rank, p.sk_epoch);
         if (++acc == acc_bufs) { acc = 0; acc_phase ^= 1; }
         continue;
       }
       if (wi.role == ROLE_FINISHER) {
-        // Stream-K finisher piece: wait for every producer of this tile (the
-        // lower-numbered clusters whose ranges reach into it), then add their
-        // partials into the TMEM accumulator, highest cluster first.
-        const long long tile_k0 = static_cast<long long>(wi.tile) * p.k_blocks;
+        // Stream-K finisher piece: wait for every producer piece of this
+        // remainder tile's tail (the spare clusters whose tail ranges meet
+        // it), then add their partials into the TMEM accumulator in the spare
+        // clusters' order.
+        const SkSplit sp = sk_split(static_cast<long long>(p.m_blocks) * p.n_blocks, p.k_blocks, num_clusters);
+        const int r = wi.tile - sp.W * num_clusters;
+        const int L = p.k_blocks - sp.m;
+        const long long t0 = static_cast<long long>(r) * L, t1 = t0 + L;
         if (elected) {
-          for (int pc = cluster_id - 1; pc >= 0; --pc) {
-            long long q0, q1;
-            sk_range(p, pc, num_clusters, q0, q1);
-            if (q1 <= tile_k0) break;
-            if (q1 <= q0) continue;  // an empty range publishes nothing
-            if (!flag_wait_eq(p.sk_flags + pc * CG + rank, p.sk_epoch)) break;
+          for (int sc = 0; sc < num_clusters - sp.R; ++sc) {
+            long long a0, b0;
+            sk_tail_range(sp, p.k_blocks, num_clusters, sc, a0, b0);
+            if (a0 >= t1) break;
+            if (b0 <= t0 || b0 <= a0) continue;
+            if (!flag_wait_eq(p.sk_flags + (r + sc) * CG + rank, p.sk_epoch)) break;
           }
         }
         named_barrier_sync(1, 128);
         for (int c32 = 0; c32 < p.tile_n / 32; ++c32) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(t_row + c32 * 32, r);
+          uint32_t rr[32];
+          tmem_ld_32x32b_x32(t_row + c32 * 32, rr);
           tmem_wait_ld();
-          for (int pc = cluster_id - 1; pc >= 0; --pc) {
-            long long q0, q1;
-            sk_range(p, pc, num_clusters, q0, q1);
-            if (q1 <= tile_k0) break;
-            if (q1 <= q0) continue;
-            const float4* src = reinterpret_cast<const float4*>(p.sk_ws + static_cast<long long>(pc * CG + rank) *
+          for (int sc = 0; sc < num_clusters - sp.R; ++sc) {
+            long long a0, b0;
+            sk_tail_range(sp, p.k_blocks, num_clusters, sc, a0, b0);
+            if (a0 >= t1) break;
+            if (b0 <= t0 || b0 <= a0) continue;
+            const float4* src = reinterpret_cast<const float4*>(p.sk_ws + static_cast<long long>((r + sc) * CG + rank) *
                                                                               C::BM * p.tile_n) + row_local;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-              const float4 a = __ldcg(src + static_cast<long long>(c32 * 8 + j) * C::BM);
-              r[4 * j] = __float_as_uint(__uint_as_float(r[4 * j]) + a.x);
-              r[4 * j + 1] = __float_as_uint(__uint_as_float(r[4 * j + 1]) + a.y);
-              r[4 * j + 2] = __float_as_uint(__uint_as_float(r[4 * j + 2]) + a.z);
-              r[4 * j + 3] = __float_as_uint(__uint_as_float(r[4 * j + 3]) + a.w);
+              const float4 v = __ldcg(src + static_cast<long long>(c32 * 8 + j) * C::BM);
+              rr[4 * j] = __float_as_uint(__uint_as_float(rr[4 * j]) + v.x);
+              rr[4 * j + 1] = __float_as_uint(__uint_as_float(rr[4 * j + 1]) + v.y);
+              rr[4 * j + 2] = __float_as_uint(__uint_as_float(rr[4 * j + 2]) + v.z);
+              rr[4 * j + 3] = __float_as_uint(__uint_as_float(rr[4 * j + 3]) + v.w);
             }
           }
-          tmem_st_32x32b_x32(t_row + c32 * 32, r);
+          tmem_st_32x32b_x32(t_row + c32 * 32, rr);
         }
         tmem_wait_st();
       }

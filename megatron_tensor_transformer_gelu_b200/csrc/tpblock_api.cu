@@ -40,7 +40,7 @@ struct DeviceInfo {
 // The reduce + residual + LayerNorm stages rows in shared memory with bulk
 // copies (1) or loads them into registers (0).
 #ifndef TP_RLN_BULK
-#define TP_RLN_BULK 1
+#define TP_RLN_BULK 0
 #endif
 
 // The attention backward makes P and dS in one dual-accumulator GEMM (1) or in
@@ -334,19 +334,24 @@ TilePlan plan_tiles_dp(const tp::GemmArgs& p, bool pair, int slots, int max_spli
   return best;
 }
 
-// Stream-K: one contiguous range of (tile, k-block) steps per cluster, so the
-// time is the steps per cluster rather than whole waves, plus the exposed
-// epilogue of every piece but the last with wide tiles, plus the fixed cost
-// of the split tiles' partials (a producer's store, its finisher's wait and
-// reads: about 3 us).
+// Stream-K (tp::sk_split): the whole waves as in the data-parallel plan, then
+// the remainder tiles split along K between their head clusters and the spare
+// clusters, so the last wave takes about R kbt / P k-blocks instead of kbt.
+// Plus the exposed epilogue of every piece but the last with wide tiles, plus
+// the fixed cost of the split tiles' partials (the producers' stores, the
+// finishers' wait and reads: about 3 us).
 constexpr double T_SK_FIX = 3.0e-6;
 
 double sk_cost(const tp::GemmArgs& p, bool pair, int clusters, int w) {
   const long long m_blocks = (p.M + (pair ? 255 : 127)) / (pair ? 256 : 128);
   const long long tiles = m_blocks * n_blocks_for(p, w);
-  const long long steps = (tiles * p.k_blocks + clusters - 1) / clusters;
+  const tp::SkSplit sp = tp::sk_split(tiles, p.k_blocks, clusters);
+  const long long last = sp.R == 0 ? 0 : (sp.m == 0 ? p.k_blocks
+                                                      : (static_cast<long long>(sp.R) * p.k_blocks + clusters - 1) /
+                                                            clusters);
+  const long long steps = static_cast<long long>(sp.W) * p.k_blocks + last;
   const double epi_weight = p.epi_mode == tp::EPI_PLAIN ? 1.0 : 2.0;
-  const long long exposed = w > 256 ? (tiles + clusters - 1) / clusters : 0;
+  const long long exposed = w > 256 ? sp.W : 0;
   return static_cast<double>(steps) * kb_cost(w) * T_KB + T_SK_FIX +
          static_cast<double>(exposed) * (w / 256.0) * T_EPI_256 * epi_weight;
 }
@@ -367,7 +372,8 @@ TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits,
     long long clusters = slots;
     while (clusters >= 2 && sk_bytes(clusters, cg, best.tile_n) > sk_area) --clusters;
     const long long steps = m_blocks * n_blocks_for(p, best.tile_n) * p.k_blocks;
-    if (clusters >= 2 && steps >= clusters) {
+    if (clusters >= 2 && steps >= clusters &&
+        tp::sk_split(m_blocks * n_blocks_for(p, best.tile_n), p.k_blocks, static_cast<int>(clusters)).m > 0) {
       best.stream_k = 1;
       best.sk_clusters = static_cast<int>(clusters);
       best.splits = 1;
@@ -377,7 +383,8 @@ TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits,
   if (g_force_tile_n || best.tile_n == 128) return best;  // a forced width, or narrow shards: as planned
   for (int w = 256; w <= (pair ? 512 : 256); w += step) {
     if (sk_bytes(slots, cg, w) > sk_area) continue;
-    if (m_blocks * n_blocks_for(p, w) * p.k_blocks < 4LL * slots) continue;  // too little work to split
+    const tp::SkSplit sp = tp::sk_split(m_blocks * n_blocks_for(p, w), p.k_blocks, slots);
+    if (sp.m == 0) continue;  // no remainder to split: the data-parallel plan is the same
     const double t = sk_cost(p, pair, slots, w);
     if (t < best_t * 0.98) {
       best_t = t;
@@ -804,14 +811,10 @@ int run_ln_backward(int S, int H, const float* V, const void* X, const void* dY,
   if (grid > LNB_MAX_CTAS) grid = LNB_MAX_CTAS;
   if (grid > S) grid = S;
   if (grid < 1) grid = 1;
-#if TP_RLN_BULK
   // Rows staged in shared memory by bulk copies (X, dY, V: 8 bytes a column),
   // 2 to 4 stages; rows too wide for two stages take the register kernel.
   const size_t stage = (static_cast<size_t>(H) * 8 + 127) & ~size_t(127);
-  const bool bulk = 2 * stage <= static_cast<size_t>(tp::rlb::MAX_STAGE_SMEM);
-#else
-  const bool bulk = false;
-#endif
+  const bool bulk = TP_RLN_BULK && 2 * stage <= static_cast<size_t>(tp::rlb::MAX_STAGE_SMEM);
   if (bulk) {
     const size_t budget = stage <= 32 * 1024 ? 96 * 1024 : tp::rlb::MAX_STAGE_SMEM;
     int nst = static_cast<int>(budget / stage);

@@ -90,10 +90,11 @@ def test_bad_arguments():
 
 
 # With the sublayers' spare partial-sum slots (3 x S x H x 4 bytes) as stream-K
-# scratch: (tile_n, splits, stream_k, pairs).  Stream-K wins where whole-tile
-# waves leave pairs idle: 64 or 128 tiles of 512 columns on 74 pairs, 256 or
-# 384 in 3.46 / 5.19 waves.  The large MLP's first GEMM (1536 tiles, 20.75
-# waves) gains under 2 % and keeps whole tiles.
+# scratch: (tile_n, splits, stream_k, pairs).  Stream-K (whole waves, then the
+# remainder tiles split along K) wins where the last wave leaves pairs idle:
+# 64 or 128 tiles of 512 columns on 74 pairs, 256 or 384 in 3.46 / 5.19 waves.
+# The large MLP's first GEMM (1536 tiles, 20.75 waves) gains under 2 % and
+# keeps whole tiles.
 SK_CASES = [
     ("mlp GEMM1", 2048, 4, 0, 4096, 4096, 0, 1, 2048 * 4096, (512, 1, 1, 74)),
     ("mlp GEMM2", 2048, 4, 1, 4096, 4096, 1, 4, 2048 * 4096, (512, 1, 1, 74)),
@@ -119,10 +120,13 @@ def test_stream_k_switch():
         # forced: as many pairs as the scratch holds 256 x 256 f32 blocks for (+ one flag each)
         L.set_gemm_stream_k(1)
         area = 10 * 2 * 128 * 256 * 4 + 256 + 10 * 2 * 8
-        tn, sp, on, pairs = L.gemm_plan_sk(600, 2, 0, 520, 1120, 0, sk_area_bytes=area)
+        # 3 x 8 = 24 tiles on 10 pairs: 2 whole waves, 4 remainder tiles split
+        tn, sp, on, pairs = L.gemm_plan_sk(600, 2, 0, 520, 1000, 0, sk_area_bytes=area)
         assert (tn, sp, on, pairs) == (256, 1, 1, 10)
+        # 3 x 10 = 30 tiles on 10 pairs: whole waves only, nothing to split
+        assert L.gemm_plan_sk(600, 2, 0, 520, 1120, 0, sk_area_bytes=area)[2] == 0
         # no scratch, no stream-K
-        assert L.gemm_plan_sk(600, 2, 0, 520, 1120, 0, sk_area_bytes=0)[2] == 0
+        assert L.gemm_plan_sk(600, 2, 0, 520, 1000, 0, sk_area_bytes=0)[2] == 0
         with pytest.raises(L.TPError):
             L.set_gemm_stream_k(2)
     finally:

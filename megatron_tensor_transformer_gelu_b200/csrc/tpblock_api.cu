@@ -49,6 +49,12 @@ struct DeviceInfo {
 #define TP_ATTN_BACK_DUAL 1
 #endif
 
+// Rows of 2049..4096 columns: 8 warps a row with 16 values a lane (0), or 16
+// warps a row with 8 values a lane (1).
+#ifndef TP_RLN_WIDE_ROWS
+#define TP_RLN_WIDE_ROWS 0
+#endif
+
 // Most K-split partial-sum slots a row-split GEMM feeding the LayerNorm may use.
 #define TP_MAX_K_SPLITS 4
 
@@ -726,7 +732,12 @@ int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, i
   if (H <= 512) np1 ? go(reduce_residual_ln_kernel<1, 2, true>, 1, 8) : go(reduce_residual_ln_kernel<1, 2, false>, 1, 8);
   else if (H <= 1024) np1 ? go(reduce_residual_ln_kernel<2, 2, true>, 2, 4) : go(reduce_residual_ln_kernel<2, 2, false>, 2, 4);
   else if (H <= 2048) np1 ? go(reduce_residual_ln_kernel<4, 2, true>, 4, 2) : go(reduce_residual_ln_kernel<4, 2, false>, 4, 2);
+#if TP_RLN_WIDE_ROWS
+  // one 512-thread CTA per row, 8 values per lane: fewer registers, more CTAs per SM
+  else if (H <= 4096) np1 ? go(reduce_residual_ln_kernel<16, 1, true>, 16, 1) : go(reduce_residual_ln_kernel<16, 1, false>, 16, 1);
+#else
   else if (H <= 4096) np1 ? go(reduce_residual_ln_kernel<8, 2, true>, 8, 1) : go(reduce_residual_ln_kernel<8, 2, false>, 8, 1);
+#endif
   else if (H <= 8192) np1 ? go(reduce_residual_ln_kernel<8, 4, true>, 8, 1) : go(reduce_residual_ln_kernel<8, 4, false>, 8, 1);
   // (one-row CTAs of 12 or 16 warps keep the generic loop: fewer registers, two CTAs per SM)
   else if (H <= 12288) go(reduce_residual_ln_kernel<12, 4, false>, 12, 1);

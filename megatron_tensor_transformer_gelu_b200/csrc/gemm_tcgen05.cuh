@@ -223,13 +223,40 @@ struct SkSplit {
   int W, R, m;
 };
 
+// The head takes SK_HEAD_EXTRA k-blocks more than the even share: a spare
+// cluster's pieces each pay a partial-sum store and a pipeline restart.
+constexpr int SK_HEAD_EXTRA = 3;
+// Most producer pieces one remainder tile's tail may have (host plans that
+// would exceed it keep whole tiles).
+constexpr int SK_MAX_PRODUCERS = 16;
+
 __host__ __device__ __forceinline__ SkSplit sk_split(long long T, int kbt, int P) {
   SkSplit s;
   s.W = static_cast<int>(T / P);
   s.R = static_cast<int>(T % P);
-  const long long m = (2LL * s.R * kbt + P) / (2LL * P);
+  const long long m = (2LL * s.R * kbt + P) / (2LL * P) + SK_HEAD_EXTRA;
   s.m = (s.R == 0 || m < 1 || m >= kbt) ? 0 : static_cast<int>(m);
   return s;
+}
+
+// The spare clusters whose tail ranges meet remainder tile r's tail
+// [r L, (r+1) L) (L = kbt - m): written to list[0..n), in order; n <= max.
+__host__ __device__ __forceinline__ int sk_producers(const SkSplit& sp, int kbt, int P, int r, int* list, int max) {
+  const long long L = kbt - sp.m;
+  const long long tt = static_cast<long long>(sp.R) * L;
+  const long long spare = P - sp.R;
+  const long long t0 = r * L, t1 = t0 + L;
+  // first s with end > t0, last s with start < t1 (ends/starts floor(tt s / spare))
+  long long s_lo = ((t0 + 1) * spare + tt - 1) / tt - 1;
+  long long s_hi = (t1 * spare + tt - 1) / tt - 1;
+  if (s_lo < 0) s_lo = 0;
+  if (s_hi > spare - 1) s_hi = spare - 1;
+  int n = 0;
+  for (long long sc = s_lo; sc <= s_hi && n < max; ++sc) {
+    const long long a = tt * sc / spare, b = tt * (sc + 1) / spare;
+    if (b > a && a < t1 && b > t0) list[n++] = static_cast<int>(sc);
+  }
+  return n;
 }
 
 // Spare cluster s's range of the remainder tiles' tail k-blocks laid end to end.
@@ -935,33 +962,25 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       if (wi.role == ROLE_FINISHER) {
         // Stream-K finisher piece: wait for every producer piece of this
         // remainder tile's tail (the spare clusters whose tail ranges meet
-        // it), then add their partials into the TMEM accumulator in the spare
-        // clusters' order.
+        // it, listed once), then add their partials into the TMEM accumulator
+        // in the spare clusters' order.
         const SkSplit sp = sk_split(static_cast<long long>(p.m_blocks) * p.n_blocks, p.k_blocks, num_clusters);
         const int r = wi.tile - sp.W * num_clusters;
-        const int L = p.k_blocks - sp.m;
-        const long long t0 = static_cast<long long>(r) * L, t1 = t0 + L;
+        int prod[SK_MAX_PRODUCERS];
+        const int nprod = sk_producers(sp, p.k_blocks, num_clusters, r, prod, SK_MAX_PRODUCERS);
         if (elected) {
-          for (int sc = 0; sc < num_clusters - sp.R; ++sc) {
-            long long a0, b0;
-            sk_tail_range(sp, p.k_blocks, num_clusters, sc, a0, b0);
-            if (a0 >= t1) break;
-            if (b0 <= t0 || b0 <= a0) continue;
-            if (!flag_wait_eq(p.sk_flags + (r + sc) * CG + rank, p.sk_epoch)) break;
-          }
+          for (int i = 0; i < nprod; ++i)
+            if (!flag_wait_eq(p.sk_flags + (r + prod[i]) * CG + rank, p.sk_epoch)) break;
         }
         named_barrier_sync(1, 128);
         for (int c32 = 0; c32 < p.tile_n / 32; ++c32) {
           uint32_t rr[32];
           tmem_ld_32x32b_x32(t_row + c32 * 32, rr);
           tmem_wait_ld();
-          for (int sc = 0; sc < num_clusters - sp.R; ++sc) {
-            long long a0, b0;
-            sk_tail_range(sp, p.k_blocks, num_clusters, sc, a0, b0);
-            if (a0 >= t1) break;
-            if (b0 <= t0 || b0 <= a0) continue;
-            const float4* src = reinterpret_cast<const float4*>(p.sk_ws + static_cast<long long>((r + sc) * CG + rank) *
-                                                                              C::BM * p.tile_n) + row_local;
+          for (int i = 0; i < nprod; ++i) {
+            const float4* src = reinterpret_cast<const float4*>(
+                                    p.sk_ws + static_cast<long long>((r + prod[i]) * CG + rank) * C::BM * p.tile_n) +
+                                row_local;
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
               const float4 v = __ldcg(src + static_cast<long long>(c32 * 8 + j) * C::BM);

@@ -248,6 +248,17 @@ struct TilePlan {
 
 // Workspace a stream-K launch needs: a 128 x w f32 partial block per CTA of
 // each of `clusters` clusters of cg CTAs, then one 8-byte flag per CTA.
+// A stream-K split is usable when no remainder tile's tail has more producer
+// pieces than a finisher lists (tp::SK_MAX_PRODUCERS).
+bool sk_split_ok(long long tiles, int kbt, int clusters) {
+  const tp::SkSplit sp = tp::sk_split(tiles, kbt, clusters);
+  if (sp.m == 0) return false;
+  int list[tp::SK_MAX_PRODUCERS + 1];
+  for (int r = 0; r < sp.R; ++r)
+    if (tp::sk_producers(sp, kbt, clusters, r, list, tp::SK_MAX_PRODUCERS + 1) > tp::SK_MAX_PRODUCERS) return false;
+  return true;
+}
+
 size_t sk_bytes(long long clusters, int cg, int w) {
   return align256(static_cast<size_t>(clusters) * cg * 128 * w * 4) + static_cast<size_t>(clusters) * cg * 8;
 }
@@ -352,9 +363,7 @@ double sk_cost(const tp::GemmArgs& p, bool pair, int clusters, int w) {
   const long long m_blocks = (p.M + (pair ? 255 : 127)) / (pair ? 256 : 128);
   const long long tiles = m_blocks * n_blocks_for(p, w);
   const tp::SkSplit sp = tp::sk_split(tiles, p.k_blocks, clusters);
-  const long long last = sp.R == 0 ? 0 : (sp.m == 0 ? p.k_blocks
-                                                      : (static_cast<long long>(sp.R) * p.k_blocks + clusters - 1) /
-                                                            clusters);
+  const long long last = sp.R == 0 ? 0 : (sp.m == 0 ? p.k_blocks : sp.m);
   const long long steps = static_cast<long long>(sp.W) * p.k_blocks + last;
   const double epi_weight = p.epi_mode == tp::EPI_PLAIN ? 1.0 : 2.0;
   const long long exposed = w > 256 ? sp.W : 0;
@@ -379,7 +388,7 @@ TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits,
     while (clusters >= 2 && sk_bytes(clusters, cg, best.tile_n) > sk_area) --clusters;
     const long long steps = m_blocks * n_blocks_for(p, best.tile_n) * p.k_blocks;
     if (clusters >= 2 && steps >= clusters &&
-        tp::sk_split(m_blocks * n_blocks_for(p, best.tile_n), p.k_blocks, static_cast<int>(clusters)).m > 0) {
+        sk_split_ok(m_blocks * n_blocks_for(p, best.tile_n), p.k_blocks, static_cast<int>(clusters))) {
       best.stream_k = 1;
       best.sk_clusters = static_cast<int>(clusters);
       best.splits = 1;
@@ -389,8 +398,7 @@ TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits,
   if (g_force_tile_n || best.tile_n == 128) return best;  // a forced width, or narrow shards: as planned
   for (int w = 256; w <= (pair ? 512 : 256); w += step) {
     if (sk_bytes(slots, cg, w) > sk_area) continue;
-    const tp::SkSplit sp = tp::sk_split(m_blocks * n_blocks_for(p, w), p.k_blocks, slots);
-    if (sp.m == 0) continue;  // no remainder to split: the data-parallel plan is the same
+    if (!sk_split_ok(m_blocks * n_blocks_for(p, w), p.k_blocks, slots)) continue;  // nothing (usable) to split
     const double t = sk_cost(p, pair, slots, w);
     if (t < best_t * 0.98) {
       best_t = t;

@@ -100,6 +100,8 @@ class TPSublayer:
         mine = (self.ops.export(self.P), self.ops.export(self.Ybuf), self.ops.export(self.flags))
         if exchange is None:
             def exchange(obj):
+                if self.world == 1:
+                    return [obj]
                 out = [None] * self.world
                 dist.all_gather_object(out, obj, group=self.group)
                 return out

@@ -44,7 +44,7 @@ def _mlp(inp, t, Y, ws, gamma=None, beta=None):
 
 
 @pytest.mark.parametrize("tile_n", [0, 256, 384, 512, 128])
-@pytest.mark.parametrize("S,H,F,t", [(600, 520, 2240, 2), (384, 1024, 4096, 4), (300, 264, 1200, 3),
+@pytest.mark.parametrize("S,H,F,t", [(600, 520, 2240, 2), (384, 1024, 4096, 4), (300, 640, 1200, 3),
                                      (1000, 768, 3072, 8)])
 def test_mlp_stream_k_matches_oracle_and_whole_tiles(cuda_device, sk_mode, tile_n, S, H, F, t):
     inp = synth.gen_mlp(S, H, F, seed=S + t)

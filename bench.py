@@ -78,9 +78,9 @@ def parse():
     ap.add_argument("--sustained-seconds", type=float, default=3.0,
                     help="length of the back-to-back headline run (0: skip)")
     ap.add_argument("--no-other-workloads", action="store_true")
-    ap.add_argument("--stream-k", choices=["auto", "on", "off"], default="auto",
-                    help="GEMM scheduling: the library's cost model (auto), stream-K wherever a GEMM has scratch "
-                         "for it (on), whole-tile waves only (off)")
+    ap.add_argument("--stream-k", choices=["off", "on", "model"], default="off",
+                    help="GEMM scheduling: whole-tile waves only (off, the library's default), stream-K wherever "
+                         "a GEMM has scratch for it (on), the library's cost model (model)")
     ap.add_argument("--tp", choices=["none", "allreduce", "rs_ag"], default="none",
                     help="split the sublayer over the GPUs (tensor parallelism across ranks, strong scaling) "
                          "instead of running one replica per GPU")
@@ -479,7 +479,7 @@ def run_ours(args, rank, world, local):
     if world > 1:
         dist.barrier()
     L.lib()  # load the CUDA library (raises if it is not built)
-    L.set_gemm_stream_k({"auto": 0, "on": 1, "off": -1}[args.stream_k])
+    L.set_gemm_stream_k({"off": 0, "on": 1, "model": 2}[args.stream_k])
     tp_mode = args.tp != "none"
     P = TPProblem(w, dev, rank, world, args.tp, L, synth, torch) if tp_mode else Problem(w, dev, rank, L, synth, torch)
     X, Y = P.X, P.Y
@@ -611,7 +611,7 @@ def run_ours(args, rank, world, local):
                 cfg[key] = getattr(w, key)
         if w.kind in ("mlp", "mlp_train"):
             cfg["act"] = "gelu_tanh"
-        if args.stream_k != "auto":
+        if args.stream_k != "off":
             cfg["stream_k"] = args.stream_k
         result = {
             "metric": metric_for(w),

@@ -418,8 +418,8 @@ def gemm_plan(M, t, row_mode, shard_k, shard_n, out_f32, b_kmajor=False, heavy_e
 
 
 def set_gemm_stream_k(mode: int) -> None:
-    """0: the cost model decides per GEMM launch; 1: stream-K wherever a
-    launch has scratch for it; -1: never."""
+    """0: whole tiles only (the default); 1: stream-K wherever a launch has
+    scratch for it; 2: the cost model decides per GEMM launch."""
     _check(lib().tp_set_gemm_stream_k(int(mode)), "tp_set_gemm_stream_k")
 
 

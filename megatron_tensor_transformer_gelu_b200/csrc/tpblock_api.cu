@@ -67,7 +67,7 @@ struct DeviceInfo {
 std::mutex g_mu;
 DeviceInfo g_dev[MAX_DEVICES];
 int g_force_tile_n = 0;  // tp_set_gemm_tile_n: 0 = cost model
-int g_stream_k = 0;      // tp_set_gemm_stream_k: 0 = cost model, 1 = wherever a workspace allows, -1 = never
+int g_stream_k = 0;      // tp_set_gemm_stream_k: 0 = whole tiles, 1 = wherever a workspace allows, 2 = cost model
 unsigned long long g_sk_epoch = 0;  // last stream-K launch's epoch (see next_sk_epoch)
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
@@ -377,11 +377,11 @@ double sk_cost(const tp::GemmArgs& p, bool pair, int clusters, int w) {
 TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits, size_t sk_area = 0) {
   double best_t = 0.0;
   TilePlan best = plan_tiles_dp(p, pair, slots, max_splits, &best_t);
-  if (g_stream_k < 0 || sk_area == 0 || p.epi_mode != tp::EPI_PLAIN) return best;
+  if (g_stream_k == 0 || sk_area == 0 || p.epi_mode != tp::EPI_PLAIN) return best;
   const int cg = pair ? 2 : 1;
   const int step = p.out_f32 ? 32 : 64;
   const long long m_blocks = (p.M + (pair ? 255 : 127)) / (pair ? 256 : 128);
-  if (g_stream_k > 0) {
+  if (g_stream_k == 1) {
     // Forced (tests): the data-parallel plan's width (or the forced width),
     // over as many clusters as the workspace holds partial blocks for.
     long long clusters = slots;
@@ -1917,7 +1917,7 @@ int tp_set_gemm_tile_n(int tile_n) {
 }
 
 int tp_set_gemm_stream_k(int mode) {
-  if (mode < -1 || mode > 1) return TP_ERR_INVALID_ARG;
+  if (mode < 0 || mode > 2) return TP_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lk(g_mu);
   g_stream_k = mode;
   return TP_OK;

@@ -70,7 +70,7 @@ def test_mlp_stream_k_matches_oracle_and_whole_tiles(cuda_device, sk_mode, tile_
     assert torch.equal(Ys[0], Ys[1]), "stream-K results differ between runs"
     ref = O.mlp_block(inp.X, inp.A, inp.B, gamma=gamma, beta=beta)
     assert rel_err(Ys[0], ref) <= TOL
-    sk_mode(-1)
+    sk_mode(0)
     Yw = torch.empty(S, H, dtype=torch.bfloat16, device="cuda")
     _mlp(inp, t, Yw, ws, gamma.cuda(), beta.cuda())
     assert rel_err(Yw, ref) <= TOL

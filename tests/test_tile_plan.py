@@ -110,12 +110,17 @@ SK_CASES = [
 @pytest.mark.parametrize("case", SK_CASES, ids=[c[0] for c in SK_CASES])
 def test_stream_k_plan_of_workload_gemms(case):
     _, M, t, row, sk, sn, f32, ms, sh, want = case
-    assert L.gemm_plan_sk(M, t, row, sk, sn, f32, max_splits=ms, sk_area_bytes=3 * sh * 4) == want
+    try:
+        L.set_gemm_stream_k(2)  # the cost model (stream-K is off by default)
+        assert L.gemm_plan_sk(M, t, row, sk, sn, f32, max_splits=ms, sk_area_bytes=3 * sh * 4) == want
+    finally:
+        L.set_gemm_stream_k(0)
 
 
 def test_stream_k_switch():
     try:
-        L.set_gemm_stream_k(-1)
+        # the default: whole tiles even with scratch
+        L.set_gemm_stream_k(0)
         assert L.gemm_plan_sk(2048, 4, 1, 4096, 4096, 1, max_splits=4, sk_area_bytes=3 * 2048 * 4096 * 4)[2] == 0
         # forced: as many pairs as the scratch holds 256 x 256 f32 blocks for (+ one flag each)
         L.set_gemm_stream_k(1)
@@ -128,6 +133,6 @@ def test_stream_k_switch():
         # no scratch, no stream-K
         assert L.gemm_plan_sk(600, 2, 0, 520, 1000, 0, sk_area_bytes=0)[2] == 0
         with pytest.raises(L.TPError):
-            L.set_gemm_stream_k(2)
+            L.set_gemm_stream_k(3)
     finally:
         L.set_gemm_stream_k(0)

@@ -21,6 +21,12 @@
 
 namespace tp {
 
+// Single-partial rows: load X and the partial of every chunk before the first
+// add (0), or add each chunk's partial as it arrives (1, fewer registers).
+#ifndef TP_RLN_LEAN
+#define TP_RLN_LEAN 0
+#endif
+
 namespace rln {
 constexpr int THREADS = 256;       // 8 warps per CTA (up to 8 warps per row)
 constexpr int MAX_WPR = 16;        // warps per row (CTAs grow to 16 warps)
@@ -116,7 +122,8 @@ __device__ __forceinline__ void store8(const ReduceLnArgs& p, long long off, con
 // row.  NP1 specialises the common single partial so that every load of a row
 // is issued before its first add.
 template <int WPR, int CH, bool NP1>
-__global__ void __launch_bounds__(rln::cta_threads(WPR)) reduce_residual_ln_kernel(const ReduceLnArgs p) {
+__global__ void __launch_bounds__(rln::cta_threads(WPR), (TP_RLN_LEAN && rln::cta_threads(WPR) == 256) ? 5 : 1)
+    reduce_residual_ln_kernel(const ReduceLnArgs p) {
   constexpr int RPC = WPR > 8 ? 1 : rln::THREADS / 32 / WPR;  // rows per CTA
   __shared__ float red[2][RPC][WPR];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -130,6 +137,22 @@ __global__ void __launch_bounds__(rln::cta_threads(WPR)) reduce_residual_ln_kern
     const long long base = row * p.H;
     float v[CH][8];
     if (NP1) {
+#if TP_RLN_LEAN
+      // each chunk's partial added as it arrives: fewer live registers, more
+      // CTAs resident per SM
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int col = ((c * WPR + wr) * 32 + lane) * 8;
+        if (live && col < p.H) {
+          float w[8];
+          if (p.x_bf16) load8_bf16(static_cast<const __nv_bfloat16*>(p.X) + base + col, v[c]);
+          else load8_f32(static_cast<const float*>(p.X) + base + col, v[c]);
+          load8_f32(p.parts + base + col, w);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[c][e] += w[e];
+        }
+      }
+#else
       float w[CH][8];
 #pragma unroll
       for (int c = 0; c < CH; ++c) {
@@ -144,6 +167,7 @@ __global__ void __launch_bounds__(rln::cta_threads(WPR)) reduce_residual_ln_kern
       for (int c = 0; c < CH; ++c)
 #pragma unroll
         for (int e = 0; e < 8; ++e) v[c][e] += w[c][e];
+#endif
     } else {
 #pragma unroll
       for (int c = 0; c < CH; ++c) {

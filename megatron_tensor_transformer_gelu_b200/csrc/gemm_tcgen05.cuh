@@ -75,6 +75,11 @@ constexpr int MAX_SHARDS = 8;
 
 enum : int { ACT_NONE = 0, ACT_GELU_TANH = 1, ACT_GELU_ERF = 2, ACT_RELU = 3 };
 
+// Kernel features, each compiled into its own instantiation so that the
+// plain GEMM's loops carry none of the others' code: FEAT_BASE (whole tiles),
+// FEAT_SK (stream-K), FEAT_DUAL (dual accumulators).
+enum : int { FEAT_BASE = 0, FEAT_SK = 1, FEAT_DUAL = 2 };
+
 template <int CG, bool WIDE = false>
 struct GemmCfg {
   static constexpr int BM = 128;                    // accumulator rows per CTA
@@ -267,9 +272,10 @@ __device__ __forceinline__ void sk_tail_range(const SkSplit& sp, int kbt, int P,
   b = tt * (s + 1) / spare;
 }
 
+template <int FEAT>
 __device__ __forceinline__ int num_work_items(const GemmArgs& p, int c, int nclusters) {
   const int num_tiles = p.m_blocks * p.n_blocks;
-  if (!p.sk) {
+  if constexpr (FEAT != FEAT_SK) {
     const int units = num_tiles * p.splits;
     return c < units ? (units - 1 - c) / nclusters + 1 : 0;
   }
@@ -288,13 +294,14 @@ __device__ __forceinline__ void split_range(const GemmArgs& p, int split, int& k
 // The idx-th of cluster c's n work items, in processing order: its whole
 // tiles first, then its remainder piece (a finisher, last) or its tail
 // pieces (producers).
+template <int FEAT>
 __device__ __forceinline__ WorkItem work_item(const GemmArgs& p, int c, int nclusters, int idx, int n) {
   WorkItem w;
   w.split = 0;
   w.slot = 0;
   w.role = ROLE_FULL;
   const int num_tiles = p.m_blocks * p.n_blocks;
-  if (!p.sk) {
+  if constexpr (FEAT != FEAT_SK) {
     const int unit = c + idx * nclusters;
     w.tile = unit % num_tiles;
     w.split = unit / num_tiles;
@@ -609,10 +616,11 @@ __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& p, int tile) {
 }
 
 // Shard, A column and B row of k-block kb.
+template <int FEAT = FEAT_BASE>
 __device__ __forceinline__ void kblock_coords(const GemmArgs& p, const TileCoord& tc, int kb, int& shard, int& a_x,
                                               int& b_y) {
   constexpr int BK = 64;
-  if (p.dual) {  // k-blocks [k/2, k) are the second product's, from its own k = 0
+  if (FEAT == FEAT_DUAL) {  // k-blocks [k/2, k) are the second product's, from its own k = 0
     const int half = p.k_blocks / 2;
     shard = tc.shard;
     b_y = (kb < half ? kb : kb - half) * BK;
@@ -672,7 +680,7 @@ __device__ __forceinline__ int b2_boxes_for(int n_valid, int n2, int rank, int b
   return (cols + C::B_BOX_N - 1) / C::B_BOX_N;
 }
 
-template <int CG, bool WIDE = false>
+template <int CG, bool WIDE = false, int FEAT = FEAT_BASE>
 __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kernel(const __grid_constant__ GemmArgs p) {
   using C = GemmCfg<CG, WIDE>;
   constexpr int STAGES = C::STAGES;
@@ -730,7 +738,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
   const bool narrow = narrow_tiles<WIDE>(p);
   const int cluster_id = blockIdx.x / CG;
   const int num_clusters = gridDim.x / CG;
-  const int num_items = num_work_items(p, cluster_id, num_clusters);
+  const int num_items = num_work_items<FEAT>(p, cluster_id, num_clusters);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -742,7 +750,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) armed[s] = -1;
       for (int idx = 0; idx < num_items && ok; ++idx) {
-        const WorkItem wi = work_item(p, cluster_id, num_clusters, idx, num_items);
+        const WorkItem wi = work_item<FEAT>(p, cluster_id, num_clusters, idx, num_items);
         const int kb_begin = wi.kb0, kb_end = wi.kb1;
         const TileCoord tc = tile_coord<CG>(p, wi.tile);
         const CUtensorMap* mA = &p.tmA[p.a_per_shard ? tc.shard : 0];
@@ -763,18 +771,21 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
             const int kp = kb + C::PREFETCH;
             if (kp < kb_end && !p.a_mnmajor) {
               int ps, pa, pb;
-              kblock_coords(p, tc, kp, ps, pa, pb);
-              if (my_a) tma_prefetch_l2_2d(mA, pa, my_row0);
-              for (int j = 0; j < my_boxes; ++j) tma_prefetch_l2_2d(&p.tmB[ps], b_x0 + j * C::B_BOX_N, pb);
+              kblock_coords<FEAT>(p, tc, kp, ps, pa, pb);
+              const bool second = FEAT == FEAT_DUAL && kp >= p.k_blocks / 2;
+              const CUtensorMap* pA = second ? &p.tmA2[p.a_per_shard ? tc.shard : 0] : mA;
+              const CUtensorMap* pB = second ? &p.tmB2[ps] : &p.tmB[ps];
+              if (my_a) tma_prefetch_l2_2d(pA, pa, my_row0);
+              for (int j = 0; j < my_boxes; ++j) tma_prefetch_l2_2d(pB, b_x0 + j * C::B_BOX_N, pb);
             }
           }
           if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
           int shard, a_x, b_y;
-          kblock_coords(p, tc, kb, shard, a_x, b_y);
+          kblock_coords<FEAT>(p, tc, kb, shard, a_x, b_y);
           uint8_t* dA = sA + stage * C::A_BYTES;
           uint8_t* dB = sB + stage * C::B_BYTES;
           // Dual accumulators: the second half of the k-blocks is the second product's.
-          const bool second = p.dual && kb >= p.k_blocks / 2;
+          const bool second = FEAT == FEAT_DUAL && kb >= p.k_blocks / 2;
           const CUtensorMap* mAk = second ? &p.tmA2[p.a_per_shard ? tc.shard : 0] : mA;
           const CUtensorMap* mBk = second ? &p.tmB2[shard] : &p.tmB[shard];
           if constexpr (CG == 1) {
@@ -841,9 +852,9 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      const int acc_bufs = p.dual ? 1 : C::ACC_BUFS;  // dual: both 256-column halves per tile
+      constexpr int acc_bufs = FEAT == FEAT_DUAL ? 1 : C::ACC_BUFS;  // dual: both 256-column halves per tile
       for (int idx = 0; idx < num_items && ok; ++idx) {
-        const WorkItem wi = work_item(p, cluster_id, num_clusters, idx, num_items);
+        const WorkItem wi = work_item<FEAT>(p, cluster_id, num_clusters, idx, num_items);
         const int kb_begin = wi.kb0, kb_end = wi.kb1;
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1)) { ok = false; break; }
         tc_fence_after();
@@ -868,9 +879,13 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
             // B K-major: like A.
             const uint64_t bd = p.b_kmajor ? sdesc_sw128(b0 + kk * 32, 16, 1024)
                                            : sdesc_sw128(b0 + kk * 2048, C::B_BOX_BYTES, 1024);
-            const bool second = p.dual && kb >= p.k_blocks / 2;
-            const uint32_t accum = ((kb != kb_begin && !(p.dual && kb == p.k_blocks / 2)) || kk != 0) ? 1u : 0u;
-            const uint32_t dt = d_tmem + (second ? static_cast<uint32_t>(C::BN) : 0u);
+            uint32_t accum = (kb != kb_begin || kk != 0) ? 1u : 0u;
+            uint32_t dt = d_tmem;
+            if constexpr (FEAT == FEAT_DUAL) {
+              const bool second = kb >= p.k_blocks / 2;
+              if (kb == p.k_blocks / 2 && kk == 0) accum = 0u;  // the second product starts its own sum
+              if (second) dt += static_cast<uint32_t>(C::BN);
+            }
             if constexpr (CG == 1) umma_bf16(dt, ad, bd, idesc, accum);
             else umma_bf16_pair(dt, ad, bd, idesc, accum);
             if constexpr (WIDE) {
@@ -914,9 +929,9 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
     uint32_t acc_phase = 0;
     int buf = 0;
     const uint32_t tempty_leader0 = CG == 2 ? mapa_shared(smem_u32(&tempty[0]), 0) : 0u;
-    const int acc_bufs = p.dual ? 1 : C::ACC_BUFS;
+    constexpr int acc_bufs = FEAT == FEAT_DUAL ? 1 : C::ACC_BUFS;
     for (int idx = 0; idx < num_items; ++idx) {
-      const WorkItem wi = work_item(p, cluster_id, num_clusters, idx, num_items);
+      const WorkItem wi = work_item<FEAT>(p, cluster_id, num_clusters, idx, num_items);
       const TileCoord tc = tile_coord<CG>(p, wi.tile);
       const int split = wi.split;
       const int y0 = tc.m0 + static_cast<int>(rank) * C::BM;
@@ -929,7 +944,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       if (!named_barrier_and(1, 128, mbar_wait(&tfull[acc], acc_phase))) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * C::BN);
-      if (wi.role == ROLE_PRODUCER) {
+      if (FEAT == FEAT_SK && wi.role == ROLE_PRODUCER) {
         // Stream-K producer piece: the raw f32 accumulator goes to this CTA's
         // block of the workspace (coalesced: float4 chunk j of row l at
         // j * 128 + l), then the TMEM buffer is handed back and the flag
@@ -959,7 +974,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
         if (++acc == acc_bufs) { acc = 0; acc_phase ^= 1; }
         continue;
       }
-      if (wi.role == ROLE_FINISHER) {
+      if (FEAT == FEAT_SK && wi.role == ROLE_FINISHER) {
         // Stream-K finisher piece: wait for every producer piece of this
         // remainder tile's tail (the spare clusters whose tail ranges meet
         // it, listed once), then add their partials into the TMEM accumulator
@@ -1000,7 +1015,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       const float rv = (p.rowvec != nullptr && grow < p.M)
                            ? __ldg(p.rowvec + static_cast<long long>(tc.shard) * p.rowvec_ld + grow)
                            : 0.0f;
-      if (p.epi_mode == EPI_DUAL_SOFTMAX) {
+      if (FEAT == FEAT_DUAL) {
         // P into staging buffer 0 and dS into buffer 1, then one store of each.
         const float rv2 = (p.rowvec2 != nullptr && grow < p.M)
                               ? __ldg(p.rowvec2 + static_cast<long long>(tc.shard) * p.rowvec_ld + grow)

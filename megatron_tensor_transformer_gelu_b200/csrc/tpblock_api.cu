@@ -105,6 +105,12 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
 
+template <int CG, bool WIDE, int FEAT>
+bool gemm_smem_attr() {
+  return cudaFuncSetAttribute(tp::gemm_tcgen05_kernel<CG, WIDE, FEAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              tp::GemmCfg<CG, WIDE>::SMEM_BYTES) == cudaSuccess;
+}
+
 // Resolve the current device's properties and the tensor-map encoder once.
 int device_ready(DeviceInfo** out) {
   int dev = 0;
@@ -123,12 +129,10 @@ int device_ready(DeviceInfo** out) {
       d.sm_count = sms;
     }
     if (d.ok) {
-      if (cudaFuncSetAttribute(tp::gemm_tcgen05_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               tp::GemmCfg<1>::SMEM_BYTES) != cudaSuccess ||
-          cudaFuncSetAttribute(tp::gemm_tcgen05_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               tp::GemmCfg<2>::SMEM_BYTES) != cudaSuccess ||
-          cudaFuncSetAttribute(tp::gemm_tcgen05_kernel<2, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               tp::GemmCfg<2, true>::SMEM_BYTES) != cudaSuccess ||
+      if (!gemm_smem_attr<1, false, tp::FEAT_BASE>() || !gemm_smem_attr<2, false, tp::FEAT_BASE>() ||
+          !gemm_smem_attr<2, true, tp::FEAT_BASE>() || !gemm_smem_attr<1, false, tp::FEAT_SK>() ||
+          !gemm_smem_attr<2, false, tp::FEAT_SK>() || !gemm_smem_attr<2, true, tp::FEAT_SK>() ||
+          !gemm_smem_attr<1, false, tp::FEAT_DUAL>() || !gemm_smem_attr<2, false, tp::FEAT_DUAL>() ||
           cudaFuncSetAttribute(tp::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                tp::attn::SMEM_BYTES) != cudaSuccess)
         d.ok = false;
@@ -442,7 +446,7 @@ struct GemmExtra {
   float epi_scale2 = 1.0f;
 };
 
-template <int CG, bool WIDE>
+template <int CG, bool WIDE, int FEAT>
 int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, const TilePlan& plan, const GemmExtra& ex,
                    cudaStream_t st) {
   using C = tp::GemmCfg<CG, WIDE>;
@@ -476,7 +480,7 @@ int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, const TilePlan& plan,
   }
   const long long units = tiles * p.splits;
   int clusters = static_cast<int>(units < slots ? units : slots);
-  if (plan.stream_k) {
+  if (FEAT == tp::FEAT_SK) {
     clusters = plan.sk_clusters;
     p.sk = 1;
     p.splits = 1;
@@ -500,7 +504,7 @@ int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, const TilePlan& plan,
   cfg.attrs = at;
   cfg.numAttrs = CG == 2 ? 2 : 1;
   ProfScope ps(K_GEMM_TC, st);
-  if (cudaLaunchKernelEx(&cfg, tp::gemm_tcgen05_kernel<CG, WIDE>, p) != cudaSuccess) return TP_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, tp::gemm_tcgen05_kernel<CG, WIDE, FEAT>, p) != cudaSuccess) return TP_ERR_CUDA;
   return launch_status();
 }
 
@@ -595,9 +599,18 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
     plan.tile_n = 256;
   }
   int r;
-  if (!pair) r = launch_gemm_tc<1, false>(dev, p, plan, ex, st);
-  else if (plan.tile_n > tp::GemmCfg<2>::BN) r = launch_gemm_tc<2, true>(dev, p, plan, ex, st);
-  else r = launch_gemm_tc<2, false>(dev, p, plan, ex, st);
+  if (dual) {
+    r = pair ? launch_gemm_tc<2, false, tp::FEAT_DUAL>(dev, p, plan, ex, st)
+             : launch_gemm_tc<1, false, tp::FEAT_DUAL>(dev, p, plan, ex, st);
+  } else if (plan.stream_k) {
+    if (!pair) r = launch_gemm_tc<1, false, tp::FEAT_SK>(dev, p, plan, ex, st);
+    else if (plan.tile_n > tp::GemmCfg<2>::BN) r = launch_gemm_tc<2, true, tp::FEAT_SK>(dev, p, plan, ex, st);
+    else r = launch_gemm_tc<2, false, tp::FEAT_SK>(dev, p, plan, ex, st);
+  } else {
+    if (!pair) r = launch_gemm_tc<1, false, tp::FEAT_BASE>(dev, p, plan, ex, st);
+    else if (plan.tile_n > tp::GemmCfg<2>::BN) r = launch_gemm_tc<2, true, tp::FEAT_BASE>(dev, p, plan, ex, st);
+    else r = launch_gemm_tc<2, false, tp::FEAT_BASE>(dev, p, plan, ex, st);
+  }
   if (splits_out) *splits_out = p.splits;
   return r;
 }

@@ -81,6 +81,9 @@ def parse():
     ap.add_argument("--stream-k", choices=["off", "on", "model"], default="off",
                     help="GEMM scheduling: whole-tile waves only (off, the library's default), stream-K wherever "
                          "a GEMM has scratch for it (on), the library's cost model (model)")
+    ap.add_argument("--attn-split", choices=["off", "last-wave", "all"], default="last-wave",
+                    help="attention kernel key split: none, the last partial wave (the library's default), every "
+                         "unit")
     ap.add_argument("--tp", choices=["none", "allreduce", "rs_ag"], default="none",
                     help="split the sublayer over the GPUs (tensor parallelism across ranks, strong scaling) "
                          "instead of running one replica per GPU")
@@ -480,6 +483,7 @@ def run_ours(args, rank, world, local):
         dist.barrier()
     L.lib()  # load the CUDA library (raises if it is not built)
     L.set_gemm_stream_k({"off": 0, "on": 1, "model": 2}[args.stream_k])
+    L.set_attn_kv_split({"off": 0, "last-wave": 1, "all": 2}[args.attn_split])
     tp_mode = args.tp != "none"
     P = TPProblem(w, dev, rank, world, args.tp, L, synth, torch) if tp_mode else Problem(w, dev, rank, L, synth, torch)
     X, Y = P.X, P.Y
@@ -613,6 +617,8 @@ def run_ours(args, rank, world, local):
             cfg["act"] = "gelu_tanh"
         if args.stream_k != "off":
             cfg["stream_k"] = args.stream_k
+        if args.attn_split != "last-wave":
+            cfg["attn_split"] = args.attn_split
         result = {
             "metric": metric_for(w),
             "value": round(value, 2),

@@ -426,17 +426,18 @@ int tp_gemm_plan(int M, int t, int row_mode, int shard_k, int shard_n, int out_f
 
 /* Stream-K scheduling of the tensor-core GEMMs.  Where a sublayer has
  * scratch to spare for it (the partial-sum slots past the first of the MLP
- * and attention workspaces) and the epilogue is the plain one, a GEMM may cut
- * the k-blocks of all its tiles, laid end to end, into one contiguous range
- * per CTA pair instead of dealing whole tiles out in waves, so that no pair
- * idles in a partly filled last wave.  A tile cut between pairs is summed by
- * the pair holding its last k-block, after a bounded wait for the others' f32
- * partials (TP_ERR_TIMEOUT through tp_device_error() if it gives up); the
- * partials are added in a fixed order, so results are run-to-run repeatable.
- * mode 0 (the default): the tile cost model chooses, per launch, between
- * whole-tile waves and stream-K; 1: every GEMM that has the scratch uses
- * stream-K (over as many pairs as the scratch holds partial blocks for); -1:
- * never.  Process-wide, not thread-safe against concurrent launches.  Returns
+ * and attention workspaces) and the epilogue is the plain one, a GEMM whose
+ * tiles leave a partly filled last wave may keep its whole waves of tiles and
+ * cut only the remainder tiles along K: each remainder tile's first k-blocks
+ * run on the pair that finishes it, the tails of all remainder tiles are
+ * spread over the pairs the last wave would leave idle.  The finishing pair
+ * adds the tails' f32 partials after a bounded wait for their flags
+ * (TP_ERR_TIMEOUT through tp_device_error() if it gives up), in a fixed
+ * order, so results are run-to-run repeatable.
+ * mode 0 (the default): whole tiles only (stream-K measured slower on B200
+ * for the MLP sublayer's GEMMs); 1: every GEMM that has the scratch and a
+ * partial last wave uses stream-K; 2: the tile cost model chooses per launch.
+ * Process-wide, not thread-safe against concurrent launches.  Returns
  * TP_ERR_INVALID_ARG for other values. */
 int tp_set_gemm_stream_k(int mode);
 
@@ -447,6 +448,28 @@ int tp_set_gemm_stream_k(int mode);
 int tp_gemm_plan_sk(int M, int t, int row_mode, int shard_k, int shard_n, int out_f32, int b_kmajor,
                     int heavy_epilogue, int slots, int max_splits, size_t sk_area_bytes, int* tile_n, int* splits,
                     int* stream_k, int* sk_clusters);
+
+/* Last-wave key split of the attention kernel (tp_qkv_attn_oproj_forward,
+ * tp_attn_forward_train, tp_attn_partial_forward).  The attention kernel runs
+ * one CTA per (head, 256 query rows) unit; U units on the GPU's SMs end with
+ * a partial wave of U mod SMs units.  mode 1 (the default): when twice that
+ * remainder fits in one wave, each of those last units runs as two CTAs over
+ * the two halves of the keys, whose softmax-weighted partial sums the second
+ * to finish merges with the first's (flash attention's combination of key
+ * ranges; a bounded wait, TP_ERR_TIMEOUT through tp_device_error() if it
+ * gives up); 0: never; 2: every unit is split (for tests).  The scratch is
+ * the workspace's partial-sum area, which the O projection overwrites
+ * afterwards.  Process-wide.  Returns TP_ERR_INVALID_ARG for other values. */
+int tp_set_attn_kv_split(int mode);
+
+/* The attention key-split plan for S query rows and nh heads on `slots`
+ * resident CTAs (148 on a B200) under `mode` (as tp_set_attn_kv_split) with
+ * scratch_bytes of scratch: writes *whole (units run over all keys), *split
+ * (units run as two half-key CTAs) and *kv_half (128-key blocks of a split
+ * unit's first half).  Host-only.  Returns TP_ERR_INVALID_ARG for S < 0,
+ * nh < 1, slots < 1, a mode outside [0, 2] or NULL outputs. */
+int tp_attn_split_plan(int S, int nh, int slots, int mode, size_t scratch_bytes, int* whole, int* split,
+                       int* kv_half);
 
 /* ------------------------------------------------------------ self-test ----
  * Diagnostic for the bounded-wait path every kernel here takes when one of its
@@ -475,7 +498,8 @@ int tp_selftest_exp2(const float* x, float* y_poly, float* y_exp2f, int n, void*
  * the launch's stream.  tp_profile_collect synchronises those events and
  * writes per kernel kind (0 tensor-core GEMM, 1 reduce+residual+LayerNorm,
  * 2 f32 CUDA-core GEMM, 3 attention, 4 LayerNorm backward, 5 the attention
- * backward's elementwise row-dot kernel): `launches` = all launches, `timed` = the
+ * backward's elementwise row-dot kernel, 6 the LayerNorm backward's sum of
+ * the per-CTA dgamma/dbeta rows): `launches` = all launches, `timed` = the
  * launches with events, `ms` = their summed device milliseconds; then it
  * clears the record.  Any output array may be NULL.  Returns the number of
  * kinds written (<= max_kinds), or -TP_ERR_CUDA.  Not thread-safe: enable,

@@ -78,6 +78,8 @@ SIGNATURES = {
     "tp_set_gemm_tile_n": (_c_int, [_c_int]),
     "tp_gemm_plan": (_c_int, [_c_int] * 10 + [ctypes.POINTER(_c_int), ctypes.POINTER(_c_int)]),
     "tp_set_gemm_stream_k": (_c_int, [_c_int]),
+    "tp_set_attn_kv_split": (_c_int, [_c_int]),
+    "tp_attn_split_plan": (_c_int, [_c_int] * 4 + [_c_size] + [ctypes.POINTER(_c_int)] * 3),
     "tp_gemm_plan_sk": (_c_int, [_c_int] * 10 + [_c_size] + [ctypes.POINTER(_c_int)] * 4),
     "tp_selftest_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
     "tp_selftest_flag_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
@@ -435,6 +437,20 @@ def gemm_plan_sk(M, t, row_mode, shard_k, shard_n, out_f32, b_kmajor=False, heav
     return tuple(o.value for o in out)
 
 
+def set_attn_kv_split(mode: int) -> None:
+    """Attention kernel's last-wave key split: 0 off, 1 the last partial wave
+    (the default), 2 every unit."""
+    _check(lib().tp_set_attn_kv_split(int(mode)), "tp_set_attn_kv_split")
+
+
+def attn_split_plan(S, nh, slots=148, mode=1, scratch_bytes=1 << 40):
+    """(whole, split, kv_half) of the attention kernel's key-split plan (host logic only)."""
+    out = [ctypes.c_int(0) for _ in range(3)]
+    _check(lib().tp_attn_split_plan(int(S), int(nh), int(slots), int(mode), int(scratch_bytes),
+                                    *[ctypes.byref(o) for o in out]), "tp_attn_split_plan")
+    return tuple(o.value for o in out)
+
+
 def selftest_wait_timeout(limit_cycles: int, stream=None):
     _check(lib().tp_selftest_wait_timeout(int(limit_cycles), _stream(stream)), "tp_selftest_wait_timeout")
 
@@ -463,7 +479,7 @@ def profile_sample(on: bool):
     _check(lib().tp_profile_sample(1 if on else 0), "tp_profile_sample")
 
 
-def profile_collect(nkinds: int = 6):
+def profile_collect(nkinds: int = 7):
     """{kernel kind: (launches, timed launches, summed ms of the timed ones)}"""
     launches = (ctypes.c_int * nkinds)()
     timed = (ctypes.c_int * nkinds)()

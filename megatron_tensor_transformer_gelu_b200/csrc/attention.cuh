@@ -25,6 +25,22 @@
 // 2^8 (log2 domain), so O is rescaled in TMEM rarely; P then stays below
 // 2^8, which bf16 and the f32 accumulator carry without loss of relative
 // precision.
+//
+// Last-wave key split.  The (head, 256-row) units are equal, so a grid of U
+// units on P resident CTAs ends with a partial wave of U mod P units.  Those
+// last units may be run as two CTAs each, over key blocks [0, kv_half) and
+// [kv_half, nkv): the same softmax-weighted sums over fewer keys.  Per warp
+// (32 query rows of a tile) the two halves meet through a flag pair in global
+// memory: each takes the claim flag with an atomic exchange of the launch's
+// epoch; the first to take it stores its unnormalised O rows and its (m, l)
+// and publishes the ready flag; the second waits (bounded) for ready, and
+// merges
+//     m = max(m1, m2),  l = l1 2^(m1-m) + l2 2^(m2-m),
+//     O = (O1 2^(m1-m) + O2 2^(m2-m)) / l
+// (the online softmax's combination of two key ranges), then stores O and
+// the row's log2 denominator.  The merge is symmetric in the two halves, so
+// results do not depend on which half arrives first.  No CTA ever waits for
+// a CTA that has not finished its main loop, so no wait can deadlock.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -66,7 +82,25 @@ struct AttnArgs {
   float* lse2;         // optional [nh, S]: log2 of each row's softmax denominator, in the
                        // units of the scores times scale_log2 (what a backward pass
                        // needs to rebuild P = 2^(s scale_log2 - lse2))
+  // Units (head, 256 query rows) in launch order: unit u = head u / nq, query
+  // block u % nq.  Blocks [0, whole) run units 0..whole-1 over every key;
+  // blocks whole + 2i and whole + 2i + 1 run unit whole + i over key blocks
+  // [0, kv_half) and [kv_half, nkv).
+  int nq;
+  int whole;
+  int kv_half;
+  float* part_o;                   // split scratch: [split units][2][4][32 col groups][32 rows] float4
+  float* part_ml;                  // [split units][2][4][2][32]: m and l of the stored rows
+  unsigned long long* part_flags;  // [split units][2][4][2]: claim, ready
+  unsigned long long epoch;        // this launch's flag value
 };
+
+// Atomic exchange with acquire-release semantics at GPU scope.
+__device__ __forceinline__ unsigned long long flag_exchange(unsigned long long* addr, unsigned long long v) {
+  unsigned long long old;
+  asm volatile("atom.acq_rel.gpu.global.exch.b64 %0, [%1], %2;" : "=l"(old) : "l"(addr), "l"(v) : "memory");
+  return old;
+}
 
 __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __grid_constant__ AttnArgs a) {
   using namespace attn;
@@ -89,15 +123,23 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * (TILES * BQ);
-  const int h = blockIdx.y;
+  const int nkv = a.S / BKV;
+  int unit = blockIdx.x, kb0 = 0, nkb = nkv, su = -1;  // su: split unit index, -1 when whole
+  if (unit >= a.whole) {
+    const int v = unit - a.whole;
+    su = v >> 1;
+    unit = a.whole + su;
+    kb0 = (v & 1) ? a.kv_half : 0;
+    nkb = (v & 1) ? nkv - a.kv_half : a.kv_half;
+  }
+  const int q0 = (unit % a.nq) * (TILES * BQ);
+  const int h = unit / a.nq;
   const int shard = h / a.heads_per_shard;
   const int hj = h % a.heads_per_shard;
   const int Hs = a.heads_per_shard * D;
   const int qcol = shard * a.shard_cols + hj * D;
   const int kcol = qcol + Hs;
   const int vcol = qcol + 2 * Hs;
-  const int nkv = a.S / BKV;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -151,15 +193,15 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
           tma_load_2d(sQ + t * TILE_BYTES + HALF_BYTES, &a.tmQKV, qcol + 64, q0 + t * BQ, q_full);
         }
       }
-      for (int j = 0; j < nkv; ++j) {
+      for (int j = 0; j < nkb; ++j) {
         const int st = j % nst;
         const uint32_t ph = (j / nst) & 1;
         if (!mbar_wait(&emptyb[st], ph ^ 1)) { ok = false; break; }
         uint8_t* d = base + st * TILE_BYTES;
         mbar_arrive_expect_tx(&fullb[st], TILE_BYTES);
         armed[st] = static_cast<int>(ph);
-        tma_load_2d(d, &a.tmQKV, col, j * BKV, &fullb[st]);
-        tma_load_2d(d + HALF_BYTES, &a.tmQKV, col + 64, j * BKV, &fullb[st]);
+        tma_load_2d(d, &a.tmQKV, col, (kb0 + j) * BKV, &fullb[st]);
+        tma_load_2d(d + HALF_BYTES, &a.tmQKV, col + 64, (kb0 + j) * BKV, &fullb[st]);
       }
       if (!ok) {
         for (int i = 0; i <= K_STAGES; ++i) {
@@ -194,10 +236,10 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
         if (t == TILES - 1) umma_commit(&k_empty[ks]);
         return true;
       };
-      for (int t = 0; t < TILES && ok && nkv > 0; ++t) ok = issue_s(0, t);
+      for (int t = 0; t < TILES && ok && nkb > 0; ++t) ok = issue_s(0, t);
       // Per block: P0 V, S0(j+1), P1 V, S1(j+1).  Tile 0's next scores are
       // ready while tile 1 is still in its exponentials, and the reverse.
-      for (int j = 0; j < nkv && ok; ++j) {
+      for (int j = 0; j < nkb && ok; ++j) {
         const int vs = j % V_STAGES;
         if (!mbar_wait(&v_full[vs], (j / V_STAGES) & 1)) { ok = false; break; }
         const uint32_t v_addr = smem_u32(sV + vs * TILE_BYTES);
@@ -214,7 +256,7 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
           umma_commit(&pv_done[t]);
           if (t == TILES - 1) umma_commit(&v_empty[vs]);
           // S_t(j+1) overwrites P_t(j): issued after P_t(j) V_j above.
-          if (j + 1 < nkv && !issue_s(j + 1, t)) { ok = false; break; }
+          if (j + 1 < nkb && !issue_s(j + 1, t)) { ok = false; break; }
         }
       }
       if (!ok) {
@@ -235,7 +277,7 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
     float m_run = -INFINITY;
     float l_run = 0.0f;
     bool ok = true;
-    for (int j = 0; j < nkv; ++j) {
+    for (int j = 0; j < nkb; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[tile], j & 1))) { ok = false; break; }
       tc_fence_after();
       float s[BKV];
@@ -315,25 +357,93 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
       mbar_arrive(&p_full[tile]);
     }
     const bool tile_valid = q0 + tile * BQ < a.S;  // the second tile of an odd tile count is not stored
-    if (ok && __all_sync(0xffffffffu, mbar_wait(&pv_done[tile], (nkv - 1) & 1)) && tile_valid) {
+    if (ok && __all_sync(0xffffffffu, mbar_wait(&pv_done[tile], (nkb - 1) & 1)) && tile_valid) {
       tc_fence_after();
-      const float inv = 1.0f / l_run;
-      const int grow = q0 + tile * BQ + r;
-      if (a.lse2) a.lse2[static_cast<long long>(h) * a.S + grow] = m_run + __log2f(l_run);
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.O) + static_cast<long long>(grow) * a.H + h * D;
+      // Split unit: the first half to claim this warp's rows stores them and
+      // is done; the second merges them with its own.
+      bool merge = false;
+      float4* po = nullptr;
+      float* pml = nullptr;
+      if (su >= 0) {
+        const int slot = (su * TILES + tile) * 4 + q;
+        unsigned long long* flags = a.part_flags + 2 * slot;
+        po = reinterpret_cast<float4*>(a.part_o) + static_cast<long long>(slot) * (D / 4) * 32;
+        pml = a.part_ml + slot * 64;
+        unsigned long long prev = 0;
+        if (lane == 0) prev = flag_exchange(&flags[0], a.epoch);
+        merge = __shfl_sync(0xffffffffu, prev == a.epoch ? 1 : 0, 0) != 0;
+        if (!merge) {
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t u[32];
-        tmem_ld_32x32b_x32(tO + c * 32, u);
-        tmem_wait_ld();
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t u[32];
+            tmem_ld_32x32b_x32(tO + c * 32, u);
+            tmem_wait_ld();
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(u[g * 8 + 0]) * inv, __uint_as_float(u[g * 8 + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(u[g * 8 + 2]) * inv, __uint_as_float(u[g * 8 + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(u[g * 8 + 4]) * inv, __uint_as_float(u[g * 8 + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(u[g * 8 + 6]) * inv, __uint_as_float(u[g * 8 + 7]) * inv);
-          *reinterpret_cast<uint4*>(orow + c * 32 + g * 8) = w;
+            for (int g = 0; g < 8; ++g)
+              __stcg(po + (c * 8 + g) * 32 + lane,
+                     make_float4(__uint_as_float(u[g * 4 + 0]), __uint_as_float(u[g * 4 + 1]),
+                                 __uint_as_float(u[g * 4 + 2]), __uint_as_float(u[g * 4 + 3])));
+          }
+          __stcg(pml + lane, m_run);
+          __stcg(pml + 32 + lane, l_run);
+          __threadfence();
+          __syncwarp();
+          if (lane == 0) flag_publish(&flags[1], a.epoch);
+        } else {
+          bool ready = true;
+          if (lane == 0) ready = flag_wait_eq(&flags[1], a.epoch);
+          ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
+          __threadfence();
+          if (!ready) merge = false;
+        }
+        if (!merge) po = nullptr;  // stored (or gave up): nothing to write here
+      }
+      if (su < 0 || po) {
+        // Row scale: 1 / l, or for a merge 2^(m_own - m) / l and 2^(m_other - m) / l,
+        // formed the same way whichever half is "own", so the sum is symmetric.
+        float s_own = 1.0f, s_oth = 0.0f, m_fin = m_run, l_fin = l_run;
+        if (po) {
+          const float m_oth = __ldcg(pml + lane);
+          const float l_oth = __ldcg(pml + 32 + lane);
+          m_fin = fmaxf(m_run, m_oth);
+          const float e_own = exp2_fast(m_run - m_fin), e_oth = exp2_fast(m_oth - m_fin);
+          l_fin = __fadd_rn(__fmul_rn(l_run, e_own), __fmul_rn(l_oth, e_oth));
+          const float inv = 1.0f / l_fin;
+          s_own = __fmul_rn(e_own, inv);
+          s_oth = __fmul_rn(e_oth, inv);
+        } else {
+          s_own = 1.0f / l_run;
+        }
+        const int grow = q0 + tile * BQ + r;
+        if (a.lse2) a.lse2[static_cast<long long>(h) * a.S + grow] = m_fin + __log2f(l_fin);
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.O) + static_cast<long long>(grow) * a.H + h * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t u[32];
+          tmem_ld_32x32b_x32(tO + c * 32, u);
+          tmem_wait_ld();
+          float o[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = __uint_as_float(u[e]) * s_own;
+          if (po) {
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+              const float4 v = __ldcg(po + (c * 8 + g) * 32 + lane);
+              o[g * 4 + 0] = __fadd_rn(o[g * 4 + 0], __fmul_rn(v.x, s_oth));
+              o[g * 4 + 1] = __fadd_rn(o[g * 4 + 1], __fmul_rn(v.y, s_oth));
+              o[g * 4 + 2] = __fadd_rn(o[g * 4 + 2], __fmul_rn(v.z, s_oth));
+              o[g * 4 + 3] = __fadd_rn(o[g * 4 + 3], __fmul_rn(v.w, s_oth));
+            }
+          }
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            uint4 w;
+            w.x = pack_bf16x2(o[g * 8 + 0], o[g * 8 + 1]);
+            w.y = pack_bf16x2(o[g * 8 + 2], o[g * 8 + 3]);
+            w.z = pack_bf16x2(o[g * 8 + 4], o[g * 8 + 5]);
+            w.w = pack_bf16x2(o[g * 8 + 6], o[g * 8 + 7]);
+            *reinterpret_cast<uint4*>(orow + c * 32 + g * 8) = w;
+          }
         }
       }
     }

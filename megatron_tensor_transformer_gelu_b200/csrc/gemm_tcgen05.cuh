@@ -1015,7 +1015,7 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
       const float rv = (p.rowvec != nullptr && grow < p.M)
                            ? __ldg(p.rowvec + static_cast<long long>(tc.shard) * p.rowvec_ld + grow)
                            : 0.0f;
-      if (FEAT == FEAT_DUAL) {
+      if constexpr (FEAT == FEAT_DUAL) {
         // P into staging buffer 0 and dS into buffer 1, then one store of each.
         const float rv2 = (p.rowvec2 != nullptr && grow < p.M)
                               ? __ldg(p.rowvec2 + static_cast<long long>(tc.shard) * p.rowvec_ld + grow)
@@ -1056,83 +1056,82 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
           }
 #endif
         }
-        if (++acc == acc_bufs) { acc = 0; acc_phase ^= 1; }
-        continue;
-      }
-      for (int c = 0; c < nchunks; ++c) {
-        for (int part = 0; part < parts; ++part) {
-          // The TMA store that last read this staging buffer must be done with it.
+      } else {
+        for (int c = 0; c < nchunks; ++c) {
+          for (int part = 0; part < parts; ++part) {
+            // The TMA store that last read this staging buffer must be done with it.
 #if TP_GEMM_WARP_STORES
-          if (lane == 0) bulk_wait_group_read<1>();
-          __syncwarp();
+            if (lane == 0) bulk_wait_group_read<1>();
+            __syncwarp();
 #else
-          if (elected) bulk_wait_group_read<1>();
-          named_barrier_sync(1, 128);
+            if (elected) bulk_wait_group_read<1>();
+            named_barrier_sync(1, 128);
 #endif
-          uint8_t* stage_row = sEpi + buf * C::EPI_BUF_BYTES + row_local * 128;
-          const uint32_t taddr = t_row + c * (p.out_f32 ? 32 : 64);
-          if (p.epi_mode == EPI_SOFTMAX) {
-            epi_chunk_softmax(taddr, stage_row, row_local, rv, p.epi_scale);
-          } else if (p.epi_mode == EPI_DSOFTMAX) {
-            const __nv_bfloat16* prow =
-                grow < p.M ? static_cast<const __nv_bfloat16*>(p.aux) + static_cast<long long>(grow) * p.ld_aux +
-                                 tc.out_col0 + c * 64
-                           : nullptr;
-            uint32_t pw[32];
-            epi_load_p64(prow, tc.n_valid - c * 64, pw);
-            epi_chunk_dsoftmax(taddr, stage_row, row_local, pw, rv, p.epi_scale);
-          } else if (p.epi_mode == EPI_GRAD) {
-            const __nv_bfloat16* urow =
-                grow < p.M ? static_cast<const __nv_bfloat16*>(p.aux) + static_cast<long long>(grow) * p.ld_aux +
-                                 tc.out_col0 + c * 64
-                           : nullptr;
-            const int nvalid = tc.n_valid - c * 64;
-            switch (p.act) {  // uniform: one branch per chunk
-              case ACT_GELU_TANH: epi_chunk_grad<ACT_GELU_TANH>(taddr, stage_row, row_local, urow, nvalid); break;
-              case ACT_GELU_ERF: epi_chunk_grad<ACT_GELU_ERF>(taddr, stage_row, row_local, urow, nvalid); break;
-              case ACT_RELU: epi_chunk_grad<ACT_RELU>(taddr, stage_row, row_local, urow, nvalid); break;
-              default: epi_chunk_grad<ACT_NONE>(taddr, stage_row, row_local, urow, nvalid); break;
-            }
-          } else if (part < parts - 1) {
-            epi_chunk<ACT_NONE>(p.out_f32, taddr, stage_row, row_local);
-          } else {
-            switch (p.act) {  // uniform: one branch per chunk
-              case ACT_GELU_TANH: epi_chunk<ACT_GELU_TANH>(p.out_f32, taddr, stage_row, row_local); break;
-              case ACT_GELU_ERF: epi_chunk<ACT_GELU_ERF>(p.out_f32, taddr, stage_row, row_local); break;
-              case ACT_RELU: epi_chunk<ACT_RELU>(p.out_f32, taddr, stage_row, row_local); break;
-              default: epi_chunk<ACT_NONE>(p.out_f32, taddr, stage_row, row_local); break;
-            }
-          }
-          if (c == nchunks - 1 && part == parts - 1) {
-            // Every accumulator column of this tile has been read: hand the
-            // TMEM buffer back to the MMA issuer before the last store.
-            tc_fence_before();
-            if constexpr (CG == 1) {
-              mbar_arrive(&tempty[acc]);
+            uint8_t* stage_row = sEpi + buf * C::EPI_BUF_BYTES + row_local * 128;
+            const uint32_t taddr = t_row + c * (p.out_f32 ? 32 : 64);
+            if (p.epi_mode == EPI_SOFTMAX) {
+              epi_chunk_softmax(taddr, stage_row, row_local, rv, p.epi_scale);
+            } else if (p.epi_mode == EPI_DSOFTMAX) {
+              const __nv_bfloat16* prow =
+                  grow < p.M ? static_cast<const __nv_bfloat16*>(p.aux) + static_cast<long long>(grow) * p.ld_aux +
+                                   tc.out_col0 + c * 64
+                             : nullptr;
+              uint32_t pw[32];
+              epi_load_p64(prow, tc.n_valid - c * 64, pw);
+              epi_chunk_dsoftmax(taddr, stage_row, row_local, pw, rv, p.epi_scale);
+            } else if (p.epi_mode == EPI_GRAD) {
+              const __nv_bfloat16* urow =
+                  grow < p.M ? static_cast<const __nv_bfloat16*>(p.aux) + static_cast<long long>(grow) * p.ld_aux +
+                                   tc.out_col0 + c * 64
+                             : nullptr;
+              const int nvalid = tc.n_valid - c * 64;
+              switch (p.act) {  // uniform: one branch per chunk
+                case ACT_GELU_TANH: epi_chunk_grad<ACT_GELU_TANH>(taddr, stage_row, row_local, urow, nvalid); break;
+                case ACT_GELU_ERF: epi_chunk_grad<ACT_GELU_ERF>(taddr, stage_row, row_local, urow, nvalid); break;
+                case ACT_RELU: epi_chunk_grad<ACT_RELU>(taddr, stage_row, row_local, urow, nvalid); break;
+                default: epi_chunk_grad<ACT_NONE>(taddr, stage_row, row_local, urow, nvalid); break;
+              }
+            } else if (part < parts - 1) {
+              epi_chunk<ACT_NONE>(p.out_f32, taddr, stage_row, row_local);
             } else {
-              __syncwarp();
-              if (lane == 0) mbar_arrive_cluster(tempty_leader0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+              switch (p.act) {  // uniform: one branch per chunk
+                case ACT_GELU_TANH: epi_chunk<ACT_GELU_TANH>(p.out_f32, taddr, stage_row, row_local); break;
+                case ACT_GELU_ERF: epi_chunk<ACT_GELU_ERF>(p.out_f32, taddr, stage_row, row_local); break;
+                case ACT_RELU: epi_chunk<ACT_RELU>(p.out_f32, taddr, stage_row, row_local); break;
+                default: epi_chunk<ACT_NONE>(p.out_f32, taddr, stage_row, row_local); break;
+              }
             }
-          }
-          fence_proxy_async_smem();
+            if (c == nchunks - 1 && part == parts - 1) {
+              // Every accumulator column of this tile has been read: hand the
+              // TMEM buffer back to the MMA issuer before the last store.
+              tc_fence_before();
+              if constexpr (CG == 1) {
+                mbar_arrive(&tempty[acc]);
+              } else {
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(tempty_leader0 + static_cast<uint32_t>(acc * sizeof(uint64_t)));
+              }
+            }
+            fence_proxy_async_smem();
 #if TP_GEMM_WARP_STORES
-          // Each warp stores its own 32 rows (a 4 KiB, 1 KiB-aligned slice of the
-          // staging buffer, so the 128-byte swizzle pattern is the same).
-          __syncwarp();
-          if (lane == 0 && y0 + q * 32 < p.M) {
-            const CUtensorMap* map = part < parts - 1 ? tmAux : tmC;
-            tma_store_3d(map, sEpi + buf * C::EPI_BUF_BYTES + q * 32 * 128, tc.n_in + c * cw, ystore + q * 32, split);
-            bulk_commit_group();
-          }
+            // Each warp stores its own 32 rows (a 4 KiB, 1 KiB-aligned slice of the
+            // staging buffer, so the 128-byte swizzle pattern is the same).
+            __syncwarp();
+            if (lane == 0 && y0 + q * 32 < p.M) {
+              const CUtensorMap* map = part < parts - 1 ? tmAux : tmC;
+              tma_store_3d(map, sEpi + buf * C::EPI_BUF_BYTES + q * 32 * 128, tc.n_in + c * cw, ystore + q * 32, split);
+              bulk_commit_group();
+            }
 #else
-          named_barrier_sync(1, 128);
-          if (elected && y0 < p.M) {
-            const CUtensorMap* map = part < parts - 1 ? tmAux : tmC;
-            tma_store_3d(map, sEpi + buf * C::EPI_BUF_BYTES, tc.n_in + c * cw, ystore, split);
-            bulk_commit_group();
-          }
+            named_barrier_sync(1, 128);
+            if (elected && y0 < p.M) {
+              const CUtensorMap* map = part < parts - 1 ? tmAux : tmC;
+              tma_store_3d(map, sEpi + buf * C::EPI_BUF_BYTES, tc.n_in + c * cw, ystore, split);
+              bulk_commit_group();
+            }
 #endif
-          buf ^= 1;
+            buf ^= 1;
+          }
         }
       }
       if (++acc == acc_bufs) { acc = 0; acc_phase ^= 1; }

@@ -68,12 +68,13 @@ std::mutex g_mu;
 DeviceInfo g_dev[MAX_DEVICES];
 int g_force_tile_n = 0;  // tp_set_gemm_tile_n: 0 = cost model
 int g_stream_k = 0;      // tp_set_gemm_stream_k: 0 = whole tiles, 1 = wherever a workspace allows, 2 = cost model
+int g_attn_split = 1;    // tp_set_attn_kv_split: 0 = off, 1 = the last partial wave, 2 = every unit
 unsigned long long g_sk_epoch = 0;  // last stream-K launch's epoch (see next_sk_epoch)
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 // ------------------------------------------------------------ event timing
 constexpr int PROF_CAP = 16384;  // launches timed between two collects
-constexpr int PROF_KINDS = 6;
+constexpr int PROF_KINDS = 7;
 bool g_prof_on = false;
 bool g_prof_sampling = true;  // record events for the launches made while set
 bool g_prof_events_made = false;
@@ -83,7 +84,9 @@ int g_prof_kind[PROF_CAP];
 int g_prof_n = 0;
 long long g_prof_launches[PROF_KINDS];  // every launch while enabled, timed or not
 
-enum Kind { K_GEMM_TC = 0, K_REDUCE_LN = 1, K_GEMM_SIMT = 2, K_ATTN = 3, K_LN_BACK = 4, K_ATTN_BACK = 5 };
+enum Kind {
+  K_GEMM_TC = 0, K_REDUCE_LN = 1, K_GEMM_SIMT = 2, K_ATTN = 3, K_LN_BACK = 4, K_ATTN_BACK = 5, K_LN_PARAMS = 6
+};
 
 struct ProfScope {
   int slot = -1;
@@ -887,7 +890,7 @@ int run_ln_backward(int S, int H, const float* V, const void* X, const void* dY,
     if (le != cudaSuccess || launch_status() != TP_OK) return TP_ERR_CUDA;
   }
   if (dgamma || dbeta) {
-    ProfScope ps(K_LN_BACK, st);
+    ProfScope ps(K_LN_PARAMS, st);
     const cudaError_t le = launch_pdl(tp::ln_grad_params_kernel, dim3(ceil_div(H, 32)),
                                       dim3(32 * tp::LNB_PARAM_SLICES), 0, st, static_cast<const float*>(partial),
                                       grid, H, dgamma, dbeta);
@@ -1007,10 +1010,45 @@ struct AttnKeep {
 // by t shards (nh / t each) of a model of hidden size H: QKV [S, 3 nh d] and O
 // [S, nh d] bf16 in the given buffers, Zsum = sum_s O_s Wo_s (f32 [S, H]; up to
 // max_splits K-split slots, *nparts used).  Arguments are already checked.
+// Last-wave key split of the attention kernel (see attention.cuh): of U =
+// nh * ceil(S / 256) units on `slots` resident CTAs, the R = U mod slots of
+// the last partial wave run as two half-key-range CTAs each when 2R CTAs fit
+// in one wave (mode 1), or every unit does (mode 2, for tests).  Scratch:
+// partial O rows, (m, l) rows and flags per split unit.
+struct AttnSplit {
+  int whole, split, kv_half;
+};
+
+size_t attn_split_bytes(long long R) {
+  return align256(static_cast<size_t>(R) * 8 * 32 * tp::attn::D * 4) + align256(static_cast<size_t>(R) * 8 * 64 * 4) +
+         static_cast<size_t>(R) * 8 * 2 * 8;
+}
+
+AttnSplit attn_split_plan(int S, int nh, int slots, int mode, size_t scratch_bytes) {
+  const int per = tp::attn::TILES * tp::attn::BQ;
+  const long long U = static_cast<long long>(nh) * ((S + per - 1) / per);
+  const int nkv = S / tp::attn::BKV;
+  AttnSplit p{static_cast<int>(U), 0, 0};
+  if (mode == 0 || U == 0 || slots < 2 || nkv < 2) return p;
+  long long R;
+  if (mode == 2) {
+    R = U;
+  } else {
+    if (nkv < 4) return p;  // halves of one key block gain nothing
+    R = U % slots;
+    if (R == 0 || 2 * R > slots) return p;
+  }
+  if (attn_split_bytes(R) > scratch_bytes) return p;
+  p.whole = static_cast<int>(U - R);
+  p.split = static_cast<int>(R);
+  p.kv_half = nkv / 2;
+  return p;
+}
+
 int attn_products(const DeviceInfo& dev, int S, int H, int nh, int d, int t, const void* in,
                   const void* const* Wqkv_shards, const void* const* Wo_shards, void* QKV, void* Obuf, float* Zsum,
                   int max_splits, int* nparts, cudaStream_t s, int kmaj, float* lse2, void* sk_ws = nullptr,
-                  size_t sk_bytes = 0) {
+                  size_t sk_bytes = 0, size_t zsum_bytes = 0) {
   *nparts = 1;
   if (S == 0) return TP_OK;
   const int Hl = nh * d;    // columns of the heads held here
@@ -1037,7 +1075,21 @@ int attn_products(const DeviceInfo& dev, int S, int H, int nh, int d, int t, con
     a.shard_cols = 3 * Hs;
     a.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
     a.lse2 = lse2;
-    dim3 grid((S + tp::attn::TILES * tp::attn::BQ - 1) / (tp::attn::TILES * tp::attn::BQ), nh);
+    a.nq = (S + tp::attn::TILES * tp::attn::BQ - 1) / (tp::attn::TILES * tp::attn::BQ);
+    // The key-split scratch is the partial-sum area, which the O projection
+    // below overwrites only after this kernel.
+    const AttnSplit sp = attn_split_plan(S, nh, dev.sm_count, g_attn_split, zsum_bytes);
+    a.whole = sp.whole;
+    a.kv_half = sp.kv_half;
+    if (sp.split > 0) {
+      uint8_t* w = reinterpret_cast<uint8_t*>(Zsum);
+      const size_t ob = align256(static_cast<size_t>(sp.split) * 8 * 32 * tp::attn::D * 4);
+      a.part_o = reinterpret_cast<float*>(w);
+      a.part_ml = reinterpret_cast<float*>(w + ob);
+      a.part_flags = reinterpret_cast<unsigned long long*>(w + ob + align256(static_cast<size_t>(sp.split) * 8 * 64 * 4));
+      a.epoch = next_sk_epoch();
+    }
+    dim3 grid(sp.whole + 2 * sp.split);
     ProfScope ps(K_ATTN, s);
     st = launch_pdl(tp::attn_fwd_kernel, grid, dim3(tp::attn::NUM_THREADS), tp::attn::SMEM_BYTES, s, a) != cudaSuccess
              ? TP_ERR_CUDA
@@ -1065,7 +1117,8 @@ int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out
   const size_t sh4 = static_cast<size_t>(S) * H * 4;
   int st = attn_products(dev, S, H, nh, d, t, in, Wqkv_shards, Wo_shards, QKV, Obuf, Zsum,
                          keep ? 1 : TP_MAX_K_SPLITS, &nparts, s, kmaj, keep ? keep->lse2 : nullptr,
-                         keep ? nullptr : reinterpret_cast<uint8_t*>(Zsum) + sh4, keep ? 0 : (TP_MAX_K_SPLITS - 1) * sh4);
+                         keep ? nullptr : reinterpret_cast<uint8_t*>(Zsum) + sh4, keep ? 0 : (TP_MAX_K_SPLITS - 1) * sh4,
+                         keep ? sh4 : TP_MAX_K_SPLITS * sh4);
   if (st != TP_OK) return st;
   return run_reduce_ln(S, H, nparts, Zsum, res, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s, dev.sm_count,
                        apply_ln);
@@ -1833,7 +1886,8 @@ int tp_attn_partial_forward(int S, int H, int nh, int d, int t, int dtype, const
   const size_t hl = static_cast<size_t>(nh) * d;
   int nparts = 1;
   return attn_products(*dev, S, H, nh, d, t, X, Wqkv_shards, Wo_shards, ws, ws + align256(static_cast<size_t>(S) * 3 * hl * 2),
-                       P, 1, &nparts, static_cast<cudaStream_t>(stream), 0, nullptr);
+                       P, 1, &nparts, static_cast<cudaStream_t>(stream), 0, nullptr, nullptr, 0,
+                       static_cast<size_t>(S) * H * 4);
 }
 
 // --------------------------------------------- peer access between ranks
@@ -1967,6 +2021,23 @@ int tp_gemm_plan(int M, int t, int row_mode, int shard_k, int shard_n, int out_f
                          tile_n, splits, nullptr, nullptr);
 }
 
+int tp_set_attn_kv_split(int mode) {
+  if (mode < 0 || mode > 2) return TP_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_attn_split = mode;
+  return TP_OK;
+}
+
+int tp_attn_split_plan(int S, int nh, int slots, int mode, size_t scratch_bytes, int* whole, int* split,
+                       int* kv_half) {
+  if (S < 0 || nh < 1 || slots < 1 || mode < 0 || mode > 2 || !whole || !split || !kv_half) return TP_ERR_INVALID_ARG;
+  const AttnSplit p = attn_split_plan(S, nh, slots, mode, scratch_bytes);
+  *whole = p.whole;
+  *split = p.split;
+  *kv_half = p.kv_half;
+  return TP_OK;
+}
+
 // ------------------------------------------------------------- self-test
 int tp_selftest_flag_wait_timeout(long long limit_cycles, void* stream) {
   if (limit_cycles < 1) return TP_ERR_INVALID_ARG;
@@ -2048,6 +2119,7 @@ const char* tp_kernel_kind_name(int kind) {
     case K_ATTN: return "attention_fwd";
     case K_LN_BACK: return "layernorm_backward";
     case K_ATTN_BACK: return "attention_backward_elementwise";
+    case K_LN_PARAMS: return "layernorm_grad_params";
     default: return "unknown";
   }
 }

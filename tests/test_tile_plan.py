@@ -136,3 +136,40 @@ def test_stream_k_switch():
             L.set_gemm_stream_k(3)
     finally:
         L.set_gemm_stream_k(0)
+
+
+# ---------------------------------------------- attention key-split plan
+def _split_bytes(R):
+    r256 = lambda x: (x + 255) // 256 * 256
+    return r256(R * 8 * 32 * 128 * 4) + r256(R * 8 * 64 * 4) + R * 8 * 2 * 8
+
+
+def test_attn_split_plan_of_the_workload():
+    # 64 heads x 8 query blocks = 512 units on 148 SMs: 3 waves + 68 units,
+    # which run as 136 half-key CTAs (8 + 8 key blocks)
+    assert L.attn_split_plan(2048, 64, slots=148, mode=1) == (444, 68, 8)
+    assert L.attn_split_plan(2048, 64, slots=148, mode=0) == (512, 0, 0)
+    assert L.attn_split_plan(2048, 64, slots=148, mode=2) == (0, 512, 8)
+    # exactly enough scratch, and one byte short
+    assert L.attn_split_plan(2048, 64, 148, 1, _split_bytes(68)) == (444, 68, 8)
+    assert L.attn_split_plan(2048, 64, 148, 1, _split_bytes(68) - 1) == (512, 0, 0)
+
+
+def test_attn_split_plan_edges():
+    # the remainder does not fit twice in a wave (248 = 148 + 100): no split
+    assert L.attn_split_plan(2048, 31, slots=148, mode=1) == (248, 0, 0)
+    # whole waves only: nothing to split
+    assert L.attn_split_plan(2048, 37, slots=148, mode=1) == (296, 0, 0)
+    # fewer units than SMs: every unit is in the partial wave
+    assert L.attn_split_plan(1024, 16, slots=148, mode=1) == (0, 64, 4)
+    # fewer than 4 key blocks: not worth it by default, possible when forced
+    assert L.attn_split_plan(384, 2, slots=148, mode=1) == (4, 0, 0)
+    assert L.attn_split_plan(384, 2, slots=148, mode=2) == (0, 4, 1)
+    # one key block cannot be halved
+    assert L.attn_split_plan(128, 2, slots=148, mode=2) == (2, 0, 0)
+    assert L.attn_split_plan(0, 2, slots=148, mode=2) == (0, 0, 0)
+    for args in ((-1, 2, 148, 1), (256, 0, 148, 1), (256, 2, 0, 1), (256, 2, 148, 3)):
+        with pytest.raises(L.TPError):
+            L.attn_split_plan(*args)
+    with pytest.raises(L.TPError):
+        L.set_attn_kv_split(3)

@@ -491,6 +491,12 @@ int tp_selftest_flag_wait_timeout(long long limit_cycles, void* stream);
  * unit.  Writes, for the n f32 inputs x (device), that evaluation into y_poly
  * and CUDA's exp2f(x) into y_exp2f (device, n each). */
 int tp_selftest_exp2(const float* x, float* y_poly, float* y_exp2f, int n, void* stream);
+/* The same with a choice of the polynomial: form 0 the degree-4 single-value
+ * evaluation (as tp_selftest_exp2), form 1 the degree-3 evaluation of two
+ * values at once with packed f32x2 arithmetic (inputs 2i and 2i + 1 share
+ * one evaluation), which is the form the attention kernel's softmax uses.
+ * Returns TP_ERR_INVALID_ARG for another form. */
+int tp_selftest_exp2_form(const float* x, float* y_poly, float* y_exp2f, int n, int form, void* stream);
 
 /* ----------------------------------------------------- kernel timing ----
  * When enabled, every kernel the library launches is counted, and the first

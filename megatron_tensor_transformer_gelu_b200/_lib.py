@@ -84,6 +84,7 @@ SIGNATURES = {
     "tp_selftest_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
     "tp_selftest_flag_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
     "tp_selftest_exp2": (_c_int, [_vp, _vp, _vp, _c_int, _vp]),
+    "tp_selftest_exp2_form": (_c_int, [_vp, _vp, _vp, _c_int, _c_int, _vp]),
     "tp_profile_enable": (_c_int, [_c_int]),
     "tp_profile_sample": (_c_int, [_c_int]),
     "tp_profile_collect": (_c_int, [ctypes.POINTER(_c_int), ctypes.POINTER(_c_int), ctypes.POINTER(ctypes.c_double),
@@ -459,11 +460,14 @@ def selftest_flag_wait_timeout(limit_cycles: int, stream=None):
     _check(lib().tp_selftest_flag_wait_timeout(int(limit_cycles), _stream(stream)), "tp_selftest_flag_wait_timeout")
 
 
-def selftest_exp2(x, stream=None):
-    """(the attention kernel's polynomial 2^x, CUDA's exp2f(x)) for a device f32 tensor x."""
+def selftest_exp2(x, stream=None, form=0):
+    """(a polynomial 2^x, CUDA's exp2f(x)) for a device f32 tensor x: form 0
+    the degree-4 single-value evaluation, form 1 the degree-3 pair (f32x2)
+    evaluation the attention kernel's softmax uses."""
     yp = torch.empty_like(x)
     yr = torch.empty_like(x)
-    _check(lib().tp_selftest_exp2(_ptr(x), _ptr(yp), _ptr(yr), x.numel(), _stream(stream)), "tp_selftest_exp2")
+    _check(lib().tp_selftest_exp2_form(_ptr(x), _ptr(yp), _ptr(yr), x.numel(), int(form), _stream(stream)),
+           "tp_selftest_exp2_form")
     return yp, yr
 
 

@@ -68,6 +68,10 @@ constexpr float RESCALE_THRESHOLD = 8.0f;
 #ifndef TP_ATTN_EXP2_POLY_EVERY
 #define TP_ATTN_EXP2_POLY_EVERY 0
 #endif
+// Softmax arithmetic on f32 pairs (f32x2 scale and row sum, three-input max).
+#ifndef TP_ATTN_X2
+#define TP_ATTN_X2 1
+#endif
 constexpr int EXP2_POLY_EVERY = TP_ATTN_EXP2_POLY_EVERY;  // 0: every exponential on the MUFU unit
 constexpr int EXP2_POLY_MOD = EXP2_POLY_EVERY > 0 ? EXP2_POLY_EVERY : 1;
 }  // namespace attn
@@ -296,16 +300,26 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
           s[96 + e] = __uint_as_float(u3[e]);
         }
       }
-      // Row max with 8 independent chains, then a tree.
+      // Row max with 8 independent chains (three-input max), then a tree.
       float m8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) m8[i] = s[i];
+#if TP_ATTN_X2
+#pragma unroll
+      for (int e = 8; e + 16 <= BKV; e += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = max3f(m8[i], s[e + i], s[e + 8 + i]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[BKV - 8 + i]);
+      const float mx = max3f(max3f(m8[0], m8[1], m8[2]), max3f(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+#else
 #pragma unroll
       for (int e = 8; e < BKV; e += 8)
 #pragma unroll
         for (int i = 0; i < 8; ++i) m8[i] = fmaxf(m8[i], s[e + i]);
       const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
                              fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+#endif
       const float m_blk = mx * a.scale_log2;
       const bool resc = m_blk > m_run + RESCALE_THRESHOLD;
       float alpha = 1.0f;
@@ -314,11 +328,39 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
         m_run = m_blk;
       }
       // p = 2^(s * scale_log2 - m) in f32, kept as bf16 pairs for the P V
-      // product; the row sum adds the f32 values in 8 independent chains.
-      // One pair in EXP2_POLY_EVERY is evaluated on the FMA pipe (exp2_poly)
-      // instead of the MUFU unit, whose exponentials bound this loop.
-      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      // product; the row sum adds the f32 values in independent chains.
+      // One pair in EXP2_POLY_EVERY is evaluated on the FMA pipe instead of
+      // the MUFU unit, whose exponentials bound this loop.
       uint32_t pk0[32], pk1[32];
+#if TP_ATTN_X2
+      // Scaling and the row sum on pairs of lanes (f32x2): half the FMA-pipe
+      // instructions.
+      const unsigned long long sc2 = f2_pack(a.scale_log2, a.scale_log2);
+      const unsigned long long nm2 = f2_pack(-m_run, -m_run);
+      unsigned long long sum4[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+      for (int e = 0; e < BKV; e += 2) {
+        const bool poly = EXP2_POLY_EVERY > 0 && (e / 2) % EXP2_POLY_MOD == EXP2_POLY_MOD - 1;
+        float x0, x1, p0, p1;
+        f2_unpack(f2_fma(f2_pack(s[e], s[e + 1]), sc2, nm2), x0, x1);
+        if (poly) {
+          exp2_poly3_pair(x0, x1, p0, p1);
+        } else {
+          p0 = exp2_fast(x0);
+          p1 = exp2_fast(x1);
+        }
+        sum4[(e / 2) & 3] = f2_add(sum4[(e / 2) & 3], f2_pack(p0, p1));
+        if (e < 64) pk0[e / 2] = pack_bf16x2(p0, p1);
+        else pk1[(e - 64) / 2] = pack_bf16x2(p0, p1);
+      }
+      float sum;
+      {
+        float a0, a1;
+        f2_unpack(f2_add(f2_add(sum4[0], sum4[1]), f2_add(sum4[2], sum4[3])), a0, a1);
+        sum = a0 + a1;
+      }
+#else
+      float sum8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int e = 0; e < BKV; e += 2) {
         const bool poly = EXP2_POLY_EVERY > 0 && (e / 2) % EXP2_POLY_MOD == EXP2_POLY_MOD - 1;
@@ -331,6 +373,7 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
         else pk1[(e - 64) / 2] = pack_bf16x2(p0, p1);
       }
       const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) + ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+#endif
       l_run = l_run * alpha + sum;
       if (j > 0) {
         // P_t(j-1) V_{j-1} must be done before P_t(j) replaces it and O_t is

@@ -451,11 +451,82 @@ __device__ __forceinline__ float exp2_poly(float x) {
   return __int_as_float(__float_as_int(p) + (n << 23));
 }
 
-// Diagnostic: exp2_poly and CUDA's exp2f side by side on n inputs.
-__global__ void selftest_exp2_kernel(const float* x, float* y_poly, float* y_ref, int n) {
+// ------------------------------------------------ packed f32 pairs (f32x2)
+// sm_100 executes add / mul / fma on two f32 lanes of a 64-bit register pair
+// in one instruction; the softmax uses them to halve its FMA-pipe work.
+__device__ __forceinline__ unsigned long long f2_pack(float a, float b) {
+  unsigned long long v;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(a), "f"(b));
+  return v;
+}
+
+__device__ __forceinline__ void f2_unpack(unsigned long long v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+
+__device__ __forceinline__ unsigned long long f2_fma(unsigned long long a, unsigned long long b,
+                                                     unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+
+__device__ __forceinline__ unsigned long long f2_add(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+__device__ __forceinline__ unsigned long long f2_sub(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair of f32 values on the FMA pipe, for the share of a
+// softmax's exponentials moved off the MUFU unit.  As exp2_poly, x = n + f
+// with n = round(x) and f in [-1/2, 1/2], but 2^f from a degree-3 polynomial
+// (coefficients fitted here for minimax relative error on [-1/2, 1/2] by the
+// Remez exchange: max relative error 7.5e-5, far below the bf16 rounding of
+// the P it feeds), evaluated on both lanes at once with f32x2 arithmetic.
+// 2^n goes into the exponent field: the bits of t = x + 1.5 * 2^23 are those
+// of 1.5 * 2^23 plus n, and (those bits << 23) is 0 mod 2^32, so adding
+// (bits(t) << 23) to the bits of 2^f adds n to its exponent.  x is clamped at
+// -125 (2^-125, not 0, below that) and must be at most 64.
+__device__ __forceinline__ void exp2_poly3_pair(float x0, float x1, float& y0, float& y1) {
+  const unsigned long long magic = f2_pack(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+  const unsigned long long x = f2_pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const unsigned long long t = f2_add(x, magic);
+  const unsigned long long f = f2_sub(x, f2_sub(t, magic));
+  unsigned long long p = f2_fma(f2_pack(0.0551716685f, 0.0551716685f), f, f2_pack(0.242611125f, 0.242611125f));
+  p = f2_fma(p, f, f2_pack(0.693260968f, 0.693260968f));
+  p = f2_fma(p, f, f2_pack(0.999928057f, 0.999928057f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
+// Diagnostic: a polynomial 2^x (degree 4 single, or the degree-3 pair form
+// the attention kernel uses) and CUDA's exp2f side by side on n inputs.
+__global__ void selftest_exp2_kernel(const float* x, float* y_poly, float* y_ref, int n, int pair) {
   for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) {
-    y_poly[i] = exp2_poly(x[i]);
     y_ref[i] = exp2f(x[i]);
+    if (!pair) {
+      y_poly[i] = exp2_poly(x[i]);
+    } else if ((i & 1) == 0) {  // inputs i and i + 1 on the two lanes
+      float y1;
+      exp2_poly3_pair(x[i], i + 1 < n ? x[i + 1] : x[i], y_poly[i], y1);
+      if (i + 1 < n) y_poly[i + 1] = y1;
+    }
   }
 }
 

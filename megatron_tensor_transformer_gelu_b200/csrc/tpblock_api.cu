@@ -2049,13 +2049,17 @@ int tp_selftest_flag_wait_timeout(long long limit_cycles, void* stream) {
 }
 
 int tp_selftest_exp2(const float* x, float* y_poly, float* y_exp2f, int n, void* stream) {
-  if (n < 0 || (n > 0 && (!x || !y_poly || !y_exp2f))) return TP_ERR_INVALID_ARG;
+  return tp_selftest_exp2_form(x, y_poly, y_exp2f, n, 0, stream);
+}
+
+int tp_selftest_exp2_form(const float* x, float* y_poly, float* y_exp2f, int n, int form, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y_poly || !y_exp2f)) || form < 0 || form > 1) return TP_ERR_INVALID_ARG;
   DeviceInfo* dev = nullptr;
   int st = device_ready(&dev);
   if (st != TP_OK) return st;
   if (n == 0) return TP_OK;
   const int blocks = ceil_div(n, 256) < 4 * dev->sm_count ? ceil_div(n, 256) : 4 * dev->sm_count;
-  tp::selftest_exp2_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_exp2f, n);
+  tp::selftest_exp2_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y_poly, y_exp2f, n, form);
   return launch_status();
 }
 

@@ -138,7 +138,9 @@ int tp_mlp_forward_ex(int S, int H, int F, int t, int dtype, int out_dtype, int 
  *
  * tp_mlp_forward_train: tp_mlp_forward (dtype bf16 only) that also keeps, in
  * the caller's `state` (>= tp_mlp_train_state_bytes()), what the backward
- * reads: U [S, F] bf16 (pre-activation), G [S, F] bf16 and V [S, H] f32.
+ * reads: U [S, F] bf16 (pre-activation), G [S, F] bf16, V [S, H] f32 and the
+ * LayerNorm's row statistics ([S][2] f32: each row's mean and
+ * 1/sqrt(var + eps), so the backward normalises with the forward's values).
  * Y is the same as tp_mlp_forward's up to rounding.
  *
  * tp_mlp_backward: from the same X, shards, gamma, eps, act and the state of
@@ -237,8 +239,9 @@ int tp_qkv_attn_oproj_forward_ex(int S, int H, int nh, int d, int t, int dtype, 
  *
  * tp_attn_forward_train: tp_qkv_attn_oproj_forward that also keeps, in the
  * caller's `state` (>= tp_attn_train_state_bytes()), QKV [S, 3H] bf16, O
- * [S, H] bf16, O Wo [S, H] f32 and each row's log2 softmax denominator per
- * head [nh, S] f32 (P is rebuilt from it in the backward).
+ * [S, H] bf16, O Wo [S, H] f32, each row's log2 softmax denominator per
+ * head [nh, S] f32 (P is rebuilt from it in the backward) and the
+ * LayerNorm's row statistics ([S][2] f32, as tp_mlp_forward_train).
  *
  * tp_attn_backward: from the same X, shards, gamma, eps and the state of one
  * tp_attn_forward_train call, and dY [S, H] bf16, writes dX [S, H] bf16,

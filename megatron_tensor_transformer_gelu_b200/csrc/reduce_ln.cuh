@@ -57,6 +57,7 @@ struct ReduceLnArgs {
   int ny_extra;               // further copies of Y written (the all-gather's stores), 0..RLN_MAX_PTRS-1
   void* y_extra[RLN_MAX_PTRS];
   int apply_ln;               // 0: Y = X + sum_p P_p only (pre-LN residual stream)
+  float* stats;               // optional [S][2]: each row's (mean, 1/sqrt(var + eps)), for a backward pass
 };
 
 __device__ __forceinline__ void load8_bf16(const __nv_bfloat16* src, float* v) {
@@ -245,6 +246,8 @@ __global__ void __launch_bounds__(rln::cta_threads(WPR), (TP_RLN_LEAN && rln::ct
     }
     const float var = tot2 / static_cast<float>(p.H);
     const float rstd = 1.0f / sqrtf(var + p.eps);
+    if (p.stats && live && wr == 0 && lane == 0)
+      *reinterpret_cast<float2*>(p.stats + 2 * row) = make_float2(mean, rstd);
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int col = ((c * WPR + wr) * 32 + lane) * 8;
@@ -411,6 +414,7 @@ __global__ void __launch_bounds__(rlb::THREADS) reduce_residual_ln_bulk_kernel(c
 #pragma unroll
     for (int w = 0; w < rlb::WARPS; ++w) tot2 += red[i & 1][1][w];
     const float rstd = 1.0f / sqrtf(tot2 * inv_h + p.eps);
+    if (p.stats && tid == 0) *reinterpret_cast<float2*>(p.stats + 2 * row) = make_float2(mean, rstd);
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int col = (c * rlb::THREADS + tid) * 8;

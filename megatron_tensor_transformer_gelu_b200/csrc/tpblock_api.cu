@@ -666,11 +666,12 @@ int run_gemm_simt(const float* A, long long lda, int M, const void* const* B, in
 int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, int x_bf16, const float* gamma,
                   const float* beta, float eps, void* Y, int y_bf16, cudaStream_t st, int dev_sms,
                   int apply_ln = 1, const float* const* part_list = nullptr, int ny_extra = 0,
-                  void* const* y_extra = nullptr) {
+                  void* const* y_extra = nullptr, float* stats = nullptr) {
   if (S == 0) return TP_OK;
   tp::ReduceLnArgs p;
   std::memset(&p, 0, sizeof(p));
   p.apply_ln = apply_ln;
+  p.stats = stats;
   p.S = S;
   p.H = H;
   p.nparts = nparts;
@@ -788,10 +789,11 @@ bool hidden_ok(int H) { return H >= 8 && H % 8 == 0 && H <= tp::rln::MAX_H; }
 
 // ------------------------------------------------------------ training state
 // Saved by tp_mlp_forward_train for tp_mlp_backward: U = X A (pre-activation,
-// bf16 [S, F]), G = Act(U) (bf16 [S, F], the row-split GEMM's input) and
-// V = G B (f32 [S, H], the row-split GEMM's output before the residual).
+// bf16 [S, F]), G = Act(U) (bf16 [S, F], the row-split GEMM's input),
+// V = G B (f32 [S, H], the row-split GEMM's output before the residual) and
+// the LayerNorm's row statistics (mean, 1/sqrt(var + eps); f32 [S][2]).
 struct TrainState {
-  size_t off_u, off_g, off_v, bytes;
+  size_t off_u, off_g, off_v, off_stats, bytes;
 };
 TrainState train_state_layout(int S, int H, int F) {
   TrainState t;
@@ -799,14 +801,15 @@ TrainState train_state_layout(int S, int H, int F) {
   t.off_u = 0;
   t.off_g = align256(sf * 2);
   t.off_v = t.off_g + align256(sf * 2);
-  t.bytes = t.off_v + align256(sh * 4);
+  t.off_stats = t.off_v + align256(sh * 4);
+  t.bytes = t.off_stats + align256(static_cast<size_t>(S) * 8);
   return t;
 }
 
 // Backward workspace: dZ (bf16 [S, H]), dU (bf16 [S, F]), the f32 row-split
 // partial of dX ([S, H]) and the LayerNorm-backward CTAs' dgamma/dbeta partial
 // rows (at most LNB_MAX_CTAS x 2 x H f32).
-constexpr int LNB_MAX_CTAS = 320;
+constexpr int LNB_MAX_CTAS = 640;
 struct BackWs {
   size_t off_dz, off_du, off_dxp, off_part, bytes;
 };
@@ -821,80 +824,54 @@ BackWs back_ws_layout(int S, int H, int F) {
   return w;
 }
 
-// LayerNorm backward + the dgamma/dbeta reduction.  Chunks of 8 per thread:
-// CH = ceil(H / 8 / 512) (1..4), threads = the chunks per CH rounded up to a
-// warp; CTAs = as many as fit two per SM's worth of threads (at most
-// LNB_MAX_CTAS, at most S).
-int run_ln_backward(int S, int H, const float* V, const void* X, const void* dY, const float* gamma, float eps,
-                    void* dZ, float* partial, float* dgamma, float* dbeta, cudaStream_t st, int dev_sms) {
+// LayerNorm backward + the dgamma/dbeta reduction.  256-thread CTAs, one row
+// at a time each, CH = ceil(H / 2048) chunks of 8 per thread; as many CTAs as
+// are resident (at most LNB_MAX_CTAS, at most S), each with 8 H bytes of
+// shared memory for its per-column sums.  stats: the forward's row (mean, r).
+int run_ln_backward(int S, int H, const float* V, const float* stats, const void* X, const void* dY,
+                    const float* gamma, void* dZ, float* partial, float* dgamma, float* dbeta, cudaStream_t st,
+                    int dev_sms) {
   tp::LnBackArgs p;
   p.S = S;
   p.H = H;
-  p.nparts = 1;
-  p.parts = V;
-  p.part_stride = static_cast<long long>(S) * H;
+  p.V = V;
+  p.stats = stats;
   p.X = static_cast<const __nv_bfloat16*>(X);
   p.dY = static_cast<const __nv_bfloat16*>(dY);
   p.gamma = gamma;
-  p.eps = eps;
   p.dZ = static_cast<__nv_bfloat16*>(dZ);
   p.partial = partial;
-  const int chunks = H / 8;
-  const int ch = ceil_div(chunks, 512);
-  const int threads = ceil_div(ceil_div(chunks, ch), 32) * 32;
-  int grid = (2048 / threads) * dev_sms / 2;
-  if (grid > LNB_MAX_CTAS) grid = LNB_MAX_CTAS;
-  if (grid > S) grid = S;
-  if (grid < 1) grid = 1;
-  // Rows staged in shared memory by bulk copies (X, dY, V: 8 bytes a column),
-  // 2 to 4 stages; rows too wide for two stages take the register kernel.
-  const size_t stage = (static_cast<size_t>(H) * 8 + 127) & ~size_t(127);
-  const bool bulk = TP_RLN_BULK && 2 * stage <= static_cast<size_t>(tp::rlb::MAX_STAGE_SMEM);
-  if (bulk) {
-    const size_t budget = stage <= 32 * 1024 ? 96 * 1024 : tp::rlb::MAX_STAGE_SMEM;
-    int nst = static_cast<int>(budget / stage);
-    nst = nst < 2 ? 2 : (nst > 4 ? 4 : nst);
-    const size_t smem = static_cast<size_t>(nst) * stage;
-    cudaError_t le = cudaSuccess;
-    auto go = [&](auto kern) {
-      int per_sm = 1;
-      if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-              cudaSuccess ||
-          cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, tp::lnbb::THREADS, smem) != cudaSuccess ||
-          per_sm < 1)
-        per_sm = 1;
-      grid = per_sm * dev_sms;
-      if (grid > LNB_MAX_CTAS) grid = LNB_MAX_CTAS;
-      if (grid > S) grid = S;
-      le = launch_pdl(kern, dim3(grid), dim3(tp::lnbb::THREADS), smem, st, p, nst, static_cast<int>(stage));
-    };
+  const size_t smem = static_cast<size_t>(H) * 8;
+  int grid = 0;
+  cudaError_t le = cudaSuccess;
+  auto go = [&](auto kern) {
+    int per_sm = 1;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, tp::lnb::THREADS, smem) != cudaSuccess ||
+        per_sm < 1)
+      per_sm = 1;
+    grid = per_sm * dev_sms;
+    if (grid > LNB_MAX_CTAS) grid = LNB_MAX_CTAS;
+    if (grid > S) grid = S;
+    le = launch_pdl(kern, dim3(grid), dim3(tp::lnb::THREADS), smem, st, p);
+  };
+  {
     ProfScope ps(K_LN_BACK, st);
     switch ((H + 2047) / 2048) {
-      case 1: go(tp::ln_backward_bulk_kernel<1>); break;
-      case 2: go(tp::ln_backward_bulk_kernel<2>); break;
-      case 3: go(tp::ln_backward_bulk_kernel<3>); break;
-      case 4: go(tp::ln_backward_bulk_kernel<4>); break;
-      case 5: case 6: go(tp::ln_backward_bulk_kernel<6>); break;
-      default: go(tp::ln_backward_bulk_kernel<8>); break;
-    }
-    if (le != cudaSuccess || launch_status() != TP_OK) return TP_ERR_CUDA;
-  } else {
-    ProfScope ps(K_LN_BACK, st);
-    cudaError_t le;
-    switch (ch) {
-      case 1: le = launch_pdl(tp::ln_backward_kernel<1>, dim3(grid), dim3(threads), 0, st, p); break;
-      case 2: le = launch_pdl(tp::ln_backward_kernel<2>, dim3(grid), dim3(threads), 0, st, p); break;
-      case 3: le = launch_pdl(tp::ln_backward_kernel<3>, dim3(grid), dim3(threads), 0, st, p); break;
-      default: le = launch_pdl(tp::ln_backward_kernel<4>, dim3(grid), dim3(threads), 0, st, p); break;
+      case 1: go(tp::ln_backward_kernel<1>); break;
+      case 2: go(tp::ln_backward_kernel<2>); break;
+      case 3: case 4: go(tp::ln_backward_kernel<4>); break;
+      default: go(tp::ln_backward_kernel<8>); break;
     }
     if (le != cudaSuccess || launch_status() != TP_OK) return TP_ERR_CUDA;
   }
   if (dgamma || dbeta) {
     ProfScope ps(K_LN_PARAMS, st);
-    const cudaError_t le = launch_pdl(tp::ln_grad_params_kernel, dim3(ceil_div(H, 32)),
+    const cudaError_t pe = launch_pdl(tp::ln_grad_params_kernel, dim3(ceil_div(H, 32)),
                                       dim3(32 * tp::LNB_PARAM_SLICES), 0, st, static_cast<const float*>(partial),
                                       grid, H, dgamma, dbeta);
-    return le != cudaSuccess ? TP_ERR_CUDA : launch_status();
+    return pe != cudaSuccess ? TP_ERR_CUDA : launch_status();
   }
   return TP_OK;
 }
@@ -1004,6 +981,7 @@ struct AttnKeep {
   void* o = nullptr;
   float* zsum = nullptr;
   float* lse2 = nullptr;
+  float* stats = nullptr;  // the LayerNorm's row (mean, 1/sqrt(var + eps))
 };
 
 // QKV, per-head attention and the row-split O projection of the nh heads held
@@ -1121,7 +1099,7 @@ int attn_core(const DeviceInfo& dev, int S, int H, int nh, int d, int t, int out
                          keep ? sh4 : TP_MAX_K_SPLITS * sh4);
   if (st != TP_OK) return st;
   return run_reduce_ln(S, H, nparts, Zsum, res, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s, dev.sm_count,
-                       apply_ln);
+                       apply_ln, nullptr, 0, nullptr, keep ? keep->stats : nullptr);
 }
 
 int check_mlp_args(int S, int H, int F, int t, int dtype, int out_dtype, const void* X, const void* const* A_shards,
@@ -1235,7 +1213,8 @@ int tp_mlp_forward_train_ex(int S, int H, int F, int t, int dtype, int out_dtype
   // V = sum_i G_i B_i in one f32 slot (no K split: the backward reads one).
   st = run_gemm_tc(*dev, G, F, S, B_shards, t, 1, Fs, H, V, H, 1, TP_ACT_NONE, s, 1, 0, nullptr, kmaj);
   if (st != TP_OK) return st;
-  return run_reduce_ln(S, H, 1, V, X, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s, dev->sm_count);
+  return run_reduce_ln(S, H, 1, V, X, 1, gamma, beta, eps, Y, out_dtype == TP_DTYPE_BF16, s, dev->sm_count, 1,
+                       nullptr, 0, nullptr, reinterpret_cast<float*>(base + L.off_stats));
 }
 
 size_t tp_mlp_backward_workspace_bytes(int S, int H, int F, int t, int dtype) {
@@ -1285,7 +1264,8 @@ int tp_mlp_backward_ex(int S, int H, int F, int t, int dtype, int w_layout, cons
   float* part = reinterpret_cast<float*>(wb + W.off_part);
   const int Fs = F / t;
   // 1. Through the LayerNorm: dZ, dgamma, dbeta.
-  st = run_ln_backward(S, H, V, X, dY, gamma, eps, dZ, part, dgamma, dbeta, s, dev->sm_count);
+  const float* stats = reinterpret_cast<const float*>(sb + L.off_stats);
+  st = run_ln_backward(S, H, V, stats, X, dY, gamma, dZ, part, dgamma, dbeta, s, dev->sm_count);
   if (st != TP_OK) return st;
   // In [out, in] storage (TP_W_OUT_IN) every weight is the transpose of its
   // [in, out] form: the backward reads B_i and A_i with the other majorness,
@@ -1388,7 +1368,7 @@ int tp_qkv_attn_oproj_forward_ex(int S, int H, int nh, int d, int t, int dtype, 
 // ------------------------------------------------- attention training step
 namespace {
 struct AttnState {
-  size_t off_qkv, off_o, off_z, off_lse, bytes;
+  size_t off_qkv, off_o, off_z, off_lse, off_stats, bytes;
 };
 AttnState attn_state_layout(int S, int H, int nh) {
   AttnState a;
@@ -1397,7 +1377,8 @@ AttnState attn_state_layout(int S, int H, int nh) {
   a.off_o = align256(s * 3 * h * 2);
   a.off_z = a.off_o + align256(s * h * 2);
   a.off_lse = a.off_z + align256(s * h * 4);
-  a.bytes = a.off_lse + align256(static_cast<size_t>(nh) * s * 4);
+  a.off_stats = a.off_lse + align256(static_cast<size_t>(nh) * s * 4);
+  a.bytes = a.off_stats + align256(s * 8);
   return a;
 }
 struct AttnBackWs {
@@ -1452,6 +1433,7 @@ int tp_attn_forward_train(int S, int H, int nh, int d, int t, int dtype, int out
   keep.o = b + L.off_o;
   keep.zsum = reinterpret_cast<float*>(b + L.off_z);
   keep.lse2 = reinterpret_cast<float*>(b + L.off_lse);
+  keep.stats = reinterpret_cast<float*>(b + L.off_stats);
   return attn_core(*dev, S, H, nh, d, t, out_dtype, X, X, Wqkv_shards, Wo_shards, gamma, beta, eps, 1, Y, nullptr,
                    static_cast<cudaStream_t>(stream), 0, &keep);
 }
@@ -1498,7 +1480,8 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
   float* D = reinterpret_cast<float*>(wb + W.off_d);
   float* part = reinterpret_cast<float*>(wb + W.off_part);
   // 1. Through the LayerNorm: dZ, dgamma, dbeta (Z = X + the O projection's output).
-  st = run_ln_backward(S, H, Vo, X, dY, gamma, eps, dZ, part, dgamma, dbeta, s, dev->sm_count);
+  const float* stats = reinterpret_cast<const float*>(sb + L.off_stats);
+  st = run_ln_backward(S, H, Vo, stats, X, dY, gamma, dZ, part, dgamma, dbeta, s, dev->sm_count);
   if (st != TP_OK) return st;
   // 2. Through the O projection: dO_s = dZ Wo_s^T (Wo_s [Hs, H] read K-major)
   //    into shard s's head columns of dO, and dWo_s = O_s^T dZ.

@@ -76,10 +76,10 @@ def test_workspace_sizes(lib):
 
 def test_attention_backward_workspace_holds_a_head_group(lib):
     """dZ, dO, dQKV (bf16), the f32 row-split partial, the [S, S] P and dS
-    matrices (bf16) of a group of heads, D [nh, S] and 320 per-CTA LayerNorm
+    matrices (bf16) of a group of heads, D [nh, S] and 640 per-CTA LayerNorm
     partial rows: 8 heads a group unless nh < 8 or 8 would pass 1 GiB."""
     def expect(S, H, nh, g):
-        return S * H * (2 + 2 + 6 + 4) + g * S * S * 4 + nh * S * 4 + 320 * 2 * H * 4
+        return S * H * (2 + 2 + 6 + 4) + g * S * S * 4 + nh * S * 4 + 640 * 2 * H * 4
     lib.tp_attn_backward_workspace_bytes.restype = ctypes.c_size_t
     assert lib.tp_attn_backward_workspace_bytes(2048, 8192, 64, 128, 4, 1) == expect(2048, 8192, 64, 8)
     assert lib.tp_attn_backward_workspace_bytes(256, 512, 4, 128, 2, 1) == expect(256, 512, 4, 4)
@@ -160,7 +160,7 @@ def test_training_argument_checks(lib):
     pda, kda = _ptrs(t)
     pdb, kdb = _ptrs(t)
     st_bytes = lib.tp_mlp_train_state_bytes(S, H, F, t, 1)
-    assert st_bytes == 2 * S * F * 2 + S * H * 4
+    assert st_bytes == 2 * S * F * 2 + S * H * 4 + S * 8  # U, G, V and the LayerNorm's row statistics
     assert lib.tp_mlp_train_state_bytes(S, H, F, t, 0) == 0      # f32 storage has no training path
     ws_bytes = lib.tp_mlp_backward_workspace_bytes(S, H, F, t, 1)
     assert ws_bytes >= S * H * 2 + S * F * 2 + S * H * 4

@@ -79,8 +79,11 @@ __device__ __forceinline__ void lnb_load8_bf16(const __nv_bfloat16* src, float (
 // dbeta's), so a thread's read-modify-write of its own chunk is conflict-free.
 // The row reduction's scratch is double-buffered by row parity, so one
 // barrier per row suffices.
+#ifndef TP_LNB_MIN_BLOCKS
+#define TP_LNB_MIN_BLOCKS 1  // CTAs per SM the register budget of the 1- and 2-chunk kernels is sized for
+#endif
 template <int CH>
-__global__ void __launch_bounds__(lnb::THREADS) ln_backward_kernel(const LnBackArgs p) {
+__global__ void __launch_bounds__(lnb::THREADS, CH <= 2 ? TP_LNB_MIN_BLOCKS : 1) ln_backward_kernel(const LnBackArgs p) {
   extern __shared__ float4 lnb_acc[];  // [4][H / 8]
   __shared__ float red[2][2][lnb::WARPS];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -187,10 +190,11 @@ __global__ void __launch_bounds__(lnb::THREADS) ln_backward_kernel(const LnBackA
 
 // dgamma[j] = sum_b partial[b][0][j], dbeta[j] = sum_b partial[b][1][j].
 // A CTA takes 32 columns with 32 warps: warp w sums the partial rows
-// b = w, w + 32, ... (each load a 128-byte row segment, four rows in flight
+// b = w, w + 32, ... (each load a 128-byte row segment, eight rows in flight
 // in separate accumulators added in a fixed order), then warp 0 adds the 32
 // warps' sums in warp order, so the result is deterministic.
 constexpr int LNB_PARAM_SLICES = 32;
+constexpr int LNB_PARAM_UNROLL = 8;
 __global__ void __launch_bounds__(32 * LNB_PARAM_SLICES)
     ln_grad_params_kernel(const float* partial, int nblk, int H, float* dgamma, float* dbeta) {
   __shared__ float sa[LNB_PARAM_SLICES][33], sb[LNB_PARAM_SLICES][33];
@@ -198,13 +202,15 @@ __global__ void __launch_bounds__(32 * LNB_PARAM_SLICES)
   griddep_wait();  // the partial rows come from the preceding kernel
   griddep_launch_dependents();
   const int j = blockIdx.x * 32 + lane;
-  float a[4] = {0.0f, 0.0f, 0.0f, 0.0f}, b[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  float a[LNB_PARAM_UNROLL], b[LNB_PARAM_UNROLL];
+#pragma unroll
+  for (int u = 0; u < LNB_PARAM_UNROLL; ++u) a[u] = b[u] = 0.0f;
   if (j < H) {
     const long long step = 2LL * H;
     int k = slice;
-    for (; k + 3 * LNB_PARAM_SLICES < nblk; k += 4 * LNB_PARAM_SLICES) {
+    for (; k + (LNB_PARAM_UNROLL - 1) * LNB_PARAM_SLICES < nblk; k += LNB_PARAM_UNROLL * LNB_PARAM_SLICES) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < LNB_PARAM_UNROLL; ++u) {
         const float* row = partial + (k + u * LNB_PARAM_SLICES) * step;
         a[u] += row[j];
         b[u] += row[H + j];
@@ -215,18 +221,24 @@ __global__ void __launch_bounds__(32 * LNB_PARAM_SLICES)
       b[0] += partial[k * step + H + j];
     }
   }
-  sa[slice][lane] = (a[0] + a[1]) + (a[2] + a[3]);
-  sb[slice][lane] = (b[0] + b[1]) + (b[2] + b[3]);
+  float ta = 0.0f, tb = 0.0f;
+#pragma unroll
+  for (int u = 0; u < LNB_PARAM_UNROLL; ++u) {
+    ta += a[u];
+    tb += b[u];
+  }
+  sa[slice][lane] = ta;
+  sb[slice][lane] = tb;
   __syncthreads();
   if (slice == 0 && j < H) {
-    float ta = 0.0f, tb = 0.0f;
+    float sa_t = 0.0f, sb_t = 0.0f;
 #pragma unroll 8
     for (int w = 0; w < LNB_PARAM_SLICES; ++w) {
-      ta += sa[w][lane];
-      tb += sb[w][lane];
+      sa_t += sa[w][lane];
+      sb_t += sb[w][lane];
     }
-    if (dgamma) dgamma[j] = ta;
-    if (dbeta) dbeta[j] = tb;
+    if (dgamma) dgamma[j] = sa_t;
+    if (dbeta) dbeta[j] = sb_t;
   }
 }
 

@@ -563,7 +563,9 @@ def run_ours(args, rank, world, local):
                 h2d.wait_event(ev_down[b])
             last.record(h2d)
 
-    e2e_steps = max(nbuf, min(args.steps, 200))
+    # As many steps as the timed region of `value`: under the power cap a
+    # shorter run is not comparable (it ends before the clocks settle).
+    e2e_steps = max(nbuf, args.steps)
     e2e_run(max(nbuf, min(args.warmup, 5)))
     barrier()
     f0 = torch.cuda.Event(enable_timing=True)

@@ -80,7 +80,7 @@ enum : int { ACT_NONE = 0, ACT_GELU_TANH = 1, ACT_GELU_ERF = 2, ACT_RELU = 3 };
 // FEAT_SK (stream-K), FEAT_DUAL (dual accumulators).
 enum : int { FEAT_BASE = 0, FEAT_SK = 1, FEAT_DUAL = 2 };
 
-template <int CG, bool WIDE = false>
+template <int CG, bool WIDE = false, int FEAT = FEAT_BASE>
 struct GemmCfg {
   static constexpr int BM = 128;                    // accumulator rows per CTA
   static constexpr int TILE_M = BM * CG;            // rows per (cluster) tile
@@ -106,7 +106,11 @@ struct GemmCfg {
 #define TP_GEMM_WARP_STORES 0
 #endif
   static_assert(!WIDE || CG == 2, "wide tiles need a CTA pair");
-  static constexpr int STAGES = WIDE ? TP_GEMM_WIDE_STAGES : (CG == 2 ? TP_GEMM_PAIR_STAGES : 4);
+  // The dual-accumulator tiles have 4 k-blocks: fewer stages (5 for a pair,
+  // 3 for a single CTA, whose B stage is twice as large), and the shared
+  // memory that frees goes to a second pair of epilogue staging buffers.
+  static constexpr int STAGES =
+      FEAT == FEAT_DUAL ? (CG == 2 ? 5 : 3) : (WIDE ? TP_GEMM_WIDE_STAGES : (CG == 2 ? TP_GEMM_PAIR_STAGES : 4));
   static constexpr int PREFETCH = TP_GEMM_L2_PREFETCH;  // k-blocks ahead (0 = off)
   static constexpr int A_BYTES = BM * BK * 2;       // 16 KiB
   static constexpr int B_BOX_N = 64;                // 64 bf16 = one 128-byte swizzle row
@@ -119,11 +123,14 @@ struct GemmCfg {
   static constexpr int ACC_BUFS = WIDE ? 1 : 2;     // accumulators in TMEM
   static constexpr int NUM_THREADS = 192;
   static constexpr int TMEM_COLS = 512;
-  // Epilogue staging: two buffers of 128 rows x 128 bytes (32 f32 or 64 bf16
-  // columns), 128-byte swizzled, drained by TMA stores.
+  // Epilogue staging: buffers of 128 rows x 128 bytes (32 f32 or 64 bf16
+  // columns), 128-byte swizzled, drained by TMA stores: two, used in turn;
+  // four for the dual tiles (a P and a dS buffer, two pairs used in turn).
   static constexpr int EPI_BUF_BYTES = BM * 128;
+  static constexpr int EPI_BUFS = FEAT == FEAT_DUAL ? 4 : 2;
   static constexpr int SMEM_BYTES =
-      STAGES * (A_BYTES + B_BYTES) + 2 * EPI_BUF_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+      STAGES * (A_BYTES + B_BYTES) + EPI_BUFS * EPI_BUF_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+  static_assert(SMEM_BYTES <= 232448, "more dynamic shared memory than a CTA may have");
   static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN, /*a_mn=*/false, /*b_mn=*/true);
   // B given K-major ([out, in] weights): one box of B_COLS_CTA rows x 64 k.
   static constexpr uint32_t IDESC_BK = idesc_bf16_f32(TILE_M, BN, /*a_mn=*/false, /*b_mn=*/false);
@@ -509,6 +516,11 @@ __device__ __forceinline__ void epi_chunk_dsoftmax(uint32_t taddr, uint8_t* stag
 __device__ __forceinline__ void epi_chunk_dual_softmax(uint32_t taddr, uint8_t* stage_p, uint8_t* stage_ds,
                                                        int row_local, float r1, float scale1, float r2,
                                                        float scale2) {
+  // P = 2^(s scale1 - r1) with the forward softmax's exponential (ex2.approx,
+  // so P is rebuilt as the forward made it), dS = (P (dp - r2)) scale2; the
+  // arithmetic on f32 pairs (f32x2), two columns per instruction.
+  const unsigned long long sc = f2_pack(scale1, scale1), nr = f2_pack(-r1, -r1);
+  const unsigned long long d2 = f2_pack(r2, r2), s2 = f2_pack(scale2, scale2);
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     uint32_t sv[32], dv[32];
@@ -521,11 +533,14 @@ __device__ __forceinline__ void epi_chunk_dual_softmax(uint32_t taddr, uint8_t* 
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int i0 = 8 * j + 2 * e;
-        const float p0 = exp2f(fmaf(__uint_as_float(sv[i0]), scale1, -r1));
-        const float p1 = exp2f(fmaf(__uint_as_float(sv[i0 + 1]), scale1, -r1));
+        float x0, x1, q0, q1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[i0]), __uint_as_float(sv[i0 + 1])), sc, nr), x0, x1);
+        const float p0 = exp2_fast(x0), p1 = exp2_fast(x1);
         wp[e] = pack_bf16x2(p0, p1);
-        wd[e] = pack_bf16x2(p0 * (__uint_as_float(dv[i0]) - r2) * scale2,
-                            p1 * (__uint_as_float(dv[i0 + 1]) - r2) * scale2);
+        const unsigned long long g =
+            f2_sub(f2_pack(__uint_as_float(dv[i0]), __uint_as_float(dv[i0 + 1])), d2);
+        f2_unpack(f2_mul(f2_mul(f2_pack(p0, p1), g), s2), q0, q1);
+        wd[e] = pack_bf16x2(q0, q1);
       }
       const int off = ((4 * h + j) ^ (row_local & 7)) << 4;
       *reinterpret_cast<uint4*>(stage_p + off) = make_uint4(wp[0], wp[1], wp[2], wp[3]);
@@ -682,14 +697,14 @@ __device__ __forceinline__ int b2_boxes_for(int n_valid, int n2, int rank, int b
 
 template <int CG, bool WIDE = false, int FEAT = FEAT_BASE>
 __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kernel(const __grid_constant__ GemmArgs p) {
-  using C = GemmCfg<CG, WIDE>;
+  using C = GemmCfg<CG, WIDE, FEAT>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * C::A_BYTES;
-  uint8_t* sEpi = sB + STAGES * C::B_BYTES;  // 2 x EPI_BUF_BYTES
-  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + 2 * C::EPI_BUF_BYTES);
+  uint8_t* sEpi = sB + STAGES * C::B_BYTES;  // EPI_BUFS x EPI_BUF_BYTES
+  uint64_t* full = reinterpret_cast<uint64_t*>(sEpi + C::EPI_BUFS * C::EPI_BUF_BYTES);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
@@ -1016,20 +1031,24 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
                            ? __ldg(p.rowvec + static_cast<long long>(tc.shard) * p.rowvec_ld + grow)
                            : 0.0f;
       if constexpr (FEAT == FEAT_DUAL) {
-        // P into staging buffer 0 and dS into buffer 1, then one store of each.
+        // P into staging buffer 2b and dS into 2b + 1, then one store of
+        // each (one bulk group); the pairs b = 0, 1 are used in turn, so a
+        // chunk is computed while the previous chunk's stores drain.
         const float rv2 = (p.rowvec2 != nullptr && grow < p.M)
                               ? __ldg(p.rowvec2 + static_cast<long long>(tc.shard) * p.rowvec_ld + grow)
                               : 0.0f;
         for (int c = 0; c < nchunks; ++c) {
+          uint8_t* sP = sEpi + (2 * buf) * C::EPI_BUF_BYTES;
+          uint8_t* sDS = sP + C::EPI_BUF_BYTES;
 #if TP_GEMM_WARP_STORES
-          if (lane == 0) bulk_wait_group_read<0>();
+          if (lane == 0) bulk_wait_group_read<1>();
           __syncwarp();
 #else
-          if (elected) bulk_wait_group_read<0>();
+          if (elected) bulk_wait_group_read<1>();
           named_barrier_sync(1, 128);
 #endif
-          epi_chunk_dual_softmax(t_row + c * 64, sEpi + row_local * 128, sEpi + C::EPI_BUF_BYTES + row_local * 128,
-                                 row_local, rv, p.epi_scale, rv2, p.epi_scale2);
+          epi_chunk_dual_softmax(t_row + c * 64, sP + row_local * 128, sDS + row_local * 128, row_local, rv,
+                                 p.epi_scale, rv2, p.epi_scale2);
           if (c == nchunks - 1) {
             tc_fence_before();
             if constexpr (CG == 1) {
@@ -1043,18 +1062,21 @@ __global__ void __launch_bounds__(GemmCfg<CG>::NUM_THREADS, 1) gemm_tcgen05_kern
 #if TP_GEMM_WARP_STORES
           __syncwarp();
           if (lane == 0 && y0 + q * 32 < p.M) {
-            tma_store_3d(tmC, sEpi + q * 32 * 128, tc.n_in + c * 64, ystore + q * 32, 0);
-            tma_store_3d(tmAux, sEpi + C::EPI_BUF_BYTES + q * 32 * 128, tc.n_in + c * 64, ystore + q * 32, 0);
-            bulk_commit_group();
+            tma_store_3d(tmC, sP + q * 32 * 128, tc.n_in + c * 64, ystore + q * 32, 0);
+            tma_store_3d(tmAux, sDS + q * 32 * 128, tc.n_in + c * 64, ystore + q * 32, 0);
           }
+          if (lane == 0) bulk_commit_group();  // an empty group keeps the count of groups per pair
 #else
           named_barrier_sync(1, 128);
-          if (elected && y0 < p.M) {
-            tma_store_3d(tmC, sEpi, tc.n_in + c * 64, ystore, 0);
-            tma_store_3d(tmAux, sEpi + C::EPI_BUF_BYTES, tc.n_in + c * 64, ystore, 0);
+          if (elected) {
+            if (y0 < p.M) {
+              tma_store_3d(tmC, sP, tc.n_in + c * 64, ystore, 0);
+              tma_store_3d(tmAux, sDS, tc.n_in + c * 64, ystore, 0);
+            }
             bulk_commit_group();
           }
 #endif
+          buf ^= 1;
         }
       } else {
         for (int c = 0; c < nchunks; ++c) {

@@ -111,7 +111,7 @@ int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b
 template <int CG, bool WIDE, int FEAT>
 bool gemm_smem_attr() {
   return cudaFuncSetAttribute(tp::gemm_tcgen05_kernel<CG, WIDE, FEAT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              tp::GemmCfg<CG, WIDE>::SMEM_BYTES) == cudaSuccess;
+                              tp::GemmCfg<CG, WIDE, FEAT>::SMEM_BYTES) == cudaSuccess;
 }
 
 // Resolve the current device's properties and the tensor-map encoder once.
@@ -452,7 +452,7 @@ struct GemmExtra {
 template <int CG, bool WIDE, int FEAT>
 int launch_gemm_tc(const DeviceInfo& dev, tp::GemmArgs& p, const TilePlan& plan, const GemmExtra& ex,
                    cudaStream_t st) {
-  using C = tp::GemmCfg<CG, WIDE>;
+  using C = tp::GemmCfg<CG, WIDE, FEAT>;
   p.m_blocks = ceil_div(p.M, C::TILE_M);
   p.tile_n = plan.tile_n;
   p.n2 = WIDE ? plan.tile_n - C::BN : 0;

@@ -59,9 +59,9 @@ def run_and_check(S, nh, t, seed, d=128):
 
 # The per-head GEMMs run over groups of up to 8 heads per launch: (256, 12, 4)
 # and (512, 10, 2) end on a partial group, with the group's heads spread over
-# several shards.
+# several shards.  S = 128 runs the score tiles on single CTAs instead of pairs.
 @pytest.mark.parametrize("S,nh,t", [(256, 2, 1), (384, 4, 2), (256, 4, 4), (512, 8, 2), (256, 12, 4),
-                                    (512, 10, 2)])
+                                    (512, 10, 2), (128, 2, 2)])
 def test_attention_backward_small(cuda_device, S, nh, t):
     run_and_check(S, nh, t, seed=S + nh + t)
 

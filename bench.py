@@ -213,7 +213,7 @@ def whole_job_tflops(flops_per_step: int, steps: int, world: int, ms_max: float)
     return world * flops_per_step * steps / (ms_max * 1e-3) / 1e12
 
 
-TENSOR_KINDS = ("gemm_tcgen05", "attention_fwd")
+TENSOR_KINDS = ("gemm_tcgen05", "attention_fwd", "attention_bwd")
 ALU_KINDS = ("gemm_simt_f32",)
 
 
@@ -345,8 +345,12 @@ class Problem:
             # Bytes of the backward's elementwise kernel: D = rowsum(dO * O) per
             # head reads dO and O once and writes D [nh, S] f32 (P and dS are
             # made in GEMM epilogues).
-            self.work = {"gemm_tcgen05": w.flops - att,          # every product but the fused forward attention
+            # The per-head products of the backward (the rebuilt scores, dV, dP,
+            # dQ and dK: 5 x att / 2) run in the two fused backward kernels,
+            # which also compute the scores and dP a second time (not counted).
+            self.work = {"gemm_tcgen05": w.flops - att - 5 * att // 2,   # the projections and their gradients
                          "attention_fwd": att,
+                         "attention_bwd": 5 * att // 2,
                          "reduce_residual_layernorm": 2 * (S * H * 8 + H * 8),
                          "layernorm_backward": S * H * (4 + 2 + 2 + 2),
                          "attention_backward_elementwise": S * H * 4 + w.nh * S * 4}

@@ -247,10 +247,11 @@ int tp_qkv_attn_oproj_forward_ex(int S, int H, int nh, int d, int t, int dtype, 
  * tp_attn_forward_train call, and dY [S, H] bf16, writes dX [S, H] bf16,
  * dWqkv_shards[s] [H, 3 (nh/t) d] and dWo_shards[s] [(nh/t) d, H] f32 (the
  * shards' layout), dgamma and dbeta [H] f32 (either may be NULL).
- * workspace >= tp_attn_backward_workspace_bytes(): it holds the [S, S] score,
- * P, dP and dS matrices of a group of heads that the per-head GEMMs process in
- * one launch each (8 heads, or fewer where nh < 8 or where 8 would take more
- * than 1 GiB).  Shapes as tp_qkv_attn_oproj_forward. */
+ * workspace >= tp_attn_backward_workspace_bytes(): dZ, dO, dQKV, the
+ * f32 partial of dX, the row dots D and the LayerNorm backward's partial
+ * rows.  The per-head products run in two fused kernels that keep the score,
+ * P, dP and dS tiles on chip (TMEM), so no [S, S] matrix is held.  Shapes as
+ * tp_qkv_attn_oproj_forward. */
 size_t tp_attn_train_state_bytes(int S, int H, int nh, int d, int t, int dtype);
 int tp_attn_forward_train(int S, int H, int nh, int d, int t, int dtype, int out_dtype, const void* X,
                           const void* const* Wqkv_shards, const void* const* Wo_shards,

@@ -483,7 +483,7 @@ def profile_sample(on: bool):
     _check(lib().tp_profile_sample(1 if on else 0), "tp_profile_sample")
 
 
-def profile_collect(nkinds: int = 7):
+def profile_collect(nkinds: int = 8):
     """{kernel kind: (launches, timed launches, summed ms of the timed ones)}"""
     launches = (ctypes.c_int * nkinds)()
     timed = (ctypes.c_int * nkinds)()

@@ -17,6 +17,7 @@
 #include "../../include/tpblock.h"
 #include "attention.cuh"
 #include "attn_backward.cuh"
+#include "attn_bwd_fused.cuh"
 #include "gemm_tcgen05.cuh"
 #include "ln_backward.cuh"
 #include "reduce_ln.cuh"
@@ -45,6 +46,11 @@ struct DeviceInfo {
 
 // The attention backward makes P and dS in one dual-accumulator GEMM (1) or in
 // a score GEMM and a dP GEMM that reads P back (0).
+// Attention backward: the fused key-major and query-major kernels (1), or
+// per-head GEMM launches over P and dS in memory (0).
+#ifndef TP_ATTN_BACK_FUSED
+#define TP_ATTN_BACK_FUSED 1
+#endif
 #ifndef TP_ATTN_BACK_DUAL
 #define TP_ATTN_BACK_DUAL 1
 #endif
@@ -74,7 +80,7 @@ PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
 // ------------------------------------------------------------ event timing
 constexpr int PROF_CAP = 16384;  // launches timed between two collects
-constexpr int PROF_KINDS = 7;
+constexpr int PROF_KINDS = 8;
 bool g_prof_on = false;
 bool g_prof_sampling = true;  // record events for the launches made while set
 bool g_prof_events_made = false;
@@ -85,7 +91,8 @@ int g_prof_n = 0;
 long long g_prof_launches[PROF_KINDS];  // every launch while enabled, timed or not
 
 enum Kind {
-  K_GEMM_TC = 0, K_REDUCE_LN = 1, K_GEMM_SIMT = 2, K_ATTN = 3, K_LN_BACK = 4, K_ATTN_BACK = 5, K_LN_PARAMS = 6
+  K_GEMM_TC = 0, K_REDUCE_LN = 1, K_GEMM_SIMT = 2, K_ATTN = 3, K_LN_BACK = 4, K_ATTN_BACK = 5, K_LN_PARAMS = 6,
+  K_ATTN_BWD = 7
 };
 
 struct ProfScope {
@@ -137,7 +144,11 @@ int device_ready(DeviceInfo** out) {
           !gemm_smem_attr<2, false, tp::FEAT_SK>() || !gemm_smem_attr<2, true, tp::FEAT_SK>() ||
           !gemm_smem_attr<1, false, tp::FEAT_DUAL>() || !gemm_smem_attr<2, false, tp::FEAT_DUAL>() ||
           cudaFuncSetAttribute(tp::attn_fwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               tp::attn::SMEM_BYTES) != cudaSuccess)
+                               tp::attn::SMEM_BYTES) != cudaSuccess ||
+          cudaFuncSetAttribute(tp::attn_bwd_dkv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tp::attb::SMEM_DKV) != cudaSuccess ||
+          cudaFuncSetAttribute(tp::attn_bwd_dq_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tp::attb::SMEM_DQ) != cudaSuccess)
         d.ok = false;
     }
     if (d.ok) {
@@ -1396,7 +1407,8 @@ int attn_back_group(int S, int nh) {
 AttnBackWs attn_back_layout(int S, int H, int nh) {
   AttnBackWs w;
   const size_t s = static_cast<size_t>(S), h = static_cast<size_t>(H);
-  const size_t ss = static_cast<size_t>(attn_back_group(S, nh)) * s * s;
+  // P and dS in memory only for the per-head GEMM form.
+  const size_t ss = TP_ATTN_BACK_FUSED ? 0 : static_cast<size_t>(attn_back_group(S, nh)) * s * s;
   w.off_dz = 0;
   w.off_do = align256(s * h * 2);
   w.off_dqkv = w.off_do + align256(s * h * 2);
@@ -1475,8 +1487,10 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
   uint8_t* dO = wb + W.off_do;
   uint8_t* dQKV = wb + W.off_dqkv;
   float* dXp = reinterpret_cast<float*>(wb + W.off_dxp);
+#if !TP_ATTN_BACK_FUSED
   __nv_bfloat16* P = reinterpret_cast<__nv_bfloat16*>(wb + W.off_p);
   __nv_bfloat16* dS = reinterpret_cast<__nv_bfloat16*>(wb + W.off_ds);
+#endif
   float* D = reinterpret_cast<float*>(wb + W.off_d);
   float* part = reinterpret_cast<float*>(wb + W.off_part);
   // 1. Through the LayerNorm: dZ, dgamma, dbeta (Z = X + the O projection's output).
@@ -1521,6 +1535,42 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
            : launch_status();
   }
   if (st != TP_OK) return st;
+#if TP_ATTN_BACK_FUSED
+  // Every head at once: dV and dK from the key-major kernel, dQ from the
+  // query-major one, straight into their columns of dQKV.
+  {
+    tp::AttnBwdArgs ab;
+    std::memset(&ab, 0, sizeof(ab));
+    if (!tmap_bf16(&ab.tmQKV, QKV, S, H3, H3, 64, tp::attb::BT) ||
+        !tmap_bf16(&ab.tmdO, dO, S, H, H, 64, tp::attb::BT))
+      return TP_ERR_CUDA;
+    ab.lse2 = lse2;
+    ab.Dvec = D;
+    ab.dQKV = reinterpret_cast<__nv_bfloat16*>(dQKV);
+    ab.ld_qkv = H3;
+    ab.S = S;
+    ab.nh = nh;
+    ab.heads_per_shard = hps;
+    ab.shard_cols = 3 * Hs;
+    ab.scale_log2 = scale_log2;
+    ab.scale = scale;
+    const dim3 grid(S / tp::attb::BT, nh);
+    {
+      ProfScope ps(K_ATTN_BWD, s);
+      if (launch_pdl(tp::attn_bwd_dkv_kernel, grid, dim3(tp::attb::NUM_THREADS), tp::attb::SMEM_DKV, s, ab) !=
+          cudaSuccess)
+        return TP_ERR_CUDA;
+    }
+    {
+      ProfScope ps(K_ATTN_BWD, s);
+      if (launch_pdl(tp::attn_bwd_dq_kernel, grid, dim3(tp::attb::NUM_THREADS), tp::attb::SMEM_DQ, s, ab) !=
+          cudaSuccess)
+        return TP_ERR_CUDA;
+    }
+    st = launch_status();
+    if (st != TP_OK) return st;
+  }
+#else
   // The heads go through in groups of G: each GEMM below is one launch over
   // the group's heads (shard j of the launch = head h0 + j, with its own A, B
   // and output).  P and dS are [S, G S] with head j in columns [j S, (j+1) S);
@@ -1631,6 +1681,7 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
       if (st != TP_OK) return st;
     }
   }
+#endif
   // 4. Through the QKV projection and the residual: dX = dZ + sum_s dQKV_s
   //    Wqkv_s^T (row split over the shards, Wqkv_s [H, 3 Hs] read K-major),
   //    then dWqkv_s = X^T dQKV_s.
@@ -2107,6 +2158,7 @@ const char* tp_kernel_kind_name(int kind) {
     case K_LN_BACK: return "layernorm_backward";
     case K_ATTN_BACK: return "attention_backward_elementwise";
     case K_LN_PARAMS: return "layernorm_grad_params";
+    case K_ATTN_BWD: return "attention_bwd";
     default: return "unknown";
   }
 }

@@ -74,12 +74,12 @@ def test_workspace_sizes(lib):
     assert lib.tp_attn_workspace_bytes(2048, 8192, 64, 128, 4, 0) == 0
 
 
-def test_attention_backward_workspace_holds_a_head_group(lib):
-    """dZ, dO, dQKV (bf16), the f32 row-split partial, the [S, S] P and dS
-    matrices (bf16) of a group of heads, D [nh, S] and 640 per-CTA LayerNorm
-    partial rows: 8 heads a group unless nh < 8 or 8 would pass 1 GiB."""
+def test_attention_backward_workspace(lib):
+    """dZ, dO, dQKV (bf16), the f32 row-split partial, D [nh, S] and 640
+    per-CTA LayerNorm partial rows; the fused attention backward keeps P and
+    dS on chip, so no [S, S] matrix is held."""
     def expect(S, H, nh, g):
-        return S * H * (2 + 2 + 6 + 4) + g * S * S * 4 + nh * S * 4 + 640 * 2 * H * 4
+        return S * H * (2 + 2 + 6 + 4) + nh * S * 4 + 640 * 2 * H * 4
     lib.tp_attn_backward_workspace_bytes.restype = ctypes.c_size_t
     assert lib.tp_attn_backward_workspace_bytes(2048, 8192, 64, 128, 4, 1) == expect(2048, 8192, 64, 8)
     assert lib.tp_attn_backward_workspace_bytes(256, 512, 4, 128, 2, 1) == expect(256, 512, 4, 4)

@@ -4,18 +4,18 @@
 //   dS = P (dP - D) / sqrt d        (D = rowsum(dO * O), lse2 from the forward)
 //   dV = P^T dO,  dK = dS^T Q,  dQ = dS K
 //
-// Two kernels, each a loop over one head's 128-row tiles with every product
-// on the 5th-generation tensor cores and the elementwise steps in between on
-// 128 threads, one TMEM lane (one row) each:
+// Two kernels, each a loop over one head's tiles with every product on the
+// 5th-generation tensor cores and the elementwise steps in between on 128
+// threads, one TMEM lane (one row) each:
 //
 //   attn_bwd_dkv_kernel  one CTA per (128 keys, head): K_j and V_j stay in
-//     shared memory while the query tiles Q_i, dO_i (and their lse2 and D
-//     values) stream through a 2-stage ring.  Per query tile:
+//     shared memory while 64-query tiles Q_i, dO_i (and their lse2 and D
+//     values) stream through a 3-stage ring.  Per query tile:
 //       S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM (lane = key);
-//       P^T and dS^T, as bf16 pairs over the first 64 columns of each;
+//       P^T and dS^T, as bf16 pairs over the first 32 columns of each;
 //       dV_j += P^T dO_i and dK_j += dS^T Q_i with A read from TMEM.
 //   attn_bwd_dq_kernel   one CTA per (128 queries, head): Q_i and dO_i stay,
-//     the key tiles K_j, V_j stream.  Per key tile:
+//     128-key tiles K_j, V_j stream through a 2-stage ring.  Per key tile:
 //       S = Q_i K_j^T and dP = dO_i V_j^T (lane = query);
 //       dS as bf16 pairs over the first 64 columns of dP;
 //       dQ_i += dS K_j with A read from TMEM.
@@ -23,12 +23,17 @@
 // S, P, dP and dS never reach memory, and no result is reduced across CTAs:
 // the key-major kernel sums dV and dK over the queries in TMEM, the
 // query-major kernel sums dQ over the keys.  The price is computing S and dP
-// twice.  TMEM: 4 x 128 f32 columns (S, dP, dV, dK) and 3 x 128 (S, dP, dQ).
-// Roles: warp 0 loads (TMA), warp 1 allocates TMEM and issues the MMAs from
-// one thread, warps 2..5 run the elementwise steps and the epilogue.  The
-// next tile's S and dP are issued after the current tile's last products by
-// the same thread, so they overwrite P and dS only after those products have
-// read them.  Every wait is bounded.
+// twice.  In the key-major kernel the S^T and dP^T of a query tile are 64
+// columns wide, so TMEM holds two of each (4 x 64 f32 columns) besides the
+// 128-column dV and dK: the tensor core computes tile t + 2's S^T and dP^T
+// (and tile t's last products) while the elementwise threads work on tile
+// t + 1.  The query-major kernel keeps 128-key tiles and one S and dP (with
+// 64-key tiles and two buffers it measured slower).  Roles: warp 0 loads (TMA),
+// warp 1 allocates TMEM and issues the MMAs from one thread, warps 2..5 run
+// the elementwise steps and the epilogue.  A buffer of S and dP is reused
+// by a later tile whose S and dP are issued after the products that read the
+// buffer's P and dS, by the same thread, so they overwrite them only once
+// those have completed.  Every wait is bounded.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -40,22 +45,29 @@ namespace tp {
 
 namespace attb {
 constexpr int D = 128;                       // head dimension
-constexpr int BT = 128;                      // rows of a key or query tile
+constexpr int BT = 128;                      // rows of the resident tile (keys or queries): TMEM lanes
+constexpr int BS = 64;                       // rows of a streamed tile: columns of S and dP
 constexpr int NUM_THREADS = 192;             // 6 warps
-constexpr int STAGES = 2;
-constexpr int HALF_BYTES = BT * 64 * 2;      // one 64-column (128 B) box of 128 rows: 16 KiB
-constexpr int TILE_BYTES = 2 * HALF_BYTES;   // 128 rows x 128 bf16: 32 KiB
-constexpr int VEC_BYTES = BT * 4;            // one tile's lse2 or D values
-constexpr int SMEM_DKV = 2 * TILE_BYTES + STAGES * (2 * TILE_BYTES + 2 * VEC_BYTES) + 1024 + 256;
-constexpr int SMEM_DQ = 2 * TILE_BYTES + STAGES * 2 * TILE_BYTES + 1024 + 256;
-constexpr uint32_t IDESC_SS = idesc_bf16_f32(BT, BT, false, false);  // A, B K-major (smem)
+constexpr int STAGES = 3;                    // streamed tiles in flight
+constexpr int HALF_T = BT * 64 * 2;          // one 64-column (128 B) box of a resident tile: 16 KiB
+constexpr int HALF_S = BS * 64 * 2;          // the same for a streamed tile: 8 KiB
+constexpr int TILE_T = 2 * HALF_T;           // 32 KiB
+constexpr int TILE_S = 2 * HALF_S;           // 16 KiB
+constexpr int VEC_BYTES = BS * 4;            // one streamed tile's lse2 or D values
+constexpr int SMEM_DKV = 2 * TILE_T + STAGES * (2 * TILE_S + 2 * VEC_BYTES) + 1024 + 256;
+constexpr int DQ_STAGES = 2;                 // key tiles (128 rows) in flight in the query-major kernel
+constexpr int SMEM_DQ = 2 * TILE_T + DQ_STAGES * 2 * TILE_T + 1024 + 256;
+constexpr uint32_t IDESC_SS = idesc_bf16_f32(BT, BS, false, false);  // S^T, dP^T: A, B K-major (smem)
+constexpr uint32_t IDESC_SQ = idesc_bf16_f32(BT, BT, false, false);  // S, dP of the query-major kernel
 constexpr uint32_t IDESC_TB = idesc_bf16_f32(BT, D, false, true);    // A from TMEM, B MN-major
 constexpr uint32_t TMEM_COLS = 512;
 }  // namespace attb
 
 struct AttnBwdArgs {
-  CUtensorMap tmQKV;        // [S, 3H] bf16, box {64, 128}
-  CUtensorMap tmdO;         // [S, nh D] bf16, box {64, 128}
+  CUtensorMap tmQKV_t;      // [S, 3H] bf16, box {64, 128}: resident tiles
+  CUtensorMap tmQKV_s;      // [S, 3H] bf16, box {64, 64}: streamed tiles
+  CUtensorMap tmdO_t;       // [S, nh D] bf16, box {64, 128}
+  CUtensorMap tmdO_s;       // [S, nh D] bf16, box {64, 64}
   const float* lse2;        // [nh, S]
   const float* Dvec;        // [nh, S]
   __nv_bfloat16* dQKV;      // [S, 3H], laid out as QKV
@@ -67,14 +79,14 @@ struct AttnBwdArgs {
   float scale;              // 1 / sqrt(D)
 };
 
-// The K-major (smem) operand of a 128 x 128 tile for the kk-th 16-element K
-// step, and the MN-major B operand for the kk-th 16-row K step (the two
-// 64-column halves HALF_BYTES apart).
-__device__ __forceinline__ uint64_t attb_kmajor(uint32_t tile, int kk) {
-  return sdesc_sw128(tile + (kk >> 2) * attb::HALF_BYTES + (kk & 3) * 32, 16, 1024);
+// K-major (smem) operand of a tile whose two 64-column boxes are `half`
+// bytes apart, for the kk-th 16-element K step; MN-major B operand of such a
+// tile for the kk-th 16-row K step.
+__device__ __forceinline__ uint64_t attb_kmajor(uint32_t tile, int half, int kk) {
+  return sdesc_sw128(tile + (kk >> 2) * half + (kk & 3) * 32, 16, 1024);
 }
-__device__ __forceinline__ uint64_t attb_mnmajor(uint32_t tile, int kk) {
-  return sdesc_sw128(tile + kk * 2048, attb::HALF_BYTES, 1024);
+__device__ __forceinline__ uint64_t attb_mnmajor(uint32_t tile, int half, int kk) {
+  return sdesc_sw128(tile + kk * 2048, static_cast<uint32_t>(half), 1024);
 }
 
 // Row r's 128 f32 accumulator columns (TMEM lane = r) as bf16 into dst.
@@ -106,23 +118,31 @@ __device__ __forceinline__ void attb_drain(uint64_t* const* bars, const int* arm
   }
 }
 
+// The MMA thread's wait for an in-flight drain after a failed wait.
+__device__ __forceinline__ void attb_mma_drain(uint64_t* drain) {
+  umma_commit(drain);
+  const uint32_t ad = smem_u32(drain);
+  const long long t0 = clock64();
+  while (!mbar_try_wait(ad, 0) && clock64() - t0 < WAIT_LIMIT_CYCLES) {}
+}
+
 __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(const __grid_constant__ AttnBwdArgs a) {
   using namespace attb;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
-  uint8_t* sV = sK + TILE_BYTES;
-  uint8_t* sQ = sV + TILE_BYTES;                 // STAGES tiles
-  uint8_t* sdO = sQ + STAGES * TILE_BYTES;       // STAGES tiles
-  float* sL = reinterpret_cast<float*>(sdO + STAGES * TILE_BYTES);  // STAGES x BT lse2 values
-  float* sD = sL + STAGES * BT;                                      // STAGES x BT D values
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sD + STAGES * BT);
+  uint8_t* sV = sK + TILE_T;
+  uint8_t* sQ = sV + TILE_T;                     // STAGES tiles
+  uint8_t* sdO = sQ + STAGES * TILE_S;           // STAGES tiles
+  float* sL = reinterpret_cast<float*>(sdO + STAGES * TILE_S);  // STAGES x BS lse2 values
+  float* sD = sL + STAGES * BS;                                  // STAGES x BS D values
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sD + STAGES * BS);
   uint64_t* kv_full = bars;
   uint64_t* q_full = bars + 1;                   // [STAGES]
   uint64_t* q_empty = q_full + STAGES;           // [STAGES]
-  uint64_t* s_full = q_empty + STAGES;
-  uint64_t* p_full = s_full + 1;
-  uint64_t* acc_full = p_full + 1;
+  uint64_t* s_full = q_empty + STAGES;           // [2]: S and dP of a buffer computed
+  uint64_t* p_full = s_full + 2;                 // [2]: P and dS of a buffer written
+  uint64_t* acc_full = p_full + 2;
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
 
@@ -133,7 +153,7 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
   const int Hs = a.heads_per_shard * D;
   const int qcol = (h / a.heads_per_shard) * a.shard_cols + (h % a.heads_per_shard) * D;
   const int kcol = qcol + Hs, vcol = qcol + 2 * Hs, ocol = h * D;
-  const int nq = a.S / BT;
+  const int nq = a.S / BS;
 
   if (threadIdx.x == 0) {
     mbar_init(kv_full, 1);
@@ -141,15 +161,18 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
     }
-    mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 128);
+    }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     mbar_fence_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&a.tmQKV);
-    tma_prefetch_desc(&a.tmdO);
+    tma_prefetch_desc(&a.tmQKV_t);
+    tma_prefetch_desc(&a.tmQKV_s);
+    tma_prefetch_desc(&a.tmdO_s);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, TMEM_COLS);
@@ -159,6 +182,7 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // S buffers at columns [0, 64) and [64, 128), dP buffers at [128, 192) and [192, 256)
   const uint32_t tS = tmem_base, tdP = tmem_base + 128, tdV = tmem_base + 256, tdK = tmem_base + 384;
   griddep_wait();  // QKV, dO, lse2 and D come from preceding kernels
   griddep_launch_dependents();
@@ -170,28 +194,28 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
       uint64_t* armed_bar[1 + STAGES] = {kv_full};
       for (int i = 0; i < STAGES; ++i) armed_bar[1 + i] = &q_full[i];
       for (int i = 0; i <= STAGES; ++i) armed[i] = -1;
-      mbar_arrive_expect_tx(kv_full, 2 * TILE_BYTES);
+      mbar_arrive_expect_tx(kv_full, 2 * TILE_T);
       armed[0] = 0;
-      tma_load_2d(sK, &a.tmQKV, kcol, j0, kv_full);
-      tma_load_2d(sK + HALF_BYTES, &a.tmQKV, kcol + 64, j0, kv_full);
-      tma_load_2d(sV, &a.tmQKV, vcol, j0, kv_full);
-      tma_load_2d(sV + HALF_BYTES, &a.tmQKV, vcol + 64, j0, kv_full);
+      tma_load_2d(sK, &a.tmQKV_t, kcol, j0, kv_full);
+      tma_load_2d(sK + HALF_T, &a.tmQKV_t, kcol + 64, j0, kv_full);
+      tma_load_2d(sV, &a.tmQKV_t, vcol, j0, kv_full);
+      tma_load_2d(sV + HALF_T, &a.tmQKV_t, vcol + 64, j0, kv_full);
       bool ok = true;
       for (int i = 0; i < nq; ++i) {
         const int st = i % STAGES;
         const uint32_t ph = (i / STAGES) & 1;
         if (!mbar_wait(&q_empty[st], ph ^ 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(&q_full[st], 2 * TILE_BYTES + 2 * VEC_BYTES);
+        mbar_arrive_expect_tx(&q_full[st], 2 * TILE_S + 2 * VEC_BYTES);
         armed[1 + st] = static_cast<int>(ph);
-        uint8_t* q = sQ + st * TILE_BYTES;
-        uint8_t* o = sdO + st * TILE_BYTES;
-        tma_load_2d(q, &a.tmQKV, qcol, i * BT, &q_full[st]);
-        tma_load_2d(q + HALF_BYTES, &a.tmQKV, qcol + 64, i * BT, &q_full[st]);
-        tma_load_2d(o, &a.tmdO, ocol, i * BT, &q_full[st]);
-        tma_load_2d(o + HALF_BYTES, &a.tmdO, ocol + 64, i * BT, &q_full[st]);
-        const long long v0 = static_cast<long long>(h) * a.S + static_cast<long long>(i) * BT;
-        bulk_load_1d(sL + st * BT, a.lse2 + v0, VEC_BYTES, &q_full[st]);
-        bulk_load_1d(sD + st * BT, a.Dvec + v0, VEC_BYTES, &q_full[st]);
+        uint8_t* q = sQ + st * TILE_S;
+        uint8_t* o = sdO + st * TILE_S;
+        tma_load_2d(q, &a.tmQKV_s, qcol, i * BS, &q_full[st]);
+        tma_load_2d(q + HALF_S, &a.tmQKV_s, qcol + 64, i * BS, &q_full[st]);
+        tma_load_2d(o, &a.tmdO_s, ocol, i * BS, &q_full[st]);
+        tma_load_2d(o + HALF_S, &a.tmdO_s, ocol + 64, i * BS, &q_full[st]);
+        const long long v0 = static_cast<long long>(h) * a.S + static_cast<long long>(i) * BS;
+        bulk_load_1d(sL + st * BS, a.lse2 + v0, VEC_BYTES, &q_full[st]);
+        bulk_load_1d(sD + st * BS, a.Dvec + v0, VEC_BYTES, &q_full[st]);
       }
       if (!ok) attb_drain(armed_bar, armed, 1 + STAGES);
     }
@@ -200,38 +224,44 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
     if (lane == 0) {
       bool ok = mbar_wait(kv_full, 0);
       const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
+      // S^T = K_j Q_i^T and dP^T = V_j dO_i^T of query tile i into buffer i & 1.
+      auto issue_sdp = [&](int i) -> bool {
+        const int st = i % STAGES, b = i & 1;
+        if (!mbar_wait(&q_full[st], (i / STAGES) & 1)) return false;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(sQ + st * TILE_S), o_addr = smem_u32(sdO + st * TILE_S);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16(tS + b * BS, attb_kmajor(k_addr, HALF_T, kk), attb_kmajor(q_addr, HALF_S, kk), IDESC_SS,
+                    kk > 0 ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_bf16(tdP + b * BS, attb_kmajor(v_addr, HALF_T, kk), attb_kmajor(o_addr, HALF_S, kk), IDESC_SS,
+                    kk > 0 ? 1u : 0u);
+        umma_commit(&s_full[b]);
+        return true;
+      };
+      for (int i = 0; i < 2 && i < nq && ok; ++i) ok = issue_sdp(i);
       for (int i = 0; i < nq && ok; ++i) {
-        const int st = i % STAGES;
-        if (!mbar_wait(&q_full[st], (i / STAGES) & 1)) { ok = false; break; }
+        const int st = i % STAGES, b = i & 1;
+        // P^T over buffer b of S^T, dS^T over buffer b of dP^T (K = the tile's queries).
+        if (!mbar_wait(&p_full[b], (i >> 1) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t q_addr = smem_u32(sQ + st * TILE_BYTES), o_addr = smem_u32(sdO + st * TILE_BYTES);
-        // S^T = K_j Q_i^T, dP^T = V_j dO_i^T (K = d).
+        const uint32_t q_addr = smem_u32(sQ + st * TILE_S), o_addr = smem_u32(sdO + st * TILE_S);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_bf16(tS, attb_kmajor(k_addr, kk), attb_kmajor(q_addr, kk), IDESC_SS, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < BS / 16; ++kk)
+          umma_bf16_tmem_a(tdV, tS + b * BS + kk * 8, attb_mnmajor(o_addr, HALF_S, kk), IDESC_TB,
+                           (i > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_bf16(tdP, attb_kmajor(v_addr, kk), attb_kmajor(o_addr, kk), IDESC_SS, kk > 0 ? 1u : 0u);
-        umma_commit(s_full);
-        // P^T over S^T's first 64 columns, dS^T over dP^T's (K = queries).
-        if (!mbar_wait(p_full, i & 1)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < BT / 16; ++kk)
-          umma_bf16_tmem_a(tdV, tS + kk * 8, attb_mnmajor(o_addr, kk), IDESC_TB, (i > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-        for (int kk = 0; kk < BT / 16; ++kk)
-          umma_bf16_tmem_a(tdK, tdP + kk * 8, attb_mnmajor(q_addr, kk), IDESC_TB, (i > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BS / 16; ++kk)
+          umma_bf16_tmem_a(tdK, tdP + b * BS + kk * 8, attb_mnmajor(q_addr, HALF_S, kk), IDESC_TB,
+                           (i > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&q_empty[st]);
+        // Tile i + 2 reuses buffer b: issued after the products above.
+        if (i + 2 < nq && !issue_sdp(i + 2)) { ok = false; break; }
       }
-      if (ok) {
-        umma_commit(acc_full);
-      } else {
-        umma_commit(drain);
-        const uint32_t ad = smem_u32(drain);
-        const long long t0 = clock64();
-        while (!mbar_try_wait(ad, 0) && clock64() - t0 < WAIT_LIMIT_CYCLES) {}
-      }
+      if (ok) umma_commit(acc_full);
+      else attb_mma_drain(drain);
     }
   } else {
     // ------------------------------------------ elementwise and epilogue
@@ -239,18 +269,19 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     bool ok = true;
     for (int i = 0; i < nq; ++i) {
-      const int st = i % STAGES;
-      if (!__all_sync(0xffffffffu, mbar_wait(s_full, i & 1))) { ok = false; break; }
+      const int st = i % STAGES, b = i & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (i >> 1) & 1))) { ok = false; break; }
       // lse2 and D of this query tile arrived with Q_i.
       if (!__all_sync(0xffffffffu, mbar_wait(&q_full[st], (i / STAGES) & 1))) { ok = false; break; }
       tc_fence_after();
-      const float* L = sL + st * BT;
-      const float* Dv = sD + st * BT;
+      const float* L = sL + st * BS;
+      const float* Dv = sD + st * BS;
+      const uint32_t tSb = tS + b * BS + lane_off, tdPb = tdP + b * BS + lane_off;
 #pragma unroll
-      for (int c = 0; c < BT / 32; ++c) {
+      for (int c = 0; c < BS / 32; ++c) {
         uint32_t us[32], ud[32], pp[16], pd[16];
-        tmem_ld_32x32b_x32(tS + lane_off + c * 32, us);
-        tmem_ld_32x32b_x32(tdP + lane_off + c * 32, ud);
+        tmem_ld_32x32b_x32(tSb + c * 32, us);
+        tmem_ld_32x32b_x32(tdPb + c * 32, ud);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -262,14 +293,14 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
           pp[e] = pack_bf16x2(p0, p1);
           pd[e] = pack_bf16x2(d0, d1);
         }
-        // Columns [16c, 16c + 16) hold queries [32c, 32c + 32) as pairs; they
-        // lie within the columns already read.
-        tmem_st_32x32b_x16(tS + lane_off + c * 16, pp);
-        tmem_st_32x32b_x16(tdP + lane_off + c * 16, pd);
+        // Columns [16c, 16c + 16) of the buffer hold queries [32c, 32c + 32)
+        // as pairs; they lie within the columns already read.
+        tmem_st_32x32b_x16(tSb + c * 16, pp);
+        tmem_st_32x32b_x16(tdPb + c * 16, pd);
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_full);
+      mbar_arrive(&p_full[b]);
     }
     if (ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0))) {
       tc_fence_after();
@@ -292,14 +323,14 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dq_kernel(const
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sdO = sQ + TILE_BYTES;
-  uint8_t* sK = sdO + TILE_BYTES;                // STAGES tiles
-  uint8_t* sV = sK + STAGES * TILE_BYTES;        // STAGES tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + STAGES * TILE_BYTES);
+  uint8_t* sdO = sQ + TILE_T;
+  uint8_t* sK = sdO + TILE_T;                    // DQ_STAGES tiles
+  uint8_t* sV = sK + DQ_STAGES * TILE_T;         // DQ_STAGES tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + DQ_STAGES * TILE_T);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = bars + 1;                  // [STAGES]
-  uint64_t* kv_empty = kv_full + STAGES;         // [STAGES]
-  uint64_t* s_full = kv_empty + STAGES;
+  uint64_t* kv_full = bars + 1;                  // [DQ_STAGES]
+  uint64_t* kv_empty = kv_full + DQ_STAGES;      // [DQ_STAGES]
+  uint64_t* s_full = kv_empty + DQ_STAGES;
   uint64_t* p_full = s_full + 1;
   uint64_t* acc_full = p_full + 1;
   uint64_t* drain = acc_full + 1;
@@ -316,7 +347,7 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dq_kernel(const
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int i = 0; i < STAGES; ++i) {
+    for (int i = 0; i < DQ_STAGES; ++i) {
       mbar_init(&kv_full[i], 1);
       mbar_init(&kv_empty[i], 1);
     }
@@ -327,8 +358,8 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dq_kernel(const
     mbar_fence_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&a.tmQKV);
-    tma_prefetch_desc(&a.tmdO);
+    tma_prefetch_desc(&a.tmQKV_t);
+    tma_prefetch_desc(&a.tmdO_t);
   }
   if (warp == 1) {
     tmem_alloc(tmem_holder, TMEM_COLS);
@@ -345,31 +376,31 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dq_kernel(const
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      int armed[1 + STAGES];
-      uint64_t* armed_bar[1 + STAGES] = {q_full};
-      for (int i = 0; i < STAGES; ++i) armed_bar[1 + i] = &kv_full[i];
-      for (int i = 0; i <= STAGES; ++i) armed[i] = -1;
-      mbar_arrive_expect_tx(q_full, 2 * TILE_BYTES);
+      int armed[1 + DQ_STAGES];
+      uint64_t* armed_bar[1 + DQ_STAGES] = {q_full};
+      for (int i = 0; i < DQ_STAGES; ++i) armed_bar[1 + i] = &kv_full[i];
+      for (int i = 0; i <= DQ_STAGES; ++i) armed[i] = -1;
+      mbar_arrive_expect_tx(q_full, 2 * TILE_T);
       armed[0] = 0;
-      tma_load_2d(sQ, &a.tmQKV, qcol, i0, q_full);
-      tma_load_2d(sQ + HALF_BYTES, &a.tmQKV, qcol + 64, i0, q_full);
-      tma_load_2d(sdO, &a.tmdO, ocol, i0, q_full);
-      tma_load_2d(sdO + HALF_BYTES, &a.tmdO, ocol + 64, i0, q_full);
+      tma_load_2d(sQ, &a.tmQKV_t, qcol, i0, q_full);
+      tma_load_2d(sQ + HALF_T, &a.tmQKV_t, qcol + 64, i0, q_full);
+      tma_load_2d(sdO, &a.tmdO_t, ocol, i0, q_full);
+      tma_load_2d(sdO + HALF_T, &a.tmdO_t, ocol + 64, i0, q_full);
       bool ok = true;
       for (int j = 0; j < nk; ++j) {
-        const int st = j % STAGES;
-        const uint32_t ph = (j / STAGES) & 1;
+        const int st = j % DQ_STAGES;
+        const uint32_t ph = (j / DQ_STAGES) & 1;
         if (!mbar_wait(&kv_empty[st], ph ^ 1)) { ok = false; break; }
-        mbar_arrive_expect_tx(&kv_full[st], 2 * TILE_BYTES);
+        mbar_arrive_expect_tx(&kv_full[st], 2 * TILE_T);
         armed[1 + st] = static_cast<int>(ph);
-        uint8_t* k = sK + st * TILE_BYTES;
-        uint8_t* v = sV + st * TILE_BYTES;
-        tma_load_2d(k, &a.tmQKV, kcol, j * BT, &kv_full[st]);
-        tma_load_2d(k + HALF_BYTES, &a.tmQKV, kcol + 64, j * BT, &kv_full[st]);
-        tma_load_2d(v, &a.tmQKV, vcol, j * BT, &kv_full[st]);
-        tma_load_2d(v + HALF_BYTES, &a.tmQKV, vcol + 64, j * BT, &kv_full[st]);
+        uint8_t* k = sK + st * TILE_T;
+        uint8_t* v = sV + st * TILE_T;
+        tma_load_2d(k, &a.tmQKV_t, kcol, j * BT, &kv_full[st]);
+        tma_load_2d(k + HALF_T, &a.tmQKV_t, kcol + 64, j * BT, &kv_full[st]);
+        tma_load_2d(v, &a.tmQKV_t, vcol, j * BT, &kv_full[st]);
+        tma_load_2d(v + HALF_T, &a.tmQKV_t, vcol + 64, j * BT, &kv_full[st]);
       }
-      if (!ok) attb_drain(armed_bar, armed, 1 + STAGES);
+      if (!ok) attb_drain(armed_bar, armed, 1 + DQ_STAGES);
     }
   } else if (warp == 1) {
     // --------------------------------------------------------- MMA issuer
@@ -377,34 +408,31 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dq_kernel(const
       bool ok = mbar_wait(q_full, 0);
       const uint32_t q_addr = smem_u32(sQ), o_addr = smem_u32(sdO);
       for (int j = 0; j < nk && ok; ++j) {
-        const int st = j % STAGES;
-        if (!mbar_wait(&kv_full[st], (j / STAGES) & 1)) { ok = false; break; }
+        const int st = j % DQ_STAGES;
+        if (!mbar_wait(&kv_full[st], (j / DQ_STAGES) & 1)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + st * TILE_BYTES), v_addr = smem_u32(sV + st * TILE_BYTES);
+        const uint32_t k_addr = smem_u32(sK + st * TILE_T), v_addr = smem_u32(sV + st * TILE_T);
         // S = Q_i K_j^T, dP = dO_i V_j^T (K = d).
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          umma_bf16(tS, attb_kmajor(q_addr, kk), attb_kmajor(k_addr, kk), IDESC_SS, kk > 0 ? 1u : 0u);
+          umma_bf16(tS, attb_kmajor(q_addr, HALF_T, kk), attb_kmajor(k_addr, HALF_T, kk), IDESC_SQ,
+                    kk > 0 ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          umma_bf16(tdP, attb_kmajor(o_addr, kk), attb_kmajor(v_addr, kk), IDESC_SS, kk > 0 ? 1u : 0u);
+          umma_bf16(tdP, attb_kmajor(o_addr, HALF_T, kk), attb_kmajor(v_addr, HALF_T, kk), IDESC_SQ,
+                    kk > 0 ? 1u : 0u);
         umma_commit(s_full);
         // dS over dP's first 64 columns (K = keys).
         if (!mbar_wait(p_full, j & 1)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk)
-          umma_bf16_tmem_a(tdQ, tdP + kk * 8, attb_mnmajor(k_addr, kk), IDESC_TB, (j > 0 || kk > 0) ? 1u : 0u);
+          umma_bf16_tmem_a(tdQ, tdP + kk * 8, attb_mnmajor(k_addr, HALF_T, kk), IDESC_TB,
+                           (j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&kv_empty[st]);
       }
-      if (ok) {
-        umma_commit(acc_full);
-      } else {
-        umma_commit(drain);
-        const uint32_t ad = smem_u32(drain);
-        const long long t0 = clock64();
-        while (!mbar_try_wait(ad, 0) && clock64() - t0 < WAIT_LIMIT_CYCLES) {}
-      }
+      if (ok) umma_commit(acc_full);
+      else attb_mma_drain(drain);
     }
   } else {
     // ------------------------------------------ elementwise and epilogue
@@ -429,6 +457,8 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dq_kernel(const
           pd[e] = pack_bf16x2((p0 * (__uint_as_float(ud[2 * e]) - Dr)) * a.scale,
                               (p1 * (__uint_as_float(ud[2 * e + 1]) - Dr)) * a.scale);
         }
+        // Columns [16c, 16c + 16) hold keys [32c, 32c + 32) as pairs; they lie
+        // within the columns already read.
         tmem_st_32x32b_x16(tdP + lane_off + c * 16, pd);
       }
       tmem_wait_st();

@@ -1541,8 +1541,10 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
   {
     tp::AttnBwdArgs ab;
     std::memset(&ab, 0, sizeof(ab));
-    if (!tmap_bf16(&ab.tmQKV, QKV, S, H3, H3, 64, tp::attb::BT) ||
-        !tmap_bf16(&ab.tmdO, dO, S, H, H, 64, tp::attb::BT))
+    if (!tmap_bf16(&ab.tmQKV_t, QKV, S, H3, H3, 64, tp::attb::BT) ||
+        !tmap_bf16(&ab.tmQKV_s, QKV, S, H3, H3, 64, tp::attb::BS) ||
+        !tmap_bf16(&ab.tmdO_t, dO, S, H, H, 64, tp::attb::BT) ||
+        !tmap_bf16(&ab.tmdO_s, dO, S, H, H, 64, tp::attb::BS))
       return TP_ERR_CUDA;
     ab.lse2 = lse2;
     ab.Dvec = D;

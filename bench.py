@@ -81,6 +81,9 @@ def parse():
     ap.add_argument("--stream-k", choices=["off", "on", "model"], default="off",
                     help="GEMM scheduling: whole-tile waves only (off, the library's default), stream-K wherever "
                          "a GEMM has scratch for it (on), the library's cost model (model)")
+    ap.add_argument("--gemm-tile-n", type=int, default=0,
+                    help="force every tensor-core GEMM's tile width (128, or 256..512 in steps of 32; 0: the "
+                         "library's cost model)")
     ap.add_argument("--attn-split", choices=["off", "last-wave", "all"], default="last-wave",
                     help="attention kernel key split: none, the last partial wave (the library's default), every "
                          "unit")
@@ -488,6 +491,8 @@ def run_ours(args, rank, world, local):
     L.lib()  # load the CUDA library (raises if it is not built)
     L.set_gemm_stream_k({"off": 0, "on": 1, "model": 2}[args.stream_k])
     L.set_attn_kv_split({"off": 0, "last-wave": 1, "all": 2}[args.attn_split])
+    if args.gemm_tile_n:
+        L.set_gemm_tile_n(args.gemm_tile_n)
     tp_mode = args.tp != "none"
     P = TPProblem(w, dev, rank, world, args.tp, L, synth, torch) if tp_mode else Problem(w, dev, rank, L, synth, torch)
     X, Y = P.X, P.Y
@@ -625,6 +630,8 @@ def run_ours(args, rank, world, local):
             cfg["stream_k"] = args.stream_k
         if args.attn_split != "last-wave":
             cfg["attn_split"] = args.attn_split
+        if args.gemm_tile_n:
+            cfg["gemm_tile_n"] = args.gemm_tile_n
         result = {
             "metric": metric_for(w),
             "value": round(value, 2),

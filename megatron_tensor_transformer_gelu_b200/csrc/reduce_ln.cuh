@@ -125,7 +125,11 @@ __device__ __forceinline__ void store8(const ReduceLnArgs& p, long long off, con
 // row.  NP1 specialises the common single partial so that every load of a row
 // is issued before its first add.
 template <int WPR, int CH, bool NP1>
-__global__ void __launch_bounds__(rln::cta_threads(WPR), (TP_RLN_LEAN && rln::cta_threads(WPR) == 256) ? 5 : 1)
+#ifndef TP_RLN_CH4_MIN_BLOCKS
+#define TP_RLN_CH4_MIN_BLOCKS 4
+#endif
+__global__ void __launch_bounds__(rln::cta_threads(WPR),
+                                  (TP_RLN_LEAN && rln::cta_threads(WPR) == 256) ? (CH <= 2 ? 5 : TP_RLN_CH4_MIN_BLOCKS) : 1)
     reduce_residual_ln_kernel(const ReduceLnArgs p) {
   constexpr int RPC = WPR > 8 ? 1 : rln::THREADS / 32 / WPR;  // rows per CTA
   __shared__ float red[2][RPC][WPR];

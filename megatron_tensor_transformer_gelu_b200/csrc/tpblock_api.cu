@@ -57,6 +57,9 @@ struct DeviceInfo {
 
 // Rows of 2049..4096 columns: 8 warps a row with 16 values a lane (0), or 16
 // warps a row with 8 values a lane (1).
+#ifndef TP_RLN_4096_WPR
+#define TP_RLN_4096_WPR 8  // warps per row of the reduce + LayerNorm kernel for 2048 < H <= 4096 (8 or 4)
+#endif
 #ifndef TP_RLN_WIDE_ROWS
 #define TP_RLN_WIDE_ROWS 0
 #endif
@@ -771,6 +774,9 @@ int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, i
 #if TP_RLN_WIDE_ROWS
   // one 512-thread CTA per row, 8 values per lane: fewer registers, more CTAs per SM
   else if (H <= 4096) np1 ? go(reduce_residual_ln_kernel<16, 1, true>, 16, 1) : go(reduce_residual_ln_kernel<16, 1, false>, 16, 1);
+#elif TP_RLN_4096_WPR == 4
+  // two rows per 256-thread CTA, 4 warps and 4 chunks per lane each
+  else if (H <= 4096) np1 ? go(reduce_residual_ln_kernel<4, 4, true>, 4, 2) : go(reduce_residual_ln_kernel<4, 4, false>, 4, 2);
 #else
   else if (H <= 4096) np1 ? go(reduce_residual_ln_kernel<8, 2, true>, 8, 1) : go(reduce_residual_ln_kernel<8, 2, false>, 8, 1);
 #endif

@@ -47,7 +47,21 @@ namespace attb {
 constexpr int D = 128;                       // head dimension
 constexpr int BT = 128;                      // rows of the resident tile (keys or queries): TMEM lanes
 constexpr int BS = 64;                       // rows of a streamed tile: columns of S and dP
-constexpr int NUM_THREADS = 192;             // 6 warps
+// Elementwise warpgroups per kernel: each takes its own columns of every tile.
+// Measured (ncu, one box): the query-major kernel 282 us with two against
+// 291-293 us with one, the key-major kernel 366-369 us with one against 376
+// us with two.
+#ifndef TP_ATTB_DKV_EWG
+#define TP_ATTB_DKV_EWG 1
+#endif
+#ifndef TP_ATTB_DQ_EWG
+#define TP_ATTB_DQ_EWG 2
+#endif
+constexpr int DKV_EWG = TP_ATTB_DKV_EWG;
+constexpr int DQ_EWG = TP_ATTB_DQ_EWG;
+// warp 0 loads, warp 1 MMAs, the rest elementwise
+constexpr int DKV_THREADS = 64 + 128 * DKV_EWG;
+constexpr int DQ_THREADS = 64 + 128 * DQ_EWG;
 constexpr int STAGES = 3;                    // streamed tiles in flight
 constexpr int HALF_T = BT * 64 * 2;          // one 64-column (128 B) box of a resident tile: 16 KiB
 constexpr int HALF_S = BS * 64 * 2;          // the same for a streamed tile: 8 KiB
@@ -89,10 +103,11 @@ __device__ __forceinline__ uint64_t attb_mnmajor(uint32_t tile, int half, int kk
   return sdesc_sw128(tile + kk * 2048, static_cast<uint32_t>(half), 1024);
 }
 
-// Row r's 128 f32 accumulator columns (TMEM lane = r) as bf16 into dst.
-__device__ __forceinline__ void attb_store_row(uint32_t t_row, __nv_bfloat16* dst) {
-#pragma unroll
-  for (int c = 0; c < attb::D / 32; ++c) {
+// f32 accumulator columns [c0 * 32, c1 * 32) of row r (TMEM lane = r) as bf16
+// into dst (which points at column 0).
+__device__ __forceinline__ void attb_store_row(uint32_t t_row, __nv_bfloat16* dst, int c0 = 0,
+                                               int c1 = attb::D / 32) {
+  for (int c = c0; c < c1; ++c) {
     uint32_t u[32];
     tmem_ld_32x32b_x32(t_row + c * 32, u);
     tmem_wait_ld();
@@ -106,6 +121,16 @@ __device__ __forceinline__ void attb_store_row(uint32_t t_row, __nv_bfloat16* ds
       *reinterpret_cast<uint4*>(dst + c * 32 + g * 8) = w;
     }
   }
+}
+
+// P, dS as bf16 pairs: of `ewg` elementwise warpgroups, group g owns columns
+// [g n, (g + 1) n) of a buffer (n = cols / ewg) and stores the pairs of its
+// rows' values there, from its first column on (only over columns it has
+// read).  The packed column that holds rows [16 kk, 16 kk + 16) of the K
+// dimension:
+__device__ __forceinline__ uint32_t attb_packed_col(int kk, int cols, int ewg) {
+  const int n = cols / ewg, q = 16 * kk, g = q / n;
+  return static_cast<uint32_t>(g * n + (q - g * n) / 2);
 }
 
 // Wait (bounded) for the copies a producer thread armed before it gave up.
@@ -126,8 +151,9 @@ __device__ __forceinline__ void attb_mma_drain(uint64_t* drain) {
   while (!mbar_try_wait(ad, 0) && clock64() - t0 < WAIT_LIMIT_CYCLES) {}
 }
 
-__global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(const __grid_constant__ AttnBwdArgs a) {
+__global__ void __launch_bounds__(attb::DKV_THREADS, 1) attn_bwd_dkv_kernel(const __grid_constant__ AttnBwdArgs a) {
   using namespace attb;
+  constexpr int EWG = DKV_EWG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sK = smem;
@@ -163,7 +189,7 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 128);
+      mbar_init(&p_full[b], 128 * EWG);
     }
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
@@ -250,11 +276,11 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
         const uint32_t q_addr = smem_u32(sQ + st * TILE_S), o_addr = smem_u32(sdO + st * TILE_S);
 #pragma unroll
         for (int kk = 0; kk < BS / 16; ++kk)
-          umma_bf16_tmem_a(tdV, tS + b * BS + kk * 8, attb_mnmajor(o_addr, HALF_S, kk), IDESC_TB,
+          umma_bf16_tmem_a(tdV, tS + b * BS + attb_packed_col(kk, BS, EWG), attb_mnmajor(o_addr, HALF_S, kk), IDESC_TB,
                            (i > 0 || kk > 0) ? 1u : 0u);
 #pragma unroll
         for (int kk = 0; kk < BS / 16; ++kk)
-          umma_bf16_tmem_a(tdK, tdP + b * BS + kk * 8, attb_mnmajor(q_addr, HALF_S, kk), IDESC_TB,
+          umma_bf16_tmem_a(tdK, tdP + b * BS + attb_packed_col(kk, BS, EWG), attb_mnmajor(q_addr, HALF_S, kk), IDESC_TB,
                            (i > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&q_empty[st]);
         // Tile i + 2 reuses buffer b: issued after the products above.
@@ -267,6 +293,8 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
     // ------------------------------------------ elementwise and epilogue
     const int r = (warp & 3) * 32 + lane;                 // key row of the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int g = (warp - 2) >> 2;                        // elementwise warpgroup
+    constexpr int GC = BS / EWG;                          // its columns (queries) of a tile
     bool ok = true;
     for (int i = 0; i < nq; ++i) {
       const int st = i % STAGES, b = i & 1;
@@ -276,16 +304,16 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
       tc_fence_after();
       const float* L = sL + st * BS;
       const float* Dv = sD + st * BS;
-      const uint32_t tSb = tS + b * BS + lane_off, tdPb = tdP + b * BS + lane_off;
+      const uint32_t tSb = tS + b * BS + lane_off + g * GC, tdPb = tdP + b * BS + lane_off + g * GC;
 #pragma unroll
-      for (int c = 0; c < BS / 32; ++c) {
+      for (int c = 0; c < GC / 32; ++c) {
         uint32_t us[32], ud[32], pp[16], pd[16];
         tmem_ld_32x32b_x32(tSb + c * 32, us);
         tmem_ld_32x32b_x32(tdPb + c * 32, ud);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const int q = c * 32 + 2 * e;
+          const int q = g * GC + c * 32 + 2 * e;
           const float p0 = exp2_fast(fmaf(__uint_as_float(us[2 * e]), a.scale_log2, -L[q]));
           const float p1 = exp2_fast(fmaf(__uint_as_float(us[2 * e + 1]), a.scale_log2, -L[q + 1]));
           const float d0 = (p0 * (__uint_as_float(ud[2 * e]) - Dv[q])) * a.scale;
@@ -293,8 +321,8 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
           pp[e] = pack_bf16x2(p0, p1);
           pd[e] = pack_bf16x2(d0, d1);
         }
-        // Columns [16c, 16c + 16) of the buffer hold queries [32c, 32c + 32)
-        // as pairs; they lie within the columns already read.
+        // The group's columns [16c, 16c + 16) hold its queries [32c, 32c + 32)
+        // as pairs; they lie within the columns it has already read.
         tmem_st_32x32b_x16(tSb + c * 16, pp);
         tmem_st_32x32b_x16(tdPb + c * 16, pd);
       }
@@ -305,8 +333,8 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
     if (ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0))) {
       tc_fence_after();
       __nv_bfloat16* row = a.dQKV + static_cast<long long>(j0 + r) * a.ld_qkv;
-      attb_store_row(tdV + lane_off, row + vcol);
-      attb_store_row(tdK + lane_off, row + kcol);
+      if (EWG == 1 || g == 0) attb_store_row(tdV + lane_off, row + vcol);
+      if (EWG == 1 || g == 1) attb_store_row(tdK + lane_off, row + kcol);
     }
   }
 
@@ -318,8 +346,9 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dkv_kernel(cons
   }
 }
 
-__global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dq_kernel(const __grid_constant__ AttnBwdArgs a) {
+__global__ void __launch_bounds__(attb::DQ_THREADS, 1) attn_bwd_dq_kernel(const __grid_constant__ AttnBwdArgs a) {
   using namespace attb;
+  constexpr int EWG = DQ_EWG;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
@@ -352,7 +381,7 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dq_kernel(const
       mbar_init(&kv_empty[i], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
+    mbar_init(p_full, 128 * EWG);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     mbar_fence_init();
@@ -427,7 +456,7 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dq_kernel(const
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BT / 16; ++kk)
-          umma_bf16_tmem_a(tdQ, tdP + kk * 8, attb_mnmajor(k_addr, HALF_T, kk), IDESC_TB,
+          umma_bf16_tmem_a(tdQ, tdP + attb_packed_col(kk, BT, EWG), attb_mnmajor(k_addr, HALF_T, kk), IDESC_TB,
                            (j > 0 || kk > 0) ? 1u : 0u);
         umma_commit(&kv_empty[st]);
       }
@@ -438,17 +467,20 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dq_kernel(const
     // ------------------------------------------ elementwise and epilogue
     const int r = (warp & 3) * 32 + lane;                 // query row of the tile == TMEM lane
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const int g = (warp - 2) >> 2;                        // elementwise warpgroup
+    constexpr int GC = BT / EWG;                          // its columns (keys) of a tile
     const long long v0 = static_cast<long long>(h) * a.S + i0 + r;
     const float lse = a.lse2[v0], Dr = a.Dvec[v0];
     bool ok = true;
     for (int j = 0; j < nk; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(s_full, j & 1))) { ok = false; break; }
       tc_fence_after();
+      const uint32_t tSg = tS + lane_off + g * GC, tdPg = tdP + lane_off + g * GC;
 #pragma unroll
-      for (int c = 0; c < BT / 32; ++c) {
+      for (int c = 0; c < GC / 32; ++c) {
         uint32_t us[32], ud[32], pd[16];
-        tmem_ld_32x32b_x32(tS + lane_off + c * 32, us);
-        tmem_ld_32x32b_x32(tdP + lane_off + c * 32, ud);
+        tmem_ld_32x32b_x32(tSg + c * 32, us);
+        tmem_ld_32x32b_x32(tdPg + c * 32, ud);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -457,9 +489,9 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dq_kernel(const
           pd[e] = pack_bf16x2((p0 * (__uint_as_float(ud[2 * e]) - Dr)) * a.scale,
                               (p1 * (__uint_as_float(ud[2 * e + 1]) - Dr)) * a.scale);
         }
-        // Columns [16c, 16c + 16) hold keys [32c, 32c + 32) as pairs; they lie
-        // within the columns already read.
-        tmem_st_32x32b_x16(tdP + lane_off + c * 16, pd);
+        // The group's columns [16c, 16c + 16) hold its keys [32c, 32c + 32)
+        // as pairs; they lie within the columns it has already read.
+        tmem_st_32x32b_x16(tdPg + c * 16, pd);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -467,7 +499,8 @@ __global__ void __launch_bounds__(attb::NUM_THREADS, 1) attn_bwd_dq_kernel(const
     }
     if (ok && __all_sync(0xffffffffu, mbar_wait(acc_full, 0))) {
       tc_fence_after();
-      attb_store_row(tdQ + lane_off, a.dQKV + static_cast<long long>(i0 + r) * a.ld_qkv + qcol);
+      attb_store_row(tdQ + lane_off, a.dQKV + static_cast<long long>(i0 + r) * a.ld_qkv + qcol,
+                     g * (D / 32 / EWG), (g + 1) * (D / 32 / EWG));
     }
   }
 

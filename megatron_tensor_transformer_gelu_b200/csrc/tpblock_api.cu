@@ -1565,13 +1565,13 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
     const dim3 grid(S / tp::attb::BT, nh);
     {
       ProfScope ps(K_ATTN_BWD, s);
-      if (launch_pdl(tp::attn_bwd_dkv_kernel, grid, dim3(tp::attb::NUM_THREADS), tp::attb::SMEM_DKV, s, ab) !=
+      if (launch_pdl(tp::attn_bwd_dkv_kernel, grid, dim3(tp::attb::DKV_THREADS), tp::attb::SMEM_DKV, s, ab) !=
           cudaSuccess)
         return TP_ERR_CUDA;
     }
     {
       ProfScope ps(K_ATTN_BWD, s);
-      if (launch_pdl(tp::attn_bwd_dq_kernel, grid, dim3(tp::attb::NUM_THREADS), tp::attb::SMEM_DQ, s, ab) !=
+      if (launch_pdl(tp::attn_bwd_dq_kernel, grid, dim3(tp::attb::DQ_THREADS), tp::attb::SMEM_DQ, s, ab) !=
           cudaSuccess)
         return TP_ERR_CUDA;
     }

@@ -452,6 +452,13 @@ int tp_set_gemm_stream_k(int mode);
 int tp_gemm_plan_sk(int M, int t, int row_mode, int shard_k, int shard_n, int out_f32, int b_kmajor,
                     int heavy_epilogue, int slots, int max_splits, size_t sk_area_bytes, int* tile_n, int* splits,
                     int* stream_k, int* sk_clusters);
+/* tp_gemm_plan_sk for a GEMM whose A operand is read M-major (a_mnmajor = 1:
+ * A stored [K, M], the weight-gradient GEMMs X^T dU, G^T dZ, O^T dZ and
+ * X^T dQKV of the backward passes), for which the 256-column tiles cost
+ * more per k-block than with a K-major A. */
+int tp_gemm_plan_ex(int M, int t, int row_mode, int shard_k, int shard_n, int out_f32, int a_mnmajor, int b_kmajor,
+                    int heavy_epilogue, int slots, int max_splits, size_t sk_area_bytes, int* tile_n, int* splits,
+                    int* stream_k, int* sk_clusters);
 
 /* Last-wave key split of the attention kernel (tp_qkv_attn_oproj_forward,
  * tp_attn_forward_train, tp_attn_partial_forward).  The attention kernel runs

@@ -81,6 +81,7 @@ SIGNATURES = {
     "tp_set_attn_kv_split": (_c_int, [_c_int]),
     "tp_attn_split_plan": (_c_int, [_c_int] * 4 + [_c_size] + [ctypes.POINTER(_c_int)] * 3),
     "tp_gemm_plan_sk": (_c_int, [_c_int] * 10 + [_c_size] + [ctypes.POINTER(_c_int)] * 4),
+    "tp_gemm_plan_ex": (_c_int, [_c_int] * 11 + [_c_size] + [ctypes.POINTER(_c_int)] * 4),
     "tp_selftest_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
     "tp_selftest_flag_wait_timeout": (_c_int, [ctypes.c_longlong, _vp]),
     "tp_selftest_exp2": (_c_int, [_vp, _vp, _vp, _c_int, _vp]),
@@ -449,6 +450,17 @@ def attn_split_plan(S, nh, slots=148, mode=1, scratch_bytes=1 << 40):
     out = [ctypes.c_int(0) for _ in range(3)]
     _check(lib().tp_attn_split_plan(int(S), int(nh), int(slots), int(mode), int(scratch_bytes),
                                     *[ctypes.byref(o) for o in out]), "tp_attn_split_plan")
+    return tuple(o.value for o in out)
+
+
+def gemm_plan_ex(M, t, row_mode, shard_k, shard_n, out_f32, a_mnmajor=False, b_kmajor=False, heavy_epilogue=False,
+                 slots=74, max_splits=1, sk_area_bytes=0):
+    """gemm_plan_sk with A read M-major (the weight-gradient GEMMs) when a_mnmajor."""
+    out = [ctypes.c_int(0) for _ in range(4)]
+    _check(lib().tp_gemm_plan_ex(int(M), int(t), int(bool(row_mode)), int(shard_k), int(shard_n),
+                                 int(bool(out_f32)), int(bool(a_mnmajor)), int(bool(b_kmajor)),
+                                 int(bool(heavy_epilogue)), int(slots), int(max_splits), int(sk_area_bytes),
+                                 *[ctypes.byref(o) for o in out]), "tp_gemm_plan_ex")
     return tuple(o.value for o in out)
 
 

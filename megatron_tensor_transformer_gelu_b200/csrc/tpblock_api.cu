@@ -301,6 +301,12 @@ unsigned long long next_sk_epoch() {
 
 constexpr double T_KB = 0.40e-6;
 constexpr double T_EPI_256 = 3.5e-6;
+// An M-major A (the weight-gradient GEMMs: X^T, G^T, O^T) costs the
+// 256-column tiles 10 % more per k-block than the model's K-major figure,
+// relative to the wide tiles: measured (ncu, one box) dWqkv 692.6 against
+// 634.5 us, dWo 238.2 against 222.1, the MLP's dA 243.1 against 221.9 and
+// dB 243.3 against 222.4 us at 256 and 512 columns.
+constexpr double MN_A_PENALTY_256 = 1.10;
 
 double per_mac_factor(int w) {
   static const int xs[] = {256, 384, 448, 480, 512};
@@ -330,7 +336,8 @@ TilePlan plan_tiles_dp(const tp::GemmArgs& p, bool pair, int slots, int max_spli
   for (int s = 1; s <= max_splits && s <= p.k_blocks; ++s) {
     const long long waves = (tiles * s + slots - 1) / slots;
     const long long kb = (p.k_blocks + s - 1) / s;
-    const double t = static_cast<double>(waves * kb) * T_KB + (s - 1) * slot_cost;
+    const double t = static_cast<double>(waves * kb) * T_KB * (p.a_mnmajor ? MN_A_PENALTY_256 : 1.0) +
+                     (s - 1) * slot_cost;
     if (t < best_t * 0.98) {  // a split must buy at least 2%
       best_t = t;
       best.splits = s;
@@ -2035,11 +2042,19 @@ int tp_set_gemm_stream_k(int mode) {
 int tp_gemm_plan_sk(int M, int t, int row_mode, int shard_k, int shard_n, int out_f32, int b_kmajor,
                     int heavy_epilogue, int slots, int max_splits, size_t sk_area_bytes, int* tile_n, int* splits,
                     int* stream_k, int* sk_clusters) {
+  return tp_gemm_plan_ex(M, t, row_mode, shard_k, shard_n, out_f32, 0, b_kmajor, heavy_epilogue, slots, max_splits,
+                         sk_area_bytes, tile_n, splits, stream_k, sk_clusters);
+}
+
+int tp_gemm_plan_ex(int M, int t, int row_mode, int shard_k, int shard_n, int out_f32, int a_mnmajor, int b_kmajor,
+                    int heavy_epilogue, int slots, int max_splits, size_t sk_area_bytes, int* tile_n, int* splits,
+                    int* stream_k, int* sk_clusters) {
   if (M < 1 || t < 1 || t > TP_MAX_SHARDS || shard_k < 1 || shard_n < 1 || slots < 1 || max_splits < 1 ||
       !tile_n || !splits)
     return TP_ERR_INVALID_ARG;
   tp::GemmArgs p;
   std::memset(&p, 0, sizeof(p));
+  p.a_mnmajor = a_mnmajor ? 1 : 0;
   p.M = M;
   p.t = t;
   p.row_mode = row_mode ? 1 : 0;

@@ -173,3 +173,20 @@ def test_attn_split_plan_edges():
             L.attn_split_plan(*args)
     with pytest.raises(L.TPError):
         L.set_attn_kv_split(3)
+
+
+# --------------------------------------- weight-gradient GEMMs (M-major A)
+# (M, t, shard_k, shard_n): the MLP's dA = X^T dU and dB = G^T dZ, the attention
+# backward's dWo = O^T dZ and dWqkv = X^T dQKV, all f32 out.  With an M-major
+# A the 256-column tiles cost 10 % more per k-block (measured), so the wide
+# tiles win; the same shapes with a K-major A keep 256.
+WGRAD_CASES = [("mlp dA", 4096, 4, 2048, 4096), ("mlp dB", 16384, 1, 2048, 4096),
+               ("attn dWo", 8192, 1, 2048, 8192), ("attn dWqkv", 8192, 4, 2048, 6144)]
+
+
+@pytest.mark.parametrize("case", WGRAD_CASES, ids=[c[0] for c in WGRAD_CASES])
+def test_weight_gradient_gemms_take_wide_tiles(case):
+    _, M, t, sk, sn = case
+    assert L.gemm_plan_ex(M, t, 0, sk, sn, True, a_mnmajor=True) == (512, 1, 0, 0)
+    assert L.gemm_plan_ex(M, t, 0, sk, sn, True, a_mnmajor=False) == (256, 1, 0, 0)
+    assert L.gemm_plan_sk(M, t, 0, sk, sn, True) == L.gemm_plan_ex(M, t, 0, sk, sn, True)

@@ -62,17 +62,6 @@ __device__ __forceinline__ void lnb_unpack8(const uint4& w, float (&v)[8]) {
   }
 }
 
-__device__ __forceinline__ void lnb_load8_bf16(const __nv_bfloat16* src, float (&v)[8]) {
-  const uint4 w = *reinterpret_cast<const uint4*>(src);
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float2 f = __bfloat1622float2(h[e]);
-    v[2 * e] = f.x;
-    v[2 * e + 1] = f.y;
-  }
-}
-
 // One row per CTA at a time, CH chunks of 8 per thread (H <= CH * 2048).  The
 // CTA's per-column dgamma/dbeta sums live in dynamic shared memory as four
 // planes of H / 8 float4 (dgamma elements 0..3 and 4..7 of each chunk, then
@@ -93,10 +82,32 @@ __global__ void __launch_bounds__(lnb::THREADS, CH <= 2 ? TP_LNB_MIN_BLOCKS : 1)
   griddep_wait();  // V, the statistics and dY come from preceding kernels
   griddep_launch_dependents();
   const float inv_h = 1.0f / static_cast<float>(p.H);
+  // The row in flight: its loads are issued one row ahead, before the
+  // current row's reduction barrier, so they overlap that row's reduction,
+  // its dZ stores and its dgamma/dbeta updates.
+  uint4 xr[CH], dyr[CH];
+  float4 var[CH], vbr[CH];
+  float2 str = make_float2(0.0f, 0.0f);
+  auto load_row = [&](int row) {
+    const long long base = static_cast<long long>(row) * p.H;
+    str = *reinterpret_cast<const float2*>(p.stats + 2LL * row);
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int k = c * lnb::THREADS + tid;
+      if (k < nch) {
+        xr[c] = *reinterpret_cast<const uint4*>(p.X + base + k * 8);
+        dyr[c] = *reinterpret_cast<const uint4*>(p.dY + base + k * 8);
+        const float4* vp = reinterpret_cast<const float4*>(p.V + base + k * 8);
+        var[c] = __ldcs(vp);
+        vbr[c] = __ldcs(vp + 1);
+      }
+    }
+  };
+  if (static_cast<int>(blockIdx.x) < p.S) load_row(blockIdx.x);
   int parity = 0;
   for (int row = blockIdx.x; row < p.S; row += gridDim.x, parity ^= 1) {
     const long long base = static_cast<long long>(row) * p.H;
-    const float2 st = *reinterpret_cast<const float2*>(p.stats + 2LL * row);
+    const float2 st = str;
     float xh[CH][8];
     uint4 dyp[CH];
     float sg = 0.0f, sgx = 0.0f;
@@ -105,11 +116,9 @@ __global__ void __launch_bounds__(lnb::THREADS, CH <= 2 ? TP_LNB_MIN_BLOCKS : 1)
       const int k = c * lnb::THREADS + tid;
       if (k < nch) {
         float x[8], dy[8], gm[8];
-        lnb_load8_bf16(p.X + base + k * 8, x);
-        dyp[c] = *reinterpret_cast<const uint4*>(p.dY + base + k * 8);
-        const float4* vp = reinterpret_cast<const float4*>(p.V + base + k * 8);
-        const float4 va = __ldcs(vp), vb = __ldcs(vp + 1);
-        const float v[8] = {va.x, va.y, va.z, va.w, vb.x, vb.y, vb.z, vb.w};
+        lnb_unpack8(xr[c], x);
+        dyp[c] = dyr[c];
+        const float v[8] = {var[c].x, var[c].y, var[c].z, var[c].w, vbr[c].x, vbr[c].y, vbr[c].z, vbr[c].w};
         lnb_unpack8(dyp[c], dy);
         lnb_gamma8(p.gamma, k * 8, gm);
 #pragma unroll
@@ -122,6 +131,7 @@ __global__ void __launch_bounds__(lnb::THREADS, CH <= 2 ? TP_LNB_MIN_BLOCKS : 1)
         }
       }
     }
+    if (row + static_cast<int>(gridDim.x) < p.S) load_row(row + gridDim.x);
     // Row sums: warp shuffles, then the 8 warps' sums in warp order.
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {

@@ -124,12 +124,20 @@ __device__ __forceinline__ void store8(const ReduceLnArgs& p, long long off, con
 // beyond) keep registers low and occupancy high; larger H uses more warps per
 // row.  NP1 specialises the common single partial so that every load of a row
 // is issued before its first add.
-template <int WPR, int CH, bool NP1>
+//
+// PF (one partial, bf16 X) loads each row group one iteration ahead: the next
+// group's loads are issued before this group's reductions, so they overlap
+// the barriers and the stores.
 #ifndef TP_RLN_CH4_MIN_BLOCKS
 #define TP_RLN_CH4_MIN_BLOCKS 4
 #endif
+#ifndef TP_RLN_PF_MIN_BLOCKS
+#define TP_RLN_PF_MIN_BLOCKS 3  // CTAs per SM the two-chunk prefetching kernel's registers are sized for
+#endif
+template <int WPR, int CH, bool NP1, bool PF = false>
 __global__ void __launch_bounds__(rln::cta_threads(WPR),
-                                  (TP_RLN_LEAN && rln::cta_threads(WPR) == 256) ? (CH <= 2 ? 5 : TP_RLN_CH4_MIN_BLOCKS) : 1)
+                                  PF ? (CH <= 2 ? TP_RLN_PF_MIN_BLOCKS : 2)
+                                     : ((TP_RLN_LEAN && rln::cta_threads(WPR) == 256) ? (CH <= 2 ? 5 : TP_RLN_CH4_MIN_BLOCKS) : 1))
     reduce_residual_ln_kernel(const ReduceLnArgs p) {
   constexpr int RPC = WPR > 8 ? 1 : rln::THREADS / 32 / WPR;  // rows per CTA
   __shared__ float red[2][RPC][WPR];
@@ -138,12 +146,45 @@ __global__ void __launch_bounds__(rln::cta_threads(WPR),
   griddep_wait();  // the partial sums come from the preceding kernel
   griddep_launch_dependents();
   const int groups = (p.S + RPC - 1) / RPC;
+  uint4 xr[PF ? CH : 1];
+  float4 pra[PF ? CH : 1], prb[PF ? CH : 1];
+  auto prefetch = [&](int gg) {
+    const long long prow = static_cast<long long>(gg) * RPC + rloc;
+    const bool plive = gg < groups && prow < p.S && rloc < RPC;
+#pragma unroll
+    for (int c = 0; c < (PF ? CH : 1); ++c) {
+      const int col = ((c * WPR + wr) * 32 + lane) * 8;
+      if (plive && col < p.H) {
+        xr[c] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.X) + prow * p.H + col);
+        const float4* src = reinterpret_cast<const float4*>(p.parts + prow * p.H + col);
+        pra[c] = __ldcs(src);
+        prb[c] = __ldcs(src + 1);
+      }
+    }
+  };
+  if constexpr (PF) prefetch(blockIdx.x);
   for (int g = blockIdx.x; g < groups; g += gridDim.x) {
     const long long row = static_cast<long long>(g) * RPC + rloc;
     const bool live = row < p.S && rloc < RPC;
     const long long base = row * p.H;
     float v[CH][8];
-    if (NP1) {
+    if constexpr (PF) {
+#pragma unroll
+      for (int c = 0; c < CH; ++c) {
+        const int col = ((c * WPR + wr) * 32 + lane) * 8;
+        if (live && col < p.H) {
+          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&xr[c]);
+          const float w[8] = {pra[c].x, pra[c].y, pra[c].z, pra[c].w, prb[c].x, prb[c].y, prb[c].z, prb[c].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h[e]);
+            v[c][2 * e] = f.x + w[2 * e];
+            v[c][2 * e + 1] = f.y + w[2 * e + 1];
+          }
+        }
+      }
+      prefetch(g + gridDim.x);
+    } else if (NP1) {
 #if TP_RLN_LEAN
       // each chunk's partial added as it arrives: fewer live registers, more
       // CTAs resident per SM

@@ -786,6 +786,7 @@ int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, i
   else if (H <= 4096) np1 ? go(reduce_residual_ln_kernel<16, 1, true>, 16, 1) : go(reduce_residual_ln_kernel<16, 1, false>, 16, 1);
 #elif TP_RLN_4096_WPR == 4
   // two rows per 256-thread CTA, 4 warps and 4 chunks per lane each
+  else if (H <= 4096 && TP_RLN_PF && np1 && x_bf16 && apply_ln) go(reduce_residual_ln_kernel<4, 4, true, true>, 4, 2);
   else if (H <= 4096) np1 ? go(reduce_residual_ln_kernel<4, 4, true>, 4, 2) : go(reduce_residual_ln_kernel<4, 4, false>, 4, 2);
 #else
   else if (H <= 4096 && TP_RLN_PF && np1 && x_bf16 && apply_ln) go(reduce_residual_ln_kernel<8, 2, true, true>, 8, 1);

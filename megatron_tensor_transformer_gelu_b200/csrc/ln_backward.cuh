@@ -40,28 +40,6 @@ struct LnBackArgs {
   float* partial;              // [gridDim.x][2][H]: per-CTA (dgamma, dbeta) sums
 };
 
-__device__ __forceinline__ void lnb_gamma8(const float* gamma, int col, float (&gm)[8]) {
-  if (gamma) {
-    const float4 ga = __ldg(reinterpret_cast<const float4*>(gamma + col));
-    const float4 gb = __ldg(reinterpret_cast<const float4*>(gamma + col) + 1);
-    gm[0] = ga.x; gm[1] = ga.y; gm[2] = ga.z; gm[3] = ga.w;
-    gm[4] = gb.x; gm[5] = gb.y; gm[6] = gb.z; gm[7] = gb.w;
-  } else {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) gm[e] = 1.0f;
-  }
-}
-
-__device__ __forceinline__ void lnb_unpack8(const uint4& w, float (&v)[8]) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&w);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float2 f = __bfloat1622float2(h[e]);
-    v[2 * e] = f.x;
-    v[2 * e + 1] = f.y;
-  }
-}
-
 // One row per CTA at a time, CH chunks of 8 per thread (H <= CH * 2048).  The
 // CTA's per-column dgamma/dbeta sums live in dynamic shared memory as four
 // planes of H / 8 float4 (dgamma elements 0..3 and 4..7 of each chunk, then
@@ -71,6 +49,28 @@ __device__ __forceinline__ void lnb_unpack8(const uint4& w, float (&v)[8]) {
 #ifndef TP_LNB_MIN_BLOCKS
 #define TP_LNB_MIN_BLOCKS 1  // CTAs per SM the register budget of the 1- and 2-chunk kernels is sized for
 #endif
+// Elementwise work on f32 pairs (fma/add/mul.rn.f32x2): with the row
+// constants folded, x̂ = Z r - mean r and dZ = g r + x̂ (-mean(g x̂) r) +
+// (-mean(g) r), two pair instructions each.
+using f2x = unsigned long long;
+
+// The two bf16 of a 32-bit word as an f32 pair (low half first).
+__device__ __forceinline__ f2x lnb_bf2(uint32_t w) {
+  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+__device__ __forceinline__ void lnb_gamma4(const float* gamma, int col, f2x (&gm)[4]) {
+  if (gamma) {
+    const ulonglong2 ga = __ldg(reinterpret_cast<const ulonglong2*>(gamma + col));
+    const ulonglong2 gb = __ldg(reinterpret_cast<const ulonglong2*>(gamma + col) + 1);
+    gm[0] = ga.x; gm[1] = ga.y; gm[2] = gb.x; gm[3] = gb.y;
+  } else {
+    const f2x one = f2_pack(1.0f, 1.0f);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) gm[e] = one;
+  }
+}
+
 template <int CH>
 __global__ void __launch_bounds__(lnb::THREADS, CH <= 2 ? TP_LNB_MIN_BLOCKS : 1) ln_backward_kernel(const LnBackArgs p) {
   extern __shared__ float4 lnb_acc[];  // [4][H / 8]
@@ -86,7 +86,7 @@ __global__ void __launch_bounds__(lnb::THREADS, CH <= 2 ? TP_LNB_MIN_BLOCKS : 1)
   // current row's reduction barrier, so they overlap that row's reduction,
   // its dZ stores and its dgamma/dbeta updates.
   uint4 xr[CH], dyr[CH];
-  float4 var[CH], vbr[CH];
+  ulonglong2 var[CH], vbr[CH];
   float2 str = make_float2(0.0f, 0.0f);
   auto load_row = [&](int row) {
     const long long base = static_cast<long long>(row) * p.H;
@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(lnb::THREADS, CH <= 2 ? TP_LNB_MIN_BLOCKS : 1)
       if (k < nch) {
         xr[c] = *reinterpret_cast<const uint4*>(p.X + base + k * 8);
         dyr[c] = *reinterpret_cast<const uint4*>(p.dY + base + k * 8);
-        const float4* vp = reinterpret_cast<const float4*>(p.V + base + k * 8);
+        const ulonglong2* vp = reinterpret_cast<const ulonglong2*>(p.V + base + k * 8);
         var[c] = __ldcs(vp);
         vbr[c] = __ldcs(vp + 1);
       }
@@ -107,31 +107,40 @@ __global__ void __launch_bounds__(lnb::THREADS, CH <= 2 ? TP_LNB_MIN_BLOCKS : 1)
   int parity = 0;
   for (int row = blockIdx.x; row < p.S; row += gridDim.x, parity ^= 1) {
     const long long base = static_cast<long long>(row) * p.H;
-    const float2 st = str;
-    float xh[CH][8];
+    const f2x r2 = f2_pack(str.y, str.y);
+    const f2x b2 = f2_pack(-str.x * str.y, -str.x * str.y);
+    f2x xh[CH][4];
     uint4 dyp[CH];
-    float sg = 0.0f, sgx = 0.0f;
+    f2x sg2 = 0ull, sgx2 = 0ull;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int k = c * lnb::THREADS + tid;
       if (k < nch) {
-        float x[8], dy[8], gm[8];
-        lnb_unpack8(xr[c], x);
+        f2x gm[4];
+        lnb_gamma4(p.gamma, k * 8, gm);
         dyp[c] = dyr[c];
-        const float v[8] = {var[c].x, var[c].y, var[c].z, var[c].w, vbr[c].x, vbr[c].y, vbr[c].z, vbr[c].w};
-        lnb_unpack8(dyp[c], dy);
-        lnb_gamma8(p.gamma, k * 8, gm);
+        const uint32_t xw[4] = {xr[c].x, xr[c].y, xr[c].z, xr[c].w};
+        const uint32_t dw[4] = {dyp[c].x, dyp[c].y, dyp[c].z, dyp[c].w};
+        const f2x v[4] = {var[c].x, var[c].y, vbr[c].x, vbr[c].y};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
+        for (int e = 0; e < 4; ++e) {
           // Z = X + V added as the forward's LayerNorm added it
-          xh[c][e] = (x[e] + v[e] - st.x) * st.y;
-          const float g = dy[e] * gm[e];
-          sg += g;
-          sgx = fmaf(g, xh[c][e], sgx);
+          xh[c][e] = f2_fma(f2_add(lnb_bf2(xw[e]), v[e]), r2, b2);
+          const f2x g = f2_mul(lnb_bf2(dw[e]), gm[e]);
+          sg2 = f2_add(sg2, g);
+          sgx2 = f2_fma(g, xh[c][e], sgx2);
         }
       }
     }
     if (row + static_cast<int>(gridDim.x) < p.S) load_row(row + gridDim.x);
+    float sg, sgx;
+    {
+      float a0, a1;
+      f2_unpack(sg2, a0, a1);
+      sg = a0 + a1;
+      f2_unpack(sgx2, a0, a1);
+      sgx = a0 + a1;
+    }
     // Row sums: warp shuffles, then the 8 warps' sums in warp order.
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
@@ -149,35 +158,36 @@ __global__ void __launch_bounds__(lnb::THREADS, CH <= 2 ? TP_LNB_MIN_BLOCKS : 1)
       tg += red[parity][0][w];
       tgx += red[parity][1][w];
     }
-    const float mg = tg * inv_h, mgx = tgx * inv_h;
+    const float c1 = -(tg * inv_h) * str.y, c2 = -(tgx * inv_h) * str.y;
+    const f2x c1p = f2_pack(c1, c1), c2p = f2_pack(c2, c2);
+    const f2x rr2 = r2;
 #pragma unroll
     for (int c = 0; c < CH; ++c) {
       const int k = c * lnb::THREADS + tid;
       if (k < nch) {
-        float dy[8], gm[8];
-        lnb_unpack8(dyp[c], dy);
-        lnb_gamma8(p.gamma, k * 8, gm);
+        f2x gm[4];
+        lnb_gamma4(p.gamma, k * 8, gm);
+        const uint32_t dw[4] = {dyp[c].x, dyp[c].y, dyp[c].z, dyp[c].w};
         uint32_t w[4];
+        ulonglong2* a = reinterpret_cast<ulonglong2*>(lnb_acc + k);
+        ulonglong2 d0 = a[0], d1 = a[nch], e0 = a[2 * nch], e1 = a[3 * nch];
+        f2x dg[4] = {d0.x, d0.y, d1.x, d1.y}, db[4] = {e0.x, e0.y, e1.x, e1.y};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float o0 = st.y * (dy[2 * e] * gm[2 * e] - mg - xh[c][2 * e] * mgx);
-          const float o1 = st.y * (dy[2 * e + 1] * gm[2 * e + 1] - mg - xh[c][2 * e + 1] * mgx);
+          const f2x dy = lnb_bf2(dw[e]);
+          const f2x dz = f2_fma(xh[c][e], c2p, f2_fma(f2_mul(dy, gm[e]), rr2, c1p));
+          float o0, o1;
+          f2_unpack(dz, o0, o1);
           __nv_bfloat162 hh = __floats2bfloat162_rn(o0, o1);
           w[e] = *reinterpret_cast<uint32_t*>(&hh);
+          dg[e] = f2_fma(dy, xh[c][e], dg[e]);
+          db[e] = f2_add(db[e], dy);
         }
         *reinterpret_cast<uint4*>(p.dZ + base + k * 8) = make_uint4(w[0], w[1], w[2], w[3]);
-        float4* a = lnb_acc + k;
-        float4 d0 = a[0], d1 = a[nch], b0 = a[2 * nch], b1 = a[3 * nch];
-        d0.x = fmaf(dy[0], xh[c][0], d0.x); d0.y = fmaf(dy[1], xh[c][1], d0.y);
-        d0.z = fmaf(dy[2], xh[c][2], d0.z); d0.w = fmaf(dy[3], xh[c][3], d0.w);
-        d1.x = fmaf(dy[4], xh[c][4], d1.x); d1.y = fmaf(dy[5], xh[c][5], d1.y);
-        d1.z = fmaf(dy[6], xh[c][6], d1.z); d1.w = fmaf(dy[7], xh[c][7], d1.w);
-        b0.x += dy[0]; b0.y += dy[1]; b0.z += dy[2]; b0.w += dy[3];
-        b1.x += dy[4]; b1.y += dy[5]; b1.z += dy[6]; b1.w += dy[7];
-        a[0] = d0;
-        a[nch] = d1;
-        a[2 * nch] = b0;
-        a[3 * nch] = b1;
+        a[0] = make_ulonglong2(dg[0], dg[1]);
+        a[nch] = make_ulonglong2(dg[2], dg[3]);
+        a[2 * nch] = make_ulonglong2(db[0], db[1]);
+        a[3 * nch] = make_ulonglong2(db[2], db[3]);
       }
     }
   }

@@ -30,6 +30,14 @@
  *  Ordering   Work is enqueued on `stream` (a cudaStream_t; NULL = legacy
  *             default stream).  No call synchronises; results are valid once
  *             the caller has synchronised the stream.
+ *  Graphs     Calls may be captured into a CUDA graph (they allocate nothing
+ *             and never synchronise; make one uncaptured call per device
+ *             first) and the graph replayed, on the default schedules.  The
+ *             forced stream-K schedule (tp_set_gemm_stream_k(1 or 2)) is not
+ *             replay-safe: its flags carry an epoch taken on the host at each
+ *             call, which a replay repeats; so is tp_peer_barrier, whose
+ *             epoch is an argument.  The attention key split clears its flags
+ *             after use, so it is replay-safe.
  *  Errors     Arguments are checked before anything is launched; a failed
  *             check returns its status and enqueues nothing.  A CUDA launch
  *             error returns TP_ERR_CUDA.  Every device-side wait is bounded:

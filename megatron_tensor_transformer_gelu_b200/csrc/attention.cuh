@@ -40,7 +40,10 @@
 // (the online softmax's combination of two key ranges), then stores O and
 // the row's log2 denominator.  The merge is symmetric in the two halves, so
 // results do not depend on which half arrives first.  No CTA ever waits for
-// a CTA that has not finished its main loop, so no wait can deadlock.
+// a CTA that has not finished its main loop, so no wait can deadlock.  The
+// flags carry the launch's epoch, so flags left by an earlier launch that
+// gave up never match; the merging half clears the pair after use, so the
+// replays of a captured launch (one epoch for all of them) start unclaimed.
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -438,6 +441,12 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
           ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
           __threadfence();
           if (!ready) merge = false;
+          // Both halves are done with the flag pair: clear it, so a replay of
+          // this launch (a CUDA graph keeps its epoch) finds it unclaimed.
+          if (ready && lane == 0) {
+            flag_publish(&flags[0], 0ull);
+            flag_publish(&flags[1], 0ull);
+          }
         }
         if (!merge) po = nullptr;  // stored (or gave up): nothing to write here
       }

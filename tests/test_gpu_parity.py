@@ -196,7 +196,10 @@ def test_linear_full_size(cuda_device, kind, t):
 
 # ------------------------------------------------------ reduce + LayerNorm
 
-@pytest.mark.parametrize("H", [8, 264, 4096, 12288, 16384])
+# H: one warp per row (8, 264), the one-CTA rows with the next row group's
+# loads issued ahead at two and four chunks per thread, ragged (2056, 4104)
+# and whole (4096, 8192), and the 12- and 16-warp rows.
+@pytest.mark.parametrize("H", [8, 264, 2056, 4096, 4104, 8192, 12288, 16384])
 @pytest.mark.parametrize("nparts", [0, 1, 3])
 def test_reduce_residual_layernorm(cuda_device, H, nparts):
     g = torch.Generator().manual_seed(H + nparts)
@@ -210,6 +213,23 @@ def test_reduce_residual_layernorm(cuda_device, H, nparts):
     torch.cuda.synchronize()
     Z = X.double().numpy() + (P[:nparts].double().numpy().sum(0) if nparts else 0.0)
     assert rel_err(Y, O.layernorm(Z, gam, bet)) <= TOL_F32
+
+
+@pytest.mark.parametrize("H", [2056, 4104])
+def test_reduce_residual_layernorm_bf16_out(cuda_device, H):
+    """The sublayers' case: one f32 partial, bf16 X and bf16 Y, rows whose
+    chunk count does not fill the CTA (the look-ahead kernel's bounds)."""
+    g = torch.Generator().manual_seed(H)
+    S = 53
+    X = torch.randn(S, H, generator=g).to(torch.bfloat16)
+    P = torch.randn(1, S, H, generator=g) * 3.0
+    gam = torch.randn(H, generator=g)
+    bet = torch.randn(H, generator=g)
+    Y = torch.empty(S, H, dtype=torch.bfloat16, device="cuda")
+    L.reduce_residual_layernorm(P.cuda(), X.cuda(), Y, gam.cuda(), bet.cuda())
+    torch.cuda.synchronize()
+    Z = X.double().numpy() + P.double().numpy().sum(0)
+    assert rel_err(Y, O.layernorm(Z, gam, bet)) <= TOL_BF16
 
 
 # --------------------------------------------------------------- attention

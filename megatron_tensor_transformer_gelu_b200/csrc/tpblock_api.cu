@@ -1547,7 +1547,8 @@ int tp_attn_backward(int S, int H, int nh, int d, int t, int dtype, const void* 
   const float scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(d)));
   {
   ProfScope ps(K_ATTN_BACK, s);
-  st = launch_pdl(tp::rowdot_kernel, dim3(ceil_div(static_cast<long long>(S) * nh * 32, 256)), dim3(256), 0, s,
+  st = launch_pdl(tp::rowdot_kernel, dim3(ceil_div(static_cast<long long>(S) * nh * 32, 256 * tp::ROWDOT_ITEMS)),
+                  dim3(256), 0, s,
                   reinterpret_cast<const __nv_bfloat16*>(dO), reinterpret_cast<const __nv_bfloat16*>(Ob), D, S, H,
                   nh) != cudaSuccess
            ? TP_ERR_CUDA

@@ -59,8 +59,14 @@ constexpr int BQ = 128;           // query rows per tile
 constexpr int TILES = 2;          // query tiles per CTA
 constexpr int BKV = 128;          // keys per block
 constexpr int NUM_THREADS = 352;  // 11 warps
-constexpr int K_STAGES = 2;
-constexpr int V_STAGES = 2;
+#ifndef TP_ATTN_K_STAGES
+#define TP_ATTN_K_STAGES 2
+#endif
+#ifndef TP_ATTN_V_STAGES
+#define TP_ATTN_V_STAGES 2
+#endif
+constexpr int K_STAGES = TP_ATTN_K_STAGES;
+constexpr int V_STAGES = TP_ATTN_V_STAGES;
 constexpr int HALF_BYTES = BQ * 64 * 2;     // one 64-column (128 B) box of 128 rows: 16 KiB
 constexpr int TILE_BYTES = 2 * HALF_BYTES;  // 128 rows x 128 bf16: 32 KiB
 constexpr int SMEM_BYTES = TILE_BYTES * (TILES + K_STAGES + V_STAGES) + 1024 + 256;
@@ -187,14 +193,16 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
       uint64_t* emptyb = is_k ? k_empty : v_empty;
       uint8_t* base = is_k ? sK : sV;
       const int col = is_k ? kcol : vcol;
-      int armed[K_STAGES + 1];
+      // armed[st]: the phase stage st's barrier expects (-1: none); armed[QS]: the Q load's
+      constexpr int QS = K_STAGES > V_STAGES ? K_STAGES : V_STAGES;
+      int armed[QS + 1];
 #pragma unroll
-      for (int i = 0; i <= K_STAGES; ++i) armed[i] = -1;
+      for (int i = 0; i <= QS; ++i) armed[i] = -1;
       bool ok = true;
       if (is_k) {
         // Tiles past S (an odd tile count) are zero-filled by the TMA.
         mbar_arrive_expect_tx(q_full, TILES * TILE_BYTES);
-        armed[K_STAGES] = 0;
+        armed[QS] = 0;
         for (int t = 0; t < TILES; ++t) {
           tma_load_2d(sQ + t * TILE_BYTES, &a.tmQKV, qcol, q0 + t * BQ, q_full);
           tma_load_2d(sQ + t * TILE_BYTES + HALF_BYTES, &a.tmQKV, qcol + 64, q0 + t * BQ, q_full);
@@ -211,9 +219,9 @@ __global__ void __launch_bounds__(attn::NUM_THREADS, 1) attn_fwd_kernel(const __
         tma_load_2d(d + HALF_BYTES, &a.tmQKV, col + 64, (kb0 + j) * BKV, &fullb[st]);
       }
       if (!ok) {
-        for (int i = 0; i <= K_STAGES; ++i) {
-          if (armed[i] < 0 || (i < K_STAGES && i >= nst)) continue;
-          const uint32_t ad = smem_u32(i == K_STAGES ? q_full : &fullb[i]);
+        for (int i = 0; i <= QS; ++i) {
+          if (armed[i] < 0 || (i < QS && i >= nst)) continue;
+          const uint32_t ad = smem_u32(i == QS ? q_full : &fullb[i]);
           const long long t0 = clock64();
           while (!mbar_try_wait(ad, static_cast<uint32_t>(armed[i])) && clock64() - t0 < WAIT_LIMIT_CYCLES) {}
         }

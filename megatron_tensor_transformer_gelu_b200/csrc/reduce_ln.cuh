@@ -124,20 +124,12 @@ __device__ __forceinline__ void store8(const ReduceLnArgs& p, long long off, con
 // beyond) keep registers low and occupancy high; larger H uses more warps per
 // row.  NP1 specialises the common single partial so that every load of a row
 // is issued before its first add.
-//
-// PF (one partial, bf16 X) loads each row group one iteration ahead: the next
-// group's loads are issued before this group's reductions, so they overlap
-// the barriers and the stores.
 #ifndef TP_RLN_CH4_MIN_BLOCKS
 #define TP_RLN_CH4_MIN_BLOCKS 4
 #endif
-#ifndef TP_RLN_PF_MIN_BLOCKS
-#define TP_RLN_PF_MIN_BLOCKS 3  // CTAs per SM the two-chunk prefetching kernel's registers are sized for
-#endif
-template <int WPR, int CH, bool NP1, bool PF = false>
+template <int WPR, int CH, bool NP1>
 __global__ void __launch_bounds__(rln::cta_threads(WPR),
-                                  PF ? (CH <= 2 ? TP_RLN_PF_MIN_BLOCKS : 2)
-                                     : ((TP_RLN_LEAN && rln::cta_threads(WPR) == 256) ? (CH <= 2 ? 5 : TP_RLN_CH4_MIN_BLOCKS) : 1))
+                                  (TP_RLN_LEAN && rln::cta_threads(WPR) == 256) ? (CH <= 2 ? 5 : TP_RLN_CH4_MIN_BLOCKS) : 1)
     reduce_residual_ln_kernel(const ReduceLnArgs p) {
   constexpr int RPC = WPR > 8 ? 1 : rln::THREADS / 32 / WPR;  // rows per CTA
   __shared__ float red[2][RPC][WPR];
@@ -146,45 +138,12 @@ __global__ void __launch_bounds__(rln::cta_threads(WPR),
   griddep_wait();  // the partial sums come from the preceding kernel
   griddep_launch_dependents();
   const int groups = (p.S + RPC - 1) / RPC;
-  uint4 xr[PF ? CH : 1];
-  float4 pra[PF ? CH : 1], prb[PF ? CH : 1];
-  auto prefetch = [&](int gg) {
-    const long long prow = static_cast<long long>(gg) * RPC + rloc;
-    const bool plive = gg < groups && prow < p.S && rloc < RPC;
-#pragma unroll
-    for (int c = 0; c < (PF ? CH : 1); ++c) {
-      const int col = ((c * WPR + wr) * 32 + lane) * 8;
-      if (plive && col < p.H) {
-        xr[c] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.X) + prow * p.H + col);
-        const float4* src = reinterpret_cast<const float4*>(p.parts + prow * p.H + col);
-        pra[c] = __ldcs(src);
-        prb[c] = __ldcs(src + 1);
-      }
-    }
-  };
-  if constexpr (PF) prefetch(blockIdx.x);
   for (int g = blockIdx.x; g < groups; g += gridDim.x) {
     const long long row = static_cast<long long>(g) * RPC + rloc;
     const bool live = row < p.S && rloc < RPC;
     const long long base = row * p.H;
     float v[CH][8];
-    if constexpr (PF) {
-#pragma unroll
-      for (int c = 0; c < CH; ++c) {
-        const int col = ((c * WPR + wr) * 32 + lane) * 8;
-        if (live && col < p.H) {
-          const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&xr[c]);
-          const float w[8] = {pra[c].x, pra[c].y, pra[c].z, pra[c].w, prb[c].x, prb[c].y, prb[c].z, prb[c].w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(h[e]);
-            v[c][2 * e] = f.x + w[2 * e];
-            v[c][2 * e + 1] = f.y + w[2 * e + 1];
-          }
-        }
-      }
-      prefetch(g + gridDim.x);
-    } else if (NP1) {
+    if (NP1) {
 #if TP_RLN_LEAN
       // each chunk's partial added as it arrives: fewer live registers, more
       // CTAs resident per SM
@@ -311,6 +270,156 @@ __global__ void __launch_bounds__(rln::cta_threads(WPR),
         float y[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) y[e] = fmaf((v[c][e] - mean) * rstd, gm[e], bt[e]);
+        store8(p, base + col, y);
+      }
+    }
+    __syncthreads();  // `red` is reused by the next row group
+  }
+}
+
+// ---------------------------------------- rows loaded one group ahead (bf16 X)
+// The common case of the sublayers (one partial, bf16 X, the LN applied; Y
+// bf16 or f32) with the row-group walk of the kernel above, plus two things:
+//  - each thread issues the loads of its next row group before the current
+//    group's two block reductions, so they overlap the barriers and stores;
+//  - the elementwise work runs on f32 pairs (add/sub/mul/fma.rn.f32x2):
+//    Z = X + P, the row sum, the centred squares and
+//    Y = (Z - mean) (r gamma) + beta take one or two pair instructions per
+//    two elements.
+// The statistics keep the two-pass form (mean, then the mean square of
+// Z - mean), reduced by warp shuffles and then across the row's warps in warp
+// order, so results are repeatable.
+#ifndef TP_RLN_PF_MIN_BLOCKS
+#define TP_RLN_PF_MIN_BLOCKS 4  // CTAs per SM the two-chunk kernel's registers are sized for
+#endif
+using rln_f2 = unsigned long long;
+
+__device__ __forceinline__ rln_f2 rln_bf2(uint32_t w) {
+  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+template <int WPR, int CH>
+__global__ void __launch_bounds__(rln::cta_threads(WPR), CH <= 2 ? TP_RLN_PF_MIN_BLOCKS : 2)
+    reduce_residual_ln_pf2_kernel(const ReduceLnArgs p) {
+  constexpr int RPC = WPR > 8 ? 1 : rln::THREADS / 32 / WPR;  // rows per CTA
+  __shared__ float red[2][RPC][WPR];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rloc = warp / WPR, wr = warp % WPR;
+  griddep_wait();  // the partial sums come from the preceding kernel
+  griddep_launch_dependents();
+  const int groups = (p.S + RPC - 1) / RPC;
+  uint4 xr[CH];
+  ulonglong2 pra[CH], prb[CH];
+  auto prefetch = [&](int gg) {
+    const long long prow = static_cast<long long>(gg) * RPC + rloc;
+    const bool plive = gg < groups && prow < p.S && rloc < RPC;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = ((c * WPR + wr) * 32 + lane) * 8;
+      if (plive && col < p.H) {
+        xr[c] = *reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(p.X) + prow * p.H + col);
+        const ulonglong2* src = reinterpret_cast<const ulonglong2*>(p.parts + prow * p.H + col);
+        pra[c] = __ldcs(src);
+        prb[c] = __ldcs(src + 1);
+      }
+    }
+  };
+  prefetch(blockIdx.x);
+  const float inv_h = 1.0f / static_cast<float>(p.H);
+  for (int g = blockIdx.x; g < groups; g += gridDim.x) {
+    const long long row = static_cast<long long>(g) * RPC + rloc;
+    const bool live = row < p.S && rloc < RPC;
+    const long long base = row * p.H;
+    rln_f2 v[CH][4];
+    rln_f2 sum2 = 0ull;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = ((c * WPR + wr) * 32 + lane) * 8;
+      if (live && col < p.H) {
+        const uint32_t xw[4] = {xr[c].x, xr[c].y, xr[c].z, xr[c].w};
+        const rln_f2 pw[4] = {pra[c].x, pra[c].y, prb[c].x, prb[c].y};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[c][e] = f2_add(rln_bf2(xw[e]), pw[e]);
+          sum2 = f2_add(sum2, v[c][e]);
+        }
+      }
+    }
+    prefetch(g + gridDim.x);
+    float s;
+    {
+      float a0, a1;
+      f2_unpack(sum2, a0, a1);
+      s = a0 + a1;
+    }
+    // mean over the row: warp shuffle, then the row's WPR warps in fixed order
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lane == 0 && rloc < RPC) red[0][rloc][wr] = s;
+    __syncthreads();
+    float tot = 0.0f;
+    if (rloc < RPC) {
+#pragma unroll
+      for (int i = 0; i < WPR; ++i) tot += red[0][rloc][i];
+    }
+    const float mean = tot * inv_h;
+    const rln_f2 mean2 = f2_pack(mean, mean);
+    rln_f2 sq2 = 0ull;
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = ((c * WPR + wr) * 32 + lane) * 8;
+      if (live && col < p.H) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[c][e] = f2_sub(v[c][e], mean2);  // centred from here on
+          sq2 = f2_fma(v[c][e], v[c][e], sq2);
+        }
+      }
+    }
+    float s2;
+    {
+      float a0, a1;
+      f2_unpack(sq2, a0, a1);
+      s2 = a0 + a1;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    if (lane == 0 && rloc < RPC) red[1][rloc][wr] = s2;
+    __syncthreads();
+    float tot2 = 0.0f;
+    if (rloc < RPC) {
+#pragma unroll
+      for (int i = 0; i < WPR; ++i) tot2 += red[1][rloc][i];
+    }
+    const float rstd = 1.0f / sqrtf(tot2 * inv_h + p.eps);
+    if (p.stats && live && wr == 0 && lane == 0)
+      *reinterpret_cast<float2*>(p.stats + 2 * row) = make_float2(mean, rstd);
+    const rln_f2 rstd2 = f2_pack(rstd, rstd);
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      const int col = ((c * WPR + wr) * 32 + lane) * 8;
+      if (live && col < p.H) {
+        rln_f2 gm[4], bt[4];
+        if (p.gamma) {
+          const ulonglong2 ga = reinterpret_cast<const ulonglong2*>(p.gamma + col)[0];
+          const ulonglong2 gb = reinterpret_cast<const ulonglong2*>(p.gamma + col)[1];
+          gm[0] = ga.x; gm[1] = ga.y; gm[2] = gb.x; gm[3] = gb.y;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) gm[e] = f2_pack(1.0f, 1.0f);
+        }
+        if (p.beta) {
+          const ulonglong2 ba = reinterpret_cast<const ulonglong2*>(p.beta + col)[0];
+          const ulonglong2 bb = reinterpret_cast<const ulonglong2*>(p.beta + col)[1];
+          bt[0] = ba.x; bt[1] = ba.y; bt[2] = bb.x; bt[3] = bb.y;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) bt[e] = 0ull;
+        }
+        float y[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          f2_unpack(f2_fma(v[c][e], f2_mul(rstd2, gm[e]), bt[e]), y[2 * e], y[2 * e + 1]);
         store8(p, base + col, y);
       }
     }

@@ -58,7 +58,7 @@ struct DeviceInfo {
 // Rows of 2049..4096 columns: 8 warps a row with 16 values a lane (0), or 16
 // warps a row with 8 values a lane (1).
 #ifndef TP_RLN_PF
-#define TP_RLN_PF 1  // single-partial bf16 rows loaded one row group ahead (reduce_ln.cuh)
+#define TP_RLN_PF 1  // single-partial bf16 rows loaded one group ahead, on f32 pairs (reduce_residual_ln_pf2_kernel)
 #endif
 #ifndef TP_RLN_4096_WPR
 #define TP_RLN_4096_WPR 8  // warps per row of the reduce + LayerNorm kernel for 2048 < H <= 4096 (8 or 4)
@@ -786,13 +786,13 @@ int run_reduce_ln(int S, int H, int nparts, const float* parts, const void* X, i
   else if (H <= 4096) np1 ? go(reduce_residual_ln_kernel<16, 1, true>, 16, 1) : go(reduce_residual_ln_kernel<16, 1, false>, 16, 1);
 #elif TP_RLN_4096_WPR == 4
   // two rows per 256-thread CTA, 4 warps and 4 chunks per lane each
-  else if (H <= 4096 && TP_RLN_PF && np1 && x_bf16 && apply_ln) go(reduce_residual_ln_kernel<4, 4, true, true>, 4, 2);
+  else if (H <= 4096 && TP_RLN_PF && np1 && x_bf16 && apply_ln) go(reduce_residual_ln_pf2_kernel<4, 4>, 4, 2);
   else if (H <= 4096) np1 ? go(reduce_residual_ln_kernel<4, 4, true>, 4, 2) : go(reduce_residual_ln_kernel<4, 4, false>, 4, 2);
 #else
-  else if (H <= 4096 && TP_RLN_PF && np1 && x_bf16 && apply_ln) go(reduce_residual_ln_kernel<8, 2, true, true>, 8, 1);
+  else if (H <= 4096 && TP_RLN_PF && np1 && x_bf16 && apply_ln) go(reduce_residual_ln_pf2_kernel<8, 2>, 8, 1);
   else if (H <= 4096) np1 ? go(reduce_residual_ln_kernel<8, 2, true>, 8, 1) : go(reduce_residual_ln_kernel<8, 2, false>, 8, 1);
 #endif
-  else if (H <= 8192 && TP_RLN_PF && np1 && x_bf16 && apply_ln) go(reduce_residual_ln_kernel<8, 4, true, true>, 8, 1);
+  else if (H <= 8192 && TP_RLN_PF && np1 && x_bf16 && apply_ln) go(reduce_residual_ln_pf2_kernel<8, 4>, 8, 1);
   else if (H <= 8192) np1 ? go(reduce_residual_ln_kernel<8, 4, true>, 8, 1) : go(reduce_residual_ln_kernel<8, 4, false>, 8, 1);
   // (one-row CTAs of 12 or 16 warps keep the generic loop: fewer registers, two CTAs per SM)
   else if (H <= 12288) go(reduce_residual_ln_kernel<12, 4, false>, 12, 1);

@@ -159,6 +159,10 @@ struct GemmArgs {
   int n_blocks_per_shard;        // column mode
   int k_blocks_per_shard;        // row mode (column mode: k blocks of K)
   int m_blocks, n_blocks, k_blocks;  // m_blocks counts TILE_M-row tiles
+  // Tile order: 0, tile t is (m block t mod m_blocks, n block t / m_blocks),
+  // so a wave shares B columns; 1, (t / n_blocks, t mod n_blocks), so a wave
+  // shares A rows (for an A too large to stay in L2 across waves).
+  int n_fastest;
   int act;
   int out_f32;
   // Split of the K loop into `splits` contiguous k-block ranges.  Work unit u
@@ -614,8 +618,8 @@ template <int CG>
 __device__ __forceinline__ TileCoord tile_coord(const GemmArgs& p, int tile) {
   using C = GemmCfg<CG>;
   TileCoord c;
-  const int mb = tile % p.m_blocks;
-  const int nb = tile / p.m_blocks;
+  const int mb = p.n_fastest ? tile / p.n_blocks : tile % p.m_blocks;
+  const int nb = p.n_fastest ? tile % p.n_blocks : tile / p.m_blocks;
   c.m0 = mb * C::TILE_M;
   if (!p.row_mode) {
     c.shard = nb / p.n_blocks_per_shard;

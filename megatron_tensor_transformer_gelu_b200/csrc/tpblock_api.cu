@@ -60,6 +60,9 @@ struct DeviceInfo {
 #ifndef TP_RLN_PF
 #define TP_RLN_PF 1  // single-partial bf16 rows loaded one group ahead, on f32 pairs (reduce_residual_ln_pf2_kernel)
 #endif
+#ifndef TP_DB_N_FASTEST
+#define TP_DB_N_FASTEST 1  // the MLP's dB GEMMs walk their tiles n fastest
+#endif
 #ifndef TP_RLN_4096_WPR
 #define TP_RLN_4096_WPR 8  // warps per row of the reduce + LayerNorm kernel for 2048 < H <= 4096 (8 or 4)
 #endif
@@ -447,6 +450,7 @@ TilePlan plan_tiles(const tp::GemmArgs& p, bool pair, int slots, int max_splits,
 // the epilogue modes of tp::GemmArgs.
 struct GemmExtra {
   int a_mnmajor = 0;                 // A stored [K, M] (row stride lda)
+  int n_fastest = 0;                 // tiles walk n fastest (GemmArgs::n_fastest)
   long long ldb = 0;                 // row stride of every B shard (0: contiguous)
   void* const* C_shards = nullptr;   // column mode: shard s writes C_shards[s] (row stride ldc_shard)
   long long ldc_shard = 0;
@@ -596,6 +600,7 @@ int run_gemm_tc(const DeviceInfo& dev, const void* A, long long lda, int M, cons
     p.epi_scale2 = ex.epi_scale2;
   }
   p.a_mnmajor = ex.a_mnmajor;
+  p.n_fastest = ex.n_fastest;
   p.epi_mode = ex.epi_mode;
   p.rowvec = ex.rowvec;
   p.rowvec_ld = ex.rowvec_ld;
@@ -1347,6 +1352,7 @@ int tp_mlp_backward_ex(int S, int H, int F, int t, int dtype, int w_layout, cons
   if (t > 1 && Fs % 256 == 0) {  // F >= 512 rows: the CTA-pair GEMM with 256-row tiles
     GemmExtra ex;
     ex.a_mnmajor = 1;
+    ex.n_fastest = TP_DB_N_FASTEST;  // G (S x F) is read once per wave, not once per column block
     ex.m_split = t;
     ex.C_shards = splitOut;
     ex.ldc_shard = H;
@@ -1355,6 +1361,7 @@ int tp_mlp_backward_ex(int S, int H, int F, int t, int dtype, int w_layout, cons
   for (int i = 0; i < t; ++i) {
     GemmExtra ex;
     ex.a_mnmajor = 1;
+    ex.n_fastest = TP_DB_N_FASTEST;
     st = run_gemm_tc(*dev, splitA + static_cast<size_t>(i) * Fs * 2, F, Fs, b1, 1, 0, S, H, splitOut[i], H, 1,
                      TP_ACT_NONE, s, 1, 0, nullptr, 0, &ex);
     if (st != TP_OK) return st;
